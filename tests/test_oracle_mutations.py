@@ -1,0 +1,121 @@
+"""Plant plausible mistakes in the oracle (on the CPU, by monkeypatching) and
+check that the pins catch every one of them."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+import oracle.wsvd_oracle as OW
+import test_oracle_pins as P
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(OW, name, fn)
+    monkeypatch.setattr(O, name, fn)
+
+
+def _decode_head_variant(kind):
+    def f(q, lat_k, scale_k, lat_v, scale_v, Bk_h, Bv_h, n, r, bits, softmax_scale=None):
+        Hd = Bk_h.shape[1]
+        latK = OW.dequantize(lat_k[:n], scale_k[:n], r, bits)
+        latV = OW.dequantize(lat_v[:n], scale_v[:n], r, bits)
+        if kind == "no_scale_K":
+            latK = OW.unpack_codes(lat_k[:n], r, bits).astype(np.float64)
+        K = latK @ np.asarray(Bk_h, np.float64)
+        V = latV @ np.asarray((Bk_h if kind == "swap_B" else Bv_h), np.float64)
+        sc = 1.0 if kind == "no_softmax_scale" else OW.default_scale(Hd, softmax_scale)
+        if kind == "sign":
+            sc = -sc
+        out, p = OW.attention(np.asarray(q, np.float64), K, V, sc)
+        if kind == "drop_last_token" and n > 1:
+            out, p = OW.attention(np.asarray(q, np.float64), K[:-1], V[:-1], sc)
+        return out, p
+    return f
+
+
+
+@pytest.mark.parametrize("kind", ["swap_B", "no_softmax_scale", "no_scale_K", "sign", "drop_last_token"])
+def test_decode_mutants_are_caught(monkeypatch, kind):
+    _patch(monkeypatch, "wsvd_decode_head", _decode_head_variant(kind))
+    with pytest.raises(AssertionError):
+        P.test_decode_matches_exact_bruteforce(8, 3, 5, 4)
+
+
+def test_nibble_order_mutant_is_caught(monkeypatch):
+    orig = OW.unpack_codes
+
+    def swapped(lat, r, bits):
+        c = orig(lat, r, bits)
+        if bits == 4:
+            c = c.reshape(c.shape[:-1] + (r // 2, 2))[..., ::-1].reshape(c.shape)
+        return c
+    _patch(monkeypatch, "unpack_codes", swapped)
+    with pytest.raises(AssertionError):
+        P.test_int4_layout_golden()
+
+
+def test_round_half_away_mutant_is_caught(monkeypatch):
+    def q_away(c, bits):
+        Q = OW.qmax(bits)
+        c32 = np.asarray(c, np.float64).astype(np.float32)
+        amax = np.max(np.abs(c32), axis=-1)
+        scale = (amax / np.float32(Q)).astype(np.float16)
+        s32 = scale.astype(np.float32)[..., None]
+        v = np.where(s32 > 0, c32 / np.where(s32 > 0, s32, 1), 0)
+        codes = np.clip(np.sign(v) * np.floor(np.abs(v) + 0.5), -Q, Q).astype(np.int64)
+        return codes, scale
+    _patch(monkeypatch, "quantize", q_away)
+    with pytest.raises(AssertionError):
+        P.test_quantize_ties_to_even_and_clamp()
+
+
+def test_scale_without_fp16_rounding_mutant_is_caught(monkeypatch):
+    def q_f32(c, bits):
+        Q = OW.qmax(bits)
+        c32 = np.asarray(c, np.float64).astype(np.float32)
+        amax = np.max(np.abs(c32), axis=-1)
+        scale = amax / np.float32(Q)
+        v = np.where(scale[..., None] > 0, c32 / np.where(scale[..., None] > 0, scale[..., None], 1), 0)
+        return np.clip(np.rint(v), -Q, Q).astype(np.int64), scale
+    _patch(monkeypatch, "quantize", q_f32)
+    with pytest.raises(AssertionError):
+        P.test_quantize_random_rows_properties(8)
+
+
+def test_unnormalised_rotation_mutant_is_caught(monkeypatch):
+    def rot(x, block):
+        x = np.asarray(x, np.float64)
+        Hn = OW.sylvester_hadamard(block)
+        out = np.empty_like(x)
+        for s in range(0, x.shape[-1], block):
+            out[..., s:s + block] = x[..., s:s + block] @ Hn
+        return out
+    _patch(monkeypatch, "block_hadamard_rotate", rot)
+    with pytest.raises(AssertionError):
+        P.test_projection_undoes_rotation()
+
+
+def test_reversed_block_order_mutant_is_caught(monkeypatch):
+    def rot(x, block):
+        x = np.asarray(x, np.float64)
+        Hn = OW.sylvester_hadamard(block) / math.sqrt(block)
+        out = np.empty_like(x)
+        E = x.shape[-1]
+        for s in range(0, E, block):
+            d = E - block - s  # writes block k into block (n-1-k)
+            out[..., d:d + block] = x[..., s:s + block] @ Hn
+        return out
+    _patch(monkeypatch, "block_hadamard_rotate", rot)
+    with pytest.raises(AssertionError):
+        P.test_block_rotation_orthonormal_and_blockwise()
+
+
+def test_shared_path_wrong_head_mutant_is_caught(monkeypatch):
+    orig = OW.shared_latent_decode
+
+    def wrong(q, lat_k, lat_v, Bk, Bv, seq_lens, softmax_scale=None):
+        return orig(q, lat_k, lat_v, Bk[::-1], Bv, seq_lens, softmax_scale)
+    _patch(monkeypatch, "shared_latent_decode", wrong)
+    with pytest.raises(AssertionError):
+        P.test_shared_latent_with_selector_factors_equals_dense()
