@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the WSVD low-rank decode step on B200.
+
+A step is one pass of the hot path over one batch: the latent append of the
+new token (block-Hadamard rotation, projection through A_Kh / A_Vh, int8/int4
+quantisation into the cache) followed by the decode-step attention over the
+per-head low-rank cache (split-L kernel + combine).  Workloads without an
+append (ragged int4, comparison shapes) time the decode alone.
+
+Prints ONE JSON line (rank 0).  `value` is tokens*heads/s over the whole job
+(sum over sequences of the attended length times heads, divided by the device
+time of the timed steps, max over ranks).  Inputs are resident in HBM before
+the timed region; L2 is flushed (a 256 MiB write) between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl wsvd|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload
+(the decode has no exchange step); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "low-rank decode-attention step µs, tokens·heads/s, HBM GB/s vs ~8 TB/s peak"
+UNIT = "tokens*heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "rank_kv_cache_wsvd_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h"],
+                  "decode": ["decode.cu", "common.cuh", "wsvd_internal.h"]}
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_digest") != source_digest(KERNEL_SOURCES[kernel]):
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [ln.split(", ") for ln in out.strip().splitlines() if ln.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workloads
+def attended_tokens(w: WL.Workload, lens_after: np.ndarray) -> int:
+    return int(lens_after.sum()) * w.H
+
+
+def alg_bytes_decode(w: WL.Workload, lens: np.ndarray) -> int:
+    rb = w.r * w.bits // 8
+    codes = int(lens.sum()) * w.H * 2 * (rb + 2)
+    weights = 2 * w.H * w.r * w.Hd * 2
+    io = w.B * w.H * w.Hd * (2 + 4)
+    return codes + weights + io
+
+
+def alg_bytes_append(w: WL.Workload) -> int:
+    rb = w.r * w.bits // 8
+    return 2 * w.H * w.E * w.r * 2 + w.B * w.E * 2 + w.B * w.H * 2 * (rb + 2) + w.B * 4 * 2
+
+
+class WsvdStep:
+    """Device-resident inputs of one workload and the launches of one step."""
+
+    def __init__(self, w: WL.Workload, seed: int = 0):
+        import torch
+
+        import rank_kv_cache_wsvd_b200 as W
+        self.W, self.torch, self.w = W, torch, w
+        self.has_append = w.append_steps > 0
+        lens_full = WL.seq_lens(w, seed)
+        lens0 = lens_full - 1 if self.has_append else lens_full
+        d = WL.decode_inputs(w, seed=seed, lens=lens_full)
+        if self.has_append:  # the new token's row is produced by the append inside each step
+            for b in range(w.B):
+                n = int(lens0[b])
+                d.lat_k[b, :, n:] = 0
+                d.lat_v[b, :, n:] = 0
+                d.scale_k[b, :, n:] = 0
+                d.scale_v[b, :, n:] = 0
+        cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
+        self.q = cu(d.q_bits.view(np.int16)).view(qdt)
+        self.lat_k, self.lat_v = cu(d.lat_k), cu(d.lat_v)
+        self.scale_k, self.scale_v = cu(d.scale_k), cu(d.scale_v)
+        self.B_k, self.B_v = cu(d.Bk), cu(d.Bv)
+        self.lens0 = cu(lens0.astype(np.int32))
+        self.lens = self.lens0.clone()
+        self.lens_after = lens_full.astype(np.int64)
+        self.out = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32, device="cuda")
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.ws = W.workspace(W.wsvd_decode_workspace_size(w.B, w.H, w.r))
+        if self.has_append:
+            ai = WL.append_inputs(w, seed=seed, steps=1)
+            self.x = cu(ai.x_bits[0].view(np.int16)).view(torch.bfloat16)
+            self.A_k, self.A_v = cu(ai.A_k), cu(ai.A_v)
+            self.ws_app = W.workspace(W.wsvd_append_workspace_size())
+            self.x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
+        self.out_host = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32).pin_memory()
+        self.launches_per_step = (1 if self.has_append else 0) + 2
+
+    def reset(self):
+        self.lens.copy_(self.lens0)
+
+    def append(self):
+        if self.has_append:
+            self.W.wsvd_latent_append(self.x, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v, self.scale_k,
+                                      self.scale_v, bits=self.w.bits, hadamard_block=self.w.hadamard_block,
+                                      workspace_buf=self.ws_app, err=self.err)
+
+    def decode(self):
+        self.W.wsvd_decode_attention(self.q, self.lat_k, self.lat_v, self.scale_k, self.scale_v, self.B_k, self.B_v,
+                                     self.lens, bits=self.w.bits, out=self.out, workspace_buf=self.ws, err=self.err)
+
+    def e2e_step(self):
+        """Public-API step with host buffers: H2D of the step inputs, append,
+        decode, D2H of the result."""
+        if self.has_append:
+            self.x.copy_(self.x_host, non_blocking=True)
+        self.q.copy_(self.q_host, non_blocking=True)
+        self.append()
+        self.decode()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = self.q_host.numel() * 2 + (self.x_host.numel() * 2 if self.has_append else 0)
+        return h2d, self.out_host.numel() * 4
+
+
+def time_comparisons(w: WL.Workload, steps: int, warmup: int, flush):
+    """Dense fp16 flash-decode and shared-latent SVD decode on the same shapes."""
+    import torch
+
+    import rank_kv_cache_wsvd_b200 as W
+    res = {}
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    ww = w.with_(R=w.R or 512)
+    dd = WL.dense_inputs(ww, seed=0)
+    q = cu(dd["q_bits"].view(np.int16)).view(torch.float16 if w.q_dtype == "fp16" else torch.bfloat16)
+    K, V, lens = cu(dd["K"]), cu(dd["V"]), cu(dd["seq_lens"])
+    del dd
+    wsd = W.workspace(W.dense_decode_workspace_size(w.B, w.H, w.Hd))
+    out = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32, device="cuda")
+    t = _time_loop(lambda: W.dense_decode_attention(q, K, V, lens, out=out, workspace_buf=wsd), steps, warmup, flush)
+    nb = int(WL.seq_lens(w).sum()) * w.H * 2 * w.Hd * 2
+    res["dense_fp16"] = {"us": t * 1e6, "alg_bytes": nb, "gbs": nb / t / 1e9}
+    del K, V
+    sd = WL.shared_inputs(ww, seed=0)
+    lk, lv, bk, bv = cu(sd["lat_k"]), cu(sd["lat_v"]), cu(sd["Bk"]), cu(sd["Bv"])
+    del sd
+    wss = W.workspace(W.shared_decode_workspace_size(w.B, w.H, ww.R))
+    t = _time_loop(lambda: W.shared_latent_svd_decode(q, lk, lv, bk, bv, lens, out=out, workspace_buf=wss), steps,
+                   warmup, flush)
+    ntok = int(WL.seq_lens(w).sum())
+    per_head = ntok * w.H * 2 * ww.R * 2
+    unique = ntok * 2 * ww.R * 2 + 2 * w.H * ww.R * w.Hd * 2
+    res["shared_latent_R%d" % ww.R] = {"us": t * 1e6, "per_head_reconstruction_bytes": per_head,
+                                       "unique_bytes": unique, "unique_gbs": unique / t / 1e9}
+    return res
+
+
+def _time_loop(fn, steps, warmup, flush):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / 1e3 / steps
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_step(w: WL.Workload, seed: int, heads: int, cache={}):
+    """One step of the float64 oracle on `heads` heads of every sequence (the
+    bounded CPU sample); returns the tokens*heads it processed."""
+    import oracle as O
+    key = (w.name, seed, heads)
+    if key not in cache:
+        lens = WL.seq_lens(w, seed)
+        q, _ = WL.query(w, seed)
+        bk, bv = WL.up_proj(w, seed)
+        blocks = {(b, h): WL.latent_cache_block(w, seed, b, h) for b in range(w.B) for h in range(heads)}
+        ai = WL.append_inputs(w, seed=seed, steps=1) if w.append_steps else None
+        cache[key] = (lens, q, bk, bv, blocks, ai)
+    lens, q, bk, bv, blocks, ai = cache[key]
+    if ai is not None:  # the append of the new token over the sampled heads
+        O.latent_project(ai.x[0], ai.A_k[:heads], ai.A_v[:heads], w.hadamard_block)
+    n = 0
+    for (b, h), (lk, sk, lv, sv) in blocks.items():
+        O.wsvd_decode_head(q[b, h], lk, sk, lv, sv, bk[h], bv[h], int(lens[b]), w.r, w.bits)
+        n += int(lens[b])
+    return n
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def run_cpu_sample(w: WL.Workload, budget_s: float, heads: int):
+    oracle_sample_step(w, 0, heads)  # build the inputs outside the timing
+    t0 = time.perf_counter()
+    n_tok, n_steps = 0, 0
+    while True:
+        n_tok += oracle_sample_step(w, 0, heads)
+        n_steps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n_tok / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n_steps} float64 oracle steps over {heads} of {w.H} heads of every sequence "
+                      f"({'append + ' if w.append_steps else ''}decode), {dt:.1f} s on "
+                      f"{len(os.sched_getaffinity(0))} host cores"}
+
+
+def sample_heads(w: WL.Workload) -> int:
+    """Heads per oracle step: about 12800 attended token-heads (tens of ms of float64 work)."""
+    per_head_tokens = w.B * (w.L_cap if not isinstance(w.lens, tuple) else sum(w.lens) // 2)
+    return max(1, min(w.H, 12800 // max(1, per_head_tokens)))
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="wsvd", choices=["wsvd", "reference"])
+    ap.add_argument("--workload", default="llava7b", choices=sorted(WL.PRESETS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-extras", action="store_true", help="skip the CPU baseline, e2e and comparison timings")
+    args = ap.parse_args()
+    w = WL.PRESETS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        heads = sample_heads(w)
+        for _ in range(max(0, args.warmup)):
+            oracle_sample_step(w, 0, heads)
+        t0 = time.perf_counter()
+        n = sum(oracle_sample_step(w, 0, heads) for _ in range(args.steps))
+        dt = time.perf_counter() - t0
+        v = n / dt
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": w.name, "sample_heads": heads},
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                 "sample": f"{heads} of {w.H} heads of every sequence per step"},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import rank_kv_cache_wsvd_b200 as W
+    W.load()  # fails loudly if the library is missing
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    st = WsvdStep(w, seed=rank)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    for _ in range(max(3, args.warmup)):
+        st.reset()
+        st.append()
+        st.decode()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.25)
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        st.reset()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        st.append()
+        e[1].record()
+        st.decode()
+        e[2].record()
+        evs.append(e)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    t_app = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    t_dec = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3
+    t_total = max_over_ranks(t_app + t_dec)
+    if int(st.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(st.err.item())}")
+
+    units = attended_tokens(w, st.lens_after) * args.steps * world
+    value = units / t_total
+    ms_per_step = t_total / args.steps * 1e3
+    peak, peak_kind = peaks()
+    dec_bytes = alg_bytes_decode(w, st.lens_after)
+    app_bytes = alg_bytes_append(w) if st.has_append else 0
+    per_app = t_app / args.steps
+    per_dec = t_dec / args.steps
+    if st.has_append and per_app >= per_dec:
+        dom, nbytes, dur, launches = "append", app_bytes, per_app, "wsvd append kernel (1 launch)"
+    else:
+        dom, nbytes, dur, launches = "decode", dec_bytes, per_dec, "wsvd decode (split-L kernel + combine)"
+    achieved = nbytes / dur / 1e9
+    traffic = ncu_traffic(dom, args.workload)
+
+    extras = {}
+    if not args.no_extras and rank == 0:
+        # end to end through the public API with host buffers (wall clock, host sync per step)
+        n_e2e = max(50, min(args.steps, 500))
+        for _ in range(10):
+            st.reset()
+            st.e2e_step()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_e2e):
+            st.reset()
+            st.e2e_step()
+            torch.cuda.current_stream().synchronize()
+        t_e2e = time.perf_counter() - t0
+        h2d, d2h = st.e2e_bytes()
+        extras["e2e"] = {"value": attended_tokens(w, st.lens_after) * n_e2e / t_e2e, "unit": UNIT,
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                         "us_per_step": t_e2e / n_e2e * 1e6, "timing": "host wall clock, stream sync per step"}
+        extras["comparisons_same_shape"] = time_comparisons(w, min(args.steps, 200), 5, flush)
+        extras["comparisons_same_shape"]["wsvd_decode"] = {"us": per_dec * 1e6, "alg_bytes": dec_bytes,
+                                                           "gbs": dec_bytes / per_dec / 1e9}
+        extras["cpu_baseline"] = run_cpu_sample(w, args.cpu_seconds, sample_heads(w))
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Hd": w.Hd, "r": w.r,
+                       "latent_bits": w.bits, "attended_tokens_per_seq": [int(x) for x in st.lens_after],
+                       "step": ("append + decode" if st.has_append else "decode"),
+                       "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
+            "step_us": ms_per_step * 1e3,
+            "breakdown_us": {"append": per_app * 1e6, "decode": per_dec * 1e6},
+            "hbm_gbs": (dec_bytes + app_bytes) / (t_total / args.steps) / 1e9,
+            "roofline": {"bound": "hbm", "kernel": launches, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                         "alg_bytes_per_launch": nbytes, "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS},
+            "gpu_launches": st.launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        for k in ("cpu_baseline", "e2e", "comparisons_same_shape"):
+            if k in extras:
+                line[k] = extras[k]
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * wsvd.h -- C ABI of the B200 (sm_100a) WSVD low-rank KV-cache decode library.
+ *
+ * The operations follow the WSVD summaries ("WSVD: Weighted Low-Rank
+ * Approximation for Fast and Efficient Execution of Low-Precision
+ * Vision-Language Models", gist.science paper 2604.02570):
+ *   - per-head factorisation W_Kh ~= A_Kh . B_Kh, A_Kh in R^{E x r},
+ *     B_Kh in R^{r x Hd}, and a per-head latent cache C_Kh of L x r values
+ *     (Arabic summary §2.a; German summary §2.A "Fein granulare SVD pro
+ *     Attention-Head");
+ *   - low-precision latents (W8A8 / W8A4) with the Hadamard rotation S1 on the
+ *     activations (German summary §2.C "Quantisierungsbewusstes Training");
+ *   - a fused decode that rebuilds K/V from latent tiles on chip and runs
+ *     q.K^T, softmax and the V product without writing K/V to memory
+ *     (Japanese summary §2.4 "システム実装：融合カーネル"; German §2.D).
+ *
+ * Conventions for every entry point:
+ *   - Array pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates, frees or synchronises; it launches on `stream` (a
+ *     cudaStream_t passed as void*, NULL = legacy default stream) and returns.
+ *   - 16-bit floats are passed as `const void*` (IEEE fp16 or bf16 bits).
+ *   - All arrays are dense row-major in the shapes given; every array pointer
+ *     must be 16-byte aligned.
+ *   - Return value: a wsvd_status.  Argument problems found on the host are
+ *     reported before anything is launched.  A launch failure returns
+ *     WSVD_ERR_CUDA (cudaGetLastError).  Problems found on the device (a
+ *     sequence length out of range, a full cache) never fault: the kernel ORs a
+ *     WSVD_DEVERR_* bit into the caller's int32 `*err` (device memory; may be
+ *     NULL) and treats the sequence as described per call.
+ *   - Outputs are written in full on every successful launch.  Results are
+ *     deterministic: the same inputs, shapes and device give the same bits.
+ */
+#ifndef WSVD_B200_H
+#define WSVD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WSVD_OK = 0,
+  WSVD_ERR_INVALID_ARG = 1,          /* null pointer, bad size, misaligned pointer */
+  WSVD_ERR_UNSUPPORTED = 2,          /* valid but not built (e.g. row bytes not a multiple of 16) */
+  WSVD_ERR_CUDA = 3,                 /* the CUDA runtime reported an error */
+  WSVD_ERR_WORKSPACE_TOO_SMALL = 4   /* workspace_bytes below the matching *_workspace_size() */
+} wsvd_status;
+
+/* 16-bit float formats for q and x. */
+enum { WSVD_DTYPE_FP16 = 0, WSVD_DTYPE_BF16 = 1 };
+
+/* Bits ORed into the caller's device error word. */
+enum {
+  WSVD_DEVERR_LEN_RANGE = 1,     /* decode: seq_lens[b] < 0 or > L_cap; that sequence's output is 0 */
+  WSVD_DEVERR_CACHE_FULL = 2,    /* append: seq_lens[b] >= L_cap (or < 0); row not written, length kept */
+  WSVD_DEVERR_PIPE_TIMEOUT = 4   /* a pipeline wait exceeded its time limit; outputs are not valid */
+};
+
+/* Human-readable name of a wsvd_status. Never NULL. */
+const char* wsvd_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int wsvd_abi_version(void);
+
+/* ---------------------------------------------------------------- footprint
+ * Bytes of a per-head latent cache: K and V codes (L_cap x r per head, `bits`
+ * per code) plus one fp16 scale per token per head for each
+ * (Arabic summary §2.a: the latent footprint per head is L x r).            */
+size_t wsvd_cache_bytes(int B, int H, int L_cap, int r, int bits);
+/* Bytes of a conventional shared fp16 latent: L_cap x R for K and for V
+ * (Arabic summary §2.a: the shared latent is L x R).                        */
+size_t shared_cache_bytes(int B, int L_cap, int R);
+/* Bytes of a dense fp16 K/V cache (L_cap x Hd per head, K and V).           */
+size_t dense_cache_bytes(int B, int H, int L_cap, int Hd);
+
+/* ---------------------------------------------------------------- WSVD decode
+ * One decode step of attention over a per-head low-rank, low-precision cache
+ * (Japanese §2.4 / German §2.D, the fused low-rank flash-decoding kernel).
+ *
+ * For each sequence b < B and head h < H, with n = seq_lens[b] tokens:
+ *   lat_K[l] = code_K[b,h,l,:] * scale_k[b,h,l]      (l < n; likewise V)
+ *   K = lat_K . B_k[h],  V = lat_V . B_v[h]          (n x Hd, never stored)
+ *   out[b,h,:] = softmax(K . q[b,h,:] * softmax_scale) . V
+ * computed in the reassociated form q' = B_k[h] . q, score_l = s_K,l
+ * (code_K,l . q'), out = ((sum_l p_l s_V,l code_V,l) / sum_l p_l) . B_v[h],
+ * fp32 accumulation.  A sequence with n = 0 gets out = 0.
+ *
+ *   B, H, Hd, r, bits : batch, heads, head dim (multiple of 32, <= 256), rank,
+ *                       bits per code (8 or 4).  Row bytes r*bits/8 must be
+ *                       16, 32, 64 or 128 (else WSVD_ERR_UNSUPPORTED).
+ *   L_cap             : rows per (b, h) in the cache; multiple of 8.
+ *   seq_lens  [B]            int32: tokens used per sequence (0 <= n <= L_cap).
+ *   q         [B][H][Hd]     fp16 or bf16 (q_dtype).
+ *   lat_k, lat_v [B][H][L_cap][r*bits/8] uint8: int8 two's complement codes,
+ *                            or int4 with element 2j in bits 0-3 and 2j+1 in
+ *                            bits 4-7 of byte j (two's complement nibbles).
+ *   scale_k, scale_v [B][H][L_cap] fp16 per-token scales.
+ *   B_k, B_v  [H][r][Hd]     fp16.
+ *   softmax_scale            0 selects 1/sqrt(Hd).
+ *   out       [B][H][Hd]     float32, written.
+ *   workspace                device scratch of at least
+ *                            wsvd_decode_workspace_size(B, H, r) bytes; no
+ *                            initial contents required; clobbered.
+ *   err                      optional device int32; WSVD_DEVERR_LEN_RANGE.
+ * Rows >= seq_lens[b] are never used: their bytes may hold anything.        */
+size_t wsvd_decode_workspace_size(int B, int H, int r);
+int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                          const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
+                          const void* scale_k, const void* scale_v, const void* B_k, const void* B_v,
+                          float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                          int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------- latent append
+ * Writes one new token per sequence into the latent cache (the projection of
+ * the new token through A_Kh / A_Vh, German §2.A, after the Hadamard rotation
+ * S1 of German §2.C), then advances its length:
+ *   x~ = x[b,:] . blockdiag(H_blk / sqrt(blk))   (Sylvester order, blk = hadamard_block)
+ *   c_K = x~ . A_k[h],  c_V = x~ . A_v[h]         (r values each, fp32)
+ *   per (b, h, K|V): scale = fp16(max_j |c_j| / Q)  (Q = 127 int8, 7 int4),
+ *   code_j = clamp(round_half_even(c_j / scale), -Q, Q) (scale 0 -> codes 0);
+ *   row seq_lens[b] of lat_k/lat_v/scale_k/scale_v is written, then
+ *   seq_lens[b] += 1.
+ * A sequence with seq_lens[b] >= L_cap (or < 0) is not written and not
+ * advanced; WSVD_DEVERR_CACHE_FULL is raised.
+ *
+ *   x          [B][E]       bf16 or fp16 (x_dtype); E % hadamard_block == 0.
+ *   A_k, A_v   [H][E][r]    fp16.
+ *   hadamard_block          power of two in [2, 1024] (1 = no rotation).
+ *   E                       multiple of 8 * hadamard_block, at most 65536.
+ *   B                       1..16.
+ *   seq_lens   [B]          int32, read and advanced in place.
+ *   workspace               at least wsvd_append_workspace_size() bytes of
+ *                           device memory that is ZERO before the first call
+ *                           (cudaMemset once); every call leaves it zero.
+ *                           Calls that share a workspace must not overlap.
+ * Rows other than seq_lens[b] are never written.                             */
+size_t wsvd_append_workspace_size(void);
+int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block,
+                       const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
+                       uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
+                       size_t workspace_bytes, int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------- comparison: dense decode
+ * The flash-decoding baseline the pages compare against (German §4
+ * "Ergebnisse"): out[b,h] = softmax(K[b,h,:n] . q[b,h] * softmax_scale) . V[b,h,:n]
+ * over a dense fp16 cache.  K, V [B][H][L_cap][Hd] fp16 (Hd in {64, 128, 256}).
+ * Other arguments as for wsvd_decode_attention.                              */
+size_t dense_decode_workspace_size(int B, int H, int Hd);
+int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q,
+                           int q_dtype, const void* K, const void* V, float softmax_scale, float* out,
+                           void* workspace, size_t workspace_bytes, int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------- comparison: shared-latent SVD decode
+ * The conventional SVD decode the pages measure against (Japanese §1, German
+ * §1): one latent per sequence shared by all heads, lat_k, lat_v
+ * [B][L_cap][R] fp16, and per-head up-projections B_k, B_v [H][R][Hd] fp16.
+ * Every head reads the whole shared latent:
+ *   K_h = lat_k[b,:n] . B_k[h], V_h = lat_v[b,:n] . B_v[h],
+ *   out[b,h] = softmax(K_h . q[b,h] * softmax_scale) . V_h.
+ * R in {128, 256, 512, 1024}.  Other arguments as for wsvd_decode_attention. */
+size_t shared_decode_workspace_size(int B, int H, int R);
+int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32_t* seq_lens,
+                             const void* q, int q_dtype, const void* lat_k, const void* lat_v,
+                             const void* B_k, const void* B_v, float softmax_scale, float* out,
+                             void* workspace, size_t workspace_bytes, int32_t* err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WSVD_B200_H */

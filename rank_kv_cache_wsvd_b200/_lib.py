@@ -1,0 +1,230 @@
+"""ctypes binding of libwsvd_b200.so: argument marshalling only.
+
+Every operation runs in the library's CUDA kernels; PyTorch only provides
+device memory and the current stream.  There is no CPU fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwsvd_b200.so")
+
+WSVD_DTYPE_FP16 = 0
+WSVD_DTYPE_BF16 = 1
+DEVERR_LEN_RANGE = 1
+DEVERR_CACHE_FULL = 2
+DEVERR_PIPE_TIMEOUT = 4
+
+_c_int, _c_size, _c_float, _p = ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
+
+# name -> (restype, argtypes); every symbol the public header declares.
+SIGNATURES = {
+    "wsvd_status_string": (ctypes.c_char_p, [_c_int]),
+    "wsvd_abi_version": (_c_int, []),
+    "wsvd_cache_bytes": (_c_size, [_c_int] * 5),
+    "shared_cache_bytes": (_c_size, [_c_int] * 3),
+    "dense_cache_bytes": (_c_size, [_c_int] * 4),
+    "wsvd_decode_workspace_size": (_c_size, [_c_int] * 3),
+    "dense_decode_workspace_size": (_c_size, [_c_int] * 3),
+    "shared_decode_workspace_size": (_c_size, [_c_int] * 3),
+    "wsvd_append_workspace_size": (_c_size, []),
+    "wsvd_decode_attention": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size,
+                                                                                        _p, _p]),
+    "wsvd_latent_append": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 7 + [_p, _c_size, _p, _p]),
+    "dense_decode_attention": (_c_int, [_c_int] * 4 + [_p, _p, _c_int, _p, _p, _c_float, _p, _p, _c_size, _p, _p]),
+    "shared_latent_svd_decode": (_c_int, [_c_int] * 5 + [_p, _p, _c_int] + [_p] * 4 + [_c_float, _p, _p, _c_size,
+                                                                                         _p, _p]),
+}
+
+_lib = None
+
+
+class WsvdError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once) and declare every entry point's signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise WsvdError(f"{path} is missing: build it with `python -m rank_kv_cache_wsvd_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        msg = load().wsvd_status_string(status).decode()
+        raise WsvdError(f"{what}: {msg} (status {status})")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise WsvdError("all tensors must be CUDA tensors")
+    if not t.is_contiguous():
+        raise WsvdError("all tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return WSVD_DTYPE_FP16
+    if t.dtype == torch.bfloat16:
+        return WSVD_DTYPE_BF16
+    raise WsvdError(f"expected fp16 or bf16, got {t.dtype}")
+
+
+def _expect(t: torch.Tensor, dtype, shape, name: str) -> None:
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise WsvdError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+# ----------------------------------------------------------------------------- sizes
+def wsvd_cache_bytes(B, H, L_cap, r, bits) -> int:
+    return load().wsvd_cache_bytes(B, H, L_cap, r, bits)
+
+
+def shared_cache_bytes(B, L_cap, R) -> int:
+    return load().shared_cache_bytes(B, L_cap, R)
+
+
+def dense_cache_bytes(B, H, L_cap, Hd) -> int:
+    return load().dense_cache_bytes(B, H, L_cap, Hd)
+
+
+def wsvd_decode_workspace_size(B, H, r) -> int:
+    return load().wsvd_decode_workspace_size(B, H, r)
+
+
+def dense_decode_workspace_size(B, H, Hd) -> int:
+    return load().dense_decode_workspace_size(B, H, Hd)
+
+
+def shared_decode_workspace_size(B, H, R) -> int:
+    return load().shared_decode_workspace_size(B, H, R)
+
+
+def wsvd_append_workspace_size() -> int:
+    return load().wsvd_append_workspace_size()
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Caller-owned scratch buffer (uint8), zero-filled."""
+    return torch.zeros(max(16, nbytes), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------- decode
+def wsvd_decode_attention(q, lat_k, lat_v, scale_k, scale_v, B_k, B_v, seq_lens, bits: int,
+                          softmax_scale: float = 0.0, out=None, workspace_buf=None, err=None, stream=None):
+    """Decode step over a per-head low-rank cache; returns out [B][H][Hd] fp32."""
+    lib = load()
+    B, H, Hd = q.shape
+    L_cap, rb = lat_k.shape[2], lat_k.shape[3]
+    r = rb * 8 // bits
+    _expect(lat_k, torch.uint8, (B, H, L_cap, rb), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, rb), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _expect(B_k, torch.float16, (H, r, Hd), "B_k")
+    _expect(B_v, torch.float16, (H, r, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, H, Hd), "out")
+    need = lib.wsvd_decode_workspace_size(B, H, r)
+    if workspace_buf is None:
+        workspace_buf = workspace(need, q.device)
+    st = lib.wsvd_decode_attention(B, H, Hd, r, bits, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q),
+                                   _ptr(lat_k), _ptr(lat_v), _ptr(scale_k), _ptr(scale_v), _ptr(B_k), _ptr(B_v),
+                                   float(softmax_scale), _ptr(out), _ptr(workspace_buf), workspace_buf.numel(),
+                                   _ptr(err), _stream(stream))
+    _check(st, "wsvd_decode_attention")
+    return out
+
+
+def dense_decode_attention(q, K, V, seq_lens, softmax_scale: float = 0.0, out=None, workspace_buf=None,
+                           err=None, stream=None):
+    lib = load()
+    B, H, Hd = q.shape
+    L_cap = K.shape[2]
+    _expect(K, torch.float16, (B, H, L_cap, Hd), "K")
+    _expect(V, torch.float16, (B, H, L_cap, Hd), "V")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    need = lib.dense_decode_workspace_size(B, H, Hd)
+    if workspace_buf is None:
+        workspace_buf = workspace(need, q.device)
+    st = lib.dense_decode_attention(B, H, Hd, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q), _ptr(K), _ptr(V),
+                                    float(softmax_scale), _ptr(out), _ptr(workspace_buf), workspace_buf.numel(),
+                                    _ptr(err), _stream(stream))
+    _check(st, "dense_decode_attention")
+    return out
+
+
+def shared_latent_svd_decode(q, lat_k, lat_v, B_k, B_v, seq_lens, softmax_scale: float = 0.0, out=None,
+                             workspace_buf=None, err=None, stream=None):
+    lib = load()
+    B, H, Hd = q.shape
+    L_cap, R = lat_k.shape[1], lat_k.shape[2]
+    _expect(lat_k, torch.float16, (B, L_cap, R), "lat_k")
+    _expect(lat_v, torch.float16, (B, L_cap, R), "lat_v")
+    _expect(B_k, torch.float16, (H, R, Hd), "B_k")
+    _expect(B_v, torch.float16, (H, R, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    need = lib.shared_decode_workspace_size(B, H, R)
+    if workspace_buf is None:
+        workspace_buf = workspace(need, q.device)
+    st = lib.shared_latent_svd_decode(B, H, Hd, R, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q), _ptr(lat_k),
+                                      _ptr(lat_v), _ptr(B_k), _ptr(B_v), float(softmax_scale), _ptr(out),
+                                      _ptr(workspace_buf), workspace_buf.numel(), _ptr(err), _stream(stream))
+    _check(st, "shared_latent_svd_decode")
+    return out
+
+
+# ----------------------------------------------------------------------------- append
+def wsvd_latent_append(x, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, bits: int,
+                       hadamard_block: int = 128, workspace_buf=None, err=None, stream=None) -> None:
+    """Quantise one new token per sequence into the cache and advance seq_lens (in place).
+
+    `workspace_buf` must be zero before its first use (the default allocation is);
+    every call leaves it zero."""
+    lib = load()
+    B, E = x.shape
+    H, _, r = A_k.shape
+    L_cap, rb = lat_k.shape[2], lat_k.shape[3]
+    _expect(A_k, torch.float16, (H, E, r), "A_k")
+    _expect(A_v, torch.float16, (H, E, r), "A_v")
+    _expect(lat_k, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if workspace_buf is None:
+        workspace_buf = workspace(lib.wsvd_append_workspace_size(), x.device)
+    st = lib.wsvd_latent_append(B, H, E, r, bits, L_cap, hadamard_block, _ptr(x), _dtype_code(x), _ptr(A_k),
+                                _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k), _ptr(scale_v),
+                                _ptr(workspace_buf), workspace_buf.numel(), _ptr(err), _stream(stream))
+    _check(st, "wsvd_latent_append")

@@ -1,0 +1,213 @@
+// C ABI of the library: host-side validation, split planning and launches.
+// No allocation, no synchronisation; every launch goes to the caller's stream.
+#include <math.h>
+
+#include "wsvd_internal.h"
+
+using namespace wsvd;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline float resolve_scale(float softmax_scale, int Hd) {
+  return softmax_scale != 0.f ? softmax_scale : (float)(1.0 / sqrt((double)Hd));
+}
+
+inline size_t partial_bytes(int B, int H, int W) {
+  return ((size_t)kMaxDecodeCtas + (size_t)B * H) * ((size_t)W + 2) * sizeof(float);
+}
+
+// Shared validation of the decode entry points.
+int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
+                 const float* out, const void* workspace) {
+  if (B < 0 || H < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
+  if (B == 0) return WSVD_OK;
+  if (B > 4096) return WSVD_ERR_UNSUPPORTED;
+  if (Hd < 32 || Hd > 256 || Hd % 32) return WSVD_ERR_UNSUPPORTED;
+  if (L_cap % 8) return WSVD_ERR_UNSUPPORTED;
+  if (q_dtype != WSVD_DTYPE_FP16 && q_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
+  if (!seq_lens || !q || !out || !workspace) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return WSVD_ERR_INVALID_ARG;
+  return WSVD_OK;
+}
+
+int run_split(int codec, int rowbytes, int qmode, SplitArgs a, const __half* Bv, float* out, int Hd,
+              cudaStream_t stream) {
+  a.ctas = split_decode_grid(codec, rowbytes, qmode, a.B, a.H, a.L_cap);
+  if (a.ctas < 1) return WSVD_ERR_UNSUPPORTED;
+  int tile = 0;
+  if (launch_split_decode(codec, rowbytes, qmode, a, &tile, stream) != cudaSuccess) return WSVD_ERR_CUDA;
+  CombineArgs c{a.B, a.H, Hd, a.W, a.L_cap, a.ctas, tile, a.seq_lens, a.partials, Bv, out, a.err};
+  if (launch_combine(c, stream) != cudaSuccess) return WSVD_ERR_CUDA;
+  return WSVD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wsvd_status_string(int status) {
+  switch (status) {
+    case WSVD_OK: return "ok";
+    case WSVD_ERR_INVALID_ARG: return "invalid argument";
+    case WSVD_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case WSVD_ERR_CUDA: return "CUDA runtime error";
+    case WSVD_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int wsvd_abi_version(void) { return 100; }
+
+size_t wsvd_cache_bytes(int B, int H, int L_cap, int r, int bits) {
+  if (B < 0 || H < 0 || L_cap < 0 || r < 0 || (bits != 8 && bits != 4)) return 0;
+  return (size_t)B * H * L_cap * ((size_t)2 * r * bits / 8 + 2 * 2);
+}
+
+size_t shared_cache_bytes(int B, int L_cap, int R) {
+  if (B < 0 || L_cap < 0 || R < 0) return 0;
+  return (size_t)B * L_cap * 2 * R * 2;
+}
+
+size_t dense_cache_bytes(int B, int H, int L_cap, int Hd) {
+  if (B < 0 || H < 0 || L_cap < 0 || Hd < 0) return 0;
+  return (size_t)B * H * L_cap * 2 * Hd * 2;
+}
+
+size_t wsvd_decode_workspace_size(int B, int H, int r) {
+  if (B < 0 || H < 0 || r < 1) return 0;
+  return partial_bytes(B, H, r);
+}
+
+size_t dense_decode_workspace_size(int B, int H, int Hd) {
+  if (B < 0 || H < 0 || Hd < 1) return 0;
+  return partial_bytes(B, H, Hd);
+}
+
+size_t shared_decode_workspace_size(int B, int H, int R) {
+  if (B < 0 || H < 0 || R < 1) return 0;
+  return partial_bytes(B, H, R) + (size_t)B * H * R * sizeof(float);
+}
+
+int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                          const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
+                          const void* scale_k, const void* scale_v, const void* B_k, const void* B_v,
+                          float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                          int32_t* err, void* stream) {
+  int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
+  if (st != WSVD_OK || B == 0) return st;
+  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
+  if (r < 1 || (r * bits) % 8) return WSVD_ERR_INVALID_ARG;
+  const int rowbytes = r * bits / 8;
+  if (rowbytes % 16 || split_decode_tile_tokens(bits == 8 ? kCodecI8 : kCodecI4, rowbytes) == 0)
+    return WSVD_ERR_UNSUPPORTED;
+  if (!lat_k || !lat_v || !scale_k || !scale_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
+      !aligned16(B_k) || !aligned16(B_v))
+    return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < wsvd_decode_workspace_size(B, H, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+
+  SplitArgs a{};
+  a.B = B; a.H = H; a.Hd = Hd; a.W = r; a.L_cap = L_cap; a.heads_share = 0;
+  a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
+  a.lat_k = lat_k; a.lat_v = lat_v;
+  a.scale_k = static_cast<const __half*>(scale_k); a.scale_v = static_cast<const __half*>(scale_v);
+  a.Bk = static_cast<const __half*>(B_k); a.qglobal = nullptr;
+  a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
+  a.partials = static_cast<float*>(workspace); a.err = err;
+  return run_split(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj, a, static_cast<const __half*>(B_v), out,
+                   Hd, as_stream(stream));
+}
+
+int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
+                           const void* K, const void* V, float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, int32_t* err, void* stream) {
+  int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
+  if (st != WSVD_OK || B == 0) return st;
+  const int rowbytes = Hd * 2;
+  if (split_decode_tile_tokens(kCodecF16, rowbytes) == 0) return WSVD_ERR_UNSUPPORTED;
+  if (!K || !V) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V)) return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < dense_decode_workspace_size(B, H, Hd)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+
+  SplitArgs a{};
+  a.B = B; a.H = H; a.Hd = Hd; a.W = Hd; a.L_cap = L_cap; a.heads_share = 0;
+  a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
+  a.lat_k = static_cast<const uint8_t*>(K); a.lat_v = static_cast<const uint8_t*>(V);
+  a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
+  a.partials = static_cast<float*>(workspace); a.err = err;
+  return run_split(kCodecF16, rowbytes, kQDirect, a, nullptr, out, Hd, as_stream(stream));
+}
+
+int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32_t* seq_lens, const void* q,
+                             int q_dtype, const void* lat_k, const void* lat_v, const void* B_k, const void* B_v,
+                             float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                             int32_t* err, void* stream) {
+  int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
+  if (st != WSVD_OK || B == 0) return st;
+  const int rowbytes = R * 2;
+  if (R < 1 || split_decode_tile_tokens(kCodecF16, rowbytes) == 0) return WSVD_ERR_UNSUPPORTED;
+  {
+    // the shared path instantiates R = 128, 256, 512, 1024 only
+    if (R != 128 && R != 256 && R != 512 && R != 1024) return WSVD_ERR_UNSUPPORTED;
+  }
+  if (!lat_k || !lat_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(B_k) || !aligned16(B_v)) return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < shared_decode_workspace_size(B, H, R)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+
+  float* partials = static_cast<float*>(workspace);
+  float* qglobal = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + partial_bytes(B, H, R));
+  if (launch_shared_qproj(B, H, Hd, R, q, q_dtype, static_cast<const __half*>(B_k), qglobal,
+                          as_stream(stream)) != cudaSuccess)
+    return WSVD_ERR_CUDA;
+  SplitArgs a{};
+  a.B = B; a.H = H; a.Hd = Hd; a.W = R; a.L_cap = L_cap; a.heads_share = 1;
+  a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
+  a.lat_k = static_cast<const uint8_t*>(lat_k); a.lat_v = static_cast<const uint8_t*>(lat_v);
+  a.qglobal = qglobal;
+  a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
+  a.partials = partials; a.err = err;
+  return run_split(kCodecF16, rowbytes, kQGlobal, a, static_cast<const __half*>(B_v), out, Hd,
+                   as_stream(stream));
+}
+
+size_t wsvd_append_workspace_size(void) { return 256; }
+
+int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x,
+                       int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens, uint8_t* lat_k,
+                       uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace, size_t workspace_bytes,
+                       int32_t* err, void* stream) {
+  if (B < 0 || H < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
+  if (B == 0) return WSVD_OK;
+  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
+  if (x_dtype != WSVD_DTYPE_FP16 && x_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
+  if (hadamard_block < 1 || hadamard_block > 1024 || (hadamard_block & (hadamard_block - 1)))
+    return WSVD_ERR_INVALID_ARG;
+  if (E % hadamard_block) return WSVD_ERR_INVALID_ARG;
+  if (B > 16 || r % 8 || r > 128 || (r * bits / 8) % 4 || E > 65536) return WSVD_ERR_UNSUPPORTED;
+  if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
+    return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
+      !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
+    return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < wsvd_append_workspace_size()) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+  const int cl = append_cluster_size(E, hadamard_block);
+  if (cl < 1) return WSVD_ERR_UNSUPPORTED;
+  if (append_smem_bytes(B, E, r, cl) > 200 * 1024) return WSVD_ERR_UNSUPPORTED;
+
+  AppendArgs a{};
+  a.B = B; a.H = H; a.E = E; a.r = r; a.bits = bits; a.L_cap = L_cap; a.blk = hadamard_block; a.cluster = cl;
+  a.hnorm = (float)(1.0 / sqrt((double)hadamard_block));
+  a.x = x; a.x_dtype = x_dtype;
+  a.Ak = static_cast<const __half*>(A_k); a.Av = static_cast<const __half*>(A_v);
+  a.seq_lens = seq_lens; a.lat_k = lat_k; a.lat_v = lat_v;
+  a.scale_k = static_cast<__half*>(scale_k); a.scale_v = static_cast<__half*>(scale_v);
+  a.counter = static_cast<int32_t*>(workspace); a.err = err;
+  if (launch_append(a, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
+  return WSVD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+// Device helpers shared by the sm_100a kernels: mbarrier + 1-D bulk-copy (TMA)
+// staging with bounded waits, and exact integer -> float32 code conversion.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wsvd_internal.h"
+
+namespace wsvd {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+// ---------------------------------------------------------------- shared memory / mbarrier
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns` of wall
+// time.  Returns false on timeout; the caller records WSVD_DEVERR_PIPE_TIMEOUT
+// and leaves the pipeline instead of spinning forever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing `bytes` of
+// transaction count on `bar`.  Both addresses 16-byte aligned, bytes % 16 == 0.
+// No multicast: the destination is this CTA only.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// L2 policy for data read exactly once (latent / KV streams): evict first, so
+// the small reused operands (B matrices, q) stay resident.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void set_err(int32_t* err, int32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ---------------------------------------------------------------- code conversion
+// int8 codes -> float32, exact.  Each byte is moved into the low mantissa byte
+// of 2^23 (after flipping its sign bit, so it reads as c + 128); subtracting
+// 2^23 + 128 leaves c exactly (IEEE-754 layout: integers below 2^24 are exact).
+__device__ __forceinline__ float2 i8_pair(uint32_t xflip, int first) {
+  const uint32_t sel0 = 0x7540u | (uint32_t)first;
+  const uint32_t sel1 = 0x7540u | (uint32_t)(first + 1);
+  float2 f;
+  f.x = __uint_as_float(__byte_perm(xflip, 0x4B000000u, sel0));
+  f.y = __uint_as_float(__byte_perm(xflip, 0x4B000000u, sel1));
+  return __fadd2_rn(f, make_float2(-8388736.f, -8388736.f));
+}
+
+// int4 codes (two's complement nibbles, element k in bits 4k..4k+3 of the word)
+// -> float32, exact.  Same mantissa trick with offset 8.
+__device__ __forceinline__ float2 i4_pair(uint32_t xflip, int k) {
+  float2 f;
+  f.x = __uint_as_float(((xflip >> (4 * k)) & 0xFu) | 0x4B000000u);
+  f.y = __uint_as_float(((xflip >> (4 * k + 4)) & 0xFu) | 0x4B000000u);
+  return __fadd2_rn(f, make_float2(-8388616.f, -8388616.f));
+}
+
+__device__ __forceinline__ float2 h2_pair(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+__device__ __forceinline__ float load_q_elem(const void* q, int dtype, size_t i) {
+  const uint16_t u = reinterpret_cast<const uint16_t*>(q)[i];
+  if (dtype == WSVD_DTYPE_BF16) return __uint_as_float(((uint32_t)u) << 16);
+  return __half2float(__ushort_as_half(u));
+}
+
+}  // namespace wsvd

@@ -1,0 +1,84 @@
+// Internal declarations shared by the kernel translation units and the C ABI layer.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/wsvd.h"
+
+namespace wsvd {
+
+// Pipeline waits give up after one second of wall time (see mbar_wait_bounded).
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+// Split-L decode: 8 consumer warps + 1 producer warp per CTA.
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kDecodeThreads = kConsumerThreads + 32;
+constexpr int kStages = 4;
+// Upper bound on the persistent grid; sizes the partial-result workspace.
+constexpr int kMaxDecodeCtas = 2048;
+
+enum Codec { kCodecI8 = 0, kCodecI4 = 1, kCodecF16 = 2 };
+enum QMode { kQProj = 0, kQDirect = 1, kQGlobal = 2 };
+
+// Arguments of the persistent split-L decode kernel (one struct for every codec).
+struct SplitArgs {
+  int B, H, Hd, W;       // W: latent width per token (r, Hd or R)
+  int L_cap;
+  int ctas;              // persistent grid size C
+  int heads_share;       // 1: the latent rows of (b, h) are the rows of b (shared-latent path)
+  const int32_t* seq_lens;
+  const void* q;
+  int q_dtype;
+  const uint8_t* lat_k;  // rows of W codes / values
+  const uint8_t* lat_v;
+  const __half* scale_k; // per-token scales (quantised codecs only)
+  const __half* scale_v;
+  const __half* Bk;      // [H][W][Hd] (kQProj)
+  const float* qglobal;  // [B][H][W] (kQGlobal)
+  float qscale;          // softmax_scale * log2(e)
+  float* partials;       // [(ctas + B*H)][W + 2]
+  int32_t* err;
+};
+
+struct CombineArgs {
+  int B, H, Hd, W, L_cap, ctas, tile;
+  const int32_t* seq_lens;
+  const float* partials;
+  const __half* Bv;      // [H][W][Hd], or nullptr for the dense path (W == Hd)
+  float* out;            // [B][H][Hd]
+  int32_t* err;
+};
+
+// Host launchers (decode.cu, shared.cu, append.cu).  Return a cudaError_t.
+cudaError_t launch_split_decode(int codec, int rowbytes, int qmode, const SplitArgs& a, int* tile_tokens,
+                                cudaStream_t stream);
+int split_decode_tile_tokens(int codec, int rowbytes);
+int split_decode_grid(int codec, int rowbytes, int qmode, int B, int H, int L_cap);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+cudaError_t launch_shared_qproj(int B, int H, int Hd, int R, const void* q, int q_dtype, const __half* Bk,
+                                float* qglobal, cudaStream_t stream);
+
+struct AppendArgs {
+  int B, H, E, r, bits, L_cap, blk, cluster;
+  float hnorm;           // 1/sqrt(blk), correctly rounded
+  const void* x;
+  int x_dtype;
+  const __half* Ak;
+  const __half* Av;
+  int32_t* seq_lens;
+  uint8_t* lat_k;
+  uint8_t* lat_v;
+  __half* scale_k;
+  __half* scale_v;
+  int32_t* counter;
+  int32_t* err;
+};
+int append_cluster_size(int E, int blk);
+size_t append_smem_bytes(int B, int E, int r, int cluster);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+}  // namespace wsvd

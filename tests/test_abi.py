@@ -1,0 +1,100 @@
+"""The C-ABI library loads on a host without a GPU, exports every symbol the
+public header declares, and its host-only entry points (sizes, validation)
+behave as documented.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+import rank_kv_cache_wsvd_b200 as W
+from rank_kv_cache_wsvd_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wsvd.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\**([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from rank_kv_cache_wsvd_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_symbols_are_exported_and_bound(lib):
+    names = _declared_functions()
+    assert len(names) >= 12, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in wsvd.h but not exported"
+        assert n in _lib.SIGNATURES, f"{n} has no Python binding signature"
+    assert set(_lib.SIGNATURES) == set(names)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.wsvd_abi_version() == 100
+    assert lib.wsvd_status_string(0) == b"ok"
+    assert lib.wsvd_status_string(4) == b"workspace too small"
+    assert lib.wsvd_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("B,H,L,r,bits", [(1, 4, 256, 16, 8), (16, 32, 4096, 32, 4), (4, 32, 32768, 64, 8)])
+def test_cache_byte_counts_match_oracle(lib, B, H, L, r, bits):
+    assert W.wsvd_cache_bytes(B, H, L, r, bits) == O.wsvd_cache_bytes(B, H, L, r, bits)
+    assert W.shared_cache_bytes(B, L, 512) == O.shared_cache_bytes(B, L, 512)
+    assert W.dense_cache_bytes(B, H, L, 128) == O.dense_cache_bytes(B, H, L, 128)
+
+
+def test_workspace_sizes_hold_only_partials(lib):
+    """The decode workspace holds split partials (r + 2 floats per slot), never
+    an L x Hd buffer: reconstructed K/V are not materialised."""
+    B, H, r, L = 4, 32, 32, 32768
+    ws = W.wsvd_decode_workspace_size(B, H, r)
+    assert ws == (2048 + B * H) * (r + 2) * 4
+    assert ws < B * H * L * 128 * 2 / 100  # far below one reconstructed K
+    assert W.dense_decode_workspace_size(B, H, 128) == (2048 + B * H) * 130 * 4
+    assert W.shared_decode_workspace_size(B, H, 512) == (2048 + B * H) * 514 * 4 + B * H * 512 * 4
+    assert W.wsvd_append_workspace_size() == 256
+
+
+def test_host_validation_rejects_before_launch(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    # null seq_lens
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 8, 256, None, p, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                     None, None) == 1
+    # bits not in {4, 8}
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 6, 256, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                     None, None) == 1
+    # row bytes not a multiple of 16 (r = 16, int4 -> 8 bytes)
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 4, 256, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                     None, None) == 2
+    # L_cap not a multiple of 8
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 8, 257, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                     None, None) == 2
+    # misaligned pointer
+    bad = ctypes.c_void_p(24)
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 8, 256, p, bad, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                     None, None) == 1
+    # workspace too small
+    assert lib.wsvd_decode_attention(1, 4, 64, 16, 8, 256, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 64,
+                                     None, None) == 4
+    # empty batch is a no-op
+    assert lib.wsvd_decode_attention(0, 4, 64, 16, 8, 256, None, None, 0, None, None, None, None, None, None,
+                                     0.0, None, None, 0, None, None) == 0
+    # append: hadamard block not a power of two / E not a multiple of it / B too large
+    assert lib.wsvd_latent_append(1, 4, 256, 16, 8, 8, 96, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 1
+    assert lib.wsvd_latent_append(1, 4, 200, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 1
+    assert lib.wsvd_latent_append(17, 4, 256, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 2
+    assert lib.wsvd_latent_append(1, 4, 256, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 8, None, None) == 4
+    # dense / shared: unsupported widths
+    assert lib.dense_decode_attention(1, 4, 48, 256, p, p, 0, p, p, 0.0, p, p, 1 << 22, None, None) == 2
+    assert lib.shared_latent_svd_decode(1, 4, 128, 384, 256, p, p, 0, p, p, p, p, 0.0, p, p, 1 << 24,
+                                        None, None) == 2
