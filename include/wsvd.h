@@ -87,9 +87,10 @@ size_t dense_cache_bytes(int B, int H, int L_cap, int Hd);
  * (code_K,l . q'), out = ((sum_l p_l s_V,l code_V,l) / sum_l p_l) . B_v[h],
  * fp32 accumulation.  A sequence with n = 0 gets out = 0.
  *
- *   B, H, Hd, r, bits : batch, heads, head dim (multiple of 32, <= 256), rank,
+ *   B, H, Hd, r, bits : batch (<= 4096), heads, head dim (32, 64, 128 or 256), rank,
  *                       bits per code (8 or 4).  Row bytes r*bits/8 must be
- *                       16, 32, 64 or 128 (else WSVD_ERR_UNSUPPORTED).
+ *                       16, 32, 64 or 128 for int8 and 16, 32 or 64 for int4
+ *                       (else WSVD_ERR_UNSUPPORTED).
  *   L_cap             : rows per (b, h) in the cache; multiple of 8.
  *   seq_lens  [B]            int32: tokens used per sequence (0 <= n <= L_cap).
  *   q         [B][H][Hd]     fp16 or bf16 (q_dtype).
@@ -101,8 +102,12 @@ size_t dense_cache_bytes(int B, int H, int L_cap, int Hd);
  *   softmax_scale            0 selects 1/sqrt(Hd).
  *   out       [B][H][Hd]     float32, written.
  *   workspace                device scratch of at least
- *                            wsvd_decode_workspace_size(B, H, r) bytes; no
- *                            initial contents required; clobbered.
+ *                            wsvd_decode_workspace_size(B, H, r) bytes that is
+ *                            ZERO before the first call (cudaMemset once):
+ *                            it holds split partials and one completion
+ *                            counter per (b, h), and every call leaves the
+ *                            counters zero.  Calls that share a workspace must
+ *                            not overlap on the GPU.
  *   err                      optional device int32; WSVD_DEVERR_LEN_RANGE.
  * Rows >= seq_lens[b] are never used: their bytes may hold anything.        */
 size_t wsvd_decode_workspace_size(int B, int H, int r);
@@ -145,8 +150,8 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
 /* ---------------------------------------------------------------- comparison: dense decode
  * The flash-decoding baseline the pages compare against (German §4
  * "Ergebnisse"): out[b,h] = softmax(K[b,h,:n] . q[b,h] * softmax_scale) . V[b,h,:n]
- * over a dense fp16 cache.  K, V [B][H][L_cap][Hd] fp16 (Hd in {64, 128, 256}).
- * Other arguments as for wsvd_decode_attention.                              */
+ * over a dense fp16 cache.  K, V [B][H][L_cap][Hd] fp16 (Hd in {32, 64, 128, 256}).
+ * Other arguments (workspace contract included) as for wsvd_decode_attention. */
 size_t dense_decode_workspace_size(int B, int H, int Hd);
 int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q,
                            int q_dtype, const void* K, const void* V, float softmax_scale, float* out,
@@ -159,7 +164,8 @@ int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_l
  * Every head reads the whole shared latent:
  *   K_h = lat_k[b,:n] . B_k[h], V_h = lat_v[b,:n] . B_v[h],
  *   out[b,h] = softmax(K_h . q[b,h] * softmax_scale) . V_h.
- * R in {128, 256, 512, 1024}.  Other arguments as for wsvd_decode_attention. */
+ * R in {128, 256, 512, 1024}.  Other arguments (workspace contract included)
+ * as for wsvd_decode_attention.                                             */
 size_t shared_decode_workspace_size(int B, int H, int R);
 int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32_t* seq_lens,
                              const void* q, int q_dtype, const void* lat_k, const void* lat_v,

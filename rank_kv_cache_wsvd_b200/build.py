@@ -32,17 +32,29 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+DIGEST = LIB + ".digest"
+
+
+def _digest(extra_flags=()) -> str:
+    """Content hash of every source, header and flag that goes into the library."""
+    import hashlib
+    h = hashlib.sha256(" ".join(NVCC_FLAGS + list(extra_flags)).encode())
+    for f in [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "wsvd.h")]:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _stale(extra_flags=()) -> bool:
+    if not os.path.exists(LIB) or not os.path.exists(DIGEST):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "wsvd.h")]
-    return any(os.path.getmtime(d) > t for d in deps)
+    with open(DIGEST) as f:
+        return f.read().strip() != _digest(extra_flags)
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     """Compile every CUDA source into one shared library; returns its path."""
-    if not force and not _stale():
+    if not force and not _stale(extra_flags):
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-o", tmp,
@@ -51,6 +63,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    with open(DIGEST, "w") as f:
+        f.write(_digest(extra_flags))
     return LIB
 
 

@@ -16,9 +16,14 @@ inline float resolve_scale(float softmax_scale, int Hd) {
   return softmax_scale != 0.f ? softmax_scale : (float)(1.0 / sqrt((double)Hd));
 }
 
+inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
+// Decode workspace: split partials (m, l, o[W]) for every slot a persistent
+// grid can use, then one completion counter per (b, h).
 inline size_t partial_bytes(int B, int H, int W) {
-  return ((size_t)kMaxDecodeCtas + (size_t)B * H) * ((size_t)W + 2) * sizeof(float);
+  return align16(((size_t)kMaxDecodeCtas + (size_t)B * H) * ((size_t)W + 2) * sizeof(float));
 }
+inline size_t decode_ws_bytes(int B, int H, int W) { return partial_bytes(B, H, W) + align16((size_t)B * H * 4); }
 
 // Shared validation of the decode entry points.
 int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
@@ -26,7 +31,7 @@ int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const
   if (B < 0 || H < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
   if (B == 0) return WSVD_OK;
   if (B > 4096) return WSVD_ERR_UNSUPPORTED;
-  if (Hd < 32 || Hd > 256 || Hd % 32) return WSVD_ERR_UNSUPPORTED;
+  if (Hd != 32 && Hd != 64 && Hd != 128 && Hd != 256) return WSVD_ERR_UNSUPPORTED;
   if (L_cap % 8) return WSVD_ERR_UNSUPPORTED;
   if (q_dtype != WSVD_DTYPE_FP16 && q_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
   if (!seq_lens || !q || !out || !workspace) return WSVD_ERR_INVALID_ARG;
@@ -34,14 +39,10 @@ int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const
   return WSVD_OK;
 }
 
-int run_split(int codec, int rowbytes, int qmode, SplitArgs a, const __half* Bv, float* out, int Hd,
-              cudaStream_t stream) {
-  a.ctas = split_decode_grid(codec, rowbytes, qmode, a.B, a.H, a.L_cap);
-  if (a.ctas < 1) return WSVD_ERR_UNSUPPORTED;
-  int tile = 0;
-  if (launch_split_decode(codec, rowbytes, qmode, a, &tile, stream) != cudaSuccess) return WSVD_ERR_CUDA;
-  CombineArgs c{a.B, a.H, Hd, a.W, a.L_cap, a.ctas, tile, a.seq_lens, a.partials, Bv, out, a.err};
-  if (launch_combine(c, stream) != cudaSuccess) return WSVD_ERR_CUDA;
+int run_decode(int codec, int rowbytes, int qmode, DecodeArgs a, void* workspace, cudaStream_t stream) {
+  a.partials = static_cast<float*>(workspace);
+  a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + partial_bytes(a.B, a.H, a.W));
+  if (launch_decode(codec, rowbytes, qmode, a, stream) != cudaSuccess) return WSVD_ERR_CUDA;
   return WSVD_OK;
 }
 
@@ -79,17 +80,17 @@ size_t dense_cache_bytes(int B, int H, int L_cap, int Hd) {
 
 size_t wsvd_decode_workspace_size(int B, int H, int r) {
   if (B < 0 || H < 0 || r < 1) return 0;
-  return partial_bytes(B, H, r);
+  return decode_ws_bytes(B, H, r);
 }
 
 size_t dense_decode_workspace_size(int B, int H, int Hd) {
   if (B < 0 || H < 0 || Hd < 1) return 0;
-  return partial_bytes(B, H, Hd);
+  return decode_ws_bytes(B, H, Hd);
 }
 
 size_t shared_decode_workspace_size(int B, int H, int R) {
   if (B < 0 || H < 0 || R < 1) return 0;
-  return partial_bytes(B, H, R) + (size_t)B * H * R * sizeof(float);
+  return decode_ws_bytes(B, H, R) + align16((size_t)B * H * R * sizeof(float));
 }
 
 int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
@@ -102,24 +103,22 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
   if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
   if (r < 1 || (r * bits) % 8) return WSVD_ERR_INVALID_ARG;
   const int rowbytes = r * bits / 8;
-  if (rowbytes % 16 || split_decode_tile_tokens(bits == 8 ? kCodecI8 : kCodecI4, rowbytes) == 0)
-    return WSVD_ERR_UNSUPPORTED;
+  if (!decode_supported(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj)) return WSVD_ERR_UNSUPPORTED;
   if (!lat_k || !lat_v || !scale_k || !scale_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
   if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
       !aligned16(B_k) || !aligned16(B_v))
     return WSVD_ERR_INVALID_ARG;
   if (workspace_bytes < wsvd_decode_workspace_size(B, H, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
 
-  SplitArgs a{};
+  DecodeArgs a{};
   a.B = B; a.H = H; a.Hd = Hd; a.W = r; a.L_cap = L_cap; a.heads_share = 0;
   a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
   a.lat_k = lat_k; a.lat_v = lat_v;
   a.scale_k = static_cast<const __half*>(scale_k); a.scale_v = static_cast<const __half*>(scale_v);
-  a.Bk = static_cast<const __half*>(B_k); a.qglobal = nullptr;
+  a.Bk = static_cast<const __half*>(B_k); a.Bv = static_cast<const __half*>(B_v); a.qglobal = nullptr;
   a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
-  a.partials = static_cast<float*>(workspace); a.err = err;
-  return run_split(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj, a, static_cast<const __half*>(B_v), out,
-                   Hd, as_stream(stream));
+  a.out = out; a.err = err;
+  return run_decode(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj, a, workspace, as_stream(stream));
 }
 
 int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
@@ -128,18 +127,19 @@ int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_l
   int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
   if (st != WSVD_OK || B == 0) return st;
   const int rowbytes = Hd * 2;
-  if (split_decode_tile_tokens(kCodecF16, rowbytes) == 0) return WSVD_ERR_UNSUPPORTED;
+  if (!decode_supported(kCodecF16, rowbytes, kQDirect)) return WSVD_ERR_UNSUPPORTED;
   if (!K || !V) return WSVD_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V)) return WSVD_ERR_INVALID_ARG;
   if (workspace_bytes < dense_decode_workspace_size(B, H, Hd)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
 
-  SplitArgs a{};
+  DecodeArgs a{};
   a.B = B; a.H = H; a.Hd = Hd; a.W = Hd; a.L_cap = L_cap; a.heads_share = 0;
   a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
   a.lat_k = static_cast<const uint8_t*>(K); a.lat_v = static_cast<const uint8_t*>(V);
+  a.Bv = nullptr;
   a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
-  a.partials = static_cast<float*>(workspace); a.err = err;
-  return run_split(kCodecF16, rowbytes, kQDirect, a, nullptr, out, Hd, as_stream(stream));
+  a.out = out; a.err = err;
+  return run_decode(kCodecF16, rowbytes, kQDirect, a, workspace, as_stream(stream));
 }
 
 int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32_t* seq_lens, const void* q,
@@ -149,29 +149,23 @@ int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32
   int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
   if (st != WSVD_OK || B == 0) return st;
   const int rowbytes = R * 2;
-  if (R < 1 || split_decode_tile_tokens(kCodecF16, rowbytes) == 0) return WSVD_ERR_UNSUPPORTED;
-  {
-    // the shared path instantiates R = 128, 256, 512, 1024 only
-    if (R != 128 && R != 256 && R != 512 && R != 1024) return WSVD_ERR_UNSUPPORTED;
-  }
+  if (R < 1 || !decode_supported(kCodecF16, rowbytes, kQGlobal)) return WSVD_ERR_UNSUPPORTED;
   if (!lat_k || !lat_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
   if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(B_k) || !aligned16(B_v)) return WSVD_ERR_INVALID_ARG;
   if (workspace_bytes < shared_decode_workspace_size(B, H, R)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
 
-  float* partials = static_cast<float*>(workspace);
-  float* qglobal = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + partial_bytes(B, H, R));
+  float* qglobal = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_ws_bytes(B, H, R));
   if (launch_shared_qproj(B, H, Hd, R, q, q_dtype, static_cast<const __half*>(B_k), qglobal,
                           as_stream(stream)) != cudaSuccess)
     return WSVD_ERR_CUDA;
-  SplitArgs a{};
+  DecodeArgs a{};
   a.B = B; a.H = H; a.Hd = Hd; a.W = R; a.L_cap = L_cap; a.heads_share = 1;
   a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
   a.lat_k = static_cast<const uint8_t*>(lat_k); a.lat_v = static_cast<const uint8_t*>(lat_v);
-  a.qglobal = qglobal;
+  a.Bv = static_cast<const __half*>(B_v); a.qglobal = qglobal;
   a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
-  a.partials = partials; a.err = err;
-  return run_split(kCodecF16, rowbytes, kQGlobal, a, static_cast<const __half*>(B_v), out, Hd,
-                   as_stream(stream));
+  a.out = out; a.err = err;
+  return run_decode(kCodecF16, rowbytes, kQGlobal, a, workspace, as_stream(stream));
 }
 
 size_t wsvd_append_workspace_size(void) { return 256; }

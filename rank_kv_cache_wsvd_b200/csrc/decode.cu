@@ -1,5 +1,5 @@
 // Persistent split-L flash-decoding over a low-rank (int8 / int4) or dense
-// (fp16) cache, for sm_100a.
+// (fp16) cache, for sm_100a.  One launch does the whole decode step.
 //
 // The fused decode of the WSVD summaries (Japanese §2.4, German §2.D) streams
 // tiles of each head's latent cache C_Kh through on-chip memory and runs
@@ -12,20 +12,41 @@
 // so the per-token work is O(r) instead of O(r * Hd) and the only bytes read
 // per token are its 2 x r codes and 2 fp16 scales.
 //
+// Arithmetic per token.  K side: q' is held as a 24-bit fixed-point integer
+// split into three byte planes, so code . q' is three dp4a chains (exact
+// integer sums) combined once in fp32; the fixed-point step is max|q'| / 2^23.
+// V side: codes are turned into exact fp32 values by placing them in the
+// mantissa of 2^23 (one byte-permute or bit-select per code) and accumulated
+// with packed fp32x2 FMAs.
+//
 // Work decomposition: the (b, h, tile) space of all sequences is flattened
 // (tiles of T tokens, t fastest) and split evenly over a persistent grid of C
-// CTAs, so ragged lengths cost nothing extra.  A CTA that crosses a (b, h)
-// boundary writes one partial (m, l, o[W]) per (b, h) it touched, into slot
-// c + b*H + h (slots of consecutive CTAs never collide because tile ranges are
-// ordered).  combine_kernel merges the partials of each (b, h) and applies
-// B_Vh.
+// CTAs, so ragged lengths cost nothing extra.  A CTA that owns all tiles of a
+// (b, h) finishes it alone; otherwise each CTA writes one partial (m, l,
+// o[W]) into slot c + b*H + h (slots of consecutive CTAs never collide because
+// tile ranges are ordered) and bumps a per-(b, h) counter; the CTA that
+// arrives last merges the partials and applies B_Vh (last-arriver pattern, no
+// waiting), then resets the counter to zero.
+//
+// Small problems (few tiles per resident CTA) use decode_cluster_kernel
+// instead: one thread-block cluster per (b, h) splits the tokens and merges
+// through distributed shared memory (see below).
 //
 // Per CTA: one producer warp issues 1-D bulk copies (TMA, no multicast) of
-// K codes, V codes and their scales into a kStages-deep shared-memory ring;
-// eight consumer warps read 16-byte segments (a token's row is split over
-// SEGS adjacent lanes), convert codes to fp32 exactly, keep a per-thread
-// online softmax and reduce across lanes / warps only at (b, h) boundaries.
+// K codes, V codes and their scales into a shared-memory ring; eight consumer
+// warps each own NTOK tokens per tile (TPT adjacent lanes per token, VPT
+// values per lane), keep a per-lane online softmax and reduce across lanes /
+// warps only at (b, h) boundaries.
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace wsvd {
 
@@ -33,80 +54,171 @@ template <int CODEC>
 struct CodecT;
 template <>
 struct CodecT<kCodecI8> {
-  static constexpr int kVals = 16;  // values per 16-byte segment
+  static constexpr int kBits = 8;
   static constexpr bool kScaled = true;
 };
 template <>
 struct CodecT<kCodecI4> {
-  static constexpr int kVals = 32;
+  static constexpr int kBits = 4;
   static constexpr bool kScaled = true;
 };
 template <>
 struct CodecT<kCodecF16> {
-  static constexpr int kVals = 8;
+  static constexpr int kBits = 16;
   static constexpr bool kScaled = false;
 };
 
-// ------------------------------------------------------------------ segment math
-// q2 / acc point at the thread's float2 pairs for this segment (kVals / 2 pairs).
-template <int CODEC>
-__device__ __forceinline__ void seg_dot(const uint4 s, const float2* q2, float2& d0, float2& d1);
-template <int CODEC>
-__device__ __forceinline__ void seg_axpy(const uint4 s, const float2 w, float2* acc);
+constexpr int kMaxParts = kMaxDecodeCtas;
+constexpr int kMaxClusterSize = 8;
 
-template <>
-__device__ __forceinline__ void seg_dot<kCodecI8>(const uint4 s, const float2* q2, float2& d0, float2& d1) {
-  const uint32_t w[4] = {s.x ^ 0x80808080u, s.y ^ 0x80808080u, s.z ^ 0x80808080u, s.w ^ 0x80808080u};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    d0 = __ffma2_rn(i8_pair(w[k], 0), q2[2 * k], d0);
-    d1 = __ffma2_rn(i8_pair(w[k], 2), q2[2 * k + 1], d1);
-  }
+// Per-(b, h) operands the producer stages next to the tiles: B_Kh and q (low-rank
+// path), q (dense path) or the projected q' (shared-latent path).  Two buffers
+// when they are small, so the next segment's operands load under the current one.
+__host__ __device__ inline size_t seg_bytes(int qmode, int W, int Hd) {
+  size_t b = qmode == kQProj ? (size_t)W * Hd * 2 + (size_t)Hd * 2 : (qmode == kQDirect ? (size_t)Hd * 2 : (size_t)W * 4);
+  return (b + 127) / 128 * 128;
 }
-template <>
-__device__ __forceinline__ void seg_axpy<kCodecI8>(const uint4 s, const float2 w2, float2* acc) {
-  const uint32_t w[4] = {s.x ^ 0x80808080u, s.y ^ 0x80808080u, s.z ^ 0x80808080u, s.w ^ 0x80808080u};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    acc[2 * k] = __ffma2_rn(i8_pair(w[k], 0), w2, acc[2 * k]);
-    acc[2 * k + 1] = __ffma2_rn(i8_pair(w[k], 2), w2, acc[2 * k + 1]);
-  }
-}
+__host__ __device__ inline int seg_nbuf(int qmode, int W, int Hd) { return seg_bytes(qmode, W, Hd) <= 17408 ? 2 : 1; }
 
-template <>
-__device__ __forceinline__ void seg_dot<kCodecI4>(const uint4 s, const float2* q2, float2& d0, float2& d1) {
-  const uint32_t w[4] = {s.x ^ 0x88888888u, s.y ^ 0x88888888u, s.z ^ 0x88888888u, s.w ^ 0x88888888u};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    d0 = __ffma2_rn(i4_pair(w[k], 0), q2[4 * k + 0], d0);
-    d1 = __ffma2_rn(i4_pair(w[k], 2), q2[4 * k + 1], d1);
-    d0 = __ffma2_rn(i4_pair(w[k], 4), q2[4 * k + 2], d0);
-    d1 = __ffma2_rn(i4_pair(w[k], 6), q2[4 * k + 3], d1);
+template <int CODEC, int VPT, int TPT, int NTOK>
+struct Cfg {
+  using CT = CodecT<CODEC>;
+  static constexpr int kCB = VPT * CT::kBits / 8;  // bytes per lane per token
+  static constexpr int kNSeg = kCB / 16;           // 16-byte shared loads per lane per token
+  static constexpr int kRB = kCB * TPT;            // bytes per token row
+  static constexpr int kW = VPT * TPT;             // values per token row
+  static constexpr int kTPP = kConsumerThreads / TPT;
+  static constexpr int kT = kTPP * NTOK;           // tokens per tile
+  static constexpr int kCodeBytes = kT * kRB;
+  static constexpr int kScaleBytes = CT::kScaled ? kT * 2 : 0;
+  static constexpr int kStageBytes = 2 * kCodeBytes + 2 * kScaleBytes;
+  static constexpr int kStageBudget = kW <= 32 ? 73728 : 57344;  // ring bytes per CTA (two CTAs per SM)
+  static constexpr int kStagesRaw = kStageBudget / kStageBytes;
+  static constexpr int kStages = kStagesRaw < 2 ? 2 : (kStagesRaw > 8 ? 8 : kStagesRaw);
+  static constexpr int kRedRaw = kConsumerWarps * TPT * (VPT + 2);
+  static constexpr int kRedFloats = kRedRaw < kConsumerThreads ? kConsumerThreads : kRedRaw;
+  static constexpr int kQW = VPT / 4;  // byte-plane words of q' per lane
+  static_assert(kCB % 16 == 0, "a lane's chunk is a whole number of 16-byte loads");
+  static_assert(kT % 8 == 0, "tile must hold a multiple of 8 tokens (16-byte scale copies)");
+  static_assert(TPT <= 32 && (TPT & (TPT - 1)) == 0, "a token's lanes share a warp");
+  // shared-memory layout (bytes)
+  static constexpr size_t kOffBar = (size_t)kStages * kStageBytes;
+  static constexpr size_t kOffQ = kOffBar + 2 * kStages * 8 + 4 * 8;  // + segment full / empty barriers
+  static constexpr size_t kOffRed = kOffQ + (size_t)kW * 4;
+  static constexpr size_t kOffRes = kOffRed + (size_t)kRedFloats * 4;
+  static constexpr size_t kOffParts = kOffRes + (size_t)(kW + 2) * 4;
+  static constexpr size_t kOffMisc = kOffParts + (size_t)kMaxParts * 4;
+  static constexpr size_t kOffPre = kOffMisc + 16 * 4;
+  // runtime part: lens / prefix (2B + 1 ints), then the segment buffers
+  __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(2 * B + 1) * 4 + 127) / 128 * 128; }
+  static size_t smem_bytes(int B, int qmode, int Hd) {
+    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd);
   }
-}
-template <>
-__device__ __forceinline__ void seg_axpy<kCodecI4>(const uint4 s, const float2 w2, float2* acc) {
-  const uint32_t w[4] = {s.x ^ 0x88888888u, s.y ^ 0x88888888u, s.z ^ 0x88888888u, s.w ^ 0x88888888u};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) acc[4 * k + p] = __ffma2_rn(i4_pair(w[k], 2 * p), w2, acc[4 * k + p]);
+  // cluster kernel: operands, the leader's partial slots, then B_Vh
+  __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
+  static size_t cluster_smem_bytes(int qmode, int Hd) {
+    return cluster_seg_off() + seg_bytes(qmode, kW, Hd) + (size_t)kMaxClusterSize * (kW + 2) * 4 +
+           (qmode == kQDirect ? 0 : (size_t)kW * Hd * 2);
   }
-}
+};
 
-template <>
-__device__ __forceinline__ void seg_dot<kCodecF16>(const uint4 s, const float2* q2, float2& d0, float2& d1) {
-  d0 = __ffma2_rn(h2_pair(s.x), q2[0], d0);
-  d1 = __ffma2_rn(h2_pair(s.y), q2[1], d1);
-  d0 = __ffma2_rn(h2_pair(s.z), q2[2], d0);
-  d1 = __ffma2_rn(h2_pair(s.w), q2[3], d1);
-}
-template <>
-__device__ __forceinline__ void seg_axpy<kCodecF16>(const uint4 s, const float2 w2, float2* acc) {
-  acc[0] = __ffma2_rn(h2_pair(s.x), w2, acc[0]);
-  acc[1] = __ffma2_rn(h2_pair(s.y), w2, acc[1]);
-  acc[2] = __ffma2_rn(h2_pair(s.z), w2, acc[2]);
-  acc[3] = __ffma2_rn(h2_pair(s.w), w2, acc[3]);
+// ------------------------------------------------------------------ per-lane query state
+template <int CODEC, int VPT>
+struct QState;
+
+template <int VPT>
+struct QState<kCodecI8, VPT> {
+  uint32_t qh[VPT / 4], qm[VPT / 4], ql[VPT / 4];  // signed high byte, unsigned middle / low bytes
+  float step;
+  __device__ __forceinline__ float dot(const uint4* seg) const {
+    int ah = 0, am = 0, al = 0;
+#pragma unroll
+    for (int k = 0; k < VPT / 4; ++k) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(seg)[k];
+      ah = dp4a_ss(w, qh[k], ah);
+      am = dp4a_su(w, qm[k], am);
+      al = dp4a_su(w, ql[k], al);
+    }
+    return fmaf((float)ah, 65536.f, fmaf((float)am, 256.f, (float)al));
+  }
+};
+
+template <int VPT>
+struct QState<kCodecI4, VPT> {
+  // byte plane word 2k holds the even elements of source word k, 2k+1 the odd ones
+  uint32_t qh[VPT / 4], qm[VPT / 4], ql[VPT / 4];
+  int ch, cm, cl;  // 8 * sum of each plane: removes the +8 offset of the nibbles
+  float step;
+  __device__ __forceinline__ float dot(const uint4* seg) const {
+    int ah = -ch, am = -cm, al = -cl;
+#pragma unroll
+    for (int k = 0; k < VPT / 8; ++k) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(seg)[k];
+      const uint32_t ev = (w & 0x0F0F0F0Fu) ^ 0x08080808u;         // c + 8 of elements 8k, 8k+2, ...
+      const uint32_t od = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // c + 8 of elements 8k+1, 8k+3, ...
+      ah = dp4a_us(ev, qh[2 * k], ah);
+      ah = dp4a_us(od, qh[2 * k + 1], ah);
+      am = dp4a_uu(ev, qm[2 * k], am);
+      am = dp4a_uu(od, qm[2 * k + 1], am);
+      al = dp4a_uu(ev, ql[2 * k], al);
+      al = dp4a_uu(od, ql[2 * k + 1], al);
+    }
+    return fmaf((float)ah, 65536.f, fmaf((float)am, 256.f, (float)al));
+  }
+};
+
+template <int VPT>
+struct QState<kCodecF16, VPT> {
+  float2 qv[VPT / 2];
+  float step;
+  __device__ __forceinline__ float dot(const uint4* seg) const {
+    float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < VPT / 4; ++k) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(seg) + 2 * k;
+      d0 = __ffma2_rn(h2_pair(w[0]), qv[2 * k], d0);
+      d1 = __ffma2_rn(h2_pair(w[1]), qv[2 * k + 1], d1);
+    }
+    return (d0.x + d0.y) + (d1.x + d1.y);
+  }
+};
+
+// acc[VPT/2] += wt * values(seg)
+template <int CODEC, int VPT>
+__device__ __forceinline__ void axpy(const uint4* seg, float wt, float2* acc) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(seg);
+  if (CODEC == kCodecI8) {
+    const float2 w2 = make_float2(wt, wt);
+#pragma unroll
+    for (int k = 0; k < VPT / 4; ++k) {
+      const uint32_t x = w[k] ^ 0x80808080u;
+      acc[2 * k] = __ffma2_rn(i8_pair(x, 0), w2, acc[2 * k]);
+      acc[2 * k + 1] = __ffma2_rn(i8_pair(x, 2), w2, acc[2 * k + 1]);
+    }
+  } else if (CODEC == kCodecI4) {
+    // Nibble k of a 16-bit half lands at bits 4k of the mantissa of 2^23, i.e.
+    // value 2^23 + 16^k (c + 8); the weight carries the matching 16^-k.
+    const float2 wa = make_float2(wt, wt * 0.0625f), wb = make_float2(wt * 0.00390625f, wt * 0.000244140625f);
+    const float2 oa = make_float2(-8388616.f, -8388736.f), ob = make_float2(-8390656.f, -8421376.f);
+#pragma unroll
+    for (int k = 0; k < VPT / 8; ++k) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t x = hlf ? (w[k] >> 16) : w[k];
+        float2 f01, f23;
+        f01.x = __uint_as_float((x & 0x000Fu) ^ 0x4B000008u);
+        f01.y = __uint_as_float((x & 0x00F0u) ^ 0x4B000080u);
+        f23.x = __uint_as_float((x & 0x0F00u) ^ 0x4B000800u);
+        f23.y = __uint_as_float((x & 0xF000u) ^ 0x4B008000u);
+        acc[4 * k + 2 * hlf] = __ffma2_rn(__fadd2_rn(f01, oa), wa, acc[4 * k + 2 * hlf]);
+        acc[4 * k + 2 * hlf + 1] = __ffma2_rn(__fadd2_rn(f23, ob), wb, acc[4 * k + 2 * hlf + 1]);
+      }
+    }
+  } else {
+    const float2 w2 = make_float2(wt, wt);
+#pragma unroll
+    for (int k = 0; k < VPT / 2; ++k) acc[k] = __ffma2_rn(h2_pair(w[k]), w2, acc[k]);
+  }
 }
 
 // ------------------------------------------------------------------ tile bookkeeping
@@ -143,44 +255,367 @@ struct TileWalk {
 
 __device__ __forceinline__ int clamp_len(int n, int L_cap) { return (n < 0 || n > L_cap) ? 0 : n; }
 
-template <int CODEC, int SEGS, int SPT>
-struct SplitCfg {
-  using CT = CodecT<CODEC>;
-  static constexpr int kVS = CT::kVals;
-  static constexpr int kVals = kVS * SPT;            // values per consumer thread
-  static constexpr int kPairs = kVals / 2;
-  static constexpr int kT = kConsumerThreads / SEGS;  // tokens per tile
-  static constexpr int kRB = SEGS * SPT * 16;         // bytes per token row
-  static constexpr int kW = SEGS * SPT * kVS;         // values per token row
-  static constexpr int kCodeBytes = kT * kRB;
-  static constexpr int kScaleBytes = CT::kScaled ? kT * 2 : 0;
-  static constexpr int kStageBytes = 2 * kCodeBytes + 2 * kScaleBytes;
-  static constexpr int kRedFloats = kConsumerWarps * SEGS * (kVals + 2);
-  static_assert(kT % 8 == 0, "tile must hold a multiple of 8 tokens (16-byte scale copies)");
-  static size_t smem_bytes(int B) {
-    return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) + (size_t)kW * 4 +
-           (size_t)kRedFloats * 4 + (size_t)(B + 1) * 4;
-  }
-};
+// CTA that owns flat tile g when G tiles are split evenly over C CTAs.
+__device__ __forceinline__ int cta_of(long long g, long long G, int C) {
+  return (int)(((g + 1) * C + G - 1) / G - 1);
+}
 
-template <int CODEC, int SEGS, int SPT, int QMODE>
-__global__ void __launch_bounds__(kDecodeThreads, 2) split_decode_kernel(const SplitArgs a) {
-  using C = SplitCfg<CODEC, SEGS, SPT>;
+// A lane's chunk of a token row from shared memory.  With two 16-byte halves,
+// lanes 4-7 of each 8-lane phase take the halves in the other order, so the
+// phase touches 32 distinct banks.
+template <int NSEG>
+__device__ __forceinline__ void load_chunk(uint4* seg, const uint8_t* p, int lane) {
+  if constexpr (NSEG == 2) {
+    const bool swap = (lane >> 2) & 1;
+    const uint4 x = *reinterpret_cast<const uint4*>(p + (swap ? 16 : 0));
+    const uint4 y = *reinterpret_cast<const uint4*>(p + (swap ? 0 : 16));
+    seg[0] = swap ? y : x;
+    seg[1] = swap ? x : y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < NSEG; ++j) seg[j] = *reinterpret_cast<const uint4*>(p + 16 * j);
+  }
+}
+
+// Consumer-group barrier (the producer warp never joins).
+__device__ __forceinline__ void csync() { named_barrier_sync(1, kConsumerThreads); }
+
+// ------------------------------------------------------------------ consumer building blocks
+// Builds this lane's query state from the staged per-(b, h) operands (see
+// seg_bytes).  Low-rank path: q' = B_Kh . q in shared memory (eight lanes per
+// row, scaled by softmax_scale * log2 e), then the lane's 24-bit fixed-point
+// byte planes (step = max|q'| / 2^23).  fp16 paths: q or the projected q'.
+// Contains consumer-group barriers.
+template <int CODEC, int VPT, int W, int QMODE>
+__device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8_t* sbuf, float* qs, float* misc,
+                                            const DecodeArgs& a, int tid, int sub) {
+  using CT = CodecT<CODEC>;
+  const int warp = tid >> 5, lane = tid & 31;
+  float amax = 0.f;
+  if (QMODE == kQProj) {
+    const __half* Bs = reinterpret_cast<const __half*>(sbuf);
+    const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * 2);
+    const int part = tid & 7, cols = a.Hd >> 3;
+    for (int j = tid >> 3; j < W; j += kConsumerThreads / 8) {
+      const __half* row = Bs + (size_t)j * a.Hd + part * cols;
+      const uint16_t* qq = qsrc + part * cols;
+      float d = 0.f;
+      for (int k = 0; k < cols; k += 2) {
+        const float2 bw = __half22float2(*reinterpret_cast<const __half2*>(row + k));
+        float q0, q1;
+        if (a.q_dtype == WSVD_DTYPE_BF16) {
+          q0 = __uint_as_float((uint32_t)qq[k] << 16);
+          q1 = __uint_as_float((uint32_t)qq[k + 1] << 16);
+        } else {
+          q0 = __half2float(__ushort_as_half(qq[k]));
+          q1 = __half2float(__ushort_as_half(qq[k + 1]));
+        }
+        d = fmaf(bw.x, q0, d);
+        d = fmaf(bw.y, q1, d);
+      }
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
+      d += __shfl_xor_sync(0xffffffffu, d, 2);
+      d += __shfl_xor_sync(0xffffffffu, d, 4);
+      d *= a.qscale;
+      amax = fmaxf(amax, fabsf(d));
+      if (part == 0) qs[j] = d;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  } else if (QMODE == kQDirect) {
+    const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf);
+    for (int j = tid; j < W; j += kConsumerThreads)
+      qs[j] = (a.q_dtype == WSVD_DTYPE_BF16 ? __uint_as_float((uint32_t)qsrc[j] << 16)
+                                            : __half2float(__ushort_as_half(qsrc[j]))) * a.qscale;
+  } else {
+    const float* qg = reinterpret_cast<const float*>(sbuf);
+    for (int j = tid; j < W; j += kConsumerThreads) qs[j] = qg[j] * a.qscale;
+  }
+  if (CT::kScaled && lane == 0) misc[warp] = amax;
+  csync();
+  if constexpr (CT::kScaled) {
+    float M = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, misc[w]);
+    const float inv = M > 0.f ? 8388607.f / M : 0.f;
+    qst.step = M > 0.f ? M / 8388607.f : 0.f;
+    auto qint = [&](int v) {
+      const int x = __float2int_rn(qs[sub * VPT + v] * inv);
+      return max(-8388607, min(8388607, x));
+    };
+    if constexpr (CODEC == kCodecI8) {
+#pragma unroll
+      for (int k = 0; k < VPT / 4; ++k) {
+        uint32_t h4 = 0, m4 = 0, l4 = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int x = qint(4 * k + i);
+          h4 |= ((uint32_t)(x >> 16) & 0xFFu) << (8 * i);
+          m4 |= ((uint32_t)(x >> 8) & 0xFFu) << (8 * i);
+          l4 |= ((uint32_t)x & 0xFFu) << (8 * i);
+        }
+        qst.qh[k] = h4;
+        qst.qm[k] = m4;
+        qst.ql[k] = l4;
+      }
+    } else {
+      int sh = 0, sm = 0, sl = 0;
+#pragma unroll
+      for (int k = 0; k < VPT / 8; ++k) {
+#pragma unroll
+        for (int par = 0; par < 2; ++par) {
+          uint32_t h4 = 0, m4 = 0, l4 = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int x = qint(8 * k + 2 * i + par);
+            const int hb = x >> 16, mb = (x >> 8) & 0xFF, lb = x & 0xFF;
+            sh += hb;
+            sm += mb;
+            sl += lb;
+            h4 |= ((uint32_t)hb & 0xFFu) << (8 * i);
+            m4 |= (uint32_t)mb << (8 * i);
+            l4 |= (uint32_t)lb << (8 * i);
+          }
+          qst.qh[2 * k + par] = h4;
+          qst.qm[2 * k + par] = m4;
+          qst.ql[2 * k + par] = l4;
+        }
+      }
+      qst.ch = 8 * sh;
+      qst.cm = 8 * sm;
+      qst.cl = 8 * sl;
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < VPT / 2; ++p) qst.qv[p] = make_float2(qs[sub * VPT + 2 * p], qs[sub * VPT + 2 * p + 1]);
+    qst.step = 1.f;
+  }
+}
+
+// One staged tile with n valid tokens: scores, lazy-rescaled online softmax and
+// the latent P.V accumulation of this lane's NTOK tokens.
+template <int CODEC, int VPT, int TPT, int NTOK>
+__device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QState<CODEC, VPT>& qst, float& m,
+                                             float& l, float2* acc, int tid) {
+  using C = Cfg<CODEC, VPT, TPT, NTOK>;
   using CT = typename C::CT;
-  constexpr int VS = C::kVS, VALS = C::kVals, NP = C::kPairs, T = C::kT, RB = C::kRB, W = C::kW;
+  constexpr int T = C::kT, RB = C::kRB, CB = C::kCB, NSEG = C::kNSeg, TPP = C::kTPP, NP = VPT / 2;
+  const int g_tok = tid / TPT, sub = tid % TPT, lane = tid & 31;
+  const __half* sck = reinterpret_cast<const __half*>(st + 2 * C::kCodeBytes);
+  float sc[NTOK];
+  float tmax = kNegInf;
+#pragma unroll
+  for (int k = 0; k < NTOK; ++k) {
+    const int tok = k * TPP + g_tok;
+    uint4 seg[NSEG];
+    load_chunk<NSEG>(seg, st + (size_t)tok * RB + sub * CB, lane);
+    float d = qst.dot(seg);
+#pragma unroll
+    for (int o = 1; o < TPT; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    const bool valid = tok < n;
+    const float skk = (CT::kScaled && valid) ? __half2float(sck[tok]) * qst.step : qst.step;
+    sc[k] = valid ? d * skk : kNegInf;
+    tmax = fmaxf(tmax, sc[k]);
+  }
+  if (tmax > m + 8.f) {  // lazy rescale: the reference moves only when a score beats it by 2^8
+    const float fr = ex2(m - tmax);
+    l *= fr;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) acc[p] = __fmul2_rn(acc[p], make_float2(fr, fr));
+    m = tmax;
+  }
+#pragma unroll
+  for (int k = 0; k < NTOK; ++k) {
+    const int tok = k * TPP + g_tok;
+    if (tok < n) {
+      const float p = ex2(sc[k] - m);
+      l += p;
+      const float wv = CT::kScaled ? p * __half2float(sck[T + tok]) : p;
+      uint4 seg[NSEG];
+      load_chunk<NSEG>(seg, st + C::kCodeBytes + (size_t)tok * RB + sub * CB, lane);
+      axpy<CODEC, VPT>(seg, wv, acc);
+    }
+  }
+}
+
+// Merges every consumer lane's (m, l, acc) into res[] = (M, L, O[W]).
+// Lanes holding the same chunk (same sub) merge by shuffles, warps through red[].
+template <int VPT, int TPT, int W>
+__device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, float* red, float* res, int tid) {
+  constexpr int NP = VPT / 2;
+  const int warp = tid >> 5, lane = tid & 31, sub = tid % TPT;
+#pragma unroll
+  for (int o = TPT; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+    const float M = fmaxf(m, mo);
+    const float f1 = (m == kNegInf) ? 0.f : ex2(m - M);
+    const float f2 = (mo == kNegInf) ? 0.f : ex2(mo - M);
+    l = l * f1 + lo * f2;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      float2 ao;
+      ao.x = __shfl_xor_sync(0xffffffffu, acc[p].x, o);
+      ao.y = __shfl_xor_sync(0xffffffffu, acc[p].y, o);
+      acc[p] = __ffma2_rn(acc[p], make_float2(f1, f1), __fmul2_rn(ao, make_float2(f2, f2)));
+    }
+    m = M;
+  }
+  if (lane < TPT) {
+    float* rw = red + (warp * TPT + sub) * (VPT + 2);
+    rw[0] = m;
+    rw[1] = l;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      rw[2 + 2 * p] = acc[p].x;
+      rw[3 + 2 * p] = acc[p].y;
+    }
+  }
+  csync();
+  float M = kNegInf;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * TPT * (VPT + 2)]);
+  float f[kConsumerWarps];
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) {
+    const float mw = red[w * TPT * (VPT + 2)];
+    f[w] = (mw == kNegInf) ? 0.f : ex2(mw - M);
+  }
+  for (int e = tid; e < W; e += kConsumerThreads) {
+    const int se = e / VPT, v = e % VPT;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) s = fmaf(f[w], red[(w * TPT + se) * (VPT + 2) + 2 + v], s);
+    res[2 + e] = s;
+  }
+  if (tid == 0) {
+    float ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) ls = fmaf(f[w], red[w * TPT * (VPT + 2) + 1], ls);
+    res[0] = M;
+    res[1] = ls;
+  }
+  csync();
+}
+
+// Merges rows p of a partial array part[p][W + 2] (m, l, o[W]), p < np, into
+// res[], staging chunks of rows in red[] (nred floats).  ldcg selects
+// L2-coherent global loads (rows written by other CTAs).
+template <int W, bool GLOBAL>
+__device__ __forceinline__ void merge_rows(const float* part, int np, float* red, int nred, float* res, int tid) {
+  const int rows = max(1, nred / (W + 2));
+  float Mrun = kNegInf;
+  for (int p0 = 0; p0 < np; p0 += rows) {
+    const int nr = min(rows, np - p0);
+    for (int i = tid; i < nr * (W + 2); i += kConsumerThreads)
+      red[i] = GLOBAL ? __ldcg(part + (size_t)p0 * (W + 2) + i) : part[(size_t)p0 * (W + 2) + i];
+    csync();
+    float M = Mrun;
+    for (int p = 0; p < nr; ++p) M = fmaxf(M, red[p * (W + 2)]);
+    const float fold = (Mrun == kNegInf) ? 0.f : ex2(Mrun - M);
+    for (int e = tid; e < W + 1; e += kConsumerThreads) {  // e = 0: l, e >= 1: o[e - 1]
+      float s2 = (p0 == 0) ? 0.f : res[1 + e] * fold;
+      for (int p = 0; p < nr; ++p) {
+        const float mp = red[p * (W + 2)];
+        if (mp != kNegInf) s2 = fmaf(ex2(mp - M), red[p * (W + 2) + 1 + e], s2);
+      }
+      res[1 + e] = s2;
+    }
+    Mrun = M;
+    csync();
+  }
+  if (tid == 0) res[0] = Mrun;
+  csync();
+}
+
+// out = O . Bv / L for the merged res[] (Bv [W][Hd] fp16, global or shared;
+// null: the dense path, out = O / L).  L = 0 (no tokens) gives zeros.
+template <int W>
+__device__ __forceinline__ void finalize_out(const float* res, const __half* Bv, float* outp, int Hd, float* red,
+                                             int tid) {
+  const float inv = res[1] > 0.f ? 1.f / res[1] : 0.f;
+  if (Bv == nullptr) {
+    for (int d = tid; d < Hd; d += kConsumerThreads) outp[d] = res[2 + d] * inv;
+    return;
+  }
+  const int ng = kConsumerThreads / Hd;  // e-groups per output column (Hd divides 256)
+  const int d = tid % Hd, grp = tid / Hd;
+  float s = 0.f;
+  for (int e = grp; e < W; e += ng) s = fmaf(res[2 + e], __half2float(Bv[(size_t)e * Hd + d]), s);
+  red[tid] = s;
+  csync();
+  if (tid < Hd) {
+    float t = 0.f;
+    for (int q = 0; q < ng; ++q) t += red[q * Hd + tid];
+    outp[tid] = t * inv;
+  }
+  csync();
+}
+
+// Producer: stage the per-(b, h) operands into a segment buffer.
+template <int W, int QMODE>
+__device__ __forceinline__ void issue_operands(uint8_t* dst, uint64_t* bar, const DecodeArgs& a, int b, int h,
+                                               uint64_t keep) {
+  const size_t bh = (size_t)b * a.H + h;
+  if (QMODE == kQProj) {
+    const uint32_t bb = (uint32_t)W * a.Hd * 2, qb = (uint32_t)a.Hd * 2;
+    mbar_arrive_expect_tx(bar, bb + qb);
+    bulk_g2s(dst, a.Bk + (size_t)h * W * a.Hd, bb, bar, keep);
+    bulk_g2s(dst + bb, static_cast<const uint16_t*>(a.q) + bh * a.Hd, qb, bar, keep);
+  } else if (QMODE == kQDirect) {
+    mbar_arrive_expect_tx(bar, (uint32_t)a.Hd * 2);
+    bulk_g2s(dst, static_cast<const uint16_t*>(a.q) + bh * a.Hd, (uint32_t)a.Hd * 2, bar, keep);
+  } else {
+    mbar_arrive_expect_tx(bar, (uint32_t)W * 4);
+    bulk_g2s(dst, a.qglobal + bh * W, (uint32_t)W * 4, bar, keep);
+  }
+}
+
+// Producer: stage tile t (n valid tokens) of (b, h) into ring stage st.
+template <int CODEC, int VPT, int TPT, int NTOK>
+__device__ __forceinline__ void issue_tile(uint8_t* st, uint64_t* bar, const DecodeArgs& a, int b, int h, int t,
+                                           int n, uint64_t pol) {
+  using C = Cfg<CODEC, VPT, TPT, NTOK>;
+  using CT = typename C::CT;
+  const size_t head_row = ((size_t)b * a.H + h) * a.L_cap + (size_t)t * C::kT;
+  const size_t row0 = a.heads_share ? (size_t)b * a.L_cap + (size_t)t * C::kT : head_row;
+  const uint32_t cb = (uint32_t)n * C::kRB;
+  const uint32_t sb = CT::kScaled ? (uint32_t)((n + 7) & ~7) * 2u : 0u;
+  mbar_arrive_expect_tx(bar, 2 * cb + 2 * sb);
+  bulk_g2s(st, a.lat_k + row0 * C::kRB, cb, bar, pol);
+  bulk_g2s(st + C::kCodeBytes, a.lat_v + row0 * C::kRB, cb, bar, pol);
+  if (CT::kScaled) {
+    bulk_g2s(st + 2 * C::kCodeBytes, a.scale_k + head_row, sb, bar, pol);
+    bulk_g2s(st + 2 * C::kCodeBytes + C::kScaleBytes, a.scale_v + head_row, sb, bar, pol);
+  }
+}
+
+// ------------------------------------------------------------------ persistent kernel
+template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+  using C = Cfg<CODEC, VPT, TPT, NTOK>;
+  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
-  uint64_t* empty = full + kStages;
-  float* qs = reinterpret_cast<float*>(empty + kStages);
-  float* red = qs + W;
-  int* pre = reinterpret_cast<int*>(red + C::kRedFloats);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + S;
+  uint64_t* segfull = empty + S;  // [2]
+  uint64_t* segempty = segfull + 2;
+  float* qs = reinterpret_cast<float*>(smem + C::kOffQ);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* res = reinterpret_cast<float*>(smem + C::kOffRes);
+  float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
+  int* pre = reinterpret_cast<int*>(smem + C::kOffPre);
+  int* lens = pre + a.B + 1;
+  uint8_t* segbuf = smem + C::seg_off(a.B);
+  const int NBUF = seg_nbuf(QMODE, W, a.Hd);
+  const uint32_t SEGB = (uint32_t)seg_bytes(QMODE, W, a.Hd);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
 
-  // Tiles per sequence (per head), exclusive prefix over sequences.
+  // Valid lengths, tiles per sequence (per head) and their exclusive prefix.
   if (warp == 0) {
     const int per = (a.B + 31) / 32;
     const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
@@ -188,7 +623,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) split_decode_kernel(const S
     for (int b = b0; b < b1; ++b) {
       const int raw = a.seq_lens[b];
       if ((raw < 0 || raw > a.L_cap) && c == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
-      sum += (clamp_len(raw, a.L_cap) + T - 1) / T;
+      const int n = clamp_len(raw, a.L_cap);
+      lens[b] = n;
+      sum += (n + T - 1) / T;
     }
     int incl = sum;
 #pragma unroll
@@ -199,362 +636,437 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) split_decode_kernel(const S
     int run = incl - sum;
     for (int b = b0; b < b1; ++b) {
       pre[b] = run;
-      run += (clamp_len(a.seq_lens[b], a.L_cap) + T - 1) / T;
+      run += (lens[b] + T - 1) / T;
     }
     if (lane == 31) pre[a.B] = incl;
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < S; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], kConsumerWarps);
+      }
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&segfull[s], 1);
+        mbar_init(&segempty[s], kConsumerWarps);
       }
       fence_mbar_init();
     }
   }
   __syncthreads();
 
+  // Sequences with no tokens get a zero output (spread over the CTAs).
+  for (int b = c; b < a.B; b += a.ctas) {
+    if (lens[b] == 0)
+      for (int i = tid; i < a.H * a.Hd; i += blockDim.x) a.out[(size_t)b * a.H * a.Hd + i] = 0.f;
+  }
+
   const TileWalk walk{pre, a.B, a.H};
   const long long G = (long long)a.H * pre[a.B];
-  const long long g_begin = G * c / a.ctas, g_end = G * (c + 1) / a.ctas;
-  if (g_begin >= g_end) return;  // uniform across the CTA; nothing was issued
+  // At most one CTA per tile, so every working CTA owns at least one tile and
+  // the CTAs that share a (b, h) are consecutive without gaps.
+  const int CW = (int)(G < a.ctas ? G : a.ctas);
+  if (c >= CW) return;  // uniform across the CTA; nothing was issued
+  const long long g_begin = G * c / CW, g_end = G * (c + 1) / CW;
 
   // ---------------------------------------------------------------- producer warp
   if (warp == kConsumerWarps) {
     if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
+      const uint64_t pol = l2_evict_first_policy(), keep = l2_evict_last_policy();
       int b, h, t;
       walk.locate(g_begin, b, h, t);
       long long issued = 0;
+      int nseg = 0, pb = -1, ph = -1;
       bool ok = true;
-      for (long long g = g_begin; g < g_end; ++g, ++issued) {
-        const int s = (int)(issued % kStages);
-        if (issued >= kStages && !mbar_wait_bounded(&empty[s], (uint32_t)(((issued / kStages) - 1) & 1))) {
+      for (long long g = g_begin; g < g_end && ok; ++g, ++issued) {
+        if (b != pb || h != ph) {  // operands of the next (b, h)
+          const int sb = nseg % NBUF;
+          if (nseg >= NBUF && !mbar_wait_bounded(&segempty[sb], (uint32_t)(((nseg / NBUF) - 1) & 1))) {
+            set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+            ok = false;
+            break;
+          }
+          issue_operands<W, QMODE>(segbuf + (size_t)sb * SEGB, &segfull[sb], a, b, h, keep);
+          ++nseg;
+          pb = b;
+          ph = h;
+        }
+        const int s = (int)(issued % S);
+        if (issued >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((issued / S) - 1) & 1))) {
           set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
           ok = false;
           break;
         }
-        const int len = a.seq_lens[b];
-        const int n = min(T, len - t * T);
-        const size_t head_row = ((size_t)b * a.H + h) * a.L_cap + (size_t)t * T;
-        const size_t row0 = a.heads_share ? (size_t)b * a.L_cap + (size_t)t * T : head_row;
-        uint8_t* st = stages + s * C::kStageBytes;
-        const uint32_t cb = (uint32_t)n * RB;
-        const uint32_t sb = CT::kScaled ? (uint32_t)((n + 7) & ~7) * 2u : 0u;
-        mbar_arrive_expect_tx(&full[s], 2 * cb + 2 * sb);
-        bulk_g2s(st, a.lat_k + row0 * RB, cb, &full[s], pol);
-        bulk_g2s(st + C::kCodeBytes, a.lat_v + row0 * RB, cb, &full[s], pol);
-        if (CT::kScaled) {
-          bulk_g2s(st + 2 * C::kCodeBytes, a.scale_k + head_row, sb, &full[s], pol);
-          bulk_g2s(st + 2 * C::kCodeBytes + C::kScaleBytes, a.scale_v + head_row, sb, &full[s], pol);
-        }
+        issue_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, &full[s], a, b, h, t,
+                                          min(T, lens[b] - t * T), pol);
         walk.advance(b, h, t);
       }
-      // Leave no copy in flight behind: wait (bounded) for the last uses of each stage.
-      const long long last = issued;
-      for (long long i = (last > kStages ? last - kStages : 0); i < last && ok; ++i) {
-        const int s = (int)(i % kStages);
-        if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kStages) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-      }
+      // Leave no copy in flight behind: wait (bounded) for the last uses of each buffer.
+      for (long long i = (issued > S ? issued - S : 0); i < issued && ok; ++i)
+        if (!mbar_wait_bounded(&full[(int)(i % S)], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      for (int k = (nseg > NBUF ? nseg - NBUF : 0); k < nseg && ok; ++k)
+        if (!mbar_wait_bounded(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     }
     return;
   }
 
   // ---------------------------------------------------------------- consumer warps
-  const int tok = tid / SEGS, sl = tid % SEGS;
-  float2 qv[NP], acc[NP];
+  const int sub = tid % TPT;
+  QState<CODEC, VPT> qst;
+  float2 acc[NP];
   float m = kNegInf, l = 0.f;
   bool timed_out = false;
+  int nseg = 0;
 
-  auto setup_query = [&](int b, int h) {
-    if (QMODE == kQProj) {
-      // q' = B_Kh . q, scaled by softmax_scale * log2(e): one warp per row of B_Kh.
-      const size_t qoff = ((size_t)b * a.H + h) * a.Hd;
-      float qr[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        qr[k] = (lane + 32 * k < a.Hd) ? load_q_elem(a.q, a.q_dtype, qoff + lane + 32 * k) : 0.f;
-      const __half* Bh = a.Bk + (size_t)h * W * a.Hd;
-      for (int j = warp; j < W; j += kConsumerWarps) {
-        float d = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (lane + 32 * k < a.Hd) d = fmaf(__half2float(Bh[(size_t)j * a.Hd + lane + 32 * k]), qr[k], d);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (lane == 0) qs[j] = d * a.qscale;
-      }
-    } else if (QMODE == kQDirect) {
-      const size_t qoff = ((size_t)b * a.H + h) * a.Hd;
-      for (int j = tid; j < W; j += kConsumerThreads) qs[j] = load_q_elem(a.q, a.q_dtype, qoff + j) * a.qscale;
-    } else {
-      const float* qg = a.qglobal + ((size_t)b * a.H + h) * W;
-      for (int j = tid; j < W; j += kConsumerThreads) qs[j] = qg[j] * a.qscale;
+  auto flush = [&](int b, int h, int c_first, int c_last) {
+    reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
+    float* outp = a.out + ((size_t)b * a.H + h) * a.Hd;
+    const __half* Bvh = a.Bv ? a.Bv + (size_t)h * W * a.Hd : nullptr;
+    if (c_first == c_last) {  // this CTA owns the whole (b, h)
+      finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
+      return;
     }
-    named_barrier_sync(1, kConsumerThreads);
-#pragma unroll
-    for (int i = 0; i < SPT; ++i) {
-      const int e0 = (sl + i * SEGS) * VS;
-#pragma unroll
-      for (int p = 0; p < VS / 2; ++p) qv[i * (VS / 2) + p] = make_float2(qs[e0 + 2 * p], qs[e0 + 2 * p + 1]);
-    }
-#pragma unroll
-    for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
-    m = kNegInf;
-    l = 0.f;
-  };
-
-  auto flush = [&](int b, int h) {
-    // Merge lanes that hold the same segment (same sl), then warps.
-#pragma unroll
-    for (int o = SEGS; o < 32; o <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-      const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-      const float M = fmaxf(m, mo);
-      const float f1 = (m == kNegInf) ? 0.f : exp2f(m - M);
-      const float f2 = (mo == kNegInf) ? 0.f : exp2f(mo - M);
-      l = l * f1 + lo * f2;
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        float2 ao;
-        ao.x = __shfl_xor_sync(0xffffffffu, acc[p].x, o);
-        ao.y = __shfl_xor_sync(0xffffffffu, acc[p].y, o);
-        acc[p] = __ffma2_rn(acc[p], make_float2(f1, f1), __fmul2_rn(ao, make_float2(f2, f2)));
-      }
-      m = M;
-    }
-    if (lane < SEGS) {
-      float* rw = red + (warp * SEGS + sl) * (VALS + 2);
-      rw[0] = m;
-      rw[1] = l;
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        rw[2 + 2 * p] = acc[p].x;
-        rw[3 + 2 * p] = acc[p].y;
-      }
-    }
-    named_barrier_sync(1, kConsumerThreads);
-    float M = kNegInf;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * SEGS * (VALS + 2)]);
-    float f[kConsumerWarps];
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float mw = red[w * SEGS * (VALS + 2)];
-      f[w] = (mw == kNegInf) ? 0.f : exp2f(mw - M);
-    }
-    float* dst = a.partials + ((size_t)c + (size_t)b * a.H + h) * (W + 2);
-    for (int e = tid; e < W; e += kConsumerThreads) {
-      const int seg = e / VS, sle = seg % SEGS, v = (seg / SEGS) * VS + e % VS;
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) s = fmaf(f[w], red[(w * SEGS + sle) * (VALS + 2) + 2 + v], s);
-      dst[2 + e] = s;
-    }
+    // Publish the partial; the last CTA of (b, h) to arrive merges and finishes.
+    const int bh = b * a.H + h;
+    float* dst = a.partials + ((size_t)c + bh) * (W + 2);
+    for (int e = tid; e < W + 2; e += kConsumerThreads) dst[e] = res[e];
+    __threadfence();
+    csync();
     if (tid == 0) {
-      float ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) ls = fmaf(f[w], red[w * SEGS * (VALS + 2) + 1], ls);
-      dst[0] = M;
-      dst[1] = ls;
+      const int prev = atomicAdd(&a.counters[bh], 1);
+      reinterpret_cast<int*>(misc)[8] = (prev == c_last - c_first) ? 1 : 0;
     }
-    named_barrier_sync(1, kConsumerThreads);
+    csync();
+    if (reinterpret_cast<int*>(misc)[8]) {
+      __threadfence();
+      merge_rows<W, true>(a.partials + ((size_t)c_first + bh) * (W + 2), c_last - c_first + 1, red, C::kRedFloats,
+                          res, tid);
+      if (tid == 0) atomicExch(&a.counters[bh], 0);
+      finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
+    }
+    csync();
   };
 
   int b, h, t;
   walk.locate(g_begin, b, h, t);
-  int cb = -1, ch = -1;
+  int cb = -1, ch = -1, c_first = 0, c_last = 0;
   long long i = 0;
   for (long long g = g_begin; g < g_end; ++g, ++i) {
     if (b != cb || h != ch) {
-      if (cb >= 0) flush(cb, ch);
-      setup_query(b, h);
+      if (cb >= 0) flush(cb, ch, c_first, c_last);
+      const int tb = walk.tiles(b);
+      const long long gf = (long long)a.H * pre[b] + (long long)h * tb;
+      c_first = cta_of(gf, G, CW);
+      c_last = cta_of(gf + tb - 1, G, CW);
+      if (a.Bv != nullptr && c == c_last) {  // the likely finisher warms B_Vh in L2
+        const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)h * W * a.Hd);
+        for (int o = tid * 128; o < W * a.Hd * 2; o += kConsumerThreads * 128) prefetch_l2(bv + o);
+      }
+      const int sb = nseg % NBUF;
+      if (!mbar_wait_bounded(&segfull[sb], (uint32_t)((nseg / NBUF) & 1), timed_out ? 0ull : kWaitLimitNs)) {
+        if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        timed_out = true;
+      }
+      build_query<CODEC, VPT, W, QMODE>(qst, segbuf + (size_t)sb * SEGB, qs, misc, a, tid, sub);
+      if (lane == 0) mbar_arrive(&segempty[sb]);  // the staged operands are consumed
+      ++nseg;
+#pragma unroll
+      for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
+      m = kNegInf;
+      l = 0.f;
       cb = b;
       ch = h;
     }
-    const int s = (int)(i % kStages);
+    const int s = (int)(i % S);
     // A timed-out wait only poisons the result (err is set); control flow stays
     // uniform so every consumer warp reaches every named barrier.
-    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kStages) & 1), timed_out ? 0ull : kWaitLimitNs)) {
+    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
       if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       timed_out = true;
     }
-    const int n = min(T, a.seq_lens[b] - t * T);
-    const bool valid = tok < n;
-    const uint8_t* st = stages + s * C::kStageBytes;
-    const uint8_t* rowk = st + tok * RB;
-    const uint8_t* rowv = st + C::kCodeBytes + tok * RB;
-
-    float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < SPT; ++j) {
-      const uint4 kc = *reinterpret_cast<const uint4*>(rowk + (sl + j * SEGS) * 16);
-      seg_dot<CODEC>(kc, &qv[j * (VS / 2)], d0, d1);
-    }
-    float d = (d0.x + d0.y) + (d1.x + d1.y);
-#pragma unroll
-    for (int o = 1; o < SEGS; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-
-    float sk = 1.f, sv = 1.f;
-    if (CT::kScaled && valid) {
-      const __half* scl = reinterpret_cast<const __half*>(st + 2 * C::kCodeBytes);
-      sk = __half2float(scl[tok]);
-      sv = __half2float(scl[T + tok]);
-    }
-    const float sc = valid ? d * sk : kNegInf;
-    if (sc > m + 8.f) {  // lazy rescale: the reference max moves only when a score beats it by 2^8
-      const float fr = exp2f(m - sc);
-      l *= fr;
-#pragma unroll
-      for (int p = 0; p < NP; ++p) acc[p] = __fmul2_rn(acc[p], make_float2(fr, fr));
-      m = sc;
-    }
-    if (valid) {
-      const float p = exp2f(sc - m);
-      l += p;
-      const float wv = p * sv;
-#pragma unroll
-      for (int j = 0; j < SPT; ++j) {
-        const uint4 vc = *reinterpret_cast<const uint4*>(rowv + (sl + j * SEGS) * 16);
-        seg_axpy<CODEC>(vc, make_float2(wv, wv), &acc[j * (VS / 2)]);
-      }
-    }
+    process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, lens[b] - t * T), qst, m, l,
+                                        acc, tid);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     walk.advance(b, h, t);
   }
-  if (cb >= 0) flush(cb, ch);
+  if (cb >= 0) flush(cb, ch, c_first, c_last);
 }
 
-// ------------------------------------------------------------------ combine
-// One CTA per (b, h): merge the partials of every CTA that touched (b, h),
-// then up-project through B_Vh (low-rank paths) or normalise (dense path).
-__global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
-  __shared__ float f[kMaxDecodeCtas];
-  __shared__ int red_i[2][8];
-  __shared__ float red_f[8];
-  extern __shared__ float o[];  // W floats
+// ------------------------------------------------------------------ cluster kernel (small problems)
+// One thread-block cluster of `cluster` CTAs per (b, h) splits the cached
+// tokens into contiguous chunks.  Each CTA issues its operand and tile copies
+// at launch (the operands before seq_lens is even read), reduces its chunk to
+// (m, l, o[W]) and stores it straight into a slot of the leader's shared
+// memory (distributed shared memory), then arrives on the leader's mbarrier.
+// The leader merges the slots in rank order and writes out[b, h] with B_Vh
+// staged in its shared memory: no global partials, counters or fences.
+template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const DecodeArgs a) {
+  using C = Cfg<CODEC, VPT, TPT, NTOK>;
+  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank(), csize = (int)cluster.num_blocks();
+  const int h = blockIdx.y, b = blockIdx.z;
 
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int T = a.tile;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stages = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + S;
+  uint64_t* segfull = empty + S;
+  uint64_t* aux = segfull + 1;  // [0]: B_Vh staged (leader), [1]: slots filled (leader)
+  float* qs = reinterpret_cast<float*>(smem + C::kOffQ);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* res = reinterpret_cast<float*>(smem + C::kOffRes);
+  float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
+  uint8_t* segbuf = smem + C::cluster_seg_off();
+  float* slots = reinterpret_cast<float*>(segbuf + seg_bytes(QMODE, W, a.Hd));  // [csize][W + 2]
+  __half* bvs = reinterpret_cast<__half*>(slots + (size_t)kMaxClusterSize * (W + 2));
 
-  // Tiles of sequences < b and of all sequences.
-  int before = 0, total = 0;
-  for (int i = tid; i < a.B; i += blockDim.x) {
-    const int tb = (clamp_len(a.seq_lens[i], a.L_cap) + T - 1) / T;
-    total += tb;
-    if (i < b) before += tb;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    before += __shfl_xor_sync(0xffffffffu, before, off);
-    total += __shfl_xor_sync(0xffffffffu, total, off);
-  }
-  if (lane == 0) {
-    red_i[0][warp] = before;
-    red_i[1][warp] = total;
-  }
-  __syncthreads();
-  before = total = 0;
-  for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
-    before += red_i[0][w];
-    total += red_i[1][w];
-  }
-  const int len = clamp_len(a.seq_lens[b], a.L_cap);
-  const int tb = (len + T - 1) / T;
-  float* outp = a.out + (size_t)bh * a.Hd;
-  if (tb == 0) {
-    for (int d = tid; d < a.Hd; d += blockDim.x) outp[d] = 0.f;
-    return;
-  }
-  const long long G = (long long)a.H * total;
-  const long long g0 = (long long)a.H * before + (long long)h * tb, g1 = g0 + tb - 1;
-  auto cta_of = [&](long long g) { return (int)(((g + 1) * a.ctas + G - 1) / G - 1); };
-  const int c0 = cta_of(g0), c1 = cta_of(g1);
-  const int np = c1 - c0 + 1;
-  const int W = a.W;
-  const float* part = a.partials + ((size_t)c0 + bh) * (W + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Token chunk of this rank (multiple of 8 tokens, so scale copies stay aligned).
+  const int chunk = ((a.L_cap + csize - 1) / csize + 7) & ~7;
+  const int lo = min(a.L_cap, rank * chunk), hi = min(a.L_cap, lo + chunk);
 
-  float M = kNegInf;
-  for (int p = tid; p < np; p += blockDim.x) M = fmaxf(M, part[(size_t)p * (W + 2)]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) red_f[warp] = M;
-  __syncthreads();
-  M = kNegInf;
-  for (int w = 0; w < (int)(blockDim.x / 32); ++w) M = fmaxf(M, red_f[w]);
-  for (int p = tid; p < np; p += blockDim.x) {
-    const float mp = part[(size_t)p * (W + 2)];
-    f[p] = (mp == kNegInf) ? 0.f : exp2f(mp - M);
-  }
-  __syncthreads();
-  float lsum = 0.f;
-  for (int p = 0; p < np; ++p) lsum = fmaf(f[p], part[(size_t)p * (W + 2) + 1], lsum);
-  for (int e = tid; e < W; e += blockDim.x) {
-    float s = 0.f;
-    for (int p = 0; p < np; ++p) s = fmaf(f[p], part[(size_t)p * (W + 2) + 2 + e], s);
-    o[e] = s;
-  }
-  __syncthreads();
-  const float inv = 1.f / lsum;
-  if (a.Bv == nullptr) {
-    for (int d = tid; d < a.Hd; d += blockDim.x) outp[d] = o[d] * inv;
-  } else {
-    const __half* Bh = a.Bv + (size_t)h * W * a.Hd;
-    for (int d = tid; d < a.Hd; d += blockDim.x) {
-      float s = 0.f;
-      for (int e = 0; e < W; ++e) s = fmaf(o[e], __half2float(Bh[(size_t)e * a.Hd + d]), s);
-      outp[d] = s * inv;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    mbar_init(segfull, 1);
+    mbar_init(&aux[0], 1);
+    mbar_init(&aux[1], csize > 1 ? csize - 1 : 1);
+    fence_mbar_init();
+    // Operands first: they do not depend on the sequence length.
+    const uint64_t keep = l2_evict_last_policy();
+    issue_operands<W, QMODE>(segbuf, segfull, a, b, h, keep);
+    if (rank == 0 && a.Bv != nullptr) {
+      const uint32_t bb = (uint32_t)W * a.Hd * 2;
+      mbar_arrive_expect_tx(&aux[0], bb);
+      for (uint32_t off = 0; off < bb; off += 32768)
+        bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, reinterpret_cast<const uint8_t*>(a.Bv + (size_t)h * W * a.Hd) + off,
+                 min(32768u, bb - off), &aux[0], keep);
     }
   }
+  cluster.barrier_arrive();  // barriers initialised; waited on before any remote access
+
+  const int raw = a.seq_lens[b];
+  if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+  const int len = clamp_len(raw, a.L_cap);
+  const int end = min(hi, len);
+  const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
+  __syncthreads();  // barrier initialisation visible to every thread of this CTA
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / S) - 1) & 1))) {
+          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        // tiles are counted from lo; issue_tile counts rows from (b, h) row 0, so
+        // pass the token offset through t with tiles of T tokens: lo is a multiple of 8,
+        // not of T, so address rows directly.
+        const int r0 = lo + i * T, n = min(T, end - r0);
+        const size_t head_row = ((size_t)b * a.H + h) * a.L_cap + r0;
+        const size_t row0 = a.heads_share ? (size_t)b * a.L_cap + r0 : head_row;
+        using CT = typename C::CT;
+        uint8_t* st = stages + (size_t)s * C::kStageBytes;
+        const uint32_t cbytes = (uint32_t)n * C::kRB;
+        const uint32_t sbytes = CT::kScaled ? (uint32_t)((n + 7) & ~7) * 2u : 0u;
+        mbar_arrive_expect_tx(&full[s], 2 * cbytes + 2 * sbytes);
+        bulk_g2s(st, a.lat_k + row0 * C::kRB, cbytes, &full[s], pol);
+        bulk_g2s(st + C::kCodeBytes, a.lat_v + row0 * C::kRB, cbytes, &full[s], pol);
+        if (CT::kScaled) {
+          bulk_g2s(st + 2 * C::kCodeBytes, a.scale_k + head_row, sbytes, &full[s], pol);
+          bulk_g2s(st + 2 * C::kCodeBytes + C::kScaleBytes, a.scale_v + head_row, sbytes, &full[s], pol);
+        }
+      }
+      for (int i = (ntiles > S ? ntiles - S : 0); i < ntiles && ok; ++i)
+        if (!mbar_wait_bounded(&full[i % S], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+    }
+    cluster.barrier_wait();
+    return;
+  }
+
+  // consumers
+  const int sub = tid % TPT;
+  QState<CODEC, VPT> qst;
+  float2 acc[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
+  float m = kNegInf, l = 0.f;
+  bool timed_out = false;
+  if (!mbar_wait_bounded(segfull, 0)) {
+    if (lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+    timed_out = true;
+  }
+  build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, a, tid, sub);
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % S;
+    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
+      if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      timed_out = true;
+    }
+    process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, end - lo - i * T), qst, m, l,
+                                        acc, tid);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
+
+  cluster.barrier_wait();  // every CTA of the cluster has initialised its barriers
+  float* leader_slots = cluster.map_shared_rank(slots, 0);
+  for (int e = tid; e < W + 2; e += kConsumerThreads) leader_slots[(size_t)rank * (W + 2) + e] = res[e];
+  csync();
+  if (rank != 0) {
+    if (tid == 0) {
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      uint32_t rbar;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(&aux[1])), "r"(0));
+      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
+    }
+    return;
+  }
+  if (csize > 1) {
+    if (tid == 0) {
+      const uint32_t addr = smem_u32(&aux[1]);
+      const uint64_t t0 = globaltimer_ns();
+      for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(addr)
+            : "memory");
+        if (done) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+          break;
+        }
+      }
+    }
+    csync();
+    merge_rows<W, false>(slots, csize, red, C::kRedFloats, res, tid);
+  }
+  const __half* Bvh = nullptr;
+  if (a.Bv != nullptr) {
+    if (!mbar_wait_bounded(&aux[0], 0, timed_out ? 0ull : kWaitLimitNs) && lane == 0)
+      set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+    Bvh = bvs;
+  }
+  finalize_out<W>(res, Bvh, a.out + ((size_t)b * a.H + h) * a.Hd, a.Hd, red, tid);
 }
 
 // ------------------------------------------------------------------ host side
 namespace {
 
+// Per-device caches of the host-side launch set-up (SM count, occupancy, the
+// dynamic shared-memory opt-in), so a decode call is one launch and no
+// repeated driver queries.
+struct HostCache {
+  std::mutex mu;
+  std::map<std::pair<const void*, int>, size_t> smem_optin;  // (kernel, device) -> bytes opted in
+  std::map<std::tuple<const void*, int, size_t>, int> occ;   // (kernel, device, smem) -> CTAs per SM
+  std::map<int, int> sms;                                    // device -> SM count
+};
+HostCache& host_cache() {
+  static HostCache c;
+  return c;
+}
+
+cudaError_t ensure_smem(const void* fn, size_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  HostCache& c = host_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  auto key = std::make_pair(fn, dev);
+  auto it = c.smem_optin.find(key);
+  if (it != c.smem_optin.end() && it->second >= smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) c.smem_optin[key] = smem;
+  return e;
+}
+
+int device_sms_and_occupancy(const void* fn, size_t smem, int threads, int* occ_out) {
+  int dev = 0, sms = 148, occ = 1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    *occ_out = 1;
+    return sms;
+  }
+  HostCache& c = host_cache();
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    auto s = c.sms.find(dev);
+    auto o = c.occ.find(std::make_tuple(fn, dev, smem));
+    if (s != c.sms.end() && o != c.occ.end()) {
+      *occ_out = o->second;
+      return s->second;
+    }
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (ensure_smem(fn, smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess || occ < 1)
+    occ = 1;
+  std::lock_guard<std::mutex> lock(c.mu);
+  c.sms[dev] = sms;
+  c.occ[std::make_tuple(fn, dev, smem)] = occ;
+  *occ_out = occ;
+  return sms;
+}
+
 struct KernelInfo {
-  const void* fn;
-  size_t smem_fixed;  // bytes without the (B + 1) prefix ints
+  const void* fn;          // persistent kernel
+  const void* cfn;         // cluster kernel (same tile shape)
+  size_t (*smem)(int B, int qmode, int Hd);
+  size_t (*csmem)(int qmode, int Hd);
   int tile;
 };
 
-template <int CODEC, int SEGS, int SPT, int QMODE>
+template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
 KernelInfo info() {
-  using C = SplitCfg<CODEC, SEGS, SPT>;
-  return KernelInfo{reinterpret_cast<const void*>(&split_decode_kernel<CODEC, SEGS, SPT, QMODE>),
-                    C::smem_bytes(0) - 4, C::kT};
+  using C = Cfg<CODEC, VPT, TPT, NTOK>;
+  return KernelInfo{reinterpret_cast<const void*>(&decode_kernel<CODEC, VPT, TPT, NTOK, QMODE>),
+                    reinterpret_cast<const void*>(&decode_cluster_kernel<CODEC, VPT, TPT, NTOK, QMODE>),
+                    &C::smem_bytes, &C::cluster_smem_bytes, C::kT};
 }
 
-// Supported instantiations: rows of 16..128 bytes for the quantised codecs,
-// 64..512 bytes (fp16 Hd 32..256) for dense, 256..2048 bytes for shared latents.
-bool pick(int codec, int rowbytes, int qmode, KernelInfo* ki) {
-  const int nseg = rowbytes / 16;
-  if (rowbytes % 16 || nseg < 1) return false;
+// Instantiated shapes.  `big` selects the variant with more tokens per lane per
+// tile (fewer, larger tiles) for long caches.
+bool pick(int codec, int rowbytes, int qmode, bool big, KernelInfo* ki) {
   if (qmode == kQProj && codec == kCodecI8) {
-    switch (nseg) {
-      case 1: *ki = info<kCodecI8, 1, 1, kQProj>(); return true;
-      case 2: *ki = info<kCodecI8, 2, 1, kQProj>(); return true;
-      case 4: *ki = info<kCodecI8, 4, 1, kQProj>(); return true;
-      case 8: *ki = info<kCodecI8, 8, 1, kQProj>(); return true;
+    switch (rowbytes) {
+      case 16: *ki = big ? info<kCodecI8, 16, 1, 4, kQProj>() : info<kCodecI8, 16, 1, 2, kQProj>(); return true;
+      case 32: *ki = big ? info<kCodecI8, 32, 1, 2, kQProj>() : info<kCodecI8, 32, 1, 1, kQProj>(); return true;
+      case 64: *ki = info<kCodecI8, 32, 2, 1, kQProj>(); return true;
+      case 128: *ki = info<kCodecI8, 32, 4, 1, kQProj>(); return true;
     }
   } else if (qmode == kQProj && codec == kCodecI4) {
-    switch (nseg) {
-      case 1: *ki = info<kCodecI4, 1, 1, kQProj>(); return true;
-      case 2: *ki = info<kCodecI4, 2, 1, kQProj>(); return true;
-      case 4: *ki = info<kCodecI4, 4, 1, kQProj>(); return true;
-      case 8: *ki = info<kCodecI4, 8, 1, kQProj>(); return true;
+    switch (rowbytes) {
+      case 16: *ki = big ? info<kCodecI4, 32, 1, 2, kQProj>() : info<kCodecI4, 32, 1, 1, kQProj>(); return true;
+      case 32: *ki = info<kCodecI4, 32, 2, 1, kQProj>(); return true;
+      case 64: *ki = info<kCodecI4, 32, 4, 1, kQProj>(); return true;
     }
   } else if (qmode == kQDirect && codec == kCodecF16) {
-    switch (nseg) {
-      case 8: *ki = info<kCodecF16, 8, 1, kQDirect>(); return true;
-      case 16: *ki = info<kCodecF16, 16, 1, kQDirect>(); return true;
-      case 32: *ki = info<kCodecF16, 32, 1, kQDirect>(); return true;
+    switch (rowbytes) {
+      case 64: *ki = info<kCodecF16, 16, 2, 2, kQDirect>(); return true;
+      case 128: *ki = info<kCodecF16, 16, 4, 2, kQDirect>(); return true;
+      case 256: *ki = info<kCodecF16, 16, 8, 2, kQDirect>(); return true;
+      case 512: *ki = info<kCodecF16, 16, 16, 2, kQDirect>(); return true;
     }
   } else if (qmode == kQGlobal && codec == kCodecF16) {
-    switch (nseg) {
-      case 16: *ki = info<kCodecF16, 16, 1, kQGlobal>(); return true;
-      case 32: *ki = info<kCodecF16, 32, 1, kQGlobal>(); return true;
-      case 64: *ki = info<kCodecF16, 32, 2, kQGlobal>(); return true;
-      case 128: *ki = info<kCodecF16, 32, 4, kQGlobal>(); return true;
+    switch (rowbytes) {
+      case 256: *ki = info<kCodecF16, 16, 8, 2, kQGlobal>(); return true;
+      case 512: *ki = info<kCodecF16, 16, 16, 2, kQGlobal>(); return true;
+      case 1024: *ki = info<kCodecF16, 16, 32, 1, kQGlobal>(); return true;
+      case 2048: *ki = info<kCodecF16, 32, 32, 1, kQGlobal>(); return true;
     }
   }
   return false;
@@ -562,51 +1074,64 @@ bool pick(int codec, int rowbytes, int qmode, KernelInfo* ki) {
 
 }  // namespace
 
-int split_decode_tile_tokens(int codec, int rowbytes) {
+bool decode_supported(int codec, int rowbytes, int qmode) {
   KernelInfo ki;
-  for (int qm : {kQProj, kQDirect, kQGlobal})
-    if (pick(codec, rowbytes, qm, &ki)) return ki.tile;
-  return 0;
+  return pick(codec, rowbytes, qmode, false, &ki) && pick(codec, rowbytes, qmode, true, &ki);
 }
 
-int split_decode_grid(int codec, int rowbytes, int qmode, int B, int H, int L_cap) {
-  KernelInfo ki;
-  if (!pick(codec, rowbytes, qmode, &ki)) return 0;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const size_t smem = ki.smem_fixed + (size_t)(B + 1) * 4;
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream) {
+  KernelInfo small, big;
+  if (!pick(codec, rowbytes, qmode, false, &small) || !pick(codec, rowbytes, qmode, true, &big))
+    return cudaErrorInvalidValue;
   int occ = 1;
-  cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ki.fn, kDecodeThreads, smem) != cudaSuccess || occ < 1)
-    occ = 1;
-  const long long tiles_max = (long long)B * H * ((L_cap + ki.tile - 1) / ki.tile);
+  const size_t smem_small = small.smem(a.B, qmode, a.Hd);
+  const int sms = device_sms_and_occupancy(small.fn, smem_small, kDecodeThreads, &occ);
+  const long long resident = (long long)sms * occ;
+  const long long tiles_small = (long long)a.B * a.H * ((a.L_cap + small.tile - 1) / small.tile);
+
+  // Few tiles per resident CTA: one cluster per (b, h), merged on chip (the
+  // low-rank and dense paths; B_Vh must fit in the leader's shared memory).
+  const size_t csmem = small.csmem(qmode, a.Hd);
+  if (tiles_small <= 2 * resident && qmode != kQGlobal && csmem <= 112 * 1024 && a.H <= 65535) {
+    const int csize = (int)std::min<long long>(kMaxClusterSize, std::max(1, (a.L_cap + 127) / 128));
+    const size_t smem = csmem;
+    cudaError_t e = ensure_smem(small.cfn, smem);
+    if (e != cudaSuccess) return e;
+    a.ctas = csize;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize, a.H, a.B);
+    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&a};
+    return cudaLaunchKernelExC(&cfg, small.cfn, args);
+  }
+
+  // Otherwise the persistent grid; the large-tile variant when there are several
+  // tiles per resident CTA.
+  const size_t smem_big = big.smem(a.B, qmode, a.Hd);
+  device_sms_and_occupancy(big.fn, smem_big, kDecodeThreads, &occ);
+  const long long tiles_big = (long long)a.B * a.H * ((a.L_cap + big.tile - 1) / big.tile);
+  const KernelInfo& ki = (tiles_big >= 4 * (long long)sms * occ) ? big : small;
+  const size_t smem = ki.smem(a.B, qmode, a.Hd);
+  device_sms_and_occupancy(ki.fn, smem, kDecodeThreads, &occ);
+  const long long tiles_max = (long long)a.B * a.H * ((a.L_cap + ki.tile - 1) / ki.tile);
   long long ctas = (long long)sms * occ;
   if (ctas > tiles_max) ctas = tiles_max;
   if (ctas > kMaxDecodeCtas) ctas = kMaxDecodeCtas;
   if (ctas < 1) ctas = 1;
-  return (int)ctas;
-}
-
-cudaError_t launch_split_decode(int codec, int rowbytes, int qmode, const SplitArgs& a, int* tile_tokens,
-                                cudaStream_t stream) {
-  KernelInfo ki;
-  if (!pick(codec, rowbytes, qmode, &ki)) return cudaErrorInvalidValue;
-  if (tile_tokens) *tile_tokens = ki.tile;
-  const size_t smem = ki.smem_fixed + (size_t)(a.B + 1) * 4;
-  cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  a.ctas = (int)ctas;
+  cudaError_t e = ensure_smem(ki.fn, smem);
   if (e != cudaSuccess) return e;
-  void* args[] = {const_cast<SplitArgs*>(&a)};
+  void* args[] = {&a};
   return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kDecodeThreads), args, smem, stream);
-}
-
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
-  const size_t smem = (size_t)a.W * 4;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  combine_kernel<<<a.B * a.H, 256, smem, stream>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace wsvd

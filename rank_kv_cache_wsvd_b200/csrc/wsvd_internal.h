@@ -17,7 +17,6 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumerThreads + 32;
-constexpr int kStages = 4;
 // Upper bound on the persistent grid; sizes the partial-result workspace.
 constexpr int kMaxDecodeCtas = 2048;
 
@@ -25,10 +24,10 @@ enum Codec { kCodecI8 = 0, kCodecI4 = 1, kCodecF16 = 2 };
 enum QMode { kQProj = 0, kQDirect = 1, kQGlobal = 2 };
 
 // Arguments of the persistent split-L decode kernel (one struct for every codec).
-struct SplitArgs {
+struct DecodeArgs {
   int B, H, Hd, W;       // W: latent width per token (r, Hd or R)
   int L_cap;
-  int ctas;              // persistent grid size C
+  int ctas;              // persistent grid size C (set by launch_decode)
   int heads_share;       // 1: the latent rows of (b, h) are the rows of b (shared-latent path)
   const int32_t* seq_lens;
   const void* q;
@@ -38,27 +37,18 @@ struct SplitArgs {
   const __half* scale_k; // per-token scales (quantised codecs only)
   const __half* scale_v;
   const __half* Bk;      // [H][W][Hd] (kQProj)
+  const __half* Bv;      // [H][W][Hd], or nullptr for the dense path (W == Hd)
   const float* qglobal;  // [B][H][W] (kQGlobal)
   float qscale;          // softmax_scale * log2(e)
-  float* partials;       // [(ctas + B*H)][W + 2]
-  int32_t* err;
-};
-
-struct CombineArgs {
-  int B, H, Hd, W, L_cap, ctas, tile;
-  const int32_t* seq_lens;
-  const float* partials;
-  const __half* Bv;      // [H][W][Hd], or nullptr for the dense path (W == Hd)
   float* out;            // [B][H][Hd]
+  float* partials;       // [(kMaxDecodeCtas + B*H)][W + 2]
+  int32_t* counters;     // [B*H], zero between calls
   int32_t* err;
 };
 
 // Host launchers (decode.cu, shared.cu, append.cu).  Return a cudaError_t.
-cudaError_t launch_split_decode(int codec, int rowbytes, int qmode, const SplitArgs& a, int* tile_tokens,
-                                cudaStream_t stream);
-int split_decode_tile_tokens(int codec, int rowbytes);
-int split_decode_grid(int codec, int rowbytes, int qmode, int B, int H, int L_cap);
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+bool decode_supported(int codec, int rowbytes, int qmode);
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream);
 cudaError_t launch_shared_qproj(int B, int H, int Hd, int R, const void* q, int q_dtype, const __half* Bk,
                                 float* qglobal, cudaStream_t stream);
 

@@ -57,11 +57,13 @@ def test_workspace_sizes_hold_only_partials(lib):
     """The decode workspace holds split partials (r + 2 floats per slot), never
     an L x Hd buffer: reconstructed K/V are not materialised."""
     B, H, r, L = 4, 32, 32, 32768
+    a16 = lambda v: (v + 15) // 16 * 16
     ws = W.wsvd_decode_workspace_size(B, H, r)
-    assert ws == (2048 + B * H) * (r + 2) * 4
+    assert ws == a16((2048 + B * H) * (r + 2) * 4) + a16(B * H * 4)  # partial slots + one counter per head
     assert ws < B * H * L * 128 * 2 / 100  # far below one reconstructed K
-    assert W.dense_decode_workspace_size(B, H, 128) == (2048 + B * H) * 130 * 4
-    assert W.shared_decode_workspace_size(B, H, 512) == (2048 + B * H) * 514 * 4 + B * H * 512 * 4
+    assert W.dense_decode_workspace_size(B, H, 128) == a16((2048 + B * H) * 130 * 4) + a16(B * H * 4)
+    assert W.shared_decode_workspace_size(B, H, 512) == (a16((2048 + B * H) * 514 * 4) + a16(B * H * 4)
+                                                         + B * H * 512 * 4)
     assert W.wsvd_append_workspace_size() == 256
 
 

@@ -31,7 +31,7 @@ def _cache(B, H, L_cap, r, bits, rng=None, fill=0):
     return lat, sc
 
 
-def _run_steps(w: WL.Workload, steps: int, lens0, blk=128, bits=None, seed=0, check_every=True):
+def _run_steps(w: WL.Workload, steps: int, lens0, blk=128, bits=None, seed=0):
     bits = w.bits if bits is None else bits
     ai = WL.append_inputs(w, seed=seed, steps=steps)
     rng = np.random.default_rng(seed + 1)
@@ -44,6 +44,7 @@ def _run_steps(w: WL.Workload, steps: int, lens0, blk=128, bits=None, seed=0, ch
     ws = W.workspace(W.wsvd_append_workspace_size())
     ties = [0, 0]
     o = dict(lat_k=lat_k, lat_v=lat_v, sk=sc_k, sv=sc_v, lens=lens)
+    before = {k: v.cpu().numpy() for k, v in g.items()}
     for s in range(steps):
         x = q_tensor(ai.x_bits[s], "bf16")
         W.wsvd_latent_append(x, A_k, A_v, g["lens"], g["lat_k"], g["lat_v"], g["sk"], g["sv"], bits=bits,
@@ -52,31 +53,29 @@ def _run_steps(w: WL.Workload, steps: int, lens0, blk=128, bits=None, seed=0, ch
         lk, sk, lv, sv, nl, oerr, ck, cv = O.latent_append(ai.x[s], ai.A_k, ai.A_v, o["lens"], o["lat_k"], o["sk"],
                                                             o["lat_v"], o["sv"], w.r, bits, blk)
         o = dict(lat_k=lk, lat_v=lv, sk=sk, sv=sv, lens=nl)
-        if check_every or s == steps - 1:
-            torch.cuda.synchronize()
-            gl = {k: v.cpu().numpy() for k, v in g.items()}
-            assert np.array_equal(gl["lens"], o["lens"]), (s, gl["lens"], o["lens"])
+        torch.cuda.synchronize()
+        gl = {k: v.cpu().numpy() for k, v in g.items()}
+        assert np.array_equal(gl["lens"], o["lens"]), (s, gl["lens"], o["lens"])
+        for b in range(w.B):
+            pos = int(prev[b])
+            if pos < 0 or pos >= w.L_cap:
+                continue
+            for which, c in (("k", ck), ("v", cv)):
+                gc = unpack(gl["lat_" + which][b, :, pos], w.r, bits)
+                oc = unpack(o["lat_" + which][b, :, pos], w.r, bits)
+                t = compare_codes(gc, gl["s" + which][b, :, pos], oc, o["s" + which][b, :, pos], c[b], bits)
+                ties[0] += t[0]
+                ties[1] += t[1]
+        # every other byte of the GPU cache is what it was before this call
+        for key in ("lat_k", "lat_v", "sk", "sv"):
+            a, bref = gl[key].copy(), before[key].copy()
             for b in range(w.B):
                 pos = int(prev[b])
-                if pos < 0 or pos >= w.L_cap:
-                    continue
-                for which, c in (("k", ck), ("v", cv)):
-                    gc = unpack(gl["lat_" + which][b, :, pos], w.r, bits)
-                    oc = unpack(o["lat_" + which][b, :, pos], w.r, bits)
-                    t = compare_codes(gc, gl["s" + which][b, :, pos], oc, o["s" + which][b, :, pos], c[b], bits)
-                    ties[0] += t[0]
-                    ties[1] += t[1]
-            # every other row is untouched: overwrite the written rows and compare bytes
-            for key in ("lat_k", "lat_v", "sk", "sv"):
-                a, bref = gl[key].copy(), o[key].copy()
-                for b in range(w.B):
-                    pos = int(prev[b])
-                    if 0 <= pos < w.L_cap:
-                        a[b, :, pos] = 0
-                        bref[b, :, pos] = 0
-                assert np.array_equal(a.view(np.uint8), bref.view(np.uint8)), (s, key)
-            if not check_every:
-                break
+                if 0 <= pos < w.L_cap:
+                    a[b, :, pos] = 0
+                    bref[b, :, pos] = 0
+            assert np.array_equal(a.view(np.uint8), bref.view(np.uint8)), (s, key)
+        before = gl
     torch.cuda.synchronize()
     return ties, int(err.item()), g, o
 
