@@ -109,6 +109,20 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def replica_throughput(units_local: float, seconds_local: float, world: int, device="cuda"):
+    """Whole-job throughput of N independent replicas: every rank processed
+    `units_local` units; the job's duration is the slowest rank's (max over
+    ranks).  Returns (units per second over all ranks, max seconds)."""
+    if world == 1:
+        return units_local / seconds_local, seconds_local
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t_max = float(t.item())
+    return units_local * world / t_max, t_max
+
+
 # ----------------------------------------------------------------------------- workloads
 def attended_tokens(w: WL.Workload, lens_after: np.ndarray) -> int:
     return int(lens_after.sum()) * w.H
@@ -358,13 +372,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     st = WsvdStep(w, seed=rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
@@ -426,12 +433,11 @@ def main():
     torch.cuda.synchronize()
     t_app = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3 / n_b * args.steps if st.has_append else 0.0
     t_dec = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3 / n_b * args.steps
-    t_total = max_over_ranks(t_step)
+    units_local = attended_tokens(w, st.lens_after) * args.steps
+    value, t_total = replica_throughput(units_local, t_step, world)
     if int(st.err.item()) != 0:
         raise RuntimeError(f"device error word {int(st.err.item())}")
 
-    units = attended_tokens(w, st.lens_after) * args.steps * world
-    value = units / t_total
     ms_per_step = t_total / args.steps * 1e3
     peak, peak_kind = peaks()
     dec_bytes = alg_bytes_decode(w, st.lens_after)
