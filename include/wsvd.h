@@ -117,6 +117,35 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
                           float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                           int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- WSVD decode without allocation
+ * The WSVD summaries have no counterpart to this entry point: it is a
+ * deployment convenience of this library.
+ *
+ * Same operation, arguments and results as wsvd_decode_attention, for callers
+ * that cannot call cudaMalloc: a serving runtime whose device memory is one
+ * pre-sized pool owned by another allocator, code that runs where a device
+ * allocation would synchronise the device or fail (inside latency-critical
+ * loops, under memory limits), or a host language binding without access to
+ * device allocation.  The scratch it needs (split partials and one counter
+ * per (b, h)) lives in a static device array of WSVD_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits; the call
+ * itself allocates nothing.
+ *   - A problem whose scratch need, wsvd_decode_workspace_size(B, H, r),
+ *     exceeds WSVD_NOALLOC_SCRATCH_BYTES is rejected with
+ *     WSVD_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call clears the counters it uses (an asynchronous memset on
+ *     `stream`), then launches the decode.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race and give wrong results.                  */
+#define WSVD_NOALLOC_SCRATCH_BYTES (2u << 20)
+int wsvd_decode_attention_noalloc(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                                  const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
+                                  const void* scale_k, const void* scale_v, const void* B_k, const void* B_v,
+                                  float softmax_scale, float* out, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------- latent append
  * Writes one new token per sequence into the latent cache (the projection of
  * the new token through A_Kh / A_Vh, German §2.A, after the Hadamard rotation

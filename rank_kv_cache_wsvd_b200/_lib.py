@@ -36,6 +36,7 @@ SIGNATURES = {
     "wsvd_append_workspace_size": (_c_size, []),
     "wsvd_decode_attention": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size,
                                                                                         _p, _p]),
+    "wsvd_decode_attention_noalloc": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _p]),
     "wsvd_latent_append": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 7 + [_p, _c_size, _p, _p]),
     "dense_decode_attention": (_c_int, [_c_int] * 4 + [_p, _p, _c_int, _p, _p, _c_float, _p, _p, _c_size, _p, _p]),
     "shared_latent_svd_decode": (_c_int, [_c_int] * 5 + [_p, _p, _c_int] + [_p] * 4 + [_c_float, _p, _p, _c_size,
