@@ -146,8 +146,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
     for (uint32_t off = 0; off < bytes; off += kPiece)
       bulk_g2s(smem + L.a_off + off, src + off, min(kPiece, bytes - off), bar_a, once);
   }
-  // Every CTA's barriers are initialised before any remote arrival.
-  cluster.sync();
+  // Every CTA's barriers are initialised before any remote access; the wait is
+  // deferred until the first access so the barrier latency overlaps the copies.
+  cluster.barrier_arrive();
 
   // 2. Rotate x: one warp per Hadamard block, butterflies with warp-level sync.
   if (!mbar_wait_bounded(bar_x, 0) && tid == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
 
   // 3. Wait for A (bounded), then the slice GEMV into this rank's slot of the leader.
   if (!mbar_wait_bounded(bar_a, 0) && tid == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+  cluster.barrier_wait();
   float* my_slot = cluster.map_shared_rank(slots, 0) + (size_t)rank * B * r;
   if (B == 1) gemv_slice<1>(As, xs, B, Ec, r, red, my_slot, tid);
   else if (B == 2) gemv_slice<2>(As, xs, B, Ec, r, red, my_slot, tid);

@@ -32,7 +32,8 @@
 // instead: one thread-block cluster per (b, h) splits the tokens and merges
 // through distributed shared memory (see below).
 //
-// Per CTA: one producer warp issues 1-D bulk copies (TMA, no multicast) of
+// Per CTA of the persistent kernel: one producer warp issues 1-D bulk copies
+// (TMA, no multicast) of
 // K codes, V codes and their scales into a shared-memory ring; eight consumer
 // warps each own NTOK tokens per tile (TPT adjacent lanes per token, VPT
 // values per lane), keep a per-lane online softmax and reduce across lanes /
@@ -68,7 +69,6 @@ struct CodecT<kCodecF16> {
   static constexpr bool kScaled = false;
 };
 
-constexpr int kMaxParts = kMaxDecodeCtas;
 constexpr int kMaxClusterSize = 8;
 
 // Per-(b, h) operands the producer stages next to the tiles: B_Kh and q (low-rank
@@ -79,6 +79,18 @@ __host__ __device__ inline size_t seg_bytes(int qmode, int W, int Hd) {
   return (b + 127) / 128 * 128;
 }
 __host__ __device__ inline int seg_nbuf(int qmode, int W, int Hd) { return seg_bytes(qmode, W, Hd) <= 17408 ? 2 : 1; }
+
+// Helper-owned shared state (after the operand buffers).
+template <int W, int PW>
+struct HelperArea {
+  float qsv[2][W];            // scaled q' (fp16 codecs read it directly)
+  uint32_t planes[2][PW];     // packed byte planes + int4 corrections
+  float qstep[2];
+  int seginfo[2][4];          // b, h, c_first, c_last
+  float res[2][W + 2];        // merged (M, L, O[W]) of a segment, consumers -> helper
+  int qi[W];                  // quantised q'
+  uint64_t bars[10];          // qready[2], qfree[2], resfull[2], resfree[2]
+};
 
 template <int CODEC, int VPT, int TPT, int NTOK>
 struct Cfg {
@@ -106,13 +118,14 @@ struct Cfg {
   static constexpr size_t kOffQ = kOffBar + 2 * kStages * 8 + 4 * 8;  // + segment full / empty barriers
   static constexpr size_t kOffRed = kOffQ + (size_t)kW * 4;
   static constexpr size_t kOffRes = kOffRed + (size_t)kRedFloats * 4;
+  static constexpr int kPlaneWords = TPT * (3 * kQW + 4);  // packed q' byte planes + corrections, per chunk
   static constexpr size_t kOffParts = kOffRes + (size_t)(kW + 2) * 4;
-  static constexpr size_t kOffMisc = kOffParts + (size_t)kMaxParts * 4;
+  static constexpr size_t kOffMisc = kOffParts + (size_t)kPlaneWords * 4;
   static constexpr size_t kOffPre = kOffMisc + 16 * 4;
   // runtime part: lens / prefix (2B + 1 ints), then the segment buffers
   __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(2 * B + 1) * 4 + 127) / 128 * 128; }
   static size_t smem_bytes(int B, int qmode, int Hd) {
-    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd);
+    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) + sizeof(HelperArea<kW, kPlaneWords>);
   }
   // cluster kernel: operands, the leader's partial slots, then B_Vh
   __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
@@ -131,15 +144,15 @@ struct QState<kCodecI8, VPT> {
   uint32_t qh[VPT / 4], qm[VPT / 4], ql[VPT / 4];  // signed high byte, unsigned middle / low bytes
   float step;
   __device__ __forceinline__ float dot(const uint4* seg) const {
-    int ah = 0, am = 0, al = 0;
+    int ah[2] = {0, 0}, am[2] = {0, 0}, al[2] = {0, 0};  // two chains per plane
 #pragma unroll
     for (int k = 0; k < VPT / 4; ++k) {
       const uint32_t w = reinterpret_cast<const uint32_t*>(seg)[k];
-      ah = dp4a_ss(w, qh[k], ah);
-      am = dp4a_su(w, qm[k], am);
-      al = dp4a_su(w, ql[k], al);
+      ah[k & 1] = dp4a_ss(w, qh[k], ah[k & 1]);
+      am[k & 1] = dp4a_su(w, qm[k], am[k & 1]);
+      al[k & 1] = dp4a_su(w, ql[k], al[k & 1]);
     }
-    return fmaf((float)ah, 65536.f, fmaf((float)am, 256.f, (float)al));
+    return fmaf((float)(ah[0] + ah[1]), 65536.f, fmaf((float)(am[0] + am[1]), 256.f, (float)(al[0] + al[1])));
   }
 };
 
@@ -150,20 +163,20 @@ struct QState<kCodecI4, VPT> {
   int ch, cm, cl;  // 8 * sum of each plane: removes the +8 offset of the nibbles
   float step;
   __device__ __forceinline__ float dot(const uint4* seg) const {
-    int ah = -ch, am = -cm, al = -cl;
+    int ah[2] = {-ch, 0}, am[2] = {-cm, 0}, al[2] = {-cl, 0};  // even / odd elements on separate chains
 #pragma unroll
     for (int k = 0; k < VPT / 8; ++k) {
       const uint32_t w = reinterpret_cast<const uint32_t*>(seg)[k];
       const uint32_t ev = (w & 0x0F0F0F0Fu) ^ 0x08080808u;         // c + 8 of elements 8k, 8k+2, ...
       const uint32_t od = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // c + 8 of elements 8k+1, 8k+3, ...
-      ah = dp4a_us(ev, qh[2 * k], ah);
-      ah = dp4a_us(od, qh[2 * k + 1], ah);
-      am = dp4a_uu(ev, qm[2 * k], am);
-      am = dp4a_uu(od, qm[2 * k + 1], am);
-      al = dp4a_uu(ev, ql[2 * k], al);
-      al = dp4a_uu(od, ql[2 * k + 1], al);
+      ah[0] = dp4a_us(ev, qh[2 * k], ah[0]);
+      ah[1] = dp4a_us(od, qh[2 * k + 1], ah[1]);
+      am[0] = dp4a_uu(ev, qm[2 * k], am[0]);
+      am[1] = dp4a_uu(od, qm[2 * k + 1], am[1]);
+      al[0] = dp4a_uu(ev, ql[2 * k], al[0]);
+      al[1] = dp4a_uu(od, ql[2 * k + 1], al[1]);
     }
-    return fmaf((float)ah, 65536.f, fmaf((float)am, 256.f, (float)al));
+    return fmaf((float)(ah[0] + ah[1]), 65536.f, fmaf((float)(am[0] + am[1]), 256.f, (float)(al[0] + al[1])));
   }
 };
 
@@ -286,40 +299,46 @@ __device__ __forceinline__ void csync() { named_barrier_sync(1, kConsumerThreads
 // row, scaled by softmax_scale * log2 e), then the lane's 24-bit fixed-point
 // byte planes (step = max|q'| / 2^23).  fp16 paths: q or the projected q'.
 // Contains consumer-group barriers.
+// q'[j] = (B_Kh . q)[j] * qscale for rows j = j0, j0 + jstep, ...: eight lanes per
+// row (part = lane & 7) sum columns part, part + 8, ... from a row-dependent
+// rotation (distinct banks across the warp's rows), then a fixed shuffle tree.
+// Every builder uses this routine, so q' is bit-identical whoever builds it.
+// Returns this lane's max |q'| over its rows.
+__device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, const DecodeArgs& a, int W, int j0,
+                                            int jstep, int part) {
+  const __half* Bs = reinterpret_cast<const __half*>(sbuf);
+  const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * 2);
+  const int cols = a.Hd >> 3;
+  float amax = 0.f;
+  for (int j = j0; j < W; j += jstep) {
+    const __half* row = Bs + (size_t)j * a.Hd;
+    float d = 0.f;
+    for (int k = 0; k < cols; ++k) {
+      const int col = ((k + j) % cols) * 8 + part;
+      const uint16_t qu = qsrc[col];
+      const float qv = (a.q_dtype == WSVD_DTYPE_BF16) ? __uint_as_float((uint32_t)qu << 16)
+                                                       : __half2float(__ushort_as_half(qu));
+      d = fmaf(__half2float(row[col]), qv, d);
+    }
+    d += __shfl_xor_sync(0xffffffffu, d, 1);
+    d += __shfl_xor_sync(0xffffffffu, d, 2);
+    d += __shfl_xor_sync(0xffffffffu, d, 4);
+    d *= a.qscale;
+    amax = fmaxf(amax, fabsf(d));
+    if (part == 0) qs[j] = d;
+  }
+  return amax;
+}
+
 template <int CODEC, int VPT, int W, int QMODE>
 __device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8_t* sbuf, float* qs, float* misc,
-                                            const DecodeArgs& a, int tid, int sub) {
+                                            uint32_t* planes, const DecodeArgs& a, int tid, int sub) {
   using CT = CodecT<CODEC>;
+  constexpr int QW = VPT / 4;
   const int warp = tid >> 5, lane = tid & 31;
   float amax = 0.f;
   if (QMODE == kQProj) {
-    const __half* Bs = reinterpret_cast<const __half*>(sbuf);
-    const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * 2);
-    const int part = tid & 7, cols = a.Hd >> 3;
-    for (int j = tid >> 3; j < W; j += kConsumerThreads / 8) {
-      const __half* row = Bs + (size_t)j * a.Hd + part * cols;
-      const uint16_t* qq = qsrc + part * cols;
-      float d = 0.f;
-      for (int k = 0; k < cols; k += 2) {
-        const float2 bw = __half22float2(*reinterpret_cast<const __half2*>(row + k));
-        float q0, q1;
-        if (a.q_dtype == WSVD_DTYPE_BF16) {
-          q0 = __uint_as_float((uint32_t)qq[k] << 16);
-          q1 = __uint_as_float((uint32_t)qq[k + 1] << 16);
-        } else {
-          q0 = __half2float(__ushort_as_half(qq[k]));
-          q1 = __half2float(__ushort_as_half(qq[k + 1]));
-        }
-        d = fmaf(bw.x, q0, d);
-        d = fmaf(bw.y, q1, d);
-      }
-      d += __shfl_xor_sync(0xffffffffu, d, 1);
-      d += __shfl_xor_sync(0xffffffffu, d, 2);
-      d += __shfl_xor_sync(0xffffffffu, d, 4);
-      d *= a.qscale;
-      amax = fmaxf(amax, fabsf(d));
-      if (part == 0) qs[j] = d;
-    }
+    amax = qprime_rows(sbuf, qs, a, W, tid >> 3, kConsumerThreads / 8, tid & 7);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   } else if (QMODE == kQDirect) {
@@ -334,56 +353,59 @@ __device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8
   if (CT::kScaled && lane == 0) misc[warp] = amax;
   csync();
   if constexpr (CT::kScaled) {
+    constexpr int TPT = W / VPT;
     float M = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, misc[w]);
     const float inv = M > 0.f ? 8388607.f / M : 0.f;
     qst.step = M > 0.f ? M / 8388607.f : 0.f;
-    auto qint = [&](int v) {
-      const int x = __float2int_rn(qs[sub * VPT + v] * inv);
+    auto qint = [&](int e) {
+      const int x = __float2int_rn(qs[e] * inv);
       return max(-8388607, min(8388607, x));
     };
-    if constexpr (CODEC == kCodecI8) {
+    // Pack each (chunk, plane word) once: planes[(s*3 + plane)*QW + k].
+    for (int idx = tid; idx < TPT * QW; idx += kConsumerThreads) {
+      const int s2 = idx / QW, k = idx % QW;
+      uint32_t h4 = 0, m4 = 0, l4 = 0;
 #pragma unroll
-      for (int k = 0; k < VPT / 4; ++k) {
-        uint32_t h4 = 0, m4 = 0, l4 = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int x = qint(4 * k + i);
-          h4 |= ((uint32_t)(x >> 16) & 0xFFu) << (8 * i);
-          m4 |= ((uint32_t)(x >> 8) & 0xFFu) << (8 * i);
-          l4 |= ((uint32_t)x & 0xFFu) << (8 * i);
-        }
-        qst.qh[k] = h4;
-        qst.qm[k] = m4;
-        qst.ql[k] = l4;
+      for (int i = 0; i < 4; ++i) {
+        // int8: element 4k+i; int4: even/odd elements of source word k/2
+        const int e = s2 * VPT + (CODEC == kCodecI8 ? 4 * k + i : 8 * (k >> 1) + 2 * i + (k & 1));
+        const int x = qint(e);
+        h4 |= ((uint32_t)(x >> 16) & 0xFFu) << (8 * i);
+        m4 |= ((uint32_t)(x >> 8) & 0xFFu) << (8 * i);
+        l4 |= ((uint32_t)x & 0xFFu) << (8 * i);
       }
-    } else {
-      int sh = 0, sm = 0, sl = 0;
-#pragma unroll
-      for (int k = 0; k < VPT / 8; ++k) {
-#pragma unroll
-        for (int par = 0; par < 2; ++par) {
-          uint32_t h4 = 0, m4 = 0, l4 = 0;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int x = qint(8 * k + 2 * i + par);
-            const int hb = x >> 16, mb = (x >> 8) & 0xFF, lb = x & 0xFF;
-            sh += hb;
-            sm += mb;
-            sl += lb;
-            h4 |= ((uint32_t)hb & 0xFFu) << (8 * i);
-            m4 |= (uint32_t)mb << (8 * i);
-            l4 |= (uint32_t)lb << (8 * i);
-          }
-          qst.qh[2 * k + par] = h4;
-          qst.qm[2 * k + par] = m4;
-          qst.ql[2 * k + par] = l4;
+      planes[(s2 * 3 + 0) * QW + k] = h4;
+      planes[(s2 * 3 + 1) * QW + k] = m4;
+      planes[(s2 * 3 + 2) * QW + k] = l4;
+    }
+    if (CODEC == kCodecI4) {
+      // 8 * sum of each plane over the chunk: removes the +8 offset of the nibbles
+      for (int s2 = tid; s2 < TPT; s2 += kConsumerThreads) {
+        int sh = 0, sm = 0, sl = 0;
+        for (int v = 0; v < VPT; ++v) {
+          const int x = qint(s2 * VPT + v);
+          sh += x >> 16;
+          sm += (x >> 8) & 0xFF;
+          sl += x & 0xFF;
         }
+        planes[TPT * 3 * QW + s2 * 3 + 0] = (uint32_t)(8 * sh);
+        planes[TPT * 3 * QW + s2 * 3 + 1] = (uint32_t)(8 * sm);
+        planes[TPT * 3 * QW + s2 * 3 + 2] = (uint32_t)(8 * sl);
       }
-      qst.ch = 8 * sh;
-      qst.cm = 8 * sm;
-      qst.cl = 8 * sl;
+    }
+    csync();
+#pragma unroll
+    for (int k = 0; k < QW; ++k) {
+      qst.qh[k] = planes[(sub * 3 + 0) * QW + k];
+      qst.qm[k] = planes[(sub * 3 + 1) * QW + k];
+      qst.ql[k] = planes[(sub * 3 + 2) * QW + k];
+    }
+    if constexpr (CODEC == kCodecI4) {
+      qst.ch = (int)planes[TPT * 3 * QW + sub * 3 + 0];
+      qst.cm = (int)planes[TPT * 3 * QW + sub * 3 + 1];
+      qst.cl = (int)planes[TPT * 3 * QW + sub * 3 + 2];
     }
   } else {
 #pragma unroll
@@ -438,117 +460,142 @@ __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QSt
   }
 }
 
-// Merges every consumer lane's (m, l, acc) into res[] = (M, L, O[W]).
-// Lanes holding the same chunk (same sub) merge by shuffles, warps through red[].
+// Butterfly reduce-scatter across the lanes that share a chunk (lane offsets
+// O, O/2, ..., TPT): each round a lane keeps half of its values and adds the
+// partner's matching half, so the values to move halve every round.
+template <int CUR, int O, int TPT>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+  if constexpr (O >= TPT) {
+    if constexpr (CUR >= 2) {
+      constexpr int HALF = CUR / 2;
+      const bool up = lane & O;
+#pragma unroll
+      for (int j = 0; j < HALF; ++j) {
+        const float send = up ? v[j] : v[j + HALF];
+        const float keep = up ? v[j + HALF] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      reduce_scatter<HALF, O / 2, TPT>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      reduce_scatter<1, O / 2, TPT>(v, lane);
+    }
+  }
+}
+
+// First element index held by a lane after reduce_scatter (values j = 0.. are consecutive).
+template <int CUR, int O, int TPT>
+__device__ __forceinline__ int scatter_base(int lane) {
+  if constexpr (O >= TPT && CUR >= 2) {
+    return ((lane & O) ? CUR / 2 : 0) + scatter_base<CUR / 2, O / 2, TPT>(lane);
+  } else {
+    return 0;
+  }
+}
+
+// Merges every consumer lane's (m, l, acc) into res[] = (M, L, O[W]): a common
+// maximum per chunk, a butterfly reduce-scatter inside each warp, then the
+// eight warps through red[] (8*W floats of warp partials, then (M, l) pairs).
 template <int VPT, int TPT, int W>
 __device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, float* red, float* res, int tid) {
   constexpr int NP = VPT / 2;
+  constexpr int FINAL = (VPT * TPT >= 32) ? VPT * TPT / 32 : 1;
   const int warp = tid >> 5, lane = tid & 31, sub = tid % TPT;
+  float M = m;
 #pragma unroll
-  for (int o = TPT; o < 32; o <<= 1) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-    const float M = fmaxf(m, mo);
-    const float f1 = (m == kNegInf) ? 0.f : ex2(m - M);
-    const float f2 = (mo == kNegInf) ? 0.f : ex2(mo - M);
-    l = l * f1 + lo * f2;
+  for (int o = TPT; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float f = (m == kNegInf) ? 0.f : ex2(m - M);
+  l *= f;
 #pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      float2 ao;
-      ao.x = __shfl_xor_sync(0xffffffffu, acc[p].x, o);
-      ao.y = __shfl_xor_sync(0xffffffffu, acc[p].y, o);
-      acc[p] = __ffma2_rn(acc[p], make_float2(f1, f1), __fmul2_rn(ao, make_float2(f2, f2)));
-    }
-    m = M;
+  for (int o = TPT; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  float v[VPT];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    v[2 * p] = acc[p].x * f;
+    v[2 * p + 1] = acc[p].y * f;
   }
-  if (lane < TPT) {
-    float* rw = red + (warp * TPT + sub) * (VPT + 2);
-    rw[0] = m;
-    rw[1] = l;
+  reduce_scatter<VPT, 16, TPT>(v, lane);
+  const int base = sub * VPT + scatter_base<VPT, 16, TPT>(lane);
+  float* wp = red + (size_t)warp * W;
 #pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      rw[2 + 2 * p] = acc[p].x;
-      rw[3 + 2 * p] = acc[p].y;
-    }
+  for (int j = 0; j < FINAL; ++j) wp[base + j] = v[j];
+  float* ml = red + (size_t)kConsumerWarps * W;
+  if (lane == 0) {
+    ml[2 * warp] = M;
+    ml[2 * warp + 1] = l;
   }
   csync();
-  float M = kNegInf;
+  float Mg = kNegInf;
 #pragma unroll
-  for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[w * TPT * (VPT + 2)]);
-  float f[kConsumerWarps];
+  for (int w = 0; w < kConsumerWarps; ++w) Mg = fmaxf(Mg, ml[2 * w]);
+  float fw[kConsumerWarps];
 #pragma unroll
-  for (int w = 0; w < kConsumerWarps; ++w) {
-    const float mw = red[w * TPT * (VPT + 2)];
-    f[w] = (mw == kNegInf) ? 0.f : ex2(mw - M);
-  }
+  for (int w = 0; w < kConsumerWarps; ++w) fw[w] = (ml[2 * w] == kNegInf) ? 0.f : ex2(ml[2 * w] - Mg);
   for (int e = tid; e < W; e += kConsumerThreads) {
-    const int se = e / VPT, v = e % VPT;
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) s = fmaf(f[w], red[(w * TPT + se) * (VPT + 2) + 2 + v], s);
+    for (int w = 0; w < kConsumerWarps; ++w) s = fmaf(fw[w], red[(size_t)w * W + e], s);
     res[2 + e] = s;
   }
   if (tid == 0) {
     float ls = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) ls = fmaf(f[w], red[w * TPT * (VPT + 2) + 1], ls);
-    res[0] = M;
+    for (int w = 0; w < kConsumerWarps; ++w) ls = fmaf(fw[w], ml[2 * w + 1], ls);
+    res[0] = Mg;
     res[1] = ls;
   }
   csync();
 }
 
-// Merges rows p of a partial array part[p][W + 2] (m, l, o[W]), p < np, into
-// res[], staging chunks of rows in red[] (nred floats).  ldcg selects
-// L2-coherent global loads (rows written by other CTAs).
+// Merges rows p < np of a partial array part[p][W + 2] = (m, l, o[W]) into
+// res[]: M = max_p m_p, then for every element (l, o[0..W)) the sum over p in
+// ascending order of 2^(m_p - M) * value.  Each element is computed by one
+// thread with the same operation order whatever the thread count, so a
+// warp and a thread block give identical bits.  ldcg selects L2-coherent
+// loads (rows written by other CTAs).
 template <int W, bool GLOBAL>
-__device__ __forceinline__ void merge_rows(const float* part, int np, float* red, int nred, float* res, int tid) {
-  const int rows = max(1, nred / (W + 2));
-  float Mrun = kNegInf;
-  for (int p0 = 0; p0 < np; p0 += rows) {
-    const int nr = min(rows, np - p0);
-    for (int i = tid; i < nr * (W + 2); i += kConsumerThreads)
-      red[i] = GLOBAL ? __ldcg(part + (size_t)p0 * (W + 2) + i) : part[(size_t)p0 * (W + 2) + i];
-    csync();
-    float M = Mrun;
-    for (int p = 0; p < nr; ++p) M = fmaxf(M, red[p * (W + 2)]);
-    const float fold = (Mrun == kNegInf) ? 0.f : ex2(Mrun - M);
-    for (int e = tid; e < W + 1; e += kConsumerThreads) {  // e = 0: l, e >= 1: o[e - 1]
-      float s2 = (p0 == 0) ? 0.f : res[1 + e] * fold;
-      for (int p = 0; p < nr; ++p) {
-        const float mp = red[p * (W + 2)];
-        if (mp != kNegInf) s2 = fmaf(ex2(mp - M), red[p * (W + 2) + 1 + e], s2);
-      }
-      res[1 + e] = s2;
+__device__ __forceinline__ float merge_elem(const float* part, int np, float M, int e) {
+  float s2 = 0.f;
+  for (int p = 0; p < np; ++p) {
+    const float mp = GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)];
+    if (mp != kNegInf) {
+      const float v = GLOBAL ? __ldcg(part + (size_t)p * (W + 2) + 1 + e) : part[(size_t)p * (W + 2) + 1 + e];
+      s2 = fmaf(ex2(mp - M), v, s2);
     }
-    Mrun = M;
-    csync();
   }
-  if (tid == 0) res[0] = Mrun;
+  return s2;
+}
+template <int W, bool GLOBAL>
+__device__ __forceinline__ float merge_max(const float* part, int np) {
+  float M = kNegInf;
+  for (int p = 0; p < np; ++p) M = fmaxf(M, GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)]);
+  return M;
+}
+// Thread-block version (consumer threads).
+template <int W, bool GLOBAL>
+__device__ __forceinline__ void merge_rows(const float* part, int np, float* res, int tid) {
+  const float M = merge_max<W, GLOBAL>(part, np);
+  for (int e = tid; e < W + 1; e += kConsumerThreads) res[1 + e] = merge_elem<W, GLOBAL>(part, np, M, e);
+  if (tid == 0) res[0] = M;
   csync();
 }
 
-// out = O . Bv / L for the merged res[] (Bv [W][Hd] fp16, global or shared;
-// null: the dense path, out = O / L).  L = 0 (no tokens) gives zeros.
+// One output column: (sum over e ascending of O[e] * Bv[e][d]) / L; dense path
+// (Bv null): O[d] / L.  L = 0 (no tokens) gives zero.
+template <int W>
+__device__ __forceinline__ float out_col(const float* res, const __half* Bv, int Hd, int d) {
+  const float inv = res[1] > 0.f ? 1.f / res[1] : 0.f;
+  if (Bv == nullptr) return res[2 + d] * inv;
+  float s = 0.f;
+  for (int e = 0; e < W; ++e) s = fmaf(res[2 + e], __half2float(Bv[(size_t)e * Hd + d]), s);
+  return s * inv;
+}
+
+// out[b, h, :] from the merged res[] (consumer threads; see out_col).
 template <int W>
 __device__ __forceinline__ void finalize_out(const float* res, const __half* Bv, float* outp, int Hd, float* red,
                                              int tid) {
-  const float inv = res[1] > 0.f ? 1.f / res[1] : 0.f;
-  if (Bv == nullptr) {
-    for (int d = tid; d < Hd; d += kConsumerThreads) outp[d] = res[2 + d] * inv;
-    return;
-  }
-  const int ng = kConsumerThreads / Hd;  // e-groups per output column (Hd divides 256)
-  const int d = tid % Hd, grp = tid / Hd;
-  float s = 0.f;
-  for (int e = grp; e < W; e += ng) s = fmaf(res[2 + e], __half2float(Bv[(size_t)e * Hd + d]), s);
-  red[tid] = s;
-  csync();
-  if (tid < Hd) {
-    float t = 0.f;
-    for (int q = 0; q < ng; ++q) t += red[q * Hd + tid];
-    outp[tid] = t * inv;
-  }
+  for (int d = tid; d < Hd; d += kConsumerThreads) outp[d] = out_col<W>(res, Bv, Hd, d);
   csync();
 }
 
@@ -591,10 +638,95 @@ __device__ __forceinline__ void issue_tile(uint8_t* st, uint64_t* bar, const Dec
 }
 
 // ------------------------------------------------------------------ persistent kernel
+// Warp roles: warps 0-7 consume tiles, warp 8 is the producer (TMA), warp 9 the
+// helper.  The helper builds each (b, h)'s query state (q' and its byte planes)
+// one segment ahead of the consumers and finishes each segment after them
+// (partial write, completion counter, last-arriver merge, B_Vh up-projection),
+// so the consumers only stream tiles and reduce their own registers.
+
+// Warp-level q' = B_Kh . q from the staged operands: lane j-rotation keeps the
+// row reads on distinct banks.  Returns max|q'| (scaled by softmax_scale * log2 e).
+template <int W, int QMODE>
+__device__ __forceinline__ float helper_qprime(const uint8_t* sbuf, float* qsv, const DecodeArgs& a, int lane) {
+  float amax = 0.f;
+  if (QMODE == kQProj) {
+    amax = qprime_rows(sbuf, qsv, a, W, lane >> 3, 4, lane & 7);
+  } else if (QMODE == kQDirect) {
+    const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf);
+    for (int j = lane; j < W; j += 32)
+      qsv[j] = (a.q_dtype == WSVD_DTYPE_BF16 ? __uint_as_float((uint32_t)qsrc[j] << 16)
+                                             : __half2float(__ushort_as_half(qsrc[j]))) * a.qscale;
+  } else {
+    const float* qg = reinterpret_cast<const float*>(sbuf);
+    for (int j = lane; j < W; j += 32) qsv[j] = qg[j] * a.qscale;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  return amax;
+}
+
+// Warp-level packing of the 24-bit fixed-point q' into byte planes (see QState).
+template <int CODEC, int VPT, int W>
+__device__ __forceinline__ void helper_planes(const float* qsv, int* qi, uint32_t* planes, float* qstep, float amax,
+                                              int lane) {
+  constexpr int TPT = W / VPT, QW = VPT / 4;
+  const float inv = amax > 0.f ? 8388607.f / amax : 0.f;
+  *qstep = amax > 0.f ? amax / 8388607.f : 0.f;
+  for (int j = lane; j < W; j += 32) qi[j] = max(-8388607, min(8388607, __float2int_rn(qsv[j] * inv)));
+  __syncwarp();
+  for (int idx = lane; idx < TPT * QW; idx += 32) {
+    const int s2 = idx / QW, k = idx % QW;
+    uint32_t h4 = 0, m4 = 0, l4 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = s2 * VPT + (CODEC == kCodecI8 ? 4 * k + i : 8 * (k >> 1) + 2 * i + (k & 1));
+      const int x = qi[e];
+      h4 |= ((uint32_t)(x >> 16) & 0xFFu) << (8 * i);
+      m4 |= ((uint32_t)(x >> 8) & 0xFFu) << (8 * i);
+      l4 |= ((uint32_t)x & 0xFFu) << (8 * i);
+    }
+    planes[(s2 * 3 + 0) * QW + k] = h4;
+    planes[(s2 * 3 + 1) * QW + k] = m4;
+    planes[(s2 * 3 + 2) * QW + k] = l4;
+  }
+  if (CODEC == kCodecI4) {
+    for (int s2 = 0; s2 < TPT; ++s2) {
+      int sh = 0, sm = 0, sl = 0;
+      for (int v = lane; v < VPT; v += 32) {
+        const int x = qi[s2 * VPT + v];
+        sh += x >> 16;
+        sm += (x >> 8) & 0xFF;
+        sl += x & 0xFF;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sh += __shfl_xor_sync(0xffffffffu, sh, o);
+        sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        sl += __shfl_xor_sync(0xffffffffu, sl, o);
+      }
+      if (lane == 0) {
+        planes[TPT * 3 * QW + s2 * 3 + 0] = (uint32_t)(8 * sh);
+        planes[TPT * 3 * QW + s2 * 3 + 1] = (uint32_t)(8 * sm);
+        planes[TPT * 3 * QW + s2 * 3 + 2] = (uint32_t)(8 * sl);
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// Warp-level out[b, h, :] (same per-column arithmetic as finalize_out).
+template <int W>
+__device__ __forceinline__ void helper_finalize(const float* res, const __half* Bv, float* outp, int Hd, int lane) {
+  for (int d = lane; d < Hd; d += 32) outp[d] = out_col<W>(res, Bv, Hd, d);
+}
+
 template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const DecodeArgs a) {
   using C = Cfg<CODEC, VPT, TPT, NTOK>;
-  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2;
+  using CT = typename C::CT;
+  using HA = HelperArea<C::kW, C::kPlaneWords>;
+  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2, QW = VPT / 4;
+  constexpr int kProducerWarp = kConsumerWarps, kHelperWarp = kConsumerWarps + 1;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
@@ -602,15 +734,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
   uint64_t* empty = full + S;
   uint64_t* segfull = empty + S;  // [2]
   uint64_t* segempty = segfull + 2;
-  float* qs = reinterpret_cast<float*>(smem + C::kOffQ);
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
-  float* res = reinterpret_cast<float*>(smem + C::kOffRes);
-  float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
   int* pre = reinterpret_cast<int*>(smem + C::kOffPre);
   int* lens = pre + a.B + 1;
   uint8_t* segbuf = smem + C::seg_off(a.B);
   const int NBUF = seg_nbuf(QMODE, W, a.Hd);
   const uint32_t SEGB = (uint32_t)seg_bytes(QMODE, W, a.Hd);
+  HA* ha = reinterpret_cast<HA*>(segbuf + (size_t)NBUF * SEGB);
+  uint64_t* qready = ha->bars;
+  uint64_t* qfree = ha->bars + 2;
+  uint64_t* resfull = ha->bars + 4;
+  uint64_t* resfree = ha->bars + 6;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
@@ -646,7 +780,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
       }
       for (int s = 0; s < 2; ++s) {
         mbar_init(&segfull[s], 1);
-        mbar_init(&segempty[s], kConsumerWarps);
+        mbar_init(&segempty[s], 1);
+        mbar_init(&qready[s], 1);
+        mbar_init(&qfree[s], kConsumerWarps);
+        mbar_init(&resfull[s], 1);
+        mbar_init(&resfree[s], 1);
       }
       fence_mbar_init();
     }
@@ -668,7 +806,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
   const long long g_begin = G * c / CW, g_end = G * (c + 1) / CW;
 
   // ---------------------------------------------------------------- producer warp
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy(), keep = l2_evict_last_policy();
       int b, h, t;
@@ -708,87 +846,235 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(const DecodeA
     return;
   }
 
+  // ---------------------------------------------------------------- helper warp
+  if (warp == kHelperWarp) {
+    int b = 0, h = 0, t = 0;
+    walk.locate(g_begin, b, h, t);
+    long long g = g_begin;
+    // next (b, h) segment of this CTA's tile range, or false at the end
+    auto next_segment = [&](int& sbk, int& shk) {
+      if (g >= g_end) return false;
+      sbk = b;
+      shk = h;
+      while (g < g_end && b == sbk && h == shk) {
+        walk.advance(b, h, t);
+        ++g;
+      }
+      return true;
+    };
+    bool timed_out = false;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (!mbar_wait_bounded(bar, parity, timed_out ? 0ull : kWaitLimitNs)) {
+        if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        timed_out = true;
+      }
+    };
+    int built = 0, done = 0;
+    bool more = true;
+    {  // segment 0: the consumers build its query state; record what finishing it needs
+      int sb_b, sb_h;
+      if (next_segment(sb_b, sb_h)) {
+        const int tb = walk.tiles(sb_b);
+        const long long gf = (long long)a.H * pre[sb_b] + (long long)sb_h * tb;
+        if (lane == 0) {
+          ha->seginfo[0][0] = sb_b;
+          ha->seginfo[0][1] = sb_h;
+          ha->seginfo[0][2] = cta_of(gf, G, CW);
+          ha->seginfo[0][3] = cta_of(gf + tb - 1, G, CW);
+        }
+        built = 1;
+      } else {
+        more = false;
+      }
+    }
+    while (true) {
+      // Build up to one segment ahead of the oldest unfinished one.
+      while (more && built <= done + 1) {
+        int sb_b, sb_h;
+        if (!next_segment(sb_b, sb_h)) {
+          more = false;
+          break;
+        }
+        const int k = built, sq = k & 1;
+        const int tb = walk.tiles(sb_b);
+        const long long gf = (long long)a.H * pre[sb_b] + (long long)sb_h * tb;
+        const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
+        if (lane == 0) {
+          ha->seginfo[sq][0] = sb_b;
+          ha->seginfo[sq][1] = sb_h;
+          ha->seginfo[sq][2] = cf;
+          ha->seginfo[sq][3] = cl;
+        }
+        if (a.Bv != nullptr && c == cl) {  // the likely finisher warms B_Vh in L2
+          const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)sb_h * W * a.Hd);
+          for (int o = lane * 128; o < W * a.Hd * 2; o += 32 * 128) prefetch_l2(bv + o);
+        }
+        wait(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1));
+        if (k >= 2) wait(&qfree[sq], (uint32_t)(((k / 2) - 1) & 1));
+        const float amax = helper_qprime<W, QMODE>(segbuf + (size_t)(k % NBUF) * SEGB, ha->qsv[sq], a, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&segempty[k % NBUF]);  // the staged operands are consumed
+        if constexpr (CT::kScaled) {
+          helper_planes<CODEC, VPT, W>(ha->qsv[sq], ha->qi, ha->planes[sq], &ha->qstep[sq], amax, lane);
+        } else {
+          if (lane == 0) ha->qstep[sq] = 1.f;
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(&qready[sq]);
+        ++built;
+      }
+      // The consumers finish the CTA's last segment themselves.
+      if (done == built || (!more && done == built - 1)) break;
+      // Finish segment `done` once the consumers have reduced it.
+      const int k = done, sr = k & 1;
+      wait(&resfull[sr], (uint32_t)((k / 2) & 1));
+      const float* res = ha->res[sr];
+      const int sb_b = ha->seginfo[sr][0], sb_h = ha->seginfo[sr][1];
+      const int cf = ha->seginfo[sr][2], cl = ha->seginfo[sr][3];
+      float* outp = a.out + ((size_t)sb_b * a.H + sb_h) * a.Hd;
+      const __half* Bvh = a.Bv ? a.Bv + (size_t)sb_h * W * a.Hd : nullptr;
+      if (cf == cl) {
+        helper_finalize<W>(res, Bvh, outp, a.Hd, lane);
+      } else {
+        const int bh = sb_b * a.H + sb_h;
+        float* dst = a.partials + ((size_t)c + bh) * (W + 2);
+        for (int e = lane; e < W + 2; e += 32) dst[e] = res[e];
+        __threadfence();  // publish before the counter bump
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(&a.counters[bh], 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == cl - cf) {  // last arriver: merge every partial of (b, h) in CTA order
+          __threadfence();
+          const int np = cl - cf + 1;
+          const float* part = a.partials + ((size_t)cf + bh) * (W + 2);
+          const float M = merge_max<W, true>(part, np);
+          float* mres = ha->res[sr];  // reuse the segment's slot for the merged result
+          for (int e = lane; e < W + 1; e += 32) mres[1 + e] = merge_elem<W, true>(part, np, M, e);
+          __syncwarp();
+          helper_finalize<W>(mres, Bvh, outp, a.Hd, lane);
+          if (lane == 0) atomicExch(&a.counters[bh], 0);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&resfree[sr]);
+      ++done;
+    }
+    return;
+  }
+
   // ---------------------------------------------------------------- consumer warps
   const int sub = tid % TPT;
   QState<CODEC, VPT> qst;
   float2 acc[NP];
   float m = kNegInf, l = 0.f;
   bool timed_out = false;
-  int nseg = 0;
-
-  auto flush = [&](int b, int h, int c_first, int c_last) {
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (!mbar_wait_bounded(bar, parity, timed_out ? 0ull : kWaitLimitNs)) {
+      if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      timed_out = true;
+    }
+  };
+  int k = 0;  // segments started
+  auto end_segment = [&](int j) {  // hand segment j to the helper
+    const int sr = j & 1;
+    if (j >= 2) wait(&resfree[sr], (uint32_t)(((j / 2) - 1) & 1));
+    reduce_to_res<VPT, TPT, W>(m, l, acc, red, ha->res[sr], tid);
+    if (tid == 0) mbar_arrive(&resfull[sr]);
+  };
+  // The CTA's last segment: every consumer thread finishes it (partial, counter,
+  // last-arriver merge, up-projection); nothing runs after it.
+  float* res = reinterpret_cast<float*>(smem + C::kOffRes);
+  float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
+  auto finish_last = [&](int b_, int h_) {
     reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
-    float* outp = a.out + ((size_t)b * a.H + h) * a.Hd;
-    const __half* Bvh = a.Bv ? a.Bv + (size_t)h * W * a.Hd : nullptr;
-    if (c_first == c_last) {  // this CTA owns the whole (b, h)
+    const int tb = walk.tiles(b_);
+    const long long gf = (long long)a.H * pre[b_] + (long long)h_ * tb;
+    const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
+    float* outp = a.out + ((size_t)b_ * a.H + h_) * a.Hd;
+    const __half* Bvh = a.Bv ? a.Bv + (size_t)h_ * W * a.Hd : nullptr;
+    if (cf == cl) {
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
       return;
     }
-    // Publish the partial; the last CTA of (b, h) to arrive merges and finishes.
-    const int bh = b * a.H + h;
+    const int bh = b_ * a.H + h_;
     float* dst = a.partials + ((size_t)c + bh) * (W + 2);
-    for (int e = tid; e < W + 2; e += kConsumerThreads) dst[e] = res[e];
-    __threadfence();
+    if (tid < W + 2) {
+      for (int e = tid; e < W + 2; e += kConsumerThreads) dst[e] = res[e];
+      __threadfence();  // publish before the counter bump
+    }
     csync();
     if (tid == 0) {
       const int prev = atomicAdd(&a.counters[bh], 1);
-      reinterpret_cast<int*>(misc)[8] = (prev == c_last - c_first) ? 1 : 0;
+      reinterpret_cast<int*>(misc)[8] = (prev == cl - cf) ? 1 : 0;
     }
     csync();
     if (reinterpret_cast<int*>(misc)[8]) {
       __threadfence();
-      merge_rows<W, true>(a.partials + ((size_t)c_first + bh) * (W + 2), c_last - c_first + 1, red, C::kRedFloats,
-                          res, tid);
+      merge_rows<W, true>(a.partials + ((size_t)cf + bh) * (W + 2), cl - cf + 1, res, tid);
       if (tid == 0) atomicExch(&a.counters[bh], 0);
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
     }
-    csync();
   };
 
   int b, h, t;
   walk.locate(g_begin, b, h, t);
-  int cb = -1, ch = -1, c_first = 0, c_last = 0;
+  int cb = -1, ch = -1;
   long long i = 0;
   for (long long g = g_begin; g < g_end; ++g, ++i) {
     if (b != cb || h != ch) {
-      if (cb >= 0) flush(cb, ch, c_first, c_last);
-      const int tb = walk.tiles(b);
-      const long long gf = (long long)a.H * pre[b] + (long long)h * tb;
-      c_first = cta_of(gf, G, CW);
-      c_last = cta_of(gf + tb - 1, G, CW);
-      if (a.Bv != nullptr && c == c_last) {  // the likely finisher warms B_Vh in L2
-        const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)h * W * a.Hd);
-        for (int o = tid * 128; o < W * a.Hd * 2; o += kConsumerThreads * 128) prefetch_l2(bv + o);
+      if (cb >= 0) end_segment(k - 1);
+      const int sq = k & 1;
+      if (k == 0) {  // first segment: build the query state with every consumer thread
+        wait(&segfull[0], 0);
+        build_query<CODEC, VPT, W, QMODE>(qst, segbuf, ha->qsv[0], misc, ha->planes[0], a, tid, sub);
+        if (tid == 0) {
+          mbar_arrive(&segempty[0]);
+          mbar_arrive(&qready[0]);  // keeps qready[0]'s phases aligned with the segments that use it
+        }
+      } else {
+        wait(&qready[sq], (uint32_t)((k / 2) & 1));
+        qst.step = ha->qstep[sq];
+        if constexpr (CT::kScaled) {
+          const uint32_t* pl = ha->planes[sq];
+#pragma unroll
+          for (int q = 0; q < QW; ++q) {
+            qst.qh[q] = pl[(sub * 3 + 0) * QW + q];
+            qst.qm[q] = pl[(sub * 3 + 1) * QW + q];
+            qst.ql[q] = pl[(sub * 3 + 2) * QW + q];
+          }
+          if constexpr (CODEC == kCodecI4) {
+            qst.ch = (int)pl[TPT * 3 * QW + sub * 3 + 0];
+            qst.cm = (int)pl[TPT * 3 * QW + sub * 3 + 1];
+            qst.cl = (int)pl[TPT * 3 * QW + sub * 3 + 2];
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < NP; ++p)
+            qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
+        }
       }
-      const int sb = nseg % NBUF;
-      if (!mbar_wait_bounded(&segfull[sb], (uint32_t)((nseg / NBUF) & 1), timed_out ? 0ull : kWaitLimitNs)) {
-        if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-        timed_out = true;
-      }
-      build_query<CODEC, VPT, W, QMODE>(qst, segbuf + (size_t)sb * SEGB, qs, misc, a, tid, sub);
-      if (lane == 0) mbar_arrive(&segempty[sb]);  // the staged operands are consumed
-      ++nseg;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qfree[sq]);
 #pragma unroll
       for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
       m = kNegInf;
       l = 0.f;
+      ++k;
       cb = b;
       ch = h;
     }
     const int s = (int)(i % S);
     // A timed-out wait only poisons the result (err is set); control flow stays
     // uniform so every consumer warp reaches every named barrier.
-    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
-      if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-      timed_out = true;
-    }
+    wait(&full[s], (uint32_t)((i / S) & 1));
     process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, lens[b] - t * T), qst, m, l,
                                         acc, tid);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     walk.advance(b, h, t);
   }
-  if (cb >= 0) flush(cb, ch, c_first, c_last);
+  if (cb >= 0) finish_last(cb, ch);
 }
 
 // ------------------------------------------------------------------ cluster kernel (small problems)
@@ -817,6 +1103,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
   float* res = reinterpret_cast<float*>(smem + C::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
+  uint32_t* planes = reinterpret_cast<uint32_t*>(smem + C::kOffParts);
   uint8_t* segbuf = smem + C::cluster_seg_off();
   float* slots = reinterpret_cast<float*>(segbuf + seg_bytes(QMODE, W, a.Hd));  // [csize][W + 2]
   __half* bvs = reinterpret_cast<__half*>(slots + (size_t)kMaxClusterSize * (W + 2));
@@ -905,7 +1192,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     if (lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     timed_out = true;
   }
-  build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, a, tid, sub);
+  build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, planes, a, tid, sub);
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % S;
     if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
@@ -953,7 +1240,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
       }
     }
     csync();
-    merge_rows<W, false>(slots, csize, red, C::kRedFloats, res, tid);
+    merge_rows<W, false>(slots, csize, res, tid);
   }
   const __half* Bvh = nullptr;
   if (a.Bv != nullptr) {
@@ -1085,7 +1372,7 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
     return cudaErrorInvalidValue;
   int occ = 1;
   const size_t smem_small = small.smem(a.B, qmode, a.Hd);
-  const int sms = device_sms_and_occupancy(small.fn, smem_small, kDecodeThreads, &occ);
+  const int sms = device_sms_and_occupancy(small.fn, smem_small, kPersistThreads, &occ);
   const long long resident = (long long)sms * occ;
   const long long tiles_small = (long long)a.B * a.H * ((a.L_cap + small.tile - 1) / small.tile);
 
@@ -1117,11 +1404,11 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
   // Otherwise the persistent grid; the large-tile variant when there are several
   // tiles per resident CTA.
   const size_t smem_big = big.smem(a.B, qmode, a.Hd);
-  device_sms_and_occupancy(big.fn, smem_big, kDecodeThreads, &occ);
+  device_sms_and_occupancy(big.fn, smem_big, kPersistThreads, &occ);
   const long long tiles_big = (long long)a.B * a.H * ((a.L_cap + big.tile - 1) / big.tile);
   const KernelInfo& ki = (tiles_big >= 4 * (long long)sms * occ) ? big : small;
   const size_t smem = ki.smem(a.B, qmode, a.Hd);
-  device_sms_and_occupancy(ki.fn, smem, kDecodeThreads, &occ);
+  device_sms_and_occupancy(ki.fn, smem, kPersistThreads, &occ);
   const long long tiles_max = (long long)a.B * a.H * ((a.L_cap + ki.tile - 1) / ki.tile);
   long long ctas = (long long)sms * occ;
   if (ctas > tiles_max) ctas = tiles_max;
@@ -1131,7 +1418,7 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
   cudaError_t e = ensure_smem(ki.fn, smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kDecodeThreads), args, smem, stream);
+  return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kPersistThreads), args, smem, stream);
 }
 
 }  // namespace wsvd

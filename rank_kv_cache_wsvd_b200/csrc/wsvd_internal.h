@@ -16,7 +16,8 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 // Split-L decode: 8 consumer warps + 1 producer warp per CTA.
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kDecodeThreads = kConsumerThreads + 32;
+constexpr int kDecodeThreads = kConsumerThreads + 32;   // cluster kernel: + producer warp
+constexpr int kPersistThreads = kConsumerThreads + 64;  // persistent kernel: + producer and helper warps
 // Upper bound on the persistent grid; sizes the partial-result workspace.
 constexpr int kMaxDecodeCtas = 2048;
 
