@@ -40,6 +40,7 @@ UNIT = "tokens*heads/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+HOST_LEAD_CYCLES = 100_000  # device sleep (~50-75 us) before each timed step
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -180,7 +181,7 @@ class WsvdStep:
             self.x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
         self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
         self.out_host = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32).pin_memory()
-        self.launches_per_step = (1 if self.has_append else 0) + 2
+        self.launches_per_step = (1 if self.has_append else 0) + 1  # append, decode
 
     def reset(self):
         self.lens.copy_(self.lens0)
@@ -195,14 +196,24 @@ class WsvdStep:
         self.W.wsvd_decode_attention(self.q, self.lat_k, self.lat_v, self.scale_k, self.scale_v, self.B_k, self.B_v,
                                      self.lens, bits=self.w.bits, out=self.out, workspace_buf=self.ws, err=self.err)
 
+    def step(self):
+        """One step through the public API: the one-call append + decode when
+        the workload appends, else the decode."""
+        if not self.has_append:
+            self.decode()
+            return
+        self.W.wsvd_append_and_decode(self.x, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v, self.scale_k,
+                                      self.scale_v, self.q, self.B_k, self.B_v, bits=self.w.bits,
+                                      hadamard_block=self.w.hadamard_block, out=self.out, append_ws=self.ws_app,
+                                      decode_ws=self.ws, err=self.err)
+
     def e2e_step(self):
         """Public-API step with host buffers: H2D of the step inputs, append,
         decode, D2H of the result."""
         if self.has_append:
             self.x.copy_(self.x_host, non_blocking=True)
         self.q.copy_(self.q_host, non_blocking=True)
-        self.append()
-        self.decode()
+        self.step()
         self.out_host.copy_(self.out, non_blocking=True)
 
     def e2e_bytes(self):
@@ -243,26 +254,20 @@ def time_comparisons(w: WL.Workload, steps: int, warmup: int, flush):
 
 
 def _time_loop(fn, steps, warmup, flush):
-    """Device time per call of `fn`, replayed from a CUDA graph, L2 flushed between calls."""
+    """Device time per call of `fn`: events on the launching stream around the
+    call; before each call the L2 is flushed and a device sleep keeps the host
+    ahead, as in the timed steps."""
     import torch
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        for _ in range(3):
-            fn()
-    torch.cuda.current_stream().wait_stream(side)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    for _ in range(max(3, warmup)):
         fn()
-    for _ in range(warmup):
-        g.replay()
     torch.cuda.synchronize()
     evs = []
     for _ in range(steps):
         flush.zero_()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        g.replay()
+        fn()
         b.record()
         evs.append((a, b))
     torch.cuda.synchronize()
@@ -375,64 +380,84 @@ def main():
     st = WsvdStep(w, seed=rank)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    # The step's launches are captured once into CUDA graphs (append, decode) and
-    # replayed, so the device timeline holds no host launch gaps.
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        for _ in range(3):
-            st.reset()
-            st.append()
-            st.decode()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    g_step, g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):  # the whole step: append, then decode
+    for _ in range(3):  # first calls (library load, per-device setup) outside everything timed
+        st.reset()
         st.append()
         st.decode()
-    if st.has_append:
-        with torch.cuda.graph(g_app):
-            st.append()
-    with torch.cuda.graph(g_dec):
-        st.decode()
-    for _ in range(max(3, args.warmup)):
         st.reset()
-        g_step.replay()
+        st.step()
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        st.reset()
+        st.step()
     torch.cuda.synchronize()
     barrier()
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     time.sleep(0.25)
+    # Timed region: per step one call of the public step (append, then the
+    # decode launched behind it), bracketed by events on its stream.  Before
+    # the first event (outside the timed interval) the L2 is flushed, the
+    # lengths are reset and a device sleep keeps the host ahead of the device.
     evs = []
     for _ in range(args.steps):
         flush.zero_()
         st.reset()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record()
-        g_step.replay()
+        st.step()
         e[1].record()
         evs.append(e)
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
     t_step = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3
-    # Breakdown (not part of `value`): the two halves replayed separately, same flush.
-    n_b = min(args.steps, 200)
+    # Per-kernel durations (the roofline's denominators): inside the step the
+    # decode overlaps the append, so each kernel is timed here as its own
+    # launch, events around it, under the same flush and host lead.
+    n_b = min(args.steps, 300)
     evs = []
     for _ in range(n_b):
         flush.zero_()
         st.reset()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record()
-        if st.has_append:
-            g_app.replay()
+        st.append()
         e[1].record()
-        g_dec.replay()
+        st.decode()
         e[2].record()
         evs.append(e)
     torch.cuda.synchronize()
     t_app = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3 / n_b * args.steps if st.has_append else 0.0
     t_dec = sum(e[1].elapsed_time(e[2]) for e in evs) / 1e3 / n_b * args.steps
+    t_sep = sum(e[0].elapsed_time(e[2]) for e in evs) / 1e3 / n_b
+    # Context (not part of `value`): the step replayed from one CUDA graph.
+    g_step = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        st.reset()
+        st.step()
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(g_step):
+        st.step()
+    n_g = min(args.steps, 300)
+    evs = []
+    for _ in range(n_g):
+        flush.zero_()
+        st.reset()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        g_step.replay()
+        e[1].record()
+        evs.append(e)
+    torch.cuda.synchronize()
+    t_graph = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3 / n_g
+    del g_step
     units_local = attended_tokens(w, st.lens_after) * args.steps
     value, t_total = replica_throughput(units_local, t_step, world)
     if int(st.err.item()) != 0:
@@ -445,9 +470,10 @@ def main():
     per_app = t_app / args.steps
     per_dec = t_dec / args.steps
     if st.has_append and per_app >= per_dec:
-        dom, nbytes, dur, launches = "append", app_bytes, per_app, "wsvd append kernel (1 launch)"
+        dom, nbytes, dur, launches = "append", app_bytes, per_app, "wsvd latent append (1 launch)"
     else:
-        dom, nbytes, dur, launches = "decode", dec_bytes, per_dec, "wsvd decode (split-L kernel + combine)"
+        dom, nbytes, dur, launches = "decode", dec_bytes, per_dec, \
+            "wsvd decode (1 launch: split-L + last-arriver combine)"
     achieved = nbytes / dur / 1e9
     traffic = ncu_traffic(dom, args.workload)
 
@@ -483,10 +509,14 @@ def main():
                        "latent_bits": w.bits, "attended_tokens_per_seq": [int(x) for x in st.lens_after],
                        "step": ("append + decode" if st.has_append else "decode"),
                        "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
-                       "launch": "one CUDA graph replay per step (append + decode)"},
+                       "launch": ("one wsvd_append_and_decode call per step (decode launched behind the "
+                                  "append as a programmatic dependent); events around the call"
+                                  if st.has_append else "one wsvd_decode_attention call per step; events around it")},
             "step_us": ms_per_step * 1e3,
             "breakdown_us": {"append": per_app * 1e6, "decode": per_dec * 1e6,
-                             "note": "each half replayed alone; includes one graph launch each"},
+                             "two_calls": t_sep * 1e6,
+                             "note": "each kernel as its own launch, events around it (same flush and host lead)"},
+            "graph_step_us": t_graph * 1e6,
             "hbm_gbs": (dec_bytes + app_bytes) / (t_total / args.steps) / 1e9,
             "roofline": {"bound": "hbm", "kernel": launches, "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,

@@ -162,7 +162,14 @@ int wsvd_decode_attention_noalloc(int B, int H, int Hd, int r, int bits, int L_c
  *   x          [B][E]       bf16 or fp16 (x_dtype); E % hadamard_block == 0.
  *   A_k, A_v   [H][E][r]    fp16.
  *   hadamard_block          power of two in [2, 1024] (1 = no rotation).
- *   E                       multiple of 8 * hadamard_block, at most 65536.
+ *   E                       multiple of hadamard_block and of 8, at most
+ *                           65536.  E is split along a cluster of up to 8
+ *                           CTAs (the largest c in {8,4,2,1} with
+ *                           E % (c * hadamard_block) == 0 and (E/c) % 8 == 0);
+ *                           WSVD_ERR_UNSUPPORTED when the rotated slice,
+ *                           B * E/c fp32 values, and the 32 KB row ring do
+ *                           not fit in 200 KB of shared memory.
+ *   r                       multiple of 8, at most 128, r * bits/8 % 4 == 0.
  *   B                       1..16.
  *   seq_lens   [B]          int32, read and advanced in place.
  *   workspace               at least wsvd_append_workspace_size() bytes of
@@ -175,6 +182,30 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
                        const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
                        uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
                        size_t workspace_bytes, int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------- one decode step
+ * wsvd_latent_append followed by wsvd_decode_attention on the same stream: the
+ * decode step of the method (append the new token's latents, then attend over
+ * the cache including it; WSVD summaries, German §2.A and §2.C).  The pages
+ * define no separate interface for it; the results are those of the two calls
+ * made back to back, bit for bit.
+ * The decode is launched as a programmatic dependent of the append: its launch
+ * and its query projection q' = B_Kh . q overlap the append, and it reads
+ * seq_lens and the cache only after the append grid has completed.  So q, B_k
+ * and B_v must already be final when this call is made (they are read while
+ * the append runs; the append itself never writes them).
+ *   append_workspace   wsvd_append_workspace_size() bytes, contract as for
+ *                      wsvd_latent_append;
+ *   decode_workspace   wsvd_decode_workspace_size(B, H, r) bytes, contract as
+ *                      for wsvd_decode_attention.
+ * Every argument of both operations is validated before anything is launched;
+ * the status codes are those of the two calls.                              */
+int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                           const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
+                           uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, const void* q,
+                           int q_dtype, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                           void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
+                           size_t decode_workspace_bytes, int32_t* err, void* stream);
 
 /* ---------------------------------------------------------------- comparison: dense decode
  * The flash-decoding baseline the pages compare against (German §4

@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     shared_decode_workspace_size,
     shared_latent_svd_decode,
     workspace,
+    wsvd_append_and_decode,
     wsvd_append_workspace_size,
     wsvd_cache_bytes,
     wsvd_decode_attention,

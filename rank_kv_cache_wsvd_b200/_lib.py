@@ -38,6 +38,8 @@ SIGNATURES = {
                                                                                         _p, _p]),
     "wsvd_decode_attention_noalloc": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _p]),
     "wsvd_latent_append": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 7 + [_p, _c_size, _p, _p]),
+    "wsvd_append_and_decode": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
+                               + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
     "dense_decode_attention": (_c_int, [_c_int] * 4 + [_p, _p, _c_int, _p, _p, _c_float, _p, _p, _c_size, _p, _p]),
     "shared_latent_svd_decode": (_c_int, [_c_int] * 5 + [_p, _p, _c_int] + [_p] * 4 + [_c_float, _p, _p, _c_size,
                                                                                          _p, _p]),
@@ -202,6 +204,44 @@ def shared_latent_svd_decode(q, lat_k, lat_v, B_k, B_v, seq_lens, softmax_scale:
                                       _ptr(lat_v), _ptr(B_k), _ptr(B_v), float(softmax_scale), _ptr(out),
                                       _ptr(workspace_buf), workspace_buf.numel(), _ptr(err), _stream(stream))
     _check(st, "shared_latent_svd_decode")
+    return out
+
+
+# ----------------------------------------------------------------------------- one step
+def wsvd_append_and_decode(x, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q, B_k, B_v, bits: int,
+                           hadamard_block: int = 128, softmax_scale: float = 0.0, out=None, append_ws=None,
+                           decode_ws=None, err=None, stream=None):
+    """Append the new token's latents, then decode over the cache including it
+    (one library call; the decode overlaps the append's tail).  Returns out
+    [B][H][Hd] fp32; seq_lens and the cache are updated in place."""
+    lib = load()
+    B, E = x.shape
+    H, _, r = A_k.shape
+    Hd = q.shape[2]
+    L_cap = lat_k.shape[2]
+    _expect(A_k, torch.float16, (H, E, r), "A_k")
+    _expect(A_v, torch.float16, (H, E, r), "A_v")
+    _expect(q, q.dtype, (B, H, Hd), "q")
+    _expect(lat_k, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _expect(B_k, torch.float16, (H, r, Hd), "B_k")
+    _expect(B_v, torch.float16, (H, r, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, H, Hd), "out")
+    if append_ws is None:
+        append_ws = workspace(lib.wsvd_append_workspace_size(), x.device)
+    if decode_ws is None:
+        decode_ws = workspace(lib.wsvd_decode_workspace_size(B, H, r), q.device)
+    st = lib.wsvd_append_and_decode(B, H, Hd, E, r, bits, L_cap, hadamard_block, _ptr(x), _dtype_code(x),
+                                    _ptr(A_k), _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k),
+                                    _ptr(scale_v), _ptr(q), _dtype_code(q), _ptr(B_k), _ptr(B_v),
+                                    float(softmax_scale), _ptr(out), _ptr(append_ws), append_ws.numel(),
+                                    _ptr(decode_ws), decode_ws.numel(), _ptr(err), _stream(stream))
+    _check(st, "wsvd_append_and_decode")
     return out
 
 

@@ -25,6 +25,8 @@ inline size_t partial_bytes(int B, int H, int W) {
 }
 inline size_t decode_ws_bytes(int B, int H, int W) { return partial_bytes(B, H, W) + align16((size_t)B * H * 4); }
 
+constexpr size_t kAppendWorkspaceBytes = 256;  // the completion counter (padded)
+
 // Shared validation of the decode entry points.
 int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
                  const float* out, const void* workspace) {
@@ -43,6 +45,67 @@ int run_decode(int codec, int rowbytes, int qmode, DecodeArgs a, void* workspace
   a.partials = static_cast<float*>(workspace);
   a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + partial_bytes(a.B, a.H, a.W));
   if (launch_decode(codec, rowbytes, qmode, a, stream) != cudaSuccess) return WSVD_ERR_CUDA;
+  return WSVD_OK;
+}
+
+
+// Validation and argument set-up of wsvd_decode_attention (shared with the
+// fused step).  Returns WSVD_OK with *a filled, or an error status.
+int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens, const void* q,
+                        int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
+                        const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                        void* workspace, size_t workspace_bytes, int32_t* err, DecodeArgs* a) {
+  int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
+  if (st != WSVD_OK || B == 0) return st;
+  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
+  if (r < 1 || (r * bits) % 8) return WSVD_ERR_INVALID_ARG;
+  const int rowbytes = r * bits / 8;
+  if (!decode_supported(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj)) return WSVD_ERR_UNSUPPORTED;
+  if (!lat_k || !lat_v || !scale_k || !scale_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
+      !aligned16(B_k) || !aligned16(B_v))
+    return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < decode_ws_bytes(B, H, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+  a->B = B; a->H = H; a->Hd = Hd; a->W = r; a->L_cap = L_cap; a->heads_share = 0;
+  a->seq_lens = seq_lens; a->q = q; a->q_dtype = q_dtype;
+  a->lat_k = lat_k; a->lat_v = lat_v;
+  a->scale_k = static_cast<const __half*>(scale_k); a->scale_v = static_cast<const __half*>(scale_v);
+  a->Bk = static_cast<const __half*>(B_k); a->Bv = static_cast<const __half*>(B_v); a->qglobal = nullptr;
+  a->qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
+  a->out = out; a->err = err;
+  return WSVD_OK;
+}
+
+// Validation and argument set-up of wsvd_latent_append (shared with the fused step).
+int prepare_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x, int x_dtype,
+                   const void* A_k, const void* A_v, int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v,
+                   void* scale_k, void* scale_v, void* workspace, size_t workspace_bytes, int32_t* err,
+                   AppendArgs* a) {
+  if (B < 0 || H < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
+  if (B == 0) return WSVD_OK;
+  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
+  if (x_dtype != WSVD_DTYPE_FP16 && x_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
+  if (hadamard_block < 1 || hadamard_block > 1024 || (hadamard_block & (hadamard_block - 1)))
+    return WSVD_ERR_INVALID_ARG;
+  if (E % hadamard_block) return WSVD_ERR_INVALID_ARG;
+  if (B > 16 || r % 8 || r > 128 || (r * bits / 8) % 4 || E > 65536) return WSVD_ERR_UNSUPPORTED;
+  if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
+    return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
+      !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
+    return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < kAppendWorkspaceBytes) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+  const int cl = append_cluster_size(E, hadamard_block);
+  if (cl < 1) return WSVD_ERR_UNSUPPORTED;
+  if (append_smem_bytes(B, E, r, cl) > 200 * 1024) return WSVD_ERR_UNSUPPORTED;
+  a->B = B; a->H = H; a->E = E; a->r = r; a->bits = bits; a->L_cap = L_cap; a->blk = hadamard_block;
+  a->cluster = cl;
+  a->hnorm = (float)(1.0 / sqrt((double)hadamard_block));
+  a->x = x; a->x_dtype = x_dtype;
+  a->Ak = static_cast<const __half*>(A_k); a->Av = static_cast<const __half*>(A_v);
+  a->seq_lens = seq_lens; a->lat_k = lat_k; a->lat_v = lat_v;
+  a->scale_k = static_cast<__half*>(scale_k); a->scale_v = static_cast<__half*>(scale_v);
+  a->counter = static_cast<int32_t*>(workspace); a->err = err;
   return WSVD_OK;
 }
 
@@ -98,27 +161,11 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
                           const void* scale_k, const void* scale_v, const void* B_k, const void* B_v,
                           float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                           int32_t* err, void* stream) {
-  int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
-  if (st != WSVD_OK || B == 0) return st;
-  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
-  if (r < 1 || (r * bits) % 8) return WSVD_ERR_INVALID_ARG;
-  const int rowbytes = r * bits / 8;
-  if (!decode_supported(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj)) return WSVD_ERR_UNSUPPORTED;
-  if (!lat_k || !lat_v || !scale_k || !scale_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
-  if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
-      !aligned16(B_k) || !aligned16(B_v))
-    return WSVD_ERR_INVALID_ARG;
-  if (workspace_bytes < wsvd_decode_workspace_size(B, H, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
-
   DecodeArgs a{};
-  a.B = B; a.H = H; a.Hd = Hd; a.W = r; a.L_cap = L_cap; a.heads_share = 0;
-  a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
-  a.lat_k = lat_k; a.lat_v = lat_v;
-  a.scale_k = static_cast<const __half*>(scale_k); a.scale_v = static_cast<const __half*>(scale_v);
-  a.Bk = static_cast<const __half*>(B_k); a.Bv = static_cast<const __half*>(B_v); a.qglobal = nullptr;
-  a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
-  a.out = out; a.err = err;
-  return run_decode(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj, a, workspace, as_stream(stream));
+  const int st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v,
+                                     B_k, B_v, softmax_scale, out, workspace, workspace_bytes, err, &a);
+  if (st != WSVD_OK || B == 0) return st;
+  return run_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a, workspace, as_stream(stream));
 }
 
 int dense_decode_attention(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const void* q, int q_dtype,
@@ -168,39 +215,40 @@ int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32
   return run_decode(kCodecF16, rowbytes, kQGlobal, a, workspace, as_stream(stream));
 }
 
-size_t wsvd_append_workspace_size(void) { return 256; }
+size_t wsvd_append_workspace_size(void) { return kAppendWorkspaceBytes; }
 
 int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x,
                        int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens, uint8_t* lat_k,
                        uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace, size_t workspace_bytes,
                        int32_t* err, void* stream) {
-  if (B < 0 || H < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
-  if (B == 0) return WSVD_OK;
-  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
-  if (x_dtype != WSVD_DTYPE_FP16 && x_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
-  if (hadamard_block < 1 || hadamard_block > 1024 || (hadamard_block & (hadamard_block - 1)))
-    return WSVD_ERR_INVALID_ARG;
-  if (E % hadamard_block) return WSVD_ERR_INVALID_ARG;
-  if (B > 16 || r % 8 || r > 128 || (r * bits / 8) % 4 || E > 65536) return WSVD_ERR_UNSUPPORTED;
-  if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
-    return WSVD_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
-      !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
-    return WSVD_ERR_INVALID_ARG;
-  if (workspace_bytes < wsvd_append_workspace_size()) return WSVD_ERR_WORKSPACE_TOO_SMALL;
-  const int cl = append_cluster_size(E, hadamard_block);
-  if (cl < 1) return WSVD_ERR_UNSUPPORTED;
-  if (append_smem_bytes(B, E, r, cl) > 200 * 1024) return WSVD_ERR_UNSUPPORTED;
-
   AppendArgs a{};
-  a.B = B; a.H = H; a.E = E; a.r = r; a.bits = bits; a.L_cap = L_cap; a.blk = hadamard_block; a.cluster = cl;
-  a.hnorm = (float)(1.0 / sqrt((double)hadamard_block));
-  a.x = x; a.x_dtype = x_dtype;
-  a.Ak = static_cast<const __half*>(A_k); a.Av = static_cast<const __half*>(A_v);
-  a.seq_lens = seq_lens; a.lat_k = lat_k; a.lat_v = lat_v;
-  a.scale_k = static_cast<__half*>(scale_k); a.scale_v = static_cast<__half*>(scale_v);
-  a.counter = static_cast<int32_t*>(workspace); a.err = err;
+  const int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, seq_lens, lat_k,
+                                lat_v, scale_k, scale_v, workspace, workspace_bytes, err, &a);
+  if (st != WSVD_OK || B == 0) return st;
   if (launch_append(a, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
+  return WSVD_OK;
+}
+
+int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                           const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
+                           uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, const void* q, int q_dtype,
+                           const void* B_k, const void* B_v, float softmax_scale, float* out,
+                           void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
+                           size_t decode_workspace_bytes, int32_t* err, void* stream) {
+  AppendArgs ap{};
+  int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, seq_lens, lat_k, lat_v,
+                          scale_k, scale_v, append_workspace, append_workspace_bytes, err, &ap);
+  if (st != WSVD_OK) return st;
+  DecodeArgs dp{};
+  st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k, B_v,
+                           softmax_scale, out, decode_workspace, decode_workspace_bytes, err, &dp);
+  if (st != WSVD_OK || B == 0) return st;
+  if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
+  dp.partials = static_cast<float*>(decode_workspace);
+  dp.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(decode_workspace) + partial_bytes(B, H, r));
+  if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, as_stream(stream), true) !=
+      cudaSuccess)
+    return WSVD_ERR_CUDA;
   return WSVD_OK;
 }
 

@@ -5,17 +5,25 @@
 // W8A8 / W8A4 quantisation).
 //
 // The work is a GEMV [B x E] . [E x r] per (h, K|V) unit, bound by reading A
-// (2 * H * E * r fp16).  Each unit is split over a thread-block cluster of
-// up to 8 CTAs along E.  Every CTA pulls its slice of x and then its
-// contiguous A slice with 1-D bulk copies (TMA, no multicast), rotates its x
-// slice with a fast Walsh-Hadamard transform (one warp per block, warp-level
-// sync only) while A is in flight, and reduces its slice to a partial
-// c[B][r].  Non-leader CTAs store their partial straight into the leader's
-// shared memory (distributed shared memory) and arrive on the leader's
-// mbarrier; the leader sums the slots in rank order (deterministic),
-// quantises and writes the row.  The last leader to finish (a completion
-// counter in the caller's workspace, reset to zero by that leader) advances
-// seq_lens.
+// (2 * H * E * r fp16) once.  Each unit is split over a thread-block cluster
+// of up to 8 CTAs along E.  Order of work in a CTA, chosen so that the A
+// stream starts at once and nothing waits behind it:
+//   1. plain loads of the CTA's x slice (small, L2-resident after the first
+//      CTA), then the first 8 A rows of every thread are put in flight with
+//      16-byte cp.async copies into a per-thread ring in shared memory;
+//   2. the x slice is rotated (fast Walsh-Hadamard transform: in registers
+//      and warp shuffles for blocks up to 128, shared-memory butterflies
+//      beyond) while A arrives;
+//   3. each thread consumes its ring slot by slot (cp.async.wait_group keeps 7
+//      rows in flight) accumulating c[b][8 columns] in registers;
+//   4. partials are reduced across the CTA (shuffles, then shared memory) and
+//      stored into the cluster leader's shared memory (DSMEM) with an arrive on
+//      its mbarrier; the leader sums the ranks in order (deterministic),
+//      quantises and writes the row.  The last leader to finish (a completion
+//      counter in the caller's workspace, reset to zero by that leader)
+//      advances seq_lens.
+// A thread only ever reads ring slots it filled itself, so the ring needs no
+// block-wide synchronisation.
 #include <cooperative_groups.h>
 
 #include <map>
@@ -29,21 +37,21 @@ namespace wsvd {
 
 constexpr int kAppendThreads = 256;
 constexpr int kAppendWarps = kAppendThreads / 32;
+constexpr int kRing = 8;  // A rows in flight per thread
 
 struct AppendSmem {
-  size_t a_off, xr_off, xs_off, slot_off, red_off, codes_off, bar_off, total;
+  size_t ring_off, xs_off, slot_off, red_off, codes_off, bar_off, total;
 };
 
 static __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// A slice | raw x slice | rotated x (fp32) | partial slots [cluster][B][r] | reduction scratch | codes | barriers
+// ring [kRing][threads] x 16 B | rotated x (fp32) [B][Ec] | partial slots [cluster][B][r]
+// | reduction scratch [warps][4][r] | codes [B][r] | barriers
 static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r, int cluster) {
   AppendSmem s;
   size_t o = 0;
-  s.a_off = o;
-  o = align_up(o + (size_t)Ec * r * 2, 128);
-  s.xr_off = o;
-  o = align_up(o + (size_t)B * Ec * 2, 128);
+  s.ring_off = o;
+  o += (size_t)kRing * kAppendThreads * 16;
   s.xs_off = o;
   o = align_up(o + (size_t)B * Ec * 4, 16);
   s.slot_off = o;
@@ -53,133 +61,207 @@ static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r,
   s.codes_off = o;
   o = align_up(o + (size_t)B * r, 16);
   s.bar_off = o;
-  o += 3 * 8;
+  o += 8;
   s.total = align_up(o, 16);
   return s;
 }
 
-// The cluster's partials: slot[rank][b][j] in the leader's shared memory.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_ring() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");
+}
+
+// Per-thread share of the CTA's A slice: rows k * nrg + rg (k = 0, 1, ...) of
+// the slice, 8 columns starting at 8 * cgi (one 16-byte piece per row).
+struct RowWalk {
+  const __half* A;  // first row of the slice
+  int r, Ec, nrg, rg, cgi, nrows;
+  __device__ __forceinline__ bool valid(int k) const { return k < nrows; }
+  __device__ __forceinline__ int row(int k) const { return k * nrg + rg; }
+  __device__ __forceinline__ void issue(uint4* ring, int k, int tid) const {
+    if (valid(k)) cp_async16(ring + (size_t)(k % kRing) * kAppendThreads + tid, A + (size_t)row(k) * r + cgi * 8);
+    cp_async_commit();  // one group per ring step, empty past the end
+  }
+};
+
+// Accumulate c[bb0 + bi][8 * cgi .. + 8] over this thread's rows, streaming
+// them through the ring (rows 0 .. kRing-1 already issued by the caller).
 template <int BB>
-__device__ __forceinline__ void gemv_slice(const __half* As, const float* xs, int B, int Ec, int r, float* red,
-                                           float* dst /* [B][r], any shared window */, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  const int ncg = r / 8, nrg = kAppendThreads / ncg;
-  const int cgi = tid % ncg, rg = tid / ncg;
-  for (int bb0 = 0; bb0 < B; bb0 += BB) {
-    float acc[BB][8];
+__device__ __forceinline__ void stream_rows(const RowWalk& w, uint4* ring, const float* xs, int B, int bb0,
+                                            float (&acc)[BB][8], int tid) {
 #pragma unroll
-    for (int bi = 0; bi < BB; ++bi)
+  for (int bi = 0; bi < BB; ++bi)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[bi][k] = 0.f;
-    for (int e = rg; e < Ec; e += nrg) {
-      const uint4 av = *reinterpret_cast<const uint4*>(As + (size_t)e * r + cgi * 8);
-      const float2 a01 = h2_pair(av.x), a23 = h2_pair(av.y), a45 = h2_pair(av.z), a67 = h2_pair(av.w);
-      const float af[8] = {a01.x, a01.y, a23.x, a23.y, a45.x, a45.y, a67.x, a67.y};
+    for (int k = 0; k < 8; ++k) acc[bi][k] = 0.f;
+  for (int k = 0; k < w.nrows; ++k) {
+    cp_async_wait_ring();  // this thread's group k is complete
+    const uint4 av = ring[(size_t)(k % kRing) * kAppendThreads + tid];
+    const float2 a01 = h2_pair(av.x), a23 = h2_pair(av.y), a45 = h2_pair(av.z), a67 = h2_pair(av.w);
+    const float af[8] = {a01.x, a01.y, a23.x, a23.y, a45.x, a45.y, a67.x, a67.y};
+    // The slot is consumed (values in registers) before it is refilled.
+    w.issue(ring, k + kRing, tid);
+    const int e = w.row(k);
 #pragma unroll
-      for (int bi = 0; bi < BB; ++bi) {
-        const float xv = (bb0 + bi < B) ? xs[(size_t)(bb0 + bi) * Ec + e] : 0.f;
+    for (int bi = 0; bi < BB; ++bi) {
+      const float xv = (bb0 + bi < B) ? xs[(size_t)(bb0 + bi) * w.Ec + e] : 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[bi][k] = fmaf(xv, af[k], acc[bi][k]);
-      }
+      for (int j = 0; j < 8; ++j) acc[bi][j] = fmaf(xv, af[j], acc[bi][j]);
     }
-    for (int o = ncg; o < 32; o <<= 1)
-#pragma unroll
-      for (int bi = 0; bi < BB; ++bi)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[bi][k] += __shfl_xor_sync(0xffffffffu, acc[bi][k], o);
-    if (lane < ncg) {
-#pragma unroll
-      for (int bi = 0; bi < BB; ++bi)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) red[(warp * BB + bi) * r + lane * 8 + k] = acc[bi][k];
-    }
-    __syncthreads();
-    for (int idx = tid; idx < BB * r; idx += kAppendThreads) {
-      const int bi = idx / r, j = idx % r;
-      if (bb0 + bi < B) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kAppendWarps; ++w) s += red[(w * BB + bi) * r + j];
-        dst[(size_t)(bb0 + bi) * r + j] = s;
-      }
-    }
-    __syncthreads();
   }
 }
 
-__global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs a) {
-  cg::cluster_group cluster = cg::this_cluster();
+// Reduce acc over the CTA (threads sharing a column group, then warps) into
+// dst[bi][j] (any shared window, e.g. the leader's slot).  Fixed order.
+template <int BB>
+__device__ __forceinline__ void reduce_cta(float (&acc)[BB][8], int ncg, int r, int nb, float* red, float* dst,
+                                           int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int o = ncg; o < 32; o <<= 1)
+#pragma unroll
+    for (int bi = 0; bi < BB; ++bi)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[bi][k] += __shfl_xor_sync(0xffffffffu, acc[bi][k], o);
+  if (lane < ncg) {
+#pragma unroll
+    for (int bi = 0; bi < BB; ++bi)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) red[(warp * BB + bi) * r + lane * 8 + k] = acc[bi][k];
+  }
+  __syncthreads();
+  for (int idx = tid; idx < nb * r; idx += kAppendThreads) {
+    const int bi = idx / r, j = idx % r;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAppendWarps; ++w) s += red[(w * BB + bi) * r + j];
+    dst[(size_t)bi * r + j] = s;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ float x_elem(uint32_t bits16, int dtype) {
+  return dtype == WSVD_DTYPE_BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((uint16_t)bits16));
+}
+
+// Butterfly stage pairs (i, i + hh) of one Hadamard block held in shared memory.
+__device__ __forceinline__ void fwht_smem_warp(float* v, int blk, int lane) {
+  for (int hh = 1; hh < blk; hh <<= 1) {
+    for (int q = lane; q < blk / 2; q += 32) {
+      const int i = (q / hh) * 2 * hh + (q % hh);
+      const float u = v[i], w = v[i + hh];
+      v[i] = u + w;
+      v[i + hh] = u - w;
+    }
+    __syncwarp();
+  }
+}
+
+template <int BB>
+__device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_group& cluster, uint8_t* smem,
+                                            const AppendSmem& L) {
   const int rank = (int)cluster.block_rank();
   const int unit = blockIdx.y, h = unit >> 1, kv = unit & 1;
   const int B = a.B, r = a.r, E = a.E;
   const int Ec = E / a.cluster, e0 = rank * Ec;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const AppendSmem L = append_layout(B, Ec, r, a.cluster);
-
-  extern __shared__ __align__(128) uint8_t smem[];
-  const __half* As = reinterpret_cast<const __half*>(smem + L.a_off);
-  const uint16_t* xr = reinterpret_cast<const uint16_t*>(smem + L.xr_off);
+  uint4* ring = reinterpret_cast<uint4*>(smem + L.ring_off);
   float* xs = reinterpret_cast<float*>(smem + L.xs_off);
   float* slots = reinterpret_cast<float*>(smem + L.slot_off);
   float* red = reinterpret_cast<float*>(smem + L.red_off);
   int8_t* codes = reinterpret_cast<int8_t*>(smem + L.codes_off);
-  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* bar_a = bar_x + 1;
-  uint64_t* bar_red = bar_x + 2;  // leader only: one arrival per non-leader CTA
+  uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);  // leader: one arrival per other rank
 
-  // 1. x slice first, then the A slice, on their way.
   if (tid == 0) {
-    mbar_init(bar_x, 1);
-    mbar_init(bar_a, 1);
     mbar_init(bar_red, a.cluster > 1 ? a.cluster - 1 : 1);
     fence_mbar_init();
-    const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
-    const uint32_t xrow = (uint32_t)Ec * 2;
-    mbar_arrive_expect_tx(bar_x, xrow * B);
-    for (int b = 0; b < B; ++b)
-      bulk_g2s(smem + L.xr_off + (size_t)b * xrow, static_cast<const uint16_t*>(a.x) + (size_t)b * E + e0, xrow,
-               bar_x, keep);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>((kv ? a.Av : a.Ak) + ((size_t)h * E + e0) * (size_t)r);
-    const uint32_t bytes = (uint32_t)Ec * r * 2;
-    mbar_arrive_expect_tx(bar_a, bytes);
-    constexpr uint32_t kPiece = 32768;
-    for (uint32_t off = 0; off < bytes; off += kPiece)
-      bulk_g2s(smem + L.a_off + off, src + off, min(kPiece, bytes - off), bar_a, once);
   }
-  // Every CTA's barriers are initialised before any remote access; the wait is
-  // deferred until the first access so the barrier latency overlaps the copies.
+  // A decode launched behind this kernel may start its own prologue (q and
+  // the B matrices only) while the append runs; it reads the cache after
+  // this grid completes.
+  griddep_launch_dependents();
+  // Every CTA's barrier is initialised before any remote access; the wait is
+  // deferred to the first remote access.
   cluster.barrier_arrive();
 
-  // 2. Rotate x: one warp per Hadamard block, butterflies with warp-level sync.
-  if (!mbar_wait_bounded(bar_x, 0) && tid == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-  const int nblk = B * (Ec / a.blk);
-  for (int blk = warp; blk < nblk; blk += kAppendWarps) {
-    const int b = blk / (Ec / a.blk), off = (blk % (Ec / a.blk)) * a.blk;
-    const uint16_t* src = xr + (size_t)b * Ec + off;
-    float* dst = xs + (size_t)b * Ec + off;
-    for (int i = lane; i < a.blk; i += 32)
-      dst[i] = (a.x_dtype == WSVD_DTYPE_BF16) ? __uint_as_float((uint32_t)src[i] << 16)
-                                              : __half2float(__ushort_as_half(src[i]));
-    __syncwarp();
-    for (int hh = 1; hh < a.blk; hh <<= 1) {
-      for (int q = lane; q < a.blk / 2; q += 32) {
-        const int i = (q / hh) * 2 * hh + (q % hh);
-        const float u = dst[i], v = dst[i + hh];
-        dst[i] = u + v;
-        dst[i + hh] = u - v;
+  // 1. x slice loads first (registers), then the A stream.
+  constexpr int kMaxChunks = 4;  // 128-element x chunks per warp held in registers (fast path)
+  const int nch = B * Ec / 128;
+  const bool fast = (Ec % 128 == 0) && a.blk <= 128 && nch <= kMaxChunks * kAppendWarps;
+  uint2 xraw[kMaxChunks];
+  const uint16_t* xg = static_cast<const uint16_t*>(a.x);
+  if (fast) {
+#pragma unroll
+    for (int t = 0; t < kMaxChunks; ++t) {
+      const int ch = warp + t * kAppendWarps;
+      if (ch < nch) {
+        const int b = ch / (Ec / 128), off = (ch % (Ec / 128)) * 128;
+        xraw[t] = __ldg(reinterpret_cast<const uint2*>(xg + (size_t)b * E + e0 + off) + lane);
       }
-      __syncwarp();
     }
+  }
+  const int ncg = r / 8, nrg = kAppendThreads / ncg;
+  RowWalk w;
+  w.A = (kv ? a.Av : a.Ak) + ((size_t)h * E + e0) * (size_t)r;
+  w.r = r; w.Ec = Ec; w.nrg = nrg; w.rg = tid / ncg; w.cgi = tid % ncg;
+  w.nrows = w.rg < Ec ? (Ec - 1 - w.rg) / nrg + 1 : 0;
+#pragma unroll 1
+  for (int k = 0; k < kRing; ++k) w.issue(ring, k, tid);
+
+  // 2. Rotate x into xs[b][e] (unnormalised; 1/sqrt(blk) is applied to c).
+  if (fast) {
+    // lane holds elements 4*lane .. 4*lane+3 of a 128-element chunk
+#pragma unroll
+    for (int t = 0; t < kMaxChunks; ++t) {
+      const int ch = warp + t * kAppendWarps;
+      if (ch >= nch) continue;  // warp-uniform
+      float v[4] = {x_elem(xraw[t].x & 0xffffu, a.x_dtype), x_elem(xraw[t].x >> 16, a.x_dtype),
+                    x_elem(xraw[t].y & 0xffffu, a.x_dtype), x_elem(xraw[t].y >> 16, a.x_dtype)};
+      if (a.blk >= 2) {
+        const float u0 = v[0] + v[1], u1 = v[0] - v[1], u2 = v[2] + v[3], u3 = v[2] - v[3];
+        v[0] = u0; v[1] = u1; v[2] = u2; v[3] = u3;
+      }
+      if (a.blk >= 4) {
+        const float u0 = v[0] + v[2], u2 = v[0] - v[2], u1 = v[1] + v[3], u3 = v[1] - v[3];
+        v[0] = u0; v[1] = u1; v[2] = u2; v[3] = u3;
+      }
+      for (int m = 1; 4 * m < a.blk; m <<= 1) {  // pair distance 4m = lane distance m
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+          v[k] = upper ? o - v[k] : v[k] + o;
+        }
+      }
+      const int b = ch / (Ec / 128), off = (ch % (Ec / 128)) * 128;
+      *reinterpret_cast<float4*>(xs + (size_t)b * Ec + off + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+  } else {
+    for (int i = tid; i < B * Ec; i += kAppendThreads) {
+      const int b = i / Ec, e = i % Ec;
+      xs[i] = x_elem(xg[(size_t)b * E + e0 + e], a.x_dtype);
+    }
+    __syncthreads();
+    const int nblk = B * (Ec / a.blk);
+    for (int blk = warp; blk < nblk; blk += kAppendWarps)
+      fwht_smem_warp(xs + (size_t)blk * a.blk, a.blk, lane);
   }
   __syncthreads();
 
-  // 3. Wait for A (bounded), then the slice GEMV into this rank's slot of the leader.
-  if (!mbar_wait_bounded(bar_a, 0) && tid == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+  // 3. + 4. Stream the A rows, reduce into this rank's slot of the leader.
   cluster.barrier_wait();
   float* my_slot = cluster.map_shared_rank(slots, 0) + (size_t)rank * B * r;
-  if (B == 1) gemv_slice<1>(As, xs, B, Ec, r, red, my_slot, tid);
-  else if (B == 2) gemv_slice<2>(As, xs, B, Ec, r, red, my_slot, tid);
-  else gemv_slice<4>(As, xs, B, Ec, r, red, my_slot, tid);
+  for (int bb0 = 0; bb0 < B; bb0 += BB) {
+    if (bb0 > 0) {
+#pragma unroll 1
+      for (int k = 0; k < kRing; ++k) w.issue(ring, k, tid);  // re-stream (L2) for the next batch rows
+    }
+    float acc[BB][8];
+    stream_rows<BB>(w, ring, xs, B, bb0, acc, tid);
+    reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, my_slot + (size_t)bb0 * r, tid);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
 
   if (rank != 0) {
     // Publish the slot (release at cluster scope) and arrive on the leader's barrier.
@@ -193,9 +275,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
     return;
   }
 
-  // 4. Leader: wait for the other ranks, sum the slots in rank order, quantise.
+  // 5. Leader: wait for the other ranks, sum the slots in rank order, quantise.
   if (a.cluster > 1) {
-    bool ok = true;
     if (tid == 0) {
       const uint32_t addr = smem_u32(bar_red);
       const uint64_t t0 = globaltimer_ns();
@@ -210,11 +291,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
             : "memory");
         if (done) break;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          ok = false;
+          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
           break;
         }
       }
-      if (!ok) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     }
     __syncthreads();
   }
@@ -264,7 +344,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
   }
   __syncthreads();
 
-  // 5. The last leader to finish advances the lengths.
+  // 6. The last leader to finish advances the lengths.
   if (tid == 0) {
     __threadfence();
     const int prev = atomicAdd(a.counter, 1);
@@ -277,6 +357,15 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendArgs
       atomicExch(a.counter, 0);
     }
   }
+}
+
+__global__ void __launch_bounds__(kAppendThreads, 4) append_kernel(const AppendArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const AppendSmem L = append_layout(a.B, a.E / a.cluster, a.r, a.cluster);
+  if (a.B == 1) append_body<1>(a, cluster, smem, L);
+  else if (a.B == 2) append_body<2>(a, cluster, smem, L);
+  else append_body<4>(a, cluster, smem, L);
 }
 
 int append_cluster_size(int E, int blk) {

@@ -96,6 +96,16 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return p;
 }
 
+// Programmatic dependent launch.  griddep_wait: returns once the grid this
+// one was launched behind (programmatic stream serialisation) has completed
+// and its memory is visible; a no-op for a normal launch.
+// griddep_launch_dependents: lets the dependent grid be scheduled before this
+// one completes (it still waits in griddep_wait for the data).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

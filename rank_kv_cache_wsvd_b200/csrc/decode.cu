@@ -748,6 +748,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
+  // Launched behind the append (programmatic dependent launch): the split plan
+  // reads seq_lens, so nothing here may run before that grid has completed.
+  griddep_wait();
 
   // Valid lengths, tiles per sequence (per head) and their exclusive prefix.
   if (warp == 0) {
@@ -1134,15 +1137,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     }
   }
   cluster.barrier_arrive();  // barriers initialised; waited on before any remote access
+  __syncthreads();           // barrier initialisation visible to every thread of this CTA
 
-  const int raw = a.seq_lens[b];
-  if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
-  const int len = clamp_len(raw, a.L_cap);
-  const int end = min(hi, len);
-  const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
-  __syncthreads();  // barrier initialisation visible to every thread of this CTA
-
+  // Everything above reads only q and the B matrices.  Under a programmatic
+  // dependent launch (behind the append that writes this step's row and
+  // seq_lens) the cache and the lengths are read only after griddep_wait.
   if (warp == kConsumerWarps) {
+    griddep_wait();
+    const int end = min(hi, clamp_len(a.seq_lens[b], a.L_cap));
+    const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
       bool ok = true;
@@ -1193,6 +1196,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     timed_out = true;
   }
   build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, planes, a, tid, sub);
+  griddep_wait();
+  const int raw = a.seq_lens[b];
+  if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0 && tid == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+  const int end = min(hi, clamp_len(raw, a.L_cap));
+  const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % S;
     if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
@@ -1366,7 +1374,7 @@ bool decode_supported(int codec, int rowbytes, int qmode) {
   return pick(codec, rowbytes, qmode, false, &ki) && pick(codec, rowbytes, qmode, true, &ki);
 }
 
-cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream) {
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream, bool pdl) {
   KernelInfo small, big;
   if (!pick(codec, rowbytes, qmode, false, &small) || !pick(codec, rowbytes, qmode, true, &big))
     return cudaErrorInvalidValue;
@@ -1390,13 +1398,15 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
     cfg.blockDim = dim3(kDecodeThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     void* args[] = {&a};
     return cudaLaunchKernelExC(&cfg, small.cfn, args);
   }
@@ -1418,7 +1428,18 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
   cudaError_t e = ensure_smem(ki.fn, smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kPersistThreads), args, smem, stream);
+  if (!pdl) return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kPersistThreads), args, smem, stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.ctas);
+  cfg.blockDim = dim3(kPersistThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, ki.fn, args);
 }
 
 }  // namespace wsvd

@@ -49,7 +49,9 @@ struct DecodeArgs {
 
 // Host launchers (decode.cu, shared.cu, append.cu).  Return a cudaError_t.
 bool decode_supported(int codec, int rowbytes, int qmode);
-cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream);
+// pdl: launch as a programmatic dependent of the preceding kernel in `stream`
+// (the kernel reads q and the B matrices before that kernel completes).
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_shared_qproj(int B, int H, int Hd, int R, const void* q, int q_dtype, const __half* Bk,
                                 float* qglobal, cudaStream_t stream);
 

@@ -1,0 +1,93 @@
+"""The one-call decode step, wsvd_append_and_decode: the latent append, then the
+decode launched behind it as a programmatic dependent (its launch and query
+projection overlap the append).  Its results must be those of the two calls
+made one after the other, bit for bit (cache rows, scales, lengths, output),
+and the oracle's two steps within the attention tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import rank_kv_cache_wsvd_b200 as W
+import workloads as WL
+from gpu_util import assert_attention_close, dev, q_tensor
+from oracle import wsvd_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # cluster decode path (few tiles), B = 1
+    "llava7b": (WL.LLAVA7B.with_(L_cap=1608), [1599]),
+    # persistent decode path, a length at the last free row and a short one
+    "long-r32": (WL.LONG[32].with_(L_cap=8192), [8000, 8191, 100, 4095]),
+    # int4 cache, fp16 query, ragged lengths
+    "ragged-int4": (WL.RAGGED.with_(B=6, E=2048), [1023, 4095, 2000, 1, 3333, 64]),
+    "pr1": (WL.PR1.with_(L_cap=264), [255]),
+}
+
+
+def _inputs(w, lens0, seed):
+    d = WL.decode_inputs(w, seed=seed, lens=np.asarray(lens0) + 1)
+    for b, n in enumerate(lens0):  # the row the append writes starts out empty
+        d.lat_k[b, :, n:] = 0
+        d.lat_v[b, :, n:] = 0
+        d.scale_k[b, :, n:] = 0
+        d.scale_v[b, :, n:] = 0
+    d.seq_lens[:] = lens0
+    ai = WL.append_inputs(w, seed=seed, steps=1)
+    return d, ai
+
+
+def _device_state(d):
+    return dict(lat_k=dev(d.lat_k), lat_v=dev(d.lat_v), sk=dev(d.scale_k), sv=dev(d.scale_v), lens=dev(d.seq_lens))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_step_equals_append_then_decode(name):
+    w, lens0 = CASES[name]
+    d, ai = _inputs(w, lens0, seed=21)
+    x = q_tensor(ai.x_bits[0], "bf16")
+    A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
+    q = q_tensor(d.q_bits, w.q_dtype)
+    two, one = _device_state(d), _device_state(d)
+    err2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    err1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    W.wsvd_latent_append(x, A_k, A_v, two["lens"], two["lat_k"], two["lat_v"], two["sk"], two["sv"], bits=w.bits,
+                         hadamard_block=w.hadamard_block, err=err2)
+    out2 = W.wsvd_decode_attention(q, two["lat_k"], two["lat_v"], two["sk"], two["sv"], B_k, B_v, two["lens"],
+                                   bits=w.bits, err=err2)
+    for rep in range(2):  # the second call proves the workspaces were left zero
+        st = _device_state(d) if rep else one
+        out1 = W.wsvd_append_and_decode(x, A_k, A_v, st["lens"], st["lat_k"], st["lat_v"], st["sk"], st["sv"], q,
+                                        B_k, B_v, bits=w.bits, hadamard_block=w.hadamard_block, err=err1)
+        torch.cuda.synchronize()
+        assert int(err1.item()) == 0 and int(err2.item()) == 0
+        for k in ("lat_k", "lat_v", "sk", "sv", "lens"):
+            assert torch.equal(st[k], two[k]), (name, k)
+        assert torch.equal(out1, out2), name
+
+    # and the oracle's append + decode
+    lk, sk, lv, sv, nl, _, _, _ = O.latent_append(ai.x[0], ai.A_k, ai.A_v, d.seq_lens, d.lat_k, d.scale_k, d.lat_v,
+                                                  d.scale_v, w.r, w.bits, w.hadamard_block)
+    ref = O.wsvd_decode(d.q, lk, sk, lv, sv, d.Bk, d.Bv, nl, w.r, w.bits)
+    assert np.array_equal(one["lens"].cpu().numpy(), np.asarray(lens0) + 1)
+    assert_attention_close(out1.cpu().numpy(), ref, f"step {name}")
+
+
+def test_step_validates_before_launching():
+    w, lens0 = CASES["llava7b"]
+    d, ai = _inputs(w, lens0, seed=3)
+    st = _device_state(d)
+    x = q_tensor(ai.x_bits[0], "bf16")
+    q = q_tensor(d.q_bits, w.q_dtype)
+    bad_B_v = dev(d.Bv)[:, :, :64].contiguous()  # wrong head dim: rejected by the binding
+    with pytest.raises(W.WsvdError):
+        W.wsvd_append_and_decode(x, dev(ai.A_k), dev(ai.A_v), st["lens"], st["lat_k"], st["lat_v"], st["sk"],
+                                 st["sv"], q, dev(d.Bk), bad_B_v, bits=w.bits)
+    # a decode-side failure in the library (too small a decode workspace) leaves the cache untouched
+    small = W.workspace(16)
+    with pytest.raises(W.WsvdError):
+        W.wsvd_append_and_decode(x, dev(ai.A_k), dev(ai.A_v), st["lens"], st["lat_k"], st["lat_v"], st["sk"],
+                                 st["sv"], q, dev(d.Bk), dev(d.Bv), bits=w.bits, decode_ws=small)
+    torch.cuda.synchronize()
+    assert np.array_equal(st["lens"].cpu().numpy(), np.asarray(lens0))
+    assert torch.equal(st["lat_k"], dev(d.lat_k))
