@@ -17,11 +17,12 @@
 //   3. each thread consumes its ring slot by slot (cp.async.wait_group keeps 7
 //      rows in flight) accumulating c[b][8 columns] in registers;
 //   4. partials are reduced across the CTA (shuffles, then shared memory) and
-//      stored into the cluster leader's shared memory (DSMEM) with an arrive on
-//      its mbarrier; the leader sums the ranks in order (deterministic),
-//      quantises and writes the row.  The last leader to finish (a completion
-//      counter in the caller's workspace, reset to zero by that leader)
-//      advances seq_lens.
+//      stored into the cluster leader's shared memory with st.async stores
+//      whose bytes complete on the leader's mbarrier; the leader sums the
+//      ranks in order (deterministic), quantises with one warp per batch row
+//      and writes the row.  The last leader to finish (a completion counter
+//      in the caller's workspace, reset to zero by that leader) advances
+//      seq_lens.
 // A thread only ever reads ring slots it filled itself, so the ring needs no
 // block-wide synchronisation.
 #include <cooperative_groups.h>
@@ -40,13 +41,13 @@ constexpr int kAppendWarps = kAppendThreads / 32;
 constexpr int kRing = 8;  // A rows in flight per thread
 
 struct AppendSmem {
-  size_t ring_off, xs_off, slot_off, red_off, codes_off, bar_off, total;
+  size_t ring_off, xs_off, slot_off, red_off, bar_off, total;
 };
 
 static __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ring [kRing][threads] x 16 B | rotated x (fp32) [B][Ec] | partial slots [cluster][B][r]
-// | reduction scratch [warps][4][r] | codes [B][r] | barriers
+// | reduction scratch [warps][4][r] | barrier
 static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r, int cluster) {
   AppendSmem s;
   size_t o = 0;
@@ -58,8 +59,6 @@ static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r,
   o = align_up(o + (size_t)cluster * B * r * 4, 16);
   s.red_off = o;
   o = align_up(o + (size_t)kAppendWarps * 4 * r * 4, 16);
-  s.codes_off = o;
-  o = align_up(o + (size_t)B * r, 16);
   s.bar_off = o;
   o += 8;
   s.total = align_up(o, 16);
@@ -114,10 +113,12 @@ __device__ __forceinline__ void stream_rows(const RowWalk& w, uint4* ring, const
 }
 
 // Reduce acc over the CTA (threads sharing a column group, then warps) into
-// dst[bi][j] (any shared window, e.g. the leader's slot).  Fixed order.
+// the slot rows bi < nb: a local store on the leader (remote_bar == 0), else an
+// st.async into the leader's slot at cluster address remote_dst that completes
+// 4 bytes per value on the leader's barrier.  Fixed summation order.
 template <int BB>
 __device__ __forceinline__ void reduce_cta(float (&acc)[BB][8], int ncg, int r, int nb, float* red, float* dst,
-                                           int tid) {
+                                           uint32_t remote_dst, uint32_t remote_bar, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
   for (int o = ncg; o < 32; o <<= 1)
 #pragma unroll
@@ -136,7 +137,8 @@ __device__ __forceinline__ void reduce_cta(float (&acc)[BB][8], int ncg, int r, 
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kAppendWarps; ++w) s += red[(w * BB + bi) * r + j];
-    dst[(size_t)bi * r + j] = s;
+    if (remote_bar) st_async_f32(remote_dst + 4u * (uint32_t)(bi * r + j), s, remote_bar);
+    else dst[(size_t)bi * r + j] = s;
   }
   __syncthreads();
 }
@@ -170,17 +172,15 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   float* xs = reinterpret_cast<float*>(smem + L.xs_off);
   float* slots = reinterpret_cast<float*>(smem + L.slot_off);
   float* red = reinterpret_cast<float*>(smem + L.red_off);
-  int8_t* codes = reinterpret_cast<int8_t*>(smem + L.codes_off);
-  uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);  // leader: one arrival per other rank
+  // Leader: completes when every other rank's slot values have landed
+  // (transaction bytes of their st.async stores).
+  uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);
 
   if (tid == 0) {
-    mbar_init(bar_red, a.cluster > 1 ? a.cluster - 1 : 1);
+    mbar_init(bar_red, 1);
     fence_mbar_init();
+    if (rank == 0 && a.cluster > 1) mbar_arrive_expect_tx(bar_red, (uint32_t)((a.cluster - 1) * B * r * 4));
   }
-  // A decode launched behind this kernel may start its own prologue (q and
-  // the B matrices only) while the append runs; it reads the cache after
-  // this grid completes.
-  griddep_launch_dependents();
   // Every CTA's barrier is initialised before any remote access; the wait is
   // deferred to the first remote access.
   cluster.barrier_arrive();
@@ -251,7 +251,8 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
 
   // 3. + 4. Stream the A rows, reduce into this rank's slot of the leader.
   cluster.barrier_wait();
-  float* my_slot = cluster.map_shared_rank(slots, 0) + (size_t)rank * B * r;
+  const uint32_t remote_slot = rank ? mapa_shared(slots + (size_t)rank * B * r, 0) : 0u;
+  const uint32_t remote_bar = rank ? mapa_shared(bar_red, 0) : 0u;
   for (int bb0 = 0; bb0 < B; bb0 += BB) {
     if (bb0 > 0) {
 #pragma unroll 1
@@ -259,87 +260,62 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     }
     float acc[BB][8];
     stream_rows<BB>(w, ring, xs, B, bb0, acc, tid);
-    reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, my_slot + (size_t)bb0 * r, tid);
+    reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, slots + (size_t)bb0 * r, remote_slot + 4u * bb0 * r,
+                   remote_bar, tid);
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
+  // The A stream is done: a decode launched behind this kernel may now be
+  // scheduled (it reads q and its B matrices, and waits for this grid to
+  // complete before it touches the cache).  Triggering here rather than at
+  // launch lets the non-leader CTAs leave first, so the decode's clusters
+  // find whole SMs.
+  griddep_launch_dependents();
+  if (rank != 0) return;  // slot values are in flight to the leader
 
-  if (rank != 0) {
-    // Publish the slot (release at cluster scope) and arrive on the leader's barrier.
-    if (tid == 0) {
-      asm volatile("fence.acq_rel.cluster;" ::: "memory");
-      const uint32_t remote = static_cast<uint32_t>(__cvta_generic_to_shared(bar_red));
-      uint32_t rbar;
-      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(remote), "r"(0));
-      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
-    }
-    return;
-  }
-
-  // 5. Leader: wait for the other ranks, sum the slots in rank order, quantise.
+  // 5. Leader: wait for the other ranks, sum the slots in rank order, quantise
+  //    (one warp per batch row; lane owns columns j = lane + 32k).
   if (a.cluster > 1) {
-    if (tid == 0) {
-      const uint32_t addr = smem_u32(bar_red);
-      const uint64_t t0 = globaltimer_ns();
-      for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr)
-            : "memory");
-        if (done) break;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-          break;
-        }
-      }
-    }
+    if (tid == 0 && !mbar_wait_cluster_bounded(bar_red, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     __syncthreads();
   }
-  float* cfin = red;  // [B][r]
-  for (int idx = tid; idx < B * r; idx += kAppendThreads) {
-    float s = 0.f;
-    for (int q = 0; q < a.cluster; ++q) s += slots[(size_t)q * B * r + idx];
-    cfin[idx] = s * a.hnorm;
-  }
-  __syncthreads();
   const int Q = (a.bits == 8) ? 127 : 7;
   const int RB = r * a.bits / 8;
   for (int b = warp; b < B; b += kAppendWarps) {
     const int pos = a.seq_lens[b];
     const bool ok = pos >= 0 && pos < a.L_cap;
-    const float* cb = cfin + (size_t)b * r;
+    float cv[4];
     float amax = 0.f;
-    for (int j = lane; j < r; j += 32) amax = fmaxf(amax, fabsf(cb[j]));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = lane + 32 * k;
+      cv[k] = 0.f;
+      if (j < r) {
+        float sum = 0.f;
+        for (int q = 0; q < a.cluster; ++q) sum += slots[((size_t)q * B + b) * r + j];
+        cv[k] = sum * a.hnorm;
+        amax = fmaxf(amax, fabsf(cv[k]));
+      }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
-    const float s = __half2float(sh);
-    for (int j = lane; j < r; j += 32) {
-      int code = 0;
-      if (s > 0.f) code = max(-Q, min(Q, __float2int_rn(__fdiv_rn(cb[j], s))));
-      codes[b * r + j] = (int8_t)code;
-    }
-    __syncwarp();
-    if (ok) {
-      const size_t row = ((size_t)b * a.H + h) * a.L_cap + pos;
-      uint32_t* dstw = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + row * RB);
-      for (int wi = lane; wi < RB / 4; wi += 32) {
-        uint32_t word = 0;
-        if (a.bits == 8) {
+    const float sc = __half2float(sh);
+    const size_t row = ((size_t)b * a.H + h) * a.L_cap + (ok ? pos : 0);
+    uint8_t* dst = (kv ? a.lat_v : a.lat_k) + row * RB;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) word |= (uint32_t)(uint8_t)codes[b * r + 4 * wi + k] << (8 * k);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) word |= ((uint32_t)codes[b * r + 8 * wi + k] & 0xFu) << (4 * k);
-        }
-        dstw[wi] = word;
+    for (int k = 0; k < 4; ++k) {
+      const int j = lane + 32 * k;
+      const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(cv[k], sc)))) : 0;
+      if (a.bits == 8) {
+        if (ok && j < r) dst[j] = (uint8_t)code;
+      } else {
+        const int hi = __shfl_down_sync(0xffffffffu, code, 1);  // column j + 1 (r is a multiple of 8)
+        if (ok && j < r && (lane & 1) == 0) dst[j / 2] = (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
       }
-      if (lane == 0) (kv ? a.scale_v : a.scale_k)[row] = sh;
-    } else if (lane == 0 && unit == 0) {
-      set_err(a.err, WSVD_DEVERR_CACHE_FULL);
+    }
+    if (lane == 0) {
+      if (ok) (kv ? a.scale_v : a.scale_k)[row] = sh;
+      else if (unit == 0) set_err(a.err, WSVD_DEVERR_CACHE_FULL);
     }
   }
   __syncthreads();

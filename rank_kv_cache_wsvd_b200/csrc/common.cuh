@@ -69,6 +69,44 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Address of `p` (this CTA's shared memory) in the shared window of cluster
+// CTA `rank`, as a shared::cluster address.
+__device__ __forceinline__ uint32_t mapa_shared(const void* p, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// 4-byte store into another cluster CTA's shared memory that completes 4
+// bytes of transaction count on that CTA's mbarrier (both shared::cluster
+// addresses).  Once the barrier phase completes the value is visible to the
+// waiting CTA; no fence is needed on either side.
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
+// Bounded wait (cluster-scope acquire) for phase `parity` of a barrier that
+// other CTAs of the cluster complete.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                          uint64_t limit_ns = kWaitLimitNs) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing `bytes` of
 // transaction count on `bar`.  Both addresses 16-byte aligned, bytes % 16 == 0.
 // No multicast: the destination is this CTA only.

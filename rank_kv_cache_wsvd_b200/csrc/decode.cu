@@ -1082,12 +1082,13 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
 
 // ------------------------------------------------------------------ cluster kernel (small problems)
 // One thread-block cluster of `cluster` CTAs per (b, h) splits the cached
-// tokens into contiguous chunks.  Each CTA issues its operand and tile copies
-// at launch (the operands before seq_lens is even read), reduces its chunk to
-// (m, l, o[W]) and stores it straight into a slot of the leader's shared
-// memory (distributed shared memory), then arrives on the leader's mbarrier.
-// The leader merges the slots in rank order and writes out[b, h] with B_Vh
-// staged in its shared memory: no global partials, counters or fences.
+// tokens into contiguous chunks.  Each CTA issues its operand copies at
+// launch and builds q' before it reads seq_lens (so under a programmatic
+// dependent launch that work overlaps the preceding append), reduces its
+// chunk to (m, l, o[W]) and stores it straight into a slot of the leader's
+// shared memory with st.async stores whose bytes complete on the leader's
+// mbarrier.  The leader merges the slots in rank order and writes out[b, h]
+// with B_Vh staged in its shared memory: no global partials, counters or fences.
 template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
 __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const DecodeArgs a) {
   using C = Cfg<CODEC, VPT, TPT, NTOK>;
@@ -1123,8 +1124,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     }
     mbar_init(segfull, 1);
     mbar_init(&aux[0], 1);
-    mbar_init(&aux[1], csize > 1 ? csize - 1 : 1);
+    mbar_init(&aux[1], 1);
     fence_mbar_init();
+    // leader: the other ranks' partial rows arrive as st.async transaction bytes
+    if (rank == 0 && csize > 1) mbar_arrive_expect_tx(&aux[1], (uint32_t)((csize - 1) * (W + 2) * 4));
     // Operands first: they do not depend on the sequence length.
     const uint64_t keep = l2_evict_last_policy();
     issue_operands<W, QMODE>(segbuf, segfull, a, b, h, keep);
@@ -1215,38 +1218,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
 
   cluster.barrier_wait();  // every CTA of the cluster has initialised its barriers
-  float* leader_slots = cluster.map_shared_rank(slots, 0);
-  for (int e = tid; e < W + 2; e += kConsumerThreads) leader_slots[(size_t)rank * (W + 2) + e] = res[e];
-  csync();
   if (rank != 0) {
-    if (tid == 0) {
-      asm volatile("fence.acq_rel.cluster;" ::: "memory");
-      uint32_t rbar;
-      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(&aux[1])), "r"(0));
-      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
-    }
+    // Partial row straight into the leader's slot; each store completes its
+    // bytes on the leader's barrier (no fence, no separate arrive).
+    const uint32_t rslot = mapa_shared(slots + (size_t)rank * (W + 2), 0), rbar = mapa_shared(&aux[1], 0);
+    for (int e = tid; e < W + 2; e += kConsumerThreads) st_async_f32(rslot + 4u * e, res[e], rbar);
     return;
   }
   if (csize > 1) {
-    if (tid == 0) {
-      const uint32_t addr = smem_u32(&aux[1]);
-      const uint64_t t0 = globaltimer_ns();
-      for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr)
-            : "memory");
-        if (done) break;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-          break;
-        }
-      }
-    }
+    for (int e = tid; e < W + 2; e += kConsumerThreads) slots[e] = res[e];
+    if (tid == 0 && !mbar_wait_cluster_bounded(&aux[1], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     csync();
     merge_rows<W, false>(slots, csize, res, tid);
   }
