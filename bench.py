@@ -181,7 +181,9 @@ class WsvdStep:
             self.x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
         self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
         self.out_host = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32).pin_memory()
-        self.launches_per_step = (1 if self.has_append else 0) + 1  # append, decode
+        # kernels per step: the append, and the decode's one or two (cluster kernel, or q' + split-L grid)
+        self.launches_per_step = (1 if self.has_append else 0) + W.wsvd_decode_launch_count(
+            w.B, w.H, w.Hd, w.r, w.bits, w.L_cap)
 
     def reset(self):
         self.lens.copy_(self.lens0)

@@ -104,13 +104,19 @@ size_t dense_cache_bytes(int B, int H, int L_cap, int Hd);
  *   workspace                device scratch of at least
  *                            wsvd_decode_workspace_size(B, H, r) bytes that is
  *                            ZERO before the first call (cudaMemset once):
- *                            it holds split partials and one completion
- *                            counter per (b, h), and every call leaves the
- *                            counters zero.  Calls that share a workspace must
- *                            not overlap on the GPU.
+ *                            it holds split partials, one completion counter
+ *                            per (b, h) and the projected queries q' [B][H][r]
+ *                            fp32, and every call leaves the counters zero.
+ *                            Calls that share a workspace must not overlap on
+ *                            the GPU.
  *   err                      optional device int32; WSVD_DEVERR_LEN_RANGE.
- * Rows >= seq_lens[b] are never used: their bytes may hold anything.        */
+ * Rows >= seq_lens[b] are never used: their bytes may hold anything.
+ * Depending on the sizes, one call launches one kernel (one cluster of CTAs
+ * per (b, h)) or two (q' for every (b, h), then the split-L grid launched
+ * behind it as a programmatic dependent); wsvd_decode_launch_count tells
+ * which, for the given sizes on the current device.                        */
 size_t wsvd_decode_workspace_size(int B, int H, int r);
+int wsvd_decode_launch_count(int B, int H, int Hd, int r, int bits, int L_cap);
 int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
                           const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
                           const void* scale_k, const void* scale_v, const void* B_k, const void* B_v,
@@ -127,7 +133,7 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
  * allocation would synchronise the device or fail (inside latency-critical
  * loops, under memory limits), or a host language binding without access to
  * device allocation.  The scratch it needs (split partials and one counter
- * per (b, h)) lives in a static device array of WSVD_NOALLOC_SCRATCH_BYTES
+ * per (b, h), the projected queries) lives in a static device array of WSVD_NOALLOC_SCRATCH_BYTES
  * that every GPU loading the library holds until the process exits; the call
  * itself allocates nothing.
  *   - A problem whose scratch need, wsvd_decode_workspace_size(B, H, r),

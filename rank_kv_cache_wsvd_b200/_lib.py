@@ -34,6 +34,7 @@ SIGNATURES = {
     "dense_decode_workspace_size": (_c_size, [_c_int] * 3),
     "shared_decode_workspace_size": (_c_size, [_c_int] * 3),
     "wsvd_append_workspace_size": (_c_size, []),
+    "wsvd_decode_launch_count": (_c_int, [_c_int] * 6),
     "wsvd_decode_attention": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size,
                                                                                         _p, _p]),
     "wsvd_decode_attention_noalloc": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _p]),
@@ -117,6 +118,11 @@ def dense_cache_bytes(B, H, L_cap, Hd) -> int:
 
 def wsvd_decode_workspace_size(B, H, r) -> int:
     return load().wsvd_decode_workspace_size(B, H, r)
+
+
+def wsvd_decode_launch_count(B, H, Hd, r, bits, L_cap) -> int:
+    """Kernels one wsvd_decode_attention call with these sizes launches on the current device."""
+    return load().wsvd_decode_launch_count(B, H, Hd, r, bits, L_cap)
 
 
 def dense_decode_workspace_size(B, H, Hd) -> int:

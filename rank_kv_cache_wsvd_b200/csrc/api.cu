@@ -19,11 +19,23 @@ inline float resolve_scale(float softmax_scale, int Hd) {
 inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
 // Decode workspace: split partials (m, l, o[W]) for every slot a persistent
-// grid can use, then one completion counter per (b, h).
+// grid can use, one completion counter per (b, h), then the projected query
+// q' [B][H][W] fp32 of the persistent path.
 inline size_t partial_bytes(int B, int H, int W) {
   return align16(((size_t)kMaxDecodeCtas + (size_t)B * H) * ((size_t)W + 2) * sizeof(float));
 }
-inline size_t decode_ws_bytes(int B, int H, int W) { return partial_bytes(B, H, W) + align16((size_t)B * H * 4); }
+inline size_t counter_bytes(int B, int H) { return align16((size_t)B * H * 4); }
+inline size_t decode_ws_bytes(int B, int H, int W) {
+  return partial_bytes(B, H, W) + counter_bytes(B, H) + align16((size_t)B * H * W * sizeof(float));
+}
+
+// Carve the caller's decode workspace into the kernel's regions.
+void bind_workspace(DecodeArgs* a, void* workspace) {
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  a->partials = reinterpret_cast<float*>(w);
+  a->counters = reinterpret_cast<int32_t*>(w + partial_bytes(a->B, a->H, a->W));
+  a->qglobal = reinterpret_cast<float*>(w + partial_bytes(a->B, a->H, a->W) + counter_bytes(a->B, a->H));
+}
 
 constexpr size_t kAppendWorkspaceBytes = 256;  // the completion counter (padded)
 
@@ -42,8 +54,7 @@ int check_common(int B, int H, int Hd, int L_cap, const int32_t* seq_lens, const
 }
 
 int run_decode(int codec, int rowbytes, int qmode, DecodeArgs a, void* workspace, cudaStream_t stream) {
-  a.partials = static_cast<float*>(workspace);
-  a.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + partial_bytes(a.B, a.H, a.W));
+  bind_workspace(&a, workspace);
   if (launch_decode(codec, rowbytes, qmode, a, stream) != cudaSuccess) return WSVD_ERR_CUDA;
   return WSVD_OK;
 }
@@ -70,7 +81,7 @@ int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const 
   a->seq_lens = seq_lens; a->q = q; a->q_dtype = q_dtype;
   a->lat_k = lat_k; a->lat_v = lat_v;
   a->scale_k = static_cast<const __half*>(scale_k); a->scale_v = static_cast<const __half*>(scale_v);
-  a->Bk = static_cast<const __half*>(B_k); a->Bv = static_cast<const __half*>(B_v); a->qglobal = nullptr;
+  a->Bk = static_cast<const __half*>(B_k); a->Bv = static_cast<const __half*>(B_v);
   a->qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
   a->out = out; a->err = err;
   return WSVD_OK;
@@ -153,7 +164,7 @@ size_t dense_decode_workspace_size(int B, int H, int Hd) {
 
 size_t shared_decode_workspace_size(int B, int H, int R) {
   if (B < 0 || H < 0 || R < 1) return 0;
-  return decode_ws_bytes(B, H, R) + align16((size_t)B * H * R * sizeof(float));
+  return decode_ws_bytes(B, H, R);
 }
 
 int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
@@ -201,18 +212,21 @@ int shared_latent_svd_decode(int B, int H, int Hd, int R, int L_cap, const int32
   if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(B_k) || !aligned16(B_v)) return WSVD_ERR_INVALID_ARG;
   if (workspace_bytes < shared_decode_workspace_size(B, H, R)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
 
-  float* qglobal = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + decode_ws_bytes(B, H, R));
-  if (launch_shared_qproj(B, H, Hd, R, q, q_dtype, static_cast<const __half*>(B_k), qglobal,
-                          as_stream(stream)) != cudaSuccess)
-    return WSVD_ERR_CUDA;
   DecodeArgs a{};
   a.B = B; a.H = H; a.Hd = Hd; a.W = R; a.L_cap = L_cap; a.heads_share = 1;
   a.seq_lens = seq_lens; a.q = q; a.q_dtype = q_dtype;
   a.lat_k = static_cast<const uint8_t*>(lat_k); a.lat_v = static_cast<const uint8_t*>(lat_v);
-  a.Bv = static_cast<const __half*>(B_v); a.qglobal = qglobal;
+  a.Bk = static_cast<const __half*>(B_k); a.Bv = static_cast<const __half*>(B_v);
   a.qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
   a.out = out; a.err = err;
   return run_decode(kCodecF16, rowbytes, kQGlobal, a, workspace, as_stream(stream));
+}
+
+int wsvd_decode_launch_count(int B, int H, int Hd, int r, int bits, int L_cap) {
+  if (B < 1 || H < 1 || L_cap < 0 || (bits != 8 && bits != 4) || r < 1 || (r * bits) % 8) return 0;
+  DecodeArgs a{};
+  a.B = B; a.H = H; a.Hd = Hd; a.W = r; a.L_cap = L_cap;
+  return decode_launch_count(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a);
 }
 
 size_t wsvd_append_workspace_size(void) { return kAppendWorkspaceBytes; }
@@ -244,8 +258,7 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
                            softmax_scale, out, decode_workspace, decode_workspace_bytes, err, &dp);
   if (st != WSVD_OK || B == 0) return st;
   if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
-  dp.partials = static_cast<float*>(decode_workspace);
-  dp.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(decode_workspace) + partial_bytes(B, H, r));
+  bind_workspace(&dp, decode_workspace);
   if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, as_stream(stream), true) !=
       cudaSuccess)
     return WSVD_ERR_CUDA;

@@ -80,16 +80,17 @@ __host__ __device__ inline size_t seg_bytes(int qmode, int W, int Hd) {
 }
 __host__ __device__ inline int seg_nbuf(int qmode, int W, int Hd) { return seg_bytes(qmode, W, Hd) <= 17408 ? 2 : 1; }
 
-// Helper-owned shared state (after the operand buffers).
-template <int W, int PW>
+// Helper-owned shared state (after the operand buffers): NQ query-state slots
+// the helper fills ahead of the consumers, two result slots it drains.
+template <int W, int PW, int NQ>
 struct HelperArea {
-  float qsv[2][W];            // scaled q' (fp16 codecs read it directly)
-  uint32_t planes[2][PW];     // packed byte planes + int4 corrections
-  float qstep[2];
-  int seginfo[2][4];          // b, h, c_first, c_last
+  float qsv[NQ][W];           // scaled q' (fp16 codecs read it directly)
+  uint32_t planes[NQ][PW];    // packed byte planes + int4 corrections
+  float qstep[NQ];
+  int seginfo[NQ][4];         // b, h, c_first, c_last
   float res[2][W + 2];        // merged (M, L, O[W]) of a segment, consumers -> helper
   int qi[W];                  // quantised q'
-  uint64_t bars[10];          // qready[2], qfree[2], resfull[2], resfree[2]
+  uint64_t bars[2 * NQ + 4];  // qready[NQ], qfree[NQ], resfull[2], resfree[2]
 };
 
 template <int CODEC, int VPT, int TPT, int NTOK>
@@ -110,6 +111,7 @@ struct Cfg {
   static constexpr int kRedRaw = kConsumerWarps * TPT * (VPT + 2);
   static constexpr int kRedFloats = kRedRaw < kConsumerThreads ? kConsumerThreads : kRedRaw;
   static constexpr int kQW = VPT / 4;  // byte-plane words of q' per lane
+  static constexpr int kNQ = kW <= 128 ? 4 : 2;  // helper query-state slots (segments built ahead)
   static_assert(kCB % 16 == 0, "a lane's chunk is a whole number of 16-byte loads");
   static_assert(kT % 8 == 0, "tile must hold a multiple of 8 tokens (16-byte scale copies)");
   static_assert(TPT <= 32 && (TPT & (TPT - 1)) == 0, "a token's lanes share a warp");
@@ -125,7 +127,7 @@ struct Cfg {
   // runtime part: lens / prefix (2B + 1 ints), then the segment buffers
   __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(2 * B + 1) * 4 + 127) / 128 * 128; }
   static size_t smem_bytes(int B, int qmode, int Hd) {
-    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) + sizeof(HelperArea<kW, kPlaneWords>);
+    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) + sizeof(HelperArea<kW, kPlaneWords, kNQ>);
   }
   // cluster kernel: operands, the leader's partial slots, then B_Vh
   __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
@@ -647,18 +649,24 @@ __device__ __forceinline__ void issue_tile(uint8_t* st, uint64_t* bar, const Dec
 // Warp-level q' = B_Kh . q from the staged operands: lane j-rotation keeps the
 // row reads on distinct banks.  Returns max|q'| (scaled by softmax_scale * log2 e).
 template <int W, int QMODE>
-__device__ __forceinline__ float helper_qprime(const uint8_t* sbuf, float* qsv, const DecodeArgs& a, int lane) {
+__device__ __forceinline__ float helper_qprime(const uint8_t* sbuf, float* qsv, const DecodeArgs& a, size_t bh,
+                                               int lane) {
   float amax = 0.f;
   if (QMODE == kQProj) {
     amax = qprime_rows(sbuf, qsv, a, W, lane >> 3, 4, lane & 7);
   } else if (QMODE == kQDirect) {
     const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf);
-    for (int j = lane; j < W; j += 32)
+    for (int j = lane; j < W; j += 32) {
       qsv[j] = (a.q_dtype == WSVD_DTYPE_BF16 ? __uint_as_float((uint32_t)qsrc[j] << 16)
                                              : __half2float(__ushort_as_half(qsrc[j]))) * a.qscale;
-  } else {
-    const float* qg = reinterpret_cast<const float*>(sbuf);
-    for (int j = lane; j < W; j += 32) qsv[j] = qg[j] * a.qscale;
+      amax = fmaxf(amax, fabsf(qsv[j]));
+    }
+  } else {  // q' projected beforehand into global memory (L2-coherent loads)
+    const float* qg = a.qglobal + bh * W;
+    for (int j = lane; j < W; j += 32) {
+      qsv[j] = __ldcg(qg + j) * a.qscale;
+      amax = fmaxf(amax, fabsf(qsv[j]));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -724,9 +732,14 @@ template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
 __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const DecodeArgs a) {
   using C = Cfg<CODEC, VPT, TPT, NTOK>;
   using CT = typename C::CT;
-  using HA = HelperArea<C::kW, C::kPlaneWords>;
-  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2, QW = VPT / 4;
+  using HA = HelperArea<C::kW, C::kPlaneWords, C::kNQ>;
+  constexpr int T = C::kT, W = C::kW, S = C::kStages, NP = VPT / 2, QW = VPT / 4, NQ = C::kNQ;
   constexpr int kProducerWarp = kConsumerWarps, kHelperWarp = kConsumerWarps + 1;
+  // How far the helper may build ahead of the oldest unfinished segment.  With
+  // q' in global memory nothing else gates a build; with operands staged by the
+  // producer (dense path) it stays one ahead, the producer being at most a
+  // ring's length ahead of the consumers.
+  constexpr int kAhead = QMODE == kQGlobal ? NQ : 2;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
@@ -742,15 +755,17 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   const uint32_t SEGB = (uint32_t)seg_bytes(QMODE, W, a.Hd);
   HA* ha = reinterpret_cast<HA*>(segbuf + (size_t)NBUF * SEGB);
   uint64_t* qready = ha->bars;
-  uint64_t* qfree = ha->bars + 2;
-  uint64_t* resfull = ha->bars + 4;
-  uint64_t* resfree = ha->bars + 6;
+  uint64_t* qfree = ha->bars + NQ;
+  uint64_t* resfull = ha->bars + 2 * NQ;
+  uint64_t* resfree = ha->bars + 2 * NQ + 2;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
-  // Launched behind the append (programmatic dependent launch): the split plan
-  // reads seq_lens, so nothing here may run before that grid has completed.
-  griddep_wait();
+  // Programmatic dependent launch: behind the append (dep 2) the split plan
+  // reads seq_lens, so nothing here may run before that grid has completed;
+  // behind the q' projection alone (dep 1) only the helper waits, before it
+  // reads q'.
+  if (a.dep == 2) griddep_wait();
 
   // Valid lengths, tiles per sequence (per head) and their exclusive prefix.
   if (warp == 0) {
@@ -784,10 +799,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       for (int s = 0; s < 2; ++s) {
         mbar_init(&segfull[s], 1);
         mbar_init(&segempty[s], 1);
-        mbar_init(&qready[s], 1);
-        mbar_init(&qfree[s], kConsumerWarps);
         mbar_init(&resfull[s], 1);
         mbar_init(&resfree[s], 1);
+      }
+      for (int s = 0; s < NQ; ++s) {
+        mbar_init(&qready[s], 1);
+        mbar_init(&qfree[s], kConsumerWarps);
       }
       fence_mbar_init();
     }
@@ -818,7 +835,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       int nseg = 0, pb = -1, ph = -1;
       bool ok = true;
       for (long long g = g_begin; g < g_end && ok; ++g, ++issued) {
-        if (b != pb || h != ph) {  // operands of the next (b, h)
+        if (QMODE != kQGlobal && (b != pb || h != ph)) {  // operands of the next (b, h)
           const int sb = nseg % NBUF;
           if (nseg >= NBUF && !mbar_wait_bounded(&segempty[sb], (uint32_t)(((nseg / NBUF) - 1) & 1))) {
             set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
@@ -874,31 +891,16 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
     };
     int built = 0, done = 0;
     bool more = true;
-    {  // segment 0: the consumers build its query state; record what finishing it needs
-      int sb_b, sb_h;
-      if (next_segment(sb_b, sb_h)) {
-        const int tb = walk.tiles(sb_b);
-        const long long gf = (long long)a.H * pre[sb_b] + (long long)sb_h * tb;
-        if (lane == 0) {
-          ha->seginfo[0][0] = sb_b;
-          ha->seginfo[0][1] = sb_h;
-          ha->seginfo[0][2] = cta_of(gf, G, CW);
-          ha->seginfo[0][3] = cta_of(gf + tb - 1, G, CW);
-        }
-        built = 1;
-      } else {
-        more = false;
-      }
-    }
+    if (QMODE == kQGlobal) griddep_wait();  // q' comes from the grid this one was launched behind
     while (true) {
-      // Build up to one segment ahead of the oldest unfinished one.
-      while (more && built <= done + 1) {
+      // Build ahead of the oldest unfinished segment (see kAhead).
+      while (more && built < done + kAhead) {
         int sb_b, sb_h;
         if (!next_segment(sb_b, sb_h)) {
           more = false;
           break;
         }
-        const int k = built, sq = k & 1;
+        const int k = built, sq = k % NQ;
         const int tb = walk.tiles(sb_b);
         const long long gf = (long long)a.H * pre[sb_b] + (long long)sb_h * tb;
         const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
@@ -912,11 +914,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
           const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)sb_h * W * a.Hd);
           for (int o = lane * 128; o < W * a.Hd * 2; o += 32 * 128) prefetch_l2(bv + o);
         }
-        wait(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1));
-        if (k >= 2) wait(&qfree[sq], (uint32_t)(((k / 2) - 1) & 1));
-        const float amax = helper_qprime<W, QMODE>(segbuf + (size_t)(k % NBUF) * SEGB, ha->qsv[sq], a, lane);
+        if (QMODE != kQGlobal) wait(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1));
+        if (k >= NQ) wait(&qfree[sq], (uint32_t)(((k / NQ) - 1) & 1));
+        const float amax = helper_qprime<W, QMODE>(segbuf + (size_t)(k % NBUF) * SEGB, ha->qsv[sq], a,
+                                                   (size_t)sb_b * a.H + sb_h, lane);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&segempty[k % NBUF]);  // the staged operands are consumed
+        if (QMODE != kQGlobal && lane == 0) mbar_arrive(&segempty[k % NBUF]);  // staged operands consumed
         if constexpr (CT::kScaled) {
           helper_planes<CODEC, VPT, W>(ha->qsv[sq], ha->qi, ha->planes[sq], &ha->qstep[sq], amax, lane);
         } else {
@@ -929,11 +932,11 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       // The consumers finish the CTA's last segment themselves.
       if (done == built || (!more && done == built - 1)) break;
       // Finish segment `done` once the consumers have reduced it.
-      const int k = done, sr = k & 1;
+      const int k = done, sr = k & 1, si = k % NQ;
       wait(&resfull[sr], (uint32_t)((k / 2) & 1));
       const float* res = ha->res[sr];
-      const int sb_b = ha->seginfo[sr][0], sb_h = ha->seginfo[sr][1];
-      const int cf = ha->seginfo[sr][2], cl = ha->seginfo[sr][3];
+      const int sb_b = ha->seginfo[si][0], sb_h = ha->seginfo[si][1];
+      const int cf = ha->seginfo[si][2], cl = ha->seginfo[si][3];
       float* outp = a.out + ((size_t)sb_b * a.H + sb_h) * a.Hd;
       const __half* Bvh = a.Bv ? a.Bv + (size_t)sb_h * W * a.Hd : nullptr;
       if (cf == cl) {
@@ -1027,35 +1030,26 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   for (long long g = g_begin; g < g_end; ++g, ++i) {
     if (b != cb || h != ch) {
       if (cb >= 0) end_segment(k - 1);
-      const int sq = k & 1;
-      if (k == 0) {  // first segment: build the query state with every consumer thread
-        wait(&segfull[0], 0);
-        build_query<CODEC, VPT, W, QMODE>(qst, segbuf, ha->qsv[0], misc, ha->planes[0], a, tid, sub);
-        if (tid == 0) {
-          mbar_arrive(&segempty[0]);
-          mbar_arrive(&qready[0]);  // keeps qready[0]'s phases aligned with the segments that use it
+      const int sq = k % NQ;
+      wait(&qready[sq], (uint32_t)((k / NQ) & 1));
+      qst.step = ha->qstep[sq];
+      if constexpr (CT::kScaled) {
+        const uint32_t* pl = ha->planes[sq];
+#pragma unroll
+        for (int q = 0; q < QW; ++q) {
+          qst.qh[q] = pl[(sub * 3 + 0) * QW + q];
+          qst.qm[q] = pl[(sub * 3 + 1) * QW + q];
+          qst.ql[q] = pl[(sub * 3 + 2) * QW + q];
+        }
+        if constexpr (CODEC == kCodecI4) {
+          qst.ch = (int)pl[TPT * 3 * QW + sub * 3 + 0];
+          qst.cm = (int)pl[TPT * 3 * QW + sub * 3 + 1];
+          qst.cl = (int)pl[TPT * 3 * QW + sub * 3 + 2];
         }
       } else {
-        wait(&qready[sq], (uint32_t)((k / 2) & 1));
-        qst.step = ha->qstep[sq];
-        if constexpr (CT::kScaled) {
-          const uint32_t* pl = ha->planes[sq];
 #pragma unroll
-          for (int q = 0; q < QW; ++q) {
-            qst.qh[q] = pl[(sub * 3 + 0) * QW + q];
-            qst.qm[q] = pl[(sub * 3 + 1) * QW + q];
-            qst.ql[q] = pl[(sub * 3 + 2) * QW + q];
-          }
-          if constexpr (CODEC == kCodecI4) {
-            qst.ch = (int)pl[TPT * 3 * QW + sub * 3 + 0];
-            qst.cm = (int)pl[TPT * 3 * QW + sub * 3 + 1];
-            qst.cl = (int)pl[TPT * 3 * QW + sub * 3 + 2];
-          }
-        } else {
-#pragma unroll
-          for (int p = 0; p < NP; ++p)
-            qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
-        }
+        for (int p = 0; p < NP; ++p)
+          qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&qfree[sq]);
@@ -1300,52 +1294,109 @@ int device_sms_and_occupancy(const void* fn, size_t smem, int threads, int* occ_
 
 struct KernelInfo {
   const void* fn;          // persistent kernel
-  const void* cfn;         // cluster kernel (same tile shape)
+  const void* cfn;         // cluster kernel (same tile shape), or null
+  int pqmode;              // query mode of the persistent kernel
   size_t (*smem)(int B, int qmode, int Hd);
   size_t (*csmem)(int qmode, int Hd);
   int tile;
 };
 
-template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
+constexpr int kNoCluster = -1;
+
+// PQ: query mode of the persistent kernel; CQ: of the cluster kernel (or
+// kNoCluster).  The low-rank codecs project q' inside the cluster kernel but
+// take it precomputed (kQGlobal) in the persistent one, whose helper warp
+// then only packs byte planes.
+template <int CODEC, int VPT, int TPT, int NTOK, int PQ, int CQ>
 KernelInfo info() {
   using C = Cfg<CODEC, VPT, TPT, NTOK>;
-  return KernelInfo{reinterpret_cast<const void*>(&decode_kernel<CODEC, VPT, TPT, NTOK, QMODE>),
-                    reinterpret_cast<const void*>(&decode_cluster_kernel<CODEC, VPT, TPT, NTOK, QMODE>),
+  const void* cfn = nullptr;
+  if constexpr (CQ != kNoCluster) cfn = reinterpret_cast<const void*>(&decode_cluster_kernel<CODEC, VPT, TPT, NTOK, CQ>);
+  return KernelInfo{reinterpret_cast<const void*>(&decode_kernel<CODEC, VPT, TPT, NTOK, PQ>), cfn, PQ,
                     &C::smem_bytes, &C::cluster_smem_bytes, C::kT};
 }
 
 // Instantiated shapes.  `big` selects the variant with more tokens per lane per
-// tile (fewer, larger tiles) for long caches.
+// tile (fewer, larger tiles) for long caches.  qmode is the caller's: kQProj
+// (low-rank), kQDirect (dense) or kQGlobal (shared latent).
 bool pick(int codec, int rowbytes, int qmode, bool big, KernelInfo* ki) {
+  constexpr int P = kQGlobal, X = kQProj;
   if (qmode == kQProj && codec == kCodecI8) {
     switch (rowbytes) {
-      case 16: *ki = big ? info<kCodecI8, 16, 1, 4, kQProj>() : info<kCodecI8, 16, 1, 2, kQProj>(); return true;
-      case 32: *ki = big ? info<kCodecI8, 32, 1, 2, kQProj>() : info<kCodecI8, 32, 1, 1, kQProj>(); return true;
-      case 64: *ki = info<kCodecI8, 32, 2, 1, kQProj>(); return true;
-      case 128: *ki = info<kCodecI8, 32, 4, 1, kQProj>(); return true;
+      case 16: *ki = big ? info<kCodecI8, 16, 1, 4, P, X>() : info<kCodecI8, 16, 1, 2, P, X>(); return true;
+      case 32: *ki = big ? info<kCodecI8, 32, 1, 2, P, X>() : info<kCodecI8, 32, 1, 1, P, X>(); return true;
+      case 64: *ki = info<kCodecI8, 32, 2, 1, P, X>(); return true;
+      case 128: *ki = info<kCodecI8, 32, 4, 1, P, X>(); return true;
     }
   } else if (qmode == kQProj && codec == kCodecI4) {
     switch (rowbytes) {
-      case 16: *ki = big ? info<kCodecI4, 32, 1, 2, kQProj>() : info<kCodecI4, 32, 1, 1, kQProj>(); return true;
-      case 32: *ki = info<kCodecI4, 32, 2, 1, kQProj>(); return true;
-      case 64: *ki = info<kCodecI4, 32, 4, 1, kQProj>(); return true;
+      case 16: *ki = big ? info<kCodecI4, 32, 1, 2, P, X>() : info<kCodecI4, 32, 1, 1, P, X>(); return true;
+      case 32: *ki = info<kCodecI4, 32, 2, 1, P, X>(); return true;
+      case 64: *ki = info<kCodecI4, 32, 4, 1, P, X>(); return true;
     }
   } else if (qmode == kQDirect && codec == kCodecF16) {
     switch (rowbytes) {
-      case 64: *ki = info<kCodecF16, 16, 2, 2, kQDirect>(); return true;
-      case 128: *ki = info<kCodecF16, 16, 4, 2, kQDirect>(); return true;
-      case 256: *ki = info<kCodecF16, 16, 8, 2, kQDirect>(); return true;
-      case 512: *ki = info<kCodecF16, 16, 16, 2, kQDirect>(); return true;
+      case 64: *ki = info<kCodecF16, 16, 2, 2, kQDirect, kQDirect>(); return true;
+      case 128: *ki = info<kCodecF16, 16, 4, 2, kQDirect, kQDirect>(); return true;
+      case 256: *ki = info<kCodecF16, 16, 8, 2, kQDirect, kQDirect>(); return true;
+      case 512: *ki = info<kCodecF16, 16, 16, 2, kQDirect, kQDirect>(); return true;
     }
   } else if (qmode == kQGlobal && codec == kCodecF16) {
     switch (rowbytes) {
-      case 256: *ki = info<kCodecF16, 16, 8, 2, kQGlobal>(); return true;
-      case 512: *ki = info<kCodecF16, 16, 16, 2, kQGlobal>(); return true;
-      case 1024: *ki = info<kCodecF16, 16, 32, 1, kQGlobal>(); return true;
-      case 2048: *ki = info<kCodecF16, 32, 32, 1, kQGlobal>(); return true;
+      case 256: *ki = info<kCodecF16, 16, 8, 2, P, kNoCluster>(); return true;
+      case 512: *ki = info<kCodecF16, 16, 16, 2, P, kNoCluster>(); return true;
+      case 1024: *ki = info<kCodecF16, 16, 32, 1, P, kNoCluster>(); return true;
+      case 2048: *ki = info<kCodecF16, 32, 32, 1, P, kNoCluster>(); return true;
     }
   }
   return false;
+}
+
+// The launch plan of one decode call: the cluster kernel (few tiles per
+// resident CTA, B_Vh fits in the leader's shared memory) or the persistent
+// grid, large-tile variant when there are several tiles per resident CTA.
+struct Plan {
+  bool cluster;
+  int csize;        // cluster path: CTAs per (b, h)
+  KernelInfo ki;    // the kernel to launch
+  size_t smem;
+  int ctas;         // persistent path: grid size
+};
+
+bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* pl) {
+  KernelInfo small, big;
+  if (!pick(codec, rowbytes, qmode, false, &small) || !pick(codec, rowbytes, qmode, true, &big)) return false;
+  int occ = 1;
+  const size_t smem_small = small.smem(a.B, small.pqmode, a.Hd);
+  const int sms = device_sms_and_occupancy(small.fn, smem_small, kPersistThreads, &occ);
+  const long long resident = (long long)sms * occ;
+  const long long tiles_small = (long long)a.B * a.H * ((a.L_cap + small.tile - 1) / small.tile);
+  const size_t csmem = small.cfn ? small.csmem(qmode, a.Hd) : 0;
+  if (small.cfn && tiles_small <= 2 * resident && csmem <= 112 * 1024 && a.H <= 65535) {
+    pl->cluster = true;
+    pl->csize = (int)std::min<long long>(kMaxClusterSize, std::max(1, (a.L_cap + 127) / 128));
+    pl->ki = small;
+    pl->smem = csmem;
+    pl->ctas = 0;
+    return true;
+  }
+  const size_t smem_big = big.smem(a.B, big.pqmode, a.Hd);
+  device_sms_and_occupancy(big.fn, smem_big, kPersistThreads, &occ);
+  const long long tiles_big = (long long)a.B * a.H * ((a.L_cap + big.tile - 1) / big.tile);
+  const KernelInfo& ki = (tiles_big >= 4 * (long long)sms * occ) ? big : small;
+  const size_t smem = ki.smem(a.B, ki.pqmode, a.Hd);
+  device_sms_and_occupancy(ki.fn, smem, kPersistThreads, &occ);
+  const long long tiles_max = (long long)a.B * a.H * ((a.L_cap + ki.tile - 1) / ki.tile);
+  long long ctas = (long long)sms * occ;
+  if (ctas > tiles_max) ctas = tiles_max;
+  if (ctas > kMaxDecodeCtas) ctas = kMaxDecodeCtas;
+  if (ctas < 1) ctas = 1;
+  pl->cluster = false;
+  pl->csize = 0;
+  pl->ki = ki;
+  pl->smem = smem;
+  pl->ctas = (int)ctas;
+  return true;
 }
 
 }  // namespace
@@ -1355,72 +1406,61 @@ bool decode_supported(int codec, int rowbytes, int qmode) {
   return pick(codec, rowbytes, qmode, false, &ki) && pick(codec, rowbytes, qmode, true, &ki);
 }
 
-cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream, bool pdl) {
-  KernelInfo small, big;
-  if (!pick(codec, rowbytes, qmode, false, &small) || !pick(codec, rowbytes, qmode, true, &big))
-    return cudaErrorInvalidValue;
-  int occ = 1;
-  const size_t smem_small = small.smem(a.B, qmode, a.Hd);
-  const int sms = device_sms_and_occupancy(small.fn, smem_small, kPersistThreads, &occ);
-  const long long resident = (long long)sms * occ;
-  const long long tiles_small = (long long)a.B * a.H * ((a.L_cap + small.tile - 1) / small.tile);
+int decode_launch_count(int codec, int rowbytes, int qmode, const DecodeArgs& a) {
+  Plan pl;
+  if (!plan_decode(codec, rowbytes, qmode, a, &pl)) return 0;
+  return (!pl.cluster && pl.ki.pqmode == kQGlobal) ? 2 : 1;
+}
 
-  // Few tiles per resident CTA: one cluster per (b, h), merged on chip (the
-  // low-rank and dense paths; B_Vh must fit in the leader's shared memory).
-  const size_t csmem = small.csmem(qmode, a.Hd);
-  if (tiles_small <= 2 * resident && qmode != kQGlobal && csmem <= 112 * 1024 && a.H <= 65535) {
-    const int csize = (int)std::min<long long>(kMaxClusterSize, std::max(1, (a.L_cap + 127) / 128));
-    const size_t smem = csmem;
-    cudaError_t e = ensure_smem(small.cfn, smem);
-    if (e != cudaSuccess) return e;
-    a.ctas = csize;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(csize, a.H, a.B);
-    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 2 : 1;
-    void* args[] = {&a};
-    return cudaLaunchKernelExC(&cfg, small.cfn, args);
-  }
-
-  // Otherwise the persistent grid; the large-tile variant when there are several
-  // tiles per resident CTA.
-  const size_t smem_big = big.smem(a.B, qmode, a.Hd);
-  device_sms_and_occupancy(big.fn, smem_big, kPersistThreads, &occ);
-  const long long tiles_big = (long long)a.B * a.H * ((a.L_cap + big.tile - 1) / big.tile);
-  const KernelInfo& ki = (tiles_big >= 4 * (long long)sms * occ) ? big : small;
-  const size_t smem = ki.smem(a.B, qmode, a.Hd);
-  device_sms_and_occupancy(ki.fn, smem, kPersistThreads, &occ);
-  const long long tiles_max = (long long)a.B * a.H * ((a.L_cap + ki.tile - 1) / ki.tile);
-  long long ctas = (long long)sms * occ;
-  if (ctas > tiles_max) ctas = tiles_max;
-  if (ctas > kMaxDecodeCtas) ctas = kMaxDecodeCtas;
-  if (ctas < 1) ctas = 1;
-  a.ctas = (int)ctas;
-  cudaError_t e = ensure_smem(ki.fn, smem);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream, bool after_append) {
+  Plan pl;
+  if (!plan_decode(codec, rowbytes, qmode, a, &pl)) return cudaErrorInvalidValue;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   void* args[] = {&a};
-  if (!pdl) return cudaLaunchKernel(ki.fn, dim3(a.ctas), dim3(kPersistThreads), args, smem, stream);
+  if (pl.cluster) {
+    cudaError_t e = ensure_smem(pl.ki.cfn, pl.smem);
+    if (e != cudaSuccess) return e;
+    a.ctas = pl.csize;
+    a.dep = after_append ? 2 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.csize, a.H, a.B);
+    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = pl.csize;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = after_append ? attr : attr + 1;
+    cfg.numAttrs = after_append ? 2 : 1;
+    return cudaLaunchKernelExC(&cfg, pl.ki.cfn, args);
+  }
+  cudaError_t e = ensure_smem(pl.ki.fn, pl.smem);
+  if (e != cudaSuccess) return e;
+  a.ctas = pl.ctas;
+  bool pdl = after_append;
+  if (pl.ki.pqmode == kQGlobal) {
+    // q' for every (b, h) first; the decode is launched behind it so that its
+    // split plan and first tiles overlap the projection (only its helper warp
+    // waits for q').  Behind an append the projection itself completes after
+    // the append, and the decode waits for everything (dep 2).
+    e = launch_qproj(a.B, a.H, a.Hd, a.W, a.q, a.q_dtype, a.Bk, a.qglobal, stream, after_append);
+    if (e != cudaSuccess) return e;
+    a.dep = after_append ? 2 : 1;
+    pdl = true;
+  } else {
+    a.dep = after_append ? 2 : 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.ctas);
   cfg.blockDim = dim3(kPersistThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, ki.fn, args);
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelExC(&cfg, pl.ki.fn, args);
 }
 
 }  // namespace wsvd

@@ -1,16 +1,16 @@
-// Conventional (shared-latent) SVD decode, the comparison path of the WSVD
-// summaries (Japanese §1, German §1): one fp16 latent [L][R] per sequence is
-// shared by all heads, and every head projects its query through its own
-// B_Kh (R x Hd) and re-reads the whole shared latent.  This file holds the
-// query projection q'_h = B_Kh . q_h (R values per (b, h)); the streaming part
-// is the split-L kernel of decode.cu run over R-wide fp16 rows with
-// heads_share = 1, and the merge + B_Vh up-projection is combine_kernel.
+// Query projection q'_{b,h} = B_Kh . q_{b,h} (W values per (b, h)) into a
+// global buffer, for the split-L kernel of decode.cu in its kQGlobal mode:
+// the per-head low-rank path (W = r, the reassociated score q . K^T =
+// (B_Kh . q) . lat_K^T of the WSVD summaries, German §2.A) and the
+// conventional shared-latent SVD decode (W = R; Japanese §1, German §1).
 #include "common.cuh"
 
 namespace wsvd {
 
-__global__ void __launch_bounds__(256) shared_qproj_kernel(int H, int Hd, int R, const void* q, int q_dtype,
-                                                           const __half* Bk, float* qglobal) {
+__global__ void __launch_bounds__(256) qproj_kernel(int H, int Hd, int R, const void* q, int q_dtype,
+                                                    const __half* Bk, float* qglobal) {
+  // A decode launched behind this kernel may start now; it waits for q'.
+  griddep_launch_dependents();
   const int bh = blockIdx.x, h = bh % H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float qr[8];
@@ -27,12 +27,24 @@ __global__ void __launch_bounds__(256) shared_qproj_kernel(int H, int Hd, int R,
     for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
     if (lane == 0) qglobal[(size_t)bh * R + j] = d;
   }
+  // Launched behind the append (programmatic dependent launch): this grid
+  // must not complete before that one, so that a decode waiting on this grid
+  // also sees the appended row.  A no-op for a normal launch.
+  griddep_wait();
 }
 
-cudaError_t launch_shared_qproj(int B, int H, int Hd, int R, const void* q, int q_dtype, const __half* Bk,
-                                float* qglobal, cudaStream_t stream) {
-  shared_qproj_kernel<<<B * H, 256, 0, stream>>>(H, Hd, R, q, q_dtype, Bk, qglobal);
-  return cudaGetLastError();
+cudaError_t launch_qproj(int B, int H, int Hd, int W, const void* q, int q_dtype, const __half* Bk, float* qglobal,
+                         cudaStream_t stream, bool after_append) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * H);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_append ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, qproj_kernel, H, Hd, W, q, q_dtype, Bk, qglobal);
 }
 
 }  // namespace wsvd

@@ -29,6 +29,7 @@ struct DecodeArgs {
   int B, H, Hd, W;       // W: latent width per token (r, Hd or R)
   int L_cap;
   int ctas;              // persistent grid size C (set by launch_decode)
+  int dep;               // programmatic dependency: 0 none, 1 only q' (qglobal), 2 everything (set by launch_decode)
   int heads_share;       // 1: the latent rows of (b, h) are the rows of b (shared-latent path)
   const int32_t* seq_lens;
   const void* q;
@@ -39,7 +40,7 @@ struct DecodeArgs {
   const __half* scale_v;
   const __half* Bk;      // [H][W][Hd] (kQProj)
   const __half* Bv;      // [H][W][Hd], or nullptr for the dense path (W == Hd)
-  const float* qglobal;  // [B][H][W] (kQGlobal)
+  float* qglobal;        // [B][H][W] projected q' (kQGlobal; workspace)
   float qscale;          // softmax_scale * log2(e)
   float* out;            // [B][H][Hd]
   float* partials;       // [(kMaxDecodeCtas + B*H)][W + 2]
@@ -49,11 +50,19 @@ struct DecodeArgs {
 
 // Host launchers (decode.cu, shared.cu, append.cu).  Return a cudaError_t.
 bool decode_supported(int codec, int rowbytes, int qmode);
-// pdl: launch as a programmatic dependent of the preceding kernel in `stream`
-// (the kernel reads q and the B matrices before that kernel completes).
-cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream, bool pdl = false);
-cudaError_t launch_shared_qproj(int B, int H, int Hd, int R, const void* q, int q_dtype, const __half* Bk,
-                                float* qglobal, cudaStream_t stream);
+// after_append: the preceding kernel in `stream` writes the cache (the fused
+// step); the decode is launched as its programmatic dependent and reads q and
+// the B matrices before that kernel completes.  The persistent path launches
+// the q' projection first (launch_qproj) and the decode behind it.
+cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cudaStream_t stream,
+                          bool after_append = false);
+// q'[b][h][:] = B_Kh . q[b, h] (W values) into qglobal.  after_append: launched
+// as a programmatic dependent of the preceding kernel, and completes only
+// after that kernel has (so a decode launched behind it may rely on both).
+cudaError_t launch_qproj(int B, int H, int Hd, int W, const void* q, int q_dtype, const __half* Bk, float* qglobal,
+                         cudaStream_t stream, bool after_append);
+// Kernels one launch_decode call issues (1, or 2 with the q' projection).
+int decode_launch_count(int codec, int rowbytes, int qmode, const DecodeArgs& a);
 
 struct AppendArgs {
   int B, H, E, r, bits, L_cap, blk, cluster;

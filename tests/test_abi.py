@@ -54,16 +54,17 @@ def test_cache_byte_counts_match_oracle(lib, B, H, L, r, bits):
 
 
 def test_workspace_sizes_hold_only_partials(lib):
-    """The decode workspace holds split partials (r + 2 floats per slot), never
+    """The decode workspace holds split partials (W + 2 floats per slot), one
+    counter per head and the projected queries q' (W floats per head), never
     an L x Hd buffer: reconstructed K/V are not materialised."""
     B, H, r, L = 4, 32, 32, 32768
     a16 = lambda v: (v + 15) // 16 * 16
+    size = lambda W_: a16((2048 + B * H) * (W_ + 2) * 4) + a16(B * H * 4) + a16(B * H * W_ * 4)
     ws = W.wsvd_decode_workspace_size(B, H, r)
-    assert ws == a16((2048 + B * H) * (r + 2) * 4) + a16(B * H * 4)  # partial slots + one counter per head
+    assert ws == size(r)
     assert ws < B * H * L * 128 * 2 / 100  # far below one reconstructed K
-    assert W.dense_decode_workspace_size(B, H, 128) == a16((2048 + B * H) * 130 * 4) + a16(B * H * 4)
-    assert W.shared_decode_workspace_size(B, H, 512) == (a16((2048 + B * H) * 514 * 4) + a16(B * H * 4)
-                                                         + B * H * 512 * 4)
+    assert W.dense_decode_workspace_size(B, H, 128) == size(128)
+    assert W.shared_decode_workspace_size(B, H, 512) == size(512)
     assert W.wsvd_append_workspace_size() == 256
 
 
@@ -100,3 +101,11 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.dense_decode_attention(1, 4, 48, 256, p, p, 0, p, p, 0.0, p, p, 1 << 22, None, None) == 2
     assert lib.shared_latent_svd_decode(1, 4, 128, 384, 256, p, p, 0, p, p, p, p, 0.0, p, p, 1 << 24,
                                         None, None) == 2
+
+
+def test_decode_launch_count_rejects_bad_sizes(lib):
+    """wsvd_decode_launch_count answers 0 for sizes the decode would reject."""
+    assert W.wsvd_decode_launch_count(0, 32, 128, 32, 8, 1600) == 0
+    assert W.wsvd_decode_launch_count(1, 32, 128, 32, 5, 1600) == 0
+    assert W.wsvd_decode_launch_count(1, 32, 128, 3, 4, 1600) == 0  # r * bits not a whole byte
+    assert W.wsvd_decode_launch_count(1, 32, 128, 24, 8, 1600) == 0  # 24-byte rows are not instantiated

@@ -91,3 +91,13 @@ def test_step_validates_before_launching():
     torch.cuda.synchronize()
     assert np.array_equal(st["lens"].cpu().numpy(), np.asarray(lens0))
     assert torch.equal(st["lat_k"], dev(d.lat_k))
+
+
+def test_decode_launch_count_matches_the_path():
+    """One kernel for the cluster path (the LLaVA layer), two for the split-L
+    grid behind its q' projection (long contexts, ragged batches)."""
+    lc = W.wsvd_decode_launch_count
+    w = WL.LLAVA7B
+    assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 1
+    for w in (WL.LONG[16], WL.LONG[32], WL.LONG[64], WL.RAGGED, WL.CMP[8192]):
+        assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 2, w.name
