@@ -183,7 +183,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   }
   // Every CTA's barrier is initialised before any remote access; the wait is
   // deferred to the first remote access.
-  cluster.barrier_arrive();
+  cluster_arrive_relaxed();
 
   // 1. x slice loads first (registers), then the A stream.
   constexpr int kMaxChunks = 4;  // 128-element x chunks per warp held in registers (fast path)
@@ -250,7 +250,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   __syncthreads();
 
   // 3. + 4. Stream the A rows, reduce into this rank's slot of the leader.
-  cluster.barrier_wait();
+  cluster_wait();
   const uint32_t remote_slot = rank ? mapa_shared(slots + (size_t)rank * B * r, 0) : 0u;
   const uint32_t remote_bar = rank ? mapa_shared(bar_red, 0) : 0u;
   for (int bb0 = 0; bb0 < B; bb0 += BB) {

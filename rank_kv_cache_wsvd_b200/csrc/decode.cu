@@ -280,15 +280,16 @@ __device__ __forceinline__ int cta_of(long long g, long long G, int C) {
 // phase touches 32 distinct banks.
 template <int NSEG>
 __device__ __forceinline__ void load_chunk(uint4* seg, const uint8_t* p, int lane) {
+  const uint32_t a = smem_u32(p);
   if constexpr (NSEG == 2) {
     const bool swap = (lane >> 2) & 1;
-    const uint4 x = *reinterpret_cast<const uint4*>(p + (swap ? 16 : 0));
-    const uint4 y = *reinterpret_cast<const uint4*>(p + (swap ? 0 : 16));
+    const uint4 x = lds128(a + (swap ? 16u : 0u));
+    const uint4 y = lds128(a + (swap ? 0u : 16u));
     seg[0] = swap ? y : x;
     seg[1] = swap ? x : y;
   } else {
 #pragma unroll
-    for (int j = 0; j < NSEG; ++j) seg[j] = *reinterpret_cast<const uint4*>(p + 16 * j);
+    for (int j = 0; j < NSEG; ++j) seg[j] = lds128(a + 16u * j);
   }
 }
 
@@ -437,7 +438,7 @@ __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QSt
 #pragma unroll
     for (int o = 1; o < TPT; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
     const bool valid = tok < n;
-    const float skk = (CT::kScaled && valid) ? __half2float(sck[tok]) * qst.step : qst.step;
+    const float skk = (CT::kScaled && valid) ? lds_half_as_float(smem_u32(sck + tok)) * qst.step : qst.step;
     sc[k] = valid ? d * skk : kNegInf;
     tmax = fmaxf(tmax, sc[k]);
   }
@@ -454,7 +455,7 @@ __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QSt
     if (tok < n) {
       const float p = ex2(sc[k] - m);
       l += p;
-      const float wv = CT::kScaled ? p * __half2float(sck[T + tok]) : p;
+      const float wv = CT::kScaled ? p * lds_half_as_float(smem_u32(sck + T + tok)) : p;
       uint4 seg[NSEG];
       load_chunk<NSEG>(seg, st + C::kCodeBytes + (size_t)tok * RB + sub * CB, lane);
       axpy<CODEC, VPT>(seg, wv, acc);
@@ -1133,7 +1134,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
                  min(32768u, bb - off), &aux[0], keep);
     }
   }
-  cluster.barrier_arrive();  // barriers initialised; waited on before any remote access
+  cluster_arrive_relaxed();  // barriers initialised; waited on before any remote access
   __syncthreads();           // barrier initialisation visible to every thread of this CTA
 
   // Everything above reads only q and the B matrices.  Under a programmatic
@@ -1176,7 +1177,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
       if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     }
-    cluster.barrier_wait();
+    cluster_wait();
     return;
   }
 
@@ -1211,7 +1212,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   }
   reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
 
-  cluster.barrier_wait();  // every CTA of the cluster has initialised its barriers
+  cluster_wait();  // every CTA of the cluster has initialised its barriers
   if (rank != 0) {
     // Partial row straight into the leader's slot; each store completes its
     // bytes on the leader's barrier (no fence, no separate arrive).
