@@ -61,8 +61,8 @@ def source_digest(files):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h"],
-                  "decode": ["decode.cu", "common.cuh", "wsvd_internal.h"]}
+KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
+                  "decode": ["decode.cu", "shared.cu", "common.cuh", "wsvd_internal.h", "api.cu"]}
 
 
 def ncu_traffic(kernel: str, workload: str):

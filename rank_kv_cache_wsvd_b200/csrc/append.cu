@@ -41,13 +41,13 @@ constexpr int kAppendWarps = kAppendThreads / 32;
 constexpr int kRing = 8;  // A rows in flight per thread
 
 struct AppendSmem {
-  size_t ring_off, xs_off, slot_off, red_off, bar_off, total;
+  size_t ring_off, xs_off, slot_off, red_off, pos_off, bar_off, total;
 };
 
 static __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ring [kRing][threads] x 16 B | rotated x (fp32) [B][Ec] | partial slots [cluster][B][r]
-// | reduction scratch [warps][4][r] | barrier
+// | reduction scratch [warps][4][r] | row positions [16] | barrier
 static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r, int cluster) {
   AppendSmem s;
   size_t o = 0;
@@ -59,6 +59,8 @@ static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r,
   o = align_up(o + (size_t)cluster * B * r * 4, 16);
   s.red_off = o;
   o = align_up(o + (size_t)kAppendWarps * 4 * r * 4, 16);
+  s.pos_off = o;
+  o += 16 * 4;
   s.bar_off = o;
   o += 8;
   s.total = align_up(o, 16);
@@ -175,7 +177,11 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   // Leader: completes when every other rank's slot values have landed
   // (transaction bytes of their st.async stores).
   uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  int* pos_sm = reinterpret_cast<int*>(smem + L.pos_off);  // leader: seq_lens[b] as read at launch
 
+  // The leader reads the row positions first so that their latency is hidden.
+  // No CTA writes seq_lens before every leader has counted itself done (below).
+  if (rank == 0 && tid < B) pos_sm[tid] = ld_relaxed_gpu(a.seq_lens + tid);
   if (tid == 0) {
     mbar_init(bar_red, 1);
     fence_mbar_init();
@@ -276,12 +282,26 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   //    (one warp per batch row; lane owns columns j = lane + 32k).
   if (a.cluster > 1) {
     if (tid == 0 && !mbar_wait_cluster_bounded(bar_red, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-    __syncthreads();
+  }
+  __syncthreads();  // slots landed; pos_sm visible
+  // 6. Completion counter, overlapping the quantisation below: this CTA's only
+  //    reads of seq_lens (at launch) are ordered before its add (acq_rel after
+  //    the CTA barrier), so the last leader may advance the lengths at once.
+  //    The row stores need no ordering with it: later kernels see both.
+  if (tid == kAppendThreads - 32) {
+    const int prev = atom_add_acq_rel_gpu(a.counter, 1);
+    if (prev == (int)gridDim.y - 1) {
+      for (int b = 0; b < B; ++b) {
+        const int pos = pos_sm[b];
+        if (pos >= 0 && pos < a.L_cap) st_relaxed_gpu(a.seq_lens + b, pos + 1);
+      }
+      st_relaxed_gpu(a.counter, 0);
+    }
   }
   const int Q = (a.bits == 8) ? 127 : 7;
   const int RB = r * a.bits / 8;
   for (int b = warp; b < B; b += kAppendWarps) {
-    const int pos = a.seq_lens[b];
+    const int pos = pos_sm[b];
     const bool ok = pos >= 0 && pos < a.L_cap;
     float cv[4];
     float amax = 0.f;
@@ -316,21 +336,6 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     if (lane == 0) {
       if (ok) (kv ? a.scale_v : a.scale_k)[row] = sh;
       else if (unit == 0) set_err(a.err, WSVD_DEVERR_CACHE_FULL);
-    }
-  }
-  __syncthreads();
-
-  // 6. The last leader to finish advances the lengths.
-  if (tid == 0) {
-    __threadfence();
-    const int prev = atomicAdd(a.counter, 1);
-    if (prev == (int)gridDim.y - 1) {
-      __threadfence();
-      for (int b = 0; b < B; ++b) {
-        const int pos = a.seq_lens[b];
-        if (pos >= 0 && pos < a.L_cap) a.seq_lens[b] = pos + 1;
-      }
-      atomicExch(a.counter, 0);
     }
   }
 }

@@ -117,7 +117,7 @@ struct Cfg {
   static_assert(TPT <= 32 && (TPT & (TPT - 1)) == 0, "a token's lanes share a warp");
   // shared-memory layout (bytes)
   static constexpr size_t kOffBar = (size_t)kStages * kStageBytes;
-  static constexpr size_t kOffQ = kOffBar + 2 * kStages * 8 + 4 * 8;  // + segment full / empty barriers
+  static constexpr size_t kOffQ = kOffBar + 2 * kStages * 8 + 6 * 8;  // + segment / auxiliary barriers
   static constexpr size_t kOffRed = kOffQ + (size_t)kW * 4;
   static constexpr size_t kOffRes = kOffRed + (size_t)kRedFloats * 4;
   static constexpr int kPlaneWords = TPT * (3 * kQW + 4);  // packed q' byte planes + corrections, per chunk
@@ -1006,18 +1006,28 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
     }
     const int bh = b_ * a.H + h_;
     float* dst = a.partials + ((size_t)c + bh) * (W + 2);
+    int* flag = reinterpret_cast<int*>(misc) + 8;
+    // The CTA that ends a head usually reaches it after the CTAs that start
+    // it: if every other contributor has already published (the counter,
+    // read with acquire, says so), this CTA is the last arriver without
+    // publishing or bumping anything itself.
+    if (tid == 0) *flag = (ld_acquire_gpu(&a.counters[bh]) == cl - cf) ? 2 : 0;
+    csync();
+    const int early = *flag;
     if (tid < W + 2) {
       for (int e = tid; e < W + 2; e += kConsumerThreads) dst[e] = res[e];
-      __threadfence();  // publish before the counter bump
+      if (!early) __threadfence();  // publish before the counter bump
     }
     csync();
-    if (tid == 0) {
-      const int prev = atomicAdd(&a.counters[bh], 1);
-      reinterpret_cast<int*>(misc)[8] = (prev == cl - cf) ? 1 : 0;
+    if (!early) {
+      if (tid == 0) {
+        const int prev = atomicAdd(&a.counters[bh], 1);
+        *flag = (prev == cl - cf) ? 1 : 0;
+      }
+      csync();
     }
-    csync();
-    if (reinterpret_cast<int*>(misc)[8]) {
-      __threadfence();
+    if (*flag) {
+      if (!early) __threadfence();
       merge_rows<W, true>(a.partials + ((size_t)cf + bh) * (W + 2), cl - cf + 1, res, tid);
       if (tid == 0) atomicExch(&a.counters[bh], 0);
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
@@ -1097,7 +1107,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + S;
   uint64_t* segfull = empty + S;
-  uint64_t* aux = segfull + 1;  // [0]: B_Vh staged (leader), [1]: slots filled (leader)
+  uint64_t* aux = segfull + 1;  // [0]: B_Vh staged (leader), [1]: slots filled (leader),
+                                // [2]: pre-staged tile count known, [3]: tile total known
   float* qs = reinterpret_cast<float*>(smem + C::kOffQ);
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
   float* res = reinterpret_cast<float*>(smem + C::kOffRes);
@@ -1120,6 +1131,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     mbar_init(segfull, 1);
     mbar_init(&aux[0], 1);
     mbar_init(&aux[1], 1);
+    mbar_init(&aux[2], 1);
+    mbar_init(&aux[3], 1);
     fence_mbar_init();
     // leader: the other ranks' partial rows arrive as st.async transaction bytes
     if (rank == 0 && csize > 1) mbar_arrive_expect_tx(&aux[1], (uint32_t)((csize - 1) * (W + 2) * 4));
@@ -1137,42 +1150,92 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   cluster_arrive_relaxed();  // barriers initialised; waited on before any remote access
   __syncthreads();           // barrier initialisation visible to every thread of this CTA
 
-  // Everything above reads only q and the B matrices.  Under a programmatic
-  // dependent launch (behind the append that writes this step's row and
-  // seq_lens) the cache and the lengths are read only after griddep_wait.
+  // Per-stage valid rows, then (after the stages) the number of tiles staged
+  // before the dependency wait and the total, for the consumers.  red[] is
+  // free until the final reduction; the producer's last write to it precedes
+  // the last tile's arrive.
+  int* tile_info = reinterpret_cast<int*>(red);
+
+  // Everything above reads only q and the B matrices.  The tiles are the fixed
+  // grid [lo + i T, lo + (i + 1) T) of this rank's rows below the length.
+  // Behind the append that writes this step's row and seq_lens (programmatic
+  // dependent launch, dep 2) the producer stages, before it waits, the rows
+  // that append cannot touch: it writes only row seq_lens[b] as it was at
+  // launch, and the value read here is that one or the advanced one, so rows
+  // below it minus one are final either way.  A tile straddling that bound is
+  // filled in two parts (its barrier completes only with the second part).
+  // The grid, and so the arithmetic, does not depend on that early read.
   if (warp == kConsumerWarps) {
-    griddep_wait();
-    const int end = min(hi, clamp_len(a.seq_lens[b], a.L_cap));
-    const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
     if (lane == 0) {
+      using CT = typename C::CT;
       const uint64_t pol = l2_evict_first_policy();
       bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
+      // rows [r0 + off, r0 + off + n) of the tile at r0 into stage st, completing on bar
+      auto copy_rows = [&](uint8_t* st, int r0, int off, int n, uint64_t* bar) {
+        const int rr = r0 + off;
+        const size_t head_row = ((size_t)b * a.H + h) * a.L_cap + rr;
+        const size_t row0 = a.heads_share ? (size_t)b * a.L_cap + rr : head_row;
+        const uint32_t cbytes = (uint32_t)n * C::kRB;
+        const uint32_t sbytes = CT::kScaled ? (uint32_t)((n + 7) & ~7) * 2u : 0u;
+        bulk_g2s(st + (size_t)off * C::kRB, a.lat_k + row0 * C::kRB, cbytes, bar, pol);
+        bulk_g2s(st + C::kCodeBytes + (size_t)off * C::kRB, a.lat_v + row0 * C::kRB, cbytes, bar, pol);
+        if (CT::kScaled) {
+          bulk_g2s(st + 2 * C::kCodeBytes + off * 2, a.scale_k + head_row, sbytes, bar, pol);
+          bulk_g2s(st + 2 * C::kCodeBytes + C::kScaleBytes + off * 2, a.scale_v + head_row, sbytes, bar, pol);
+        }
+      };
+      auto tile_bytes = [&](int n) {
+        return 2u * (uint32_t)n * C::kRB + (CT::kScaled ? 4u * (uint32_t)((n + 7) & ~7) : 0u);
+      };
+      auto claim = [&](int i) {  // stage of tile i, free for reuse
         const int s = i % S;
         if (i >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / S) - 1) & 1))) {
           set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
           ok = false;
-          break;
         }
-        // tiles are counted from lo; issue_tile counts rows from (b, h) row 0, so
-        // pass the token offset through t with tiles of T tokens: lo is a multiple of 8,
-        // not of T, so address rows directly.
-        const int r0 = lo + i * T, n = min(T, end - r0);
-        const size_t head_row = ((size_t)b * a.H + h) * a.L_cap + r0;
-        const size_t row0 = a.heads_share ? (size_t)b * a.L_cap + r0 : head_row;
-        using CT = typename C::CT;
-        uint8_t* st = stages + (size_t)s * C::kStageBytes;
-        const uint32_t cbytes = (uint32_t)n * C::kRB;
-        const uint32_t sbytes = CT::kScaled ? (uint32_t)((n + 7) & ~7) * 2u : 0u;
-        mbar_arrive_expect_tx(&full[s], 2 * cbytes + 2 * sbytes);
-        bulk_g2s(st, a.lat_k + row0 * C::kRB, cbytes, &full[s], pol);
-        bulk_g2s(st + C::kCodeBytes, a.lat_v + row0 * C::kRB, cbytes, &full[s], pol);
-        if (CT::kScaled) {
-          bulk_g2s(st + 2 * C::kCodeBytes, a.scale_k + head_row, sbytes, &full[s], pol);
-          bulk_g2s(st + 2 * C::kCodeBytes + C::kScaleBytes, a.scale_v + head_row, sbytes, &full[s], pol);
+        return s;
+      };
+      int pre_end = lo;
+      if (a.dep == 2) {
+        const int v = clamp_len(ld_relaxed_gpu(a.seq_lens + b), a.L_cap);
+        pre_end = max(lo, min(hi, v - 1) & ~7);
+      }
+      const int npre = (pre_end - lo) / T, part = (pre_end - lo) % T;  // whole tiles below the bound, rows of the next
+      tile_info[S] = npre;
+      mbar_arrive(&aux[2]);
+      for (int i = 0; i < npre && ok; ++i) {
+        const int s = claim(i);
+        if (!ok) break;
+        tile_info[s] = T;
+        mbar_arrive_expect_tx(&full[s], tile_bytes(T));
+        copy_rows(stages + (size_t)s * C::kStageBytes, lo + i * T, 0, T, &full[s]);
+      }
+      if (ok && part > 0) {
+        const int s = claim(npre);
+        if (ok) {
+          mbar_expect_tx(&full[s], tile_bytes(part));  // no arrive yet: the rest follows after the wait
+          copy_rows(stages + (size_t)s * C::kStageBytes, lo + npre * T, 0, part, &full[s]);
         }
       }
-      for (int i = (ntiles > S ? ntiles - S : 0); i < ntiles && ok; ++i)
+      griddep_wait();
+      const int raw = a.seq_lens[b];
+      if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+      const int end = max(pre_end, min(hi, clamp_len(raw, a.L_cap)));  // pre_end <= end holds by construction
+      const int total = end > lo ? (end - lo + T - 1) / T : 0;         // > npre whenever part > 0
+      tile_info[S + 1] = total;
+      mbar_arrive(&aux[3]);
+      for (int i = npre; i < total && ok; ++i) {
+        const int r0 = lo + i * T, n = min(T, end - r0);
+        const bool split = (i == npre && part > 0);
+        const int s = split ? i % S : claim(i);  // a split tile's stage was claimed before the wait
+        if (!ok) break;
+        tile_info[s] = n;
+        const int off = split ? part : 0;
+        mbar_arrive_expect_tx(&full[s], n > off ? tile_bytes(n) - tile_bytes(off) : 0u);
+        if (n > off) copy_rows(stages + (size_t)s * C::kStageBytes, r0, off, n - off, &full[s]);
+      }
+      const int issued = ok ? total : 0;
+      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
         if (!mbar_wait_bounded(&full[i % S], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
@@ -1181,7 +1244,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     return;
   }
 
-  // consumers
+  // consumers: every staged tile reaches them through the producer, which
+  // waits on the preceding grid before staging anything that grid may write.
   const int sub = tid % TPT;
   QState<CODEC, VPT> qst;
   float2 acc[NP];
@@ -1189,27 +1253,34 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
   float m = kNegInf, l = 0.f;
   bool timed_out = false;
-  if (!mbar_wait_bounded(segfull, 0)) {
-    if (lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-    timed_out = true;
-  }
-  build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, planes, a, tid, sub);
-  griddep_wait();
-  const int raw = a.seq_lens[b];
-  if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0 && tid == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
-  const int end = min(hi, clamp_len(raw, a.L_cap));
-  const int ntiles = end > lo ? (end - lo + T - 1) / T : 0;
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i % S;
-    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / S) & 1), timed_out ? 0ull : kWaitLimitNs)) {
+  auto cwait = [&](uint64_t* bar, uint32_t parity) {
+    if (!mbar_wait_bounded(bar, parity, timed_out ? 0ull : kWaitLimitNs)) {
       if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       timed_out = true;
     }
-    process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, end - lo - i * T), qst, m, l,
-                                        acc, tid);
+  };
+  cwait(segfull, 0);
+  build_query<CODEC, VPT, W, QMODE>(qst, segbuf, qs, misc, planes, a, tid, sub);
+  const int max_tiles = (hi - lo + T - 1) / T;
+  cwait(&aux[2], 0);
+  const int npre = timed_out ? 0 : min(tile_info[S], max_tiles);
+  int total = -1;
+  for (int i = 0; i < max_tiles; ++i) {
+    if (i >= npre) {
+      if (total < 0) {
+        cwait(&aux[3], 0);
+        total = timed_out ? 0 : min(tile_info[S + 1], max_tiles);
+      }
+      if (i >= total) break;
+    }
+    const int s = i % S;
+    cwait(&full[s], (uint32_t)((i / S) & 1));
+    if (timed_out) break;
+    process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, tile_info[s], qst, m, l, acc, tid);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
+  csync();  // every consumer has read its last tile_info before red[] is reused
   reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
 
   cluster_wait();  // every CTA of the cluster has initialised its barriers
