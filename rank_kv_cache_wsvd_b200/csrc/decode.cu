@@ -145,6 +145,21 @@ template <int VPT>
 struct QState<kCodecI8, VPT> {
   uint32_t qh[VPT / 4], qm[VPT / 4], ql[VPT / 4];  // signed high byte, unsigned middle / low bytes
   float step;
+  // Lanes that read their chunk's two 16-byte halves in swapped order (see
+  // load_chunk) hold their plane words in that order too.
+  __device__ __forceinline__ void swap_halves(bool sw) {
+    constexpr int H = VPT / 8;
+#pragma unroll
+    for (int k = 0; k < H; ++k) {
+      const uint32_t h0 = qh[k], m0 = qm[k], l0 = ql[k];
+      qh[k] = sw ? qh[k + H] : h0;
+      qh[k + H] = sw ? h0 : qh[k + H];
+      qm[k] = sw ? qm[k + H] : m0;
+      qm[k + H] = sw ? m0 : qm[k + H];
+      ql[k] = sw ? ql[k + H] : l0;
+      ql[k + H] = sw ? l0 : ql[k + H];
+    }
+  }
   __device__ __forceinline__ float dot(const uint4* seg) const {
     int ah[2] = {0, 0}, am[2] = {0, 0}, al[2] = {0, 0};  // two chains per plane
 #pragma unroll
@@ -164,6 +179,7 @@ struct QState<kCodecI4, VPT> {
   uint32_t qh[VPT / 4], qm[VPT / 4], ql[VPT / 4];
   int ch, cm, cl;  // 8 * sum of each plane: removes the +8 offset of the nibbles
   float step;
+  __device__ __forceinline__ void swap_halves(bool) {}
   __device__ __forceinline__ float dot(const uint4* seg) const {
     int ah[2] = {-ch, 0}, am[2] = {-cm, 0}, al[2] = {-cl, 0};  // even / odd elements on separate chains
 #pragma unroll
@@ -186,6 +202,15 @@ template <int VPT>
 struct QState<kCodecF16, VPT> {
   float2 qv[VPT / 2];
   float step;
+  __device__ __forceinline__ void swap_halves(bool sw) {
+    constexpr int H = VPT / 4;
+#pragma unroll
+    for (int k = 0; k < H; ++k) {
+      const float2 t = qv[k];
+      qv[k] = sw ? qv[k + H] : t;
+      qv[k + H] = sw ? t : qv[k + H];
+    }
+  }
   __device__ __forceinline__ float dot(const uint4* seg) const {
     float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -278,15 +303,19 @@ __device__ __forceinline__ int cta_of(long long g, long long G, int C) {
 // A lane's chunk of a token row from shared memory.  With two 16-byte halves,
 // lanes 4-7 of each 8-lane phase take the halves in the other order, so the
 // phase touches 32 distinct banks.
+__device__ __forceinline__ bool swapped_lane(int lane) { return (lane >> 2) & 1; }
+
 template <int NSEG>
 __device__ __forceinline__ void load_chunk(uint4* seg, const uint8_t* p, int lane) {
   const uint32_t a = smem_u32(p);
   if constexpr (NSEG == 2) {
-    const bool swap = (lane >> 2) & 1;
-    const uint4 x = lds128(a + (swap ? 16u : 0u));
-    const uint4 y = lds128(a + (swap ? 0u : 16u));
-    seg[0] = swap ? y : x;
-    seg[1] = swap ? x : y;
+    // Lanes 4-7 of every eight read the second half first (rows of 32 bytes
+    // would otherwise put two lanes of a quarter-warp on the same banks).
+    // The halves stay in that order: those lanes keep their query state and
+    // accumulators permuted to match (swap_halves, reduce_to_res).
+    const uint32_t off = swapped_lane(lane) ? 16u : 0u;
+    seg[0] = lds128(a + off);
+    seg[1] = lds128(a + (off ^ 16u));
   } else {
 #pragma unroll
     for (int j = 0; j < NSEG; ++j) seg[j] = lds128(a + 16u * j);
@@ -415,6 +444,7 @@ __device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8
     for (int p = 0; p < VPT / 2; ++p) qst.qv[p] = make_float2(qs[sub * VPT + 2 * p], qs[sub * VPT + 2 * p + 1]);
     qst.step = 1.f;
   }
+  if constexpr (Cfg<CODEC, VPT, W / VPT, 1>::kNSeg == 2) qst.swap_halves(swapped_lane(tid & 31));
 }
 
 // One staged tile with n valid tokens: scores, lazy-rescaled online softmax and
@@ -499,7 +529,7 @@ __device__ __forceinline__ int scatter_base(int lane) {
 // Merges every consumer lane's (m, l, acc) into res[] = (M, L, O[W]): a common
 // maximum per chunk, a butterfly reduce-scatter inside each warp, then the
 // eight warps through red[] (8*W floats of warp partials, then (M, l) pairs).
-template <int VPT, int TPT, int W>
+template <int VPT, int TPT, int W, int NSEG>
 __device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, float* red, float* res, int tid) {
   constexpr int NP = VPT / 2;
   constexpr int FINAL = (VPT * TPT >= 32) ? VPT * TPT / 32 : 1;
@@ -512,10 +542,12 @@ __device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, flo
 #pragma unroll
   for (int o = TPT; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   float v[VPT];
+  const bool sw = NSEG == 2 && swapped_lane(lane);  // accumulators of a swapped lane hold the halves permuted
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
-    v[2 * p] = acc[p].x * f;
-    v[2 * p + 1] = acc[p].y * f;
+    const float2 x = (NSEG == 2 && sw) ? acc[p ^ (NP / 2)] : acc[p];
+    v[2 * p] = x.x * f;
+    v[2 * p + 1] = x.y * f;
   }
   reduce_scatter<VPT, 16, TPT>(v, lane);
   const int base = sub * VPT + scatter_base<VPT, 16, TPT>(lane);
@@ -986,7 +1018,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   auto end_segment = [&](int j) {  // hand segment j to the helper
     const int sr = j & 1;
     if (j >= 2) wait(&resfree[sr], (uint32_t)(((j / 2) - 1) & 1));
-    reduce_to_res<VPT, TPT, W>(m, l, acc, red, ha->res[sr], tid);
+    reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, ha->res[sr], tid);
     if (tid == 0) mbar_arrive(&resfull[sr]);
   };
   // The CTA's last segment: every consumer thread finishes it (partial, counter,
@@ -994,7 +1026,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   float* res = reinterpret_cast<float*>(smem + C::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
   auto finish_last = [&](int b_, int h_) {
-    reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
+    reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
     const int tb = walk.tiles(b_);
     const long long gf = (long long)a.H * pre[b_] + (long long)h_ * tb;
     const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
@@ -1062,6 +1094,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
         for (int p = 0; p < NP; ++p)
           qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
       }
+      if constexpr (C::kNSeg == 2) qst.swap_halves(swapped_lane(lane));
       __syncwarp();
       if (lane == 0) mbar_arrive(&qfree[sq]);
 #pragma unroll
@@ -1281,7 +1314,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     if (lane == 0) mbar_arrive(&empty[s]);
   }
   csync();  // every consumer has read its last tile_info before red[] is reused
-  reduce_to_res<VPT, TPT, W>(m, l, acc, red, res, tid);
+  reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
 
   cluster_wait();  // every CTA of the cluster has initialised its barriers
   if (rank != 0) {
