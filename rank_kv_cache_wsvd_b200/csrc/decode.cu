@@ -126,8 +126,14 @@ struct Cfg {
   static constexpr size_t kOffPre = kOffMisc + 16 * 4;
   // runtime part: lens / prefix (2B + 1 ints), then the segment buffers
   __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(2 * B + 1) * 4 + 127) / 128 * 128; }
+  // B_Vh of the CTA's last segment, staged for its finish (low-rank codecs, up
+  // to 16 KB so that two CTAs still fit an SM; larger ones read global memory).
+  __host__ __device__ static size_t bv_stage_bytes(int Hd) {
+    return (CT::kScaled && (size_t)kW * Hd * 2 <= 16384) ? (size_t)kW * Hd * 2 : 0;
+  }
   static size_t smem_bytes(int B, int qmode, int Hd) {
-    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) + sizeof(HelperArea<kW, kPlaneWords, kNQ>);
+    return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) +
+           (sizeof(HelperArea<kW, kPlaneWords, kNQ>) + 127) / 128 * 128 + bv_stage_bytes(Hd);
   }
   // cluster kernel: operands, the leader's partial slots, then B_Vh
   __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
@@ -787,6 +793,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   const int NBUF = seg_nbuf(QMODE, W, a.Hd);
   const uint32_t SEGB = (uint32_t)seg_bytes(QMODE, W, a.Hd);
   HA* ha = reinterpret_cast<HA*>(segbuf + (size_t)NBUF * SEGB);
+  __half* bv_last = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(ha) + (sizeof(HA) + 127) / 128 * 128);
+  uint64_t* bvbar = segempty + 2;  // B_Vh of the last segment staged
   uint64_t* qready = ha->bars;
   uint64_t* qfree = ha->bars + NQ;
   uint64_t* resfull = ha->bars + 2 * NQ;
@@ -835,6 +843,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
         mbar_init(&resfull[s], 1);
         mbar_init(&resfree[s], 1);
       }
+      mbar_init(bvbar, 1);
       for (int s = 0; s < NQ; ++s) {
         mbar_init(&qready[s], 1);
         mbar_init(&qfree[s], kConsumerWarps);
@@ -890,7 +899,21 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
                                           min(T, lens[b] - t * T), pol);
         walk.advance(b, h, t);
       }
+      // B_Vh of the CTA's last segment, for the consumers' finish (issued after
+      // the tiles so that it does not compete with the first ones).
+      const bool stage_bv = C::bv_stage_bytes(a.Hd) > 0 && a.Bv != nullptr;
+      if (stage_bv) {
+        int lb, lh, lt;
+        walk.locate(g_end - 1, lb, lh, lt);
+        const uint32_t bytes = (uint32_t)W * a.Hd * 2;
+        mbar_arrive_expect_tx(bvbar, bytes);
+        for (uint32_t off = 0; off < bytes; off += 32768)
+          bulk_g2s(reinterpret_cast<uint8_t*>(bv_last) + off,
+                   reinterpret_cast<const uint8_t*>(a.Bv + (size_t)lh * W * a.Hd) + off, min(32768u, bytes - off),
+                   bvbar, keep);
+      }
       // Leave no copy in flight behind: wait (bounded) for the last uses of each buffer.
+      if (stage_bv && !mbar_wait_bounded(bvbar, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       for (long long i = (issued > S ? issued - S : 0); i < issued && ok; ++i)
         if (!mbar_wait_bounded(&full[(int)(i % S)], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       for (int k = (nseg > NBUF ? nseg - NBUF : 0); k < nseg && ok; ++k)
@@ -1026,24 +1049,35 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   float* res = reinterpret_cast<float*>(smem + C::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
   auto finish_last = [&](int b_, int h_) {
-    reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
     const int tb = walk.tiles(b_);
     const long long gf = (long long)a.H * pre[b_] + (long long)h_ * tb;
     const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
+    const int bh = b_ * a.H + h_;
+    // The CTA that ends a head usually reaches it after the CTAs that start
+    // it: if every other contributor has already published (the counter,
+    // read with acquire, says so), this CTA is the last arriver without
+    // publishing or bumping anything itself.  The read is issued before the
+    // reduction so that its latency overlaps it (an early, lower count only
+    // sends this CTA down the publishing path).
+    const int seen = (cf != cl && tid == 0) ? ld_acquire_gpu(&a.counters[bh]) : 0;
+    reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
     float* outp = a.out + ((size_t)b_ * a.H + h_) * a.Hd;
-    const __half* Bvh = a.Bv ? a.Bv + (size_t)h_ * W * a.Hd : nullptr;
+    const __half* Bvh = nullptr;
+    if (a.Bv != nullptr) {
+      if (C::bv_stage_bytes(a.Hd) > 0) {  // staged by the producer
+        wait(bvbar, 0);
+        Bvh = bv_last;
+      } else {
+        Bvh = a.Bv + (size_t)h_ * W * a.Hd;
+      }
+    }
     if (cf == cl) {
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
       return;
     }
-    const int bh = b_ * a.H + h_;
     float* dst = a.partials + ((size_t)c + bh) * (W + 2);
     int* flag = reinterpret_cast<int*>(misc) + 8;
-    // The CTA that ends a head usually reaches it after the CTAs that start
-    // it: if every other contributor has already published (the counter,
-    // read with acquire, says so), this CTA is the last arriver without
-    // publishing or bumping anything itself.
-    if (tid == 0) *flag = (ld_acquire_gpu(&a.counters[bh]) == cl - cf) ? 2 : 0;
+    if (tid == 0) *flag = (seen == cl - cf) ? 2 : 0;
     csync();
     const int early = *flag;
     if (tid < W + 2) {

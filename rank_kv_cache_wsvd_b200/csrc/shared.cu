@@ -7,22 +7,23 @@
 
 namespace wsvd {
 
+// Block (bh, y) computes q' elements j = 8 y + warp of one (b, h), each as a
+// full-warp reduction of B_Kh[j, :] . q: every block lives about one memory
+// round trip, so a decode launched behind this kernel is not kept from its SMs.
 __global__ void __launch_bounds__(256) qproj_kernel(int H, int Hd, int R, const void* q, int q_dtype,
                                                     const __half* Bk, float* qglobal) {
   // A decode launched behind this kernel may start now; it waits for q'.
   griddep_launch_dependents();
   const int bh = blockIdx.x, h = bh % H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float qr[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    qr[k] = (lane + 32 * k < Hd) ? load_q_elem(q, q_dtype, (size_t)bh * Hd + lane + 32 * k) : 0.f;
-  const __half* Bh = Bk + (size_t)h * R * Hd;
-  for (int j = warp; j < R; j += 8) {
+  const int j = blockIdx.y * 8 + warp;
+  if (j < R) {
+    const __half* Bj = Bk + ((size_t)h * R + j) * Hd;
     float d = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      if (lane + 32 * k < Hd) d = fmaf(__half2float(Bh[(size_t)j * Hd + lane + 32 * k]), qr[k], d);
+      if (lane + 32 * k < Hd)
+        d = fmaf(__half2float(Bj[lane + 32 * k]), load_q_elem(q, q_dtype, (size_t)bh * Hd + lane + 32 * k), d);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
     if (lane == 0) qglobal[(size_t)bh * R + j] = d;
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(256) qproj_kernel(int H, int Hd, int R, const 
 cudaError_t launch_qproj(int B, int H, int Hd, int W, const void* q, int q_dtype, const __half* Bk, float* qglobal,
                          cudaStream_t stream, bool after_append) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(B * H);
+  cfg.gridDim = dim3(B * H, (W + 7) / 8);
   cfg.blockDim = dim3(256);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
