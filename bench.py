@@ -129,27 +129,28 @@ def attended_tokens(w: WL.Workload, lens_after: np.ndarray) -> int:
     return int(lens_after.sum()) * w.H
 
 
-def alg_bytes_decode(w: WL.Workload, lens: np.ndarray) -> int:
+def alg_bytes_decode(w: WL.Workload, lens: np.ndarray, w8: bool = False) -> int:
     rb = w.r * w.bits // 8
     codes = int(lens.sum()) * w.H * 2 * (rb + 2)
-    weights = 2 * w.H * w.r * w.Hd * 2
+    weights = 2 * w.H * (w.r * w.Hd + w.Hd * 4) if w8 else 2 * w.H * w.r * w.Hd * 2  # B_K, B_V (+ column scales)
     io = w.B * w.H * w.Hd * (2 + 4)
     return codes + weights + io
 
 
-def alg_bytes_append(w: WL.Workload) -> int:
+def alg_bytes_append(w: WL.Workload, w8: bool = False) -> int:
     rb = w.r * w.bits // 8
-    return 2 * w.H * w.E * w.r * 2 + w.B * w.E * 2 + w.B * w.H * 2 * (rb + 2) + w.B * 4 * 2
+    weights = 2 * w.H * (w.E * w.r + w.r * 4) if w8 else 2 * w.H * w.E * w.r * 2  # A_K, A_V (+ column scales)
+    return weights + w.B * w.E * 2 + w.B * w.H * 2 * (rb + 2) + w.B * 4 * 2
 
 
 class WsvdStep:
     """Device-resident inputs of one workload and the launches of one step."""
 
-    def __init__(self, w: WL.Workload, seed: int = 0):
+    def __init__(self, w: WL.Workload, seed: int = 0, w8: bool = False):
         import torch
 
         import rank_kv_cache_wsvd_b200 as W
-        self.W, self.torch, self.w = W, torch, w
+        self.W, self.torch, self.w, self.w8 = W, torch, w, w8
         self.has_append = w.append_steps > 0
         lens_full = WL.seq_lens(w, seed)
         lens0 = lens_full - 1 if self.has_append else lens_full
@@ -167,6 +168,10 @@ class WsvdStep:
         self.lat_k, self.lat_v = cu(d.lat_k), cu(d.lat_v)
         self.scale_k, self.scale_v = cu(d.scale_k), cu(d.scale_v)
         self.B_k, self.B_v = cu(d.Bk), cu(d.Bv)
+        if w8:  # int8 weights, one fp32 scale per output column
+            bkq, sbk = WL.quantize_weights_w8(d.Bk)
+            bvq, sbv = WL.quantize_weights_w8(d.Bv)
+            self.B_k, self.B_v, self.sB_k, self.sB_v = cu(bkq), cu(bvq), cu(sbk), cu(sbv)
         self.lens0 = cu(lens0.astype(np.int32))
         self.lens = self.lens0.clone()
         self.lens_after = lens_full.astype(np.int64)
@@ -177,6 +182,10 @@ class WsvdStep:
             ai = WL.append_inputs(w, seed=seed, steps=1)
             self.x = cu(ai.x_bits[0].view(np.int16)).view(torch.bfloat16)
             self.A_k, self.A_v = cu(ai.A_k), cu(ai.A_v)
+            if w8:
+                akq, sak = WL.quantize_weights_w8(ai.A_k)
+                avq, sav = WL.quantize_weights_w8(ai.A_v)
+                self.A_k, self.A_v, self.sA_k, self.sA_v = cu(akq), cu(avq), cu(sak), cu(sav)
             self.ws_app = W.workspace(W.wsvd_append_workspace_size())
             self.x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
         self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
@@ -189,20 +198,40 @@ class WsvdStep:
         self.lens.copy_(self.lens0)
 
     def append(self):
-        if self.has_append:
+        if not self.has_append:
+            return
+        if self.w8:
+            self.W.wsvd_latent_append_w8(self.x, self.A_k, self.A_v, self.sA_k, self.sA_v, self.lens, self.lat_k,
+                                         self.lat_v, self.scale_k, self.scale_v, bits=self.w.bits,
+                                         hadamard_block=self.w.hadamard_block, workspace_buf=self.ws_app,
+                                         err=self.err)
+        else:
             self.W.wsvd_latent_append(self.x, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v, self.scale_k,
                                       self.scale_v, bits=self.w.bits, hadamard_block=self.w.hadamard_block,
                                       workspace_buf=self.ws_app, err=self.err)
 
     def decode(self):
-        self.W.wsvd_decode_attention(self.q, self.lat_k, self.lat_v, self.scale_k, self.scale_v, self.B_k, self.B_v,
-                                     self.lens, bits=self.w.bits, out=self.out, workspace_buf=self.ws, err=self.err)
+        if self.w8:
+            self.W.wsvd_decode_attention_w8(self.q, self.lat_k, self.lat_v, self.scale_k, self.scale_v, self.B_k,
+                                            self.B_v, self.sB_k, self.sB_v, self.lens, bits=self.w.bits,
+                                            out=self.out, workspace_buf=self.ws, err=self.err)
+        else:
+            self.W.wsvd_decode_attention(self.q, self.lat_k, self.lat_v, self.scale_k, self.scale_v, self.B_k,
+                                         self.B_v, self.lens, bits=self.w.bits, out=self.out, workspace_buf=self.ws,
+                                         err=self.err)
 
     def step(self):
         """One step through the public API: the one-call append + decode when
         the workload appends, else the decode."""
         if not self.has_append:
             self.decode()
+            return
+        if self.w8:
+            self.W.wsvd_append_and_decode_w8(self.x, self.A_k, self.A_v, self.sA_k, self.sA_v, self.lens, self.lat_k,
+                                             self.lat_v, self.scale_k, self.scale_v, self.q, self.B_k, self.B_v,
+                                             self.sB_k, self.sB_v, bits=self.w.bits,
+                                             hadamard_block=self.w.hadamard_block, out=self.out,
+                                             append_ws=self.ws_app, decode_ws=self.ws, err=self.err)
             return
         self.W.wsvd_append_and_decode(self.x, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v, self.scale_k,
                                       self.scale_v, self.q, self.B_k, self.B_v, bits=self.w.bits,
@@ -339,6 +368,8 @@ def main():
     ap.add_argument("--workload", default="llava7b", choices=sorted(WL.PRESETS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-extras", action="store_true", help="skip the CPU baseline, e2e and comparison timings")
+    ap.add_argument("--weights", default="fp16", choices=["fp16", "int8"],
+                    help="low-rank factors A, B as fp16, or int8 with per-column scales (W8)")
     args = ap.parse_args()
     w = WL.PRESETS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -379,7 +410,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    st = WsvdStep(w, seed=rank)
+    w8 = args.weights == "int8"
+    st = WsvdStep(w, seed=rank, w8=w8)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
     for _ in range(3):  # first calls (library load, per-device setup) outside everything timed
@@ -467,8 +499,8 @@ def main():
 
     ms_per_step = t_total / args.steps * 1e3
     peak, peak_kind = peaks()
-    dec_bytes = alg_bytes_decode(w, st.lens_after)
-    app_bytes = alg_bytes_append(w) if st.has_append else 0
+    dec_bytes = alg_bytes_decode(w, st.lens_after, w8)
+    app_bytes = alg_bytes_append(w, w8) if st.has_append else 0
     per_app = t_app / args.steps
     per_dec = t_dec / args.steps
     if st.has_append and per_app >= per_dec:
@@ -477,7 +509,7 @@ def main():
         dom, nbytes, dur, launches = "decode", dec_bytes, per_dec, \
             "wsvd decode (1 launch: split-L + last-arriver combine)"
     achieved = nbytes / dur / 1e9
-    traffic = ncu_traffic(dom, args.workload)
+    traffic = ncu_traffic(dom, args.workload + ("_w8" if w8 else ""))
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -508,7 +540,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "Hd": w.Hd, "r": w.r,
-                       "latent_bits": w.bits, "attended_tokens_per_seq": [int(x) for x in st.lens_after],
+                       "latent_bits": w.bits, "weights": args.weights,
+                       "attended_tokens_per_seq": [int(x) for x in st.lens_after],
                        "step": ("append + decode" if st.has_append else "decode"),
                        "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
                        "launch": ("one wsvd_append_and_decode call per step (decode launched behind the "

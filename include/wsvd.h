@@ -213,6 +213,36 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
                            void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
                            size_t decode_workspace_bytes, int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- int8 weights (W8)
+ * The same three operations with the low-rank factors stored as int8 weights
+ * (the "W8" of the method's W8A8 / W8A4 configurations, German §2.C): every
+ * weight matrix has one fp32 scale per output column,
+ *   A_h[e][j] = A_k[h][e][j] * sA_k[h][j]   (A_k, A_v  [H][E][r] int8, sA_* [H][r]  fp32),
+ *   B_h[j][d] = B_k[h][j][d] * sB_k[h][d]   (B_k, B_v  [H][r][Hd] int8, sB_* [H][Hd] fp32),
+ * and the results are those of the fp16 entry points given those dequantised
+ * weights (the kernels fold each scale in once: into q for B_k, after the
+ * column sums for A and B_v).  The pages fix no granularity for the weight
+ * scales; per output column is this library's reading.  Int8 matrices must be
+ * 16-byte aligned; scales are read with plain loads.  Every other argument,
+ * the workspace contracts and the status codes are those of the fp16 entry
+ * points. */
+int wsvd_decode_attention_w8(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                             const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
+                             const void* scale_k, const void* scale_v, const int8_t* B_k, const int8_t* B_v,
+                             const float* sB_k, const float* sB_v, float softmax_scale, float* out, void* workspace,
+                             size_t workspace_bytes, int32_t* err, void* stream);
+int wsvd_latent_append_w8(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x,
+                          int x_dtype, const int8_t* A_k, const int8_t* A_v, const float* sA_k, const float* sA_v,
+                          int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                          void* workspace, size_t workspace_bytes, int32_t* err, void* stream);
+int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                              const void* x, int x_dtype, const int8_t* A_k, const int8_t* A_v, const float* sA_k,
+                              const float* sA_v, int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k,
+                              void* scale_v, const void* q, int q_dtype, const int8_t* B_k, const int8_t* B_v,
+                              const float* sB_k, const float* sB_v, float softmax_scale, float* out,
+                              void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
+                              size_t decode_workspace_bytes, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------- comparison: dense decode
  * The flash-decoding baseline the pages compare against (German §4
  * "Ergebnisse"): out[b,h] = softmax(K[b,h,:n] . q[b,h] * softmax_scale) . V[b,h,:n]

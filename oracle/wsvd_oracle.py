@@ -266,6 +266,18 @@ def latent_append(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r: int,
 
 
 # ----------------------------------------------------------------------------- footprint
+# ----------------------------------------------------------------------------- int8 weights
+def dequantize_weights(wq: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Int8 weight matrices wq [H][K][N] with one scale per output column,
+    scale [H][N]: W[h][k][n] = wq[h][k][n] * scale[h][n] (float64).
+
+    The "W8" of the method's W8A8 / W8A4 configurations (de §2.C): the low-rank
+    factors A_h (E x r, output columns r) and B_h (r x Hd, output columns Hd)
+    stored as 8-bit weights.  The pages fix no scale granularity; one scale per
+    output column is the reading taken here."""
+    return np.asarray(wq, np.float64) * np.asarray(scale, np.float64)[:, None, :]
+
+
 def wsvd_cache_bytes(B: int, H: int, L_cap: int, r: int, bits: int) -> int:
     """Per-head latent cache: K and V codes (L x r each, bits per code) plus one
     fp16 scale per token per head for each (ar §2.a: footprint L x r per head)."""

@@ -41,6 +41,11 @@ SIGNATURES = {
     "wsvd_latent_append": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 7 + [_p, _c_size, _p, _p]),
     "wsvd_append_and_decode": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
+    "wsvd_decode_attention_w8": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 8 + [_c_float, _p, _p, _c_size,
+                                                                                           _p, _p]),
+    "wsvd_latent_append_w8": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 9 + [_p, _c_size, _p, _p]),
+    "wsvd_append_and_decode_w8": (_c_int, [_c_int] * 8 + [_p, _c_int] + [_p] * 9 + [_p, _c_int] + [_p] * 4
+                                  + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
     "dense_decode_attention": (_c_int, [_c_int] * 4 + [_p, _p, _c_int, _p, _p, _c_float, _p, _p, _c_size, _p, _p]),
     "shared_latent_svd_decode": (_c_int, [_c_int] * 5 + [_p, _p, _c_int] + [_p] * 4 + [_c_float, _p, _p, _c_size,
                                                                                          _p, _p]),
@@ -248,6 +253,98 @@ def wsvd_append_and_decode(x, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v
                                     float(softmax_scale), _ptr(out), _ptr(append_ws), append_ws.numel(),
                                     _ptr(decode_ws), decode_ws.numel(), _ptr(err), _stream(stream))
     _check(st, "wsvd_append_and_decode")
+    return out
+
+
+# ----------------------------------------------------------------------------- int8 weights
+def _w8(t, s, shape_t, shape_s, name):
+    _expect(t, torch.int8, shape_t, name)
+    _expect(s, torch.float32, shape_s, "scales of " + name)
+
+
+def wsvd_decode_attention_w8(q, lat_k, lat_v, scale_k, scale_v, B_k, B_v, sB_k, sB_v, seq_lens, bits: int,
+                             softmax_scale: float = 0.0, out=None, workspace_buf=None, err=None, stream=None):
+    """Decode with int8 B_k, B_v [H][r][Hd] and per-column fp32 scales [H][Hd]."""
+    lib = load()
+    B, H, Hd = q.shape
+    L_cap, rb = lat_k.shape[2], lat_k.shape[3]
+    r = rb * 8 // bits
+    _expect(lat_k, torch.uint8, (B, H, L_cap, rb), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, rb), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _w8(B_k, sB_k, (H, r, Hd), (H, Hd), "B_k")
+    _w8(B_v, sB_v, (H, r, Hd), (H, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, H, Hd), "out")
+    if workspace_buf is None:
+        workspace_buf = workspace(lib.wsvd_decode_workspace_size(B, H, r), q.device)
+    st = lib.wsvd_decode_attention_w8(B, H, Hd, r, bits, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q),
+                                      _ptr(lat_k), _ptr(lat_v), _ptr(scale_k), _ptr(scale_v), _ptr(B_k), _ptr(B_v),
+                                      _ptr(sB_k), _ptr(sB_v), float(softmax_scale), _ptr(out), _ptr(workspace_buf),
+                                      workspace_buf.numel(), _ptr(err), _stream(stream))
+    _check(st, "wsvd_decode_attention_w8")
+    return out
+
+
+def wsvd_latent_append_w8(x, A_k, A_v, sA_k, sA_v, seq_lens, lat_k, lat_v, scale_k, scale_v, bits: int,
+                          hadamard_block: int = 128, workspace_buf=None, err=None, stream=None) -> None:
+    """Append with int8 A_k, A_v [H][E][r] and per-column fp32 scales [H][r]."""
+    lib = load()
+    B, E = x.shape
+    H, _, r = A_k.shape
+    L_cap = lat_k.shape[2]
+    _w8(A_k, sA_k, (H, E, r), (H, r), "A_k")
+    _w8(A_v, sA_v, (H, E, r), (H, r), "A_v")
+    _expect(lat_k, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if workspace_buf is None:
+        workspace_buf = workspace(lib.wsvd_append_workspace_size(), x.device)
+    st = lib.wsvd_latent_append_w8(B, H, E, r, bits, L_cap, hadamard_block, _ptr(x), _dtype_code(x), _ptr(A_k),
+                                   _ptr(A_v), _ptr(sA_k), _ptr(sA_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v),
+                                   _ptr(scale_k), _ptr(scale_v), _ptr(workspace_buf), workspace_buf.numel(),
+                                   _ptr(err), _stream(stream))
+    _check(st, "wsvd_latent_append_w8")
+
+
+def wsvd_append_and_decode_w8(x, A_k, A_v, sA_k, sA_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q, B_k, B_v,
+                              sB_k, sB_v, bits: int, hadamard_block: int = 128, softmax_scale: float = 0.0,
+                              out=None, append_ws=None, decode_ws=None, err=None, stream=None):
+    """wsvd_append_and_decode with int8 weights (A: [H][E][r] + [H][r] scales;
+    B: [H][r][Hd] + [H][Hd] scales)."""
+    lib = load()
+    B, E = x.shape
+    H, _, r = A_k.shape
+    Hd = q.shape[2]
+    L_cap = lat_k.shape[2]
+    _w8(A_k, sA_k, (H, E, r), (H, r), "A_k")
+    _w8(A_v, sA_v, (H, E, r), (H, r), "A_v")
+    _w8(B_k, sB_k, (H, r, Hd), (H, Hd), "B_k")
+    _w8(B_v, sB_v, (H, r, Hd), (H, Hd), "B_v")
+    _expect(lat_k, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_k")
+    _expect(lat_v, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_v")
+    _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, H, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, H, Hd), "out")
+    if append_ws is None:
+        append_ws = workspace(lib.wsvd_append_workspace_size(), x.device)
+    if decode_ws is None:
+        decode_ws = workspace(lib.wsvd_decode_workspace_size(B, H, r), q.device)
+    st = lib.wsvd_append_and_decode_w8(B, H, Hd, E, r, bits, L_cap, hadamard_block, _ptr(x), _dtype_code(x),
+                                       _ptr(A_k), _ptr(A_v), _ptr(sA_k), _ptr(sA_v), _ptr(seq_lens), _ptr(lat_k),
+                                       _ptr(lat_v), _ptr(scale_k), _ptr(scale_v), _ptr(q), _dtype_code(q),
+                                       _ptr(B_k), _ptr(B_v), _ptr(sB_k), _ptr(sB_v), float(softmax_scale),
+                                       _ptr(out), _ptr(append_ws), append_ws.numel(), _ptr(decode_ws),
+                                       decode_ws.numel(), _ptr(err), _stream(stream))
+    _check(st, "wsvd_append_and_decode_w8")
     return out
 
 

@@ -64,8 +64,9 @@ int run_decode(int codec, int rowbytes, int qmode, DecodeArgs a, void* workspace
 // fused step).  Returns WSVD_OK with *a filled, or an error status.
 int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens, const void* q,
                         int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
-                        const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
-                        void* workspace, size_t workspace_bytes, int32_t* err, DecodeArgs* a) {
+                        const void* scale_v, const void* B_k, const void* B_v, const float* sB_k, const float* sB_v,
+                        int w8, float softmax_scale, float* out, void* workspace, size_t workspace_bytes, int32_t* err,
+                        DecodeArgs* a) {
   int st = check_common(B, H, Hd, L_cap, seq_lens, q, q_dtype, out, workspace);
   if (st != WSVD_OK || B == 0) return st;
   if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
@@ -73,6 +74,7 @@ int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const 
   const int rowbytes = r * bits / 8;
   if (!decode_supported(bits == 8 ? kCodecI8 : kCodecI4, rowbytes, kQProj)) return WSVD_ERR_UNSUPPORTED;
   if (!lat_k || !lat_v || !scale_k || !scale_v || !B_k || !B_v) return WSVD_ERR_INVALID_ARG;
+  if (w8 && (!sB_k || !sB_v)) return WSVD_ERR_INVALID_ARG;
   if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
       !aligned16(B_k) || !aligned16(B_v))
     return WSVD_ERR_INVALID_ARG;
@@ -81,7 +83,7 @@ int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const 
   a->seq_lens = seq_lens; a->q = q; a->q_dtype = q_dtype;
   a->lat_k = lat_k; a->lat_v = lat_v;
   a->scale_k = static_cast<const __half*>(scale_k); a->scale_v = static_cast<const __half*>(scale_v);
-  a->Bk = static_cast<const __half*>(B_k); a->Bv = static_cast<const __half*>(B_v);
+  a->Bk = B_k; a->Bv = B_v; a->sBk = sB_k; a->sBv = sB_v; a->w8 = w8;
   a->qscale = resolve_scale(softmax_scale, Hd) * 1.4426950408889634f;
   a->out = out; a->err = err;
   return WSVD_OK;
@@ -89,9 +91,9 @@ int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const 
 
 // Validation and argument set-up of wsvd_latent_append (shared with the fused step).
 int prepare_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x, int x_dtype,
-                   const void* A_k, const void* A_v, int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v,
-                   void* scale_k, void* scale_v, void* workspace, size_t workspace_bytes, int32_t* err,
-                   AppendArgs* a) {
+                   const void* A_k, const void* A_v, const float* sA_k, const float* sA_v, int w8,
+                   int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
+                   size_t workspace_bytes, int32_t* err, AppendArgs* a) {
   if (B < 0 || H < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
   if (B == 0) return WSVD_OK;
   if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
@@ -102,6 +104,7 @@ int prepare_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard
   if (B > 16 || r % 8 || r > 128 || (r * bits / 8) % 4 || E > 65536) return WSVD_ERR_UNSUPPORTED;
   if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
     return WSVD_ERR_INVALID_ARG;
+  if (w8 && (!sA_k || !sA_v)) return WSVD_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
       !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
     return WSVD_ERR_INVALID_ARG;
@@ -113,10 +116,34 @@ int prepare_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard
   a->cluster = cl;
   a->hnorm = (float)(1.0 / sqrt((double)hadamard_block));
   a->x = x; a->x_dtype = x_dtype;
-  a->Ak = static_cast<const __half*>(A_k); a->Av = static_cast<const __half*>(A_v);
+  a->Ak = A_k; a->Av = A_v; a->sAk = sA_k; a->sAv = sA_v; a->w8 = w8;
   a->seq_lens = seq_lens; a->lat_k = lat_k; a->lat_v = lat_v;
   a->scale_k = static_cast<__half*>(scale_k); a->scale_v = static_cast<__half*>(scale_v);
   a->counter = static_cast<int32_t*>(workspace); a->err = err;
+  return WSVD_OK;
+}
+
+// The append, then the decode launched behind it as a programmatic dependent
+// (shared by the fp16 and int8-weight one-call steps).
+int run_step(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block, const void* x, int x_dtype,
+             const void* A_k, const void* A_v, const float* sA_k, const float* sA_v, int32_t* seq_lens, uint8_t* lat_k,
+             uint8_t* lat_v, void* scale_k, void* scale_v, const void* q, int q_dtype, const void* B_k,
+             const void* B_v, const float* sB_k, const float* sB_v, int w8, float softmax_scale, float* out,
+             void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
+             size_t decode_workspace_bytes, int32_t* err, void* stream) {
+  AppendArgs ap{};
+  int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, sA_k, sA_v, w8, seq_lens,
+                          lat_k, lat_v, scale_k, scale_v, append_workspace, append_workspace_bytes, err, &ap);
+  if (st != WSVD_OK) return st;
+  DecodeArgs dp{};
+  st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k, B_v,
+                           sB_k, sB_v, w8, softmax_scale, out, decode_workspace, decode_workspace_bytes, err, &dp);
+  if (st != WSVD_OK || B == 0) return st;
+  if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
+  bind_workspace(&dp, decode_workspace);
+  if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, as_stream(stream), true) !=
+      cudaSuccess)
+    return WSVD_ERR_CUDA;
   return WSVD_OK;
 }
 
@@ -174,7 +201,20 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
                           int32_t* err, void* stream) {
   DecodeArgs a{};
   const int st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v,
-                                     B_k, B_v, softmax_scale, out, workspace, workspace_bytes, err, &a);
+                                     B_k, B_v, nullptr, nullptr, 0, softmax_scale, out, workspace, workspace_bytes, err,
+                                     &a);
+  if (st != WSVD_OK || B == 0) return st;
+  return run_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a, workspace, as_stream(stream));
+}
+
+int wsvd_decode_attention_w8(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                             const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
+                             const void* scale_k, const void* scale_v, const int8_t* B_k, const int8_t* B_v,
+                             const float* sB_k, const float* sB_v, float softmax_scale, float* out, void* workspace,
+                             size_t workspace_bytes, int32_t* err, void* stream) {
+  DecodeArgs a{};
+  const int st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v,
+                                     B_k, B_v, sB_k, sB_v, 1, softmax_scale, out, workspace, workspace_bytes, err, &a);
   if (st != WSVD_OK || B == 0) return st;
   return run_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a, workspace, as_stream(stream));
 }
@@ -236,8 +276,20 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
                        uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace, size_t workspace_bytes,
                        int32_t* err, void* stream) {
   AppendArgs a{};
-  const int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, seq_lens, lat_k,
-                                lat_v, scale_k, scale_v, workspace, workspace_bytes, err, &a);
+  const int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, nullptr, nullptr, 0,
+                                seq_lens, lat_k, lat_v, scale_k, scale_v, workspace, workspace_bytes, err, &a);
+  if (st != WSVD_OK || B == 0) return st;
+  if (launch_append(a, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
+  return WSVD_OK;
+}
+
+int wsvd_latent_append_w8(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x,
+                          int x_dtype, const int8_t* A_k, const int8_t* A_v, const float* sA_k, const float* sA_v,
+                          int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                          void* workspace, size_t workspace_bytes, int32_t* err, void* stream) {
+  AppendArgs a{};
+  const int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, sA_k, sA_v, 1,
+                                seq_lens, lat_k, lat_v, scale_k, scale_v, workspace, workspace_bytes, err, &a);
   if (st != WSVD_OK || B == 0) return st;
   if (launch_append(a, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
   return WSVD_OK;
@@ -249,20 +301,21 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
                            const void* B_k, const void* B_v, float softmax_scale, float* out,
                            void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
                            size_t decode_workspace_bytes, int32_t* err, void* stream) {
-  AppendArgs ap{};
-  int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, seq_lens, lat_k, lat_v,
-                          scale_k, scale_v, append_workspace, append_workspace_bytes, err, &ap);
-  if (st != WSVD_OK) return st;
-  DecodeArgs dp{};
-  st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k, B_v,
-                           softmax_scale, out, decode_workspace, decode_workspace_bytes, err, &dp);
-  if (st != WSVD_OK || B == 0) return st;
-  if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
-  bind_workspace(&dp, decode_workspace);
-  if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, as_stream(stream), true) !=
-      cudaSuccess)
-    return WSVD_ERR_CUDA;
-  return WSVD_OK;
+  return run_step(B, H, Hd, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, nullptr, nullptr, seq_lens,
+                  lat_k, lat_v, scale_k, scale_v, q, q_dtype, B_k, B_v, nullptr, nullptr, 0, softmax_scale, out,
+                  append_workspace, append_workspace_bytes, decode_workspace, decode_workspace_bytes, err, stream);
+}
+
+int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                              const void* x, int x_dtype, const int8_t* A_k, const int8_t* A_v, const float* sA_k,
+                              const float* sA_v, int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k,
+                              void* scale_v, const void* q, int q_dtype, const int8_t* B_k, const int8_t* B_v,
+                              const float* sB_k, const float* sB_v, float softmax_scale, float* out,
+                              void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
+                              size_t decode_workspace_bytes, int32_t* err, void* stream) {
+  return run_step(B, H, Hd, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, sA_k, sA_v, seq_lens, lat_k,
+                  lat_v, scale_k, scale_v, q, q_dtype, B_k, B_v, sB_k, sB_v, 1, softmax_scale, out, append_workspace,
+                  append_workspace_bytes, decode_workspace, decode_workspace_bytes, err, stream);
 }
 
 }  // extern "C"

@@ -75,23 +75,33 @@ __device__ __forceinline__ void cp_async_wait_ring() {
   asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");
 }
 
+__device__ __forceinline__ void cp_async8(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+
 // Per-thread share of the CTA's A slice: rows k * nrg + rg (k = 0, 1, ...) of
-// the slice, 8 columns starting at 8 * cgi (one 16-byte piece per row).
+// the slice, 8 columns starting at 8 * cgi: one 16-byte piece per row (fp16),
+// or 8 bytes (int8 A) in the first half of the ring slot.
+template <bool W8>
 struct RowWalk {
-  const __half* A;  // first row of the slice
+  const uint8_t* A;  // first row of the slice
   int r, Ec, nrg, rg, cgi, nrows;
   __device__ __forceinline__ bool valid(int k) const { return k < nrows; }
   __device__ __forceinline__ int row(int k) const { return k * nrg + rg; }
   __device__ __forceinline__ void issue(uint4* ring, int k, int tid) const {
-    if (valid(k)) cp_async16(ring + (size_t)(k % kRing) * kAppendThreads + tid, A + (size_t)row(k) * r + cgi * 8);
+    if (valid(k)) {
+      const uint8_t* src = A + ((size_t)row(k) * r + cgi * 8) * (W8 ? 1 : 2);
+      if (W8) cp_async8(ring + (size_t)(k % kRing) * kAppendThreads + tid, src);
+      else cp_async16(ring + (size_t)(k % kRing) * kAppendThreads + tid, src);
+    }
     cp_async_commit();  // one group per ring step, empty past the end
   }
 };
 
 // Accumulate c[bb0 + bi][8 * cgi .. + 8] over this thread's rows, streaming
 // them through the ring (rows 0 .. kRing-1 already issued by the caller).
-template <int BB>
-__device__ __forceinline__ void stream_rows(const RowWalk& w, uint4* ring, const float* xs, int B, int bb0,
+template <int BB, bool W8>
+__device__ __forceinline__ void stream_rows(const RowWalk<W8>& w, uint4* ring, const float* xs, int B, int bb0,
                                             float (&acc)[BB][8], int tid) {
 #pragma unroll
   for (int bi = 0; bi < BB; ++bi)
@@ -100,7 +110,18 @@ __device__ __forceinline__ void stream_rows(const RowWalk& w, uint4* ring, const
   for (int k = 0; k < w.nrows; ++k) {
     cp_async_wait_ring();  // this thread's group k is complete
     const uint4 av = ring[(size_t)(k % kRing) * kAppendThreads + tid];
-    const float2 a01 = h2_pair(av.x), a23 = h2_pair(av.y), a45 = h2_pair(av.z), a67 = h2_pair(av.w);
+    float2 a01, a23, a45, a67;
+    if (W8) {  // int8 codes -> fp32, exact
+      a01 = i8_pair(av.x ^ 0x80808080u, 0);
+      a23 = i8_pair(av.x ^ 0x80808080u, 2);
+      a45 = i8_pair(av.y ^ 0x80808080u, 0);
+      a67 = i8_pair(av.y ^ 0x80808080u, 2);
+    } else {
+      a01 = h2_pair(av.x);
+      a23 = h2_pair(av.y);
+      a45 = h2_pair(av.z);
+      a67 = h2_pair(av.w);
+    }
     const float af[8] = {a01.x, a01.y, a23.x, a23.y, a45.x, a45.y, a67.x, a67.y};
     // The slot is consumed (values in registers) before it is refilled.
     w.issue(ring, k + kRing, tid);
@@ -162,7 +183,7 @@ __device__ __forceinline__ void fwht_smem_warp(float* v, int blk, int lane) {
   }
 }
 
-template <int BB>
+template <int BB, bool W8>
 __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_group& cluster, uint8_t* smem,
                                             const AppendSmem& L) {
   const int rank = (int)cluster.block_rank();
@@ -208,8 +229,8 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     }
   }
   const int ncg = r / 8, nrg = kAppendThreads / ncg;
-  RowWalk w;
-  w.A = (kv ? a.Av : a.Ak) + ((size_t)h * E + e0) * (size_t)r;
+  RowWalk<W8> w;
+  w.A = static_cast<const uint8_t*>(kv ? a.Av : a.Ak) + ((size_t)h * E + e0) * (size_t)r * (W8 ? 1 : 2);
   w.r = r; w.Ec = Ec; w.nrg = nrg; w.rg = tid / ncg; w.cgi = tid % ncg;
   w.nrows = w.rg < Ec ? (Ec - 1 - w.rg) / nrg + 1 : 0;
 #pragma unroll 1
@@ -265,7 +286,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
       for (int k = 0; k < kRing; ++k) w.issue(ring, k, tid);  // re-stream (L2) for the next batch rows
     }
     float acc[BB][8];
-    stream_rows<BB>(w, ring, xs, B, bb0, acc, tid);
+    stream_rows<BB, W8>(w, ring, xs, B, bb0, acc, tid);
     reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, slots + (size_t)bb0 * r, remote_slot + 4u * bb0 * r,
                    remote_bar, tid);
   }
@@ -313,6 +334,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
         float sum = 0.f;
         for (int q = 0; q < a.cluster; ++q) sum += slots[((size_t)q * B + b) * r + j];
         cv[k] = sum * a.hnorm;
+        if (W8) cv[k] *= (kv ? a.sAv : a.sAk)[(size_t)h * r + j];  // column scale of int8 A
         amax = fmaxf(amax, fabsf(cv[k]));
       }
     }
@@ -340,13 +362,15 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   }
 }
 
+// One kernel per weight format, so that each gets its own register allocation.
+template <bool W8>
 __global__ void __launch_bounds__(kAppendThreads, 4) append_kernel(const AppendArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const AppendSmem L = append_layout(a.B, a.E / a.cluster, a.r, a.cluster);
-  if (a.B == 1) append_body<1>(a, cluster, smem, L);
-  else if (a.B == 2) append_body<2>(a, cluster, smem, L);
-  else append_body<4>(a, cluster, smem, L);
+  if (a.B == 1) append_body<1, W8>(a, cluster, smem, L);
+  else if (a.B == 2) append_body<2, W8>(a, cluster, smem, L);
+  else append_body<4, W8>(a, cluster, smem, L);
 }
 
 int append_cluster_size(int E, int blk) {
@@ -361,19 +385,21 @@ size_t append_smem_bytes(int B, int E, int r, int cluster) {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   const size_t smem = append_smem_bytes(a.B, a.E, a.r, a.cluster);
+  void (*kern)(const AppendArgs) = a.w8 ? append_kernel<true> : append_kernel<false>;
   {
-    // Opt in to the dynamic shared memory once per device and size.
+    // Opt in to the dynamic shared memory once per device, kernel and size.
     static std::mutex mu;
-    static std::map<int, size_t> done;
+    static std::map<std::pair<int, int>, size_t> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    auto it = done.find(dev);
+    const auto key = std::make_pair(dev, a.w8);
+    auto it = done.find(key);
     if (it == done.end() || it->second < smem) {
-      e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      done[dev] = smem;
+      done[key] = smem;
     }
   }
   cudaLaunchConfig_t cfg = {};
@@ -388,7 +414,7 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, append_kernel, a);
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace wsvd

@@ -259,6 +259,11 @@ __device__ __forceinline__ float2 i4_pair(uint32_t xflip, int k) {
   return __fadd2_rn(f, make_float2(-8388616.f, -8388616.f));
 }
 
+// Element idx of a B matrix stored as fp16 or (w8) as int8, as float32 (exact).
+__device__ __forceinline__ float bmat_elem(const void* base, int w8, size_t idx) {
+  return w8 ? (float)static_cast<const int8_t*>(base)[idx] : __half2float(static_cast<const __half*>(base)[idx]);
+}
+
 __device__ __forceinline__ float2 h2_pair(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }

@@ -342,21 +342,30 @@ __device__ __forceinline__ void csync() { named_barrier_sync(1, kConsumerThreads
 // rotation (distinct banks across the warp's rows), then a fixed shuffle tree.
 // Every builder uses this routine, so q' is bit-identical whoever builds it.
 // Returns this lane's max |q'| over its rows.
-__device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, const DecodeArgs& a, int W, int j0,
-                                            int jstep, int part) {
-  const __half* Bs = reinterpret_cast<const __half*>(sbuf);
-  const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * 2);
+__device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, const DecodeArgs& a, int h, int W,
+                                            int j0, int jstep, int part) {
+  const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * (a.w8 ? 1 : 2));
+  const float* colscale = a.w8 ? a.sBk + (size_t)h * a.Hd : nullptr;  // int8 B_K: folded into q
   const int cols = a.Hd >> 3;
   float amax = 0.f;
+  auto qval = [&](int col) {
+    const uint16_t qu = qsrc[col];
+    return (a.q_dtype == WSVD_DTYPE_BF16) ? __uint_as_float((uint32_t)qu << 16) : __half2float(__ushort_as_half(qu));
+  };
   for (int j = j0; j < W; j += jstep) {
-    const __half* row = Bs + (size_t)j * a.Hd;
     float d = 0.f;
-    for (int k = 0; k < cols; ++k) {
-      const int col = ((k + j) % cols) * 8 + part;
-      const uint16_t qu = qsrc[col];
-      const float qv = (a.q_dtype == WSVD_DTYPE_BF16) ? __uint_as_float((uint32_t)qu << 16)
-                                                       : __half2float(__ushort_as_half(qu));
-      d = fmaf(__half2float(row[col]), qv, d);
+    if (colscale) {  // int8 B_K
+      const int8_t* row = reinterpret_cast<const int8_t*>(sbuf) + (size_t)j * a.Hd;
+      for (int k = 0; k < cols; ++k) {
+        const int col = ((k + j) % cols) * 8 + part;
+        d = fmaf((float)row[col], qval(col) * colscale[col], d);
+      }
+    } else {
+      const __half* row = reinterpret_cast<const __half*>(sbuf) + (size_t)j * a.Hd;
+      for (int k = 0; k < cols; ++k) {
+        const int col = ((k + j) % cols) * 8 + part;
+        d = fmaf(__half2float(row[col]), qval(col), d);
+      }
     }
     d += __shfl_xor_sync(0xffffffffu, d, 1);
     d += __shfl_xor_sync(0xffffffffu, d, 2);
@@ -376,7 +385,7 @@ __device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8
   const int warp = tid >> 5, lane = tid & 31;
   float amax = 0.f;
   if (QMODE == kQProj) {
-    amax = qprime_rows(sbuf, qs, a, W, tid >> 3, kConsumerThreads / 8, tid & 7);
+    amax = qprime_rows(sbuf, qs, a, blockIdx.y, W, tid >> 3, kConsumerThreads / 8, tid & 7);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   } else if (QMODE == kQDirect) {
@@ -621,22 +630,36 @@ __device__ __forceinline__ void merge_rows(const float* part, int np, float* res
   csync();
 }
 
-// One output column: (sum over e ascending of O[e] * Bv[e][d]) / L; dense path
-// (Bv null): O[d] / L.  L = 0 (no tokens) gives zero.
+// Up-projection operand: B_Vh (fp16, or int8 with per-column scales sv).
+struct BvRef {
+  const void* p;   // [W][Hd], or null on the dense path
+  int w8;
+  const float* sv;  // w8: [Hd]
+};
+
+// One output column: (sum over e ascending of O[e] * Bv[e][d]) (* sv[d] for
+// int8 B_V) / L; dense path (no B_V): O[d] / L.  L = 0 (no tokens) gives zero.
 template <int W>
-__device__ __forceinline__ float out_col(const float* res, const __half* Bv, int Hd, int d) {
+__device__ __forceinline__ float out_col(const float* res, const BvRef& bv, int Hd, int d) {
   const float inv = res[1] > 0.f ? 1.f / res[1] : 0.f;
-  if (Bv == nullptr) return res[2 + d] * inv;
+  if (bv.p == nullptr) return res[2 + d] * inv;
   float s = 0.f;
-  for (int e = 0; e < W; ++e) s = fmaf(res[2 + e], __half2float(Bv[(size_t)e * Hd + d]), s);
+  if (bv.w8) {
+    const int8_t* B8 = static_cast<const int8_t*>(bv.p);
+    for (int e = 0; e < W; ++e) s = fmaf(res[2 + e], (float)B8[(size_t)e * Hd + d], s);
+    s *= bv.sv[d];
+  } else {
+    const __half* Bh = static_cast<const __half*>(bv.p);
+    for (int e = 0; e < W; ++e) s = fmaf(res[2 + e], __half2float(Bh[(size_t)e * Hd + d]), s);
+  }
   return s * inv;
 }
 
 // out[b, h, :] from the merged res[] (consumer threads; see out_col).
 template <int W>
-__device__ __forceinline__ void finalize_out(const float* res, const __half* Bv, float* outp, int Hd, float* red,
+__device__ __forceinline__ void finalize_out(const float* res, const BvRef& bv, float* outp, int Hd, float* red,
                                              int tid) {
-  for (int d = tid; d < Hd; d += kConsumerThreads) outp[d] = out_col<W>(res, Bv, Hd, d);
+  for (int d = tid; d < Hd; d += kConsumerThreads) outp[d] = out_col<W>(res, bv, Hd, d);
   csync();
 }
 
@@ -646,9 +669,9 @@ __device__ __forceinline__ void issue_operands(uint8_t* dst, uint64_t* bar, cons
                                                uint64_t keep) {
   const size_t bh = (size_t)b * a.H + h;
   if (QMODE == kQProj) {
-    const uint32_t bb = (uint32_t)W * a.Hd * 2, qb = (uint32_t)a.Hd * 2;
+    const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), qb = (uint32_t)a.Hd * 2;
     mbar_arrive_expect_tx(bar, bb + qb);
-    bulk_g2s(dst, a.Bk + (size_t)h * W * a.Hd, bb, bar, keep);
+    bulk_g2s(dst, static_cast<const uint8_t*>(a.Bk) + (size_t)h * bb, bb, bar, keep);
     bulk_g2s(dst + bb, static_cast<const uint16_t*>(a.q) + bh * a.Hd, qb, bar, keep);
   } else if (QMODE == kQDirect) {
     mbar_arrive_expect_tx(bar, (uint32_t)a.Hd * 2);
@@ -692,7 +715,7 @@ __device__ __forceinline__ float helper_qprime(const uint8_t* sbuf, float* qsv, 
                                                int lane) {
   float amax = 0.f;
   if (QMODE == kQProj) {
-    amax = qprime_rows(sbuf, qsv, a, W, lane >> 3, 4, lane & 7);
+    amax = qprime_rows(sbuf, qsv, a, (int)(bh % a.H), W, lane >> 3, 4, lane & 7);
   } else if (QMODE == kQDirect) {
     const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf);
     for (int j = lane; j < W; j += 32) {
@@ -763,8 +786,8 @@ __device__ __forceinline__ void helper_planes(const float* qsv, int* qi, uint32_
 
 // Warp-level out[b, h, :] (same per-column arithmetic as finalize_out).
 template <int W>
-__device__ __forceinline__ void helper_finalize(const float* res, const __half* Bv, float* outp, int Hd, int lane) {
-  for (int d = lane; d < Hd; d += 32) outp[d] = out_col<W>(res, Bv, Hd, d);
+__device__ __forceinline__ void helper_finalize(const float* res, const BvRef& bv, float* outp, int Hd, int lane) {
+  for (int d = lane; d < Hd; d += 32) outp[d] = out_col<W>(res, bv, Hd, d);
 }
 
 template <int CODEC, int VPT, int TPT, int NTOK, int QMODE>
@@ -905,12 +928,12 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       if (stage_bv) {
         int lb, lh, lt;
         walk.locate(g_end - 1, lb, lh, lt);
-        const uint32_t bytes = (uint32_t)W * a.Hd * 2;
+        const uint32_t bytes = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2);
         mbar_arrive_expect_tx(bvbar, bytes);
         for (uint32_t off = 0; off < bytes; off += 32768)
           bulk_g2s(reinterpret_cast<uint8_t*>(bv_last) + off,
-                   reinterpret_cast<const uint8_t*>(a.Bv + (size_t)lh * W * a.Hd) + off, min(32768u, bytes - off),
-                   bvbar, keep);
+                   static_cast<const uint8_t*>(a.Bv) + (size_t)lh * bytes + off, min(32768u, bytes - off), bvbar,
+                   keep);
       }
       // Leave no copy in flight behind: wait (bounded) for the last uses of each buffer.
       if (stage_bv && !mbar_wait_bounded(bvbar, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
@@ -967,8 +990,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
           ha->seginfo[sq][3] = cl;
         }
         if (a.Bv != nullptr && c == cl) {  // the likely finisher warms B_Vh in L2
-          const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)sb_h * W * a.Hd);
-          for (int o = lane * 128; o < W * a.Hd * 2; o += 32 * 128) prefetch_l2(bv + o);
+          const int bytes = W * a.Hd * (a.w8 ? 1 : 2);
+          const char* bv = static_cast<const char*>(a.Bv) + (size_t)sb_h * bytes;
+          for (int o = lane * 128; o < bytes; o += 32 * 128) prefetch_l2(bv + o);
         }
         if (QMODE != kQGlobal) wait(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1));
         if (k >= NQ) wait(&qfree[sq], (uint32_t)(((k / NQ) - 1) & 1));
@@ -994,7 +1018,8 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       const int sb_b = ha->seginfo[si][0], sb_h = ha->seginfo[si][1];
       const int cf = ha->seginfo[si][2], cl = ha->seginfo[si][3];
       float* outp = a.out + ((size_t)sb_b * a.H + sb_h) * a.Hd;
-      const __half* Bvh = a.Bv ? a.Bv + (size_t)sb_h * W * a.Hd : nullptr;
+      const BvRef Bvh{a.Bv ? static_cast<const uint8_t*>(a.Bv) + (size_t)sb_h * W * a.Hd * (a.w8 ? 1 : 2) : nullptr,
+                      a.w8, a.w8 ? a.sBv + (size_t)sb_h * a.Hd : nullptr};
       if (cf == cl) {
         helper_finalize<W>(res, Bvh, outp, a.Hd, lane);
       } else {
@@ -1062,13 +1087,13 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
     const int seen = (cf != cl && tid == 0) ? ld_acquire_gpu(&a.counters[bh]) : 0;
     reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
     float* outp = a.out + ((size_t)b_ * a.H + h_) * a.Hd;
-    const __half* Bvh = nullptr;
+    BvRef Bvh{nullptr, a.w8, a.w8 ? a.sBv + (size_t)h_ * a.Hd : nullptr};
     if (a.Bv != nullptr) {
       if (C::bv_stage_bytes(a.Hd) > 0) {  // staged by the producer
         wait(bvbar, 0);
-        Bvh = bv_last;
+        Bvh.p = bv_last;
       } else {
-        Bvh = a.Bv + (size_t)h_ * W * a.Hd;
+        Bvh.p = static_cast<const uint8_t*>(a.Bv) + (size_t)h_ * W * a.Hd * (a.w8 ? 1 : 2);
       }
     }
     if (cf == cl) {
@@ -1207,10 +1232,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     const uint64_t keep = l2_evict_last_policy();
     issue_operands<W, QMODE>(segbuf, segfull, a, b, h, keep);
     if (rank == 0 && a.Bv != nullptr) {
-      const uint32_t bb = (uint32_t)W * a.Hd * 2;
+      const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2);
       mbar_arrive_expect_tx(&aux[0], bb);
       for (uint32_t off = 0; off < bb; off += 32768)
-        bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, reinterpret_cast<const uint8_t*>(a.Bv + (size_t)h * W * a.Hd) + off,
+        bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, static_cast<const uint8_t*>(a.Bv) + (size_t)h * bb + off,
                  min(32768u, bb - off), &aux[0], keep);
     }
   }
@@ -1364,11 +1389,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     csync();
     merge_rows<W, false>(slots, csize, res, tid);
   }
-  const __half* Bvh = nullptr;
+  BvRef Bvh{nullptr, a.w8, a.w8 ? a.sBv + (size_t)h * a.Hd : nullptr};
   if (a.Bv != nullptr) {
     if (!mbar_wait_bounded(&aux[0], 0, timed_out ? 0ull : kWaitLimitNs) && lane == 0)
       set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-    Bvh = bvs;
+    Bvh.p = bvs;
   }
   finalize_out<W>(res, Bvh, a.out + ((size_t)b * a.H + h) * a.Hd, a.Hd, red, tid);
 }
@@ -1585,7 +1610,7 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
     // split plan and first tiles overlap the projection (only its helper warp
     // waits for q').  Behind an append the projection itself completes after
     // the append, and the decode waits for everything (dep 2).
-    e = launch_qproj(a.B, a.H, a.Hd, a.W, a.q, a.q_dtype, a.Bk, a.qglobal, stream, after_append);
+    e = launch_qproj(a.B, a.H, a.Hd, a.W, a.q, a.q_dtype, a.Bk, a.sBk, a.w8, a.qglobal, stream, after_append);
     if (e != cudaSuccess) return e;
     a.dep = after_append ? 2 : 1;
     pdl = true;

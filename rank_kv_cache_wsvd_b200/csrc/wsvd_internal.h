@@ -38,8 +38,11 @@ struct DecodeArgs {
   const uint8_t* lat_v;
   const __half* scale_k; // per-token scales (quantised codecs only)
   const __half* scale_v;
-  const __half* Bk;      // [H][W][Hd] (kQProj)
-  const __half* Bv;      // [H][W][Hd], or nullptr for the dense path (W == Hd)
+  const void* Bk;        // [H][W][Hd] fp16, or int8 when w8
+  const void* Bv;        // [H][W][Hd] fp16, or int8 when w8; nullptr for the dense path (W == Hd)
+  const float* sBk;      // w8: per-column scales [H][Hd] of B_k (B_k[h][j][d] * sBk[h][d])
+  const float* sBv;      // w8: per-column scales [H][Hd] of B_v
+  int w8;                // 1: B_k, B_v are int8 with per-column fp32 scales
   float* qglobal;        // [B][H][W] projected q' (kQGlobal; workspace)
   float qscale;          // softmax_scale * log2(e)
   float* out;            // [B][H][Hd]
@@ -59,8 +62,8 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
 // q'[b][h][:] = B_Kh . q[b, h] (W values) into qglobal.  after_append: launched
 // as a programmatic dependent of the preceding kernel, and completes only
 // after that kernel has (so a decode launched behind it may rely on both).
-cudaError_t launch_qproj(int B, int H, int Hd, int W, const void* q, int q_dtype, const __half* Bk, float* qglobal,
-                         cudaStream_t stream, bool after_append);
+cudaError_t launch_qproj(int B, int H, int Hd, int W, const void* q, int q_dtype, const void* Bk, const float* sBk,
+                         int w8, float* qglobal, cudaStream_t stream, bool after_append);
 // Kernels one launch_decode call issues (1, or 2 with the q' projection).
 int decode_launch_count(int codec, int rowbytes, int qmode, const DecodeArgs& a);
 
@@ -69,8 +72,11 @@ struct AppendArgs {
   float hnorm;           // 1/sqrt(blk), correctly rounded
   const void* x;
   int x_dtype;
-  const __half* Ak;
-  const __half* Av;
+  const void* Ak;        // [H][E][r] fp16, or int8 when w8
+  const void* Av;
+  const float* sAk;      // w8: per-column scales [H][r] (A_k[h][e][j] * sAk[h][j])
+  const float* sAv;
+  int w8;                // 1: A_k, A_v are int8 with per-column fp32 scales
   int32_t* seq_lens;
   uint8_t* lat_k;
   uint8_t* lat_v;

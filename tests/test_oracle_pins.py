@@ -409,3 +409,16 @@ def test_footprint_against_pages_and_arrays():
     assert nb == O.wsvd_cache_bytes(w.B, w.H, w.L_cap, w.r, w.bits)
     s = W.shared_inputs(W.CMP[2048].with_(B=1, L_cap=16, lens=16))
     assert s["lat_k"].nbytes + s["lat_v"].nbytes == O.shared_cache_bytes(1, 16, 512)
+
+
+def test_dequantize_weights_scales_each_output_column():
+    """Hand-computed: one scale per output column (last axis), shared by every
+    row of the contraction axis; a per-row scale would give other numbers."""
+    wq = np.array([[[1, -2], [3, 4]]], np.int8)         # [H=1][K=2][N=2]
+    s = np.array([[0.5, 2.0]], np.float32)               # [H][N]
+    got = O.dequantize_weights(wq, s)
+    assert np.array_equal(got, np.array([[[0.5, -4.0], [1.5, 8.0]]]))
+    # an int8 matrix with unit scales is the matrix itself
+    rng = np.random.default_rng(0)
+    q = rng.integers(-127, 128, size=(3, 5, 7)).astype(np.int8)
+    assert np.array_equal(O.dequantize_weights(q, np.ones((3, 7), np.float32)), q.astype(np.float64))

@@ -77,3 +77,16 @@ def test_append_inputs_outliers():
     assert a.x.shape == (3, 2, 4096) and a.A_k.shape == (32, 4096, 32)
     big = np.abs(a.x).max(axis=(0, 1)) > 20
     assert 1 <= big.sum() <= 8
+
+
+def test_w8_weight_recipe_hits_the_code_range_per_column():
+    """Per output column: every code in [-127, 127], the largest magnitude 127,
+    and the dequantised matrix within half a step of the fp16 one."""
+    ai = W.append_inputs(W.PR1, seed=0, steps=1)
+    q, s = W.quantize_weights_w8(ai.A_k)
+    assert q.dtype == np.int8 and s.dtype == np.float32 and s.shape == (W.PR1.H, W.PR1.r)
+    assert np.abs(q.astype(int)).max() <= 127
+    assert np.all(np.abs(q.astype(int)).max(axis=1) == 127)
+    back = q.astype(np.float64) * s.astype(np.float64)[:, None, :]
+    # half a step, plus the float32 rounding of w / scale (up to 127 * 2^-24 code units)
+    assert np.all(np.abs(back - ai.A_k.astype(np.float64)) <= (0.5 + 1e-4) * s.astype(np.float64)[:, None, :])

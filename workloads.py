@@ -267,6 +267,18 @@ def append_inputs(w: Workload, seed: int = 0, steps: Optional[int] = None) -> Ap
     return AppendInputs(w, xv, xb, ak, av)
 
 
+def quantize_weights_w8(Wf: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Input recipe of the int8-weight (W8) workloads: each weight matrix
+    [H][K][N] (fp16) is stored as symmetric int8 with one fp32 scale per output
+    column, scale[h][n] = max_k |W[h][k][n]| / 127 (1 for an all-zero column),
+    code = clamp(round_half_even(W / scale), -127, 127)."""
+    w = np.asarray(Wf, np.float32)
+    scale = (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)
+    scale[scale == 0] = 1.0
+    q = np.clip(np.rint(w / scale[:, None, :]), -127, 127).astype(np.int8)
+    return q, scale
+
+
 # ----------------------------------------------------------------------------- comparisons
 def dense_block(w: Workload, seed: int, b: int, h: int) -> Tuple[np.ndarray, np.ndarray]:
     """Dense K, V [L_cap][Hd] fp16 ~ N(0,1) for one (b, h)."""
