@@ -243,6 +243,24 @@ int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int 
                               void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
                               size_t decode_workspace_bytes, int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- latent rotation S2 (weight preparation)
+ * Folds an orthogonal rotation S2 of each head's latent space into the
+ * low-rank factors (the "Outlier-Smoothing" transforms S1, S2 of the WSVD
+ * summaries, German §2.C and Arabic §2.c; S2 is learned jointly with A and B,
+ * and given here):
+ *   A'_k[h] = A_k[h] . S2_k[h],   B'_k[h] = S2_k[h]^T . B_k[h]   (same for V).
+ * With S2 . S2^T = I the rebuilt keys and values c . B are unchanged, while
+ * the cache then holds the rotated latents c . S2, which are what the append
+ * quantises.  Run once at model load; the other entry points take A', B'.
+ *   S2_k, S2_v            [H][r][r] float32, orthogonal (not checked).
+ *   A_k, A_v              [H][E][r] fp16;  A_k_out, A_v_out same shape, written.
+ *   B_k, B_v              [H][r][Hd] fp16; B_k_out, B_v_out same shape, written.
+ * fp32 dot products over r, each result rounded once to fp16.  Outputs must not
+ * alias inputs; r <= 128, H <= 65535.  Launches four small kernels on `stream`. */
+int wsvd_fold_latent_rotation(int H, int E, int r, int Hd, const float* S2_k, const float* S2_v, const void* A_k,
+                              const void* A_v, const void* B_k, const void* B_v, void* A_k_out, void* A_v_out,
+                              void* B_k_out, void* B_v_out, void* stream);
+
 /* ---------------------------------------------------------------- comparison: dense decode
  * The flash-decoding baseline the pages compare against (German §4
  * "Ergebnisse"): out[b,h] = softmax(K[b,h,:n] . q[b,h] * softmax_scale) . V[b,h,:n]

@@ -266,6 +266,24 @@ def latent_append(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r: int,
 
 
 # ----------------------------------------------------------------------------- footprint
+# ----------------------------------------------------------------------------- latent rotation S2
+def fold_latent_rotation(A: np.ndarray, B: np.ndarray, S2: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Fold an orthogonal rotation S2 of each head's latent space into its
+    factors: A' = A . S2 (A [H][E][r]) and B' = S2^T . B (B [H][r][Hd]),
+    S2 [H][r][r] orthogonal (float64).
+
+    The pages introduce orthogonal transforms S1 (the Hadamard rotation of the
+    activations) and S2, learned jointly with A and B to smooth what is
+    quantised (de §2.C "Outlier-Smoothing", ar §2.c).  Reading taken: S2 acts
+    on the r-dimensional latent of each head (one for K, one for V), so the
+    cache holds rotated latents c . S2 and, since S2 . S2^T = I, folding it
+    into A and B leaves c . B unchanged."""
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    S2 = np.asarray(S2, np.float64)
+    return np.einsum("her,hrs->hes", A, S2), np.einsum("hrs,hrd->hsd", S2, B)
+
+
 # ----------------------------------------------------------------------------- int8 weights
 def dequantize_weights(wq: np.ndarray, scale: np.ndarray) -> np.ndarray:
     """Int8 weight matrices wq [H][K][N] with one scale per output column,

@@ -46,6 +46,7 @@ SIGNATURES = {
     "wsvd_latent_append_w8": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 9 + [_p, _c_size, _p, _p]),
     "wsvd_append_and_decode_w8": (_c_int, [_c_int] * 8 + [_p, _c_int] + [_p] * 9 + [_p, _c_int] + [_p] * 4
                                   + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
+    "wsvd_fold_latent_rotation": (_c_int, [_c_int] * 4 + [_p] * 11),
     "dense_decode_attention": (_c_int, [_c_int] * 4 + [_p, _p, _c_int, _p, _p, _c_float, _p, _p, _c_size, _p, _p]),
     "shared_latent_svd_decode": (_c_int, [_c_int] * 5 + [_p, _p, _c_int] + [_p] * 4 + [_c_float, _p, _p, _c_size,
                                                                                          _p, _p]),
@@ -346,6 +347,25 @@ def wsvd_append_and_decode_w8(x, A_k, A_v, sA_k, sA_v, seq_lens, lat_k, lat_v, s
                                        decode_ws.numel(), _ptr(err), _stream(stream))
     _check(st, "wsvd_append_and_decode_w8")
     return out
+
+
+# ----------------------------------------------------------------------------- latent rotation
+def wsvd_fold_latent_rotation(S2_k, S2_v, A_k, A_v, B_k, B_v, stream=None):
+    """A' = A . S2 and B' = S2^T . B per head (weight preparation).  Returns
+    (A_k', A_v', B_k', B_v') as new fp16 tensors."""
+    lib = load()
+    H, E, r = A_k.shape
+    Hd = B_k.shape[2]
+    for t, shape, name in ((S2_k, (H, r, r), "S2_k"), (S2_v, (H, r, r), "S2_v")):
+        _expect(t, torch.float32, shape, name)
+    for t, shape, name in ((A_k, (H, E, r), "A_k"), (A_v, (H, E, r), "A_v"), (B_k, (H, r, Hd), "B_k"),
+                           (B_v, (H, r, Hd), "B_v")):
+        _expect(t, torch.float16, shape, name)
+    outs = [torch.empty_like(t) for t in (A_k, A_v, B_k, B_v)]
+    st = lib.wsvd_fold_latent_rotation(H, E, r, Hd, _ptr(S2_k), _ptr(S2_v), _ptr(A_k), _ptr(A_v), _ptr(B_k),
+                                       _ptr(B_v), *[_ptr(o) for o in outs], _stream(stream))
+    _check(st, "wsvd_fold_latent_rotation")
+    return tuple(outs)
 
 
 # ----------------------------------------------------------------------------- append

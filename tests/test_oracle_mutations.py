@@ -119,3 +119,27 @@ def test_shared_path_wrong_head_mutant_is_caught(monkeypatch):
     _patch(monkeypatch, "shared_latent_decode", wrong)
     with pytest.raises(AssertionError):
         P.test_shared_latent_with_selector_factors_equals_dense()
+
+
+@pytest.mark.parametrize("kind", ["B_not_transposed", "A_transposed_rotation", "dequant_per_row"])
+def test_rotation_and_weight_mutants_are_caught(monkeypatch, kind):
+    """Folding S2 (not S2^T) into B, rotating A by S2^T, or scaling int8 weights
+    per row instead of per output column: the pins must fail."""
+    if kind == "dequant_per_row":
+        _patch(monkeypatch, "dequantize_weights",
+               lambda wq, s: np.asarray(wq, np.float64) * np.asarray(s, np.float64)[:, :, None]
+               if np.shape(s)[1] == np.shape(wq)[1] else np.asarray(wq, np.float64) * 0.0)
+        with pytest.raises(AssertionError):
+            P.test_dequantize_weights_scales_each_output_column()
+        return
+
+    def fold(A, B, S2):
+        A = np.asarray(A, np.float64)
+        B = np.asarray(B, np.float64)
+        S2 = np.asarray(S2, np.float64)
+        if kind == "B_not_transposed":
+            return np.einsum("her,hrs->hes", A, S2), np.einsum("hsr,hrd->hsd", S2, B)
+        return np.einsum("her,hsr->hes", A, S2), np.einsum("hrs,hrd->hsd", S2, B)
+    _patch(monkeypatch, "fold_latent_rotation", fold)
+    with pytest.raises(AssertionError):
+        P.test_fold_latent_rotation_pins()

@@ -422,3 +422,37 @@ def test_dequantize_weights_scales_each_output_column():
     rng = np.random.default_rng(0)
     q = rng.integers(-127, 128, size=(3, 5, 7)).astype(np.int8)
     assert np.array_equal(O.dequantize_weights(q, np.ones((3, 7), np.float32)), q.astype(np.float64))
+
+
+def test_fold_latent_rotation_pins():
+    """S2 = I leaves the factors unchanged; a hand-worked 2 x 2 rotation; and
+    for a random orthogonal S2 the rebuilt keys c . B and the attention output
+    over unquantised latents are unchanged (to float64 rounding), while the
+    latents themselves do change."""
+    rng = np.random.default_rng(3)
+    A = rng.standard_normal((2, 8, 4))
+    B = rng.standard_normal((2, 4, 6))
+    I = np.broadcast_to(np.eye(4), (2, 4, 4))
+    a2, b2 = O.fold_latent_rotation(A, B, I)
+    assert np.array_equal(a2, A) and np.array_equal(b2, B)
+    # a quarter turn in the latent plane: columns (x, y) -> (-y, x)
+    R = np.array([[[0.0, 1.0], [-1.0, 0.0]]])
+    a, b = O.fold_latent_rotation(np.array([[[1.0, 2.0]]]), np.array([[[3.0], [5.0]]]), R)
+    assert np.array_equal(a, np.array([[[-2.0, 1.0]]])) and np.array_equal(b, np.array([[[-5.0], [3.0]]]))
+    # invariance for a random orthogonal S2 (one per head)
+    w = W.PR1
+    S2 = W.latent_rotation(w, seed=1).astype(np.float64)
+    assert np.allclose(np.einsum("hrs,hts->hrt", S2, S2), np.eye(w.r)[None], atol=1e-6)
+    x = rng.standard_normal((3, 8))
+    A = rng.standard_normal((w.H, 8, w.r))
+    B = rng.standard_normal((w.H, w.r, w.Hd))
+    A2, B2 = O.fold_latent_rotation(A, B, S2)
+    c, c2 = np.einsum("le,her->hlr", x, A), np.einsum("le,her->hlr", x, A2)
+    assert not np.allclose(c, c2)
+    K, K2 = np.einsum("hlr,hrd->hld", c, B), np.einsum("hlr,hrd->hld", c2, B2)
+    assert np.allclose(K, K2, rtol=1e-5, atol=1e-5)   # S2 is float32-orthogonal
+    q = rng.standard_normal(w.Hd)
+    for h in range(w.H):
+        o1, _ = O.attention(q, K[h], K[h], 0.125)
+        o2, _ = O.attention(q, K2[h], K2[h], 0.125)
+        assert np.allclose(o1, o2, rtol=1e-5, atol=1e-5)

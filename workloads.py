@@ -33,6 +33,7 @@ import numpy as np
 _T_Q, _T_LK, _T_LV, _T_BK, _T_BV, _T_LEN, _T_OUTL = 1, 2, 3, 4, 5, 6, 7
 _T_X, _T_AK, _T_AV, _T_XOUT = 10, 11, 12, 13
 _T_DK, _T_DV, _T_SK, _T_SV, _T_SBK, _T_SBV = 20, 21, 22, 23, 24, 25
+_T_S2K, _T_S2V = 30, 31
 
 
 def _rng(seed: int, *key: int) -> np.random.Generator:
@@ -265,6 +266,17 @@ def append_inputs(w: Workload, seed: int = 0, steps: Optional[int] = None) -> Ap
     ak = (_rng(seed, _T_AK).standard_normal((w.H, w.E, w.r)) * sd).astype(np.float16)
     av = (_rng(seed, _T_AV).standard_normal((w.H, w.E, w.r)) * sd).astype(np.float16)
     return AppendInputs(w, xv, xb, ak, av)
+
+
+def latent_rotation(w: Workload, seed: int = 0, which: str = "k") -> np.ndarray:
+    """Synthetic orthogonal latent rotations S2 [H][r][r] (float32): the Q
+    factor of a Gaussian matrix per head, sign-fixed so that diag(R) > 0."""
+    g = _rng(seed, _T_S2K if which == "k" else _T_S2V).standard_normal((w.H, w.r, w.r))
+    out = np.empty_like(g)
+    for h in range(w.H):
+        q, rr = np.linalg.qr(g[h])
+        out[h] = q * np.sign(np.diag(rr))[None, :]
+    return out.astype(np.float32)
 
 
 def quantize_weights_w8(Wf: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
