@@ -265,6 +265,49 @@ def latent_append(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r: int,
     return lat_k, scale_k, lat_v, scale_v, lens.astype(np.int32), err, ck, cv
 
 
+def latent_prefill(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r: int, bits: int, block: int):
+    """Write a block of T new tokens per sequence into the latent cache (the
+    prompt's tokens, e.g. the image tokens of a vision-language prompt, in one
+    call instead of T single-token appends).
+
+    x [B][T][E].  Each token is rotated, projected and quantised exactly as by
+    latent_append (the per-head projection of German §2.A after the rotation
+    S1 and the W8A8 / W8A4 quantiser of German §2.C): token t of sequence b
+    goes to row seq_lens[b] + t, then seq_lens[b] += T.  The pages describe
+    the cache and its per-token quantiser, not a block interface; the block
+    write is read as the same rows that T successive appends would write.
+    A sequence whose block does not fit (seq_lens[b] < 0 or
+    seq_lens[b] + T > L_cap) is left untouched and flagged.
+    Returns (lat_k, scale_k, lat_v, scale_v, seq_lens, err_rows, ck, cv) with
+    ck, cv [B][T][H][r] float64."""
+    x = np.asarray(x, np.float64)
+    B, T, E = x.shape
+    xt = block_hadamard_rotate(x, block)
+    H = np.shape(A_k)[0]
+    ck = np.stack([xt @ np.asarray(A_k[h], np.float64) for h in range(H)], axis=2)  # [B][T][H][r]
+    cv = np.stack([xt @ np.asarray(A_v[h], np.float64) for h in range(H)], axis=2)
+    lat_k, lat_v = lat_k.copy(), lat_v.copy()
+    scale_k, scale_v = scale_k.copy(), scale_v.copy()
+    lens = np.asarray(seq_lens, np.int64).copy()
+    L_cap = lat_k.shape[2]
+    err = np.zeros(B, bool)
+    for b in range(B):
+        pos = int(lens[b])
+        if pos < 0 or pos + T > L_cap:
+            err[b] = True
+            continue
+        for t in range(T):
+            for h in range(H):
+                codes, s = quantize(ck[b, t, h], bits)
+                lat_k[b, h, pos + t] = pack_codes(codes, bits)
+                scale_k[b, h, pos + t] = s
+                codes, s = quantize(cv[b, t, h], bits)
+                lat_v[b, h, pos + t] = pack_codes(codes, bits)
+                scale_v[b, h, pos + t] = s
+        lens[b] = pos + T
+    return lat_k, scale_k, lat_v, scale_v, lens.astype(np.int32), err, ck, cv
+
+
 # ----------------------------------------------------------------------------- footprint
 # ----------------------------------------------------------------------------- latent rotation S2
 def fold_latent_rotation(A: np.ndarray, B: np.ndarray, S2: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:

@@ -143,3 +143,56 @@ def test_rotation_and_weight_mutants_are_caught(monkeypatch, kind):
     _patch(monkeypatch, "fold_latent_rotation", fold)
     with pytest.raises(AssertionError):
         P.test_fold_latent_rotation_pins()
+
+
+def _prefill_variant(kind):
+    orig = OW.latent_prefill
+
+    def f(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r, bits, block):
+        x = np.asarray(x, np.float64)
+        if kind == "batch_rows_swapped" and x.shape[0] > 1:
+            x = x[::-1]
+        if kind == "tokens_reversed":
+            x = x[:, ::-1]
+        lens = np.asarray(seq_lens, np.int64)
+        if kind == "accept_overflow":  # refuses only a full cache, clips the block at L_cap
+            L_cap, T = lat_k.shape[2], x.shape[1]
+            res = list(orig(x, A_k, A_v, lens, lat_k, scale_k, lat_v, scale_v, r, bits, block))
+            res[:5] = [lat_k.copy(), scale_k.copy(), lat_v.copy(), scale_v.copy(), lens.astype(np.int32)]
+            res[5] = np.ones(x.shape[0], bool)
+            for b in range(x.shape[0]):
+                pos = int(lens[b])
+                if 0 <= pos < L_cap:
+                    n = min(T, L_cap - pos)
+                    one = orig(x[b:b + 1, :n], A_k, A_v, lens[b:b + 1], lat_k[b:b + 1], scale_k[b:b + 1],
+                               lat_v[b:b + 1], scale_v[b:b + 1], r, bits, block)
+                    for i in range(4):
+                        res[i][b] = one[i][0]
+                    res[4][b] = pos + n
+                    res[5][b] = False
+            return tuple(res)
+        out = list(orig(x, A_k, A_v, seq_lens, lat_k, scale_k, lat_v, scale_v, r, bits, block))
+        if kind == "advance_by_one":
+            out[4] = np.where(out[5], out[4], np.asarray(seq_lens, np.int32) + 1).astype(np.int32)
+        return tuple(out)
+    return f
+
+
+@pytest.mark.parametrize("kind", ["batch_rows_swapped", "tokens_reversed", "accept_overflow", "advance_by_one"])
+def test_prefill_mutants_are_caught(monkeypatch, kind):
+    """A token written to another sequence's or another position's row, a
+    block clipped at the capacity instead of refused, or the length advanced
+    by one instead of T: at least one prefill pin must fail."""
+    _patch(monkeypatch, "latent_prefill", _prefill_variant(kind))
+    failed = 0
+    for bits in (8, 4):
+        try:
+            P.test_prefill_equals_successive_appends(bits)
+        except AssertionError:
+            failed += 1
+    for pin in (P.test_prefill_projection_is_one_dense_matmul, P.test_prefill_capacity_boundary_and_empty_block):
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0

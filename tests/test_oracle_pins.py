@@ -392,6 +392,68 @@ def test_append_writes_one_row_and_advances():
                 assert np.all(np.abs(codes * float(s) - ck[b, h]) <= float(s) / 2 * (1 + 1e-6) + 1e-12)
 
 
+# ----------------------------------------------------------------------------- prefill (block of T tokens)
+def _prefill_case(seed, B=3, T=4, H=2, E=256, r=8, L_cap=9, bits=8):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, T, E))
+    Ak = (rng.standard_normal((H, E, r)) / 16).astype(np.float16)
+    Av = (rng.standard_normal((H, E, r)) / 16).astype(np.float16)
+    rb = r * bits // 8
+    lat = rng.integers(0, 256, size=(B, H, L_cap, rb), dtype=np.uint8)
+    sc = rng.uniform(0, 1, (B, H, L_cap)).astype(np.float16)
+    return x, Ak, Av, lat, sc
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_prefill_equals_successive_appends(bits):
+    """The block write is the rows that T single-token appends write, one after
+    the other (and T = 1 is the append itself)."""
+    r, T = 8, 4
+    x, Ak, Av, lat, sc = _prefill_case(21, T=T, r=r, bits=bits)
+    lens = np.array([0, 2, 5], np.int32)  # 5 + 4 = 9 = L_cap: fits exactly
+    got = O.latent_prefill(x, Ak, Av, lens, lat, sc, lat, sc, r, bits, 128)
+    state = [lat, sc, lat, sc, lens]
+    for t in range(T):
+        lk, sk, lv, sv, nl, err, _, _ = O.latent_append(x[:, t], Ak, Av, state[4], state[0], state[1], state[2],
+                                                        state[3], r, bits, 128)
+        assert not err.any()
+        state = [lk, sk, lv, sv, nl]
+    for g, s in zip(got[:5], state):
+        assert np.array_equal(g, s)
+    assert not got[5].any()
+    one = O.latent_prefill(x[:, :1], Ak, Av, lens, lat, sc, lat, sc, r, bits, 128)
+    app = O.latent_append(x[:, 0], Ak, Av, lens, lat, sc, lat, sc, r, bits, 128)
+    for g, s in zip(one[:6], app[:6]):
+        assert np.array_equal(g, s)
+
+
+def test_prefill_projection_is_one_dense_matmul():
+    """c[b,t,h] = (x[b,t] . blockdiag(H/sqrt(blk))) . A_h as one library matmul
+    over all B*T rows: catches a transposed rotation, a swapped head index or a
+    token mixed into another token's row."""
+    x, Ak, Av, lat, sc = _prefill_case(22, B=2, T=5, H=3, E=256, r=8, L_cap=5)
+    Hn = scipy.linalg.hadamard(128) / math.sqrt(128)
+    Rt = scipy.linalg.block_diag(Hn, Hn)
+    X = x.reshape(-1, 256) @ Rt
+    _, _, _, _, _, _, ck, cv = O.latent_prefill(x, Ak, Av, np.zeros(2, np.int32), lat, sc, lat, sc, 8, 8, 128)
+    for h in range(3):
+        assert np.allclose(ck[:, :, h].reshape(-1, 8), X @ Ak[h].astype(np.float64), rtol=1e-12, atol=1e-12)
+        assert np.allclose(cv[:, :, h].reshape(-1, 8), X @ Av[h].astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_capacity_boundary_and_empty_block():
+    x, Ak, Av, lat, sc = _prefill_case(23, T=4, L_cap=9)
+    lens = np.array([6, -1, 5], np.int32)  # 6 + 4 > 9 refused; negative refused; 5 + 4 = 9 fits
+    lk, sk, lv, sv, nl, err, _, _ = O.latent_prefill(x, Ak, Av, lens, lat, sc, lat, sc, 8, 8, 128)
+    assert list(err) == [True, True, False] and list(nl) == [6, -1, 9]
+    for b in (0, 1):
+        assert np.array_equal(lk[b], lat[b]) and np.array_equal(sk[b], sc[b])
+        assert np.array_equal(lv[b], lat[b]) and np.array_equal(sv[b], sc[b])
+    assert np.array_equal(lk[2, :, :5], lat[2, :, :5]) and not np.array_equal(lk[2, :, 5:], lat[2, :, 5:])
+    e = O.latent_prefill(x[:, :0], Ak, Av, lens, lat, sc, lat, sc, 8, 8, 128)
+    assert np.array_equal(e[0], lat) and np.array_equal(e[4], np.array([6, -1, 5], np.int32)) and e[5][1]
+
+
 # ----------------------------------------------------------------------------- footprint
 def test_footprint_against_pages_and_arrays():
     g = {t[0]: float(t[1]) for t in _golden_lines("footprint.txt")}

@@ -268,6 +268,16 @@ def append_inputs(w: Workload, seed: int = 0, steps: Optional[int] = None) -> Ap
     return AppendInputs(w, xv, xb, ak, av)
 
 
+def prefill_inputs(w: Workload, seed: int = 0, T: int = 576) -> AppendInputs:
+    """A block of T new tokens per sequence for the prefill latent write: the
+    append recipe drawn for T steps and laid out [B][T][E], so that token t of
+    the block is the activation step t of successive appends would take
+    (x has shape [B][T][E] here, not [steps][B][E])."""
+    ai = append_inputs(w, seed, steps=T)
+    return AppendInputs(w, np.ascontiguousarray(ai.x.transpose(1, 0, 2)),
+                        np.ascontiguousarray(ai.x_bits.transpose(1, 0, 2)), ai.A_k, ai.A_v)
+
+
 def latent_rotation(w: Workload, seed: int = 0, which: str = "k") -> np.ndarray:
     """Synthetic orthogonal latent rotations S2 [H][r][r] (float32): the Q
     factor of a Gaussian matrix per head, sign-fixed so that diag(R) > 0."""
