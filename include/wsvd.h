@@ -189,6 +189,39 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
                        uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
                        size_t workspace_bytes, int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- prefill latent write
+ * Writes a block of T new tokens per sequence (a prompt, e.g. the image tokens
+ * of a vision-language prompt) into the latent cache in one call: token t of
+ * sequence b is rotated, projected and quantised as by wsvd_latent_append
+ * (German §2.A projection, German §2.C rotation S1 and W8A8 / W8A4 quantiser)
+ * and stored at row seq_lens[b] + t; then seq_lens[b] += T.  The pages give
+ * no block interface; the rows written are those of T successive appends.
+ * A sequence with seq_lens[b] < 0 or seq_lens[b] + T > L_cap is not written
+ * and not advanced; WSVD_DEVERR_CACHE_FULL is raised.
+ * The projection runs as a GEMM on the tensor cores: the rotated activations
+ * are split into two fp16 halves (hi + lo, 22 significant bits after an exact
+ * per-token power-of-two scaling), each multiplied by the fp16 weights with
+ * fp32 accumulation.
+ *
+ *   x          [B][T][E]    bf16 or fp16 (x_dtype); the rotated values times
+ *                           their power-of-two scale must stay finite in fp16
+ *                           (any finite bf16 input does).
+ *   A_k, A_v   [H][E][r]    fp16.
+ *   hadamard_block          power of two in [1, 1024], E % hadamard_block == 0.
+ *   E                       multiple of 32, at most 16384.
+ *   r                       8, 16, 32, 64 or 128.
+ *   seq_lens   [B]          int32, read and advanced in place.
+ *   workspace               at least wsvd_prefill_workspace_size(B, T, E)
+ *                           bytes (the split rotated activations; no zeroing
+ *                           needed).  Calls that share it must not overlap.
+ * T = 0 (or B = 0) launches nothing.  Three launches otherwise (rotate,
+ * GEMM + quantiser, length advance), all on `stream`.                       */
+size_t wsvd_prefill_workspace_size(int B, int T, int E);
+int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, int L_cap, int hadamard_block,
+                        const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
+                        uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
+                        size_t workspace_bytes, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------- one decode step
  * wsvd_latent_append followed by wsvd_decode_attention on the same stream: the
  * decode step of the method (append the new token's latents, then attend over

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libwsvd_b200.so")
-SOURCES = ["api.cu", "decode.cu", "shared.cu", "append.cu", "noalloc.cu", "fold.cu"]
+SOURCES = ["api.cu", "decode.cu", "shared.cu", "append.cu", "noalloc.cu", "fold.cu", "prefill.cu"]
 HEADERS = ["common.cuh", "wsvd_internal.h"]
 
 NVCC_FLAGS = [

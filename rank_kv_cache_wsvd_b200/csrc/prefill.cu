@@ -1,0 +1,365 @@
+// Prefill latent write for sm_100a: a block of T new tokens per sequence (a
+// prompt, e.g. the image tokens of a vision-language prompt) is rotated by the
+// block Hadamard S1, projected through A_Kh / A_Vh and quantised into cache
+// rows seq_lens[b] .. seq_lens[b] + T - 1 (WSVD summaries: German §2.A for the
+// per-head projection, German §2.C for S1 and the W8A8 / W8A4 quantiser; every
+// row is the one a single-token append of that token would write).
+//
+// Unlike the one-token append (a GEMV bound by reading A), the block is a real
+// GEMM: C[M x N] = X~[M x E] . W[E x N] with M = B*T token rows and
+// N = 2*H*r latent columns (K heads, then V heads), W[e][n] = A_kv[h][e][j].
+// Three launches:
+//   1. prefill_rotate_kernel: one CTA per token row rotates it in shared
+//      memory (normalised FWHT), scales it by a power of two p_m (exact) so
+//      that its largest element lies in [2^14, 2^15), and splits every value v
+//      into two fp16 halves hi + lo = v to within 2^-22 relative;
+//   2. prefill_gemm_kernel: 64 x 128 output tiles on the tensor cores
+//      (mma.sync m16n8k16, fp16 x fp16 -> fp32), the hi and the lo operand
+//      each multiplied by the same fp16 weight fragment, so that the product
+//      carries the rotated activation to fp32-like precision (one fp16
+//      product alone would move the codes by up to a few hundredths of a
+//      step, far more than the quantiser's rounding ties allow); tiles stream
+//      through a three-stage cp.async ring; the epilogue stages the fp32
+//      tile in shared memory, undoes p_m (exact) and quantises each
+//      (token, head) row of r values with one warp: amax, fp16 scale,
+//      round-half-even codes, row write;
+//   3. prefill_advance_kernel: seq_lens[b] += T, or the block is refused.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace wsvd {
+
+namespace {
+
+constexpr int kRotThreads = 256;
+constexpr int kBM = 64, kBN = 128, kBK = 32;
+constexpr int kGemmThreads = 256;  // 8 warps: 2 along M x 4 along N, 32 x 32 outputs each
+constexpr int kStages = 3;
+constexpr int kAStride = kBK + 8;  // halves per shared row of an activation tile (80 B: the 8 rows of an
+                                   // ldmatrix phase land on distinct 16-byte bank groups)
+constexpr int kBStride = kBN + 8;  // halves per shared row of the weight tile (272 B, same reason)
+constexpr int kCStride = kBN + 4;  // floats per shared row of the epilogue tile
+constexpr int kATileHalves = kBM * kAStride;
+constexpr int kBTileHalves = kBK * kBStride;
+constexpr int kStageHalves = 2 * kATileHalves + kBTileHalves;  // hi, lo, weights
+constexpr size_t kGemmSmem = std::max<size_t>((size_t)kStages * kStageHalves * 2, (size_t)kBM * kCStride * 4);
+
+struct PrefillArgs {
+  int B, T, M, H, E, r, bits, L_cap, N;
+  const __half* xhi;  // [M][E]
+  const __half* xlo;  // [M][E]
+  const float* inv_p; // [M]: 1 / p_m
+  const __half* Ak;   // [H][E][r]
+  const __half* Av;
+  const int32_t* seq_lens;
+  uint8_t* lat_k;
+  uint8_t* lat_v;
+  __half* scale_k;
+  __half* scale_v;
+};
+
+__device__ __forceinline__ float x_value(uint16_t bits16, int dtype) {
+  return dtype == WSVD_DTYPE_BF16 ? __uint_as_float((uint32_t)bits16 << 16) : __half2float(__ushort_as_half(bits16));
+}
+
+// ------------------------------------------------------------------ 1. rotate + split
+__global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void* x, int x_dtype, int E, int blk,
+                                                                     float hnorm, __half* xhi, __half* xlo,
+                                                                     float* inv_p) {
+  extern __shared__ __align__(16) float xs[];
+  __shared__ float wmax[kRotThreads / 32];
+  const int m = blockIdx.x, tid = threadIdx.x;
+  const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)m * E;
+  for (int i = tid; i < E; i += kRotThreads) xs[i] = x_value(xr[i], x_dtype);
+  __syncthreads();
+  // Butterfly stages of distance 1, 2, ..., blk/2: pairs (i, i + hh) with bit
+  // hh of i clear never leave an aligned block of blk values (Sylvester order).
+  for (int hh = 1; hh < blk; hh <<= 1) {
+    for (int q = tid; q < E / 2; q += kRotThreads) {
+      const int i = (q / hh) * 2 * hh + (q % hh);
+      const float u = xs[i], v = xs[i + hh];
+      xs[i] = u + v;
+      xs[i + hh] = u - v;
+    }
+    __syncthreads();
+  }
+  float amax = 0.f;
+  for (int i = tid; i < E; i += kRotThreads) {
+    const float v = xs[i] * hnorm;
+    xs[i] = v;
+    amax = fmaxf(amax, fabsf(v));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((tid & 31) == 0) wmax[tid >> 5] = amax;
+  __syncthreads();
+  amax = 0.f;
+#pragma unroll
+  for (int w = 0; w < kRotThreads / 32; ++w) amax = fmaxf(amax, wmax[w]);
+  // p = 2^k with amax * p in [2^14, 2^15) for a normal amax (amax in [2^e, 2^(e+1)));
+  // k is clamped so that both 2^k and 2^-k are normal floats.
+  int k = 0;
+  if (amax > 0.f) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+    k = max(-126, min(126, 14 - e));
+  }
+  const float p = __uint_as_float((uint32_t)(127 + k) << 23);
+  for (int i = tid; i < E; i += kRotThreads) {
+    const float v = xs[i] * p;
+    const __half hi = __float2half_rn(v);
+    xhi[(size_t)m * E + i] = hi;
+    xlo[(size_t)m * E + i] = __float2half_rn(v - __half2float(hi));
+  }
+  if (tid == 0) inv_p[m] = __uint_as_float((uint32_t)(127 - k) << 23);
+}
+
+// ------------------------------------------------------------------ 2. GEMM + quantise
+// 16-byte cp.async; a false `valid` copies nothing and zero-fills the destination.
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// d += a . b for one 16 x 8 x 16 tile (fp16 operands, fp32 accumulators).
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Stage k-tile kt of the CTA's operands: activation rows m0.. (hi and lo: one
+// 16-byte piece each per thread) and weight rows k0.. x columns n0.. (two
+// pieces per thread; a piece is 8 consecutive latent columns of one head).
+__device__ __forceinline__ void load_stage(const PrefillArgs& a, __half* st, int m0, int n0, int kt, int tid) {
+  const int k0 = kt * kBK;
+  {
+    const int row = tid >> 2, ch = tid & 3;
+    const bool ok = m0 + row < a.M;
+    const size_t off = ok ? (size_t)(m0 + row) * a.E + k0 + ch * 8 : 0;
+    cp_async16_zfill(st + row * kAStride + ch * 8, a.xhi + off, ok);
+    cp_async16_zfill(st + kATileHalves + row * kAStride + ch * 8, a.xlo + off, ok);
+  }
+  const int HR = a.H * a.r;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int idx = tid + i * kGemmThreads;
+    const int krow = idx >> 4, ch = idx & 15;
+    const int n = n0 + ch * 8;
+    const bool ok = n < a.N;
+    const __half* src = a.Ak;
+    if (ok) {
+      const int kv = n / HR, rem = n - kv * HR;
+      const int h = rem / a.r, j = rem - h * a.r;
+      src = (kv ? a.Av : a.Ak) + ((size_t)h * a.E + k0 + krow) * a.r + j;
+    }
+    cp_async16_zfill(st + 2 * kATileHalves + krow * kBStride + ch * 8, src, ok);
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const PrefillArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __half* sm = reinterpret_cast<__half*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 2, wn = warp & 3;  // warp tile: rows wm*32.., columns wn*32..
+  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
+  const int KT = a.E / kBK;
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[i][j][k] = 0.f;
+
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < KT) load_stage(a, sm + s * kStageHalves, m0, n0, s, tid);
+    cp_async_commit_group();
+  }
+  for (int kt = 0; kt < KT; ++kt) {
+    cp_async_wait_group<kStages - 2>();  // k-tile kt has landed (this thread's copies)
+    __syncthreads();                     // everyone's copies; and slot (kt - 1) % kStages is free
+    {
+      const int nk = kt + kStages - 1;
+      if (nk < KT) load_stage(a, sm + (nk % kStages) * kStageHalves, m0, n0, nk, tid);
+      cp_async_commit_group();
+    }
+    const __half* st = sm + (kt % kStages) * kStageHalves;
+    const uint32_t ahi_base = smem_u32(st), alo_base = smem_u32(st + kATileHalves),
+                   b_base = smem_u32(st + 2 * kATileHalves);
+#pragma unroll
+    for (int kk = 0; kk < kBK; kk += 16) {
+      uint32_t ahi[2][4], alo[2][4], bq[2][4];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        const uint32_t off = (uint32_t)(((wm * 32 + mi * 16 + (lane & 15)) * kAStride + kk + (lane >> 4) * 8) * 2);
+        ldmatrix_x4(ahi[mi], ahi_base + off);
+        ldmatrix_x4(alo[mi], alo_base + off);
+      }
+#pragma unroll
+      for (int nj = 0; nj < 2; ++nj) {
+        const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = wn * 32 + nj * 16 + (lane >> 4) * 8;
+        ldmatrix_x4_trans(bq[nj], b_base + (uint32_t)((krow * kBStride + col) * 2));
+      }
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+          const uint32_t b0 = bq[ni >> 1][(ni & 1) * 2], b1 = bq[ni >> 1][(ni & 1) * 2 + 1];
+          mma_16816(acc[mi][ni], ahi[mi], b0, b1);
+          mma_16816(acc[mi][ni], alo[mi], b0, b1);
+        }
+    }
+  }
+  cp_async_wait_group<0>();
+  __syncthreads();  // every warp is done with the ring: it becomes the epilogue tile
+
+  float* cs = reinterpret_cast<float*>(smem_raw);
+  {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < 4; ++ni) {
+        const int row = wm * 32 + mi * 16 + g, col = wn * 32 + ni * 8 + 2 * t;
+        *reinterpret_cast<float2*>(cs + row * kCStride + col) = make_float2(acc[mi][ni][0], acc[mi][ni][1]);
+        *reinterpret_cast<float2*>(cs + (row + 8) * kCStride + col) = make_float2(acc[mi][ni][2], acc[mi][ni][3]);
+      }
+  }
+  __syncthreads();
+
+  // One warp per (token row, head) unit of r columns; lane owns j = lane + 32q.
+  const int Q = a.bits == 8 ? 127 : 7;
+  const int RB = a.r * a.bits / 8;
+  const int HR = a.H * a.r;
+  const int heads = kBN / a.r;
+  for (int u = warp; u < kBM * heads; u += kGemmThreads / 32) {
+    const int i = u / heads, hh = u - i * heads;
+    const int m = m0 + i, n = n0 + hh * a.r;
+    if (m >= a.M || n >= a.N) continue;  // warp-uniform
+    const int b = m / a.T, t = m - b * a.T;
+    const int pos = a.seq_lens[b];
+    if (pos < 0 || (long long)pos + a.T > a.L_cap) continue;  // refused block (flagged by the advance kernel)
+    const int kv = n / HR, h = (n - kv * HR) / a.r;
+    const float ip = a.inv_p[m];
+    float cv[4];
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = lane + 32 * q;
+      cv[q] = j < a.r ? cs[i * kCStride + hh * a.r + j] * ip : 0.f;
+      amax = fmaxf(amax, fabsf(cv[q]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
+    const float sc = __half2float(sh);
+    const size_t row = ((size_t)b * a.H + h) * a.L_cap + pos + t;
+    uint8_t* dst = (kv ? a.lat_v : a.lat_k) + row * RB;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = lane + 32 * q;
+      const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(cv[q], sc)))) : 0;
+      if (a.bits == 8) {
+        if (j < a.r) dst[j] = (uint8_t)code;
+      } else {
+        const int hi = __shfl_down_sync(0xffffffffu, code, 1);  // column j + 1 (r is a multiple of 8)
+        if (j < a.r && (lane & 1) == 0) dst[j / 2] = (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+      }
+    }
+    if (lane == 0) (kv ? a.scale_v : a.scale_k)[row] = sh;
+  }
+}
+
+// ------------------------------------------------------------------ 3. lengths
+__global__ void prefill_advance_kernel(int32_t* seq_lens, int B, int T, int L_cap, int32_t* err) {
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int pos = seq_lens[b];
+    if (pos >= 0 && (long long)pos + T <= L_cap) seq_lens[b] = pos + T;
+    else set_err(err, WSVD_DEVERR_CACHE_FULL);
+  }
+}
+
+inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+}  // namespace wsvd
+
+extern "C" size_t wsvd_prefill_workspace_size(int B, int T, int E) {
+  if (B < 1 || T < 1 || E < 1) return 0;
+  const size_t M = (size_t)B * T;
+  return 2 * wsvd::align16(M * E * 2) + wsvd::align16(M * 4);
+}
+
+extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, int L_cap, int hadamard_block,
+                                   const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
+                                   uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,
+                                   size_t workspace_bytes, int32_t* err, void* stream) {
+  using namespace wsvd;
+  if (B < 0 || T < 0 || H < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return WSVD_OK;
+  if (bits != 8 && bits != 4) return WSVD_ERR_INVALID_ARG;
+  if (x_dtype != WSVD_DTYPE_FP16 && x_dtype != WSVD_DTYPE_BF16) return WSVD_ERR_INVALID_ARG;
+  if (hadamard_block < 1 || hadamard_block > 1024 || (hadamard_block & (hadamard_block - 1)))
+    return WSVD_ERR_INVALID_ARG;
+  if (E % hadamard_block) return WSVD_ERR_INVALID_ARG;
+  if (r % 8 || 128 % r || E % kBK || E > 16384) return WSVD_ERR_UNSUPPORTED;
+  const long long M = (long long)B * T, N = 2LL * H * r;
+  if (M > (1LL << 30) || (M + kBM - 1) / kBM > 0x7fffffffLL || (N + kBN - 1) / kBN > 65535) return WSVD_ERR_UNSUPPORTED;
+  if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
+    return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
+      !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
+    return WSVD_ERR_INVALID_ARG;
+  if (workspace_bytes < wsvd_prefill_workspace_size(B, T, E)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const size_t xbytes = align16((size_t)M * E * 2);
+  PrefillArgs a{};
+  a.B = B; a.T = T; a.M = (int)M; a.H = H; a.E = E; a.r = r; a.bits = bits; a.L_cap = L_cap; a.N = (int)N;
+  a.xhi = reinterpret_cast<const __half*>(w);
+  a.xlo = reinterpret_cast<const __half*>(w + xbytes);
+  a.inv_p = reinterpret_cast<const float*>(w + 2 * xbytes);
+  a.Ak = static_cast<const __half*>(A_k);
+  a.Av = static_cast<const __half*>(A_v);
+  a.seq_lens = seq_lens;
+  a.lat_k = lat_k; a.lat_v = lat_v;
+  a.scale_k = static_cast<__half*>(scale_k); a.scale_v = static_cast<__half*>(scale_v);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t rot_smem = (size_t)E * 4;
+  if (cudaFuncSetAttribute(prefill_rotate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rot_smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(prefill_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) !=
+          cudaSuccess)
+    return WSVD_ERR_CUDA;
+  prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(
+      x, x_dtype, E, hadamard_block, (float)(1.0 / sqrt((double)hadamard_block)), reinterpret_cast<__half*>(w),
+      reinterpret_cast<__half*>(w + xbytes), reinterpret_cast<float*>(w + 2 * xbytes));
+  const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)((N + kBN - 1) / kBN));
+  prefill_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(a);
+  prefill_advance_kernel<<<1, 128, 0, s>>>(seq_lens, B, T, L_cap, err);
+  return cudaGetLastError() == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
+}

@@ -109,3 +109,27 @@ def test_decode_launch_count_rejects_bad_sizes(lib):
     assert W.wsvd_decode_launch_count(1, 32, 128, 32, 5, 1600) == 0
     assert W.wsvd_decode_launch_count(1, 32, 128, 3, 4, 1600) == 0  # r * bits not a whole byte
     assert W.wsvd_decode_launch_count(1, 32, 128, 24, 8, 1600) == 0  # 24-byte rows are not instantiated
+
+
+def test_prefill_workspace_and_host_validation(lib):
+    """The prefill scratch holds the split rotated activations (two fp16 copies
+    of the B x T x E block) and one power-of-two scale per token row; bad
+    shapes are refused before anything is launched."""
+    a16 = lambda v: (v + 15) // 16 * 16
+    assert W.wsvd_prefill_workspace_size(1, 576, 4096) == 2 * a16(576 * 4096 * 2) + a16(576 * 4)
+    assert W.wsvd_prefill_workspace_size(0, 576, 4096) == 0
+    p = ctypes.c_void_p(16)
+    ws = W.wsvd_prefill_workspace_size(2, 3, 256)
+    args = lambda B=2, T=3, H=4, E=256, r=16, bits=8, L=64, blk=128, ptr=p, nbytes=ws: (
+        B, T, H, E, r, bits, L, blk, ptr, 1, p, p, p, p, p, p, p, p, nbytes, None, None)
+    assert lib.wsvd_latent_prefill(*args(blk=96)) == 1            # block not a power of two
+    assert lib.wsvd_latent_prefill(*args(bits=6)) == 1            # bits not in {4, 8}
+    assert lib.wsvd_latent_prefill(*args(r=24)) == 2              # r must divide the 128-column tile
+    assert lib.wsvd_latent_prefill(*args(E=272, blk=16)) == 2     # E not a multiple of the 32-wide k tile
+    assert lib.wsvd_latent_prefill(*args(E=32768)) == 2           # row does not fit the rotation's shared memory
+    assert lib.wsvd_latent_prefill(*args(ptr=ctypes.c_void_p(24))) == 1  # misaligned x
+    assert lib.wsvd_latent_prefill(*args(ptr=None)) == 1          # null x
+    assert lib.wsvd_latent_prefill(*args(nbytes=ws - 16)) == 4    # workspace too small
+    assert lib.wsvd_latent_prefill(*args(T=0, ptr=None)) == 0     # empty block: nothing launched
+    assert lib.wsvd_latent_prefill(*args(B=0, ptr=None)) == 0
+    assert lib.wsvd_latent_prefill(*args(T=-1)) == 1
