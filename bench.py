@@ -284,6 +284,60 @@ def time_comparisons(w: WL.Workload, steps: int, warmup: int, flush):
     return res
 
 
+def time_prefill(w: WL.Workload, T: int, steps: int, warmup: int, flush):
+    """The prefill latent write of a T-token block per sequence (the image
+    tokens of the prompt) into an empty cache: device time per call, events
+    around it, L2 flushed and the lengths reset before each call.  The work is
+    a GEMM [B*T x E] . [E x 2*H*r]; the kernels multiply it twice (the hi and
+    lo fp16 halves of the rotated activations), so the tensor-core FLOPs are
+    twice the useful ones."""
+    import torch
+
+    import rank_kv_cache_wsvd_b200 as W
+    pi = WL.prefill_inputs(w, seed=0, T=T)
+    x = torch.from_numpy(pi.x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    A_k, A_v = torch.from_numpy(pi.A_k).cuda(), torch.from_numpy(pi.A_v).cuda()
+    L_cap = max(w.L_cap, T)
+    rb = w.r * w.bits // 8
+    lk = torch.zeros((w.B, w.H, L_cap, rb), dtype=torch.uint8, device="cuda")
+    lv = torch.zeros_like(lk)
+    sk = torch.zeros((w.B, w.H, L_cap), dtype=torch.float16, device="cuda")
+    sv = torch.zeros_like(sk)
+    lens = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = W.workspace(W.wsvd_prefill_workspace_size(w.B, T, w.E))
+    call = lambda: W.wsvd_latent_prefill(x, A_k, A_v, lens, lk, lv, sk, sv, bits=w.bits,
+                                         hadamard_block=w.hadamard_block, workspace_buf=ws, err=err)
+    for _ in range(max(3, warmup)):
+        lens.zero_()
+        call()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        lens.zero_()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"prefill device error word {int(err.item())}")
+    t = sum(a.elapsed_time(b) for a, b in evs) / 1e3 / steps
+    M, N = w.B * T, 2 * w.H * w.r
+    flops = 2.0 * M * w.E * N
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak = json.load(open(pk))["bf16_tflops"] if os.path.exists(pk) else 1590.0
+    return {"T": T, "us": t * 1e6, "launches": 3, "useful_tflops": flops / t / 1e12,
+            "tensor_tflops": 2 * flops / t / 1e12, "peak_tflops": peak,
+            "peak_kind": "measured bf16 burst (fp16 has the same nominal rate)" if os.path.exists(pk) else "fallback",
+            "frac_useful": flops / t / 1e12 / peak, "frac_tensor": 2 * flops / t / 1e12 / peak,
+            "weights_bytes": 2 * w.H * w.E * w.r * 2, "activation_bytes": M * w.E * 2,
+            "note": "mma.sync m16n8k16 fp16 tiles (hi + lo split of the rotated activations)"}
+
+
 def _time_loop(fn, steps, warmup, flush):
     """Device time per call of `fn`: events on the launching stream around the
     call; before each call the L2 is flushed and a device sleep keeps the host
@@ -358,6 +412,40 @@ def sample_heads(w: WL.Workload) -> int:
     return max(1, min(w.H, 12800 // max(1, per_head_tokens)))
 
 
+def run_prefill_line(w: WL.Workload, args, world: int, rank: int, barrier):
+    """`--op prefill`: one JSON line for the prompt-block latent write (tokens
+    written per second), each rank an independent replica."""
+    import torch
+    if not w.prefill_tokens:
+        raise SystemExit(f"workload {w.name} has no prefill block")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    barrier()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.25)
+    pf = time_prefill(w, w.prefill_tokens, args.steps, args.warmup, flush)
+    clk = clocks.stop()
+    barrier()
+    t = pf["us"] * 1e-6
+    value, t_total = replica_throughput(w.B * w.prefill_tokens * args.steps, t * args.steps, world)
+    if rank == 0:
+        line = {
+            "metric": "prefill latent write: prompt tokens written into the low-rank cache per second",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16 (hi + lo split), f32 accumulate", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.prefill_tokens, "E": w.E, "H": w.H, "r": w.r,
+                       "latent_bits": w.bits, "l2": "flushed between timed calls (256 MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "prefill (rotate + GEMM/quantise + advance, 3 launches)",
+                         "achieved": pf["tensor_tflops"], "peak": pf["peak_tflops"], "unit": "TFLOP/s",
+                         "frac": pf["frac_tensor"], "peak_kind": pf["peak_kind"], "traffic": None,
+                         "useful_tflops": pf["useful_tflops"]},
+            "prefill": pf, "gpu_launches": 3 * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -370,6 +458,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the CPU baseline, e2e and comparison timings")
     ap.add_argument("--weights", default="fp16", choices=["fp16", "int8"],
                     help="low-rank factors A, B as fp16, or int8 with per-column scales (W8)")
+    ap.add_argument("--op", default="step", choices=["step", "prefill"],
+                    help="step: the decode step (append + decode); prefill: the prompt-block latent write alone")
     args = ap.parse_args()
     w = WL.PRESETS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -409,6 +499,12 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
+
+    if args.op == "prefill":
+        run_prefill_line(w, args, world, rank, barrier)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     w8 = args.weights == "int8"
     st = WsvdStep(w, seed=rank, w8=w8)
@@ -532,6 +628,8 @@ def main():
         extras["comparisons_same_shape"] = time_comparisons(w, min(args.steps, 200), 5, flush)
         extras["comparisons_same_shape"]["wsvd_decode"] = {"us": per_dec * 1e6, "alg_bytes": dec_bytes,
                                                            "gbs": dec_bytes / per_dec / 1e9}
+        if st.has_append and w.prefill_tokens:
+            extras["prefill"] = time_prefill(w, w.prefill_tokens, min(args.steps, 200), 5, flush)
         extras["cpu_baseline"] = run_cpu_sample(w, args.cpu_seconds, sample_heads(w))
 
     if rank == 0:
@@ -559,7 +657,7 @@ def main():
             "gpu_launches": st.launches_per_step * args.steps,
             "clocks": clk,
         }
-        for k in ("cpu_baseline", "e2e", "comparisons_same_shape"):
+        for k in ("cpu_baseline", "e2e", "comparisons_same_shape", "prefill"):
             if k in extras:
                 line[k] = extras[k]
         print(json.dumps(line), flush=True)

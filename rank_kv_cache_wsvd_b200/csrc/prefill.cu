@@ -18,7 +18,9 @@
 //      each multiplied by the same fp16 weight fragment, so that the product
 //      carries the rotated activation to fp32-like precision (one fp16
 //      product alone would move the codes by up to a few hundredths of a
-//      step, far more than the quantiser's rounding ties allow); tiles stream
+//      step, far more than the quantiser's rounding ties allow); each 32-wide
+//      k-tile is accumulated from zero on the tensor cores and added to an
+//      fp32 register total; tiles stream
 //      through a three-stage cp.async ring; the epilogue stages the fp32
 //      tile in shared memory, undoes p_m (exact) and quantises each
 //      (token, head) row of r values with one warp: amax, fp16 scale,
@@ -206,6 +208,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
     const __half* st = sm + (kt % kStages) * kStageHalves;
     const uint32_t ahi_base = smem_u32(st), alo_base = smem_u32(st + kATileHalves),
                    b_base = smem_u32(st + 2 * kATileHalves);
+    // The tensor cores' fp32 accumulation is not round-to-nearest; a running
+    // sum held in the MMA accumulator over all of E drifts by a fraction of an
+    // ulp per MMA.  Each k-tile therefore starts from zero (four MMAs deep)
+    // and is added to the fp32 total with an ordinary rounded add.
+    float part[2][4][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) part[i][j][k] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < kBK; kk += 16) {
       uint32_t ahi[2][4], alo[2][4], bq[2][4];
@@ -226,10 +239,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 #pragma unroll
         for (int ni = 0; ni < 4; ++ni) {
           const uint32_t b0 = bq[ni >> 1][(ni & 1) * 2], b1 = bq[ni >> 1][(ni & 1) * 2 + 1];
-          mma_16816(acc[mi][ni], ahi[mi], b0, b1);
-          mma_16816(acc[mi][ni], alo[mi], b0, b1);
+          mma_16816(part[mi][ni], ahi[mi], b0, b1);
+          mma_16816(part[mi][ni], alo[mi], b0, b1);
         }
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[i][j][k] = __fadd_rn(acc[i][j][k], part[i][j][k]);
   }
   cp_async_wait_group<0>();
   __syncthreads();  // every warp is done with the ring: it becomes the epilogue tile

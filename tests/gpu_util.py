@@ -62,13 +62,17 @@ def _fp16_neighbours(x32: np.ndarray):
     return lo, hi, (lo.astype(np.float64) + hi.astype(np.float64)) / 2
 
 
-def compare_codes(g_codes, g_scale, o_codes, o_scale, o_c, bits: int, tie_tol: float = 1e-3):
+def compare_codes(g_codes, g_scale, o_codes, o_scale, o_c, bits: int, tie_tol: float = 1e-3,
+                  scale_tol: float = 2.0 ** -20, stats: dict = None):
     """Codes must match the oracle exactly except +-1 at counted rounding ties.
 
     A code tie: the oracle's float32 ratio v = c / scale has |frac(|v|) - 0.5| <=
-    tie_tol.  A scale tie: the oracle's float32 max|c| / Q lies within 2^-20
-    (relative) of an fp16 rounding midpoint; then the GPU scale may be the other
-    neighbour and every code of that row may move by +-1.
+    tie_tol.  A scale tie: the oracle's float32 max|c| / Q lies within scale_tol
+    (relative; 2^-20 for the fp32 paths) of an fp16 rounding midpoint; then the
+    GPU scale may be the other neighbour and every code of that row may move by
+    +-1.  `stats`, if given, collects the largest distance to the tie of every
+    accepted mismatch ("scale_dist" relative, "code_dist" in code units): a
+    measure of the kernel's error.
     Returns (n_code_ties, n_scale_ties)."""
     Q = 127 if bits == 8 else 7
     g_codes = np.asarray(g_codes, np.int64).reshape(-1, np.shape(g_codes)[-1])
@@ -84,7 +88,10 @@ def compare_codes(g_codes, g_scale, o_codes, o_scale, o_c, bits: int, tie_tol: f
         lo, hi, mid = _fp16_neighbours(ratio)
         bad = np.nonzero(~same_scale)[0]
         for i in bad:
-            near = abs(float(ratio[i]) - mid[i]) <= 2.0 ** -20 * abs(float(ratio[i]))
+            dist = abs(float(ratio[i]) - mid[i]) / max(abs(float(ratio[i])), 1e-30)
+            if stats is not None:
+                stats["scale_dist"] = max(stats.get("scale_dist", 0.0), dist)
+            near = dist <= scale_tol
             other_ok = float(g_scale[i]) in (float(lo[i]), float(hi[i]))
             assert near and other_ok, f"row {i}: scale {g_scale[i]} vs oracle {o_scale[i]} is not a rounding tie"
             assert np.all(np.abs(g_codes[i] - o_codes[i]) <= 1), f"row {i}: codes off by more than 1"
@@ -97,6 +104,8 @@ def compare_codes(g_codes, g_scale, o_codes, o_scale, o_c, bits: int, tie_tol: f
         s32 = o_scale[rows].astype(np.float32)[:, None]
         v = np.where(s32 > 0, c32[rows] / np.where(s32 > 0, s32, 1), 0).astype(np.float64)
         frac = np.abs(np.abs(v) - np.floor(np.abs(v)) - 0.5)
+        if stats is not None:
+            stats["code_dist"] = max(stats.get("code_dist", 0.0), float(frac[mism].max()))
         for i, j in zip(*mism):
             assert abs(d[i, j]) == 1 and frac[i, j] <= tie_tol, \
                 f"row {rows[i]} col {j}: gpu {g_codes[rows[i], j]} oracle {o_codes[rows[i], j]} v={v[i, j]!r}"

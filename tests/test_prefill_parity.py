@@ -14,6 +14,15 @@ from gpu_util import compare_codes, dev, q_tensor, unpack
 
 pytestmark = pytest.mark.gpu
 
+# Tie windows of the prefill.  Its latents come from the tensor cores: each
+# 32-wide k-tile is summed on them from zero (hi and lo halves, four MMAs
+# deep, fp32 accumulation that rounds toward zero) and the k-tiles are added
+# in fp32 with round-to-nearest, so c carries a few 1e-7 of max|c| more error
+# than the fp32 GEMV of the single-token append.  The scale window is four
+# times the append's 2^-20; the code window stays 1e-3 of a step.
+SCALE_TOL = 2.0 ** -18
+CODE_TOL = 1e-3
+
 
 @pytest.fixture(scope="module", autouse=True)
 def _lib():
@@ -50,6 +59,7 @@ def _run(w: WL.Workload, T: int, lens0, bits=None, blk=None, x_dtype="bf16", see
     gl = {k: v.cpu().numpy() for k, v in g.items()}
     assert np.array_equal(gl["lens"], olens), (gl["lens"], olens)
     ties = [0, 0]
+    stats = {}
     written = np.zeros((w.B, w.L_cap), bool)
     for b in range(w.B):
         pos = int(lens[b])
@@ -60,7 +70,8 @@ def _run(w: WL.Workload, T: int, lens0, bits=None, blk=None, x_dtype="bf16", see
             gc = unpack(gl["lat_" + which][b, :, pos:pos + T], w.r, bits)         # [H][T][r]
             oc = unpack((olk if which == "k" else olv)[b, :, pos:pos + T], w.r, bits)
             os_ = (osk if which == "k" else osv)[b, :, pos:pos + T]
-            t = compare_codes(gc, gl["s" + which][b, :, pos:pos + T], oc, os_, c[b].transpose(1, 0, 2), bits)
+            t = compare_codes(gc, gl["s" + which][b, :, pos:pos + T], oc, os_, c[b].transpose(1, 0, 2), bits,
+                              tie_tol=CODE_TOL, scale_tol=SCALE_TOL, stats=stats)
             ties[0] += t[0]
             ties[1] += t[1]
     # every byte outside the written rows is what it was before the call
@@ -70,6 +81,8 @@ def _run(w: WL.Workload, T: int, lens0, bits=None, blk=None, x_dtype="bf16", see
         keep = ~written[:, None, :]
         assert np.array_equal(np.where(keep[..., None] if a.ndim == 4 else keep, a, 0),
                               np.where(keep[..., None] if r_.ndim == 4 else keep, r_, 0)), key
+    print(f"prefill {w.name} T={T}: code ties {ties[0]}, scale ties {ties[1]}, largest distance to a tie "
+          f"(scale, relative) {stats.get('scale_dist', 0.0):.3g}, (code, steps) {stats.get('code_dist', 0.0):.3g}")
     return ties, int(err.item()), gl, bool(oerr.any())
 
 

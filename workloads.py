@@ -116,6 +116,7 @@ class Workload:
     x_outlier_frac: float = 0.0
     x_outlier_gain: float = 1.0
     R: int = 0  # shared-latent rank for the comparison paths (0 = not used)
+    prefill_tokens: int = 0  # prompt block written by one prefill call (0 = not measured)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -125,7 +126,7 @@ PR1 = Workload("pr1 b1 h4 hd64 r16 L256 int8", B=1, H=4, Hd=64, r=16, bits=8, L_
                q_dtype="fp16", E=256)
 LLAVA7B = Workload("llava7b-layer b1 h32 hd128 r32 L1600(576 vision+1024 text) int8 + append E4096",
                    B=1, H=32, Hd=128, r=32, bits=8, L_cap=1600, lens=1600, q_dtype="bf16",
-                   E=4096, append_steps=1)
+                   E=4096, append_steps=1, prefill_tokens=576)
 RAGGED = Workload("ragged b16 h32 hd128 r32 L~U[1024,4096] int4 student-t+outliers",
                   B=16, H=32, Hd=128, r=32, bits=4, L_cap=4096, lens=(1024, 4096), q_dtype="fp16",
                   latent="student_t_outliers")
