@@ -92,8 +92,9 @@ def test_llava_image_block_576_tokens():
     w = WL.LLAVA7B
     ties, err, g, _ = _run(w, 576, [0], seed=3)
     assert err == 0 and list(g["lens"]) == [576]
-    n_codes = 576 * w.H * 2 * w.r
-    assert ties[0] <= max(4, n_codes // 20000) and ties[1] <= 4, ties
+    n_rows = 576 * w.H * 2
+    # ties are rare: a code within CODE_TOL of a half step, a scale within SCALE_TOL of an fp16 midpoint
+    assert ties[0] <= max(4, n_rows * w.r // 20000) and ties[1] <= max(4, n_rows // 1000), ties
 
 
 def test_ragged_rows_int4_and_exact_fit():
@@ -128,8 +129,8 @@ def test_outlier_channels_long_context_recipe():
     w = WL.LONG[64].with_(L_cap=160)
     ties, err, g, _ = _run(w, 64, [0, 10, 96, 50], seed=11)
     assert err == 0 and list(g["lens"]) == [64, 74, 160, 114]
-    n_codes = 64 * w.B * w.H * 2 * w.r
-    assert ties[0] <= max(4, n_codes // 20000), ties
+    n_rows = 64 * w.B * w.H * 2
+    assert ties[0] <= max(4, n_rows * w.r // 20000) and ties[1] <= max(4, n_rows // 1000), ties
 
 
 def test_refused_blocks_are_flagged_and_untouched():
