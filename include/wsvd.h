@@ -208,7 +208,7 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
  *                           (any finite bf16 input does).
  *   A_k, A_v   [H][E][r]    fp16.
  *   hadamard_block          power of two in [1, 1024], E % hadamard_block == 0.
- *   E                       multiple of 32, at most 16384.
+ *   E                       multiple of 64, at most 16384.
  *   r                       8, 16, 32, 64 or 128.
  *   seq_lens   [B]          int32, read and advanced in place.
  *   workspace               at least wsvd_prefill_workspace_size(B, T, E)

@@ -18,9 +18,9 @@
 //      each multiplied by the same fp16 weight fragment, so that the product
 //      carries the rotated activation to fp32-like precision (one fp16
 //      product alone would move the codes by up to a few hundredths of a
-//      step, far more than the quantiser's rounding ties allow); each 32-wide
-//      k-tile is accumulated from zero on the tensor cores and added to an
-//      fp32 register total; tiles stream
+//      step, far more than the quantiser's rounding ties allow); each 64-wide
+//      k-tile of the hi half is accumulated from zero on the tensor cores and
+//      added to an fp32 register total; tiles stream
 //      through a three-stage cp.async ring; the epilogue stages the fp32
 //      tile in shared memory, undoes p_m (exact) and quantises each
 //      (token, head) row of r values with one warp: amax, fp16 scale,
@@ -35,10 +35,10 @@ namespace wsvd {
 namespace {
 
 constexpr int kRotThreads = 256;
-constexpr int kBM = 64, kBN = 128, kBK = 32;
+constexpr int kBM = 64, kBN = 128, kBK = 64;
 constexpr int kGemmThreads = 256;  // 8 warps: 2 along M x 4 along N, 32 x 32 outputs each
 constexpr int kStages = 3;
-constexpr int kAStride = kBK + 8;  // halves per shared row of an activation tile (80 B: the 8 rows of an
+constexpr int kAStride = kBK + 8;  // halves per shared row of an activation tile (144 B: the 8 rows of an
                                    // ldmatrix phase land on distinct 16-byte bank groups)
 constexpr int kBStride = kBN + 8;  // halves per shared row of the weight tile (272 B, same reason)
 constexpr int kCStride = kBN + 4;  // floats per shared row of the epilogue tile
@@ -147,13 +147,15 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Stage k-tile kt of the CTA's operands: activation rows m0.. (hi and lo: one
-// 16-byte piece each per thread) and weight rows k0.. x columns n0.. (two
+// Stage k-tile kt of the CTA's operands: activation rows m0.. (hi and lo: two
+// 16-byte pieces each per thread) and weight rows k0.. x columns n0.. (four
 // pieces per thread; a piece is 8 consecutive latent columns of one head).
 __device__ __forceinline__ void load_stage(const PrefillArgs& a, __half* st, int m0, int n0, int kt, int tid) {
   const int k0 = kt * kBK;
-  {
-    const int row = tid >> 2, ch = tid & 3;
+#pragma unroll
+  for (int i = 0; i < kBM * kBK / 8 / kGemmThreads; ++i) {
+    const int idx = tid + i * kGemmThreads;
+    const int row = idx / (kBK / 8), ch = idx % (kBK / 8);
     const bool ok = m0 + row < a.M;
     const size_t off = ok ? (size_t)(m0 + row) * a.E + k0 + ch * 8 : 0;
     cp_async16_zfill(st + row * kAStride + ch * 8, a.xhi + off, ok);
@@ -161,7 +163,7 @@ __device__ __forceinline__ void load_stage(const PrefillArgs& a, __half* st, int
   }
   const int HR = a.H * a.r;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < kBK * kBN / 8 / kGemmThreads; ++i) {
     const int idx = tid + i * kGemmThreads;
     const int krow = idx >> 4, ch = idx & 15;
     const int n = n0 + ch * 8;
@@ -184,13 +186,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
   const int KT = a.E / kBK;
 
-  float acc[2][4][4];
+  // acc: the hi half's products, k-tile by k-tile (below); acc_lo: the lo
+  // half's, kept on the tensor cores over all of E (its sum is ~2^-11 of c,
+  // so its drift is far below the hi half's rounding).  Separate accumulators
+  // also make the hi and lo MMAs independent of each other.
+  float acc[2][4][4], acc_lo[2][4][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[i][j][k] = 0.f;
+      for (int k = 0; k < 4; ++k) acc[i][j][k] = acc_lo[i][j][k] = 0.f;
 
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
@@ -210,8 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
                    b_base = smem_u32(st + 2 * kATileHalves);
     // The tensor cores' fp32 accumulation is not round-to-nearest; a running
     // sum held in the MMA accumulator over all of E drifts by a fraction of an
-    // ulp per MMA.  Each k-tile therefore starts from zero (four MMAs deep)
-    // and is added to the fp32 total with an ordinary rounded add.
+    // ulp per MMA.  Each k-tile of the hi half therefore starts from zero
+    // (four MMAs deep) and is added to the fp32 total with a rounded add.
     float part[2][4][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
         for (int ni = 0; ni < 4; ++ni) {
           const uint32_t b0 = bq[ni >> 1][(ni & 1) * 2], b1 = bq[ni >> 1][(ni & 1) * 2 + 1];
           mma_16816(part[mi][ni], ahi[mi], b0, b1);
-          mma_16816(part[mi][ni], alo[mi], b0, b1);
+          mma_16816(acc_lo[mi][ni], alo[mi], b0, b1);
         }
     }
 #pragma unroll
@@ -252,6 +258,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   }
   cp_async_wait_group<0>();
   __syncthreads();  // every warp is done with the ring: it becomes the epilogue tile
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[i][j][k] = __fadd_rn(acc[i][j][k], acc_lo[i][j][k]);
 
   float* cs = reinterpret_cast<float*>(smem_raw);
   {

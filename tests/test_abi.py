@@ -125,7 +125,7 @@ def test_prefill_workspace_and_host_validation(lib):
     assert lib.wsvd_latent_prefill(*args(blk=96)) == 1            # block not a power of two
     assert lib.wsvd_latent_prefill(*args(bits=6)) == 1            # bits not in {4, 8}
     assert lib.wsvd_latent_prefill(*args(r=24)) == 2              # r must divide the 128-column tile
-    assert lib.wsvd_latent_prefill(*args(E=272, blk=16)) == 2     # E not a multiple of the 32-wide k tile
+    assert lib.wsvd_latent_prefill(*args(E=272, blk=16)) == 2     # E not a multiple of the 64-wide k tile
     assert lib.wsvd_latent_prefill(*args(E=32768)) == 2           # row does not fit the rotation's shared memory
     assert lib.wsvd_latent_prefill(*args(ptr=ctypes.c_void_p(24))) == 1  # misaligned x
     assert lib.wsvd_latent_prefill(*args(ptr=None)) == 1          # null x

@@ -15,9 +15,9 @@ from gpu_util import compare_codes, dev, q_tensor, unpack
 pytestmark = pytest.mark.gpu
 
 # Tie windows of the prefill.  Its latents come from the tensor cores: each
-# 32-wide k-tile is summed on them from zero (hi and lo halves, four MMAs
-# deep, fp32 accumulation that rounds toward zero) and the k-tiles are added
-# in fp32 with round-to-nearest, so c carries a few 1e-7 of max|c| more error
+# 64-wide k-tile of the hi half is summed on them from zero (four MMAs deep,
+# fp32 accumulation that rounds toward zero) and the k-tiles are added in
+# fp32 with round-to-nearest, so c carries a few 1e-7 of max|c| more error
 # than the fp32 GEMV of the single-token append.  The scale window is four
 # times the append's 2^-20; the code window stays 1e-3 of a step.
 SCALE_TOL = 2.0 ** -18
