@@ -36,8 +36,13 @@ namespace {
 
 constexpr int kRotThreads = 256;
 constexpr int kBM = 64, kBN = 128, kBK = 64;
-constexpr int kGemmThreads = 512;  // 16 warps: 2 along M x 8 along N, 32 x 16 outputs each
-constexpr int kWarpsN = 8;
+constexpr int kWarpsN = 8;                      // warps along N (2 along M): 16 warps of 32 x 16 outputs
+constexpr int kGemmThreads = 64 * kWarpsN;
+constexpr int kWN = kBN / kWarpsN;              // columns per warp
+constexpr int kNI = kWN / 8;                    // n8 MMA tiles per warp
+constexpr int kNJ = kWN / 16;                   // ldmatrix.x4.trans per k16 step (two n8 tiles each)
+constexpr int kAPieces = kBM * kBK / 8 / kGemmThreads;   // 16-byte activation pieces per thread (hi and lo each)
+constexpr int kWPieces = kBK * kBN / 8 / kGemmThreads;   // 16-byte weight pieces per thread
 constexpr int kStages = 3;
 constexpr int kAStride = kBK + 8;  // halves per shared row of an activation tile (144 B: the 8 rows of an
                                    // ldmatrix phase land on distinct 16-byte bank groups)
@@ -153,25 +158,30 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // the weight tile (a piece is 8 consecutive latent columns of one head).  The
 // sources are resolved once, so a k-tile only adds its offset.
 struct CopyPlan {
-  const __half* xhi;    // row m0 + arow of the split activations, column ach * 8
-  const __half* xlo;
-  const __half* w[2];   // weight row krow of the piece's head, its first column
-  uint32_t a_dst, w_dst[2];
-  bool a_ok, w_ok[2];
+  const __half* xhi[kAPieces];  // row m0 + arow of the split activations, column ach * 8
+  const __half* xlo[kAPieces];
+  const __half* w[kWPieces];    // weight row krow of the piece's head, its first column
+  uint32_t a_dst[kAPieces], w_dst[kWPieces];
+  bool a_ok[kAPieces], w_ok[kWPieces];
 };
 
 __device__ __forceinline__ CopyPlan plan_copies(const PrefillArgs& a, int m0, int n0, int tid) {
-  static_assert(kBM * kBK / 8 == kGemmThreads && kBK * kBN / 8 == 2 * kGemmThreads, "one / two pieces per thread");
+  static_assert(kAPieces * kGemmThreads * 8 == kBM * kBK && kWPieces * kGemmThreads * 8 == kBK * kBN,
+                "whole pieces per thread");
   CopyPlan p;
-  const int arow = tid / (kBK / 8), ach = tid % (kBK / 8);
-  p.a_ok = m0 + arow < a.M;
-  const size_t aoff = p.a_ok ? (size_t)(m0 + arow) * a.E + ach * 8 : 0;
-  p.xhi = a.xhi + aoff;
-  p.xlo = a.xlo + aoff;
-  p.a_dst = (uint32_t)(arow * kAStride + ach * 8);
+#pragma unroll
+  for (int i = 0; i < kAPieces; ++i) {
+    const int idx = tid + i * kGemmThreads;
+    const int arow = idx / (kBK / 8), ach = idx % (kBK / 8);
+    p.a_ok[i] = m0 + arow < a.M;
+    const size_t aoff = p.a_ok[i] ? (size_t)(m0 + arow) * a.E + ach * 8 : 0;
+    p.xhi[i] = a.xhi + aoff;
+    p.xlo[i] = a.xlo + aoff;
+    p.a_dst[i] = (uint32_t)(arow * kAStride + ach * 8);
+  }
   const int HR = a.H * a.r;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < kWPieces; ++i) {
     const int idx = tid + i * kGemmThreads;
     const int krow = idx / (kBN / 8), ch = idx % (kBN / 8);
     const int n = n0 + ch * 8;
@@ -191,17 +201,20 @@ __device__ __forceinline__ CopyPlan plan_copies(const PrefillArgs& a, int m0, in
 // pointers stay inside the arrays but are not read).
 __device__ __forceinline__ void load_stage(const PrefillArgs& a, const CopyPlan& p, __half* st, int kt) {
   const int k0 = kt * kBK;
-  cp_async16_zfill(st + p.a_dst, p.xhi + k0, p.a_ok);
-  cp_async16_zfill(st + kATileHalves + p.a_dst, p.xlo + k0, p.a_ok);
 #pragma unroll
-  for (int i = 0; i < 2; ++i) cp_async16_zfill(st + p.w_dst[i], p.w[i] + (size_t)k0 * a.r, p.w_ok[i]);
+  for (int i = 0; i < kAPieces; ++i) {
+    cp_async16_zfill(st + p.a_dst[i], p.xhi[i] + k0, p.a_ok[i]);
+    cp_async16_zfill(st + kATileHalves + p.a_dst[i], p.xlo[i] + k0, p.a_ok[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kWPieces; ++i) cp_async16_zfill(st + p.w_dst[i], p.w[i] + (size_t)k0 * a.r, p.w_ok[i]);
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __half* sm = reinterpret_cast<__half*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp / kWarpsN, wn = warp % kWarpsN;  // warp tile: rows wm*32.., columns wn*16..
+  const int wm = warp / kWarpsN, wn = warp % kWarpsN;  // warp tile: rows wm*32.., columns wn*kWN..
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
   const int KT = a.E / kBK;
   const CopyPlan plan = plan_copies(a, m0, n0, tid);
@@ -210,11 +223,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   // half's, kept on the tensor cores over all of E (its sum is ~2^-11 of c,
   // so its drift is far below the hi half's rounding).  Separate accumulators
   // also make the hi and lo MMAs independent of each other.
-  float acc[2][2][4], acc_lo[2][2][4];
+  float acc[2][kNI][4], acc_lo[2][kNI][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < kNI; ++j)
 #pragma unroll
       for (int k = 0; k < 4; ++k) acc[i][j][k] = acc_lo[i][j][k] = 0.f;
 
@@ -238,39 +251,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
     // sum held in the MMA accumulator over all of E drifts by a fraction of an
     // ulp per MMA.  Each k-tile of the hi half therefore starts from zero
     // (four MMAs deep) and is added to the fp32 total with a rounded add.
-    float part[2][2][4];
+    float part[2][kNI][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+      for (int j = 0; j < kNI; ++j)
 #pragma unroll
         for (int k = 0; k < 4; ++k) part[i][j][k] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < kBK; kk += 16) {
-      uint32_t ahi[2][4], alo[2][4], bq[4];
+      uint32_t ahi[2][4], alo[2][4], bq[kNJ][4];
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi) {
         const uint32_t off = (uint32_t)(((wm * 32 + mi * 16 + (lane & 15)) * kAStride + kk + (lane >> 4) * 8) * 2);
         ldmatrix_x4(ahi[mi], ahi_base + off);
         ldmatrix_x4(alo[mi], alo_base + off);
       }
-      {
+#pragma unroll
+      for (int nj = 0; nj < kNJ; ++nj) {
         const int krow = kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int col = wn * 16 + (lane >> 4) * 8;
-        ldmatrix_x4_trans(bq, b_base + (uint32_t)((krow * kBStride + col) * 2));
+        const int col = wn * kWN + nj * 16 + (lane >> 4) * 8;
+        ldmatrix_x4_trans(bq[nj], b_base + (uint32_t)((krow * kBStride + col) * 2));
       }
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 2; ++ni) {
-          mma_16816(part[mi][ni], ahi[mi], bq[2 * ni], bq[2 * ni + 1]);
-          mma_16816(acc_lo[mi][ni], alo[mi], bq[2 * ni], bq[2 * ni + 1]);
+        for (int ni = 0; ni < kNI; ++ni) {
+          const uint32_t b0 = bq[ni >> 1][(ni & 1) * 2], b1 = bq[ni >> 1][(ni & 1) * 2 + 1];
+          mma_16816(part[mi][ni], ahi[mi], b0, b1);
+          mma_16816(acc_lo[mi][ni], alo[mi], b0, b1);
         }
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+      for (int j = 0; j < kNI; ++j)
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[i][j][k] = __fadd_rn(acc[i][j][k], part[i][j][k]);
   }
@@ -279,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < kNI; ++j)
 #pragma unroll
       for (int k = 0; k < 4; ++k) acc[i][j][k] = __fadd_rn(acc[i][j][k], acc_lo[i][j][k]);
 
@@ -289,8 +304,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 #pragma unroll
     for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-      for (int ni = 0; ni < 2; ++ni) {
-        const int row = wm * 32 + mi * 16 + g, col = wn * 16 + ni * 8 + 2 * t;
+      for (int ni = 0; ni < kNI; ++ni) {
+        const int row = wm * 32 + mi * 16 + g, col = wn * kWN + ni * 8 + 2 * t;
         *reinterpret_cast<float2*>(cs + row * kCStride + col) = make_float2(acc[mi][ni][0], acc[mi][ni][1]);
         *reinterpret_cast<float2*>(cs + (row + 8) * kCStride + col) = make_float2(acc[mi][ni][2], acc[mi][ni][3]);
       }
