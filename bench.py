@@ -62,7 +62,8 @@ def source_digest(files):
 
 
 KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
-                  "decode": ["decode.cu", "shared.cu", "common.cuh", "wsvd_internal.h", "api.cu"]}
+                  "decode": ["decode.cu", "shared.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
+                  "prefill_gemm": ["prefill.cu", "common.cuh", "wsvd_internal.h"]}
 
 
 def ncu_traffic(kernel: str, workload: str):
@@ -439,7 +440,9 @@ def run_prefill_line(w: WL.Workload, args, world: int, rank: int, barrier):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "kernel": "prefill (rotate + GEMM/quantise + advance, 3 launches)",
                          "achieved": pf["tensor_tflops"], "peak": pf["peak_tflops"], "unit": "TFLOP/s",
-                         "frac": pf["frac_tensor"], "peak_kind": pf["peak_kind"], "traffic": None,
+                         "frac": pf["frac_tensor"], "peak_kind": pf["peak_kind"],
+                         "traffic": ncu_traffic("prefill_gemm", "llava7b" if w is WL.LLAVA7B else w.name),
+                         "traffic_kernel": "prefill_gemm_kernel (DRAM bytes per launch, ncu)",
                          "useful_tflops": pf["useful_tflops"]},
             "prefill": pf, "gpu_launches": 3 * args.steps, "clocks": clk,
         }
