@@ -36,8 +36,10 @@ namespace {
 
 constexpr int kRotThreads = 256;
 constexpr int kBM = 64, kBN = 128, kBK = 64;
-constexpr int kWarpsN = 8;                      // warps along N (2 along M): 16 warps of 32 x 16 outputs
-constexpr int kGemmThreads = 64 * kWarpsN;
+constexpr int kWarpsM = 2, kWarpsN = 8;         // 16 warps of 32 x 16 outputs
+constexpr int kGemmThreads = 32 * kWarpsM * kWarpsN;
+constexpr int kWM = kBM / kWarpsM;              // rows per warp
+constexpr int kMI = kWM / 16;                   // m16 MMA tiles per warp
 constexpr int kWN = kBN / kWarpsN;              // columns per warp
 constexpr int kNI = kWN / 8;                    // n8 MMA tiles per warp
 constexpr int kNJ = kWN / 16;                   // ldmatrix.x4.trans per k16 step (two n8 tiles each)
@@ -78,14 +80,22 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
   extern __shared__ __align__(16) float xs[];
   __shared__ float wmax[kRotThreads / 32];
   const int m = blockIdx.x, tid = threadIdx.x;
-  const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)m * E;
-  for (int i = tid; i < E; i += kRotThreads) xs[i] = x_value(xr[i], x_dtype);
+  const int E4 = E / 4;  // E is a multiple of 64: rows are whole 8-byte groups of four values
+  const uint2* xr = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + (size_t)m * E);
+  float4* xs4 = reinterpret_cast<float4*>(xs);
+  for (int i = tid; i < E4; i += kRotThreads) {
+    const uint2 v = xr[i];
+    xs4[i] = make_float4(x_value((uint16_t)(v.x & 0xffffu), x_dtype), x_value((uint16_t)(v.x >> 16), x_dtype),
+                         x_value((uint16_t)(v.y & 0xffffu), x_dtype), x_value((uint16_t)(v.y >> 16), x_dtype));
+  }
   __syncthreads();
-  // Butterfly stages of distance 1, 2, ..., blk/2: pairs (i, i + hh) with bit
-  // hh of i clear never leave an aligned block of blk values (Sylvester order).
-  for (int hh = 1; hh < blk; hh <<= 1) {
+  // Butterfly stages of distance hh = 1, 2, ..., blk/2: pairs (i, i + hh) with
+  // bit hh of i clear never leave an aligned block of blk values (Sylvester
+  // order).  Pair q of a stage: q's bits above log2(hh) move up by one.
+  for (int sh = 0; (1 << sh) < blk; ++sh) {
+    const int hh = 1 << sh;
     for (int q = tid; q < E / 2; q += kRotThreads) {
-      const int i = (q / hh) * 2 * hh + (q % hh);
+      const int i = ((q >> sh) << (sh + 1)) | (q & (hh - 1));
       const float u = xs[i], v = xs[i + hh];
       xs[i] = u + v;
       xs[i + hh] = u - v;
@@ -93,10 +103,11 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
     __syncthreads();
   }
   float amax = 0.f;
-  for (int i = tid; i < E; i += kRotThreads) {
-    const float v = xs[i] * hnorm;
-    xs[i] = v;
-    amax = fmaxf(amax, fabsf(v));
+  for (int i = tid; i < E4; i += kRotThreads) {
+    float4 v = xs4[i];
+    v.x *= hnorm; v.y *= hnorm; v.z *= hnorm; v.w *= hnorm;
+    xs4[i] = v;
+    amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -113,11 +124,20 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
     k = max(-126, min(126, 14 - e));
   }
   const float p = __uint_as_float((uint32_t)(127 + k) << 23);
-  for (int i = tid; i < E; i += kRotThreads) {
-    const float v = xs[i] * p;
-    const __half hi = __float2half_rn(v);
-    xhi[(size_t)m * E + i] = hi;
-    xlo[(size_t)m * E + i] = __float2half_rn(v - __half2float(hi));
+  uint2* hi4 = reinterpret_cast<uint2*>(xhi + (size_t)m * E);
+  uint2* lo4 = reinterpret_cast<uint2*>(xlo + (size_t)m * E);
+  auto split = [&](float v, __half& hi) {  // hi = fp16(v), returns fp16(v - hi)
+    hi = __float2half_rn(v);
+    return __float2half_rn(v - __half2float(hi));
+  };
+  for (int i = tid; i < E4; i += kRotThreads) {
+    const float4 v = xs4[i];
+    __half h0, h1, h2, h3;
+    const __half l0 = split(v.x * p, h0), l1 = split(v.y * p, h1), l2 = split(v.z * p, h2), l3 = split(v.w * p, h3);
+    hi4[i] = make_uint2((uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16),
+                        (uint32_t)__half_as_ushort(h2) | ((uint32_t)__half_as_ushort(h3) << 16));
+    lo4[i] = make_uint2((uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16),
+                        (uint32_t)__half_as_ushort(l2) | ((uint32_t)__half_as_ushort(l3) << 16));
   }
   if (tid == 0) inv_p[m] = __uint_as_float((uint32_t)(127 - k) << 23);
 }
@@ -214,7 +234,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __half* sm = reinterpret_cast<__half*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp / kWarpsN, wn = warp % kWarpsN;  // warp tile: rows wm*32.., columns wn*kWN..
+  const int wm = warp / kWarpsN, wn = warp % kWarpsN;  // warp tile: rows wm*kWM.., columns wn*kWN..
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
   const int KT = a.E / kBK;
   const CopyPlan plan = plan_copies(a, m0, n0, tid);
@@ -223,9 +243,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   // half's, kept on the tensor cores over all of E (its sum is ~2^-11 of c,
   // so its drift is far below the hi half's rounding).  Separate accumulators
   // also make the hi and lo MMAs independent of each other.
-  float acc[2][kNI][4], acc_lo[2][kNI][4];
+  float acc[kMI][kNI][4], acc_lo[kMI][kNI][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < kMI; ++i)
 #pragma unroll
     for (int j = 0; j < kNI; ++j)
 #pragma unroll
@@ -251,19 +271,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
     // sum held in the MMA accumulator over all of E drifts by a fraction of an
     // ulp per MMA.  Each k-tile of the hi half therefore starts from zero
     // (four MMAs deep) and is added to the fp32 total with a rounded add.
-    float part[2][kNI][4];
+    float part[kMI][kNI][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kMI; ++i)
 #pragma unroll
       for (int j = 0; j < kNI; ++j)
 #pragma unroll
         for (int k = 0; k < 4; ++k) part[i][j][k] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < kBK; kk += 16) {
-      uint32_t ahi[2][4], alo[2][4], bq[kNJ][4];
+      uint32_t ahi[kMI][4], alo[kMI][4], bq[kNJ][4];
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        const uint32_t off = (uint32_t)(((wm * 32 + mi * 16 + (lane & 15)) * kAStride + kk + (lane >> 4) * 8) * 2);
+      for (int mi = 0; mi < kMI; ++mi) {
+        const uint32_t off = (uint32_t)(((wm * kWM + mi * 16 + (lane & 15)) * kAStride + kk + (lane >> 4) * 8) * 2);
         ldmatrix_x4(ahi[mi], ahi_base + off);
         ldmatrix_x4(alo[mi], alo_base + off);
       }
@@ -274,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
         ldmatrix_x4_trans(bq[nj], b_base + (uint32_t)((krow * kBStride + col) * 2));
       }
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi)
+      for (int mi = 0; mi < kMI; ++mi)
 #pragma unroll
         for (int ni = 0; ni < kNI; ++ni) {
           const uint32_t b0 = bq[ni >> 1][(ni & 1) * 2], b1 = bq[ni >> 1][(ni & 1) * 2 + 1];
@@ -283,7 +303,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
         }
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kMI; ++i)
 #pragma unroll
       for (int j = 0; j < kNI; ++j)
 #pragma unroll
@@ -292,7 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   cp_async_wait_group<0>();
   __syncthreads();  // every warp is done with the ring: it becomes the epilogue tile
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < kMI; ++i)
 #pragma unroll
     for (int j = 0; j < kNI; ++j)
 #pragma unroll
@@ -302,10 +322,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
+    for (int mi = 0; mi < kMI; ++mi)
 #pragma unroll
       for (int ni = 0; ni < kNI; ++ni) {
-        const int row = wm * 32 + mi * 16 + g, col = wn * kWN + ni * 8 + 2 * t;
+        const int row = wm * kWM + mi * 16 + g, col = wn * kWN + ni * 8 + 2 * t;
         *reinterpret_cast<float2*>(cs + row * kCStride + col) = make_float2(acc[mi][ni][0], acc[mi][ni][1]);
         *reinterpret_cast<float2*>(cs + (row + 8) * kCStride + col) = make_float2(acc[mi][ni][2], acc[mi][ni][3]);
       }
