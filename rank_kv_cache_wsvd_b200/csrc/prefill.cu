@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kRotThreads = 256;
 constexpr int kBM = 64, kBN = 128, kBK = 64;
-constexpr int kWarpsM = 2, kWarpsN = 8;         // 16 warps of 32 x 16 outputs
+constexpr int kWarpsM = 4, kWarpsN = 4;         // 16 warps of 16 x 32 outputs
 constexpr int kGemmThreads = 32 * kWarpsM * kWarpsN;
 constexpr int kWM = kBM / kWarpsM;              // rows per warp
 constexpr int kMI = kWM / 16;                   // m16 MMA tiles per warp
