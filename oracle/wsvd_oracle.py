@@ -165,6 +165,49 @@ def wsvd_decode(q, lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r: int, bit
     return out
 
 
+def wsvd_decode_gqa(q, lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r: int, bits: int,
+                    softmax_scale: Optional[float] = None) -> np.ndarray:
+    """Grouped-query decode over a per-head low-rank cache: out [B][Hq][Hd].
+
+    Hq query heads share Hkv latent heads (Hq = G * Hkv): query head g reads
+    latent head g // G with that head's factors, i.e. consecutive query heads
+    form a group, as in grouped-query attention.  q [B][Hq][Hd]; lat_*,
+    scale_* over Hkv heads; Bk, Bv [Hkv][r][Hd].  The pages describe one
+    query per latent head; this is the grouped reading of the same decode
+    (each query head is the plain decode of ja §2.4 / de §2.D over its
+    group's latent)."""
+    B, Hq, Hd = q.shape
+    Hkv = lat_k.shape[1]
+    if Hq % Hkv:
+        raise ValueError("query heads must be a multiple of latent heads")
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, Hd), np.float64)
+    for b in range(B):
+        n = int(seq_lens[b])
+        for g in range(Hq):
+            j = g // G
+            out[b, g], _ = wsvd_decode_head(q[b, g], lat_k[b, j], scale_k[b, j], lat_v[b, j], scale_v[b, j],
+                                            Bk[j], Bv[j], n, r, bits, softmax_scale)
+    return out
+
+
+def wsvd_decode_multi(q, lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r: int, bits: int,
+                      softmax_scale: Optional[float] = None) -> np.ndarray:
+    """Decode of Tq new tokens per sequence at once (a speculative or chunked
+    decode step): out [B][Tq][Hq][Hd].
+
+    q [B][Tq][Hq][Hd]; the Tq tokens are the last Tq cached rows of each
+    sequence, so query t of sequence b sees rows [0, seq_lens[b] - Tq + 1 + t)
+    (causal inside the block, everything before it).  Latent heads may be
+    grouped as in wsvd_decode_gqa.  A query that sees no row gets 0."""
+    B, Tq, Hq, Hd = q.shape
+    out = np.zeros((B, Tq, Hq, Hd), np.float64)
+    for t in range(Tq):
+        n_t = np.maximum(np.asarray(seq_lens, np.int64) - Tq + 1 + t, 0)
+        out[:, t] = wsvd_decode_gqa(q[:, t], lat_k, scale_k, lat_v, scale_v, Bk, Bv, n_t, r, bits, softmax_scale)
+    return out
+
+
 def dense_decode(q, K, V, seq_lens, softmax_scale: Optional[float] = None) -> np.ndarray:
     """Textbook decode over a dense fp16 KV cache: the flash-decoding baseline
     the pages compare against (de §4 "Ergebnisse").  K, V [B][H][L_cap][Hd]."""

@@ -196,3 +196,30 @@ def test_prefill_mutants_are_caught(monkeypatch, kind):
         except AssertionError:
             failed += 1
     assert failed > 0
+
+
+def test_gqa_strided_grouping_mutant_is_caught(monkeypatch):
+    """Query head g reading latent head g % Hkv (strided groups) instead of g // G."""
+    def strided(q, lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r, bits, softmax_scale=None):
+        B, Hq, Hd = q.shape
+        Hkv = lat_k.shape[1]
+        out = np.zeros((B, Hq, Hd))
+        for b in range(B):
+            for g in range(Hq):
+                j = g % Hkv
+                out[b, g], _ = OW.wsvd_decode_head(q[b, g], lat_k[b, j], scale_k[b, j], lat_v[b, j], scale_v[b, j],
+                                                   Bk[j], Bv[j], int(seq_lens[b]), r, bits, softmax_scale)
+        return out
+    _patch(monkeypatch, "wsvd_decode_gqa", strided)
+    with pytest.raises(AssertionError):
+        P.test_gqa_matches_torch_grouped_sdpa(8)
+
+
+def test_multi_token_visibility_mutant_is_caught(monkeypatch):
+    """Every query of the block seeing the whole block (no causal step) must fail."""
+    def no_causal(q, lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r, bits, softmax_scale=None):
+        return np.stack([OW.wsvd_decode_gqa(q[:, t], lat_k, scale_k, lat_v, scale_v, Bk, Bv, seq_lens, r, bits,
+                                            softmax_scale) for t in range(q.shape[1])], axis=1)
+    _patch(monkeypatch, "wsvd_decode_multi", no_causal)
+    with pytest.raises(AssertionError):
+        P.test_multi_token_decode_is_causal_inside_the_block()

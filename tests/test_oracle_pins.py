@@ -365,6 +365,86 @@ def test_wsvd_equals_shared_when_each_head_owns_its_block():
     assert np.allclose(w, s, rtol=1e-12, atol=1e-14)
 
 
+# ----------------------------------------------------------------------------- grouped and multi-token queries
+def _gqa_case(seed, B=2, Hq=6, Hkv=2, Hd=8, r=4, L=11, bits=8):
+    rng = np.random.default_rng(seed)
+    Q = O.qmax(bits)
+    ck = rng.integers(-Q, Q + 1, size=(B, Hkv, L, r))
+    cv = rng.integers(-Q, Q + 1, size=(B, Hkv, L, r))
+    sk = rng.uniform(0.01, 0.1, (B, Hkv, L)).astype(np.float16)
+    sv = rng.uniform(0.01, 0.1, (B, Hkv, L)).astype(np.float16)
+    Bk = (rng.standard_normal((Hkv, r, Hd)) / 2).astype(np.float16)
+    Bv = (rng.standard_normal((Hkv, r, Hd)) / 2).astype(np.float16)
+    return ck, cv, sk, sv, Bk, Bv, rng
+
+
+def _rebuilt(codes, scale, Bm):
+    """K or V of every (b, latent head) rebuilt with plain numpy: [B][Hkv][L][Hd]."""
+    lat = codes.astype(np.float64) * scale.astype(np.float64)[..., None]
+    return np.einsum("bjlr,jrd->bjld", lat, Bm.astype(np.float64))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_gqa_matches_torch_grouped_sdpa(bits):
+    """Query head g reads latent head g // G: torch's SDPA with enable_gqa (which
+    groups consecutive query heads) on the rebuilt K, V is the reference; a
+    strided grouping (g % Hkv) or a swapped factor fails it."""
+    ck, cv, sk, sv, Bk, Bv, rng = _gqa_case(31, bits=bits)
+    B, Hkv, L, r = ck.shape
+    Hq, Hd = 6, Bk.shape[2]
+    q = rng.standard_normal((B, Hq, Hd)).astype(np.float16)
+    lens = np.array([L, 4])
+    out = O.wsvd_decode_gqa(q, O.pack_codes(ck, bits), sk, O.pack_codes(cv, bits), sv, Bk, Bv, lens, r, bits)
+    K, V = _rebuilt(ck, sk, Bk), _rebuilt(cv, sv, Bv)
+    for b in range(B):
+        n = lens[b]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b].astype(np.float64))[None, :, None, :], torch.from_numpy(K[b, :, :n])[None],
+            torch.from_numpy(V[b, :, :n])[None], scale=1.0 / math.sqrt(Hd), enable_gqa=True)[0, :, 0].numpy()
+        assert np.allclose(out[b], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_gqa_with_one_query_per_head_is_the_decode_and_expands_to_it():
+    """G = 1 is wsvd_decode itself; G > 1 equals wsvd_decode on a cache whose
+    latent heads and factors are each repeated G times."""
+    ck, cv, sk, sv, Bk, Bv, rng = _gqa_case(32, Hq=2, Hkv=2)
+    lk, lv = O.pack_codes(ck, 8), O.pack_codes(cv, 8)
+    lens = np.array([11, 7])
+    q2 = rng.standard_normal((2, 2, 8))
+    assert np.array_equal(O.wsvd_decode_gqa(q2, lk, sk, lv, sv, Bk, Bv, lens, 4, 8),
+                          O.wsvd_decode(q2, lk, sk, lv, sv, Bk, Bv, lens, 4, 8))
+    q6 = rng.standard_normal((2, 6, 8))
+    rep = lambda a, ax: np.repeat(a, 3, axis=ax)
+    want = O.wsvd_decode(q6, rep(lk, 1), rep(sk, 1), rep(lv, 1), rep(sv, 1), rep(Bk, 0), rep(Bv, 0), lens, 4, 8)
+    assert np.array_equal(O.wsvd_decode_gqa(q6, lk, sk, lv, sv, Bk, Bv, lens, 4, 8), want)
+
+
+def test_multi_token_decode_is_causal_inside_the_block():
+    """Tq new tokens at once: query t sees rows [0, len - Tq + 1 + t).  Checked
+    against torch's SDPA with an explicit boolean mask built from that rule,
+    and Tq = 1 against the single-token grouped decode."""
+    ck, cv, sk, sv, Bk, Bv, rng = _gqa_case(33, L=13)
+    B, Hkv, L, r = ck.shape
+    Hq, Hd, Tq = 6, 8, 4
+    lk, lv = O.pack_codes(ck, 8), O.pack_codes(cv, 8)
+    lens = np.array([13, 9])
+    q = rng.standard_normal((B, Tq, Hq, Hd))
+    out = O.wsvd_decode_multi(q, lk, sk, lv, sv, Bk, Bv, lens, r, 8)
+    K, V = _rebuilt(ck, sk, Bk), _rebuilt(cv, sv, Bv)
+    for b in range(B):
+        n = lens[b]
+        mask = np.zeros((Tq, n), bool)
+        for t in range(Tq):
+            mask[t, :n - Tq + 1 + t] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b].transpose(1, 0, 2))[None], torch.from_numpy(K[b, :, :n])[None],
+            torch.from_numpy(V[b, :, :n])[None], attn_mask=torch.from_numpy(mask), scale=1.0 / math.sqrt(Hd),
+            enable_gqa=True)[0].numpy().transpose(1, 0, 2)
+        assert np.allclose(out[b], ref, rtol=1e-12, atol=1e-14)
+    one = O.wsvd_decode_multi(q[:, -1:], lk, sk, lv, sv, Bk, Bv, lens, r, 8)[:, 0]
+    assert np.array_equal(one, O.wsvd_decode_gqa(q[:, -1], lk, sk, lv, sv, Bk, Bv, lens, r, 8))
+
+
 # ----------------------------------------------------------------------------- append
 def test_append_writes_one_row_and_advances():
     rng = np.random.default_rng(15)
