@@ -90,3 +90,15 @@ def test_w8_weight_recipe_hits_the_code_range_per_column():
     back = q.astype(np.float64) * s.astype(np.float64)[:, None, :]
     # half a step, plus the float32 rounding of w / scale (up to 127 * 2^-24 code units)
     assert np.all(np.abs(back - ai.A_k.astype(np.float64)) <= (0.5 + 1e-4) * s.astype(np.float64)[:, None, :])
+
+
+def test_prefill_inputs_are_the_append_steps_as_one_block():
+    """Token t of the prefill block is the activation of append step t (same seed),
+    laid out [B][T][E]; the factors are the append's."""
+    w = W.LONG[16].with_(B=3)
+    p = W.prefill_inputs(w, seed=4, T=5)
+    a = W.append_inputs(w, seed=4, steps=5)
+    assert p.x.shape == (3, 5, 4096) and p.x_bits.shape == (3, 5, 4096)
+    assert np.array_equal(p.x, a.x.transpose(1, 0, 2)) and np.array_equal(p.x_bits, a.x_bits.transpose(1, 0, 2))
+    assert np.array_equal(p.A_k, a.A_k) and np.array_equal(p.A_v, a.A_v)
+    assert p.x.flags["C_CONTIGUOUS"] and W.LLAVA7B.prefill_tokens == 576
