@@ -142,8 +142,10 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
  *     that first call before any stream capture.
- *   - Every call clears the counters it uses (an asynchronous memset on
- *     `stream`), then launches the decode.
+ *   - Arguments are validated as by wsvd_decode_attention, in the same
+ *     order, before anything is queued on `stream`; then the call clears the
+ *     per-(b, h) counters (an asynchronous memset of 4 * B * H bytes on
+ *     `stream`) and launches the decode.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other threads) race and give wrong results.                  */
 #define WSVD_NOALLOC_SCRATCH_BYTES (2u << 20)
@@ -246,6 +248,35 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
                            void* append_workspace, size_t append_workspace_bytes, void* decode_workspace,
                            size_t decode_workspace_bytes, int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- one decode step from host buffers
+ * wsvd_append_and_decode for a caller whose per-step inputs and output live in
+ * host memory (a serving loop that receives the new token's activation and
+ * query from the host and returns the attention output there).  The pages
+ * have no counterpart: it exists so that one library call covers a whole
+ * step, copies included.  On `stream`, in order:
+ *   x_host [B][E] and q_host [B][H][Hd] (16-bit, x_dtype / q_dtype) are
+ *   copied into step_workspace; the append and the decode run as in
+ *   wsvd_append_and_decode on those copies; out [B][H][Hd] fp32 is copied to
+ *   out_host.
+ * The call returns once everything is queued; out_host is valid after the
+ * stream is synchronised.  Page-locked (pinned) host buffers make the copies
+ * asynchronous; pageable ones also work, with the driver's staging.
+ *   step_workspace   device memory of at least
+ *                    wsvd_step_host_workspace_size(B, H, Hd, E, r) bytes that is
+ *                    ZERO before the first call; it holds the append and
+ *                    decode workspaces (their counters are left zero) and the
+ *                    device copies of x, q and out.  Calls that share it must
+ *                    not overlap on the GPU.
+ * Every other argument is as for wsvd_append_and_decode (device pointers).
+ * All arguments are validated before anything is queued.                    */
+size_t wsvd_step_host_workspace_size(int B, int H, int Hd, int E, int r);
+int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                                const void* x_host, int x_dtype, const void* A_k, const void* A_v,
+                                int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                                const void* q_host, int q_dtype, const void* B_k, const void* B_v,
+                                float softmax_scale, float* out_host, void* step_workspace,
+                                size_t step_workspace_bytes, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------- int8 weights (W8)
  * The same three operations with the low-rank factors stored as int8 weights
  * (the "W8" of the method's W8A8 / W8A4 configurations, German §2.C): every
@@ -288,8 +319,9 @@ int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int 
  *   S2_k, S2_v            [H][r][r] float32, orthogonal (not checked).
  *   A_k, A_v              [H][E][r] fp16;  A_k_out, A_v_out same shape, written.
  *   B_k, B_v              [H][r][Hd] fp16; B_k_out, B_v_out same shape, written.
- * fp32 dot products over r, each result rounded once to fp16.  Outputs must not
- * alias inputs; r <= 128, H <= 65535.  Launches four small kernels on `stream`. */
+ * fp32 dot products over r, each result rounded once to fp16.  No output may
+ * share a byte with any input or with another output (WSVD_ERR_INVALID_ARG);
+ * r <= 128, H <= 65535.  Launches four small kernels on `stream`.           */
 int wsvd_fold_latent_rotation(int H, int E, int r, int Hd, const float* S2_k, const float* S2_v, const void* A_k,
                               const void* A_v, const void* B_k, const void* B_v, void* A_k_out, void* A_v_out,
                               void* B_k_out, void* B_v_out, void* stream);

@@ -102,14 +102,6 @@ def quantize(c: np.ndarray, bits: int) -> Tuple[np.ndarray, np.ndarray]:
     return codes, scale
 
 
-def quantize_ratio(c: np.ndarray, scale: np.ndarray) -> np.ndarray:
-    """float32 c / scale as the quantiser sees it (used to spot rounding ties)."""
-    c32 = np.asarray(c, dtype=np.float64).astype(np.float32)
-    s32 = np.asarray(scale, dtype=np.float16).astype(np.float32)[..., None]
-    safe = np.where(s32 > 0, s32, np.float32(1.0))
-    return np.where(s32 > 0, c32 / safe, np.float32(0.0)).astype(np.float32)
-
-
 # ----------------------------------------------------------------------------- attention
 def softmax(s: np.ndarray) -> np.ndarray:
     """p_l = exp(s_l - max s) / sum_k exp(s_k - max s)."""

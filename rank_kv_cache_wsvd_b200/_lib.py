@@ -43,6 +43,9 @@ SIGNATURES = {
     "wsvd_latent_prefill": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_size, _p, _p]),
     "wsvd_append_and_decode": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
+    "wsvd_step_host_workspace_size": (_c_size, [_c_int] * 5),
+    "wsvd_append_and_decode_host": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
+                                    + [_c_float, _p, _p, _c_size, _p, _p]),
     "wsvd_decode_attention_w8": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 8 + [_c_float, _p, _p, _c_size,
                                                                                            _p, _p]),
     "wsvd_latent_append_w8": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 9 + [_p, _c_size, _p, _p]),
@@ -261,6 +264,59 @@ def wsvd_append_and_decode(x, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v
                                     _ptr(decode_ws), decode_ws.numel(), _ptr(err), _stream(stream))
     _check(st, "wsvd_append_and_decode")
     return out
+
+
+def wsvd_step_host_workspace_size(B, H, Hd, E, r) -> int:
+    return load().wsvd_step_host_workspace_size(B, H, Hd, E, r)
+
+
+class StepFromHost:
+    """One decode step whose per-step inputs and output are host buffers:
+    wsvd_append_and_decode_host with every argument checked and converted
+    once, here, so that a call is one C call with no Python-side checks.
+
+    x_host [B][E] and q_host [B][H][Hd] (16-bit) and out_host [B][H][Hd]
+    fp32 are CPU tensors, ideally pinned; the device tensors (weights, cache,
+    seq_lens) are bound as given.  After `__call__` the step is queued on the
+    stream given here; out_host is valid once that stream is synchronised.
+    The caller keeps every bound tensor alive and unchanged in shape."""
+
+    def __init__(self, x_host, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q_host, B_k, B_v, out_host,
+                 bits: int, hadamard_block: int = 128, softmax_scale: float = 0.0, err=None, stream=None):
+        lib = load()
+        B, E = x_host.shape
+        H, _, r = A_k.shape
+        Hd = q_host.shape[2]
+        L_cap = lat_k.shape[2]
+        for t, name in ((x_host, "x_host"), (q_host, "q_host"), (out_host, "out_host")):
+            if t.is_cuda or not t.is_contiguous():
+                raise WsvdError(f"{name} must be a contiguous host tensor")
+        _expect(out_host, torch.float32, (B, H, Hd), "out_host")
+        _expect(q_host, q_host.dtype, (B, H, Hd), "q_host")
+        _expect(A_k, torch.float16, (H, E, r), "A_k")
+        _expect(A_v, torch.float16, (H, E, r), "A_v")
+        _expect(lat_k, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_k")
+        _expect(lat_v, torch.uint8, (B, H, L_cap, r * bits // 8), "lat_v")
+        _expect(scale_k, torch.float16, (B, H, L_cap), "scale_k")
+        _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
+        _expect(B_k, torch.float16, (H, r, Hd), "B_k")
+        _expect(B_v, torch.float16, (H, r, Hd), "B_v")
+        _expect(seq_lens, torch.int32, (B,), "seq_lens")
+        self.workspace = workspace(lib.wsvd_step_host_workspace_size(B, H, Hd, E, r), A_k.device)
+        self._keep = (x_host, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q_host, B_k, B_v, out_host, err)
+        self.h2d_bytes = x_host.numel() * 2 + q_host.numel() * 2
+        self.d2h_bytes = out_host.numel() * 4
+        self._fn = lib.wsvd_append_and_decode_host
+        self._args = (B, H, Hd, E, r, bits, L_cap, hadamard_block, x_host.data_ptr(), _dtype_code(x_host),
+                      _ptr(A_k), _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k),
+                      _ptr(scale_v), q_host.data_ptr(), _dtype_code(q_host), _ptr(B_k), _ptr(B_v),
+                      float(softmax_scale), out_host.data_ptr(), _ptr(self.workspace), self.workspace.numel(),
+                      _ptr(err), _stream(stream))
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st:
+            _check(st, "wsvd_append_and_decode_host")
 
 
 # ----------------------------------------------------------------------------- int8 weights

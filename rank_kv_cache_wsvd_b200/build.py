@@ -53,12 +53,35 @@ def _stale(extra_flags=()) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile every CUDA source into one shared library; returns its path."""
+    """Compile every CUDA source into one shared library; returns its path.
+
+    Each translation unit is compiled to an object in its own nvcc process (in
+    parallel), then the objects are linked into the library."""
     if not force and not _stale(extra_flags):
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(os.path.dirname(HERE), "_build")
+    os.makedirs(objdir, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.splitext(src)[0] + ".o")
+        cmd = [nvcc(), *compile_flags, *extra_flags, "-I", INCLUDE, "-c", "-o", obj, os.path.join(CSRC, src)]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, r
+
+    with ThreadPoolExecutor(max_workers=min(len(SOURCES), os.cpu_count() or 1)) as ex:
+        results = list(ex.map(compile_one, SOURCES))
+    for src, _, r in results:
+        if verbose or r.returncode:
+            sys.stdout.write(r.stdout)
+            sys.stderr.write(r.stderr)
+        if r.returncode:
+            raise subprocess.CalledProcessError(r.returncode, f"nvcc {src}")
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-o", tmp,
-           *[os.path.join(CSRC, f) for f in SOURCES]]
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *[o for _, o, _ in results]]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -149,6 +149,23 @@ int run_step(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadama
 
 }  // namespace
 
+int wsvd::decode_with_scratch(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens, const void* q,
+                        int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
+                        const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                        void* scratch, size_t scratch_bytes, int32_t* err, cudaStream_t stream) {
+  DecodeArgs a{};
+  const int st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v,
+                                     B_k, B_v, nullptr, nullptr, 0, softmax_scale, out, scratch, scratch_bytes, err,
+                                     &a);
+  if (st != WSVD_OK || B == 0) return st;
+  // Only the counters must start at zero: partials and q' are written before
+  // they are read.
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + partial_bytes(B, H, r), 0, counter_bytes(B, H), stream) !=
+      cudaSuccess)
+    return WSVD_ERR_CUDA;
+  return run_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a, scratch, stream);
+}
+
 extern "C" {
 
 const char* wsvd_status_string(int status) {
@@ -304,6 +321,64 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
   return run_step(B, H, Hd, E, r, bits, L_cap, hadamard_block, x, x_dtype, A_k, A_v, nullptr, nullptr, seq_lens,
                   lat_k, lat_v, scale_k, scale_v, q, q_dtype, B_k, B_v, nullptr, nullptr, 0, softmax_scale, out,
                   append_workspace, append_workspace_bytes, decode_workspace, decode_workspace_bytes, err, stream);
+}
+
+// Step workspace of wsvd_append_and_decode_host: the append counter, the
+// decode workspace, then device copies of x, q and out.
+struct StepHostLayout {
+  size_t app, dec, x, q, out, total;
+};
+inline StepHostLayout step_host_layout(int B, int H, int Hd, int E, int r) {
+  StepHostLayout l;
+  l.app = 0;
+  l.dec = align16(kAppendWorkspaceBytes);
+  l.x = l.dec + decode_ws_bytes(B, H, r);
+  l.q = l.x + align16((size_t)B * E * 2);
+  l.out = l.q + align16((size_t)B * H * Hd * 2);
+  l.total = l.out + align16((size_t)B * H * Hd * 4);
+  return l;
+}
+
+size_t wsvd_step_host_workspace_size(int B, int H, int Hd, int E, int r) {
+  if (B < 0 || H < 0 || Hd < 1 || E < 1 || r < 1) return 0;
+  return step_host_layout(B, H, Hd, E, r).total;
+}
+
+int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                                const void* x_host, int x_dtype, const void* A_k, const void* A_v,
+                                int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                                const void* q_host, int q_dtype, const void* B_k, const void* B_v,
+                                float softmax_scale, float* out_host, void* step_workspace,
+                                size_t step_workspace_bytes, int32_t* err, void* stream) {
+  if (B < 0 || H < 1 || Hd < 1 || E < 1 || r < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
+  if (B == 0) return WSVD_OK;
+  if (!x_host || !q_host || !out_host || !step_workspace) return WSVD_ERR_INVALID_ARG;
+  if (!aligned16(step_workspace)) return WSVD_ERR_INVALID_ARG;
+  const StepHostLayout l = step_host_layout(B, H, Hd, E, r);
+  if (step_workspace_bytes < l.total) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* w = static_cast<uint8_t*>(step_workspace);
+  void* x_dev = w + l.x;
+  void* q_dev = w + l.q;
+  float* out_dev = reinterpret_cast<float*>(w + l.out);
+  AppendArgs ap{};
+  int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x_dev, x_dtype, A_k, A_v, nullptr, nullptr, 0,
+                          seq_lens, lat_k, lat_v, scale_k, scale_v, w + l.app, kAppendWorkspaceBytes, err, &ap);
+  if (st != WSVD_OK) return st;
+  DecodeArgs dp{};
+  st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q_dev, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k,
+                           B_v, nullptr, nullptr, 0, softmax_scale, out_dev, w + l.dec, l.x - l.dec, err, &dp);
+  if (st != WSVD_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, (size_t)B * E * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(q_dev, q_host, (size_t)B * H * Hd * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return WSVD_ERR_CUDA;
+  if (launch_append(ap, s) != cudaSuccess) return WSVD_ERR_CUDA;
+  bind_workspace(&dp, w + l.dec);
+  if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, s, true) != cudaSuccess)
+    return WSVD_ERR_CUDA;
+  if (cudaMemcpyAsync(out_host, out_dev, (size_t)B * H * Hd * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return WSVD_ERR_CUDA;
+  return WSVD_OK;
 }
 
 int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,

@@ -40,6 +40,12 @@ __global__ void fold_b_kernel(int r, int Hd, const __half* B, const float* S2, _
   }
 }
 
+// Byte ranges [p, p + n) and [q, q + m) share at least one byte.
+inline bool overlap(const void* p, size_t n, const void* q, size_t m) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+  return a < b + m && b < a + n;
+}
+
 inline unsigned grid_x(size_t n) { return (unsigned)std::min<size_t>((n + 255) / 256, 1024); }
 
 }  // namespace
@@ -53,7 +59,18 @@ extern "C" int wsvd_fold_latent_rotation(int H, int E, int r, int Hd, const floa
   if (H < 1 || E < 1 || r < 1 || r > 128 || Hd < 1 || H > 65535) return WSVD_ERR_INVALID_ARG;
   if (!S2_k || !S2_v || !A_k || !A_v || !B_k || !B_v || !A_k_out || !A_v_out || !B_k_out || !B_v_out)
     return WSVD_ERR_INVALID_ARG;
-  if (A_k_out == A_k || A_v_out == A_v || B_k_out == B_k || B_v_out == B_v) return WSVD_ERR_INVALID_ARG;
+  // No output may share a byte with any input or with another output.
+  const size_t na = (size_t)H * E * r * 2, nb = (size_t)H * r * Hd * 2, ns = (size_t)H * r * r * 4;
+  const void* outs[4] = {A_k_out, A_v_out, B_k_out, B_v_out};
+  const size_t out_n[4] = {na, na, nb, nb};
+  const void* ins[6] = {A_k, A_v, B_k, B_v, S2_k, S2_v};
+  const size_t in_n[6] = {na, na, nb, nb, ns, ns};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 6; ++i)
+      if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return WSVD_ERR_INVALID_ARG;
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return WSVD_ERR_INVALID_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 ga(grid_x((size_t)E * r), H), gb(grid_x((size_t)r * Hd), H);
   fold_a_kernel<<<ga, 256, 0, s>>>(E, r, static_cast<const __half*>(A_k), S2_k, static_cast<__half*>(A_k_out));

@@ -41,17 +41,16 @@ extern "C" int wsvd_decode_attention_noalloc(int B, int H, int Hd, int r, int bi
                                              const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
                                              const void* scale_v, const void* B_k, const void* B_v,
                                              float softmax_scale, float* out, int32_t* err, void* stream) {
+  // The first checks of wsvd_decode_attention, in its order, before any CUDA
+  // call; the rest of its validation runs with the scratch address below.
+  if (B < 0 || H < 1 || L_cap < 0) return WSVD_ERR_INVALID_ARG;
   if (B == 0) return WSVD_OK;
-  if (B < 0 || H < 1 || r < 1) return WSVD_ERR_INVALID_ARG;
-  const size_t need = wsvd_decode_workspace_size(B, H, r);
-  if (need == 0) return WSVD_ERR_INVALID_ARG;
-  if (need > kScratchBytes) return WSVD_ERR_WORKSPACE_TOO_SMALL;  // beyond the static scratch limit
   void* scratch = nullptr;
   const int st = scratch_address(&scratch);
   if (st != WSVD_OK) return st;
-  // The array keeps the previous call's contents: the counters must start at zero.
-  if (cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return WSVD_ERR_CUDA;
-  return wsvd_decode_attention(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k,
-                               B_v, softmax_scale, out, scratch, kScratchBytes, err, stream);
+  // A problem that needs more than the static array is refused as
+  // WSVD_ERR_WORKSPACE_TOO_SMALL, like an undersized caller workspace.
+  return wsvd::decode_with_scratch(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v,
+                                   B_k, B_v, softmax_scale, out, scratch, kScratchBytes, err,
+                                   reinterpret_cast<cudaStream_t>(stream));
 }

@@ -86,6 +86,15 @@ struct AppendArgs {
   int32_t* err;
 };
 int append_cluster_size(int E, int blk);
+// wsvd_decode_attention with caller-provided scratch that is NOT zero on entry
+// (the no-allocation entry point's static array): validates every argument
+// exactly as wsvd_decode_attention does, and only then clears the per-(b, h)
+// counters (an asynchronous memset on `stream`) and launches.  Nothing is
+// queued when validation fails.
+int decode_with_scratch(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens, const void* q,
+                        int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
+                        const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                        void* scratch, size_t scratch_bytes, int32_t* err, cudaStream_t stream);
 size_t append_smem_bytes(int B, int E, int r, int cluster);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 

@@ -133,3 +133,53 @@ def test_prefill_workspace_and_host_validation(lib):
     assert lib.wsvd_latent_prefill(*args(T=0, ptr=None)) == 0     # empty block: nothing launched
     assert lib.wsvd_latent_prefill(*args(B=0, ptr=None)) == 0
     assert lib.wsvd_latent_prefill(*args(T=-1)) == 1
+
+
+def test_noalloc_checks_come_first_and_match_the_workspace_entry_point(lib):
+    """The no-allocation decode answers the first argument checks exactly as
+    wsvd_decode_attention does, before any CUDA call (so on this host too)."""
+    p = ctypes.c_void_p(16)
+    for B, H, L_cap, want in [(0, 0, 64, 1), (-1, 4, 64, 1), (1, 4, -8, 1), (0, 4, 64, 0)]:
+        ws = lib.wsvd_decode_attention(B, H, 64, 16, 8, L_cap, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 1 << 20,
+                                       None, None)
+        na = lib.wsvd_decode_attention_noalloc(B, H, 64, 16, 8, L_cap, p, p, 0, p, p, p, p, p, p, 0.0, p, None,
+                                               None)
+        assert ws == na == want, (B, H, L_cap, ws, na)
+
+
+def test_fold_rejects_overlapping_outputs(lib):
+    """Outputs may share no byte with any input or with each other: exact
+    aliasing, a partial overlap and two overlapping outputs are refused before
+    any launch."""
+    H, E, r, Hd = 2, 64, 16, 64
+    na, nb, ns = H * E * r * 2, H * r * Hd * 2, H * r * r * 4
+    base = 1 << 20
+    S2k, S2v = base, base + ns
+    Ak, Av = base + 2 * ns, base + 2 * ns + na
+    Bk, Bv = Av + na, Av + na + nb
+    free = Bv + nb + 4096
+    outs = [free, free + na, free + 2 * na, free + 2 * na + nb]
+
+    def call(o):
+        return lib.wsvd_fold_latent_rotation(H, E, r, Hd, *[ctypes.c_void_p(v) for v in
+                                                             (S2k, S2v, Ak, Av, Bk, Bv, *o)], None)
+    assert call([Ak, outs[1], outs[2], outs[3]]) == 1              # A_k_out is A_k
+    assert call([outs[0], Av + 16, outs[2], outs[3]]) == 1         # A_v_out starts inside A_v
+    assert call([outs[0], outs[1], S2v + ns - 16, outs[3]]) == 1   # B_k_out runs into S2_v's tail
+    assert call([outs[0], outs[0] + 16, outs[2], outs[3]]) == 1    # two outputs overlap
+
+
+def test_step_from_host_validation(lib):
+    """wsvd_append_and_decode_host refuses null host buffers and a small step
+    workspace before anything is queued; its workspace holds the append and
+    decode workspaces plus device copies of x, q and out."""
+    B, H, Hd, E, r = 1, 4, 64, 256, 16
+    a16 = lambda v: (v + 15) // 16 * 16
+    need = W.wsvd_step_host_workspace_size(B, H, Hd, E, r)
+    assert need == 256 + W.wsvd_decode_workspace_size(B, H, r) + a16(B * E * 2) + a16(B * H * Hd * 2) + \
+        a16(B * H * Hd * 4)
+    p = ctypes.c_void_p(16)
+    args = lambda xh=p, nbytes=need: (B, H, Hd, E, r, 8, 64, 128, xh, 1, p, p, p, p, p, p, p, p, 0, p, p, 0.0, p, p,
+                                      nbytes, None, None)
+    assert lib.wsvd_append_and_decode_host(*args(xh=None)) == 1
+    assert lib.wsvd_append_and_decode_host(*args(nbytes=need - 16)) == 4

@@ -62,6 +62,28 @@ def test_long_context_sampled_heads(r):
         assert_attention_close(gpu[b, h][None], ref[None], f"long r{r} b{b} h{h}")
 
 
+def test_comparison_shape_l2048_full():
+    """The WSVD arm of the comparison workload at its own shape (B 8, H 32,
+    r 32 int8, fp16 query, L 2048): every (b, h) against the oracle."""
+    d = WL.decode_inputs(WL.CMP[2048], seed=0)
+    gpu, err = run_gpu(d)
+    assert err == 0
+    assert_attention_close(gpu, oracle(d), "cmp L2048")
+
+
+def test_comparison_shape_l8192_sampled_heads():
+    """The WSVD arm at L 8192 (B 8, H 32) in the bench's launch configuration;
+    the oracle recomputes a sample of heads from their seeds."""
+    w = WL.CMP[8192]
+    d = WL.decode_inputs(w, seed=0)
+    gpu, err = run_gpu(d)
+    assert err == 0 and np.all(np.isfinite(gpu))
+    for b, h in [(0, 0), (2, 13), (5, 31), (7, 7), (7, 30)]:
+        lk, sk, lv, sv = WL.latent_cache_block(w, 0, b, h)
+        ref, _ = O.wsvd_decode_head(d.q[b, h], lk, sk, lv, sv, d.Bk[h], d.Bv[h], int(d.seq_lens[b]), w.r, 8)
+        assert_attention_close(gpu[b, h][None], ref[None], f"cmp L8192 b{b} h{h}")
+
+
 TINY = [1, 2, 3, 7, 8, 33, 255, 256, 257]
 
 

@@ -101,3 +101,32 @@ def test_decode_launch_count_matches_the_path():
     assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 1
     for w in (WL.LONG[16], WL.LONG[32], WL.LONG[64], WL.RAGGED, WL.CMP[8192]):
         assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 2, w.name
+
+
+@pytest.mark.parametrize("name", ["llava7b", "long-r32"])
+def test_step_from_host_buffers_equals_device_step(name):
+    """wsvd_append_and_decode_host (x and q copied in from host memory, out
+    copied back) gives bit for bit what wsvd_append_and_decode gives on the
+    same values already on the device, on two steps in a row."""
+    w, lens0 = CASES[name]
+    d, ai = _inputs(w, lens0, seed=33)
+    qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
+    x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
+    out_host = torch.full((w.B, w.H, w.Hd), float("nan"), dtype=torch.float32).pin_memory()
+    A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
+    dv, hs = _device_state(d), _device_state(d)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    step = W.StepFromHost(x_host, A_k, A_v, hs["lens"], hs["lat_k"], hs["lat_v"], hs["sk"], hs["sv"], q_host, B_k,
+                          B_v, out_host, bits=w.bits, hadamard_block=w.hadamard_block, err=err)
+    for rep in range(2):
+        out_dev = W.wsvd_append_and_decode(x_host.cuda(), A_k, A_v, dv["lens"], dv["lat_k"], dv["lat_v"], dv["sk"],
+                                           dv["sv"], q_host.cuda(), B_k, B_v, bits=w.bits,
+                                           hadamard_block=w.hadamard_block)
+        step()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert torch.equal(out_host, out_dev.cpu()), (name, rep)
+        for k in ("lat_k", "lat_v", "sk", "sv", "lens"):
+            assert torch.equal(hs[k], dv[k]), (name, k, rep)
+    assert np.array_equal(hs["lens"].cpu().numpy(), np.asarray(lens0) + 2)
