@@ -248,6 +248,18 @@ class WsvdStep:
         self.step()
         self.out_host.copy_(self.out, non_blocking=True)
 
+    def e2e_callable(self):
+        """The public call of one step from host buffers: the one-call
+        wsvd_append_and_decode_host (fp16 weights, appending workloads), else
+        the Python-level copies around the device call."""
+        if self.has_append and not self.w8:
+            self.e2e_call_name = "wsvd_append_and_decode_host"
+            return self.W.StepFromHost(self.x_host, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v,
+                                       self.scale_k, self.scale_v, self.q_host, self.B_k, self.B_v, self.out_host,
+                                       bits=self.w.bits, hadamard_block=self.w.hadamard_block, err=self.err)
+        self.e2e_call_name = "copies + " + ("wsvd_append_and_decode_w8" if self.has_append else "wsvd_decode_attention")
+        return self.e2e_step
+
     def e2e_bytes(self):
         h2d = self.q_host.numel() * 2 + (self.x_host.numel() * 2 if self.has_append else 0)
         return h2d, self.out_host.numel() * 4
@@ -360,10 +372,108 @@ def _time_loop(fn, steps, warmup, flush):
     return sum(a.elapsed_time(b) for a, b in evs) / 1e3 / steps
 
 
+# ----------------------------------------------------------------------------- sweep
+SWEEP = ["long_r16", "long_r32", "long_r64", "cmp_l2048", "cmp_l8192", "ragged"]
+
+
+def device_decode_inputs(w: WL.Workload, seed: int):
+    """Decode inputs of a full-size workload built on the device (seconds, not
+    the minutes the host generator needs at these sizes) with the workload's
+    recipe: latents N(0,1) (or Student-t nu = 3 with the workload's x20
+    outlier channels) per (b, h, token, channel), per-token scale
+    fp16(max|x| / Q), codes round-half-even(x / scale) clamped to +-Q, int4
+    packed two per byte (element 2j low nibble); q and B_K, B_V drawn by the
+    host generator.  Measurement inputs only: parity tests use workloads.py."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + seed)
+    lens = WL.seq_lens(w, seed)
+    Q = 127 if w.bits == 8 else 7
+    rb = w.r * w.bits // 8
+    gains = torch.from_numpy(WL._outlier_channels(w, seed)).float().cuda() if w.latent != "normal" else None
+
+    def lat():
+        out = torch.empty((w.B, w.H, w.L_cap, rb), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((w.B, w.H, w.L_cap), dtype=torch.float16, device="cuda")
+        for b in range(w.B):
+            x = torch.randn((w.H, w.L_cap, w.r), generator=g, device="cuda")
+            if gains is not None:  # Student-t with 3 degrees of freedom: z / sqrt(chi2_3 / 3)
+                c = torch.randn((3, w.H, w.L_cap, w.r), generator=g, device="cuda").square().sum(0)
+                x = x / torch.sqrt(c / 3.0) * gains[:, None, :]
+            s16 = (x.abs().amax(-1) / Q).half()
+            s = s16.float()[..., None]
+            codes = torch.where(s > 0, torch.round(x / torch.where(s > 0, s, torch.ones_like(s))),
+                                torch.zeros_like(x)).clamp_(-Q, Q).to(torch.int16)
+            if w.bits == 8:
+                out[b] = codes.to(torch.int8).view(torch.uint8)
+            else:
+                nib = (codes & 0xF).to(torch.uint8)
+                out[b] = nib[..., 0::2] | (nib[..., 1::2] << 4)
+            sc[b] = s16
+        return out, sc
+
+    lk, sk = lat()
+    lv, sv = lat()
+    q, qb = WL.query(w, seed)
+    bk, bv = WL.up_proj(w, seed)
+    qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
+    qt = torch.from_numpy(qb.view(np.int16).copy()).cuda().view(qdt)
+    return dict(q=qt, lat_k=lk, lat_v=lv, scale_k=sk, scale_v=sv, B_k=torch.from_numpy(bk).cuda(),
+                B_v=torch.from_numpy(bv).cuda(), seq_lens=torch.from_numpy(lens.astype(np.int32)).cuda(),
+                lens=lens)
+
+
+def run_sweep(names, steps: int, flush, peak: float):
+    """Decode-only timing of the 4K-32K workloads: the WSVD decode and the
+    in-library dense fp16 decode on the same shape (events around each call,
+    L2 flushed before it, host kept ahead), with the HBM fraction of the WSVD
+    decode and its speedup against 0.85 x the KV-byte ratio."""
+    import torch
+
+    import rank_kv_cache_wsvd_b200 as W
+    rows = {}
+    for name in names:
+        w = WL.PRESETS[name]
+        t = device_decode_inputs(w, 0)
+        lens = t.pop("lens")
+        ws = W.workspace(W.wsvd_decode_workspace_size(w.B, w.H, w.r))
+        out = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        call = lambda: W.wsvd_decode_attention(t["q"], t["lat_k"], t["lat_v"], t["scale_k"], t["scale_v"], t["B_k"],
+                                               t["B_v"], t["seq_lens"], bits=w.bits, out=out, workspace_buf=ws,
+                                               err=err)
+        t_w = _time_loop(call, steps, 5, flush)
+        if int(err.item()) != 0:
+            raise RuntimeError(f"sweep {name}: device error word {int(err.item())}")
+        del t
+        K = torch.randn((w.B, w.H, w.L_cap, w.Hd), device="cuda").half()
+        V = torch.randn_like(K)
+        qd = torch.randn((w.B, w.H, w.Hd), device="cuda").half()
+        lens_t = torch.from_numpy(lens.astype(np.int32)).cuda()
+        wsd = W.workspace(W.dense_decode_workspace_size(w.B, w.H, w.Hd))
+        t_d = _time_loop(lambda: W.dense_decode_attention(qd, K, V, lens_t, out=out, workspace_buf=wsd), steps, 5,
+                         flush)
+        del K, V
+        nb = alg_bytes_decode(w, lens)
+        dense_bytes = int(lens.sum()) * w.H * 2 * w.Hd * 2
+        ratio = dense_bytes / (int(lens.sum()) * w.H * 2 * (w.r * w.bits // 8 + 2))
+        gbs = nb / t_w / 1e9
+        rows[name] = {"decode_us": t_w * 1e6, "alg_bytes": nb, "gbs": gbs, "frac": gbs / peak,
+                      "dense_fp16_us": t_d * 1e6, "dense_gbs": dense_bytes / t_d / 1e9,
+                      "speedup_vs_dense": t_d / t_w, "kv_byte_ratio": ratio, "speedup_target": 0.85 * ratio,
+                      "launches": W.wsvd_decode_launch_count(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap),
+                      "tokens_heads_per_s": int(lens.sum()) * w.H / t_w}
+        torch.cuda.empty_cache()
+    return rows
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample_step(w: WL.Workload, seed: int, heads: int, cache={}):
     """One step of the float64 oracle on `heads` heads of every sequence (the
-    bounded CPU sample); returns the tokens*heads it processed."""
+    bounded CPU sample): the full latent append of the new token (rotation,
+    projection, quantiser, row write, length advance) when the workload
+    appends, then the decode of every sampled (b, h).  Returns the
+    tokens*heads it attended."""
     import oracle as O
     key = (w.name, seed, heads)
     if key not in cache:
@@ -371,11 +481,18 @@ def oracle_sample_step(w: WL.Workload, seed: int, heads: int, cache={}):
         q, _ = WL.query(w, seed)
         bk, bv = WL.up_proj(w, seed)
         blocks = {(b, h): WL.latent_cache_block(w, seed, b, h) for b in range(w.B) for h in range(heads)}
-        ai = WL.append_inputs(w, seed=seed, steps=1) if w.append_steps else None
-        cache[key] = (lens, q, bk, bv, blocks, ai)
-    lens, q, bk, bv, blocks, ai = cache[key]
-    if ai is not None:  # the append of the new token over the sampled heads
-        O.latent_project(ai.x[0], ai.A_k[:heads], ai.A_v[:heads], w.hadamard_block)
+        app = None
+        if w.append_steps:
+            ai = WL.append_inputs(w, seed=seed, steps=1)
+            rb = w.r * w.bits // 8
+            lat = np.zeros((w.B, heads, w.L_cap, rb), np.uint8)
+            sc = np.zeros((w.B, heads, w.L_cap), np.float16)
+            app = (ai.x[0], ai.A_k[:heads], ai.A_v[:heads], (lens - 1).astype(np.int32), lat, sc)
+        cache[key] = (lens, q, bk, bv, blocks, app)
+    lens, q, bk, bv, blocks, app = cache[key]
+    if app is not None:
+        x, ak, av, lens0, lat, sc = app
+        O.latent_append(x, ak, av, lens0, lat, sc, lat, sc, w.r, w.bits, w.hadamard_block)
     n = 0
     for (b, h), (lk, sk, lv, sv) in blocks.items():
         O.wsvd_decode_head(q[b, h], lk, sk, lv, sv, bk[h], bv[h], int(lens[b]), w.r, w.bits)
@@ -391,20 +508,40 @@ def cpu_threads():
         return 1
 
 
+def _cpu_leg(w: WL.Workload, budget_s: float, heads: int, threads):
+    """Oracle steps for about budget_s seconds; threads=None leaves the BLAS
+    pools as they are (all cores), else limits them to that many threads."""
+    from contextlib import nullcontext
+    try:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=threads) if threads else nullcontext()
+    except Exception:
+        ctx = nullcontext()
+    with ctx:
+        cores = cpu_threads()
+        oracle_sample_step(w, 0, heads)  # inputs built outside the timing
+        t0 = time.perf_counter()
+        n_tok, n_steps = 0, 0
+        while True:
+            n_tok += oracle_sample_step(w, 0, heads)
+            n_steps += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+    return {"value": n_tok / dt, "unit": UNIT, "cores": cores, "steps": n_steps, "seconds": dt}
+
+
 def run_cpu_sample(w: WL.Workload, budget_s: float, heads: int):
-    oracle_sample_step(w, 0, heads)  # build the inputs outside the timing
-    t0 = time.perf_counter()
-    n_tok, n_steps = 0, 0
-    while True:
-        n_tok += oracle_sample_step(w, 0, heads)
-        n_steps += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": n_tok / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n_steps} float64 oracle steps over {heads} of {w.H} heads of every sequence "
-                      f"({'append + ' if w.append_steps else ''}decode), {dt:.1f} s on "
-                      f"{len(os.sched_getaffinity(0))} host cores"}
+    """The float64 oracle as it stands on a bounded sample, timed twice: with
+    its BLAS pools limited to one thread and with all of the host's cores.
+    The line's value is the all-cores leg."""
+    one = _cpu_leg(w, budget_s / 2, heads, 1)
+    allc = _cpu_leg(w, budget_s / 2, heads, None)
+    work = ("latent append (rotate, project, quantise, write) + " if w.append_steps else "") + "decode"
+    return {"value": allc["value"], "unit": UNIT, "cores": allc["cores"], "kind": "oracle",
+            "sample": f"float64 oracle steps over {heads} of {w.H} heads of every sequence ({work}); "
+                      f"{len(os.sched_getaffinity(0))} host cores available",
+            "single_thread": one, "all_cores": allc}
 
 
 def sample_heads(w: WL.Workload) -> int:
@@ -457,7 +594,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="wsvd", choices=["wsvd", "reference"])
     ap.add_argument("--workload", default="llava7b", choices=sorted(WL.PRESETS))
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0,
+                    help="CPU baseline budget, split between the one-thread and all-cores legs")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the decode-only sweep over the 4K-32K workloads (default line only)")
     ap.add_argument("--no-extras", action="store_true", help="skip the CPU baseline, e2e and comparison timings")
     ap.add_argument("--weights", default="fp16", choices=["fp16", "int8"],
                     help="low-rank factors A, B as fp16, or int8 with per-column scales (W8)")
@@ -612,28 +752,43 @@ def main():
 
     extras = {}
     if not args.no_extras and rank == 0:
-        # end to end through the public API with host buffers (wall clock, host sync per step)
+        # End to end through the public API with host buffers: one library call
+        # per step (H2D of x and q from pinned memory, append, decode, D2H of
+        # out) and a stream synchronisation; host wall clock around the two.
+        # The length reset that lets every step append the same row is done
+        # before the clock starts.
         n_e2e = max(50, min(args.steps, 500))
+        fn = st.e2e_callable()
+        stream = torch.cuda.current_stream()
         for _ in range(10):
             st.reset()
-            st.e2e_step()
+            fn()
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
+        t_e2e = 0.0
         for _ in range(n_e2e):
             st.reset()
-            st.e2e_step()
-            torch.cuda.current_stream().synchronize()
-        t_e2e = time.perf_counter() - t0
+            stream.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            stream.synchronize()
+            t_e2e += time.perf_counter() - t0
         h2d, d2h = st.e2e_bytes()
         extras["e2e"] = {"value": attended_tokens(w, st.lens_after) * n_e2e / t_e2e, "unit": UNIT,
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                         "us_per_step": t_e2e / n_e2e * 1e6, "timing": "host wall clock, stream sync per step"}
+                         "us_per_step": t_e2e / n_e2e * 1e6,
+                         "timing": "host wall clock around one library call + stream sync per step",
+                         "call": st.e2e_call_name}
         extras["comparisons_same_shape"] = time_comparisons(w, min(args.steps, 200), 5, flush)
         extras["comparisons_same_shape"]["wsvd_decode"] = {"us": per_dec * 1e6, "alg_bytes": dec_bytes,
                                                            "gbs": dec_bytes / per_dec / 1e9}
         if st.has_append and w.prefill_tokens:
             extras["prefill"] = time_prefill(w, w.prefill_tokens, min(args.steps, 200), 5, flush)
         extras["cpu_baseline"] = run_cpu_sample(w, args.cpu_seconds, sample_heads(w))
+        if not args.no_sweep and args.workload == "llava7b":
+            extras["sweep"] = run_sweep(SWEEP, 300, flush, peaks()[0])
+            extras["sweep"]["note"] = ("decode-only, events around each call, L2 flushed before it; frac = "
+                                       "algorithmic GB/s / peak (%s); target frac >= 0.70 and speedup_vs_dense "
+                                       ">= speedup_target = 0.85 x kv_byte_ratio" % peaks()[1])
 
     if rank == 0:
         line = {
@@ -660,7 +815,7 @@ def main():
             "gpu_launches": st.launches_per_step * args.steps,
             "clocks": clk,
         }
-        for k in ("cpu_baseline", "e2e", "comparisons_same_shape", "prefill"):
+        for k in ("cpu_baseline", "e2e", "comparisons_same_shape", "prefill", "sweep"):
             if k in extras:
                 line[k] = extras[k]
         print(json.dumps(line), flush=True)
