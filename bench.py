@@ -467,6 +467,67 @@ def run_sweep(names, steps: int, flush, peak: float):
     return rows
 
 
+# ----------------------------------------------------------------------------- grouped / multi-token decode
+# (workload, Hq query heads, Tq tokens per step): G = Hq / w.H query heads per latent head.
+GROUPED = {
+    "gqa_llava": (WL.LLAVA7B.with_(H=8), 32, 1),      # LLaVA layer, 4 query heads per latent head
+    "multi_long": (WL.LONG[32].with_(H=8), 32, 4),    # 32K context, G 4, 4 tokens per step: 16 queries per head
+}
+
+
+def alg_bytes_grouped(w: WL.Workload, lens, Hq: int, Tq: int) -> int:
+    rb = w.r * w.bits // 8
+    return int(np.sum(lens)) * w.H * 2 * (rb + 2) + 2 * w.H * w.r * w.Hd * 2 + w.B * Tq * Hq * w.Hd * (2 + 4)
+
+
+def run_grouped(name: str, steps: int, flush, peak: float):
+    """Device time of one wsvd_decode_multi call on a grouped workload (events
+    around the call, L2 flushed before it), its HBM fraction, the tensor-core
+    work it executes, and for comparison the one-query kernel run once per
+    query of a head (what serving these queries without the grouped kernel
+    reads: the cache once per query)."""
+    import torch
+
+    import rank_kv_cache_wsvd_b200 as W
+    w, Hq, Tq = GROUPED[name]
+    G = Hq // w.H
+    t = device_decode_inputs(w, 0)
+    lens = t.pop("lens")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
+    q = torch.randn((w.B, Tq, Hq, w.Hd), generator=g, device="cuda").to(qdt)
+    ws = W.workspace(W.wsvd_decode_multi_workspace_size(w.B, Tq, Hq, w.H, w.r, w.L_cap))
+    out = torch.empty((w.B, Tq, Hq, w.Hd), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    call = lambda: W.wsvd_decode_multi(q, t["lat_k"], t["lat_v"], t["scale_k"], t["scale_v"], t["B_k"], t["B_v"],
+                                       t["seq_lens"], bits=w.bits, out=out, workspace_buf=ws, err=err)
+    t_g = _time_loop(call, steps, 5, flush)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"grouped {name}: device error word {int(err.item())}")
+    q1 = q[:, 0, ::G].contiguous()  # one query per latent head
+    ws1 = W.workspace(W.wsvd_decode_workspace_size(w.B, w.H, w.r))
+    out1 = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32, device="cuda")
+    t_1 = _time_loop(lambda: W.wsvd_decode_attention(q1, t["lat_k"], t["lat_v"], t["scale_k"], t["scale_v"],
+                                                     t["B_k"], t["B_v"], t["seq_lens"], bits=w.bits, out=out1,
+                                                     workspace_buf=ws1), steps, 5, flush)
+    nq = G * Tq
+    nb = alg_bytes_grouped(w, lens, Hq, Tq)
+    units = sum(max(0, int(n) - Tq + 1 + tq) for n in lens for tq in range(Tq)) * Hq  # attended (token, query head)
+    tiles = int(np.sum((lens + 127) // 128)) * w.H * ((nq + 15) // 16)
+    nq_cta = 4 if nq <= 4 else (8 if nq <= 8 else 16)
+    ns, no = (3 * nq_cta + 15) // 16 * 16, 2 * nq_cta
+    mo = 64 if w.r <= 64 else 128
+    mma_ops = tiles * (2 * 128 * ns * max(32, w.r) + 2 * mo * no * 128)  # executed (padded) MMA operations
+    del t
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "Hq": Hq, "Hkv": w.H, "G": G, "Tq": Tq, "us": t_g * 1e6, "alg_bytes": nb,
+            "gbs": nb / t_g / 1e9, "frac": nb / t_g / 1e9 / peak, "units_per_s": units / t_g,
+            "tensor_tops_executed": mma_ops / t_g / 1e12,
+            "one_query_kernel_us": t_1 * 1e6, "one_query_kernel_x_queries_us": t_1 * 1e6 * nq,
+            "speedup_vs_one_query_per_call": t_1 * nq / t_g}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample_step(w: WL.Workload, seed: int, heads: int, cache={}):
     """One step of the float64 oracle on `heads` heads of every sequence (the
@@ -601,8 +662,10 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the CPU baseline, e2e and comparison timings")
     ap.add_argument("--weights", default="fp16", choices=["fp16", "int8"],
                     help="low-rank factors A, B as fp16, or int8 with per-column scales (W8)")
-    ap.add_argument("--op", default="step", choices=["step", "prefill"],
-                    help="step: the decode step (append + decode); prefill: the prompt-block latent write alone")
+    ap.add_argument("--op", default="step", choices=["step", "prefill", "grouped"],
+                    help="step: the decode step (append + decode); prefill: the prompt-block latent write alone; "
+                         "grouped: the grouped-query / multi-token decode (--grouped-workload)")
+    ap.add_argument("--grouped-workload", default="multi_long", choices=sorted(GROUPED))
     args = ap.parse_args()
     w = WL.PRESETS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -642,6 +705,37 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
+
+    if args.op == "grouped":
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        barrier()
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.start()
+        time.sleep(0.25)
+        gr = run_grouped(args.grouped_workload, args.steps, flush, peaks()[0])
+        clk = clocks.stop()
+        barrier()
+        t = gr["us"] * 1e-6
+        value, t_total = replica_throughput(gr["units_per_s"] * t * args.steps, t * args.steps, world)
+        if rank == 0:
+            peak, kind = peaks()
+            print(json.dumps({
+                "metric": "grouped / multi-token low-rank decode: attended (token, query head) pairs per second",
+                "value": value, "unit": "token*query_heads/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": t_total / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "s8 x s8 -> s32 scores, f16 x f16 -> f32 values",
+                "data": "synthetic",
+                "config": {"workload": args.grouped_workload, "shape": gr["workload"], "Hq": gr["Hq"],
+                           "Hkv": gr["Hkv"], "Tq": gr["Tq"], "l2": "flushed between timed calls (256 MiB write)",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": {"bound": "hbm", "kernel": "grouped_decode_kernel (1 launch)", "achieved": gr["gbs"],
+                             "peak": peak, "unit": "GB/s", "frac": gr["gbs"] / peak, "peak_kind": kind,
+                             "traffic": None, "alg_bytes_per_launch": gr["alg_bytes"],
+                             "tensor_tops_executed": gr["tensor_tops_executed"]},
+                "grouped": gr, "gpu_launches": args.steps, "clocks": clk}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     if args.op == "prefill":
         run_prefill_line(w, args, world, rank, barrier)
@@ -785,6 +879,7 @@ def main():
             extras["prefill"] = time_prefill(w, w.prefill_tokens, min(args.steps, 200), 5, flush)
         extras["cpu_baseline"] = run_cpu_sample(w, args.cpu_seconds, sample_heads(w))
         if not args.no_sweep and args.workload == "llava7b":
+            extras["grouped"] = {k: run_grouped(k, 300, flush, peaks()[0]) for k in GROUPED}
             extras["sweep"] = run_sweep(SWEEP, 300, flush, peaks()[0])
             extras["sweep"]["note"] = ("decode-only, events around each call, L2 flushed before it; frac = "
                                        "algorithmic GB/s / peak (%s); target frac >= 0.70 and speedup_vs_dense "
@@ -815,7 +910,7 @@ def main():
             "gpu_launches": st.launches_per_step * args.steps,
             "clocks": clk,
         }
-        for k in ("cpu_baseline", "e2e", "comparisons_same_shape", "prefill", "sweep"):
+        for k in ("cpu_baseline", "e2e", "comparisons_same_shape", "prefill", "sweep", "grouped"):
             if k in extras:
                 line[k] = extras[k]
         print(json.dumps(line), flush=True)

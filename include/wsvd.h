@@ -123,6 +123,49 @@ int wsvd_decode_attention(int B, int H, int Hd, int r, int bits, int L_cap, cons
                           float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                           int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- grouped and multi-token decode
+ * The decode of wsvd_decode_attention for several queries per latent head
+ * (the fused low-rank decode of Japanese §2.4 / German §2.D, which the pages
+ * describe for one query per head and token):
+ *   - Hq query heads share Hkv latent heads (grouped-query attention):
+ *     query head g reads latent head g / G, G = Hq / Hkv (consecutive query
+ *     heads form a group), with that head's cache and factors;
+ *   - Tq new tokens per sequence are decoded at once (a chunked or
+ *     speculative step): they are the last Tq cached rows, and query token t
+ *     of sequence b attends to rows [0, seq_lens[b] - Tq + 1 + t) (causal
+ *     inside the block).  A query that sees no row gets out = 0.
+ * Per query: out = softmax(K . q * softmax_scale) . V over its visible rows,
+ * K = lat_K . B_k[h], V = lat_V . B_v[h] (h its latent head), computed
+ * reassociated as in wsvd_decode_attention.  One tile of cached latents is
+ * read once for all G * Tq queries of its latent head; the score and value
+ * products run on the tensor cores (int8 scores against a 24-bit fixed-point
+ * q'; values in fp16 hi + lo halves with fp32 accumulation).
+ *
+ *   q         [B][Tq][Hq][Hd] fp16 or bf16 (wsvd_decode_gqa: [B][Hq][Hd]).
+ *   lat_k, lat_v [B][Hkv][L_cap][r*bits/8], scale_k, scale_v [B][Hkv][L_cap],
+ *             B_k, B_v [Hkv][r][Hd]: formats as for wsvd_decode_attention.
+ *   out       [B][Tq][Hq][Hd] float32 (wsvd_decode_gqa: [B][Hq][Hd]).
+ *   Hq a multiple of Hkv; G * Tq <= 64; Hd in {32, 64, 128, 256}; row bytes
+ *   r*bits/8 in {16, 32, 64} (int8 r = 16, 32, 64; int4 r = 32, 64, 128);
+ *   L_cap a multiple of 8; B <= 65535.  Else WSVD_ERR_UNSUPPORTED.
+ *   workspace  at least wsvd_decode_multi_workspace_size(...) bytes, ZERO
+ *             before the first call; it holds split partials and one counter
+ *             per (sequence, latent head, group of 16 queries); every call
+ *             leaves the counters zero.  Calls sharing it must not overlap.
+ *   err        optional; WSVD_DEVERR_LEN_RANGE as for wsvd_decode_attention.
+ * One launch per call.                                                       */
+size_t wsvd_decode_multi_workspace_size(int B, int Tq, int Hq, int Hkv, int r, int L_cap);
+int wsvd_decode_multi(int B, int Tq, int Hq, int Hkv, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                      const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
+                      const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                      void* workspace, size_t workspace_bytes, int32_t* err, void* stream);
+/* wsvd_decode_multi with Tq = 1.                                            */
+size_t wsvd_decode_gqa_workspace_size(int B, int Hq, int Hkv, int r, int L_cap);
+int wsvd_decode_gqa(int B, int Hq, int Hkv, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
+                    const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v, const void* scale_k,
+                    const void* scale_v, const void* B_k, const void* B_v, float softmax_scale, float* out,
+                    void* workspace, size_t workspace_bytes, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------- WSVD decode without allocation
  * The WSVD summaries have no counterpart to this entry point: it is a
  * deployment convenience of this library.

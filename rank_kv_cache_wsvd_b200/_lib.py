@@ -43,6 +43,10 @@ SIGNATURES = {
     "wsvd_latent_prefill": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_size, _p, _p]),
     "wsvd_append_and_decode": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
+    "wsvd_decode_multi_workspace_size": (_c_size, [_c_int] * 6),
+    "wsvd_decode_multi": (_c_int, [_c_int] * 8 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size, _p, _p]),
+    "wsvd_decode_gqa_workspace_size": (_c_size, [_c_int] * 5),
+    "wsvd_decode_gqa": (_c_int, [_c_int] * 7 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size, _p, _p]),
     "wsvd_step_host_workspace_size": (_c_size, [_c_int] * 5),
     "wsvd_append_and_decode_host": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                     + [_c_float, _p, _p, _c_size, _p, _p]),
@@ -183,6 +187,65 @@ def wsvd_decode_attention(q, lat_k, lat_v, scale_k, scale_v, B_k, B_v, seq_lens,
                                    float(softmax_scale), _ptr(out), _ptr(workspace_buf), workspace_buf.numel(),
                                    _ptr(err), _stream(stream))
     _check(st, "wsvd_decode_attention")
+    return out
+
+
+def wsvd_decode_multi_workspace_size(B, Tq, Hq, Hkv, r, L_cap) -> int:
+    return load().wsvd_decode_multi_workspace_size(B, Tq, Hq, Hkv, r, L_cap)
+
+
+def wsvd_decode_multi(q, lat_k, lat_v, scale_k, scale_v, B_k, B_v, seq_lens, bits: int,
+                      softmax_scale: float = 0.0, out=None, workspace_buf=None, err=None, stream=None):
+    """Grouped / multi-token decode: q [B][Tq][Hq][Hd] over a cache of Hkv latent
+    heads (query head g reads latent head g // (Hq // Hkv)); query token t
+    sees rows [0, seq_lens[b] - Tq + 1 + t).  Returns out [B][Tq][Hq][Hd] fp32."""
+    lib = load()
+    B, Tq, Hq, Hd = q.shape
+    Hkv, L_cap, rb = lat_k.shape[1], lat_k.shape[2], lat_k.shape[3]
+    r = rb * 8 // bits
+    _expect(lat_k, torch.uint8, (B, Hkv, L_cap, rb), "lat_k")
+    _expect(lat_v, torch.uint8, (B, Hkv, L_cap, rb), "lat_v")
+    _expect(scale_k, torch.float16, (B, Hkv, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, Hkv, L_cap), "scale_v")
+    _expect(B_k, torch.float16, (Hkv, r, Hd), "B_k")
+    _expect(B_v, torch.float16, (Hkv, r, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, Tq, Hq, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, Tq, Hq, Hd), "out")
+    if workspace_buf is None:
+        workspace_buf = workspace(lib.wsvd_decode_multi_workspace_size(B, Tq, Hq, Hkv, r, L_cap), q.device)
+    st = lib.wsvd_decode_multi(B, Tq, Hq, Hkv, Hd, r, bits, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q),
+                               _ptr(lat_k), _ptr(lat_v), _ptr(scale_k), _ptr(scale_v), _ptr(B_k), _ptr(B_v),
+                               float(softmax_scale), _ptr(out), _ptr(workspace_buf), workspace_buf.numel(), _ptr(err),
+                               _stream(stream))
+    _check(st, "wsvd_decode_multi")
+    return out
+
+
+def wsvd_decode_gqa(q, lat_k, lat_v, scale_k, scale_v, B_k, B_v, seq_lens, bits: int, softmax_scale: float = 0.0,
+                    out=None, workspace_buf=None, err=None, stream=None):
+    """Grouped-query decode: q [B][Hq][Hd] over Hkv latent heads; out [B][Hq][Hd] fp32."""
+    lib = load()
+    B, Hq, Hd = q.shape
+    Hkv, L_cap, rb = lat_k.shape[1], lat_k.shape[2], lat_k.shape[3]
+    r = rb * 8 // bits
+    _expect(lat_k, torch.uint8, (B, Hkv, L_cap, rb), "lat_k")
+    _expect(lat_v, torch.uint8, (B, Hkv, L_cap, rb), "lat_v")
+    _expect(scale_k, torch.float16, (B, Hkv, L_cap), "scale_k")
+    _expect(scale_v, torch.float16, (B, Hkv, L_cap), "scale_v")
+    _expect(B_k, torch.float16, (Hkv, r, Hd), "B_k")
+    _expect(B_v, torch.float16, (Hkv, r, Hd), "B_v")
+    _expect(seq_lens, torch.int32, (B,), "seq_lens")
+    if out is None:
+        out = torch.empty((B, Hq, Hd), dtype=torch.float32, device=q.device)
+    _expect(out, torch.float32, (B, Hq, Hd), "out")
+    if workspace_buf is None:
+        workspace_buf = workspace(lib.wsvd_decode_gqa_workspace_size(B, Hq, Hkv, r, L_cap), q.device)
+    st = lib.wsvd_decode_gqa(B, Hq, Hkv, Hd, r, bits, L_cap, _ptr(seq_lens), _ptr(q), _dtype_code(q), _ptr(lat_k),
+                             _ptr(lat_v), _ptr(scale_k), _ptr(scale_v), _ptr(B_k), _ptr(B_v), float(softmax_scale),
+                             _ptr(out), _ptr(workspace_buf), workspace_buf.numel(), _ptr(err), _stream(stream))
+    _check(st, "wsvd_decode_gqa")
     return out
 
 

@@ -13,8 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libwsvd_b200.so")
-SOURCES = ["api.cu", "decode.cu", "shared.cu", "append.cu", "noalloc.cu", "fold.cu", "prefill.cu"]
-HEADERS = ["common.cuh", "wsvd_internal.h"]
+SOURCES = ["api.cu", "decode.cu", "shared.cu", "append.cu", "noalloc.cu", "fold.cu", "prefill.cu", "grouped.cu"]
+HEADERS = ["common.cuh", "wsvd_internal.h", "tc05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -183,3 +183,36 @@ def test_step_from_host_validation(lib):
                                       nbytes, None, None)
     assert lib.wsvd_append_and_decode_host(*args(xh=None)) == 1
     assert lib.wsvd_append_and_decode_host(*args(nbytes=need - 16)) == 4
+
+
+def test_grouped_decode_workspace_and_validation(lib):
+    """Grouped / multi-token decode: the workspace holds split partials (at most
+    64 splits of 128-token tiles) of up to 16 queries per (sequence, latent
+    head, query chunk) and one counter per chunk; unsupported shapes are
+    refused before anything is launched."""
+    a16 = lambda v: (v + 15) // 16 * 16
+    B, Tq, Hq, Hkv, r, L = 2, 4, 32, 8, 32, 1600
+    nq, nqc, slots = 16, 1, 13  # G * Tq = 16 queries; ceil(1600 / 128) = 13 tiles
+    want = a16(B * Hkv * nqc * slots * nq * (r + 2) * 4) + a16(B * Hkv * nqc * 4)
+    assert W.wsvd_decode_multi_workspace_size(B, Tq, Hq, Hkv, r, L) == want
+    assert lib.wsvd_decode_gqa_workspace_size(B, Hq, Hkv, r, L) == W.wsvd_decode_multi_workspace_size(
+        B, 1, Hq, Hkv, r, L)
+    # G * Tq = 32 queries: two chunks of 16; 64-split cap at 32768 tokens
+    assert W.wsvd_decode_multi_workspace_size(1, 4, 32, 4, 32, 32768) == \
+        a16(1 * 4 * 2 * 64 * 16 * 34 * 4) + a16(1 * 4 * 2 * 4)
+    p = ctypes.c_void_p(16)
+    ws = 1 << 24
+    args = lambda B=1, Tq=1, Hq=8, Hkv=2, Hd=64, r=32, bits=8, L=64, qp=p: (
+        B, Tq, Hq, Hkv, Hd, r, bits, L, p, qp, 0, p, p, p, p, p, p, 0.0, p, p, ws, None, None)
+    assert lib.wsvd_decode_multi(*args(Hq=6, Hkv=4)) == 1      # Hq not a multiple of Hkv
+    assert lib.wsvd_decode_multi(*args(Tq=9, Hq=16, Hkv=2)) == 2  # G * Tq = 72 > 64
+    assert lib.wsvd_decode_multi(*args(r=8)) == 2               # 8-byte rows
+    assert lib.wsvd_decode_multi(*args(Hd=48)) == 2
+    assert lib.wsvd_decode_multi(*args(L=60)) == 2              # L_cap not a multiple of 8
+    assert lib.wsvd_decode_multi(*args(bits=6)) == 1
+    assert lib.wsvd_decode_multi(*args(qp=None)) == 1
+    assert lib.wsvd_decode_multi(*args(qp=ctypes.c_void_p(24))) == 1
+    assert lib.wsvd_decode_multi(*args(B=0, qp=None)) == 0
+    small = list(args())
+    small[20] = 16
+    assert lib.wsvd_decode_multi(*small) == 4

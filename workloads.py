@@ -34,6 +34,7 @@ _T_Q, _T_LK, _T_LV, _T_BK, _T_BV, _T_LEN, _T_OUTL = 1, 2, 3, 4, 5, 6, 7
 _T_X, _T_AK, _T_AV, _T_XOUT = 10, 11, 12, 13
 _T_DK, _T_DV, _T_SK, _T_SV, _T_SBK, _T_SBV = 20, 21, 22, 23, 24, 25
 _T_S2K, _T_S2V = 30, 31
+_T_QM = 40
 
 
 def _rng(seed: int, *key: int) -> np.random.Generator:
@@ -154,6 +155,14 @@ def seq_lens(w: Workload, seed: int = 0) -> np.ndarray:
 def query(w: Workload, seed: int = 0) -> Tuple[np.ndarray, np.ndarray]:
     """q [B][H][Hd] ~ N(0,1) in the workload's dtype -> (float32 exact, uint16 bits)."""
     q = _rng(seed, _T_Q).standard_normal((w.B, w.H, w.Hd), dtype=np.float32)
+    return to_dtype_exact(q, w.q_dtype)
+
+
+def multi_query(w: Workload, seed: int, Tq: int, Hq: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Queries of a grouped / multi-token decode, q [B][Tq][Hq][Hd] ~ N(0,1) in
+    the workload's dtype -> (float32 exact, uint16 bits).  The cache of such a
+    workload has w.H = Hkv latent heads."""
+    q = _rng(seed, _T_QM).standard_normal((w.B, Tq, Hq, w.Hd), dtype=np.float32)
     return to_dtype_exact(q, w.q_dtype)
 
 
