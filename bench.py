@@ -348,7 +348,8 @@ def time_prefill(w: WL.Workload, T: int, steps: int, warmup: int, flush):
             "peak_kind": "measured bf16 burst (fp16 has the same nominal rate)" if os.path.exists(pk) else "fallback",
             "frac_useful": flops / t / 1e12 / peak, "frac_tensor": 2 * flops / t / 1e12 / peak,
             "weights_bytes": 2 * w.H * w.E * w.r * 2, "activation_bytes": M * w.E * 2,
-            "note": "mma.sync m16n8k16 fp16 tiles (hi + lo split of the rotated activations)"}
+            "note": "tcgen05 kind::f16 128x64 tiles, TMA-fed, accumulators in tensor memory (hi + lo split of the "
+                    "rotated activations); rotation + split and the length advance are separate launches"}
 
 
 def _time_loop(fn, steps, warmup, flush):

@@ -26,9 +26,14 @@
 //      (token, head) row of r values with one warp: amax, fp16 scale,
 //      round-half-even codes, row write;
 //   3. prefill_advance_kernel: seq_lens[b] += T, or the block is refused.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
+#include "tc05.cuh"
 
 namespace wsvd {
 
@@ -375,6 +380,319 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
   }
 }
 
+// ------------------------------------------------------------------ 2'. GEMM + quantise on tcgen05
+// The same product and epilogue on the fifth-generation tensor cores, for
+// shapes whose 64- (r <= 64) or 128-column (r = 128) output tiles hold whole
+// heads of one side (K or V): 128 x BN output tiles, one CTA each.
+//   warp 4   TMA producer: per 64-wide k-tile, the hi and lo activation tiles
+//            [128 x 64] (2-D tensor maps, 128-byte swizzle, K-major) and the
+//            weight tile [64 x BN] as BN / NG boxes of one head's NG columns
+//            (3-D tensor map over A [H][E][r], swizzle of NG * 2 bytes; the
+//            operand is N-major) into a four-stage mbarrier ring;
+//   warp 5   allocates tensor memory; one lane issues per k-tile four MMAs of
+//            the hi half into a fresh accumulator (double-buffered) and four
+//            of the lo half into one accumulator kept over all of E;
+//   warps 0-3  thread t <-> output row t <-> tensor-memory lane t: add each
+//            k-tile's hi sum to an fp32 register total with a round-to-nearest
+//            add, then add the lo sum, undo p_m and quantise every head of the
+//            row in registers (no cross-thread reduction: a thread holds whole
+//            heads), writing codes and scales straight to the cache.
+// Numerics are those of the mma.sync kernel above: each k-tile of the hi half
+// is summed from zero on the tensor cores, k-tiles are added with rounding to
+// nearest, the lo half keeps one tensor-core sum.
+constexpr int kTcBM = 128, kTcBK = 64, kTcStages = 4, kTcThreads = 192;
+
+template <int R>
+struct TcCfg {
+  static constexpr int BN = R <= 64 ? 64 : 128;          // output columns per tile (whole heads)
+  static constexpr int NG = R <= 64 ? R : 64;            // columns per weight box (one head, or half of r = 128)
+  static constexpr int SW = NG == 16 ? 6 : (NG == 32 ? 4 : 2);  // descriptor swizzle: 32 / 64 / 128 bytes
+  static constexpr int A_BYTES = kTcBM * kTcBK * 2;
+  static constexpr int W_BYTES = kTcBK * BN * 2;
+  static constexpr int STAGE = 2 * A_BYTES + W_BYTES;
+  static constexpr int TCOLS = 3 * BN <= 256 ? 256 : 512;
+  static constexpr int SMEM = kTcStages * STAGE + 1024 + 256;
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle-atom alignment");
+};
+
+struct TcArgs {
+  int M, T, H, bits, L_cap, KT;
+  const float* inv_p;
+  const int32_t* seq_lens;
+  uint8_t* lat_k;
+  uint8_t* lat_v;
+  __half* scale_k;
+  __half* scale_v;
+  int32_t* err;
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int R>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_xhi, const __grid_constant__ CUtensorMap tm_xlo,
+                      const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
+                      const TcArgs a) {
+  using C = TcCfg<R>;
+  constexpr int BN = C::BN, NG = C::NG, S = kTcStages;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
+  uint8_t* smem = smem_raw + (base - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::STAGE);
+  uint64_t* empty = full + S;
+  uint64_t* hfull = empty + S;  // [2] a k-tile's hi sum is in tensor memory
+  uint64_t* hfree = hfull + 2;  // [2] the epilogue has read it (128 arrivals)
+  uint64_t* done = hfree + 2;   // every MMA of the tile has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.y * BN;
+  const int HR = a.H * R;
+  const int kv = n0 >= HR ? 1 : 0, nl = n0 - kv * HR;  // tile columns within the K or the V side
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&hfull[i], 1);
+      mbar_init(&hfree[i], 128);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) tc05::alloc(tmem_slot, C::TCOLS);
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  bool timed_out = false;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (!mbar_wait_bounded(bar, parity, timed_out ? 0ull : kWaitLimitNs)) {
+      if (!timed_out) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      timed_out = true;
+    }
+  };
+  const int KT = a.KT;
+
+  if (warp == 4) {
+    if (lane == 0) {  // ---------------------------------------------- TMA producer
+      const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % S;
+        if (kt >= S) wait(&empty[s], (uint32_t)(((kt / S) - 1) & 1));
+        const uint32_t st = base + (uint32_t)(s * C::STAGE);
+        mbar_arrive_expect_tx(&full[s], C::STAGE);
+        tma_load_2d(st, &tm_xhi, kt * kTcBK, m0, &full[s]);
+        tma_load_2d(st + C::A_BYTES, &tm_xlo, kt * kTcBK, m0, &full[s]);
+#pragma unroll
+        for (int g = 0; g < BN / NG; ++g) {
+          const int col = nl + g * NG;
+          tma_load_3d(st + 2 * C::A_BYTES + g * (kTcBK * NG * 2), wmap, col % R, kt * kTcBK, col / R, &full[s]);
+        }
+      }
+      for (int kt = std::max(0, KT - S); kt < KT; ++kt) wait(&full[kt % S], (uint32_t)((kt / S) & 1));
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {  // ---------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = tc05::instr_desc(1, 0, 0, 0, 1, kTcBM, BN);
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % S;
+        wait(&full[s], (uint32_t)((kt / S) & 1));
+        if (kt >= 2) wait(&hfree[kt & 1], (uint32_t)(((kt >> 1) - 1) & 1));
+        tc05::fence_after_sync();
+        const uint32_t st = base + (uint32_t)(s * C::STAGE);
+        const uint32_t dh = tmem + (uint32_t)((kt & 1) * BN), dl = tmem + (uint32_t)(2 * BN);
+#pragma unroll
+        for (int kk = 0; kk < kTcBK / 16; ++kk) {
+          const uint64_t bd = tc05::smem_desc_sw(st + 2 * C::A_BYTES + kk * 32 * NG, 128 * NG, 16 * NG, C::SW);
+          tc05::mma_f16(dh, tc05::smem_desc_sw(st + kk * 32, 16, 1024, 2), bd, idesc, kk > 0);
+          tc05::mma_f16(dl, tc05::smem_desc_sw(st + C::A_BYTES + kk * 32, 16, 1024, 2), bd, idesc, kt > 0 || kk > 0);
+        }
+        tc05::commit(&empty[s]);
+        tc05::commit(&hfull[kt & 1]);
+      }
+      tc05::commit(done);
+      wait(done, 0);  // every MMA has completed before the allocation is released
+    }
+    __syncwarp();
+  } else {  // -------------------------------------------------------- epilogue, thread = output row
+    const int row = tid;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float tot[BN];
+#pragma unroll
+    for (int c = 0; c < BN; ++c) tot[c] = 0.f;
+    for (int kt = 0; kt < KT; ++kt) {
+      wait(&hfull[kt & 1], (uint32_t)((kt >> 1) & 1));
+      tc05::fence_after_sync();
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tc05::ld32(lane_base + (uint32_t)((kt & 1) * BN + c0), v);
+        tc05::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
+      }
+      tc05::fence_before_sync();
+      mbar_arrive(&hfree[kt & 1]);
+    }
+    wait(done, 0);
+    tc05::fence_after_sync();
+#pragma unroll
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t v[32];
+      tc05::ld32(lane_base + (uint32_t)(2 * BN + c0), v);
+      tc05::wait_ld();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
+    }
+    tc05::fence_before_sync();
+    const int m = m0 + row;
+    if (m < a.M) {
+      const int b = m / a.T, t = m - b * a.T;
+      const int pos = a.seq_lens[b];
+      if (pos >= 0 && (long long)pos + a.T <= a.L_cap) {  // else refused (flagged by the advance kernel)
+        const float ip = a.inv_p[m];
+        const int Q = a.bits == 8 ? 127 : 7;
+        constexpr int HEADS = BN / R < 1 ? 1 : BN / R;
+#pragma unroll
+        for (int hb = 0; hb < HEADS; ++hb) {
+          const int h = (nl + hb * R) / R;
+          float amax = 0.f;
+#pragma unroll
+          for (int j = 0; j < R; ++j) {
+            tot[hb * R + j] *= ip;
+            amax = fmaxf(amax, fabsf(tot[hb * R + j]));
+          }
+          const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
+          const float sc = __half2float(sh);
+          const size_t crow = ((size_t)b * a.H + h) * a.L_cap + pos + t;
+          if (a.bits == 8) {
+            uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * R);
+#pragma unroll
+            for (int j4 = 0; j4 < R / 4; ++j4) {
+              uint32_t w = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 4 * j4 + k], sc)))) : 0;
+                w |= ((uint32_t)code & 0xFFu) << (8 * k);
+              }
+              dst[j4] = w;
+            }
+          } else {
+            uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * (R / 2));
+#pragma unroll
+            for (int j8 = 0; j8 < R / 8; ++j8) {
+              uint32_t w = 0;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 8 * j8 + k], sc)))) : 0;
+                w |= ((uint32_t)code & 0xFu) << (4 * k);
+              }
+              dst[j8] = w;
+            }
+          }
+          (kv ? a.scale_v : a.scale_k)[crow] = sh;
+        }
+      }
+    }
+  }
+  tc05::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc05::fence_after_sync();
+    tc05::dealloc(tmem, C::TCOLS);
+  }
+}
+
+// Tensor maps are encoded on the host through the driver's entry point (no
+// link-time dependence on the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+CUtensorMapSwizzle swizzle_for(int inner_bytes) {
+  return inner_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                           : (inner_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Activations [M][E] fp16: boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool encode_act_map(CUtensorMap* tm, const void* base, int M, int E) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)E, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)E * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcBM};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Weights [H][E][r] fp16 as a 3-D tensor (j, e, h): boxes of NG columns x 64 rows of one head.
+bool encode_weight_map(CUtensorMap* tm, const void* base, int H, int E, int r, int NG) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)r, (cuuint64_t)E, (cuuint64_t)H};
+  const cuuint64_t strides[2] = {(cuuint64_t)r * 2, (cuuint64_t)E * r * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)NG, (cuuint32_t)kTcBK, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(NG * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R>
+cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, int32_t* err, cudaStream_t s) {
+  using C = TcCfg<R>;
+  CUtensorMap mh, ml, mk, mv;
+  if (!encode_act_map(&mh, pa.xhi, pa.M, pa.E) || !encode_act_map(&ml, pa.xlo, pa.M, pa.E) ||
+      !encode_weight_map(&mk, A_k, pa.H, pa.E, R, C::NG) || !encode_weight_map(&mv, A_v, pa.H, pa.E, R, C::NG))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  TcArgs ta{};
+  ta.M = pa.M; ta.T = pa.T; ta.H = pa.H; ta.bits = pa.bits; ta.L_cap = pa.L_cap; ta.KT = pa.E / kTcBK;
+  ta.inv_p = pa.inv_p; ta.seq_lens = pa.seq_lens;
+  ta.lat_k = pa.lat_k; ta.lat_v = pa.lat_v; ta.scale_k = pa.scale_k; ta.scale_v = pa.scale_v; ta.err = err;
+  const dim3 grid((unsigned)((pa.M + kTcBM - 1) / kTcBM), (unsigned)(pa.N / C::BN));
+  prefill_tc_kernel<R><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
+  return cudaGetLastError();
+}
+
+// The tcgen05 path serves r in {16, 32, 64, 128} when every output tile holds
+// whole heads of one side (H * r a multiple of the tile width).
+bool tc_supported(int H, int r) {
+  if (r != 16 && r != 32 && r != 64 && r != 128) return false;
+  const int bn = r <= 64 ? 64 : 128;
+  return ((long long)H * r) % bn == 0;
+}
+
 // ------------------------------------------------------------------ 3. lengths
 __global__ void prefill_advance_kernel(int32_t* seq_lens, int B, int T, int L_cap, int32_t* err) {
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
@@ -442,8 +760,19 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
   prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(
       x, x_dtype, E, hadamard_block, (float)(1.0 / sqrt((double)hadamard_block)), reinterpret_cast<__half*>(w),
       reinterpret_cast<__half*>(w + xbytes), reinterpret_cast<float*>(w + 2 * xbytes));
-  const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)((N + kBN - 1) / kBN));
-  prefill_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(a);
+  if (tc_supported(H, r)) {
+    cudaError_t e = cudaSuccess;
+    switch (r) {
+      case 16: e = launch_tc<16>(a, A_k, A_v, err, s); break;
+      case 32: e = launch_tc<32>(a, A_k, A_v, err, s); break;
+      case 64: e = launch_tc<64>(a, A_k, A_v, err, s); break;
+      default: e = launch_tc<128>(a, A_k, A_v, err, s); break;
+    }
+    if (e != cudaSuccess) return WSVD_ERR_CUDA;
+  } else {
+    const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)((N + kBN - 1) / kBN));
+    prefill_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(a);
+  }
   prefill_advance_kernel<<<1, 128, 0, s>>>(seq_lens, B, T, L_cap, err);
   return cudaGetLastError() == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
 }

@@ -21,6 +21,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);  // descriptor version 1, layout 0 (none)
 }
 
+// Swizzled variant: `layout` 2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle
+// (the patterns TMA writes with CU_TENSOR_MAP_SWIZZLE_128B / 64B / 32B; the
+// atom -- 8 rows of the swizzle width -- must be aligned to its own size).
+//   K-major:  rows of the swizzle width, sbo = next 8-row group (lbo unused);
+//   MN-major: sbo = next 8-row group along K, lbo = next swizzle-width group along M/N.
+__device__ __forceinline__ uint64_t smem_desc_sw(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return smem_desc(saddr, lbo, sbo) | ((uint64_t)layout << 61);
+}
+
 // Instruction descriptor of a dense MMA (cta_group::1).
 //   cfmt: accumulator 1 = f32, 2 = s32; afmt / bfmt: kind::f16 0 = f16, kind::i8 1 = signed;
 //   amaj / bmaj: 0 = K-major, 1 = MN-major.
@@ -86,6 +95,18 @@ __device__ __forceinline__ void ld8(uint32_t taddr, uint32_t (&v)[8]) {
                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
                : "r"(taddr)
                : "memory");
+}
+// 32 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
 }
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
