@@ -147,6 +147,94 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
   if (tid == 0) inv_p[m] = __uint_as_float((uint32_t)(127 - k) << 23);
 }
 
+// Register / shuffle version of the same rotation for rows of E = 128 * EPT
+// values (EPT a power of two <= 64) and blocks of at most 32 * EPT: 128
+// threads, thread i holds the EPT consecutive values i*EPT ..; butterfly
+// distances below EPT stay in registers, distances EPT .. 16*EPT are lane
+// exchanges inside the warp, so the only block-wide step is the maximum.
+// The arithmetic per value is the shared-memory kernel's (the same adds and
+// subtracts in the same stage order, the same normalisation, p_m and split).
+template <int EPT>
+__global__ void __launch_bounds__(128) prefill_rotate_reg_kernel(const void* x, int x_dtype, int E, int blk,
+                                                                 float hnorm, __half* xhi, __half* xlo,
+                                                                 float* inv_p) {
+  __shared__ float wmax[4];
+  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)m * E + (size_t)tid * EPT;
+  float v[EPT];
+#pragma unroll
+  for (int k = 0; k < EPT; k += 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(xr + k);
+    v[k] = x_value((uint16_t)(w.x & 0xffffu), x_dtype);
+    v[k + 1] = x_value((uint16_t)(w.x >> 16), x_dtype);
+    v[k + 2] = x_value((uint16_t)(w.y & 0xffffu), x_dtype);
+    v[k + 3] = x_value((uint16_t)(w.y >> 16), x_dtype);
+  }
+  // distances inside the thread's EPT values
+#pragma unroll
+  for (int hh = 1; hh < EPT; hh <<= 1) {
+    if (hh >= blk) break;
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      if (i & hh) continue;
+      const float u = v[i], w = v[i + hh];
+      v[i] = u + w;
+      v[i + hh] = u - w;
+    }
+  }
+  // distances EPT, 2 EPT, ...: partner lane tid ^ d holds element i +- d*EPT
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    if (d * EPT >= blk) break;
+    const bool upper = lane & d;
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], d);
+      v[i] = upper ? o - v[i] : v[i] + o;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) {
+    v[i] *= hnorm;
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) wmax[tid >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  int k = 0;
+  if (amax > 0.f) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 127;
+    k = max(-126, min(126, 14 - e));
+  }
+  const float p = __uint_as_float((uint32_t)(127 + k) << 23);
+  uint2* hi4 = reinterpret_cast<uint2*>(xhi + (size_t)m * E + (size_t)tid * EPT);
+  uint2* lo4 = reinterpret_cast<uint2*>(xlo + (size_t)m * E + (size_t)tid * EPT);
+#pragma unroll
+  for (int i = 0; i < EPT; i += 4) {
+    uint32_t hw[2], lw[2];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float t = v[i + q] * p;
+      const __half h = __float2half_rn(t);
+      const __half l = __float2half_rn(t - __half2float(h));
+      const int wi = q >> 1, sh = 16 * (q & 1);
+      if ((q & 1) == 0) {
+        hw[wi] = (uint32_t)__half_as_ushort(h);
+        lw[wi] = (uint32_t)__half_as_ushort(l);
+      } else {
+        hw[wi] |= (uint32_t)__half_as_ushort(h) << sh;
+        lw[wi] |= (uint32_t)__half_as_ushort(l) << sh;
+      }
+    }
+    hi4[i / 4] = make_uint2(hw[0], hw[1]);
+    lo4[i / 4] = make_uint2(lw[0], lw[1]);
+  }
+  if (tid == 0) inv_p[m] = __uint_as_float((uint32_t)(127 - k) << 23);
+}
+
 // ------------------------------------------------------------------ 2. GEMM + quantise
 // 16-byte cp.async; a false `valid` copies nothing and zero-fills the destination.
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
@@ -757,9 +845,25 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
       cudaFuncSetAttribute(prefill_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) !=
           cudaSuccess)
     return WSVD_ERR_CUDA;
-  prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(
-      x, x_dtype, E, hadamard_block, (float)(1.0 / sqrt((double)hadamard_block)), reinterpret_cast<__half*>(w),
-      reinterpret_cast<__half*>(w + xbytes), reinterpret_cast<float*>(w + 2 * xbytes));
+  const float hnorm = (float)(1.0 / sqrt((double)hadamard_block));
+  __half* whi = reinterpret_cast<__half*>(w);
+  __half* wlo = reinterpret_cast<__half*>(w + xbytes);
+  float* winv = reinterpret_cast<float*>(w + 2 * xbytes);
+  const int ept = E / 128;
+  const bool reg_path = E % 128 == 0 && (ept & (ept - 1)) == 0 && ept >= 4 && ept <= 64 &&
+                        hadamard_block <= 32 * ept;
+  if (reg_path) {
+    switch (ept) {
+      case 4: prefill_rotate_reg_kernel<4><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+      case 8: prefill_rotate_reg_kernel<8><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+      case 16: prefill_rotate_reg_kernel<16><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+      case 32: prefill_rotate_reg_kernel<32><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+      default: prefill_rotate_reg_kernel<64><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+    }
+  } else {
+    prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo,
+                                                                     winv);
+  }
   if (tc_supported(H, r)) {
     cudaError_t e = cudaSuccess;
     switch (r) {
