@@ -980,7 +980,9 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
           cid = next;
         }
         // This CTA has made its last claim; the last CTA to get here clears
-        // the claim counters for the next call.
+        // the claim counters for the next call (the fence orders this CTA's
+        // claims before its count).
+        __threadfence();
         if (atomicAdd(a.work + 1, 1) == (int)gridDim.x - 1) {
           atomicExch(a.work, 0);
           atomicExch(a.work + 1, 0);
