@@ -65,6 +65,7 @@ struct GroupedArgs {
   const __half* Bv;
   float qscale;      // softmax_scale * log2 e
   float* out;        // [B][Tq][Hq][Hd]
+  const uint8_t* qplanes;  // [B * Hkv * nqc] blocks of the q' planes (score operand layout) + steps
   float* partials;   // [B * Hkv * nqc][slot_stride][NQ][r + 2]
   int32_t* counters; // [B * Hkv * nqc], zero between calls
   int32_t* err;
@@ -93,19 +94,19 @@ struct GCfg {
   static constexpr int PB = kGTok * NO * 2;
   static constexpr int LBO_PL = NS * 16;
   static constexpr int PL = NS * KB;
+  static constexpr int QBLOCK = PL + NQ * 4;                     // per query group: planes, then steps
   static constexpr int OFF_AK = S * STAGE;
   static constexpr int OFF_VC = OFF_AK + 2 * AK;
   static constexpr int OFF_P = OFF_VC + 2 * VC;
   static constexpr int OFF_PL = OFF_P + 2 * PB;
-  static constexpr int OFF_QP = OFF_PL + PL;                     // float qp[NQ][R]
-  static constexpr int OFF_STEP = OFF_QP + NQ * R * 4;           // float step[NQ], inv[NQ]
+  static constexpr int OFF_STEP = OFF_PL + PL;                   // float step[NQ] (staged with the planes)
   static constexpr int OFF_WMAX = OFF_STEP + 2 * NQ * 4;         // float wmax[2][4][NQ]
   static constexpr int OFF_WSV = OFF_WMAX + 2 * 4 * NQ * 4;      // uint32 wsv[2][4]
   static constexpr int OFF_LSUM = OFF_WSV + 8 * 4;               // float lsum[4][NQ]
   static constexpr int OFF_RES = OFF_LSUM + 4 * NQ * 4;          // float res[NQ][R + 2]
   static constexpr int OFF_MISC = OFF_RES + NQ * (R + 2) * 4;    // int flag, uint32 tmem base
   static constexpr int OFF_BAR = (OFF_MISC + 16 + 7) / 8 * 8;
-  static constexpr int NBAR = 2 * S + 8;
+  static constexpr int NBAR = 2 * S + 9;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8;
   // Shared memory requested at launch: at least enough that no more CTAs are
   // resident on an SM than its 512 tensor-memory columns can serve at once
@@ -181,6 +182,61 @@ __device__ __forceinline__ uint4 i4x8_to_h(uint32_t w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// q' of every query of one (b, latent head, query chunk) group, as the score
+// operand the decode kernel stages: q'_q = (B_Kh . q_q) * softmax_scale * log2 e
+// (8 lanes per row, a fixed shuffle tree), quantised with step max|q'_q| / 8355711
+// and written as three signed byte planes in the K-major no-swizzle layout,
+// followed by the NQ steps.  One CTA per group; the decode grid is launched
+// behind it as a programmatic dependent.
+template <int CODEC, int RB, int NQ>
+__global__ void __launch_bounds__(128) grouped_qproj_kernel(const GroupedArgs a, uint8_t* qplanes) {
+  using C = GCfg<CODEC, RB, NQ>;
+  constexpr int R = C::R, NS = C::NS;
+  __shared__ float qp[NQ * R];
+  __shared__ float inv[NQ];
+  griddep_launch_dependents();
+  const int grp = blockIdx.x, t = threadIdx.x, lane = t & 31;
+  const int qc = grp % a.nqc, hkv = (grp / a.nqc) % a.Hkv, b = grp / (a.nqc * a.Hkv);
+  const int nq = min(NQ, a.G * a.Tq - qc * NQ);
+  const int part = lane & 7;
+  for (int row = t >> 3; row < NQ * R; row += 128 / 8) {
+    const int ql = row / R, j = row % R;
+    float d = 0.f;
+    if (ql < nq) {
+      const int qg = qc * NQ + ql, tq = qg / a.G, g = qg % a.G;
+      const size_t qrow = (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd;
+      const __half* brow = a.Bk + ((size_t)hkv * R + j) * a.Hd;
+      for (int k = part; k < a.Hd; k += 8) d = fmaf(__half2float(brow[k]), load_q_elem(a.q, a.q_dtype, qrow + k), d);
+    }
+    d += __shfl_xor_sync(0xffffffffu, d, 1);
+    d += __shfl_xor_sync(0xffffffffu, d, 2);
+    d += __shfl_xor_sync(0xffffffffu, d, 4);
+    if (part == 0) qp[row] = d * a.qscale;
+  }
+  __syncthreads();
+  uint8_t* blk = qplanes + (size_t)grp * C::QBLOCK;
+  float* steps = reinterpret_cast<float*>(blk + C::PL);
+  if (t < NQ) {
+    float m = 0.f;
+    for (int j = 0; j < R; ++j) m = fmaxf(m, fabsf(qp[t * R + j]));
+    steps[t] = m > 0.f ? m / (float)kQMax : 0.f;
+    inv[t] = m > 0.f ? (float)kQMax / m : 0.f;
+  }
+  __syncthreads();
+  for (int idx = t; idx < NS * C::KB; idx += 128) {
+    const int n = idx / C::KB, k = idx % C::KB;
+    int dig = 0;
+    if (n < 3 * NQ && k < R) {
+      const int ql = n / 3, p = n % 3;
+      const int x = max(-kQMax, min(kQMax, __float2int_rn(qp[ql * R + k] * inv[ql])));
+      const int l0 = ((x + 128) & 255) - 128, x1 = (x - l0) >> 8;
+      const int m0 = ((x1 + 128) & 255) - 128, h0 = (x1 - m0) >> 8;
+      dig = p == 0 ? h0 : (p == 1 ? m0 : l0);
+    }
+    blk[(k >> 4) * C::LBO_PL + (n >> 3) * 128 + (n & 7) * 16 + (k & 15)] = (uint8_t)(int8_t)dig;
+  }
+}
+
 template <int CODEC, int RB, int NQ>
 __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const GroupedArgs a) {
   using C = GCfg<CODEC, RB, NQ>;
@@ -214,9 +270,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   uint8_t* ring = smem;
   const uint32_t s_ak = smem_u32(smem + C::OFF_AK), s_vc = smem_u32(smem + C::OFF_VC);
   const uint32_t s_p = smem_u32(smem + C::OFF_P), s_pl = smem_u32(smem + C::OFF_PL);
-  float* qp = reinterpret_cast<float*>(smem + C::OFF_QP);
   float* stepv = reinterpret_cast<float*>(smem + C::OFF_STEP);
-  float* invv = stepv + NQ;
   float* wmax = reinterpret_cast<float*>(smem + C::OFF_WMAX);
   uint32_t* wsv = reinterpret_cast<uint32_t*>(smem + C::OFF_WSV);
   float* lsum = reinterpret_cast<float*>(smem + C::OFF_LSUM);
@@ -229,6 +283,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   uint64_t* sready = conv + 2;  // [2] score MMAs done (commit)
   uint64_t* pfull = sready + 2; // [2] P~ written (128 arrivals)
   uint64_t* oready = pfull + 2; // [2] value MMAs done (commit)
+  uint64_t* pready = oready + 2; // the group's q' planes and steps are staged
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -241,6 +296,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       mbar_init(&pfull[s], kGConsumers);
       mbar_init(&oready[s], 1);
     }
+    mbar_init(pready, 1);
     fence_mbar_init();
   }
   if (warp == kGMmaWarp) tc05::alloc(tmem_slot, C::TCOLS);
@@ -261,7 +317,16 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
+      const int gidx = (b * a.Hkv + hkv) * a.nqc + qc;
       for (int i = 0; i < ntiles; ++i) {
+        if (i == min(S, ntiles)) {  // the ring is primed: now the planes (they come from the preceding grid)
+          griddep_wait();
+          mbar_arrive_expect_tx(pready, (uint32_t)C::QBLOCK);
+          bulk_g2s(smem + C::OFF_PL, a.qplanes + (size_t)gidx * C::QBLOCK, (uint32_t)C::PL, pready,
+                   l2_evict_last_policy());
+          bulk_g2s(smem + C::OFF_STEP, a.qplanes + (size_t)gidx * C::QBLOCK + C::PL, (uint32_t)(NQ * 4), pready,
+                   l2_evict_last_policy());
+        }
         const int s = i % S;
         if (i >= S) wait(&empty[s], (uint32_t)(((i / S) - 1) & 1));
         const int r0 = t_begin + i * kGTok, n = min(kGTok, t_end - r0);
@@ -273,8 +338,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         bulk_g2s(st + 2 * kGTok * RB, a.scale_k + head_row + r0, sb, &full[s], pol);
         bulk_g2s(st + 2 * kGTok * RB + 2 * kGTok, a.scale_v + head_row + r0, sb, &full[s], pol);
       }
-      // no copy left in flight: the last uses of every stage have landed
+      if (ntiles <= S) {  // fewer tiles than stages: the planes follow the last tile
+        griddep_wait();
+        mbar_arrive_expect_tx(pready, (uint32_t)C::QBLOCK);
+        bulk_g2s(smem + C::OFF_PL, a.qplanes + (size_t)gidx * C::QBLOCK, (uint32_t)C::PL, pready,
+                 l2_evict_last_policy());
+        bulk_g2s(smem + C::OFF_STEP, a.qplanes + (size_t)gidx * C::QBLOCK + C::PL, (uint32_t)(NQ * 4), pready,
+                 l2_evict_last_policy());
+      }
+      // no copy left in flight: the last uses of every stage and the planes have landed
       for (int i = max(0, ntiles - S); i < ntiles; ++i) wait(&full[i % S], (uint32_t)((i / S) & 1));
+      wait(pready, 0);
     }
   } else if (warp == kGMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -292,6 +366,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
                        tc05::smem_desc(s_pl + kk * 2 * C::LBO_PL, C::LBO_PL, 128), idesc_s, kk > 0);
         tc05::commit(&sready[j & 1]);
       };
+      wait(pready, 0);  // the q' planes (score operand B) are staged
       scores(0);
       for (int i = 0; i < ntiles; ++i) {
         if (i + 1 < ntiles) scores(i + 1);
@@ -312,40 +387,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   } else {
     // ------------------------------------------------------------ consumers
     const int t = tid;  // token slot of the tile, tensor-memory lane
-    // q'_q = B_Kh . q_q * softmax_scale * log2 e for the CTA's queries
-    for (int idx = t; idx < NQ * R; idx += kGConsumers) {
-      const int ql = idx / R, j = idx % R;
-      float d = 0.f;
-      if (ql < nq) {
-        const int qg = qc * NQ + ql, tq = qg / a.G, g = qg % a.G;
-        const size_t qrow = (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd;
-        const __half* brow = a.Bk + ((size_t)hkv * R + j) * a.Hd;
-        for (int k = 0; k < a.Hd; ++k) d = fmaf(__half2float(brow[k]), load_q_elem(a.q, a.q_dtype, qrow + k), d);
-        d *= a.qscale;
-      }
-      qp[idx] = d;
-    }
-    named_barrier_sync(1, kGConsumers);
-    if (t < NQ) {
-      float m = 0.f;
-      for (int j = 0; j < R; ++j) m = fmaxf(m, fabsf(qp[t * R + j]));
-      stepv[t] = m > 0.f ? m / (float)kQMax : 0.f;
-      invv[t] = m > 0.f ? (float)kQMax / m : 0.f;
-    }
-    named_barrier_sync(1, kGConsumers);
-    // signed byte planes of q' (rows 3 q + plane, K-major, zero padding)
-    for (int idx = t; idx < NS * C::KB; idx += kGConsumers) {
-      const int n = idx / C::KB, k = idx % C::KB;
-      int dig = 0;
-      if (n < 3 * NQ && k < R) {
-        const int ql = n / 3, p = n % 3;
-        const int x = max(-kQMax, min(kQMax, __float2int_rn(qp[ql * R + k] * invv[ql])));
-        const int l0 = ((x + 128) & 255) - 128, x1 = (x - l0) >> 8;
-        const int m0 = ((x1 + 128) & 255) - 128, h0 = (x1 - m0) >> 8;
-        dig = p == 0 ? h0 : (p == 1 ? m0 : l0);
-      }
-      smem[C::OFF_PL + (k >> 4) * C::LBO_PL + (n >> 3) * 128 + (n & 7) * 16 + (k & 15)] = (uint8_t)(int8_t)dig;
-    }
+    wait(pready, 0);  // the group's steps (and planes) are staged
     float step[NQ];
     int nvis[NQ];  // rows visible to each query
 #pragma unroll
@@ -435,7 +477,6 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 
     float sk_cur, sv_cur;
     int pos_cur, e_prev = 0;
-    tc05::fence_proxy_async_smem();  // the planes, before the first hand-over
     convert(0, sk_cur, sv_cur, pos_cur);
     for (int i = 0; i < ntiles; ++i) {
       if (i >= 1) accumulate(i - 1, e_prev);
@@ -585,32 +626,39 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 // ---------------------------------------------------------------- host side
 int nq_per_cta(int nq_group) { return nq_group <= 4 ? 4 : (nq_group <= 8 ? 8 : 16); }
 
+struct GroupedKernels {
+  const void* qproj;   // grouped_qproj_kernel
+  const void* decode;  // grouped_decode_kernel
+  size_t smem;
+};
+
 template <int CODEC, int RB, int NQ>
-const void* kernel_of(size_t* smem) {
-  *smem = GCfg<CODEC, RB, NQ>::SMEM;
-  return reinterpret_cast<const void*>(&grouped_decode_kernel<CODEC, RB, NQ>);
+GroupedKernels kernels_of() {
+  return GroupedKernels{reinterpret_cast<const void*>(&grouped_qproj_kernel<CODEC, RB, NQ>),
+                        reinterpret_cast<const void*>(&grouped_decode_kernel<CODEC, RB, NQ>),
+                        (size_t)GCfg<CODEC, RB, NQ>::SMEM};
 }
 
 template <int CODEC, int RB>
-const void* pick_nq(int nq, size_t* smem) {
+GroupedKernels pick_nq(int nq) {
   switch (nq) {
-    case 4: return kernel_of<CODEC, RB, 4>(smem);
-    case 8: return kernel_of<CODEC, RB, 8>(smem);
-    default: return kernel_of<CODEC, RB, 16>(smem);
+    case 4: return kernels_of<CODEC, RB, 4>();
+    case 8: return kernels_of<CODEC, RB, 8>();
+    default: return kernels_of<CODEC, RB, 16>();
   }
 }
 
-const void* pick_grouped(int bits, int rb, int nq, size_t* smem) {
+bool pick_grouped(int bits, int rb, int nq, GroupedKernels* k) {
   if (bits == 8) {
-    if (rb == 16) return pick_nq<kCodecI8, 16>(nq, smem);
-    if (rb == 32) return pick_nq<kCodecI8, 32>(nq, smem);
-    if (rb == 64) return pick_nq<kCodecI8, 64>(nq, smem);
+    if (rb == 16) { *k = pick_nq<kCodecI8, 16>(nq); return true; }
+    if (rb == 32) { *k = pick_nq<kCodecI8, 32>(nq); return true; }
+    if (rb == 64) { *k = pick_nq<kCodecI8, 64>(nq); return true; }
   } else {
-    if (rb == 16) return pick_nq<kCodecI4, 16>(nq, smem);
-    if (rb == 32) return pick_nq<kCodecI4, 32>(nq, smem);
-    if (rb == 64) return pick_nq<kCodecI4, 64>(nq, smem);
+    if (rb == 16) { *k = pick_nq<kCodecI4, 16>(nq); return true; }
+    if (rb == 32) { *k = pick_nq<kCodecI4, 32>(nq); return true; }
+    if (rb == 64) { *k = pick_nq<kCodecI4, 64>(nq); return true; }
   }
-  return nullptr;
+  return false;
 }
 
 std::mutex g_mu;
@@ -647,7 +695,7 @@ inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
 struct GroupedShape {
   int nq, nqc, slots;
-  size_t partial_bytes, total;
+  size_t partial_bytes, counter_bytes, plane_bytes, total;
 };
 GroupedShape grouped_shape(int B, int Tq, int Hq, int Hkv, int r, int L_cap) {
   GroupedShape s{};
@@ -657,7 +705,11 @@ GroupedShape grouped_shape(int B, int Tq, int Hq, int Hkv, int r, int L_cap) {
   const int tiles_cap = std::max(1, (L_cap + kGTok - 1) / kGTok);
   s.slots = std::min(tiles_cap, kMaxGroupedSplits);
   s.partial_bytes = align16((size_t)B * Hkv * s.nqc * s.slots * s.nq * (r + 2) * sizeof(float));
-  s.total = s.partial_bytes + align16((size_t)B * Hkv * s.nqc * 4);
+  s.counter_bytes = align16((size_t)B * Hkv * s.nqc * 4);
+  // q' planes per group: (3 nq rounded up to 16) rows of max(32, r) bytes, then nq fp32 steps
+  const size_t qblock = (size_t)((3 * s.nq + 15) / 16 * 16) * (r < 32 ? 32 : r) + (size_t)s.nq * 4;
+  s.plane_bytes = align16((size_t)B * Hkv * s.nqc * qblock);
+  s.total = s.partial_bytes + s.counter_bytes + s.plane_bytes;
   return s;
 }
 
@@ -696,11 +748,11 @@ extern "C" int wsvd_decode_multi(int B, int Tq, int Hq, int Hkv, int Hd, int r, 
   const GroupedShape sh = grouped_shape(B, Tq, Hq, Hkv, r, L_cap);
   if ((size_t)Hkv * sh.nqc > 65535) return WSVD_ERR_UNSUPPORTED;
   if (workspace_bytes < sh.total) return WSVD_ERR_WORKSPACE_TOO_SMALL;
-  size_t smem = 0;
-  const void* fn = pick_grouped(bits, rb, sh.nq, &smem);
-  if (!fn) return WSVD_ERR_UNSUPPORTED;
+  GroupedKernels gk{};
+  if (!pick_grouped(bits, rb, sh.nq, &gk)) return WSVD_ERR_UNSUPPORTED;
+  const size_t smem = gk.smem;
   int sms = 148, occ = 1;
-  if (device_setup(fn, smem, &sms, &occ) != cudaSuccess) return WSVD_ERR_CUDA;
+  if (device_setup(gk.decode, smem, &sms, &occ) != cudaSuccess) return WSVD_ERR_CUDA;
 
   GroupedArgs ga{};
   ga.B = B; ga.Tq = Tq; ga.Hq = Hq; ga.Hkv = Hkv; ga.G = G; ga.Hd = Hd; ga.L_cap = L_cap;
@@ -720,14 +772,32 @@ extern "C" int wsvd_decode_multi(int B, int Tq, int Hq, int Hkv, int Hd, int r, 
   ga.out = out;
   ga.partials = static_cast<float*>(workspace);
   ga.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + sh.partial_bytes);
+  uint8_t* planes = static_cast<uint8_t*>(workspace) + sh.partial_bytes + sh.counter_bytes;
+  ga.qplanes = planes;
   ga.err = err;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  {  // q' planes of every query group
+    void* pargs[] = {&ga, &planes};
+    cudaLaunchConfig_t pcfg = {};
+    pcfg.gridDim = dim3((unsigned)groups);
+    pcfg.blockDim = dim3(128);
+    pcfg.stream = st;
+    if (cudaLaunchKernelExC(&pcfg, gk.qproj, pargs) != cudaSuccess) return WSVD_ERR_CUDA;
+  }
+  // The decode grid behind it as a programmatic dependent: it starts streaming
+  // tiles while the projection runs and stages the planes after griddepcontrol.wait.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   void* args[] = {&ga};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ga.nsplit, Hkv * sh.nqc, B);
   cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  return cudaLaunchKernelExC(&cfg, fn, args) == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, gk.decode, args) == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
 }
 
 extern "C" size_t wsvd_decode_gqa_workspace_size(int B, int Hq, int Hkv, int r, int L_cap) {

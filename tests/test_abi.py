@@ -195,13 +195,14 @@ def test_grouped_decode_workspace_and_validation(lib):
     a16 = lambda v: (v + 15) // 16 * 16
     B, Tq, Hq, Hkv, r, L = 2, 4, 32, 8, 32, 1600
     nq, nqc, slots = 16, 1, 13  # G * Tq = 16 queries; ceil(1600 / 128) = 13 tiles
-    want = a16(B * Hkv * nqc * slots * nq * (r + 2) * 4) + a16(B * Hkv * nqc * 4)
+    qblock = 48 * 32 + 16 * 4    # q' planes of a group: 3 x 16 rows of 32 bytes, then 16 steps
+    want = a16(B * Hkv * nqc * slots * nq * (r + 2) * 4) + a16(B * Hkv * nqc * 4) + a16(B * Hkv * nqc * qblock)
     assert W.wsvd_decode_multi_workspace_size(B, Tq, Hq, Hkv, r, L) == want
     assert lib.wsvd_decode_gqa_workspace_size(B, Hq, Hkv, r, L) == W.wsvd_decode_multi_workspace_size(
         B, 1, Hq, Hkv, r, L)
     # G * Tq = 32 queries: two chunks of 16; 64-split cap at 32768 tokens
     assert W.wsvd_decode_multi_workspace_size(1, 4, 32, 4, 32, 32768) == \
-        a16(1 * 4 * 2 * 64 * 16 * 34 * 4) + a16(1 * 4 * 2 * 4)
+        a16(1 * 4 * 2 * 64 * 16 * 34 * 4) + a16(1 * 4 * 2 * 4) + a16(1 * 4 * 2 * qblock)
     p = ctypes.c_void_p(16)
     ws = 1 << 24
     args = lambda B=1, Tq=1, Hq=8, Hkv=2, Hd=64, r=32, bits=8, L=64, qp=p: (
