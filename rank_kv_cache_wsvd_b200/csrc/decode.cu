@@ -1341,45 +1341,77 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
         const int v = clamp_len(ld_relaxed_gpu(a.seq_lens + b), a.L_cap);
         pre_end = max(lo, min(hi, v - 1) & ~7);
       }
-      const int npre = (pre_end - lo) / T, part = (pre_end - lo) % T;  // whole tiles below the bound, rows of the next
-      tile_info[S] = npre;
-      mbar_arrive(&aux[2]);
-      for (int i = 0; i < npre && ok; ++i) {
-        const int s = claim(i);
-        if (!ok) break;
-        tile_info[s] = T;
-        mbar_arrive_expect_tx(&full[s], tile_bytes(T));
-        copy_rows(stages + (size_t)s * C::kStageBytes, lo + i * T, 0, T, &full[s]);
-      }
-      if (ok && part > 0) {
-        const int s = claim(npre);
-        if (ok) {
-          mbar_expect_tx(&full[s], tile_bytes(part));  // no arrive yet: the rest follows after the wait
-          copy_rows(stages + (size_t)s * C::kStageBytes, lo + npre * T, 0, part, &full[s]);
+      if (a.dep == 2 && hi > lo && pre_end == hi) {
+        // Every row of this rank lies below the bound: the rows are final and
+        // the final length is above hi whichever value the early read saw, so
+        // the tiles, their counts and their arithmetic are those of the plain
+        // decode; they are handed over without waiting for the append.  The
+        // leader still waits before it exits, so the grid never completes
+        // before the grid it was launched behind.
+        const int total = (hi - lo + T - 1) / T;
+        tile_info[S] = total;
+        mbar_arrive(&aux[2]);
+        for (int i = 0; i < total && ok; ++i) {
+          const int s = claim(i);
+          if (!ok) break;
+          const int n = min(T, hi - (lo + i * T));
+          tile_info[s] = n;
+          mbar_arrive_expect_tx(&full[s], tile_bytes(n));
+          copy_rows(stages + (size_t)s * C::kStageBytes, lo + i * T, 0, n, &full[s]);
         }
+        tile_info[S + 1] = total;
+        mbar_arrive(&aux[3]);
+        if (rank == 0) {
+          griddep_wait();
+          const int raw = a.seq_lens[b];
+          if ((raw < 0 || raw > a.L_cap) && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+        }
+        const int issued = ok ? total : 0;
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          if (!mbar_wait_bounded(&full[i % S], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      } else {
+        const int npre = (pre_end - lo) / T, part = (pre_end - lo) % T;  // whole tiles below the bound, rows of the next
+        tile_info[S] = npre;
+        mbar_arrive(&aux[2]);
+        for (int i = 0; i < npre && ok; ++i) {
+          const int s = claim(i);
+          if (!ok) break;
+          tile_info[s] = T;
+          mbar_arrive_expect_tx(&full[s], tile_bytes(T));
+          copy_rows(stages + (size_t)s * C::kStageBytes, lo + i * T, 0, T, &full[s]);
+        }
+        if (ok && part > 0) {
+          const int s = claim(npre);
+          if (ok) {
+            mbar_expect_tx(&full[s], tile_bytes(part));  // no arrive yet: the rest follows after the wait
+            copy_rows(stages + (size_t)s * C::kStageBytes, lo + npre * T, 0, part, &full[s]);
+          }
+        }
+        griddep_wait();
+        const int raw = a.seq_lens[b];
+        if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+        const int end = max(pre_end, min(hi, clamp_len(raw, a.L_cap)));  // pre_end <= end holds by construction
+        const int total = end > lo ? (end - lo + T - 1) / T : 0;         // > npre whenever part > 0
+        tile_info[S + 1] = total;
+        mbar_arrive(&aux[3]);
+        for (int i = npre; i < total && ok; ++i) {
+          const int r0 = lo + i * T, n = min(T, end - r0);
+          const bool split = (i == npre && part > 0);
+          const int s = split ? i % S : claim(i);  // a split tile's stage was claimed before the wait
+          if (!ok) break;
+          tile_info[s] = n;
+          const int off = split ? part : 0;
+          mbar_arrive_expect_tx(&full[s], n > off ? tile_bytes(n) - tile_bytes(off) : 0u);
+          if (n > off) copy_rows(stages + (size_t)s * C::kStageBytes, r0, off, n - off, &full[s]);
+        }
+        const int issued = ok ? total : 0;
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          if (!mbar_wait_bounded(&full[i % S], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+        if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       }
-      griddep_wait();
-      const int raw = a.seq_lens[b];
-      if ((raw < 0 || raw > a.L_cap) && rank == 0 && h == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
-      const int end = max(pre_end, min(hi, clamp_len(raw, a.L_cap)));  // pre_end <= end holds by construction
-      const int total = end > lo ? (end - lo + T - 1) / T : 0;         // > npre whenever part > 0
-      tile_info[S + 1] = total;
-      mbar_arrive(&aux[3]);
-      for (int i = npre; i < total && ok; ++i) {
-        const int r0 = lo + i * T, n = min(T, end - r0);
-        const bool split = (i == npre && part > 0);
-        const int s = split ? i % S : claim(i);  // a split tile's stage was claimed before the wait
-        if (!ok) break;
-        tile_info[s] = n;
-        const int off = split ? part : 0;
-        mbar_arrive_expect_tx(&full[s], n > off ? tile_bytes(n) - tile_bytes(off) : 0u);
-        if (n > off) copy_rows(stages + (size_t)s * C::kStageBytes, r0, off, n - off, &full[s]);
-      }
-      const int issued = ok ? total : 0;
-      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % S], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-      if (!mbar_wait_bounded(segfull, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-      if (rank == 0 && a.Bv != nullptr && !mbar_wait_bounded(&aux[0], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     }
     cluster_wait();
     return;
