@@ -916,7 +916,10 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   // the CTAs that share a (b, h) are consecutive without gaps.  Dynamic plan:
   // every CTA takes part (it may claim nothing).
   const int CW = dyn ? a.ctas : (int)(G < a.ctas ? G : a.ctas);
-  if (!dyn && c >= CW) return;  // uniform across the CTA; nothing was issued
+  if (!dyn && c >= CW) {  // uniform across the CTA; nothing was issued
+    if (a.dep == 1) griddep_wait();  // the grid never completes before the q' grid it was launched behind
+    return;
+  }
 
   // ---------------------------------------------------------------- producer warp
   if (warp == kProducerWarp) {

@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   if (split >= ncontrib) {  // no cached token for this CTA (uniform exit before any set-up)
     if (split == 0)
       for (int i = tid; i < nq * a.Hd; i += kGThreads) out_row(i / a.Hd)[i % a.Hd] = 0.f;
+    griddep_wait();  // the grid never completes before the projection grid it was launched behind
     return;
   }
   const int t_begin = split * span;
