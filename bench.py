@@ -63,7 +63,8 @@ def source_digest(files):
 
 KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
                   "decode": ["decode.cu", "shared.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
-                  "prefill_gemm": ["prefill.cu", "common.cuh", "wsvd_internal.h"]}
+                  "prefill_gemm": ["prefill.cu", "common.cuh", "wsvd_internal.h", "tc05.cuh"],
+                  "grouped": ["grouped.cu", "common.cuh", "wsvd_internal.h", "tc05.cuh"]}
 
 
 def ncu_traffic(kernel: str, workload: str):
@@ -731,7 +732,9 @@ def main():
                            "parallelism": f"replicas x{world}"},
                 "roofline": {"bound": "hbm", "kernel": "grouped_decode_kernel (1 launch)", "achieved": gr["gbs"],
                              "peak": peak, "unit": "GB/s", "frac": gr["gbs"] / peak, "peak_kind": kind,
-                             "traffic": None, "alg_bytes_per_launch": gr["alg_bytes"],
+                             "traffic": ncu_traffic("grouped", args.grouped_workload),
+                             "traffic_kernel": "grouped_decode_kernel (DRAM bytes per launch, ncu)",
+                             "alg_bytes_per_launch": gr["alg_bytes"],
                              "tensor_tops_executed": gr["tensor_tops_executed"]},
                 "grouped": gr, "gpu_launches": args.steps, "clocks": clk}), flush=True)
         if world > 1:
