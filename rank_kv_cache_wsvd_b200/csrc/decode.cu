@@ -1644,11 +1644,15 @@ bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* 
   // With several tiles per CTA the work is claimed dynamically, in chunks of
   // whole tiles of one (b, h): about 16 chunks per CTA, at most 32 per (b, h)
   // (the workspace's partial slots), so that CTAs that stream faster take more.
+  // A chunk also carries at least ~64 KB, so that the hand-off at its end (a
+  // reduction across the consumer warps) stays small next to its streaming.
   int chunk = 0;
   if (tiles_max > ctas) {
     const long long tph = (a.L_cap + ki.tile - 1) / ki.tile;
     const long long want = (tiles_max + 16 * ctas - 1) / (16 * ctas);
-    chunk = (int)std::max<long long>(1, std::max<long long>(want, (tph + 31) / 32));
+    const long long tile_bytes = (long long)ki.tile * (2 * rowbytes + (codec == kCodecF16 ? 0 : 4));
+    const long long min_tiles = (65536 + tile_bytes - 1) / tile_bytes;
+    chunk = (int)std::max<long long>(std::max<long long>(1, min_tiles), std::max<long long>(want, (tph + 31) / 32));
   }
   pl->cluster = false;
   pl->csize = 0;
