@@ -19,13 +19,12 @@ inline float resolve_scale(float softmax_scale, int Hd) {
 inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
 // Decode workspace: split partials (m, l, o[W]) for every slot a persistent
-// grid can use, one completion counter per (b, h) and the two claim counters
-// of the dynamic plan, then the projected query q' [B][H][W] fp32 of the
-// persistent path.
+// grid can use, one completion counter per (b, h), then the projected query
+// q' [B][H][W] fp32 of the persistent path.
 inline size_t partial_bytes(int B, int H, int W) {
-  return align16((size_t)decode_partial_slots(B, H) * ((size_t)W + 2) * sizeof(float));
+  return align16(((size_t)kMaxDecodeCtas + (size_t)B * H) * ((size_t)W + 2) * sizeof(float));
 }
-inline size_t counter_bytes(int B, int H) { return align16(((size_t)B * H + 2) * 4); }
+inline size_t counter_bytes(int B, int H) { return align16((size_t)B * H * 4); }
 inline size_t decode_ws_bytes(int B, int H, int W) {
   return partial_bytes(B, H, W) + counter_bytes(B, H) + align16((size_t)B * H * W * sizeof(float));
 }
@@ -35,7 +34,6 @@ void bind_workspace(DecodeArgs* a, void* workspace) {
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a->partials = reinterpret_cast<float*>(w);
   a->counters = reinterpret_cast<int32_t*>(w + partial_bytes(a->B, a->H, a->W));
-  a->work = a->counters + (size_t)a->B * a->H;
   a->qglobal = reinterpret_cast<float*>(w + partial_bytes(a->B, a->H, a->W) + counter_bytes(a->B, a->H));
 }
 

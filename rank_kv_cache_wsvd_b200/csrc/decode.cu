@@ -82,26 +82,15 @@ __host__ __device__ inline int seg_nbuf(int qmode, int W, int Hd) { return seg_b
 
 // Helper-owned shared state (after the operand buffers): NQ query-state slots
 // the helper fills ahead of the consumers, two result slots it drains.
-// One segment -- a run of tiles of one (b, h) -- as the producer hands it to
-// the helper and the consumer warps.  Its partial (m, l, o) goes to slot ps;
-// the head's np partials occupy slots p0 .. p0 + np - 1 and are merged in slot
-// order by whichever of its segments finishes last.  nt = 0 ends the queue.
-struct SegDesc {
-  int b, h, t0, nt, ps, p0, np, pad;
-};
-constexpr int kSegQ = 4;  // depth of the descriptor queue
-
 template <int W, int PW, int NQ>
 struct HelperArea {
   float qsv[NQ][W];           // scaled q' (fp16 codecs read it directly)
   uint32_t planes[NQ][PW];    // packed byte planes + int4 corrections
   float qstep[NQ];
-  SegDesc seg[NQ];            // descriptor of each built segment
-  SegDesc sq[kSegQ];          // descriptor queue, producer -> helper and consumers
+  int seginfo[NQ][4];         // b, h, c_first, c_last
   float res[2][W + 2];        // merged (M, L, O[W]) of a segment, consumers -> helper
   int qi[W];                  // quantised q'
   uint64_t bars[2 * NQ + 4];  // qready[NQ], qfree[NQ], resfull[2], resfree[2]
-  uint64_t sqbars[2 * kSegQ]; // sqfull[kSegQ], sqfree[kSegQ]
 };
 
 template <int CODEC, int VPT, int TPT, int NTOK>
@@ -135,11 +124,16 @@ struct Cfg {
   static constexpr size_t kOffParts = kOffRes + (size_t)(kW + 2) * 4;
   static constexpr size_t kOffMisc = kOffParts + (size_t)kPlaneWords * 4;
   static constexpr size_t kOffPre = kOffMisc + 16 * 4;
-  // runtime part: tile prefix, lens, chunk prefix (3B + 2 ints), then the segment buffers
-  __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(3 * B + 2) * 4 + 127) / 128 * 128; }
+  // runtime part: lens / prefix (2B + 1 ints), then the segment buffers
+  __host__ __device__ static size_t seg_off(int B) { return (kOffPre + (size_t)(2 * B + 1) * 4 + 127) / 128 * 128; }
+  // B_Vh of the CTA's last segment, staged for its finish (low-rank codecs, up
+  // to 16 KB so that two CTAs still fit an SM; larger ones read global memory).
+  __host__ __device__ static size_t bv_stage_bytes(int Hd) {
+    return (CT::kScaled && (size_t)kW * Hd * 2 <= 16384) ? (size_t)kW * Hd * 2 : 0;
+  }
   static size_t smem_bytes(int B, int qmode, int Hd) {
     return seg_off(B) + seg_nbuf(qmode, kW, Hd) * seg_bytes(qmode, kW, Hd) +
-           (sizeof(HelperArea<kW, kPlaneWords, kNQ>) + 127) / 128 * 128;
+           (sizeof(HelperArea<kW, kPlaneWords, kNQ>) + 127) / 128 * 128 + bv_stage_bytes(Hd);
   }
   // cluster kernel: operands, the leader's partial slots, then B_Vh
   __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
@@ -612,7 +606,6 @@ __device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, flo
 template <int W, bool GLOBAL>
 __device__ __forceinline__ float merge_elem(const float* part, int np, float M, int e) {
   float s2 = 0.f;
-#pragma unroll 4
   for (int p = 0; p < np; ++p) {
     const float mp = GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)];
     if (mp != kNegInf) {
@@ -625,7 +618,6 @@ __device__ __forceinline__ float merge_elem(const float* part, int np, float M, 
 template <int W, bool GLOBAL>
 __device__ __forceinline__ float merge_max(const float* part, int np) {
   float M = kNegInf;
-#pragma unroll 4
   for (int p = 0; p < np; ++p) M = fmaxf(M, GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)]);
   return M;
 }
@@ -820,66 +812,49 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
   int* pre = reinterpret_cast<int*>(smem + C::kOffPre);
   int* lens = pre + a.B + 1;
-  int* cpre = lens + a.B;  // dynamic plan: chunk prefix (H chunks-of-heads per sequence)
   uint8_t* segbuf = smem + C::seg_off(a.B);
   const int NBUF = seg_nbuf(QMODE, W, a.Hd);
   const uint32_t SEGB = (uint32_t)seg_bytes(QMODE, W, a.Hd);
   HA* ha = reinterpret_cast<HA*>(segbuf + (size_t)NBUF * SEGB);
+  __half* bv_last = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(ha) + (sizeof(HA) + 127) / 128 * 128);
+  uint64_t* bvbar = segempty + 2;  // B_Vh of the last segment staged
   uint64_t* qready = ha->bars;
   uint64_t* qfree = ha->bars + NQ;
   uint64_t* resfull = ha->bars + 2 * NQ;
   uint64_t* resfree = ha->bars + 2 * NQ + 2;
-  uint64_t* sqfull = ha->sqbars;           // [kSegQ] a segment descriptor is in the queue
-  uint64_t* sqfree = ha->sqbars + kSegQ;   // [kSegQ] the helper and every consumer warp have read it
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
-  const bool dyn = a.chunk_tiles > 0;
   // Programmatic dependent launch: behind the append (dep 2) the split plan
   // reads seq_lens, so nothing here may run before that grid has completed;
   // behind the q' projection alone (dep 1) only the helper waits, before it
   // reads q'.
   if (a.dep == 2) griddep_wait();
 
-  // Valid lengths, tiles per sequence (per head) and their exclusive prefix;
-  // for the dynamic plan also the prefix of chunks (H chunk rows per sequence).
+  // Valid lengths, tiles per sequence (per head) and their exclusive prefix.
   if (warp == 0) {
     const int per = (a.B + 31) / 32;
     const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
-    int sum = 0, csum = 0;
+    int sum = 0;
     for (int b = b0; b < b1; ++b) {
       const int raw = a.seq_lens[b];
       if ((raw < 0 || raw > a.L_cap) && c == 0) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
       const int n = clamp_len(raw, a.L_cap);
       lens[b] = n;
-      const int tb = (n + T - 1) / T;
-      sum += tb;
-      if (dyn) csum += a.H * ((tb + a.chunk_tiles - 1) / a.chunk_tiles);
+      sum += (n + T - 1) / T;
     }
-    int incl = sum, cincl = csum;
+    int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      const int cv = __shfl_up_sync(0xffffffffu, cincl, o);
-      if (lane >= o) {
-        incl += v;
-        cincl += cv;
-      }
+      if (lane >= o) incl += v;
     }
-    int run = incl - sum, crun = cincl - csum;
+    int run = incl - sum;
     for (int b = b0; b < b1; ++b) {
-      const int tb = (lens[b] + T - 1) / T;
       pre[b] = run;
-      run += tb;
-      if (dyn) {
-        cpre[b] = crun;
-        crun += a.H * ((tb + a.chunk_tiles - 1) / a.chunk_tiles);
-      }
+      run += (lens[b] + T - 1) / T;
     }
-    if (lane == 31) {
-      pre[a.B] = incl;
-      if (dyn) cpre[a.B] = cincl;
-    }
+    if (lane == 31) pre[a.B] = incl;
     if (lane == 0) {
       for (int s = 0; s < S; ++s) {
         mbar_init(&full[s], 1);
@@ -891,13 +866,10 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
         mbar_init(&resfull[s], 1);
         mbar_init(&resfree[s], 1);
       }
+      mbar_init(bvbar, 1);
       for (int s = 0; s < NQ; ++s) {
         mbar_init(&qready[s], 1);
         mbar_init(&qfree[s], kConsumerWarps);
-      }
-      for (int s = 0; s < kSegQ; ++s) {
-        mbar_init(&sqfull[s], 1);
-        mbar_init(&sqfree[s], 1 + kConsumerWarps);
       }
       fence_mbar_init();
     }
@@ -912,102 +884,62 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
 
   const TileWalk walk{pre, a.B, a.H};
   const long long G = (long long)a.H * pre[a.B];
-  // Static plan: the flattened tiles split evenly, at most one CTA per tile, so
-  // the CTAs that share a (b, h) are consecutive without gaps.  Dynamic plan:
-  // every CTA takes part (it may claim nothing).
-  const int CW = dyn ? a.ctas : (int)(G < a.ctas ? G : a.ctas);
-  if (!dyn && c >= CW) {  // uniform across the CTA; nothing was issued
+  // At most one CTA per tile, so every working CTA owns at least one tile and
+  // the CTAs that share a (b, h) are consecutive without gaps.
+  const int CW = (int)(G < a.ctas ? G : a.ctas);
+  if (c >= CW) {  // uniform across the CTA; nothing was issued
     if (a.dep == 1) griddep_wait();  // the grid never completes before the q' grid it was launched behind
     return;
   }
+  const long long g_begin = G * c / CW, g_end = G * (c + 1) / CW;
 
   // ---------------------------------------------------------------- producer warp
   if (warp == kProducerWarp) {
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy(), keep = l2_evict_last_policy();
+      int b, h, t;
+      walk.locate(g_begin, b, h, t);
       long long issued = 0;
-      int nseg = 0, nemit = 0;
+      int nseg = 0, pb = -1, ph = -1;
       bool ok = true;
-      auto emit = [&](const SegDesc& d) {  // hand a descriptor to the helper and the consumers
-        const int s = nemit % kSegQ;
-        if (nemit >= kSegQ && !mbar_wait_bounded(&sqfree[s], (uint32_t)(((nemit / kSegQ) - 1) & 1))) {
-          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-          ok = false;
-        }
-        ha->sq[s] = d;
-        mbar_arrive(&sqfull[s]);
-        ++nemit;
-      };
-      auto stream = [&](int b, int h, int t0, int nt) {  // operands (dense path) and tiles of a segment
-        if (QMODE != kQGlobal && ok) {
+      for (long long g = g_begin; g < g_end && ok; ++g, ++issued) {
+        if (QMODE != kQGlobal && (b != pb || h != ph)) {  // operands of the next (b, h)
           const int sb = nseg % NBUF;
           if (nseg >= NBUF && !mbar_wait_bounded(&segempty[sb], (uint32_t)(((nseg / NBUF) - 1) & 1))) {
             set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
             ok = false;
-          }
-          if (ok) issue_operands<W, QMODE>(segbuf + (size_t)sb * SEGB, &segfull[sb], a, b, h, keep);
-          ++nseg;
-        }
-        for (int tt = 0; tt < nt && ok; ++tt, ++issued) {
-          const int s = (int)(issued % S);
-          if (issued >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((issued / S) - 1) & 1))) {
-            set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-            ok = false;
             break;
           }
-          const int t = t0 + tt;
-          issue_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, &full[s], a, b, h, t,
-                                            min(T, lens[b] - t * T), pol);
+          issue_operands<W, QMODE>(segbuf + (size_t)sb * SEGB, &segfull[sb], a, b, h, keep);
+          ++nseg;
+          pb = b;
+          ph = h;
         }
-      };
-      if (dyn) {
-        // Chunks of chunk_tiles tiles of one (b, h), numbered sequence by
-        // sequence, head by head; claimed one ahead so that the claim's
-        // latency overlaps the previous chunk's copies.
-        const int NCH = cpre[a.B];
-        int cid = atomicAdd(a.work, 1);
-        while (ok && cid < NCH) {
-          const int next = atomicAdd(a.work, 1);
-          int lo = 0, hi = a.B - 1;  // the sequence: the largest b with cpre[b] <= cid
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (cpre[mid] <= cid) lo = mid;
-            else hi = mid - 1;
-          }
-          const int b = lo, tb = walk.tiles(b);
-          const int nch = (tb + a.chunk_tiles - 1) / a.chunk_tiles;
-          const int rem = cid - cpre[b], h = rem / nch, k = rem % nch;
-          const int t0 = k * a.chunk_tiles, nt = min(a.chunk_tiles, tb - t0);
-          emit(SegDesc{b, h, t0, nt, cid, cid - k, nch, 0});
-          stream(b, h, t0, nt);
-          cid = next;
+        const int s = (int)(issued % S);
+        if (issued >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((issued / S) - 1) & 1))) {
+          set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+          ok = false;
+          break;
         }
-        // This CTA has made its last claim; the last CTA to get here clears
-        // the claim counters for the next call (the fence orders this CTA's
-        // claims before its count).
-        __threadfence();
-        if (atomicAdd(a.work + 1, 1) == (int)gridDim.x - 1) {
-          atomicExch(a.work, 0);
-          atomicExch(a.work + 1, 0);
-        }
-      } else {
-        long long g = G * c / CW;
-        const long long g_end = G * (c + 1) / CW;
-        while (ok && g < g_end) {
-          int b, h, t;
-          walk.locate(g, b, h, t);
-          const int tb = walk.tiles(b);
-          const int nt = (int)(((long long)(tb - t) < g_end - g) ? (long long)(tb - t) : g_end - g);
-          const long long gf = (long long)a.H * pre[b] + (long long)h * tb;
-          const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
-          const int bh = b * a.H + h;
-          emit(SegDesc{b, h, t, nt, c + bh, cf + bh, cl - cf + 1, 0});
-          stream(b, h, t, nt);
-          g += nt;
-        }
+        issue_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, &full[s], a, b, h, t,
+                                          min(T, lens[b] - t * T), pol);
+        walk.advance(b, h, t);
       }
-      emit(SegDesc{0, 0, 0, 0, 0, 0, 0, 0});  // end of the queue (also after an error)
+      // B_Vh of the CTA's last segment, for the consumers' finish (issued after
+      // the tiles so that it does not compete with the first ones).
+      const bool stage_bv = C::bv_stage_bytes(a.Hd) > 0 && a.Bv != nullptr;
+      if (stage_bv) {
+        int lb, lh, lt;
+        walk.locate(g_end - 1, lb, lh, lt);
+        const uint32_t bytes = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2);
+        mbar_arrive_expect_tx(bvbar, bytes);
+        for (uint32_t off = 0; off < bytes; off += 32768)
+          bulk_g2s(reinterpret_cast<uint8_t*>(bv_last) + off,
+                   static_cast<const uint8_t*>(a.Bv) + (size_t)lh * bytes + off, min(32768u, bytes - off), bvbar,
+                   keep);
+      }
       // Leave no copy in flight behind: wait (bounded) for the last uses of each buffer.
+      if (stage_bv && !mbar_wait_bounded(bvbar, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       for (long long i = (issued > S ? issued - S : 0); i < issued && ok; ++i)
         if (!mbar_wait_bounded(&full[(int)(i % S)], (uint32_t)((i / S) & 1))) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
       for (int k = (nseg > NBUF ? nseg - NBUF : 0); k < nseg && ok; ++k)
@@ -1018,6 +950,20 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
 
   // ---------------------------------------------------------------- helper warp
   if (warp == kHelperWarp) {
+    int b = 0, h = 0, t = 0;
+    walk.locate(g_begin, b, h, t);
+    long long g = g_begin;
+    // next (b, h) segment of this CTA's tile range, or false at the end
+    auto next_segment = [&](int& sbk, int& shk) {
+      if (g >= g_end) return false;
+      sbk = b;
+      shk = h;
+      while (g < g_end && b == sbk && h == shk) {
+        walk.advance(b, h, t);
+        ++g;
+      }
+      return true;
+    };
     bool timed_out = false;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (!mbar_wait_bounded(bar, parity, timed_out ? 0ull : kWaitLimitNs)) {
@@ -1025,33 +971,36 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
         timed_out = true;
       }
     };
-    int built = 0, done = 0, nread = 0;
+    int built = 0, done = 0;
     bool more = true;
     if (QMODE == kQGlobal) griddep_wait();  // q' comes from the grid this one was launched behind
     while (true) {
       // Build ahead of the oldest unfinished segment (see kAhead).
       while (more && built < done + kAhead) {
-        const int qs = nread % kSegQ;
-        wait(&sqfull[qs], (uint32_t)((nread / kSegQ) & 1));
-        const SegDesc d = ha->sq[qs];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sqfree[qs]);
-        ++nread;
-        if (d.nt == 0) {
+        int sb_b, sb_h;
+        if (!next_segment(sb_b, sb_h)) {
           more = false;
           break;
         }
         const int k = built, sq = k % NQ;
-        if (lane == 0) ha->seg[sq] = d;
-        if (a.Bv != nullptr && d.np > 1) {  // a merge may fall to this CTA: warm B_Vh in L2
+        const int tb = walk.tiles(sb_b);
+        const long long gf = (long long)a.H * pre[sb_b] + (long long)sb_h * tb;
+        const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
+        if (lane == 0) {
+          ha->seginfo[sq][0] = sb_b;
+          ha->seginfo[sq][1] = sb_h;
+          ha->seginfo[sq][2] = cf;
+          ha->seginfo[sq][3] = cl;
+        }
+        if (a.Bv != nullptr && c == cl) {  // the likely finisher warms B_Vh in L2
           const int bytes = W * a.Hd * (a.w8 ? 1 : 2);
-          const char* bv = static_cast<const char*>(a.Bv) + (size_t)d.h * bytes;
+          const char* bv = static_cast<const char*>(a.Bv) + (size_t)sb_h * bytes;
           for (int o = lane * 128; o < bytes; o += 32 * 128) prefetch_l2(bv + o);
         }
         if (QMODE != kQGlobal) wait(&segfull[k % NBUF], (uint32_t)((k / NBUF) & 1));
         if (k >= NQ) wait(&qfree[sq], (uint32_t)(((k / NQ) - 1) & 1));
         const float amax = helper_qprime<W, QMODE>(segbuf + (size_t)(k % NBUF) * SEGB, ha->qsv[sq], a,
-                                                   (size_t)d.b * a.H + d.h, lane);
+                                                   (size_t)sb_b * a.H + sb_h, lane);
         __syncwarp();
         if (QMODE != kQGlobal && lane == 0) mbar_arrive(&segempty[k % NBUF]);  // staged operands consumed
         if constexpr (CT::kScaled) {
@@ -1066,30 +1015,32 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       // The consumers finish the CTA's last segment themselves.
       if (done == built || (!more && done == built - 1)) break;
       // Finish segment `done` once the consumers have reduced it.
-      const int k = done, sr = k & 1;
+      const int k = done, sr = k & 1, si = k % NQ;
       wait(&resfull[sr], (uint32_t)((k / 2) & 1));
       const float* res = ha->res[sr];
-      const SegDesc d = ha->seg[k % NQ];
-      float* outp = a.out + ((size_t)d.b * a.H + d.h) * a.Hd;
-      const BvRef Bvh{a.Bv ? static_cast<const uint8_t*>(a.Bv) + (size_t)d.h * W * a.Hd * (a.w8 ? 1 : 2) : nullptr,
-                      a.w8, a.w8 ? a.sBv + (size_t)d.h * a.Hd : nullptr};
-      if (d.np == 1) {
+      const int sb_b = ha->seginfo[si][0], sb_h = ha->seginfo[si][1];
+      const int cf = ha->seginfo[si][2], cl = ha->seginfo[si][3];
+      float* outp = a.out + ((size_t)sb_b * a.H + sb_h) * a.Hd;
+      const BvRef Bvh{a.Bv ? static_cast<const uint8_t*>(a.Bv) + (size_t)sb_h * W * a.Hd * (a.w8 ? 1 : 2) : nullptr,
+                      a.w8, a.w8 ? a.sBv + (size_t)sb_h * a.Hd : nullptr};
+      if (cf == cl) {
         helper_finalize<W>(res, Bvh, outp, a.Hd, lane);
       } else {
-        const int bh = d.b * a.H + d.h;
-        float* dst = a.partials + (size_t)d.ps * (W + 2);
+        const int bh = sb_b * a.H + sb_h;
+        float* dst = a.partials + ((size_t)c + bh) * (W + 2);
         for (int e = lane; e < W + 2; e += 32) dst[e] = res[e];
         __threadfence();  // publish before the counter bump
         __syncwarp();
         int prev = 0;
         if (lane == 0) prev = atomicAdd(&a.counters[bh], 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == d.np - 1) {  // last arriver: merge every partial of (b, h) in slot order
+        if (prev == cl - cf) {  // last arriver: merge every partial of (b, h) in CTA order
           __threadfence();
-          const float* part = a.partials + (size_t)d.p0 * (W + 2);
-          const float M = merge_max<W, true>(part, d.np);
+          const int np = cl - cf + 1;
+          const float* part = a.partials + ((size_t)cf + bh) * (W + 2);
+          const float M = merge_max<W, true>(part, np);
           float* mres = ha->res[sr];  // reuse the segment's slot for the merged result
-          for (int e = lane; e < W + 1; e += 32) mres[1 + e] = merge_elem<W, true>(part, d.np, M, e);
+          for (int e = lane; e < W + 1; e += 32) mres[1 + e] = merge_elem<W, true>(part, np, M, e);
           __syncwarp();
           helper_finalize<W>(mres, Bvh, outp, a.Hd, lane);
           if (lane == 0) atomicExch(&a.counters[bh], 0);
@@ -1114,16 +1065,7 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       timed_out = true;
     }
   };
-  int nread = 0;
-  auto read_desc = [&]() {
-    const int qs = nread % kSegQ;
-    wait(&sqfull[qs], (uint32_t)((nread / kSegQ) & 1));
-    const SegDesc d = ha->sq[qs];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sqfree[qs]);
-    ++nread;
-    return d;
-  };
+  int k = 0;  // segments started
   auto end_segment = [&](int j) {  // hand segment j to the helper
     const int sr = j & 1;
     if (j >= 2) wait(&resfree[sr], (uint32_t)(((j / 2) - 1) & 1));
@@ -1134,26 +1076,36 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
   // last-arriver merge, up-projection); nothing runs after it.
   float* res = reinterpret_cast<float*>(smem + C::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
-  auto finish_last = [&](const SegDesc& d) {
-    const int bh = d.b * a.H + d.h;
-    // The CTA that ends a head usually reaches it after the other segments of
-    // the head: if every other contributor has already published (the counter,
+  auto finish_last = [&](int b_, int h_) {
+    const int tb = walk.tiles(b_);
+    const long long gf = (long long)a.H * pre[b_] + (long long)h_ * tb;
+    const int cf = cta_of(gf, G, CW), cl = cta_of(gf + tb - 1, G, CW);
+    const int bh = b_ * a.H + h_;
+    // The CTA that ends a head usually reaches it after the CTAs that start
+    // it: if every other contributor has already published (the counter,
     // read with acquire, says so), this CTA is the last arriver without
     // publishing or bumping anything itself.  The read is issued before the
     // reduction so that its latency overlaps it (an early, lower count only
     // sends this CTA down the publishing path).
-    const int seen = (d.np > 1 && tid == 0) ? ld_acquire_gpu(&a.counters[bh]) : 0;
+    const int seen = (cf != cl && tid == 0) ? ld_acquire_gpu(&a.counters[bh]) : 0;
     reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
-    float* outp = a.out + ((size_t)d.b * a.H + d.h) * a.Hd;
-    const BvRef Bvh{a.Bv ? static_cast<const uint8_t*>(a.Bv) + (size_t)d.h * W * a.Hd * (a.w8 ? 1 : 2) : nullptr,
-                    a.w8, a.w8 ? a.sBv + (size_t)d.h * a.Hd : nullptr};
-    if (d.np == 1) {
+    float* outp = a.out + ((size_t)b_ * a.H + h_) * a.Hd;
+    BvRef Bvh{nullptr, a.w8, a.w8 ? a.sBv + (size_t)h_ * a.Hd : nullptr};
+    if (a.Bv != nullptr) {
+      if (C::bv_stage_bytes(a.Hd) > 0) {  // staged by the producer
+        wait(bvbar, 0);
+        Bvh.p = bv_last;
+      } else {
+        Bvh.p = static_cast<const uint8_t*>(a.Bv) + (size_t)h_ * W * a.Hd * (a.w8 ? 1 : 2);
+      }
+    }
+    if (cf == cl) {
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
       return;
     }
-    float* dst = a.partials + (size_t)d.ps * (W + 2);
+    float* dst = a.partials + ((size_t)c + bh) * (W + 2);
     int* flag = reinterpret_cast<int*>(misc) + 8;
-    if (tid == 0) *flag = (seen == d.np - 1) ? 2 : 0;
+    if (tid == 0) *flag = (seen == cl - cf) ? 2 : 0;
     csync();
     const int early = *flag;
     if (tid < W + 2) {
@@ -1164,69 +1116,68 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
     if (!early) {
       if (tid == 0) {
         const int prev = atomicAdd(&a.counters[bh], 1);
-        *flag = (prev == d.np - 1) ? 1 : 0;
+        *flag = (prev == cl - cf) ? 1 : 0;
       }
       csync();
     }
     if (*flag) {
       if (!early) __threadfence();
-      merge_rows<W, true>(a.partials + (size_t)d.p0 * (W + 2), d.np, res, tid);
+      merge_rows<W, true>(a.partials + ((size_t)cf + bh) * (W + 2), cl - cf + 1, res, tid);
       if (tid == 0) atomicExch(&a.counters[bh], 0);
       finalize_out<W>(res, Bvh, outp, a.Hd, red, tid);
     }
   };
 
-  int k = 0;  // segments started
+  int b, h, t;
+  walk.locate(g_begin, b, h, t);
+  int cb = -1, ch = -1;
   long long i = 0;
-  SegDesc d = read_desc();
-  while (d.nt > 0) {
-    const int sq = k % NQ;
-    wait(&qready[sq], (uint32_t)((k / NQ) & 1));
-    qst.step = ha->qstep[sq];
-    if constexpr (CT::kScaled) {
-      const uint32_t* pl = ha->planes[sq];
+  for (long long g = g_begin; g < g_end; ++g, ++i) {
+    if (b != cb || h != ch) {
+      if (cb >= 0) end_segment(k - 1);
+      const int sq = k % NQ;
+      wait(&qready[sq], (uint32_t)((k / NQ) & 1));
+      qst.step = ha->qstep[sq];
+      if constexpr (CT::kScaled) {
+        const uint32_t* pl = ha->planes[sq];
 #pragma unroll
-      for (int q = 0; q < QW; ++q) {
-        qst.qh[q] = pl[(sub * 3 + 0) * QW + q];
-        qst.qm[q] = pl[(sub * 3 + 1) * QW + q];
-        qst.ql[q] = pl[(sub * 3 + 2) * QW + q];
+        for (int q = 0; q < QW; ++q) {
+          qst.qh[q] = pl[(sub * 3 + 0) * QW + q];
+          qst.qm[q] = pl[(sub * 3 + 1) * QW + q];
+          qst.ql[q] = pl[(sub * 3 + 2) * QW + q];
+        }
+        if constexpr (CODEC == kCodecI4) {
+          qst.ch = (int)pl[TPT * 3 * QW + sub * 3 + 0];
+          qst.cm = (int)pl[TPT * 3 * QW + sub * 3 + 1];
+          qst.cl = (int)pl[TPT * 3 * QW + sub * 3 + 2];
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+          qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
       }
-      if constexpr (CODEC == kCodecI4) {
-        qst.ch = (int)pl[TPT * 3 * QW + sub * 3 + 0];
-        qst.cm = (int)pl[TPT * 3 * QW + sub * 3 + 1];
-        qst.cl = (int)pl[TPT * 3 * QW + sub * 3 + 2];
-      }
-    } else {
-#pragma unroll
-      for (int p = 0; p < NP; ++p)
-        qst.qv[p] = make_float2(ha->qsv[sq][sub * VPT + 2 * p], ha->qsv[sq][sub * VPT + 2 * p + 1]);
-    }
-    if constexpr (C::kNSeg == 2) qst.swap_halves(swapped_lane(lane));
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&qfree[sq]);
-#pragma unroll
-    for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
-    m = kNegInf;
-    l = 0.f;
-    ++k;
-    for (int tt = 0; tt < d.nt; ++tt, ++i) {
-      const int s = (int)(i % S);
-      // A timed-out wait only poisons the result (err is set); control flow stays
-      // uniform so every consumer warp reaches every named barrier.
-      wait(&full[s], (uint32_t)((i / S) & 1));
-      process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, lens[d.b] - (d.t0 + tt) * T),
-                                          qst, m, l, acc, tid);
+      if constexpr (C::kNSeg == 2) qst.swap_halves(swapped_lane(lane));
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) mbar_arrive(&qfree[sq]);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
+      m = kNegInf;
+      l = 0.f;
+      ++k;
+      cb = b;
+      ch = h;
     }
-    const SegDesc nd = read_desc();
-    if (nd.nt == 0) {
-      finish_last(d);
-      break;
-    }
-    end_segment(k - 1);
-    d = nd;
+    const int s = (int)(i % S);
+    // A timed-out wait only poisons the result (err is set); control flow stays
+    // uniform so every consumer warp reaches every named barrier.
+    wait(&full[s], (uint32_t)((i / S) & 1));
+    process_tile<CODEC, VPT, TPT, NTOK>(stages + (size_t)s * C::kStageBytes, min(T, lens[b] - t * T), qst, m, l,
+                                        acc, tid);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    walk.advance(b, h, t);
   }
+  if (cb >= 0) finish_last(cb, ch);
 }
 
 // ------------------------------------------------------------------ cluster kernel (small problems)
@@ -1609,7 +1560,6 @@ struct Plan {
   KernelInfo ki;    // the kernel to launch
   size_t smem;
   int ctas;         // persistent path: grid size
-  int chunk_tiles;  // persistent path: > 0 selects the dynamic plan with chunks of this many tiles
 };
 
 bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* pl) {
@@ -1627,7 +1577,6 @@ bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* 
     pl->ki = small;
     pl->smem = csmem;
     pl->ctas = 0;
-    pl->chunk_tiles = 0;
     return true;
   }
   const size_t smem_big = big.smem(a.B, big.pqmode, a.Hd);
@@ -1641,25 +1590,11 @@ bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* 
   if (ctas > tiles_max) ctas = tiles_max;
   if (ctas > kMaxDecodeCtas) ctas = kMaxDecodeCtas;
   if (ctas < 1) ctas = 1;
-  // With several tiles per CTA the work is claimed dynamically, in chunks of
-  // whole tiles of one (b, h): about 16 chunks per CTA, at most 32 per (b, h)
-  // (the workspace's partial slots), so that CTAs that stream faster take more.
-  // A chunk also carries at least ~64 KB, so that the hand-off at its end (a
-  // reduction across the consumer warps) stays small next to its streaming.
-  int chunk = 0;
-  if (tiles_max > ctas) {
-    const long long tph = (a.L_cap + ki.tile - 1) / ki.tile;
-    const long long want = (tiles_max + 16 * ctas - 1) / (16 * ctas);
-    const long long tile_bytes = (long long)ki.tile * (2 * rowbytes + (codec == kCodecF16 ? 0 : 4));
-    const long long min_tiles = (65536 + tile_bytes - 1) / tile_bytes;
-    chunk = (int)std::max<long long>(std::max<long long>(1, min_tiles), std::max<long long>(want, (tph + 31) / 32));
-  }
   pl->cluster = false;
   pl->csize = 0;
   pl->ki = ki;
   pl->smem = smem;
   pl->ctas = (int)ctas;
-  pl->chunk_tiles = chunk;
   return true;
 }
 
@@ -1704,7 +1639,6 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
   cudaError_t e = ensure_smem(pl.ki.fn, pl.smem);
   if (e != cudaSuccess) return e;
   a.ctas = pl.ctas;
-  a.chunk_tiles = pl.chunk_tiles;
   bool pdl = after_append;
   if (pl.ki.pqmode == kQGlobal) {
     // q' for every (b, h) first; the decode is launched behind it so that its

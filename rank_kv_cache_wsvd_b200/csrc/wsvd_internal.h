@@ -18,14 +18,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumerThreads + 32;   // cluster kernel: + producer warp
 constexpr int kPersistThreads = kConsumerThreads + 64;  // persistent kernel: + producer and helper warps
-// Upper bound on the persistent grid.
+// Upper bound on the persistent grid; sizes the partial-result workspace.
 constexpr int kMaxDecodeCtas = 2048;
-// Partial-result slots of the decode workspace: enough for every CTA of the
-// static plan, and for the dynamic plan's chunks (at most 32 per (b, h)).
-__host__ __device__ inline long long decode_partial_slots(int B, int H) {
-  const long long bh = (long long)B * H;
-  return (bh * 32 > kMaxDecodeCtas ? bh * 32 : kMaxDecodeCtas) + bh;
-}
 
 enum Codec { kCodecI8 = 0, kCodecI4 = 1, kCodecF16 = 2 };
 enum QMode { kQProj = 0, kQDirect = 1, kQGlobal = 2 };
@@ -35,7 +29,6 @@ struct DecodeArgs {
   int B, H, Hd, W;       // W: latent width per token (r, Hd or R)
   int L_cap;
   int ctas;              // persistent grid size C (set by launch_decode)
-  int chunk_tiles;       // > 0: tiles are claimed dynamically in chunks of this many tiles of one (b, h)
   int dep;               // programmatic dependency: 0 none, 1 only q' (qglobal), 2 everything (set by launch_decode)
   int heads_share;       // 1: the latent rows of (b, h) are the rows of b (shared-latent path)
   const int32_t* seq_lens;
@@ -53,9 +46,8 @@ struct DecodeArgs {
   float* qglobal;        // [B][H][W] projected q' (kQGlobal; workspace)
   float qscale;          // softmax_scale * log2(e)
   float* out;            // [B][H][Hd]
-  float* partials;       // [decode_partial_slots(B, H)][W + 2]
+  float* partials;       // [(kMaxDecodeCtas + B*H)][W + 2]
   int32_t* counters;     // [B*H], zero between calls
-  int32_t* work;         // [2]: dynamic plan's claim counter and finished-CTA count, zero between calls
   int32_t* err;
 };
 

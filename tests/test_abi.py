@@ -54,14 +54,12 @@ def test_cache_byte_counts_match_oracle(lib, B, H, L, r, bits):
 
 
 def test_workspace_sizes_hold_only_partials(lib):
-    """The decode workspace holds split partials (W + 2 floats per slot; slots
-    for a 2048-CTA grid or 32 chunks per head, plus one per head), one counter
-    per head and two claim counters, and the projected queries q' (W floats
-    per head), never an L x Hd buffer: reconstructed K/V are not materialised."""
+    """The decode workspace holds split partials (W + 2 floats per slot), one
+    counter per head and the projected queries q' (W floats per head), never
+    an L x Hd buffer: reconstructed K/V are not materialised."""
     B, H, r, L = 4, 32, 32, 32768
     a16 = lambda v: (v + 15) // 16 * 16
-    slots = max(2048, 32 * B * H) + B * H
-    size = lambda W_: a16(slots * (W_ + 2) * 4) + a16((B * H + 2) * 4) + a16(B * H * W_ * 4)
+    size = lambda W_: a16((2048 + B * H) * (W_ + 2) * 4) + a16(B * H * 4) + a16(B * H * W_ * 4)
     ws = W.wsvd_decode_workspace_size(B, H, r)
     assert ws == size(r)
     assert ws < B * H * L * 128 * 2 / 100  # far below one reconstructed K

@@ -10,16 +10,11 @@ counts: no interleaving deadlocks, and no waiter ever falls two phases behind
 a barrier (which a parity wait cannot tell from the phase it wants).
 
 The ring sizes, slot counts and hand-off rules mirror decode.cu: S tile
-stages, NBUF operand buffers, NQ query-state slots, two result slots, and a
-queue of kSegQ segment descriptors through which the producer hands each
-segment (a run of tiles of one (b, h): a piece of the CTA's static range, or a
-chunk it claimed) to the helper and the consumers, followed by an end marker;
-a queue slot is reused once the helper and all eight consumer warps have read
-it.  The consumers read the next descriptor before handing a segment over, and
-finish the CTA's last segment themselves.  The helper builds segment k only
-while k < done + kAhead (kAhead = NQ when q' comes precomputed, 2 when the
-producer stages operands).  A model of the protocol, not of the arithmetic: a
-change to the kernel's hand-off rules must be mirrored here.
+stages, NBUF operand buffers, NQ query-state slots, two result slots; the
+helper builds segment k only while k < done + kAhead (kAhead = NQ when q'
+comes precomputed, 2 when the producer stages operands).  A model of the
+protocol, not of the arithmetic: a change to the kernel's hand-off rules
+must be mirrored here.
 """
 import random
 
@@ -39,59 +34,45 @@ class Bar:
 
 
 def segments_of(tiles):
-    """Tile counts of the runs of equal (b, h) in a CTA's tile list."""
     segs = []
-    prev = None
     for bh in tiles:
-        if bh != prev:
-            segs.append(0)
-            prev = bh
-        segs[-1] += 1
+        if not segs or segs[-1] != bh:
+            segs.append(bh)
     return segs
 
 
-def run(segs, S, NBUF, NQ, qglobal, rng, kAhead=None, Q=4, helper_frees=True):
+def run(tiles, S, NBUF, NQ, qglobal, rng, kAhead=None):
     kAhead = kAhead or (NQ if qglobal else 2)
     full = [Bar(1) for _ in range(S)]
     empty = [Bar(8) for _ in range(S)]
     segfull, segempty = [Bar(1) for _ in range(2)], [Bar(1) for _ in range(2)]
     qready, qfree = [Bar(1) for _ in range(NQ)], [Bar(8) for _ in range(NQ)]
     resfull, resfree = [Bar(1) for _ in range(2)], [Bar(1) for _ in range(2)]
-    sqfull, sqfree = [Bar(1) for _ in range(Q)], [Bar(9 if helper_frees else 8) for _ in range(Q)]
-    queue = list(segs) + [0]  # descriptors in emission order; 0 tiles ends the queue
+    nseg = len(segments_of(tiles))
     hazards = []
 
     def producer():
         issued = k = 0
-        for n, nt in enumerate(queue):
-            if n >= Q:  # queue slot free: read by the helper and the eight consumer warps
-                yield sqfree[n % Q], n // Q - 1
-            sqfull[n % Q].arrive()
-            if nt == 0:
-                return
-            if not qglobal:
+        prev = None
+        for bh in tiles:
+            if not qglobal and bh != prev:
                 if k >= NBUF:
                     yield segempty[k % NBUF], k // NBUF - 1
                 segfull[k % NBUF].arrive()
                 k += 1
-            for _ in range(nt):
-                s = issued % S
-                if issued >= S:
-                    yield empty[s], issued // S - 1
-                full[s].arrive()
-                issued += 1
+                prev = bh
+            s = issued % S
+            if issued >= S:
+                yield empty[s], issued // S - 1
+            full[s].arrive()
+            issued += 1
 
     def helper():
-        built = done = nread = 0
+        built = done = 0
         more = True
         while True:
             while more and built < done + kAhead:
-                yield sqfull[nread % Q], nread // Q
-                if helper_frees:
-                    sqfree[nread % Q].arrive()
-                nt = queue[nread]
-                nread += 1
-                if nt == 0:
+                if built >= nseg:
                     more = False
                     break
                 k = built
@@ -110,37 +91,25 @@ def run(segs, S, NBUF, NQ, qglobal, rng, kAhead=None, Q=4, helper_frees=True):
             done += 1
 
     def consumers():
-        k = i = nread = 0
-
-        def read():
-            nonlocal nread
-            yield sqfull[nread % Q], nread // Q
-            for _ in range(8):
-                sqfree[nread % Q].arrive()
-            nread += 1
-
-        yield from read()
-        nt = queue[0]
-        while nt > 0:
-            yield qready[k % NQ], k // NQ
-            for _ in range(8):
-                qfree[k % NQ].arrive()
-            k += 1
-            for _ in range(nt):
-                s = i % S
-                yield full[s], i // S
+        k = i = 0
+        prev = None
+        for bh in tiles:
+            if bh != prev:
+                if prev is not None:  # hand segment k - 1 to the helper
+                    j = k - 1
+                    if j >= 2:
+                        yield resfree[j & 1], j // 2 - 1
+                    resfull[j & 1].arrive()
+                yield qready[k % NQ], k // NQ
                 for _ in range(8):
-                    empty[s].arrive()
-                i += 1
-            yield from read()
-            nxt = queue[nread - 1]
-            if nxt == 0:
-                return  # finish the last segment here
-            j = k - 1  # hand segment k - 1 to the helper
-            if j >= 2:
-                yield resfree[j & 1], j // 2 - 1
-            resfull[j & 1].arrive()
-            nt = nxt
+                    qfree[k % NQ].arrive()
+                k += 1
+                prev = bh
+            s = i % S
+            yield full[s], i // S
+            for _ in range(8):
+                empty[s].arrive()
+            i += 1
 
     roles = [producer(), helper(), consumers()]
     waiting = [next(g, None) for g in roles]
@@ -176,7 +145,6 @@ def cta_tiles(lens, H, T, C, c):
 
 @pytest.mark.parametrize("qglobal", [True, False])
 def test_no_deadlock_or_phase_aliasing(qglobal):
-    """Static plan: every CTA's range of the flattened (b, h, tile) space."""
     rng = random.Random(11 if qglobal else 12)
     runs = 0
     for _ in range(60):
@@ -190,23 +158,11 @@ def test_no_deadlock_or_phase_aliasing(qglobal):
             if not tiles:
                 continue
             for S, NBUF, NQ in ((4, 2, 4), (2, 1, 4), (3, 2, 2), (8, 2, 4), (2, 2, 2)):
-                ok, hazards = run(segments_of(tiles), S, NBUF, NQ, qglobal, rng)
+                ok, hazards = run(tiles, S, NBUF, NQ, qglobal, rng)
                 runs += 1
                 assert ok, (segments_of(tiles), S, NBUF, NQ)
                 assert not hazards, (segments_of(tiles), S, NBUF, NQ)
     assert runs > 200
-
-
-@pytest.mark.parametrize("qglobal", [True, False])
-def test_dynamic_chunks_no_deadlock_or_phase_aliasing(qglobal):
-    """Dynamic plan: a CTA claims any number of chunks (none included) of one
-    to a few tiles each, in any order of heads."""
-    rng = random.Random(21 if qglobal else 22)
-    for _ in range(400):
-        segs = [rng.randint(1, 4) for _ in range(rng.choice([0, 1, 2, 3, 5, 9, 17]))]
-        S, NBUF, NQ = rng.choice(((4, 2, 4), (2, 1, 4), (3, 2, 2), (8, 2, 4), (2, 2, 2)))
-        ok, hazards = run(segs, S, NBUF, NQ, qglobal, rng)
-        assert ok and not hazards, (segs, S, NBUF, NQ)
 
 
 def test_model_catches_a_helper_that_runs_too_far_ahead():
@@ -221,20 +177,6 @@ def test_model_catches_a_helper_that_runs_too_far_ahead():
         for c in range(3):
             tiles = cta_tiles(lens, 32, 64, 37, c)
             if tiles:
-                ok, hazards = run(segments_of(tiles), 2, 1, 4, True, rng, kAhead=8, Q=16)
+                ok, hazards = run(tiles, 2, 1, 4, True, rng, kAhead=8)
                 bad += (not ok) or bool(hazards)
-    assert bad > 0
-
-
-def test_model_catches_a_queue_slot_freed_without_the_helper():
-    """The check is not vacuous for the descriptor queue either: if a slot were
-    reused once the consumers alone had read it, the helper (which reads
-    descriptors only as far as kAhead allows) falls a full queue cycle behind
-    on some schedules."""
-    rng = random.Random(9)
-    bad = 0
-    for _ in range(300):
-        segs = [rng.randint(1, 3) for _ in range(rng.randint(6, 17))]
-        ok, hazards = run(segs, 4, 2, 2, True, rng, helper_frees=False)
-        bad += (not ok) or bool(hazards)
     assert bad > 0
