@@ -189,8 +189,15 @@ class WsvdStep:
                 avq, sav = WL.quantize_weights_w8(ai.A_v)
                 self.A_k, self.A_v, self.sA_k, self.sA_v = cu(akq), cu(avq), cu(sak), cu(sav)
             self.ws_app = W.workspace(W.wsvd_append_workspace_size())
-            self.x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-        self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
+            # the step's host inputs in one pinned buffer, q right after x (one copy per step)
+            nx, nq = w.B * w.E, w.B * w.H * w.Hd
+            io = torch.empty(nx + nq, dtype=torch.int16).pin_memory()
+            io[:nx] = torch.from_numpy(ai.x_bits[0].view(np.int16).reshape(-1).copy())
+            io[nx:] = torch.from_numpy(d.q_bits.view(np.int16).reshape(-1).copy())
+            self.x_host = io[:nx].view(torch.bfloat16).view(w.B, w.E)
+            self.q_host = io[nx:].view(qdt).view(w.B, w.H, w.Hd)
+        else:
+            self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
         self.out_host = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32).pin_memory()
         # kernels per step: the append, and the decode's one or two (cluster kernel, or q' + split-L grid)
         self.launches_per_step = (1 if self.has_append else 0) + W.wsvd_decode_launch_count(

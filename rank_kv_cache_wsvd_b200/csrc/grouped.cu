@@ -183,35 +183,51 @@ __device__ __forceinline__ uint4 i4x8_to_h(uint32_t w) {
 }
 
 // q' of every query of one (b, latent head, query chunk) group, as the score
-// operand the decode kernel stages: q'_q = (B_Kh . q_q) * softmax_scale * log2 e
-// (8 lanes per row, a fixed shuffle tree), quantised with step max|q'_q| / 8355711
-// and written as three signed byte planes in the K-major no-swizzle layout,
-// followed by the NQ steps.  One CTA per group; the decode grid is launched
-// behind it as a programmatic dependent.
+// operand the decode kernel stages: q'_q = (B_Kh . q_q) * softmax_scale * log2 e,
+// quantised with step max|q'_q| / 8355711 and written as three signed byte
+// planes in the K-major no-swizzle layout, followed by the NQ steps.  One CTA
+// per group: B_Kh and the group's query rows are first staged in shared memory
+// with coalesced 16-byte loads; each output is then a dot product over the
+// head dimension in a fixed (row-rotated) order.  The decode grid is launched
+// behind this one as a programmatic dependent.
 template <int CODEC, int RB, int NQ>
 __global__ void __launch_bounds__(128) grouped_qproj_kernel(const GroupedArgs a, uint8_t* qplanes) {
   using C = GCfg<CODEC, RB, NQ>;
   constexpr int R = C::R, NS = C::NS;
-  __shared__ float qp[NQ * R];
-  __shared__ float inv[NQ];
+  extern __shared__ __align__(16) uint8_t psm[];
+  __half* bks = reinterpret_cast<__half*>(psm);                         // [R][Hd]
+  float* qs = reinterpret_cast<float*>(psm + (size_t)R * a.Hd * 2);     // [NQ][Hd]
+  float* qp = qs + (size_t)NQ * a.Hd;                                   // [NQ][R]
+  float* inv = qp + NQ * R;                                             // [NQ]
   griddep_launch_dependents();
-  const int grp = blockIdx.x, t = threadIdx.x, lane = t & 31;
+  const int grp = blockIdx.x, t = threadIdx.x;
   const int qc = grp % a.nqc, hkv = (grp / a.nqc) % a.Hkv, b = grp / (a.nqc * a.Hkv);
   const int nq = min(NQ, a.G * a.Tq - qc * NQ);
-  const int part = lane & 7;
-  for (int row = t >> 3; row < NQ * R; row += 128 / 8) {
-    const int ql = row / R, j = row % R;
-    float d = 0.f;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.Bk + (size_t)hkv * R * a.Hd);
+    uint4* dst = reinterpret_cast<uint4*>(bks);
+    for (int i = t; i < R * a.Hd / 8; i += 128) dst[i] = src[i];
+  }
+  for (int i = t; i < NQ * a.Hd; i += 128) {
+    const int ql = i / a.Hd, k = i % a.Hd;
+    float v = 0.f;
     if (ql < nq) {
       const int qg = qc * NQ + ql, tq = qg / a.G, g = qg % a.G;
-      const size_t qrow = (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd;
-      const __half* brow = a.Bk + ((size_t)hkv * R + j) * a.Hd;
-      for (int k = part; k < a.Hd; k += 8) d = fmaf(__half2float(brow[k]), load_q_elem(a.q, a.q_dtype, qrow + k), d);
+      v = load_q_elem(a.q, a.q_dtype, (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd + k);
     }
-    d += __shfl_xor_sync(0xffffffffu, d, 1);
-    d += __shfl_xor_sync(0xffffffffu, d, 2);
-    d += __shfl_xor_sync(0xffffffffu, d, 4);
-    if (part == 0) qp[row] = d * a.qscale;
+    qs[i] = v;
+  }
+  __syncthreads();
+  for (int o = t; o < NQ * R; o += 128) {
+    const int ql = o / R, j = o % R;
+    const __half* brow = bks + (size_t)j * a.Hd;
+    const float* qrow = qs + (size_t)ql * a.Hd;
+    float d = 0.f;
+    for (int kk = 0; kk < a.Hd; ++kk) {
+      const int k = (kk + j) & (a.Hd - 1);  // rows start at different columns: distinct banks
+      d = fmaf(__half2float(brow[k]), qrow[k], d);
+    }
+    qp[o] = d * a.qscale;
   }
   __syncthreads();
   uint8_t* blk = qplanes + (size_t)grp * C::QBLOCK;
@@ -235,6 +251,10 @@ __global__ void __launch_bounds__(128) grouped_qproj_kernel(const GroupedArgs a,
     }
     blk[(k >> 4) * C::LBO_PL + (n >> 3) * 128 + (n & 7) * 16 + (k & 15)] = (uint8_t)(int8_t)dig;
   }
+}
+
+__host__ inline size_t qproj_smem_bytes(int R, int NQ, int Hd) {
+  return (size_t)R * Hd * 2 + (size_t)NQ * Hd * 4 + (size_t)NQ * R * 4 + (size_t)NQ * 4;
 }
 
 template <int CODEC, int RB, int NQ>
@@ -779,9 +799,13 @@ extern "C" int wsvd_decode_multi(int B, int Tq, int Hq, int Hkv, int Hd, int r, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   {  // q' planes of every query group
     void* pargs[] = {&ga, &planes};
+    const size_t psmem = qproj_smem_bytes(r, sh.nq, Hd);
+    if (cudaFuncSetAttribute(gk.qproj, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem) != cudaSuccess)
+      return WSVD_ERR_CUDA;
     cudaLaunchConfig_t pcfg = {};
     pcfg.gridDim = dim3((unsigned)groups);
     pcfg.blockDim = dim3(128);
+    pcfg.dynamicSmemBytes = psmem;
     pcfg.stream = st;
     if (cudaLaunchKernelExC(&pcfg, gk.qproj, pargs) != cudaSuccess) return WSVD_ERR_CUDA;
   }
