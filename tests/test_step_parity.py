@@ -103,17 +103,25 @@ def test_decode_launch_count_matches_the_path():
         assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 2, w.name
 
 
-@pytest.mark.parametrize("name", ["llava7b", "long-r32"])
-def test_step_from_host_buffers_equals_device_step(name):
+@pytest.mark.parametrize("name,adjacent", [("llava7b", False), ("llava7b", True), ("long-r32", True)])
+def test_step_from_host_buffers_equals_device_step(name, adjacent):
     """wsvd_append_and_decode_host (x and q copied in from host memory, out
     copied back) gives bit for bit what wsvd_append_and_decode gives on the
-    same values already on the device, on two steps in a row."""
+    same values already on the device, on two steps in a row; with q right
+    after x in one pinned buffer (one copy) and in separate buffers."""
     w, lens0 = CASES[name]
     lens0 = [min(n, w.L_cap - 2) for n in lens0]  # two steps in a row: room for two appended rows
     d, ai = _inputs(w, lens0, seed=33)
     qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
-    x_host = torch.from_numpy(ai.x_bits[0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-    q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
+    xb = torch.from_numpy(ai.x_bits[0].view(np.int16).copy())
+    qb = torch.from_numpy(d.q_bits.view(np.int16).copy())
+    if adjacent:
+        io = torch.cat([xb.reshape(-1), qb.reshape(-1)]).pin_memory()
+        x_host = io[:xb.numel()].view(torch.bfloat16).view(xb.shape)
+        q_host = io[xb.numel():].view(qdt).view(qb.shape)
+    else:
+        x_host = xb.view(torch.bfloat16).pin_memory()
+        q_host = qb.view(qdt).pin_memory()
     out_host = torch.full((w.B, w.H, w.Hd), float("nan"), dtype=torch.float32).pin_memory()
     A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
     dv, hs = _device_state(d), _device_state(d)
