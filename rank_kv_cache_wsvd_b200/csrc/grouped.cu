@@ -103,7 +103,9 @@ struct GCfg {
   static constexpr int OFF_WMAX = OFF_STEP + 2 * NQ * 4;         // float wmax[2][4][NQ]
   static constexpr int OFF_WSV = OFF_WMAX + 2 * 4 * NQ * 4;      // uint32 wsv[2][4]
   static constexpr int OFF_LSUM = OFF_WSV + 8 * 4;               // float lsum[4][NQ]
-  static constexpr int OFF_RES = OFF_LSUM + 4 * NQ * 4;          // float res[NQ][R + 2]
+  static constexpr int OFF_BC = OFF_LSUM + 4 * NQ * 4;           // float2 bc[2][NQ] (new maximum, rescale)
+  static constexpr int OFF_MRUN = OFF_BC + 2 * NQ * 8;            // float mrun[NQ], int be[2]
+  static constexpr int OFF_RES = OFF_MRUN + NQ * 4 + 16;          // float res[NQ][R + 2]
   static constexpr int OFF_MISC = OFF_RES + NQ * (R + 2) * 4;    // int flag, uint32 tmem base
   static constexpr int OFF_BAR = (OFF_MISC + 16 + 7) / 8 * 8;
   static constexpr int NBAR = 2 * S + 9;
@@ -296,6 +298,9 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   uint32_t* wsv = reinterpret_cast<uint32_t*>(smem + C::OFF_WSV);
   float* lsum = reinterpret_cast<float*>(smem + C::OFF_LSUM);
   float* res = reinterpret_cast<float*>(smem + C::OFF_RES);
+  float2* bc = reinterpret_cast<float2*>(smem + C::OFF_BC);  // per tile parity: each query's new maximum, rescale
+  float* mrun = reinterpret_cast<float*>(smem + C::OFF_MRUN); // running maximum per query
+  int* be = reinterpret_cast<int*>(smem + C::OFF_MRUN + NQ * 4); // per tile parity: the P~ exponent
   int* flag = reinterpret_cast<int*>(smem + C::OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -459,14 +464,14 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     const int orow = MO == 64 ? (lane < 16 ? warp * 16 + lane : -1) : t;
     const bool holder = orow >= 0 && orow < R;
     const bool warp_holds = MO == 64 ? warp * 16 < R : warp * 32 < R;
-    float m[NQ], l[NQ], macc[NQ], acc[NQ];
+    float l[NQ], macc[NQ], acc[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-      m[q] = kNegInf;
       l[q] = 0.f;
       macc[q] = kNegInf;
       acc[q] = 0.f;
     }
+    if (t < NQ) mrun[t] = kNegInf;  // ordered before its first use by the tile barriers
     // Fold tile j's value accumulator (scaled by 2^-e) into acc, relative to m.
     auto accumulate = [&](int j, int e) {
       wait(&oready[j & 1], (uint32_t)((j >> 1) & 1));
@@ -483,13 +488,15 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         }
         tc05::wait_ld();
         const float unscale = __int_as_float((127 - e) << 23);
+        const float2* bj = bc + (j & 1) * NQ;  // maxima after tile j
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          if (m[q] != kNegInf) {
+          const float mq = bj[q].x;
+          if (mq != kNegInf) {
             const float d = (__uint_as_float(v[q]) + __uint_as_float(v[NQ + q])) * unscale;
-            const float f = macc[q] == kNegInf ? 0.f : ex2(macc[q] - m[q]);
+            const float f = macc[q] == kNegInf ? 0.f : ex2(macc[q] - mq);
             acc[q] = fmaf(acc[q], f, d);
-            macc[q] = m[q];
+            macc[q] = mq;
           }
         }
       }
@@ -534,26 +541,35 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       if (lane == 0) wsv[(i & 1) * 4 + warp] = svm;
       tc05::fence_before_sync();
       named_barrier_sync(1, kGConsumers);
-      // per-tile P~ scale 2^e: puts the largest s_V of the tile in [2^14, 2^15)
-      uint32_t svmax = 0;
+      // One thread per query: the tile maximum over the four warps, the new
+      // running maximum and the rescale of the old one; one thread: the P~
+      // scale 2^e that puts the largest s_V of the tile in [2^14, 2^15).
+      float2* bi = bc + (i & 1) * NQ;
+      if (t < NQ) {
+        float tmax = wm[t];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) svmax = max(svmax, wsv[(i & 1) * 4 + w]);
-      const float svmf = __half2float(__ushort_as_half((uint16_t)svmax));
-      const int e = svmf > 0.f ? 14 - (((__float_as_int(svmf) >> 23) & 0xFF) - 127) : 0;
+        for (int w = 1; w < 4; ++w) tmax = fmaxf(tmax, wm[w * NQ + t]);
+        const float mold = mrun[t], mnew = fmaxf(mold, tmax);
+        bi[t] = make_float2(mnew, mnew == kNegInf ? 1.f : ex2(mold - mnew));
+        mrun[t] = mnew;
+      } else if (t == kGConsumers - 1) {
+        uint32_t svmax = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) svmax = max(svmax, wsv[(i & 1) * 4 + w]);
+        const float svmf = __half2float(__ushort_as_half((uint16_t)svmax));
+        be[i & 1] = svmf > 0.f ? 14 - (((__float_as_int(svmf) >> 23) & 0xFF) - 127) : 0;
+      }
+      named_barrier_sync(1, kGConsumers);
+      const int e = be[i & 1];
       const float svs = (pos_cur < len) ? sv_cur * __int_as_float((127 + e) << 23) : 0.f;
       uint32_t pw[NO / 2];  // fp16 pairs of the P~ row: hi[0..NQ), lo[0..NQ), zero padding
 #pragma unroll
       for (int k = 0; k < NO / 2; ++k) pw[k] = 0u;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        float tmax = wm[q];
-#pragma unroll
-        for (int w = 1; w < 4; ++w) tmax = fmaxf(tmax, wm[w * NQ + q]);
-        const float mnew = fmaxf(m[q], tmax);
-        const float fr = mnew == kNegInf ? 1.f : ex2(m[q] - mnew);
-        const float p = s[q] == kNegInf ? 0.f : ex2(s[q] - mnew);
-        l[q] = fmaf(l[q], fr, p);
-        m[q] = mnew;
+        const float2 mf = bi[q];
+        const float p = s[q] == kNegInf ? 0.f : ex2(s[q] - mf.x);
+        l[q] = fmaf(l[q], mf.y, p);
         const float pt = p > 0.f ? p * svs : 0.f;
         const __half hi = __float2half_rn(pt);
         const __half lo = __float2half_rn(pt - __half2float(hi));
@@ -587,10 +603,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       for (int q = 0; q < NQ; ++q) res[q * (R + 2) + 2 + orow] = acc[q];
     named_barrier_sync(1, kGConsumers);
     if (t < NQ) {
-      float mt = kNegInf;  // m[t] without indexing the register array at run time
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) mt = q == t ? m[q] : mt;
-      res[t * (R + 2)] = mt;
+      res[t * (R + 2)] = mrun[t];
       res[t * (R + 2) + 1] = ((lsum[t] + lsum[NQ + t]) + lsum[2 * NQ + t]) + lsum[3 * NQ + t];
     }
     named_barrier_sync(1, kGConsumers);
