@@ -301,9 +301,8 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
  *   copied into step_workspace; the append and the decode run as in
  *   wsvd_append_and_decode on those copies; out [B][H][Hd] fp32 is copied to
  *   out_host.
- * When q_host starts right after the B*E x values in host memory, x and q go
- * in one copy.  The call returns once everything is queued; out_host is valid
- * after the stream is synchronised.  Page-locked (pinned) host buffers make the copies
+ * The call returns once everything is queued; out_host is valid after the
+ * stream is synchronised.  Page-locked (pinned) host buffers make the copies
  * asynchronous; pageable ones also work, with the driver's staging.
  *   step_workspace   device memory of at least
  *                    wsvd_step_host_workspace_size(B, H, Hd, E, r) bytes that is

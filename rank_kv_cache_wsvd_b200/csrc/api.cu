@@ -369,14 +369,9 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
                            B_v, nullptr, nullptr, 0, softmax_scale, out_dev, w + l.dec, l.x - l.dec, err, &dp);
   if (st != WSVD_OK) return st;
   cudaStream_t s = as_stream(stream);
-  const size_t xb = (size_t)B * E * 2, qb = (size_t)B * H * Hd * 2;
-  if (static_cast<const uint8_t*>(q_host) == static_cast<const uint8_t*>(x_host) + xb && l.q == l.x + xb) {
-    // q follows x in host memory as in the workspace: one copy
-    if (cudaMemcpyAsync(x_dev, x_host, xb + qb, cudaMemcpyHostToDevice, s) != cudaSuccess) return WSVD_ERR_CUDA;
-  } else if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-             cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+  if (cudaMemcpyAsync(x_dev, x_host, (size_t)B * E * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(q_dev, q_host, (size_t)B * H * Hd * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return WSVD_ERR_CUDA;
-  }
   if (launch_append(ap, s) != cudaSuccess) return WSVD_ERR_CUDA;
   bind_workspace(&dp, w + l.dec);
   if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, s, true) != cudaSuccess)

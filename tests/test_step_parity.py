@@ -107,8 +107,8 @@ def test_decode_launch_count_matches_the_path():
 def test_step_from_host_buffers_equals_device_step(name, adjacent):
     """wsvd_append_and_decode_host (x and q copied in from host memory, out
     copied back) gives bit for bit what wsvd_append_and_decode gives on the
-    same values already on the device, on two steps in a row; with q right
-    after x in one pinned buffer (one copy) and in separate buffers."""
+    same values already on the device, on two steps in a row; with x and q
+    in one pinned buffer and in separate ones."""
     w, lens0 = CASES[name]
     lens0 = [min(n, w.L_cap - 2) for n in lens0]  # two steps in a row: room for two appended rows
     d, ai = _inputs(w, lens0, seed=33)
