@@ -72,6 +72,7 @@ extern "C" int wsvd_fold_latent_rotation(int H, int E, int r, int Hd, const floa
       if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return WSVD_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();  // the status below is these launches', not an earlier call's
   const dim3 ga(grid_x((size_t)E * r), H), gb(grid_x((size_t)r * Hd), H);
   fold_a_kernel<<<ga, 256, 0, s>>>(E, r, static_cast<const __half*>(A_k), S2_k, static_cast<__half*>(A_k_out));
   fold_a_kernel<<<ga, 256, 0, s>>>(E, r, static_cast<const __half*>(A_v), S2_v, static_cast<__half*>(A_v_out));

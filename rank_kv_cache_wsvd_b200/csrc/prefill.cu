@@ -769,6 +769,7 @@ cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, i
   ta.inv_p = pa.inv_p; ta.seq_lens = pa.seq_lens;
   ta.lat_k = pa.lat_k; ta.lat_v = pa.lat_v; ta.scale_k = pa.scale_k; ta.scale_v = pa.scale_v; ta.err = err;
   const dim3 grid((unsigned)((pa.M + kTcBM - 1) / kTcBM), (unsigned)(pa.N / C::BN));
+  (void)cudaGetLastError();
   prefill_tc_kernel<R><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
   return cudaGetLastError();
 }
@@ -839,6 +840,7 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
   a.scale_k = static_cast<__half*>(scale_k); a.scale_v = static_cast<__half*>(scale_v);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();  // the status below is these launches', not an earlier call's
   const size_t rot_smem = (size_t)E * 4;
   if (cudaFuncSetAttribute(prefill_rotate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rot_smem) !=
           cudaSuccess ||
