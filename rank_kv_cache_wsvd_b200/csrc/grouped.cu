@@ -81,11 +81,12 @@ struct GCfg {
   static constexpr int NGRAN = MO == 64 ? 8 : 16;
   static constexpr int NS = (3 * NQ + 15) / 16 * 16;       // score columns: three planes per query
   static constexpr int NO = (2 * NQ + NGRAN - 1) / NGRAN * NGRAN;  // value columns: hi and lo per query
-  static constexpr int TRAW = 2 * NS + 2 * NO;
+  static constexpr int NV = 3;  // value operand / P~ / value accumulator buffers (tile i folded two tiles later)
+  static constexpr int TRAW = 2 * NS + NV * NO;
   static constexpr int TCOLS = TRAW <= 32 ? 32 : TRAW <= 64 ? 64 : TRAW <= 128 ? 128 : TRAW <= 256 ? 256 : 512;
   // shared memory, bytes
   static constexpr int STAGE = 2 * kGTok * RB + 2 * kGTok * 2;   // K codes, V codes, K scales, V scales
-  static constexpr int S = STAGE <= 9216 ? 6 : 4;
+  static constexpr int S = STAGE <= 9216 ? 4 : 3;
   static constexpr int AK = kGTok * KB;                          // K-major int8: chunk c at c * 2048
   static constexpr int LBO_A = kGTok * 16;
   static constexpr int LBO_V = R * 16;                           // MN-major fp16: 8-token groups
@@ -97,18 +98,18 @@ struct GCfg {
   static constexpr int QBLOCK = PL + NQ * 4;                     // per query group: planes, then steps
   static constexpr int OFF_AK = S * STAGE;
   static constexpr int OFF_VC = OFF_AK + 2 * AK;
-  static constexpr int OFF_P = OFF_VC + 2 * VC;
-  static constexpr int OFF_PL = OFF_P + 2 * PB;
+  static constexpr int OFF_P = OFF_VC + NV * VC;
+  static constexpr int OFF_PL = OFF_P + NV * PB;
   static constexpr int OFF_STEP = OFF_PL + PL;                   // float step[NQ] (staged with the planes)
   static constexpr int OFF_WMAX = OFF_STEP + 2 * NQ * 4;         // float wmax[2][4][NQ]
   static constexpr int OFF_WSV = OFF_WMAX + 2 * 4 * NQ * 4;      // uint32 wsv[2][4]
   static constexpr int OFF_LSUM = OFF_WSV + 8 * 4;               // float lsum[4][NQ]
-  static constexpr int OFF_BC = OFF_LSUM + 4 * NQ * 4;           // float2 bc[2][NQ] (new maximum, rescale)
-  static constexpr int OFF_MRUN = OFF_BC + 2 * NQ * 8;            // float mrun[NQ], int be[2]
+  static constexpr int OFF_BC = OFF_LSUM + 4 * NQ * 4;           // float2 bc[3][NQ] (new maximum, rescale)
+  static constexpr int OFF_MRUN = OFF_BC + 3 * NQ * 8;            // float mrun[NQ], int be[3]
   static constexpr int OFF_RES = OFF_MRUN + NQ * 4 + 16;          // float res[NQ][R + 2]
   static constexpr int OFF_MISC = OFF_RES + NQ * (R + 2) * 4;    // int flag, uint32 tmem base
   static constexpr int OFF_BAR = (OFF_MISC + 16 + 7) / 8 * 8;
-  static constexpr int NBAR = 2 * S + 9;
+  static constexpr int NBAR = 2 * S + 11;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8;
   // Shared memory requested at launch: at least enough that no more CTAs are
   // resident on an SM than its 512 tensor-memory columns can serve at once
@@ -210,14 +211,21 @@ __global__ void __launch_bounds__(128) grouped_qproj_kernel(const GroupedArgs a,
     uint4* dst = reinterpret_cast<uint4*>(bks);
     for (int i = t; i < R * a.Hd / 8; i += 128) dst[i] = src[i];
   }
-  for (int i = t; i < NQ * a.Hd; i += 128) {
-    const int ql = i / a.Hd, k = i % a.Hd;
-    float v = 0.f;
+  for (int i = t; i < NQ * a.Hd / 8; i += 128) {  // 8 query values per 16-byte load
+    const int ql = i / (a.Hd / 8), k8 = i % (a.Hd / 8);
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
     if (ql < nq) {
       const int qg = qc * NQ + ql, tq = qg / a.G, g = qg % a.G;
-      v = load_q_elem(a.q, a.q_dtype, (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd + k);
+      w = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) +
+                                         (((size_t)b * a.Tq + tq) * a.Hq + (size_t)hkv * a.G + g) * a.Hd)[k8];
     }
-    qs[i] = v;
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint16_t h16 = (uint16_t)(u[c >> 1] >> (16 * (c & 1)));
+      qs[ql * a.Hd + 8 * k8 + c] = a.q_dtype == WSVD_DTYPE_BF16 ? __uint_as_float((uint32_t)h16 << 16)
+                                                                 : __half2float(__ushort_as_half(h16));
+    }
   }
   __syncthreads();
   for (int o = t; o < NQ * R; o += 128) {
@@ -305,11 +313,12 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + S;
+  constexpr int NV = C::NV;
   uint64_t* conv = empty + S;   // [2] tile operands widened (128 arrivals)
   uint64_t* sready = conv + 2;  // [2] score MMAs done (commit)
-  uint64_t* pfull = sready + 2; // [2] P~ written (128 arrivals)
-  uint64_t* oready = pfull + 2; // [2] value MMAs done (commit)
-  uint64_t* pready = oready + 2; // the group's q' planes and steps are staged
+  uint64_t* pfull = sready + 2; // [NV] P~ written (128 arrivals)
+  uint64_t* oready = pfull + NV; // [NV] value MMAs done (commit)
+  uint64_t* pready = oready + NV; // the group's q' planes and steps are staged
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -319,6 +328,8 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     for (int s = 0; s < 2; ++s) {
       mbar_init(&conv[s], kGConsumers);
       mbar_init(&sready[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(&pfull[s], kGConsumers);
       mbar_init(&oready[s], 1);
     }
@@ -396,18 +407,19 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       scores(0);
       for (int i = 0; i < ntiles; ++i) {
         if (i + 1 < ntiles) scores(i + 1);
-        wait(&pfull[i & 1], (uint32_t)((i >> 1) & 1));
+        const int vb = i % NV;
+        wait(&pfull[vb], (uint32_t)((i / NV) & 1));
         tc05::fence_after_sync();
-        const uint32_t d = tmem + (uint32_t)(2 * NS + (i & 1) * NO);
-        const uint32_t vbase = s_vc + (uint32_t)((i & 1) * C::VC), pbase = s_p + (uint32_t)((i & 1) * C::PB);
+        const uint32_t d = tmem + (uint32_t)(2 * NS + vb * NO);
+        const uint32_t vbase = s_vc + (uint32_t)(vb * C::VC), pbase = s_p + (uint32_t)(vb * C::PB);
 #pragma unroll
         for (int kk = 0; kk < kGTok / 16; ++kk)
           tc05::mma_f16(d, tc05::smem_desc(vbase + kk * 2 * C::LBO_V, C::LBO_V, 128),
                         tc05::smem_desc(pbase + kk * 2 * C::LBO_P, C::LBO_P, 128), idesc_o, kk > 0);
-        tc05::commit(&oready[i & 1]);
+        tc05::commit(&oready[vb]);
       }
       // every MMA has completed before the allocation is released
-      wait(&oready[(ntiles - 1) & 1], (uint32_t)(((ntiles - 1) >> 1) & 1));
+      wait(&oready[(ntiles - 1) % NV], (uint32_t)(((ntiles - 1) / NV) & 1));
     }
     __syncwarp();
   } else {
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       wait(&full[s], (uint32_t)((j / S) & 1));
       const uint8_t* st = ring + (size_t)s * C::STAGE;
       const uint32_t ak = s_ak + (uint32_t)((j & 1) * C::AK) + (uint32_t)((t >> 3) * 128 + (t & 7) * 16);
-      const uint32_t vc = s_vc + (uint32_t)((j & 1) * C::VC) + (uint32_t)((t >> 3) * C::LBO_V + (t & 7) * 16);
+      const uint32_t vc = s_vc + (uint32_t)((j % NV) * C::VC) + (uint32_t)((t >> 3) * C::LBO_V + (t & 7) * 16);
       const uint32_t kr = smem_u32(st + t * RB), vr = smem_u32(st + kGTok * RB + t * RB);
 #pragma unroll
       for (int c = 0; c < RB / 16; ++c) {
@@ -472,13 +484,16 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       acc[q] = 0.f;
     }
     if (t < NQ) mrun[t] = kNegInf;  // ordered before its first use by the tile barriers
-    // Fold tile j's value accumulator (scaled by 2^-e) into acc, relative to m.
-    auto accumulate = [&](int j, int e) {
-      wait(&oready[j & 1], (uint32_t)((j >> 1) & 1));
+    // Fold tile j's value accumulator (scaled by 2^-e_j) into acc, relative to
+    // the maxima after tile j.
+    auto accumulate = [&](int j) {
+      const int vb = j % NV;
+      wait(&oready[vb], (uint32_t)((j / NV) & 1));
       tc05::fence_after_sync();
       if (warp_holds) {
+        const int e = be[vb];
         uint32_t v[(2 * NQ + 7) / 8 * 8];
-        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(2 * NS + (j & 1) * NO);
+        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(2 * NS + vb * NO);
 #pragma unroll
         for (int c = 0; c < (2 * NQ + 7) / 8; ++c) {
           uint32_t w8[8];
@@ -488,7 +503,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         }
         tc05::wait_ld();
         const float unscale = __int_as_float((127 - e) << 23);
-        const float2* bj = bc + (j & 1) * NQ;  // maxima after tile j
+        const float2* bj = bc + vb * NQ;  // maxima after tile j
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const float mq = bj[q].x;
@@ -504,10 +519,12 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     };
 
     float sk_cur, sv_cur;
-    int pos_cur, e_prev = 0;
+    int pos_cur;
     convert(0, sk_cur, sv_cur, pos_cur);
     for (int i = 0; i < ntiles; ++i) {
-      if (i >= 1) accumulate(i - 1, e_prev);
+      // tile i - 2's value product was issued a whole tile ago; its buffers
+      // (value operand, P~, accumulator) are then free for tile i + 1
+      if (i >= 2) accumulate(i - 2);
       float sk_n = 0.f, sv_n = 0.f;
       int pos_n = 0;
       if (i + 1 < ntiles) convert(i + 1, sk_n, sv_n, pos_n);
@@ -544,7 +561,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       // One thread per query: the tile maximum over the four warps, the new
       // running maximum and the rescale of the old one; one thread: the P~
       // scale 2^e that puts the largest s_V of the tile in [2^14, 2^15).
-      float2* bi = bc + (i & 1) * NQ;
+      float2* bi = bc + (i % NV) * NQ;
       if (t < NQ) {
         float tmax = wm[t];
 #pragma unroll
@@ -557,10 +574,10 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 #pragma unroll
         for (int w = 0; w < 4; ++w) svmax = max(svmax, wsv[(i & 1) * 4 + w]);
         const float svmf = __half2float(__ushort_as_half((uint16_t)svmax));
-        be[i & 1] = svmf > 0.f ? 14 - (((__float_as_int(svmf) >> 23) & 0xFF) - 127) : 0;
+        be[i % NV] = svmf > 0.f ? 14 - (((__float_as_int(svmf) >> 23) & 0xFF) - 127) : 0;
       }
       named_barrier_sync(1, kGConsumers);
-      const int e = be[i & 1];
+      const int e = be[i % NV];
       const float svs = (pos_cur < len) ? sv_cur * __int_as_float((127 + e) << 23) : 0.f;
       uint32_t pw[NO / 2];  // fp16 pairs of the P~ row: hi[0..NQ), lo[0..NQ), zero padding
 #pragma unroll
@@ -577,18 +594,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         pw[q >> 1] |= hb << (16 * (q & 1));
         pw[(NQ + q) >> 1] |= lb << (16 * ((NQ + q) & 1));
       }
-      const uint32_t pa = s_p + (uint32_t)((i & 1) * C::PB) + (uint32_t)((t >> 3) * C::LBO_P + (t & 7) * 16);
+      const uint32_t pa = s_p + (uint32_t)((i % NV) * C::PB) + (uint32_t)((t >> 3) * C::LBO_P + (t & 7) * 16);
 #pragma unroll
       for (int c = 0; c < NO / 8; ++c)
         sts128(pa + c * 128, make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
       tc05::fence_proxy_async_smem();
-      mbar_arrive(&pfull[i & 1]);
-      e_prev = e;
+      mbar_arrive(&pfull[i % NV]);
       sk_cur = sk_n;
       sv_cur = sv_n;
       pos_cur = pos_n;
     }
-    accumulate(ntiles - 1, e_prev);
+    for (int j = max(0, ntiles - 2); j < ntiles; ++j) accumulate(j);
 
     // CTA partial per query: (m, l, O[R])
 #pragma unroll

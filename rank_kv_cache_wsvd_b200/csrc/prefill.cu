@@ -478,8 +478,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 //            (3-D tensor map over A [H][E][r], swizzle of NG * 2 bytes; the
 //            operand is N-major) into a four-stage mbarrier ring;
 //   warp 5   allocates tensor memory; one lane issues per k-tile four MMAs of
-//            the hi half into a fresh accumulator (double-buffered) and four
-//            of the lo half into one accumulator kept over all of E;
+//            the hi half into a fresh accumulator (one of NH, so that it runs
+//            up to NH k-tiles ahead of the epilogue) and four of the lo half
+//            into one accumulator kept over all of E;
 //   warps 0-3  thread t <-> output row t <-> tensor-memory lane t: add each
 //            k-tile's hi sum to an fp32 register total with a round-to-nearest
 //            add, then add the lo sum, undo p_m and quantise every head of the
@@ -498,7 +499,10 @@ struct TcCfg {
   static constexpr int A_BYTES = kTcBM * kTcBK * 2;
   static constexpr int W_BYTES = kTcBK * BN * 2;
   static constexpr int STAGE = 2 * A_BYTES + W_BYTES;
-  static constexpr int TCOLS = 3 * BN <= 256 ? 256 : 512;
+  // NH fresh accumulators for the hi k-tile sums (the MMA warp runs up to NH
+  // k-tiles ahead of the epilogue), then the lo accumulator: all 512 columns.
+  static constexpr int NH = BN == 64 ? 6 : 3;
+  static constexpr int TCOLS = 512;
   static constexpr int SMEM = kTcStages * STAGE + 1024 + 256;
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle-atom alignment");
 };
@@ -543,9 +547,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = smem_raw + (base - raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::STAGE);
   uint64_t* empty = full + S;
-  uint64_t* hfull = empty + S;  // [2] a k-tile's hi sum is in tensor memory
-  uint64_t* hfree = hfull + 2;  // [2] the epilogue has read it (128 arrivals)
-  uint64_t* done = hfree + 2;   // every MMA of the tile has completed
+  constexpr int NH = C::NH;
+  uint64_t* hfull = empty + S;   // [NH] a k-tile's hi sum is in tensor memory
+  uint64_t* hfree = hfull + NH;  // [NH] the epilogue has read it (128 arrivals)
+  uint64_t* done = hfree + NH;   // every MMA of the tile has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -557,7 +562,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NH; ++i) {
       mbar_init(&hfull[i], 1);
       mbar_init(&hfree[i], 128);
     }
@@ -603,10 +608,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % S;
         wait(&full[s], (uint32_t)((kt / S) & 1));
-        if (kt >= 2) wait(&hfree[kt & 1], (uint32_t)(((kt >> 1) - 1) & 1));
+        const int hb = kt % NH;
+        if (kt >= NH) wait(&hfree[hb], (uint32_t)(((kt / NH) - 1) & 1));
         tc05::fence_after_sync();
         const uint32_t st = base + (uint32_t)(s * C::STAGE);
-        const uint32_t dh = tmem + (uint32_t)((kt & 1) * BN), dl = tmem + (uint32_t)(2 * BN);
+        const uint32_t dh = tmem + (uint32_t)(hb * BN), dl = tmem + (uint32_t)(NH * BN);
 #pragma unroll
         for (int kk = 0; kk < kTcBK / 16; ++kk) {
           const uint64_t bd = tc05::smem_desc_sw(st + 2 * C::A_BYTES + kk * 32 * NG, 128 * NG, 16 * NG, C::SW);
@@ -614,7 +620,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc05::mma_f16(dl, tc05::smem_desc_sw(st + C::A_BYTES + kk * 32, 16, 1024, 2), bd, idesc, kt > 0 || kk > 0);
         }
         tc05::commit(&empty[s]);
-        tc05::commit(&hfull[kt & 1]);
+        tc05::commit(&hfull[hb]);
       }
       tc05::commit(done);
       wait(done, 0);  // every MMA has completed before the allocation is released
@@ -627,25 +633,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
     for (int c = 0; c < BN; ++c) tot[c] = 0.f;
     for (int kt = 0; kt < KT; ++kt) {
-      wait(&hfull[kt & 1], (uint32_t)((kt >> 1) & 1));
+      const int hb = kt % NH;
+      wait(&hfull[hb], (uint32_t)((kt / NH) & 1));
       tc05::fence_after_sync();
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
-        tc05::ld32(lane_base + (uint32_t)((kt & 1) * BN + c0), v);
+        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0), v);
         tc05::wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
       }
       tc05::fence_before_sync();
-      mbar_arrive(&hfree[kt & 1]);
+      mbar_arrive(&hfree[hb]);
     }
     wait(done, 0);
     tc05::fence_after_sync();
 #pragma unroll
     for (int c0 = 0; c0 < BN; c0 += 32) {
       uint32_t v[32];
-      tc05::ld32(lane_base + (uint32_t)(2 * BN + c0), v);
+      tc05::ld32(lane_base + (uint32_t)(NH * BN + c0), v);
       tc05::wait_ld();
 #pragma unroll
       for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
