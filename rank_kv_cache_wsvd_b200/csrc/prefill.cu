@@ -491,9 +491,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 // nearest, the lo half keeps one tensor-core sum.
 constexpr int kTcBM = 128, kTcBK = 64, kTcStages = 4, kTcThreads = 192;
 
-template <int R>
+template <int R, int BN_>
 struct TcCfg {
-  static constexpr int BN = R <= 64 ? 64 : 128;          // output columns per tile (whole heads)
+  static constexpr int BN = BN_;                          // output columns per tile (whole heads)
   static constexpr int NG = R <= 64 ? R : 64;            // columns per weight box (one head, or half of r = 128)
   static constexpr int SW = NG == 16 ? 6 : (NG == 32 ? 4 : 2);  // descriptor swizzle: 32 / 64 / 128 bytes
   static constexpr int A_BYTES = kTcBM * kTcBK * 2;
@@ -502,6 +502,8 @@ struct TcCfg {
   // NH fresh accumulators for the hi k-tile sums (the MMA warp runs up to NH
   // k-tiles ahead of the epilogue), then the lo accumulator: all 512 columns.
   static constexpr int NH = BN == 64 ? 6 : 3;
+  static_assert(BN == 64 || BN == 128, "tile width");
+  static_assert(R <= BN, "whole heads per tile");
   static constexpr int TCOLS = 512;
   static constexpr int SMEM = kTcStages * STAGE + 1024 + 256;
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle-atom alignment");
@@ -534,12 +536,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
-template <int R>
+template <int R, int BN_>
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_xhi, const __grid_constant__ CUtensorMap tm_xlo,
                       const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
                       const TcArgs a) {
-  using C = TcCfg<R>;
+  using C = TcCfg<R, BN_>;
   constexpr int BN = C::BN, NG = C::NG, S = kTcStages;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -762,14 +764,15 @@ bool encode_weight_map(CUtensorMap* tm, const void* base, int H, int E, int r, i
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int R>
+template <int R, int BN>
 cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, int32_t* err, cudaStream_t s) {
-  using C = TcCfg<R>;
+  using C = TcCfg<R, BN>;
   CUtensorMap mh, ml, mk, mv;
   if (!encode_act_map(&mh, pa.xhi, pa.M, pa.E) || !encode_act_map(&ml, pa.xlo, pa.M, pa.E) ||
       !encode_weight_map(&mk, A_k, pa.H, pa.E, R, C::NG) || !encode_weight_map(&mv, A_v, pa.H, pa.E, R, C::NG))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(prefill_tc_kernel<R, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   TcArgs ta{};
   ta.M = pa.M; ta.T = pa.T; ta.H = pa.H; ta.bits = pa.bits; ta.L_cap = pa.L_cap; ta.KT = pa.E / kTcBK;
@@ -777,16 +780,21 @@ cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, i
   ta.lat_k = pa.lat_k; ta.lat_v = pa.lat_v; ta.scale_k = pa.scale_k; ta.scale_v = pa.scale_v; ta.err = err;
   const dim3 grid((unsigned)((pa.M + kTcBM - 1) / kTcBM), (unsigned)(pa.N / C::BN));
   (void)cudaGetLastError();
-  prefill_tc_kernel<R><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
+  prefill_tc_kernel<R, BN><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
   return cudaGetLastError();
 }
 
-// The tcgen05 path serves r in {16, 32, 64, 128} when every output tile holds
-// whole heads of one side (H * r a multiple of the tile width).
-bool tc_supported(int H, int r) {
-  if (r != 16 && r != 32 && r != 64 && r != 128) return false;
-  const int bn = r <= 64 ? 64 : 128;
-  return ((long long)H * r) % bn == 0;
+// Output tile width of the tcgen05 path: 128 columns when the tiles hold whole
+// heads of one side and there are enough of them to fill the device (every
+// tile re-reads the activation rows of its m-tile from L2, so wider tiles
+// halve that traffic); otherwise 64 (r <= 64), or 0 when the path does not
+// apply.
+int tc_tile_width(long long M, int H, int r) {
+  if (r != 16 && r != 32 && r != 64 && r != 128) return 0;
+  const long long hr = (long long)H * r, mt = (M + kTcBM - 1) / kTcBM;
+  if (hr % 128 == 0 && (r == 128 || mt * (2 * hr / 128) >= 64)) return 128;
+  if (r <= 64 && hr % 64 == 0) return 64;
+  return 0;
 }
 
 // ------------------------------------------------------------------ 3. lengths
@@ -873,13 +881,22 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
     prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo,
                                                                      winv);
   }
-  if (tc_supported(H, r)) {
+  const int bn = tc_tile_width(M, H, r);
+  if (bn) {
     cudaError_t e = cudaSuccess;
-    switch (r) {
-      case 16: e = launch_tc<16>(a, A_k, A_v, err, s); break;
-      case 32: e = launch_tc<32>(a, A_k, A_v, err, s); break;
-      case 64: e = launch_tc<64>(a, A_k, A_v, err, s); break;
-      default: e = launch_tc<128>(a, A_k, A_v, err, s); break;
+    if (bn == 128) {
+      switch (r) {
+        case 16: e = launch_tc<16, 128>(a, A_k, A_v, err, s); break;
+        case 32: e = launch_tc<32, 128>(a, A_k, A_v, err, s); break;
+        case 64: e = launch_tc<64, 128>(a, A_k, A_v, err, s); break;
+        default: e = launch_tc<128, 128>(a, A_k, A_v, err, s); break;
+      }
+    } else {
+      switch (r) {
+        case 16: e = launch_tc<16, 64>(a, A_k, A_v, err, s); break;
+        case 32: e = launch_tc<32, 64>(a, A_k, A_v, err, s); break;
+        default: e = launch_tc<64, 64>(a, A_k, A_v, err, s); break;
+      }
     }
     if (e != cudaSuccess) return WSVD_ERR_CUDA;
   } else {

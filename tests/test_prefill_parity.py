@@ -97,7 +97,8 @@ def _run(w: WL.Workload, T: int, lens0, bits=None, blk=None, x_dtype="bf16", see
 
 def test_llava_image_block_576_tokens():
     """The 576 image tokens of the LLaVA-7B-shaped layer in one call (B 1, H 32,
-    E 4096, r 32, int8, 128-block Hadamard): nine 64-row tiles x 16 column tiles."""
+    E 4096, r 32, int8, 128-block Hadamard): five 128-row tiles (the last one
+    ragged) x 16 column tiles of 128."""
     w = WL.LLAVA7B
     ties, err, g, _ = _run(w, 576, [0], seed=3)
     assert err == 0 and list(g["lens"]) == [576]
@@ -121,6 +122,16 @@ def test_column_tiles_heads_and_formats(H, r, bits):
     w = WL.Workload("pf-cols", B=2, H=H, Hd=64, r=r, bits=bits, L_cap=16, lens=0, E=256)
     ties, err, g, _ = _run(w, 5, [0, 9], seed=H * 100 + r)
     assert err == 0 and list(g["lens"]) == [5, 14]
+
+
+def test_wide_tiles_of_eight_small_heads():
+    """r 16 int4 with 128-column tiles (eight heads per tile): 4096 token rows
+    over 16 heads fill the device with the wide tiles."""
+    w = WL.Workload("pf-wide", B=2, H=16, Hd=64, r=16, bits=4, L_cap=2100, lens=0, E=256)
+    ties, err, g, _ = _run(w, 2048, [0, 52], seed=21)
+    assert err == 0 and list(g["lens"]) == [2048, 2100]
+    code_bound, scale_bound = tie_bounds(2048 * w.B * w.H * 2, w.r)
+    assert ties[0] <= code_bound and ties[1] <= scale_bound, (ties, code_bound, scale_bound)
 
 
 @pytest.mark.parametrize("E,blk,x_dtype", [(256, 1, "fp16"), (1024, 256, "bf16"), (2048, 64, "bf16"),
