@@ -858,8 +858,9 @@ def main():
     extras = {}
     if not args.no_extras and rank == 0:
         # End to end through the public API with host buffers: one library call
-        # per step (H2D of x and q from pinned memory, append, decode, D2H of
-        # out) and a stream synchronisation; host wall clock around the two.
+        # per step (x and q brought in from pinned host memory, append, decode,
+        # out delivered to pinned host memory) and a stream synchronisation;
+        # host wall clock around the two.
         # The length reset that lets every step append the same row is done
         # before the clock starts.
         n_e2e = max(50, min(args.steps, 500))

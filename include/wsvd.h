@@ -296,20 +296,30 @@ int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_c
  * host memory (a serving loop that receives the new token's activation and
  * query from the host and returns the attention output there).  The pages
  * have no counterpart: it exists so that one library call covers a whole
- * step, copies included.  On `stream`, in order:
+ * step, host transfers included.  On `stream`, in order:
  *   x_host [B][E] and q_host [B][H][Hd] (16-bit, x_dtype / q_dtype) are
- *   copied into step_workspace; the append and the decode run as in
- *   wsvd_append_and_decode on those copies; out [B][H][Hd] fp32 is copied to
- *   out_host.
+ *   brought into step_workspace; the append and the decode run as in
+ *   wsvd_append_and_decode on those device copies; out [B][H][Hd] fp32 is
+ *   delivered to out_host.
+ * How the bytes move depends on the host memory:
+ *   - x_host, q_host and out_host all page-locked and mapped into the device's
+ *     address space (every cudaHostAlloc / cudaMallocHost allocation under
+ *     unified addressing), 16-byte aligned, with B*E*2 and B*H*Hd*2 multiples
+ *     of 16: a small kernel reads x and q from host memory (the append is
+ *     launched behind it as a programmatic dependent and streams A_k, A_v in
+ *     the meantime), and the decode stores out straight into out_host.  No
+ *     copy-engine transfer is queued.
+ *   - otherwise: cudaMemcpyAsync copies in and out (pageable memory goes
+ *     through the driver's staging).
  * The call returns once everything is queued; out_host is valid after the
- * stream is synchronised.  Page-locked (pinned) host buffers make the copies
- * asynchronous; pageable ones also work, with the driver's staging.
+ * stream is synchronised, and the host may rewrite x_host and q_host only
+ * after that (they are read while the step runs).
  *   step_workspace   device memory of at least
  *                    wsvd_step_host_workspace_size(B, H, Hd, E, r) bytes that is
  *                    ZERO before the first call; it holds the append and
  *                    decode workspaces (their counters are left zero) and the
- *                    device copies of x, q and out.  Calls that share it must
- *                    not overlap on the GPU.
+ *                    device copies of x, q (and out, for the copy route).
+ *                    Calls that share it must not overlap on the GPU.
  * Every other argument is as for wsvd_append_and_decode (device pointers).
  * All arguments are validated before anything is queued.                    */
 size_t wsvd_step_host_workspace_size(int B, int H, int Hd, int E, int r);

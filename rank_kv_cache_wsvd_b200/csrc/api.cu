@@ -2,6 +2,9 @@
 // No allocation, no synchronisation; every launch goes to the caller's stream.
 #include <math.h>
 
+#include <algorithm>
+
+#include "common.cuh"
 #include "wsvd_internal.h"
 
 using namespace wsvd;
@@ -35,6 +38,32 @@ void bind_workspace(DecodeArgs* a, void* workspace) {
   a->partials = reinterpret_cast<float*>(w);
   a->counters = reinterpret_cast<int32_t*>(w + partial_bytes(a->B, a->H, a->W));
   a->qglobal = reinterpret_cast<float*>(w + partial_bytes(a->B, a->H, a->W) + counter_bytes(a->B, a->H));
+}
+
+// Device address of pinned host memory that is mapped into the device's
+// address space (every cudaHostAlloc / cudaMallocHost allocation under unified
+// addressing), or nullptr for any other pointer.
+void* mapped_device_pointer(const void* host) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
+// The step's inputs from mapped host memory into the step workspace, 16 bytes
+// per thread and load, uncached (the host rewrites these buffers every step).
+// The append is launched behind it as a programmatic dependent: it streams its
+// weights at once and reads x after griddepcontrol.wait.
+__global__ void __launch_bounds__(256) step_ingest_kernel(const uint4* x_src, uint4* x_dst, int nx, const uint4* q_src,
+                                                          uint4* q_dst, int nq) {
+  griddep_launch_dependents();
+  const int stride = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nx + nq; i += stride) {
+    if (i < nx) x_dst[i] = __ldcv(x_src + i);
+    else q_dst[i - nx] = __ldcv(q_src + (i - nx));
+  }
 }
 
 constexpr size_t kAppendWorkspaceBytes = 256;  // the completion counter (padded)
@@ -359,7 +388,15 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
   uint8_t* w = static_cast<uint8_t*>(step_workspace);
   void* x_dev = w + l.x;
   void* q_dev = w + l.q;
-  float* out_dev = reinterpret_cast<float*>(w + l.out);
+  const size_t xbytes = (size_t)B * E * 2, qbytes = (size_t)B * H * Hd * 2, obytes = (size_t)B * H * Hd * 4;
+  // Pinned (mapped) host buffers are read and written in place by the
+  // kernels; any other host memory goes through copies.
+  void* xm = mapped_device_pointer(x_host);
+  void* qm = xm ? mapped_device_pointer(q_host) : nullptr;
+  void* om = qm ? mapped_device_pointer(out_host) : nullptr;
+  const bool in_place = om && aligned16(xm) && aligned16(qm) && aligned16(om) && xbytes % 16 == 0 &&
+                        qbytes % 16 == 0 && (xbytes + qbytes) / 16 <= 0x7fffffffu;
+  float* out_dev = in_place ? static_cast<float*>(om) : reinterpret_cast<float*>(w + l.out);
   AppendArgs ap{};
   int st = prepare_append(B, H, E, r, bits, L_cap, hadamard_block, x_dev, x_dtype, A_k, A_v, nullptr, nullptr, 0,
                           seq_lens, lat_k, lat_v, scale_k, scale_v, w + l.app, kAppendWorkspaceBytes, err, &ap);
@@ -369,14 +406,23 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
                            B_v, nullptr, nullptr, 0, softmax_scale, out_dev, w + l.dec, l.x - l.dec, err, &dp);
   if (st != WSVD_OK) return st;
   cudaStream_t s = as_stream(stream);
-  if (cudaMemcpyAsync(x_dev, x_host, (size_t)B * E * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(q_dev, q_host, (size_t)B * H * Hd * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  (void)cudaGetLastError();  // the status below is these launches', not an earlier call's
+  if (in_place) {
+    const int nx = (int)(xbytes / 16), nq = (int)(qbytes / 16);
+    const int grid = std::min(148, (nx + nq + 255) / 256);
+    step_ingest_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(xm), static_cast<uint4*>(x_dev), nx,
+                                            static_cast<const uint4*>(qm), static_cast<uint4*>(q_dev), nq);
+    if (cudaGetLastError() != cudaSuccess) return WSVD_ERR_CUDA;
+    ap.dep = 1;
+  } else if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+             cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
     return WSVD_ERR_CUDA;
+  }
   if (launch_append(ap, s) != cudaSuccess) return WSVD_ERR_CUDA;
   bind_workspace(&dp, w + l.dec);
   if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, s, true) != cudaSuccess)
     return WSVD_ERR_CUDA;
-  if (cudaMemcpyAsync(out_host, out_dev, (size_t)B * H * Hd * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  if (!in_place && cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return WSVD_ERR_CUDA;
   return WSVD_OK;
 }

@@ -212,22 +212,26 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   // deferred to the first remote access.
   cluster_arrive_relaxed();
 
-  // 1. x slice loads first (registers), then the A stream.
+  // 1. x slice loads first (registers), then the A stream.  Behind the grid
+  // that writes x, the A stream goes first and x is read after the wait.
   constexpr int kMaxChunks = 4;  // 128-element x chunks per warp held in registers (fast path)
   const int nch = B * Ec / 128;
   const bool fast = (Ec % 128 == 0) && a.blk <= 128 && nch <= kMaxChunks * kAppendWarps;
   uint2 xraw[kMaxChunks];
   const uint16_t* xg = static_cast<const uint16_t*>(a.x);
-  if (fast) {
+  auto load_x = [&]() {
+    if (fast) {
 #pragma unroll
-    for (int t = 0; t < kMaxChunks; ++t) {
-      const int ch = warp + t * kAppendWarps;
-      if (ch < nch) {
-        const int b = ch / (Ec / 128), off = (ch % (Ec / 128)) * 128;
-        xraw[t] = __ldg(reinterpret_cast<const uint2*>(xg + (size_t)b * E + e0 + off) + lane);
+      for (int t = 0; t < kMaxChunks; ++t) {
+        const int ch = warp + t * kAppendWarps;
+        if (ch < nch) {
+          const int b = ch / (Ec / 128), off = (ch % (Ec / 128)) * 128;
+          xraw[t] = __ldcg(reinterpret_cast<const uint2*>(xg + (size_t)b * E + e0 + off) + lane);
+        }
       }
     }
-  }
+  };
+  if (!a.dep) load_x();
   const int ncg = r / 8, nrg = kAppendThreads / ncg;
   RowWalk<W8> w;
   w.A = static_cast<const uint8_t*>(kv ? a.Av : a.Ak) + ((size_t)h * E + e0) * (size_t)r * (W8 ? 1 : 2);
@@ -235,6 +239,10 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   w.nrows = w.rg < Ec ? (Ec - 1 - w.rg) / nrg + 1 : 0;
 #pragma unroll 1
   for (int k = 0; k < kRing; ++k) w.issue(ring, k, tid);
+  if (a.dep) {
+    griddep_wait();
+    load_x();
+  }
 
   // 2. Rotate x into xs[b][e] (unnormalised; 1/sqrt(blk) is applied to c).
   if (fast) {
@@ -407,13 +415,15 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kAppendThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.dep ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

@@ -185,6 +185,20 @@ __device__ __forceinline__ uint4 i4x8_to_h(uint32_t w) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// An integer below 2^22 in magnitude to fp32, exactly, on the FMA pipe:
+// adding it to the bits of 1.5 * 2^23 lands it in that float's mantissa.
+__device__ __forceinline__ float small_int_to_f32(uint32_t v) {
+  return __int_as_float((int)v + 0x4B400000) - 12582912.f;
+}
+
+// Score of query q from its three plane sums (h 2^16 + m 2^8 + l); every plane
+// sum is below 128 * 127 * 127 < 2^21 in magnitude.
+template <int N>
+__device__ __forceinline__ float plane_sum(const uint32_t (&sv)[N], int q) {
+  return fmaf(small_int_to_f32(sv[3 * q]), 65536.f,
+              fmaf(small_int_to_f32(sv[3 * q + 1]), 256.f, small_int_to_f32(sv[3 * q + 2])));
+}
+
 // q' of every query of one (b, latent head, query chunk) group, as the score
 // operand the decode kernel stages: q'_q = (B_Kh . q_q) * softmax_scale * log2 e,
 // quantised with step max|q'_q| / 8355711 and written as three signed byte
@@ -428,6 +442,7 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     wait(pready, 0);  // the group's steps (and planes) are staged
     float step[NQ];
     int nvis[NQ];  // rows visible to each query
+    const int vis_min = len - a.Tq + 1 + (qc * NQ) / a.G;  // the chunk's first query sees the fewest
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       step[q] = stepv[q];
@@ -476,16 +491,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     const int orow = MO == 64 ? (lane < 16 ? warp * 16 + lane : -1) : t;
     const bool holder = orow >= 0 && orow < R;
     const bool warp_holds = MO == 64 ? warp * 16 < R : warp * 32 < R;
-    float l[NQ], macc[NQ], acc[NQ];
+    float l[NQ], acc[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       l[q] = 0.f;
-      macc[q] = kNegInf;
       acc[q] = 0.f;
     }
     if (t < NQ) mrun[t] = kNegInf;  // ordered before its first use by the tile barriers
-    // Fold tile j's value accumulator (scaled by 2^-e_j) into acc, relative to
-    // the maxima after tile j.
+    // Fold tile j's value accumulator (scaled by 2^-e_j) into acc, rescaled
+    // from the maxima before tile j to the maxima after it (the factor tile
+    // j's softmax step broadcast: 0 while nothing was seen, 1 while a query
+    // still sees nothing, when its columns are zero).
     auto accumulate = [&](int j) {
       const int vb = j % NV;
       wait(&oready[vb], (uint32_t)((j / NV) & 1));
@@ -503,16 +519,11 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         }
         tc05::wait_ld();
         const float unscale = __int_as_float((127 - e) << 23);
-        const float2* bj = bc + vb * NQ;  // maxima after tile j
+        const float2* bj = bc + vb * NQ;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          const float mq = bj[q].x;
-          if (mq != kNegInf) {
-            const float d = (__uint_as_float(v[q]) + __uint_as_float(v[NQ + q])) * unscale;
-            const float f = macc[q] == kNegInf ? 0.f : ex2(macc[q] - mq);
-            acc[q] = fmaf(acc[q], f, d);
-            macc[q] = mq;
-          }
+          const float d = (__uint_as_float(v[q]) + __uint_as_float(v[NQ + q])) * unscale;
+          acc[q] = fmaf(acc[q], bj[q].y, d);
         }
       }
       tc05::fence_before_sync();
@@ -545,11 +556,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       }
       float s[NQ];
       float* wm = wmax + (i & 1) * 4 * NQ;
+      // Every row of a tile below the first query's horizon is visible to all
+      // real queries: no per-query test there.
+      if (nq == NQ && t_begin + (i + 1) * kGTok <= vis_min) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) s[q] = plane_sum(sv32, q) * step[q] * sk_cur;
+      } else {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) s[q] = pos_cur < nvis[q] ? plane_sum(sv32, q) * step[q] * sk_cur : kNegInf;
+      }
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        const float combo = fmaf((float)(int)sv32[3 * q], 65536.f,
-                                 fmaf((float)(int)sv32[3 * q + 1], 256.f, (float)(int)sv32[3 * q + 2]));
-        s[q] = pos_cur < nvis[q] ? combo * step[q] * sk_cur : kNegInf;
         const float mx = warp_max_f32(s[q]);
         if (lane == 0) wm[warp * NQ + q] = mx;
       }
@@ -567,7 +584,9 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 #pragma unroll
         for (int w = 1; w < 4; ++w) tmax = fmaxf(tmax, wm[w * NQ + t]);
         const float mold = mrun[t], mnew = fmaxf(mold, tmax);
-        bi[t] = make_float2(mnew, mnew == kNegInf ? 1.f : ex2(mold - mnew));
+        // .x: the maximum the tile's exponentials are taken against (0 while
+        // the query sees nothing, so that -inf - .x stays -inf); .y: rescale
+        bi[t] = make_float2(mnew == kNegInf ? 0.f : mnew, mnew == kNegInf ? 1.f : ex2(mold - mnew));
         mrun[t] = mnew;
       } else if (t == kGConsumers - 1) {
         uint32_t svmax = 0;
@@ -581,18 +600,19 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       const float svs = (pos_cur < len) ? sv_cur * __int_as_float((127 + e) << 23) : 0.f;
       uint32_t pw[NO / 2];  // fp16 pairs of the P~ row: hi[0..NQ), lo[0..NQ), zero padding
 #pragma unroll
-      for (int k = 0; k < NO / 2; ++k) pw[k] = 0u;
+      for (int k = NQ; k < NO / 2; ++k) pw[k] = 0u;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const float2 mf = bi[q];
-        const float p = s[q] == kNegInf ? 0.f : ex2(s[q] - mf.x);
-        l[q] = fmaf(l[q], mf.y, p);
-        const float pt = p > 0.f ? p * svs : 0.f;
-        const __half hi = __float2half_rn(pt);
-        const __half lo = __float2half_rn(pt - __half2float(hi));
-        const uint32_t hb = __half_as_ushort(hi), lb = __half_as_ushort(lo);
-        pw[q >> 1] |= hb << (16 * (q & 1));
-        pw[(NQ + q) >> 1] |= lb << (16 * ((NQ + q) & 1));
+      for (int q = 0; q < NQ; q += 2) {
+        const float2 m0 = bi[q], m1 = bi[q + 1];
+        const float p0 = ex2(s[q] - m0.x), p1 = ex2(s[q + 1] - m1.x);  // 0 for a row the query does not see
+        l[q] = fmaf(l[q], m0.y, p0);
+        l[q + 1] = fmaf(l[q + 1], m1.y, p1);
+        const float t0 = p0 * svs, t1 = p1 * svs;
+        const __half2 hi = __floats2half2_rn(t0, t1);
+        const float2 hf = __half22float2(hi);
+        const __half2 lo = __floats2half2_rn(t0 - hf.x, t1 - hf.y);
+        pw[q >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+        pw[(NQ + q) >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
       }
       const uint32_t pa = s_p + (uint32_t)((i % NV) * C::PB) + (uint32_t)((t >> 3) * C::LBO_P + (t & 7) * 16);
 #pragma unroll
@@ -680,13 +700,14 @@ struct GroupedKernels {
   const void* qproj;   // grouped_qproj_kernel
   const void* decode;  // grouped_decode_kernel
   size_t smem;
+  int tmem_ctas;       // CTAs per SM that the 512 tensor-memory columns serve at once
 };
 
 template <int CODEC, int RB, int NQ>
 GroupedKernels kernels_of() {
   return GroupedKernels{reinterpret_cast<const void*>(&grouped_qproj_kernel<CODEC, RB, NQ>),
                         reinterpret_cast<const void*>(&grouped_decode_kernel<CODEC, RB, NQ>),
-                        (size_t)GCfg<CODEC, RB, NQ>::SMEM};
+                        (size_t)GCfg<CODEC, RB, NQ>::SMEM, GCfg<CODEC, RB, NQ>::TMEM_CTAS};
 }
 
 template <int CODEC, int RB>
@@ -715,8 +736,11 @@ std::mutex g_mu;
 std::map<std::pair<const void*, int>, int> g_occ;  // (kernel, device) -> resident CTAs per SM (smem opted in)
 std::map<int, int> g_sms;
 
-// Opts the kernel into its shared memory and returns (SMs, resident CTAs per SM).
-cudaError_t device_setup(const void* fn, size_t smem, int* sms, int* occ) {
+// Opts the kernel into its shared memory and returns (SMs, resident CTAs per
+// SM).  The residency is worked out from the kernel's registers, its shared
+// memory and its tensor-memory columns (the occupancy query knows nothing of
+// the last).
+cudaError_t device_setup(const void* fn, size_t smem, int tmem_ctas, int* sms, int* occ) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -730,14 +754,33 @@ cudaError_t device_setup(const void* fn, size_t smem, int* sms, int* occ) {
   }
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int n = 148, o = 1;
+  int n = 148, sm_smem = 233472, sm_regs = 65536, reserved = 1024;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kGThreads, smem) != cudaSuccess || o < 1) o = 1;
+  cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  cudaFuncAttributes fa{};
+  int o = tmem_ctas;
+  if (cudaFuncGetAttributes(&fa, fn) == cudaSuccess && fa.numRegs > 0) {
+    const int warp_regs = (fa.numRegs * 32 + 255) / 256 * 256;  // allocated per warp in 256-register units
+    o = std::min(o, sm_regs / (warp_regs * (kGThreads / 32)));
+  }
+  o = std::min(o, (int)(sm_smem / (smem + (size_t)reserved)));
+  o = std::max(o, 1);
   g_occ[key] = o;
   g_sms[dev] = n;
   *occ = o;
   *sms = n;
   return cudaSuccess;
+}
+
+// Splits per (b, latent head, query chunk): as many as fill the resident CTA
+// slots in one wave (a grid a little over a whole number of waves leaves a
+// tail as long as a CTA), never more than there are tiles or partial slots.
+int grouped_splits(long long groups, int tiles_cap, int slots, int sms, int occ) {
+  const long long resident = (long long)sms * occ;
+  const long long per_group = groups >= resident ? 1 : resident / groups;
+  return (int)std::max<long long>(1, std::min<long long>(std::min<long long>(tiles_cap, slots), per_group));
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -802,15 +845,14 @@ extern "C" int wsvd_decode_multi(int B, int Tq, int Hq, int Hkv, int Hd, int r, 
   if (!pick_grouped(bits, rb, sh.nq, &gk)) return WSVD_ERR_UNSUPPORTED;
   const size_t smem = gk.smem;
   int sms = 148, occ = 1;
-  if (device_setup(gk.decode, smem, &sms, &occ) != cudaSuccess) return WSVD_ERR_CUDA;
+  if (device_setup(gk.decode, smem, gk.tmem_ctas, &sms, &occ) != cudaSuccess) return WSVD_ERR_CUDA;
 
   GroupedArgs ga{};
   ga.B = B; ga.Tq = Tq; ga.Hq = Hq; ga.Hkv = Hkv; ga.G = G; ga.Hd = Hd; ga.L_cap = L_cap;
   ga.nqc = sh.nqc;
   const int tiles_cap = std::max(1, (L_cap + kGTok - 1) / kGTok);
   const long long groups = (long long)B * Hkv * sh.nqc;
-  const long long target = 2LL * sms * occ;  // two waves of resident CTAs
-  int nsplit = (int)std::min<long long>(sh.slots, std::max<long long>(1, (target + groups - 1) / groups));
+  const int nsplit = grouped_splits(groups, tiles_cap, sh.slots, sms, occ);
   ga.chunk_tiles = (tiles_cap + nsplit - 1) / nsplit;
   ga.nsplit = (tiles_cap + ga.chunk_tiles - 1) / ga.chunk_tiles;
   ga.slot_stride = sh.slots;

@@ -84,6 +84,7 @@ struct AppendArgs {
   __half* scale_v;
   int32_t* counter;
   int32_t* err;
+  int dep;               // 1: launched as a programmatic dependent of the grid that writes x (read after the wait)
 };
 int append_cluster_size(int E, int blk);
 // wsvd_decode_attention with caller-provided scratch that is NOT zero on entry

@@ -103,39 +103,53 @@ def test_decode_launch_count_matches_the_path():
         assert lc(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap) == 2, w.name
 
 
-@pytest.mark.parametrize("name,adjacent", [("llava7b", False), ("llava7b", True), ("long-r32", True)])
-def test_step_from_host_buffers_equals_device_step(name, adjacent):
-    """wsvd_append_and_decode_host (x and q copied in from host memory, out
-    copied back) gives bit for bit what wsvd_append_and_decode gives on the
-    same values already on the device, on two steps in a row; with x and q
-    in one pinned buffer and in separate ones."""
+@pytest.mark.parametrize("name,memory", [("llava7b", "pinned"), ("llava7b", "pinned-one-buffer"),
+                                         ("llava7b", "pageable"), ("long-r32", "pinned"), ("ragged-int4", "pinned")])
+def test_step_from_host_buffers_equals_device_step(name, memory):
+    """wsvd_append_and_decode_host gives bit for bit what wsvd_append_and_decode
+    gives on the same values already on the device, on two steps in a row
+    whose host inputs differ (the second step's values are written into the
+    same host buffers).  Pinned buffers are read and written by the kernels in
+    place; pageable ones go through copies."""
     w, lens0 = CASES[name]
     lens0 = [min(n, w.L_cap - 2) for n in lens0]  # two steps in a row: room for two appended rows
     d, ai = _inputs(w, lens0, seed=33)
+    ai2 = WL.append_inputs(w, seed=34, steps=1)
+    q2_bits = WL.decode_inputs(w, seed=35, lens=np.asarray(lens0) + 1).q_bits
     qdt = torch.float16 if w.q_dtype == "fp16" else torch.bfloat16
-    xb = torch.from_numpy(ai.x_bits[0].view(np.int16).copy())
-    qb = torch.from_numpy(d.q_bits.view(np.int16).copy())
-    if adjacent:
+    xs = [torch.from_numpy(a.x_bits[0].view(np.int16).copy()) for a in (ai, ai2)]
+    qs = [torch.from_numpy(b.view(np.int16).copy()) for b in (d.q_bits, q2_bits)]
+    xb, qb = xs[0], qs[0]
+    if memory == "pinned-one-buffer":
         io = torch.cat([xb.reshape(-1), qb.reshape(-1)]).pin_memory()
         x_host = io[:xb.numel()].view(torch.bfloat16).view(xb.shape)
         q_host = io[xb.numel():].view(qdt).view(qb.shape)
-    else:
+    elif memory == "pinned":
         x_host = xb.view(torch.bfloat16).pin_memory()
         q_host = qb.view(qdt).pin_memory()
-    out_host = torch.full((w.B, w.H, w.Hd), float("nan"), dtype=torch.float32).pin_memory()
+    else:
+        x_host = xb.view(torch.bfloat16).clone()
+        q_host = qb.view(qdt).clone()
+    out_host = torch.full((w.B, w.H, w.Hd), float("nan"), dtype=torch.float32)
+    if memory != "pageable":
+        out_host = out_host.pin_memory()
+    assert x_host.is_pinned() == (memory != "pageable") and out_host.is_pinned() == (memory != "pageable")
     A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
     dv, hs = _device_state(d), _device_state(d)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     step = W.StepFromHost(x_host, A_k, A_v, hs["lens"], hs["lat_k"], hs["lat_v"], hs["sk"], hs["sv"], q_host, B_k,
                           B_v, out_host, bits=w.bits, hadamard_block=w.hadamard_block, err=err)
     for rep in range(2):
+        x_host.view(torch.int16).copy_(xs[rep].view(x_host.shape))
+        q_host.view(torch.int16).copy_(qs[rep].view(q_host.shape))
         out_dev = W.wsvd_append_and_decode(x_host.cuda(), A_k, A_v, dv["lens"], dv["lat_k"], dv["lat_v"], dv["sk"],
                                            dv["sv"], q_host.cuda(), B_k, B_v, bits=w.bits,
                                            hadamard_block=w.hadamard_block)
+        torch.cuda.synchronize()
         step()
         torch.cuda.synchronize()
         assert int(err.item()) == 0
-        assert torch.equal(out_host, out_dev.cpu()), (name, rep)
+        assert torch.equal(out_host, out_dev.cpu()), (name, memory, rep)
         for k in ("lat_k", "lat_v", "sk", "sv", "lens"):
-            assert torch.equal(hs[k], dv[k]), (name, k, rep)
+            assert torch.equal(hs[k], dv[k]), (name, memory, k, rep)
     assert np.array_equal(hs["lens"].cpu().numpy(), np.asarray(lens0) + 2)
