@@ -256,15 +256,18 @@ class WsvdStep:
         self.step()
         self.out_host.copy_(self.out, non_blocking=True)
 
-    def e2e_callable(self):
-        """The public call of one step from host buffers: the one-call
-        wsvd_append_and_decode_host (fp16 weights, appending workloads), else
-        the Python-level copies around the device call."""
+    def e2e_callable(self, graph=True):
+        """The public call of one step from host buffers: StepFromHost (fp16
+        weights, appending workloads) -- one launch of the captured step graph,
+        or with graph=False one wsvd_append_and_decode_host call -- else the
+        Python-level copies around the device call."""
         if self.has_append and not self.w8:
-            self.e2e_call_name = "wsvd_append_and_decode_host"
+            self.e2e_call_name = ("wsvd_step_host_graph_launch (wsvd_append_and_decode_host captured once)" if graph
+                                  else "wsvd_append_and_decode_host")
             return self.W.StepFromHost(self.x_host, self.A_k, self.A_v, self.lens, self.lat_k, self.lat_v,
                                        self.scale_k, self.scale_v, self.q_host, self.B_k, self.B_v, self.out_host,
-                                       bits=self.w.bits, hadamard_block=self.w.hadamard_block, err=self.err)
+                                       bits=self.w.bits, hadamard_block=self.w.hadamard_block, err=self.err,
+                                       graph=graph)
         self.e2e_call_name = "copies + " + ("wsvd_append_and_decode_w8" if self.has_append else "wsvd_decode_attention")
         return self.e2e_step
 
@@ -864,26 +867,40 @@ def main():
         # The length reset that lets every step append the same row is done
         # before the clock starts.
         n_e2e = max(50, min(args.steps, 500))
-        fn = st.e2e_callable()
         stream = torch.cuda.current_stream()
-        for _ in range(10):
-            st.reset()
-            fn()
-        torch.cuda.synchronize()
-        t_e2e = 0.0
-        for _ in range(n_e2e):
-            st.reset()
-            stream.synchronize()
-            t0 = time.perf_counter()
-            fn()
-            stream.synchronize()
-            t_e2e += time.perf_counter() - t0
+
+        def wall_per_step(fn):
+            for _ in range(10):
+                st.reset()
+                fn()
+            torch.cuda.synchronize()
+            total = 0.0
+            for _ in range(n_e2e):
+                st.reset()
+                stream.synchronize()
+                t0 = time.perf_counter()
+                fn()
+                stream.synchronize()
+                total += time.perf_counter() - t0
+            return total
+
+        fn = st.e2e_callable(graph=True)
+        t_e2e = wall_per_step(fn)
+        call_name = st.e2e_call_name
+        direct = None
+        if st.has_append and not w8:
+            fd = st.e2e_callable(graph=False)
+            direct = {"us_per_step": wall_per_step(fd) / n_e2e * 1e6, "call": st.e2e_call_name}
+        if hasattr(fn, "close"):
+            fn.close()
         h2d, d2h = st.e2e_bytes()
         extras["e2e"] = {"value": attended_tokens(w, st.lens_after) * n_e2e / t_e2e, "unit": UNIT,
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "us_per_step": t_e2e / n_e2e * 1e6,
                          "timing": "host wall clock around one library call + stream sync per step",
-                         "call": st.e2e_call_name}
+                         "call": call_name}
+        if direct is not None:
+            extras["e2e"]["direct_call"] = direct
         extras["comparisons_same_shape"] = time_comparisons(w, min(args.steps, 200), 5, flush)
         extras["comparisons_same_shape"]["wsvd_decode"] = {"us": per_dec * 1e6, "alg_bytes": dec_bytes,
                                                            "gbs": dec_bytes / per_dec / 1e9}

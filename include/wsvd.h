@@ -330,6 +330,36 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
                                 float softmax_scale, float* out_host, void* step_workspace,
                                 size_t step_workspace_bytes, int32_t* err, void* stream);
 
+/* ---------------------------------------------------------------- the host-buffer step as one graph
+ * The launches of one wsvd_append_and_decode_host call captured once into a
+ * CUDA graph, replayed per step with one cudaGraphLaunch (a serving loop's
+ * per-step cost is then one call, and the device runs the step's three
+ * kernels without waiting for the host between them).  The pages have no
+ * counterpart.
+ * wsvd_step_host_graph_create takes the arguments of
+ * wsvd_append_and_decode_host (minus the stream) and binds them: every
+ * pointer, the shapes and softmax_scale are fixed in the graph, so each launch
+ * reads the host buffers' current contents and the device state (seq_lens,
+ * the cache) as it is at that point in the stream.  It validates exactly as
+ * wsvd_append_and_decode_host does and runs nothing on the GPU.  It needs
+ * the in-place route (x_host, q_host, out_host pinned, mapped and aligned as
+ * described there) and returns WSVD_ERR_UNSUPPORTED otherwise.  On success
+ * *graph receives a handle; on failure it is set to NULL.
+ * wsvd_step_host_graph_launch queues one step on `stream` (WSVD_ERR_INVALID_ARG
+ * for a NULL handle, WSVD_ERR_CUDA if the launch fails).  Launches of one
+ * handle must not overlap on the GPU (they share the step workspace).
+ * wsvd_step_host_graph_destroy releases the handle (NULL is ignored); no
+ * launch of it may still be pending.                                          */
+typedef struct wsvd_step_graph wsvd_step_graph;
+int wsvd_step_host_graph_create(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                                const void* x_host, int x_dtype, const void* A_k, const void* A_v,
+                                int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                                const void* q_host, int q_dtype, const void* B_k, const void* B_v,
+                                float softmax_scale, float* out_host, void* step_workspace,
+                                size_t step_workspace_bytes, int32_t* err, wsvd_step_graph** graph);
+int wsvd_step_host_graph_launch(wsvd_step_graph* graph, void* stream);
+void wsvd_step_host_graph_destroy(wsvd_step_graph* graph);
+
 /* ---------------------------------------------------------------- int8 weights (W8)
  * The same three operations with the low-rank factors stored as int8 weights
  * (the "W8" of the method's W8A8 / W8A4 configurations, German §2.C): every

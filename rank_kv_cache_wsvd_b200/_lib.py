@@ -50,6 +50,10 @@ SIGNATURES = {
     "wsvd_step_host_workspace_size": (_c_size, [_c_int] * 5),
     "wsvd_append_and_decode_host": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                     + [_c_float, _p, _p, _c_size, _p, _p]),
+    "wsvd_step_host_graph_create": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
+                                    + [_c_float, _p, _p, _c_size, _p, _p]),
+    "wsvd_step_host_graph_launch": (_c_int, [_p, _p]),
+    "wsvd_step_host_graph_destroy": (None, [_p]),
     "wsvd_decode_attention_w8": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 8 + [_c_float, _p, _p, _c_size,
                                                                                            _p, _p]),
     "wsvd_latent_append_w8": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 9 + [_p, _c_size, _p, _p]),
@@ -341,11 +345,16 @@ class StepFromHost:
     x_host [B][E] and q_host [B][H][Hd] (16-bit) and out_host [B][H][Hd]
     fp32 are CPU tensors, ideally pinned; the device tensors (weights, cache,
     seq_lens) are bound as given.  After `__call__` the step is queued on the
-    stream given here; out_host is valid once that stream is synchronised.
-    The caller keeps every bound tensor alive and unchanged in shape."""
+    stream given here; out_host is valid once that stream is synchronised,
+    and x_host, q_host may be rewritten for the next step only after that.
+    With `graph` (the default when all three host buffers are pinned) the
+    step's launches are captured once into a CUDA graph
+    (wsvd_step_host_graph_create) and a call is one graph launch.  The caller
+    keeps every bound tensor alive and unchanged in shape."""
 
     def __init__(self, x_host, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q_host, B_k, B_v, out_host,
-                 bits: int, hadamard_block: int = 128, softmax_scale: float = 0.0, err=None, stream=None):
+                 bits: int, hadamard_block: int = 128, softmax_scale: float = 0.0, err=None, stream=None,
+                 graph=None):
         lib = load()
         B, E = x_host.shape
         H, _, r = A_k.shape
@@ -369,17 +378,50 @@ class StepFromHost:
         self._keep = (x_host, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, q_host, B_k, B_v, out_host, err)
         self.h2d_bytes = x_host.numel() * 2 + q_host.numel() * 2
         self.d2h_bytes = out_host.numel() * 4
+        self._lib = lib
         self._fn = lib.wsvd_append_and_decode_host
-        self._args = (B, H, Hd, E, r, bits, L_cap, hadamard_block, x_host.data_ptr(), _dtype_code(x_host),
-                      _ptr(A_k), _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k),
-                      _ptr(scale_v), q_host.data_ptr(), _dtype_code(q_host), _ptr(B_k), _ptr(B_v),
-                      float(softmax_scale), out_host.data_ptr(), _ptr(self.workspace), self.workspace.numel(),
-                      _ptr(err), _stream(stream))
+        args = (B, H, Hd, E, r, bits, L_cap, hadamard_block, x_host.data_ptr(), _dtype_code(x_host),
+                _ptr(A_k), _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k),
+                _ptr(scale_v), q_host.data_ptr(), _dtype_code(q_host), _ptr(B_k), _ptr(B_v),
+                float(softmax_scale), out_host.data_ptr(), _ptr(self.workspace), self.workspace.numel(),
+                _ptr(err))
+        self._args = args + (_stream(stream),)
+        self._graph = None
+        if graph is None:
+            graph = x_host.is_pinned() and q_host.is_pinned() and out_host.is_pinned()
+        if graph:
+            handle = ctypes.c_void_p()
+            st = lib.wsvd_step_host_graph_create(*args, ctypes.byref(handle))
+            _check(st, "wsvd_step_host_graph_create")
+            self._graph = handle
+            self._launch = lib.wsvd_step_host_graph_launch
+            self._gargs = (handle, _stream(stream))
+
+    @property
+    def uses_graph(self) -> bool:
+        return self._graph is not None
 
     def __call__(self) -> None:
+        if self._graph is not None:
+            st = self._launch(*self._gargs)
+            if st:
+                _check(st, "wsvd_step_host_graph_launch")
+            return
         st = self._fn(*self._args)
         if st:
             _check(st, "wsvd_append_and_decode_host")
+
+    def close(self) -> None:
+        """Releases the captured graph (no step of it may still be pending)."""
+        if self._graph is not None:
+            self._lib.wsvd_step_host_graph_destroy(self._graph)
+            self._graph = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ----------------------------------------------------------------------------- int8 weights

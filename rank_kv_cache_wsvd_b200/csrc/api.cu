@@ -1,8 +1,11 @@
 // C ABI of the library: host-side validation, split planning and launches.
 // No allocation, no synchronisation; every launch goes to the caller's stream.
+// (The captured host-buffer step is the one exception: creating it builds and
+// instantiates a CUDA graph, once.)
 #include <math.h>
 
 #include <algorithm>
+#include <new>
 
 #include "common.cuh"
 #include "wsvd_internal.h"
@@ -425,6 +428,67 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
   if (!in_place && cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return WSVD_ERR_CUDA;
   return WSVD_OK;
+}
+
+struct wsvd_step_graph {
+  cudaGraphExec_t exec;
+};
+
+int wsvd_step_host_graph_create(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
+                                const void* x_host, int x_dtype, const void* A_k, const void* A_v,
+                                int32_t* seq_lens, uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v,
+                                const void* q_host, int q_dtype, const void* B_k, const void* B_v,
+                                float softmax_scale, float* out_host, void* step_workspace,
+                                size_t step_workspace_bytes, int32_t* err, wsvd_step_graph** graph) {
+  if (!graph) return WSVD_ERR_INVALID_ARG;
+  *graph = nullptr;
+  // Only the in-place route can be captured (a copy from pageable memory cannot).
+  const size_t xbytes = (size_t)(B > 0 ? B : 0) * (E > 0 ? E : 0) * 2;
+  const size_t qbytes = (size_t)(B > 0 ? B : 0) * (H > 0 ? H : 0) * (Hd > 0 ? Hd : 0) * 2;
+  void* xm = x_host ? mapped_device_pointer(x_host) : nullptr;
+  void* qm = q_host ? mapped_device_pointer(q_host) : nullptr;
+  void* om = out_host ? mapped_device_pointer(out_host) : nullptr;
+  if (B > 0 && !(xm && qm && om && aligned16(xm) && aligned16(qm) && aligned16(om) && xbytes % 16 == 0 &&
+                 qbytes % 16 == 0))
+    return WSVD_ERR_UNSUPPORTED;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return WSVD_ERR_CUDA;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return WSVD_ERR_CUDA;
+  }
+  const int st = wsvd_append_and_decode_host(B, H, Hd, E, r, bits, L_cap, hadamard_block, x_host, x_dtype, A_k, A_v,
+                                             seq_lens, lat_k, lat_v, scale_k, scale_v, q_host, q_dtype, B_k, B_v,
+                                             softmax_scale, out_host, step_workspace, step_workspace_bytes, err, cs);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(cs, &g);
+  cudaStreamDestroy(cs);
+  if (st != WSVD_OK || ce != cudaSuccess || !g) {
+    if (g) cudaGraphDestroy(g);
+    (void)cudaGetLastError();
+    return st != WSVD_OK ? st : WSVD_ERR_CUDA;
+  }
+  cudaGraphExec_t ex = nullptr;
+  const cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
+  cudaGraphDestroy(g);
+  if (ie != cudaSuccess) return WSVD_ERR_CUDA;
+  *graph = new (std::nothrow) wsvd_step_graph{ex};
+  if (!*graph) {
+    cudaGraphExecDestroy(ex);
+    return WSVD_ERR_CUDA;
+  }
+  return WSVD_OK;
+}
+
+int wsvd_step_host_graph_launch(wsvd_step_graph* graph, void* stream) {
+  if (!graph) return WSVD_ERR_INVALID_ARG;
+  return cudaGraphLaunch(graph->exec, as_stream(stream)) == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
+}
+
+void wsvd_step_host_graph_destroy(wsvd_step_graph* graph) {
+  if (!graph) return;
+  cudaGraphExecDestroy(graph->exec);
+  delete graph;
 }
 
 int wsvd_append_and_decode_w8(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,

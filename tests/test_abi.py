@@ -185,6 +185,22 @@ def test_step_from_host_validation(lib):
     assert lib.wsvd_append_and_decode_host(*args(nbytes=need - 16)) == 4
 
 
+def test_step_graph_needs_pinned_buffers_and_a_handle(lib):
+    """The captured host-buffer step refuses host pointers that are not pinned
+    and mapped (WSVD_ERR_UNSUPPORTED, handle set to NULL) and a missing handle
+    slot; a NULL handle is refused by launch and ignored by destroy."""
+    B, H, Hd, E, r = 1, 4, 64, 256, 16
+    need = W.wsvd_step_host_workspace_size(B, H, Hd, E, r)
+    p = ctypes.c_void_p(16)
+    args = (B, H, Hd, E, r, 8, 64, 128, p, 1, p, p, p, p, p, p, p, p, 0, p, p, 0.0, p, p, need, None)
+    h = ctypes.c_void_p(1234)
+    assert lib.wsvd_step_host_graph_create(*args, ctypes.byref(h)) == 2
+    assert h.value is None
+    assert lib.wsvd_step_host_graph_create(*args, None) == 1
+    assert lib.wsvd_step_host_graph_launch(None, None) == 1
+    lib.wsvd_step_host_graph_destroy(None)
+
+
 def test_grouped_decode_workspace_and_validation(lib):
     """Grouped / multi-token decode: the workspace holds split partials (at most
     64 splits of 128-token tiles) of up to 16 queries per (sequence, latent

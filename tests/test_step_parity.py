@@ -104,13 +104,15 @@ def test_decode_launch_count_matches_the_path():
 
 
 @pytest.mark.parametrize("name,memory", [("llava7b", "pinned"), ("llava7b", "pinned-one-buffer"),
-                                         ("llava7b", "pageable"), ("long-r32", "pinned"), ("ragged-int4", "pinned")])
+                                         ("llava7b", "pinned-direct"), ("llava7b", "pageable"), ("long-r32", "pinned"),
+                                         ("ragged-int4", "pinned"), ("ragged-int4", "pinned-direct")])
 def test_step_from_host_buffers_equals_device_step(name, memory):
     """wsvd_append_and_decode_host gives bit for bit what wsvd_append_and_decode
     gives on the same values already on the device, on two steps in a row
     whose host inputs differ (the second step's values are written into the
     same host buffers).  Pinned buffers are read and written by the kernels in
-    place; pageable ones go through copies."""
+    place (replayed from one captured graph, or one direct call per step);
+    pageable ones go through copies."""
     w, lens0 = CASES[name]
     lens0 = [min(n, w.L_cap - 2) for n in lens0]  # two steps in a row: room for two appended rows
     d, ai = _inputs(w, lens0, seed=33)
@@ -124,7 +126,7 @@ def test_step_from_host_buffers_equals_device_step(name, memory):
         io = torch.cat([xb.reshape(-1), qb.reshape(-1)]).pin_memory()
         x_host = io[:xb.numel()].view(torch.bfloat16).view(xb.shape)
         q_host = io[xb.numel():].view(qdt).view(qb.shape)
-    elif memory == "pinned":
+    elif memory in ("pinned", "pinned-direct"):
         x_host = xb.view(torch.bfloat16).pin_memory()
         q_host = qb.view(qdt).pin_memory()
     else:
@@ -138,7 +140,9 @@ def test_step_from_host_buffers_equals_device_step(name, memory):
     dv, hs = _device_state(d), _device_state(d)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     step = W.StepFromHost(x_host, A_k, A_v, hs["lens"], hs["lat_k"], hs["lat_v"], hs["sk"], hs["sv"], q_host, B_k,
-                          B_v, out_host, bits=w.bits, hadamard_block=w.hadamard_block, err=err)
+                          B_v, out_host, bits=w.bits, hadamard_block=w.hadamard_block, err=err,
+                          graph=False if memory == "pinned-direct" else None)
+    assert step.uses_graph == (memory in ("pinned", "pinned-one-buffer"))
     for rep in range(2):
         x_host.view(torch.int16).copy_(xs[rep].view(x_host.shape))
         q_host.view(torch.int16).copy_(qs[rep].view(q_host.shape))
