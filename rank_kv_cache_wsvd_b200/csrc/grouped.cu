@@ -364,77 +364,73 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     }
   };
 
+  // The producer and MMA warps run their loops converged (every lane waits,
+  // one elected lane issues), so that copies and MMAs issue at full rate.
   if (warp == kGProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      const int gidx = (b * a.Hkv + hkv) * a.nqc + qc;
-      for (int i = 0; i < ntiles; ++i) {
-        if (i == min(S, ntiles)) {  // the ring is primed: now the planes (they come from the preceding grid)
-          griddep_wait();
-          mbar_arrive_expect_tx(pready, (uint32_t)C::QBLOCK);
-          bulk_g2s(smem + C::OFF_PL, a.qplanes + (size_t)gidx * C::QBLOCK, (uint32_t)C::PL, pready,
-                   l2_evict_last_policy());
-          bulk_g2s(smem + C::OFF_STEP, a.qplanes + (size_t)gidx * C::QBLOCK + C::PL, (uint32_t)(NQ * 4), pready,
-                   l2_evict_last_policy());
-        }
-        const int s = i % S;
-        if (i >= S) wait(&empty[s], (uint32_t)(((i / S) - 1) & 1));
-        const int r0 = t_begin + i * kGTok, n = min(kGTok, t_end - r0);
-        const uint32_t cb = (uint32_t)n * RB, sb = (uint32_t)((n + 7) & ~7) * 2u;
-        uint8_t* st = ring + (size_t)s * C::STAGE;
-        mbar_arrive_expect_tx(&full[s], 2 * cb + 2 * sb);
-        bulk_g2s(st, a.lat_k + (head_row + r0) * RB, cb, &full[s], pol);
-        bulk_g2s(st + kGTok * RB, a.lat_v + (head_row + r0) * RB, cb, &full[s], pol);
-        bulk_g2s(st + 2 * kGTok * RB, a.scale_k + head_row + r0, sb, &full[s], pol);
-        bulk_g2s(st + 2 * kGTok * RB + 2 * kGTok, a.scale_v + head_row + r0, sb, &full[s], pol);
-      }
-      if (ntiles <= S) {  // fewer tiles than stages: the planes follow the last tile
-        griddep_wait();
-        mbar_arrive_expect_tx(pready, (uint32_t)C::QBLOCK);
-        bulk_g2s(smem + C::OFF_PL, a.qplanes + (size_t)gidx * C::QBLOCK, (uint32_t)C::PL, pready,
-                 l2_evict_last_policy());
-        bulk_g2s(smem + C::OFF_STEP, a.qplanes + (size_t)gidx * C::QBLOCK + C::PL, (uint32_t)(NQ * 4), pready,
-                 l2_evict_last_policy());
-      }
-      // no copy left in flight: the last uses of every stage and the planes have landed
-      for (int i = max(0, ntiles - S); i < ntiles; ++i) wait(&full[i % S], (uint32_t)((i / S) & 1));
-      wait(pready, 0);
+    const uint64_t pol = l2_evict_first_policy();
+    const int gidx = (b * a.Hkv + hkv) * a.nqc + qc;
+    auto stage_planes = [&]() {  // the q' planes and steps (written by the preceding grid)
+      griddep_wait();
+      mbar_arrive_expect_tx_warp(pready, (uint32_t)C::QBLOCK);
+      bulk_g2s_warp(smem + C::OFF_PL, a.qplanes + (size_t)gidx * C::QBLOCK, (uint32_t)C::PL, pready,
+                    l2_evict_last_policy());
+      bulk_g2s_warp(smem + C::OFF_STEP, a.qplanes + (size_t)gidx * C::QBLOCK + C::PL, (uint32_t)(NQ * 4), pready,
+                    l2_evict_last_policy());
+    };
+    for (int i = 0; i < ntiles; ++i) {
+      if (i == min(S, ntiles)) stage_planes();  // the ring is primed: now the planes
+      const int s = i % S;
+      if (i >= S) wait(&empty[s], (uint32_t)(((i / S) - 1) & 1));
+      __syncwarp();
+      const int r0 = t_begin + i * kGTok, n = min(kGTok, t_end - r0);
+      const uint32_t cb = (uint32_t)n * RB, sb = (uint32_t)((n + 7) & ~7) * 2u;
+      uint8_t* st = ring + (size_t)s * C::STAGE;
+      mbar_arrive_expect_tx_warp(&full[s], 2 * cb + 2 * sb);
+      bulk_g2s_warp(st, a.lat_k + (head_row + r0) * RB, cb, &full[s], pol);
+      bulk_g2s_warp(st + kGTok * RB, a.lat_v + (head_row + r0) * RB, cb, &full[s], pol);
+      bulk_g2s_warp(st + 2 * kGTok * RB, a.scale_k + head_row + r0, sb, &full[s], pol);
+      bulk_g2s_warp(st + 2 * kGTok * RB + 2 * kGTok, a.scale_v + head_row + r0, sb, &full[s], pol);
     }
+    if (ntiles <= S) stage_planes();  // fewer tiles than stages: the planes follow the last tile
+    // no copy left in flight: the last uses of every stage and the planes have landed
+    for (int i = max(0, ntiles - S); i < ntiles; ++i) wait(&full[i % S], (uint32_t)((i / S) & 1));
+    wait(pready, 0);
+    __syncwarp();
   } else if (warp == kGMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = tc05::instr_desc(2, 1, 1, 0, 0, kGTok, NS);
-      constexpr uint32_t idesc_o = tc05::instr_desc(1, 0, 0, 1, 1, MO, NO);
-      auto scores = [&](int j) {
-        wait(&conv[j & 1], (uint32_t)((j >> 1) & 1));
-        tc05::fence_after_sync();
-        const uint32_t d = tmem + (uint32_t)((j & 1) * NS);
-        const uint32_t abase = s_ak + (uint32_t)((j & 1) * C::AK);
+    constexpr uint32_t idesc_s = tc05::instr_desc(2, 1, 1, 0, 0, kGTok, NS);
+    constexpr uint32_t idesc_o = tc05::instr_desc(1, 0, 0, 1, 1, MO, NO);
+    auto scores = [&](int j) {
+      wait(&conv[j & 1], (uint32_t)((j >> 1) & 1));
+      __syncwarp();
+      tc05::fence_after_sync();
+      const uint32_t d = tmem + (uint32_t)((j & 1) * NS);
+      const uint32_t abase = s_ak + (uint32_t)((j & 1) * C::AK);
 #pragma unroll
-        for (int kk = 0; kk < C::KS; ++kk)
-          tc05::mma_i8(d, tc05::smem_desc(abase + kk * 2 * C::LBO_A, C::LBO_A, 128),
-                       tc05::smem_desc(s_pl + kk * 2 * C::LBO_PL, C::LBO_PL, 128), idesc_s, kk > 0);
-        tc05::commit(&sready[j & 1]);
-      };
-      wait(pready, 0);  // the q' planes (score operand B) are staged
-      scores(0);
-      for (int i = 0; i < ntiles; ++i) {
-        if (i + 1 < ntiles) scores(i + 1);
-        const int vb = i % NV;
-        wait(&pfull[vb], (uint32_t)((i / NV) & 1));
-        tc05::fence_after_sync();
-        const uint32_t d = tmem + (uint32_t)(2 * NS + vb * NO);
-        const uint32_t vbase = s_vc + (uint32_t)(vb * C::VC), pbase = s_p + (uint32_t)(vb * C::PB);
+      for (int kk = 0; kk < C::KS; ++kk)
+        tc05::mma_i8_warp(d, tc05::smem_desc(abase + kk * 2 * C::LBO_A, C::LBO_A, 128),
+                          tc05::smem_desc(s_pl + kk * 2 * C::LBO_PL, C::LBO_PL, 128), idesc_s, kk > 0);
+      tc05::commit_warp(&sready[j & 1]);
+    };
+    wait(pready, 0);  // the q' planes (score operand B) are staged
+    scores(0);
+    for (int i = 0; i < ntiles; ++i) {
+      if (i + 1 < ntiles) scores(i + 1);
+      const int vb = i % NV;
+      wait(&pfull[vb], (uint32_t)((i / NV) & 1));
+      __syncwarp();
+      tc05::fence_after_sync();
+      const uint32_t d = tmem + (uint32_t)(2 * NS + vb * NO);
+      const uint32_t vbase = s_vc + (uint32_t)(vb * C::VC), pbase = s_p + (uint32_t)(vb * C::PB);
 #pragma unroll
-        for (int kk = 0; kk < kGTok / 16; ++kk)
-          tc05::mma_f16(d, tc05::smem_desc(vbase + kk * 2 * C::LBO_V, C::LBO_V, 128),
-                        tc05::smem_desc(pbase + kk * 2 * C::LBO_P, C::LBO_P, 128), idesc_o, kk > 0);
-        tc05::commit(&oready[vb]);
-      }
-      // every MMA has completed before the allocation is released
-      wait(&oready[(ntiles - 1) % NV], (uint32_t)(((ntiles - 1) / NV) & 1));
+      for (int kk = 0; kk < kGTok / 16; ++kk)
+        tc05::mma_f16_warp(d, tc05::smem_desc(vbase + kk * 2 * C::LBO_V, C::LBO_V, 128),
+                           tc05::smem_desc(pbase + kk * 2 * C::LBO_P, C::LBO_P, 128), idesc_o, kk > 0);
+      tc05::commit_warp(&oready[vb]);
     }
+    // every MMA has completed before the allocation is released
+    wait(&oready[(ntiles - 1) % NV], (uint32_t)(((ntiles - 1) / NV) & 1));
     __syncwarp();
   } else {
     // ------------------------------------------------------------ consumers

@@ -527,6 +527,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+// Warp-level forms: a converged warp calls them, one elected lane issues.
+__device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      "\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                                 uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
                                             uint64_t* bar) {
   asm volatile(
@@ -586,47 +606,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
   const int KT = a.KT;
 
-  if (warp == 4) {
-    if (lane == 0) {  // ---------------------------------------------- TMA producer
-      const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % S;
-        if (kt >= S) wait(&empty[s], (uint32_t)(((kt / S) - 1) & 1));
-        const uint32_t st = base + (uint32_t)(s * C::STAGE);
-        mbar_arrive_expect_tx(&full[s], C::STAGE);
-        tma_load_2d(st, &tm_xhi, kt * kTcBK, m0, &full[s]);
-        tma_load_2d(st + C::A_BYTES, &tm_xlo, kt * kTcBK, m0, &full[s]);
+  // The producer and MMA warps run their loops converged (every lane waits,
+  // one elected lane issues), so that the copies and MMAs issue at full rate.
+  if (warp == 4) {  // ------------------------------------------------------ TMA producer
+    const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      if (kt >= S) wait(&empty[s], (uint32_t)(((kt / S) - 1) & 1));
+      __syncwarp();
+      const uint32_t st = base + (uint32_t)(s * C::STAGE);
+      mbar_arrive_expect_tx_warp(&full[s], C::STAGE);
+      tma_load_2d_warp(st, &tm_xhi, kt * kTcBK, m0, &full[s]);
+      tma_load_2d_warp(st + C::A_BYTES, &tm_xlo, kt * kTcBK, m0, &full[s]);
 #pragma unroll
-        for (int g = 0; g < BN / NG; ++g) {
-          const int col = nl + g * NG;
-          tma_load_3d(st + 2 * C::A_BYTES + g * (kTcBK * NG * 2), wmap, col % R, kt * kTcBK, col / R, &full[s]);
-        }
+      for (int g = 0; g < BN / NG; ++g) {
+        const int col = nl + g * NG;
+        tma_load_3d_warp(st + 2 * C::A_BYTES + g * (kTcBK * NG * 2), wmap, col % R, kt * kTcBK, col / R, &full[s]);
       }
-      for (int kt = std::max(0, KT - S); kt < KT; ++kt) wait(&full[kt % S], (uint32_t)((kt / S) & 1));
     }
-  } else if (warp == 5) {
-    if (lane == 0) {  // ---------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = tc05::instr_desc(1, 0, 0, 0, 1, kTcBM, BN);
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % S;
-        wait(&full[s], (uint32_t)((kt / S) & 1));
-        const int hb = kt % NH;
-        if (kt >= NH) wait(&hfree[hb], (uint32_t)(((kt / NH) - 1) & 1));
-        tc05::fence_after_sync();
-        const uint32_t st = base + (uint32_t)(s * C::STAGE);
-        const uint32_t dh = tmem + (uint32_t)(hb * BN), dl = tmem + (uint32_t)(NH * BN);
+    for (int kt = std::max(0, KT - S); kt < KT; ++kt) wait(&full[kt % S], (uint32_t)((kt / S) & 1));
+    __syncwarp();
+  } else if (warp == 5) {  // ----------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = tc05::instr_desc(1, 0, 0, 0, 1, kTcBM, BN);
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      wait(&full[s], (uint32_t)((kt / S) & 1));
+      const int hb = kt % NH;
+      if (kt >= NH) wait(&hfree[hb], (uint32_t)(((kt / NH) - 1) & 1));
+      __syncwarp();
+      tc05::fence_after_sync();
+      const uint32_t st = base + (uint32_t)(s * C::STAGE);
+      const uint32_t dh = tmem + (uint32_t)(hb * BN), dl = tmem + (uint32_t)(NH * BN);
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 16; ++kk) {
-          const uint64_t bd = tc05::smem_desc_sw(st + 2 * C::A_BYTES + kk * 32 * NG, 128 * NG, 16 * NG, C::SW);
-          tc05::mma_f16(dh, tc05::smem_desc_sw(st + kk * 32, 16, 1024, 2), bd, idesc, kk > 0);
-          tc05::mma_f16(dl, tc05::smem_desc_sw(st + C::A_BYTES + kk * 32, 16, 1024, 2), bd, idesc, kt > 0 || kk > 0);
-        }
-        tc05::commit(&empty[s]);
-        tc05::commit(&hfull[hb]);
+      for (int kk = 0; kk < kTcBK / 16; ++kk) {
+        const uint64_t bd = tc05::smem_desc_sw(st + 2 * C::A_BYTES + kk * 32 * NG, 128 * NG, 16 * NG, C::SW);
+        tc05::mma_f16_warp(dh, tc05::smem_desc_sw(st + kk * 32, 16, 1024, 2), bd, idesc, kk > 0);
+        tc05::mma_f16_warp(dl, tc05::smem_desc_sw(st + C::A_BYTES + kk * 32, 16, 1024, 2), bd, idesc,
+                           kt > 0 || kk > 0);
       }
-      tc05::commit(done);
-      wait(done, 0);  // every MMA has completed before the allocation is released
+      tc05::commit_warp(&empty[s]);
+      tc05::commit_warp(&hfull[hb]);
     }
+    tc05::commit_warp(done);
+    wait(done, 0);  // every MMA has completed before the allocation is released
     __syncwarp();
   } else {  // -------------------------------------------------------- epilogue, thread = output row
     const int row = tid;
@@ -639,12 +661,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       wait(&hfull[hb], (uint32_t)((kt / NH) & 1));
       tc05::fence_after_sync();
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0), v);
+      for (int c0 = 0; c0 < BN; c0 += 64) {  // two loads in flight per wait
+        uint32_t va[32], vb[32];
+        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0), va);
+        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0 + 32), vb);
         tc05::wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
+        for (int c = 0; c < 32; ++c) {
+          tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(va[c]));
+          tot[c0 + 32 + c] = __fadd_rn(tot[c0 + 32 + c], __uint_as_float(vb[c]));
+        }
       }
       tc05::fence_before_sync();
       mbar_arrive(&hfree[hb]);
