@@ -200,6 +200,9 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   int* pos_sm = reinterpret_cast<int*>(smem + L.pos_off);  // leader: seq_lens[b] as read at launch
 
+  // The leader reads the row positions first so that their latency is hidden.
+  // No CTA writes seq_lens before every leader has counted itself done (below).
+  if (rank == 0 && tid < B) pos_sm[tid] = ld_relaxed_gpu(a.seq_lens + tid);
   if (tid == 0) {
     mbar_init(bar_red, 1);
     fence_mbar_init();
@@ -240,14 +243,6 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     griddep_wait();
     load_x();
   }
-  // Leader, thread 0: the row positions, loaded now (with the A rows and the
-  // x slice already in flight) and stored once the rotation below has waited
-  // for its own loads anyway.
-  int pl[16];
-  if (rank == 0 && tid == 0) {
-#pragma unroll
-    for (int b = 0; b < 16; ++b) pl[b] = b < B ? ld_relaxed_gpu(a.seq_lens + b) : 0;
-  }
 
   // 2. Rotate x into xs[b][e] (unnormalised; 1/sqrt(blk) is applied to c).
   if (fast) {
@@ -287,11 +282,6 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     for (int blk = warp; blk < nblk; blk += kAppendWarps)
       fwht_smem_warp(xs + (size_t)blk * a.blk, a.blk, lane);
   }
-  if (rank == 0 && tid == 0) {
-#pragma unroll
-    for (int b = 0; b < 16; ++b)
-      if (b < B) pos_sm[b] = pl[b];
-  }
   __syncthreads();
 
   // 3. + 4. Stream the A rows, reduce into this rank's slot of the leader.
@@ -309,13 +299,6 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
                    remote_bar, tid);
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
-  // Leader, thread 0: its completion count, ordered after its reads of the
-  // lengths by the release add.  The leader whose add completes the count
-  // advances seq_lens at its end (after an acquire fence); every leader read
-  // the lengths before its add, and no other CTA reads them.  The add's
-  // round trip overlaps the cluster reduction and the quantisation.
-  int prev_done = -1;
-  if (rank == 0 && tid == 0) prev_done = atom_add_release_gpu(a.counter, 1);
   // The A stream is done: a decode launched behind this kernel may now be
   // scheduled (it reads q and its B matrices, and waits for this grid to
   // complete before it touches the cache).  Triggering here rather than at
@@ -329,7 +312,21 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   if (a.cluster > 1) {
     if (tid == 0 && !mbar_wait_cluster_bounded(bar_red, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
   }
-  __syncthreads();  // slots landed
+  __syncthreads();  // slots landed; pos_sm visible
+  // 6. Completion counter, overlapping the quantisation below: this CTA's only
+  //    reads of seq_lens (at launch) are ordered before its add (acq_rel after
+  //    the CTA barrier), so the last leader may advance the lengths at once.
+  //    The row stores need no ordering with it: later kernels see both.
+  if (tid == kAppendThreads - 32) {
+    const int prev = atom_add_acq_rel_gpu(a.counter, 1);
+    if (prev == (int)gridDim.y - 1) {
+      for (int b = 0; b < B; ++b) {
+        const int pos = pos_sm[b];
+        if (pos >= 0 && pos < a.L_cap) st_relaxed_gpu(a.seq_lens + b, pos + 1);
+      }
+      st_relaxed_gpu(a.counter, 0);
+    }
+  }
   const int Q = (a.bits == 8) ? 127 : 7;
   const int RB = r * a.bits / 8;
   for (int b = warp; b < B; b += kAppendWarps) {
@@ -370,16 +367,6 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
       if (ok) (kv ? a.scale_v : a.scale_k)[row] = sh;
       else if (unit == 0) set_err(a.err, WSVD_DEVERR_CACHE_FULL);
     }
-  }
-  // 6. The leader that completed the count advances the lengths (the row
-  //    stores above need no ordering with it: later kernels see both).
-  if (tid == 0 && prev_done == (int)gridDim.y - 1) {
-    fence_acq_rel_gpu();
-    for (int b = 0; b < B; ++b) {
-      const int pos = pos_sm[b];
-      if (pos >= 0 && pos < a.L_cap) st_relaxed_gpu(a.seq_lens + b, pos + 1);
-    }
-    st_relaxed_gpu(a.counter, 0);
   }
 }
 

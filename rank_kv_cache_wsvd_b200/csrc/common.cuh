@@ -221,14 +221,6 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t* p, int v) {
   return old;
 }
 
-// Release-only add: this thread's earlier accesses are ordered before it.
-__device__ __forceinline__ int atom_add_release_gpu(int32_t* p, int v) {
-  int old;
-  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 __device__ __forceinline__ void set_err(int32_t* err, int32_t bits) {
   if (err) atomicOr(err, bits);
 }
