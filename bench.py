@@ -798,7 +798,9 @@ def main():
     # Per-kernel durations (the roofline's denominators): inside the step the
     # decode overlaps the append, so each kernel is timed here as its own
     # launch, events around it, under the same flush and host lead.
-    n_b = min(args.steps, 300)
+    # At least 100 samples: the two kernels are close at small shapes and the
+    # event clock ticks in about a microsecond.
+    n_b = min(max(args.steps, 100), 300)
     evs = []
     for _ in range(n_b):
         flush.zero_()
