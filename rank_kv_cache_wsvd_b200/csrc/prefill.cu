@@ -569,7 +569,7 @@ __device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap
 // Quantise one finished row of a column tile (whole heads of one side) into
 // the cache: x 1/p_m, then per head the append's fp32 decisions.
 template <int R, int BN>
-__device__ __forceinline__ void quantise_tile_row(const TcArgs& a, int m, int kv, int nl, float (&tot)[BN]) {
+__device__ __forceinline__ void quantise_tile_row(const TcArgs& a, int m, int kv, int nl, float* tot) {
   if (m >= a.M) return;
   const int b = m / a.T, t = m - b * a.T;
   const int pos = a.seq_lens[b];
@@ -577,38 +577,39 @@ __device__ __forceinline__ void quantise_tile_row(const TcArgs& a, int m, int kv
   const float ip = a.inv_p[m];
   const int Q = a.bits == 8 ? 127 : 7;
   constexpr int HEADS = BN / R;
-#pragma unroll
+#pragma unroll 1
   for (int hb = 0; hb < HEADS; ++hb) {
     const int h = (nl + hb * R) / R;
+    float* c = tot + hb * R;
     float amax = 0.f;
-#pragma unroll
+#pragma unroll 8
     for (int j = 0; j < R; ++j) {
-      tot[hb * R + j] *= ip;
-      amax = fmaxf(amax, fabsf(tot[hb * R + j]));
+      c[j] *= ip;
+      amax = fmaxf(amax, fabsf(c[j]));
     }
     const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
     const float sc = __half2float(sh);
     const size_t crow = ((size_t)b * a.H + h) * a.L_cap + pos + t;
     if (a.bits == 8) {
       uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * R);
-#pragma unroll
+#pragma unroll 2
       for (int j4 = 0; j4 < R / 4; ++j4) {
         uint32_t w = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 4 * j4 + k], sc)))) : 0;
+          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(c[4 * j4 + k], sc)))) : 0;
           w |= ((uint32_t)code & 0xFFu) << (8 * k);
         }
         dst[j4] = w;
       }
     } else {
       uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * (R / 2));
-#pragma unroll
+#pragma unroll 1
       for (int j8 = 0; j8 < R / 8; ++j8) {
         uint32_t w = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 8 * j8 + k], sc)))) : 0;
+          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(c[8 * j8 + k], sc)))) : 0;
           w |= ((uint32_t)code & 0xFu) << (4 * k);
         }
         dst[j8] = w;
@@ -616,6 +617,46 @@ __device__ __forceinline__ void quantise_tile_row(const TcArgs& a, int m, int kv
     }
     (kv ? a.scale_v : a.scale_k)[crow] = sh;
   }
+}
+
+// The end of one k segment of output tile `tile` for the epilogue thread of
+// `row` (all 128 epilogue threads call it together): quantise directly when
+// the segment is the whole k range; else store the partial row sums, count
+// the segment, and let the tile's last segment sum every partial in k order
+// and quantise.  Kept out of line so that the k-tile loop's registers hold
+// only the running sums.
+template <int R, int BN>
+__device__ __noinline__ void finish_segment(const TcArgs& a, float* tot, int tile, bool whole, int row, int cta,
+                                            int ctas, int* last_flag) {
+  const int mi = tile / a.ntn, ni = tile - mi * a.ntn;
+  const int m0 = mi * kTcBM, n0 = ni * BN, HR = a.H * R;
+  const int kv = n0 >= HR ? 1 : 0, nl = n0 - kv * HR;
+  if (whole) {
+    quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
+    return;
+  }
+  const long long tu0 = (long long)tile * a.KT;
+  const int cf = sk_cta_of(tu0, a.units, ctas), cl = sk_cta_of(tu0 + a.KT - 1, a.units, ctas);
+  float* slot = a.partials + (size_t)(tile + cta) * (BN * kTcBM);
+#pragma unroll 8
+  for (int c = 0; c < BN; ++c) slot[c * kTcBM + row] = tot[c];
+  __threadfence();  // publish before the count
+  named_barrier_sync(1, 128);
+  if (row == 0) *last_flag = atomicAdd(&a.counters[tile], 1) == cl - cf;
+  named_barrier_sync(1, 128);
+  if (*last_flag) {  // the tile's last segment: sum every segment's partial in k order
+    __threadfence();
+#pragma unroll 4
+    for (int c = 0; c < BN; ++c) {
+      float v = __ldcg(a.partials + (size_t)(tile + cf) * (BN * kTcBM) + c * kTcBM + row);
+      for (int q = cf + 1; q <= cl; ++q)
+        v = __fadd_rn(v, __ldcg(a.partials + (size_t)(tile + q) * (BN * kTcBM) + c * kTcBM + row));
+      tot[c] = v;
+    }
+    quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
+    if (row == 0) a.counters[tile] = 0;
+  }
+  named_barrier_sync(1, 128);  // last_flag is read before the next segment writes it
 }
 
 template <int R, int BN_>
@@ -644,9 +685,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int cta = blockIdx.x, ctas = gridDim.x;
   const long long u0 = sk_begin(cta, a.units, ctas), u1 = sk_begin(cta + 1, a.units, ctas);
   const int HR = a.H * R;
-  // tile of unit u: row tile, column start, K or V side, column within the side
-  auto tile_of = [&](long long u, int& tile, int& m0, int& kv, int& nl) {
-    tile = (int)(u / KT);
+  // row start, K or V side and column within the side of output tile `tile`
+  auto tile_at = [&](int tile, int& m0, int& kv, int& nl) {
     const int mi = tile / a.ntn, ni = tile - mi * a.ntn;
     m0 = mi * kTcBM;
     const int n0 = ni * BN;
@@ -687,11 +727,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // The producer and MMA warps run their loops converged (every lane waits,
   // one elected lane issues), so that the copies and MMAs issue at full rate.
   if (warp == 4) {  // ------------------------------------------------------ TMA producer
+    int tile = (int)(u0 / KT), kt = (int)(u0 - (long long)tile * KT), m0 = 0, kv = 0, nl = 0;
+    tile_at(tile, m0, kv, nl);
     for (int i = 0; i < n_units; ++i) {
-      const long long u = u0 + i;
-      int tile, m0, kv, nl;
-      tile_of(u, tile, m0, kv, nl);
-      const int kt = (int)(u - (long long)tile * KT);
+      if (i > 0 && ++kt == KT) {  // next unit: the k-tile, then the tile, advance without a division
+        kt = 0;
+        tile_at(++tile, m0, kv, nl);
+      }
       const int s = i % S;
       if (i >= S) wait(&empty[s], (uint32_t)(((i / S) - 1) & 1));
       __syncwarp();
@@ -710,10 +752,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else if (warp == 5) {  // ----------------------------------------------- MMA issuer
     constexpr uint32_t idesc = tc05::instr_desc(1, 0, 0, 0, 1, kTcBM, BN);
-    int seg = 0;  // segments started by this CTA
-    for (int i = 0; i < n_units; ++i) {
-      const long long u = u0 + i;
-      const bool first = i == 0 || u % KT == 0, last = i + 1 == n_units || (u + 1) % KT == 0;
+    int seg = 0;                                            // segments started by this CTA
+    int kt = (int)(u0 - (u0 / KT) * KT);                    // k-tile of the current unit
+    for (int i = 0; i < n_units; ++i, kt = (kt + 1 == KT) ? 0 : kt + 1) {
+      const bool first = i == 0 || kt == 0, last = i + 1 == n_units || kt + 1 == KT;
       const int s = i % S;
       wait(&full[s], (uint32_t)((i / S) & 1));
       const int hb = i % NH, lb = seg & 1;
@@ -747,25 +789,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
     for (int c = 0; c < BN; ++c) tot[c] = 0.f;
     auto add_cols = [&](uint32_t col0) {  // tot += tensor-memory columns col0 .. col0 + BN - 1, round to nearest
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 64) {  // two loads in flight per wait
+      if constexpr (BN == 64) {  // two loads in flight per wait
         uint32_t va[32], vb[32];
-        tc05::ld32(lane_base + col0 + (uint32_t)c0, va);
-        tc05::ld32(lane_base + col0 + (uint32_t)(c0 + 32), vb);
+        tc05::ld32(lane_base + col0, va);
+        tc05::ld32(lane_base + col0 + 32u, vb);
         tc05::wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(va[c]));
-          tot[c0 + 32 + c] = __fadd_rn(tot[c0 + 32 + c], __uint_as_float(vb[c]));
+          tot[c] = __fadd_rn(tot[c], __uint_as_float(va[c]));
+          tot[32 + c] = __fadd_rn(tot[32 + c], __uint_as_float(vb[c]));
+        }
+      } else {  // one load per wait: 128 running sums leave no registers for more
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tc05::ld32(lane_base + col0 + (uint32_t)c0, v);
+          tc05::wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
         }
       }
     };
     int seg = 0, kb = 0;
+    int tile = (int)(u0 / KT), kt = (int)(u0 - (long long)tile * KT);
     for (int i = 0; i < n_units; ++i) {
-      const long long u = u0 + i;
-      const int kt = (int)(u % KT);
+      if (i > 0 && ++kt == KT) {
+        kt = 0;
+        ++tile;
+      }
       if (i == 0 || kt == 0) kb = kt;
-      const bool last = i + 1 == n_units || (u + 1) % KT == 0;
+      const bool last = i + 1 == n_units || kt + 1 == KT;
       const int hb = i % NH;
       wait(&hfull[hb], (uint32_t)((i / NH) & 1));
       tc05::fence_after_sync();
@@ -781,33 +834,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc05::fence_before_sync();
       mbar_arrive(&lofree[lb]);
       ++seg;
-      int tile, m0, kv, nl;
-      tile_of(u, tile, m0, kv, nl);
-      if (kb == 0 && kt == KT - 1) {  // the whole k range: quantise directly
-        quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
-      } else {
-        const long long tu0 = (long long)tile * KT;
-        const int cf = sk_cta_of(tu0, a.units, ctas), cl = sk_cta_of(tu0 + KT - 1, a.units, ctas);
-        float* slot = a.partials + (size_t)(tile + cta) * (BN * kTcBM);
+      {
+        float spill[BN];  // the running sums stay in registers; only this copy goes out of line
 #pragma unroll
-        for (int c = 0; c < BN; ++c) slot[c * kTcBM + row] = tot[c];
-        __threadfence();  // publish before the count
-        named_barrier_sync(1, 128);
-        if (tid == 0) *last_flag = atomicAdd(&a.counters[tile], 1) == cl - cf;
-        named_barrier_sync(1, 128);
-        if (*last_flag) {  // the tile's last segment: sum every segment's partial in k order
-          __threadfence();
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            float v = __ldcg(a.partials + (size_t)(tile + cf) * (BN * kTcBM) + c * kTcBM + row);
-            for (int q = cf + 1; q <= cl; ++q)
-              v = __fadd_rn(v, __ldcg(a.partials + (size_t)(tile + q) * (BN * kTcBM) + c * kTcBM + row));
-            tot[c] = v;
-          }
-          quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
-          if (tid == 0) a.counters[tile] = 0;
-        }
-        named_barrier_sync(1, 128);  // last_flag is read before the next segment writes it
+        for (int c = 0; c < BN; ++c) spill[c] = tot[c];
+        finish_segment<R, BN>(a, spill, tile, kb == 0 && kt == KT - 1, row, cta, ctas, last_flag);
       }
 #pragma unroll
       for (int c = 0; c < BN; ++c) tot[c] = 0.f;
