@@ -329,7 +329,7 @@ def time_prefill(w: WL.Workload, T: int, steps: int, warmup: int, flush):
     sv = torch.zeros_like(sk)
     lens = torch.zeros(w.B, dtype=torch.int32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = W.workspace(W.wsvd_prefill_workspace_size(w.B, T, w.H, w.E, w.r))
+    ws = W.workspace(W.wsvd_prefill_workspace_size(w.B, T, w.E))
     call = lambda: W.wsvd_latent_prefill(x, A_k, A_v, lens, lk, lv, sk, sv, bits=w.bits,
                                          hadamard_block=w.hadamard_block, workspace_buf=ws, err=err)
     for _ in range(max(3, warmup)):

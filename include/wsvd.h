@@ -256,20 +256,12 @@ int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hada
  *   E                       multiple of 64, at most 16384.
  *   r                       8, 16, 32, 64 or 128.
  *   seq_lens   [B]          int32, read and advanced in place.
- *   workspace               at least wsvd_prefill_workspace_size(B, T, H, E, r)
- *                           bytes, ZERO before the first call (every call
- *                           leaves its counters zero again): the split rotated
- *                           activations, then (tensor-core path) one segment
- *                           counter per output tile and the partial row sums
- *                           of the tiles' k segments.  Calls that share it
- *                           must not overlap on the GPU.
+ *   workspace               at least wsvd_prefill_workspace_size(B, T, E)
+ *                           bytes (the split rotated activations; no zeroing
+ *                           needed).  Calls that share it must not overlap.
  * T = 0 (or B = 0) launches nothing.  Three launches otherwise (rotate,
- * GEMM + quantiser, length advance), all on `stream`.  The GEMM is split
- * stream-K over the device's SMs when H*r is a multiple of 64 and r is 16, 32,
- * 64 or 128: the (output tile, 64-wide k-tile) units are cut into one equal
- * range per CTA; a tile's k segments are summed in k order by the last of them
- * to finish (deterministic for a given device), then quantised.             */
-size_t wsvd_prefill_workspace_size(int B, int T, int H, int E, int r);
+ * GEMM + quantiser, length advance), all on `stream`.                       */
+size_t wsvd_prefill_workspace_size(int B, int T, int E);
 int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, int L_cap, int hadamard_block,
                         const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
                         uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, void* workspace,

@@ -39,7 +39,7 @@ SIGNATURES = {
                                                                                         _p, _p]),
     "wsvd_decode_attention_noalloc": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _p]),
     "wsvd_latent_append": (_c_int, [_c_int] * 7 + [_p, _c_int] + [_p] * 7 + [_p, _c_size, _p, _p]),
-    "wsvd_prefill_workspace_size": (_c_size, [_c_int] * 5),
+    "wsvd_prefill_workspace_size": (_c_size, [_c_int] * 3),
     "wsvd_latent_prefill": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_size, _p, _p]),
     "wsvd_append_and_decode": (_c_int, [_c_int] * 8 + [_p, _c_int, _p, _p] + [_p] * 5 + [_p, _c_int, _p, _p]
                                + [_c_float, _p, _p, _c_size, _p, _c_size, _p, _p]),
@@ -156,8 +156,8 @@ def wsvd_append_workspace_size() -> int:
     return load().wsvd_append_workspace_size()
 
 
-def wsvd_prefill_workspace_size(B, T, H, E, r) -> int:
-    return load().wsvd_prefill_workspace_size(B, T, H, E, r)
+def wsvd_prefill_workspace_size(B, T, E) -> int:
+    return load().wsvd_prefill_workspace_size(B, T, E)
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
@@ -577,7 +577,7 @@ def wsvd_latent_prefill(x, A_k, A_v, seq_lens, lat_k, lat_v, scale_k, scale_v, b
     _expect(scale_v, torch.float16, (B, H, L_cap), "scale_v")
     _expect(seq_lens, torch.int32, (B,), "seq_lens")
     if workspace_buf is None:
-        workspace_buf = workspace(lib.wsvd_prefill_workspace_size(B, T, H, E, r), x.device)
+        workspace_buf = workspace(lib.wsvd_prefill_workspace_size(B, T, E), x.device)
     st = lib.wsvd_latent_prefill(B, T, H, E, r, bits, L_cap, hadamard_block, _ptr(x), _dtype_code(x), _ptr(A_k),
                                  _ptr(A_v), _ptr(seq_lens), _ptr(lat_k), _ptr(lat_v), _ptr(scale_k), _ptr(scale_v),
                                  _ptr(workspace_buf), workspace_buf.numel(), _ptr(err), _stream(stream))

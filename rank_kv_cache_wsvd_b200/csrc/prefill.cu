@@ -499,44 +499,18 @@ struct TcCfg {
   static constexpr int A_BYTES = kTcBM * kTcBK * 2;
   static constexpr int W_BYTES = kTcBK * BN * 2;
   static constexpr int STAGE = 2 * A_BYTES + W_BYTES;
-  // Tensor memory: NH fresh accumulators for the hi k-tile sums (the MMA warp
-  // runs up to NH k-tiles ahead of the epilogue), then two lo accumulators
-  // (one per segment, alternating, so that a segment's lo sum is read while
-  // the next segment accumulates): all 512 columns.
-  static constexpr int NH = BN == 64 ? 6 : 2;
-  static constexpr int TCOLS = 512;
-  static constexpr int NBAR = 2 * kTcStages + 2 * NH + 4 + 1;
-  static constexpr int SMEM = kTcStages * STAGE + 1024 + NBAR * 8 + 64;
-  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle-atom alignment");
+  // NH fresh accumulators for the hi k-tile sums (the MMA warp runs up to NH
+  // k-tiles ahead of the epilogue), then the lo accumulator: all 512 columns.
+  static constexpr int NH = BN == 64 ? 6 : 3;
   static_assert(BN == 64 || BN == 128, "tile width");
   static_assert(R <= BN, "whole heads per tile");
-  static_assert((NH + 2) * BN == TCOLS, "tensor memory budget");
+  static constexpr int TCOLS = 512;
+  static constexpr int SMEM = kTcStages * STAGE + 1024 + 256;
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle-atom alignment");
 };
-
-// Stream-K schedule: the (tile, k-tile) units of the whole GEMM, tile-major,
-// are cut into gridDim.x equal contiguous ranges, one per CTA.  A CTA's range
-// crosses tile boundaries; each piece of it within one tile is a segment.  A
-// segment that covers its tile's whole k range quantises directly; otherwise
-// every segment stores its partial row sums and the last of the tile's
-// segments to finish sums them in k order (deterministic) and quantises.
-// Segment (tile, cta) owns partial slot tile + cta: along the unit order both
-// grow by at most one per segment, so the slots are distinct.
-__host__ __device__ inline long long sk_begin(long long cta, long long units, long long ctas) {
-  return cta * units / ctas;
-}
-__device__ inline int sk_cta_of(long long u, long long units, int ctas) {
-  int c = (int)(u * ctas / units);
-  while (c + 1 < ctas && sk_begin(c + 1, units, ctas) <= u) ++c;
-  while (c > 0 && sk_begin(c, units, ctas) > u) --c;
-  return c;
-}
 
 struct TcArgs {
   int M, T, H, bits, L_cap, KT;
-  int ntn;             // column tiles
-  long long units;     // tiles * KT
-  float* partials;     // [tiles + ctas][BN][128] partial row sums, column-major per slot
-  int32_t* counters;   // [tiles] finished segments per tile, zero between calls
   const float* inv_p;
   const int32_t* seq_lens;
   uint8_t* lat_k;
@@ -546,6 +520,13 @@ struct TcArgs {
   int32_t* err;
 };
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
 // Warp-level forms: a converged warp calls them, one elected lane issues.
 __device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
   asm volatile(
@@ -566,97 +547,13 @@ __device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
-// Quantise one finished row of a column tile (whole heads of one side) into
-// the cache: x 1/p_m, then per head the append's fp32 decisions.
-template <int R, int BN>
-__device__ __forceinline__ void quantise_tile_row(const TcArgs& a, int m, int kv, int nl, float* tot) {
-  if (m >= a.M) return;
-  const int b = m / a.T, t = m - b * a.T;
-  const int pos = a.seq_lens[b];
-  if (pos < 0 || (long long)pos + a.T > a.L_cap) return;  // refused (flagged by the advance kernel)
-  const float ip = a.inv_p[m];
-  const int Q = a.bits == 8 ? 127 : 7;
-  constexpr int HEADS = BN / R;
-#pragma unroll 1
-  for (int hb = 0; hb < HEADS; ++hb) {
-    const int h = (nl + hb * R) / R;
-    float* c = tot + hb * R;
-    float amax = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < R; ++j) {
-      c[j] *= ip;
-      amax = fmaxf(amax, fabsf(c[j]));
-    }
-    const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
-    const float sc = __half2float(sh);
-    const size_t crow = ((size_t)b * a.H + h) * a.L_cap + pos + t;
-    if (a.bits == 8) {
-      uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * R);
-#pragma unroll 2
-      for (int j4 = 0; j4 < R / 4; ++j4) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(c[4 * j4 + k], sc)))) : 0;
-          w |= ((uint32_t)code & 0xFFu) << (8 * k);
-        }
-        dst[j4] = w;
-      }
-    } else {
-      uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * (R / 2));
-#pragma unroll 1
-      for (int j8 = 0; j8 < R / 8; ++j8) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(c[8 * j8 + k], sc)))) : 0;
-          w |= ((uint32_t)code & 0xFu) << (4 * k);
-        }
-        dst[j8] = w;
-      }
-    }
-    (kv ? a.scale_v : a.scale_k)[crow] = sh;
-  }
-}
-
-// The end of one k segment of output tile `tile` for the epilogue thread of
-// `row` (all 128 epilogue threads call it together): quantise directly when
-// the segment is the whole k range; else store the partial row sums, count
-// the segment, and let the tile's last segment sum every partial in k order
-// and quantise.  Kept out of line so that the k-tile loop's registers hold
-// only the running sums.
-template <int R, int BN>
-__device__ __noinline__ void finish_segment(const TcArgs& a, float* tot, int tile, bool whole, int row, int cta,
-                                            int ctas, int* last_flag) {
-  const int mi = tile / a.ntn, ni = tile - mi * a.ntn;
-  const int m0 = mi * kTcBM, n0 = ni * BN, HR = a.H * R;
-  const int kv = n0 >= HR ? 1 : 0, nl = n0 - kv * HR;
-  if (whole) {
-    quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
-    return;
-  }
-  const long long tu0 = (long long)tile * a.KT;
-  const int cf = sk_cta_of(tu0, a.units, ctas), cl = sk_cta_of(tu0 + a.KT - 1, a.units, ctas);
-  float* slot = a.partials + (size_t)(tile + cta) * (BN * kTcBM);
-#pragma unroll 8
-  for (int c = 0; c < BN; ++c) slot[c * kTcBM + row] = tot[c];
-  __threadfence();  // publish before the count
-  named_barrier_sync(1, 128);
-  if (row == 0) *last_flag = atomicAdd(&a.counters[tile], 1) == cl - cf;
-  named_barrier_sync(1, 128);
-  if (*last_flag) {  // the tile's last segment: sum every segment's partial in k order
-    __threadfence();
-#pragma unroll 4
-    for (int c = 0; c < BN; ++c) {
-      float v = __ldcg(a.partials + (size_t)(tile + cf) * (BN * kTcBM) + c * kTcBM + row);
-      for (int q = cf + 1; q <= cl; ++q)
-        v = __fadd_rn(v, __ldcg(a.partials + (size_t)(tile + q) * (BN * kTcBM) + c * kTcBM + row));
-      tot[c] = v;
-    }
-    quantise_tile_row<R, BN>(a, m0 + row, kv, nl, tot);
-    if (row == 0) a.counters[tile] = 0;
-  }
-  named_barrier_sync(1, 128);  // last_flag is read before the next segment writes it
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
 }
 
 template <int R, int BN_>
@@ -665,34 +562,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
                       const TcArgs a) {
   using C = TcCfg<R, BN_>;
-  constexpr int BN = C::BN, NG = C::NG, S = kTcStages, NH = C::NH;
+  constexpr int BN = C::BN, NG = C::NG, S = kTcStages;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
   uint8_t* smem = smem_raw + (base - raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::STAGE);
   uint64_t* empty = full + S;
+  constexpr int NH = C::NH;
   uint64_t* hfull = empty + S;   // [NH] a k-tile's hi sum is in tensor memory
   uint64_t* hfree = hfull + NH;  // [NH] the epilogue has read it (128 arrivals)
-  uint64_t* lodone = hfree + NH; // [2] a segment's lo sum is complete
-  uint64_t* lofree = lodone + 2; // [2] the epilogue has read it (128 arrivals)
-  uint64_t* done = lofree + 2;   // every MMA of the CTA has completed
+  uint64_t* done = hfree + NH;   // every MMA of the tile has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int KT = a.KT;
-  const int cta = blockIdx.x, ctas = gridDim.x;
-  const long long u0 = sk_begin(cta, a.units, ctas), u1 = sk_begin(cta + 1, a.units, ctas);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.y * BN;
   const int HR = a.H * R;
-  // row start, K or V side and column within the side of output tile `tile`
-  auto tile_at = [&](int tile, int& m0, int& kv, int& nl) {
-    const int mi = tile / a.ntn, ni = tile - mi * a.ntn;
-    m0 = mi * kTcBM;
-    const int n0 = ni * BN;
-    kv = n0 >= HR ? 1 : 0;
-    nl = n0 - kv * HR;
-  };
+  const int kv = n0 >= HR ? 1 : 0, nl = n0 - kv * HR;  // tile columns within the K or the V side
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
@@ -701,10 +587,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = 0; i < NH; ++i) {
       mbar_init(&hfull[i], 1);
       mbar_init(&hfree[i], 128);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&lodone[i], 1);
-      mbar_init(&lofree[i], 128);
     }
     mbar_init(done, 1);
     fence_mbar_init();
@@ -722,22 +604,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       timed_out = true;
     }
   };
-  const int n_units = (int)(u1 - u0);
+  const int KT = a.KT;
 
   // The producer and MMA warps run their loops converged (every lane waits,
   // one elected lane issues), so that the copies and MMAs issue at full rate.
   if (warp == 4) {  // ------------------------------------------------------ TMA producer
-    int tile = (int)(u0 / KT), kt = (int)(u0 - (long long)tile * KT), m0 = 0, kv = 0, nl = 0;
-    tile_at(tile, m0, kv, nl);
-    for (int i = 0; i < n_units; ++i) {
-      if (i > 0 && ++kt == KT) {  // next unit: the k-tile, then the tile, advance without a division
-        kt = 0;
-        tile_at(++tile, m0, kv, nl);
-      }
-      const int s = i % S;
-      if (i >= S) wait(&empty[s], (uint32_t)(((i / S) - 1) & 1));
+    const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      if (kt >= S) wait(&empty[s], (uint32_t)(((kt / S) - 1) & 1));
       __syncwarp();
-      const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
       const uint32_t st = base + (uint32_t)(s * C::STAGE);
       mbar_arrive_expect_tx_warp(&full[s], C::STAGE);
       tma_load_2d_warp(st, &tm_xhi, kt * kTcBK, m0, &full[s]);
@@ -748,36 +624,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_load_3d_warp(st + 2 * C::A_BYTES + g * (kTcBK * NG * 2), wmap, col % R, kt * kTcBK, col / R, &full[s]);
       }
     }
-    for (int i = max(0, n_units - S); i < n_units; ++i) wait(&full[i % S], (uint32_t)((i / S) & 1));
+    for (int kt = std::max(0, KT - S); kt < KT; ++kt) wait(&full[kt % S], (uint32_t)((kt / S) & 1));
     __syncwarp();
   } else if (warp == 5) {  // ----------------------------------------------- MMA issuer
     constexpr uint32_t idesc = tc05::instr_desc(1, 0, 0, 0, 1, kTcBM, BN);
-    int seg = 0;                                            // segments started by this CTA
-    int kt = (int)(u0 - (u0 / KT) * KT);                    // k-tile of the current unit
-    for (int i = 0; i < n_units; ++i, kt = (kt + 1 == KT) ? 0 : kt + 1) {
-      const bool first = i == 0 || kt == 0, last = i + 1 == n_units || kt + 1 == KT;
-      const int s = i % S;
-      wait(&full[s], (uint32_t)((i / S) & 1));
-      const int hb = i % NH, lb = seg & 1;
-      if (i >= NH) wait(&hfree[hb], (uint32_t)(((i / NH) - 1) & 1));
-      if (first && seg >= 2) wait(&lofree[lb], (uint32_t)(((seg >> 1) - 1) & 1));
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      wait(&full[s], (uint32_t)((kt / S) & 1));
+      const int hb = kt % NH;
+      if (kt >= NH) wait(&hfree[hb], (uint32_t)(((kt / NH) - 1) & 1));
       __syncwarp();
       tc05::fence_after_sync();
       const uint32_t st = base + (uint32_t)(s * C::STAGE);
-      const uint32_t dh = tmem + (uint32_t)(hb * BN), dl = tmem + (uint32_t)((NH + lb) * BN);
+      const uint32_t dh = tmem + (uint32_t)(hb * BN), dl = tmem + (uint32_t)(NH * BN);
 #pragma unroll
       for (int kk = 0; kk < kTcBK / 16; ++kk) {
         const uint64_t bd = tc05::smem_desc_sw(st + 2 * C::A_BYTES + kk * 32 * NG, 128 * NG, 16 * NG, C::SW);
         tc05::mma_f16_warp(dh, tc05::smem_desc_sw(st + kk * 32, 16, 1024, 2), bd, idesc, kk > 0);
         tc05::mma_f16_warp(dl, tc05::smem_desc_sw(st + C::A_BYTES + kk * 32, 16, 1024, 2), bd, idesc,
-                           !first || kk > 0);
+                           kt > 0 || kk > 0);
       }
       tc05::commit_warp(&empty[s]);
       tc05::commit_warp(&hfull[hb]);
-      if (last) {
-        tc05::commit_warp(&lodone[lb]);
-        ++seg;
-      }
     }
     tc05::commit_warp(done);
     wait(done, 0);  // every MMA has completed before the allocation is released
@@ -788,60 +656,84 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float tot[BN];
 #pragma unroll
     for (int c = 0; c < BN; ++c) tot[c] = 0.f;
-    auto add_cols = [&](uint32_t col0) {  // tot += tensor-memory columns col0 .. col0 + BN - 1, round to nearest
-      if constexpr (BN == 64) {  // two loads in flight per wait
+    for (int kt = 0; kt < KT; ++kt) {
+      const int hb = kt % NH;
+      wait(&hfull[hb], (uint32_t)((kt / NH) & 1));
+      tc05::fence_after_sync();
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 64) {  // two loads in flight per wait
         uint32_t va[32], vb[32];
-        tc05::ld32(lane_base + col0, va);
-        tc05::ld32(lane_base + col0 + 32u, vb);
+        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0), va);
+        tc05::ld32(lane_base + (uint32_t)(hb * BN + c0 + 32), vb);
         tc05::wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          tot[c] = __fadd_rn(tot[c], __uint_as_float(va[c]));
-          tot[32 + c] = __fadd_rn(tot[32 + c], __uint_as_float(vb[c]));
-        }
-      } else {  // one load per wait: 128 running sums leave no registers for more
-#pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t v[32];
-          tc05::ld32(lane_base + col0 + (uint32_t)c0, v);
-          tc05::wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
+          tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(va[c]));
+          tot[c0 + 32 + c] = __fadd_rn(tot[c0 + 32 + c], __uint_as_float(vb[c]));
         }
       }
-    };
-    int seg = 0, kb = 0;
-    int tile = (int)(u0 / KT), kt = (int)(u0 - (long long)tile * KT);
-    for (int i = 0; i < n_units; ++i) {
-      if (i > 0 && ++kt == KT) {
-        kt = 0;
-        ++tile;
-      }
-      if (i == 0 || kt == 0) kb = kt;
-      const bool last = i + 1 == n_units || kt + 1 == KT;
-      const int hb = i % NH;
-      wait(&hfull[hb], (uint32_t)((i / NH) & 1));
-      tc05::fence_after_sync();
-      add_cols((uint32_t)(hb * BN));
       tc05::fence_before_sync();
       mbar_arrive(&hfree[hb]);
-      if (!last) continue;
-      // ---- end of a segment: its lo sum, then its row sums are complete
-      const int lb = seg & 1;
-      wait(&lodone[lb], (uint32_t)((seg >> 1) & 1));
-      tc05::fence_after_sync();
-      add_cols((uint32_t)((NH + lb) * BN));
-      tc05::fence_before_sync();
-      mbar_arrive(&lofree[lb]);
-      ++seg;
-      {
-        float spill[BN];  // the running sums stay in registers; only this copy goes out of line
+    }
+    wait(done, 0);
+    tc05::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < BN; ++c) spill[c] = tot[c];
-        finish_segment<R, BN>(a, spill, tile, kb == 0 && kt == KT - 1, row, cta, ctas, last_flag);
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t v[32];
+      tc05::ld32(lane_base + (uint32_t)(NH * BN + c0), v);
+      tc05::wait_ld();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) tot[c0 + c] = __fadd_rn(tot[c0 + c], __uint_as_float(v[c]));
+    }
+    tc05::fence_before_sync();
+    const int m = m0 + row;
+    if (m < a.M) {
+      const int b = m / a.T, t = m - b * a.T;
+      const int pos = a.seq_lens[b];
+      if (pos >= 0 && (long long)pos + a.T <= a.L_cap) {  // else refused (flagged by the advance kernel)
+        const float ip = a.inv_p[m];
+        const int Q = a.bits == 8 ? 127 : 7;
+        constexpr int HEADS = BN / R < 1 ? 1 : BN / R;
+#pragma unroll
+        for (int hb = 0; hb < HEADS; ++hb) {
+          const int h = (nl + hb * R) / R;
+          float amax = 0.f;
+#pragma unroll
+          for (int j = 0; j < R; ++j) {
+            tot[hb * R + j] *= ip;
+            amax = fmaxf(amax, fabsf(tot[hb * R + j]));
+          }
+          const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
+          const float sc = __half2float(sh);
+          const size_t crow = ((size_t)b * a.H + h) * a.L_cap + pos + t;
+          if (a.bits == 8) {
+            uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * R);
+#pragma unroll
+            for (int j4 = 0; j4 < R / 4; ++j4) {
+              uint32_t w = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 4 * j4 + k], sc)))) : 0;
+                w |= ((uint32_t)code & 0xFFu) << (8 * k);
+              }
+              dst[j4] = w;
+            }
+          } else {
+            uint32_t* dst = reinterpret_cast<uint32_t*>((kv ? a.lat_v : a.lat_k) + crow * (R / 2));
+#pragma unroll
+            for (int j8 = 0; j8 < R / 8; ++j8) {
+              uint32_t w = 0;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(tot[hb * R + 8 * j8 + k], sc)))) : 0;
+                w |= ((uint32_t)code & 0xFu) << (4 * k);
+              }
+              dst[j8] = w;
+            }
+          }
+          (kv ? a.scale_v : a.scale_k)[crow] = sh;
+        }
       }
-#pragma unroll
-      for (int c = 0; c < BN; ++c) tot[c] = 0.f;
     }
   }
   tc05::fence_before_sync();
@@ -898,18 +790,8 @@ bool encode_weight_map(CUtensorMap* tm, const void* base, int H, int E, int r, i
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kMaxStreamCtas = 256;  // stream-K grid cap (partial slots are sized for it)
-constexpr int kMinUnitsPerCta = 8;   // at least this many k-tiles per CTA (so no CTA's range is empty)
-
-// Stream-K grid: one CTA per SM, fewer when the GEMM has few k-tile units.
-inline int stream_ctas(long long units, int sms) {
-  long long c = std::min<long long>(std::min(sms, kMaxStreamCtas), units / kMinUnitsPerCta);
-  return (int)std::max<long long>(1, c);
-}
-
 template <int R, int BN>
-cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, float* partials, int32_t* counters,
-                      int32_t* err, cudaStream_t s) {
+cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, int32_t* err, cudaStream_t s) {
   using C = TcCfg<R, BN>;
   CUtensorMap mh, ml, mk, mv;
   if (!encode_act_map(&mh, pa.xhi, pa.M, pa.E) || !encode_act_map(&ml, pa.xlo, pa.M, pa.E) ||
@@ -918,48 +800,27 @@ cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, f
   cudaError_t e =
       cudaFuncSetAttribute(prefill_tc_kernel<R, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return cudaErrorInvalidValue;
   TcArgs ta{};
   ta.M = pa.M; ta.T = pa.T; ta.H = pa.H; ta.bits = pa.bits; ta.L_cap = pa.L_cap; ta.KT = pa.E / kTcBK;
-  ta.ntn = pa.N / BN;
-  const long long tiles = (long long)((pa.M + kTcBM - 1) / kTcBM) * ta.ntn;
-  ta.units = tiles * ta.KT;
-  ta.partials = partials; ta.counters = counters;
   ta.inv_p = pa.inv_p; ta.seq_lens = pa.seq_lens;
   ta.lat_k = pa.lat_k; ta.lat_v = pa.lat_v; ta.scale_k = pa.scale_k; ta.scale_v = pa.scale_v; ta.err = err;
-  const int ctas = stream_ctas(ta.units, sms);
+  const dim3 grid((unsigned)((pa.M + kTcBM - 1) / kTcBM), (unsigned)(pa.N / C::BN));
   (void)cudaGetLastError();
-  prefill_tc_kernel<R, BN><<<ctas, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
+  prefill_tc_kernel<R, BN><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
   return cudaGetLastError();
 }
 
-// Output tile width of the tcgen05 path: 128 columns when the tiles hold
-// whole heads of one side (every tile re-reads its activation rows from L2,
-// so wider tiles halve that traffic), else 64 (r <= 64), or 0 when the path
-// does not apply (the mma.sync GEMM runs instead).
-int tc_tile_width(int H, int r) {
+// Output tile width of the tcgen05 path: 128 columns when the tiles hold whole
+// heads of one side and there are enough of them to fill the device (every
+// tile re-reads the activation rows of its m-tile from L2, so wider tiles
+// halve that traffic); otherwise 64 (r <= 64), or 0 when the path does not
+// apply.
+int tc_tile_width(long long M, int H, int r) {
   if (r != 16 && r != 32 && r != 64 && r != 128) return 0;
-  const long long hr = (long long)H * r;
-  if (hr % 128 == 0) return 128;
+  const long long hr = (long long)H * r, mt = (M + kTcBM - 1) / kTcBM;
+  if (hr % 128 == 0 && (r == 128 || mt * (2 * hr / 128) >= 64)) return 128;
   if (r <= 64 && hr % 64 == 0) return 64;
   return 0;
-}
-
-// Workspace of the stream-K GEMM: per-tile segment counters, then the
-// partial slots (tiles + the largest grid), each 128 rows x BN fp32.
-struct TcScratch {
-  size_t counter_bytes, partial_bytes;
-};
-inline TcScratch tc_scratch(long long M, int H, int r) {
-  TcScratch t{0, 0};
-  const int bn = tc_tile_width(H, r);
-  if (!bn) return t;
-  const long long tiles = (M + kTcBM - 1) / kTcBM * (2LL * H * r / bn);
-  t.counter_bytes = (size_t)(tiles * 4 + 15) / 16 * 16;
-  t.partial_bytes = (size_t)(tiles + kMaxStreamCtas) * kTcBM * bn * 4;
-  return t;
 }
 
 // ------------------------------------------------------------------ 3. lengths
@@ -978,11 +839,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 }  // namespace wsvd
 
-extern "C" size_t wsvd_prefill_workspace_size(int B, int T, int H, int E, int r) {
-  if (B < 1 || T < 1 || H < 1 || E < 1 || r < 1) return 0;
+extern "C" size_t wsvd_prefill_workspace_size(int B, int T, int E) {
+  if (B < 1 || T < 1 || E < 1) return 0;
   const size_t M = (size_t)B * T;
-  const wsvd::TcScratch t = wsvd::tc_scratch((long long)M, H, r);
-  return 2 * wsvd::align16(M * E * 2) + wsvd::align16(M * 4) + t.counter_bytes + t.partial_bytes;
+  return 2 * wsvd::align16(M * E * 2) + wsvd::align16(M * 4);
 }
 
 extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, int L_cap, int hadamard_block,
@@ -1005,7 +865,7 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
   if (!aligned16(x) || !aligned16(A_k) || !aligned16(A_v) || !aligned16(lat_k) || !aligned16(lat_v) ||
       !aligned16(scale_k) || !aligned16(scale_v) || !aligned16(workspace))
     return WSVD_ERR_INVALID_ARG;
-  if (workspace_bytes < wsvd_prefill_workspace_size(B, T, H, E, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < wsvd_prefill_workspace_size(B, T, E)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
 
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t xbytes = align16((size_t)M * E * 2);
@@ -1014,9 +874,6 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
   a.xhi = reinterpret_cast<const __half*>(w);
   a.xlo = reinterpret_cast<const __half*>(w + xbytes);
   a.inv_p = reinterpret_cast<const float*>(w + 2 * xbytes);
-  const TcScratch tcs = tc_scratch(M, H, r);
-  int32_t* counters = reinterpret_cast<int32_t*>(w + 2 * xbytes + align16((size_t)M * 4));
-  float* partials = reinterpret_cast<float*>(w + 2 * xbytes + align16((size_t)M * 4) + tcs.counter_bytes);
   a.Ak = static_cast<const __half*>(A_k);
   a.Av = static_cast<const __half*>(A_v);
   a.seq_lens = seq_lens;
@@ -1050,21 +907,21 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
     prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo,
                                                                      winv);
   }
-  const int bn = tc_tile_width(H, r);
+  const int bn = tc_tile_width(M, H, r);
   if (bn) {
     cudaError_t e = cudaSuccess;
     if (bn == 128) {
       switch (r) {
-        case 16: e = launch_tc<16, 128>(a, A_k, A_v, partials, counters, err, s); break;
-        case 32: e = launch_tc<32, 128>(a, A_k, A_v, partials, counters, err, s); break;
-        case 64: e = launch_tc<64, 128>(a, A_k, A_v, partials, counters, err, s); break;
-        default: e = launch_tc<128, 128>(a, A_k, A_v, partials, counters, err, s); break;
+        case 16: e = launch_tc<16, 128>(a, A_k, A_v, err, s); break;
+        case 32: e = launch_tc<32, 128>(a, A_k, A_v, err, s); break;
+        case 64: e = launch_tc<64, 128>(a, A_k, A_v, err, s); break;
+        default: e = launch_tc<128, 128>(a, A_k, A_v, err, s); break;
       }
     } else {
       switch (r) {
-        case 16: e = launch_tc<16, 64>(a, A_k, A_v, partials, counters, err, s); break;
-        case 32: e = launch_tc<32, 64>(a, A_k, A_v, partials, counters, err, s); break;
-        default: e = launch_tc<64, 64>(a, A_k, A_v, partials, counters, err, s); break;
+        case 16: e = launch_tc<16, 64>(a, A_k, A_v, err, s); break;
+        case 32: e = launch_tc<32, 64>(a, A_k, A_v, err, s); break;
+        default: e = launch_tc<64, 64>(a, A_k, A_v, err, s); break;
       }
     }
     if (e != cudaSuccess) return WSVD_ERR_CUDA;

@@ -113,22 +113,13 @@ def test_decode_launch_count_rejects_bad_sizes(lib):
 
 def test_prefill_workspace_and_host_validation(lib):
     """The prefill scratch holds the split rotated activations (two fp16 copies
-    of the B x T x E block), one power-of-two scale per token row and, for the
-    stream-K tensor-core GEMM, one counter per 128-row x 128-column output
-    tile and partial slots for the tiles plus the largest grid (256 CTAs);
-    bad shapes are refused before anything is launched."""
+    of the B x T x E block) and one power-of-two scale per token row; bad
+    shapes are refused before anything is launched."""
     a16 = lambda v: (v + 15) // 16 * 16
-    tiles = 5 * (2 * 32 * 32 // 128)  # 576 rows -> 5 row tiles; 2048 columns -> 16 column tiles
-    assert W.wsvd_prefill_workspace_size(1, 576, 32, 4096, 32) == \
-        2 * a16(576 * 4096 * 2) + a16(576 * 4) + a16(tiles * 4) + (tiles + 256) * 128 * 128 * 4
-    # 64-wide tiles when H * r is a multiple of 64 only; none when the mma.sync GEMM runs (r = 8)
-    assert W.wsvd_prefill_workspace_size(2, 3, 2, 256, 32) == \
-        2 * a16(6 * 256 * 2) + a16(6 * 4) + a16(2 * 4) + (2 + 256) * 128 * 64 * 4
-    assert W.wsvd_prefill_workspace_size(2, 3, 3, 256, 32) == 2 * a16(6 * 256 * 2) + a16(6 * 4)  # H * r = 96
-    assert W.wsvd_prefill_workspace_size(2, 3, 3, 256, 8) == 2 * a16(6 * 256 * 2) + a16(6 * 4)
-    assert W.wsvd_prefill_workspace_size(0, 576, 32, 4096, 32) == 0
+    assert W.wsvd_prefill_workspace_size(1, 576, 4096) == 2 * a16(576 * 4096 * 2) + a16(576 * 4)
+    assert W.wsvd_prefill_workspace_size(0, 576, 4096) == 0
     p = ctypes.c_void_p(16)
-    ws = W.wsvd_prefill_workspace_size(2, 3, 4, 256, 16)
+    ws = W.wsvd_prefill_workspace_size(2, 3, 256)
     args = lambda B=2, T=3, H=4, E=256, r=16, bits=8, L=64, blk=128, ptr=p, nbytes=ws: (
         B, T, H, E, r, bits, L, blk, ptr, 1, p, p, p, p, p, p, p, p, nbytes, None, None)
     assert lib.wsvd_latent_prefill(*args(blk=96)) == 1            # block not a power of two

@@ -134,12 +134,11 @@ def test_wide_tiles_of_eight_small_heads():
     assert ties[0] <= code_bound and ties[1] <= scale_bound, (ties, code_bound, scale_bound)
 
 
-def test_stream_k_segments_cross_tiles_and_repeat_bit_for_bit():
-    """E 1152 (18 k-tiles of 64) over 12 output tiles: 216 k-tile units cut
-    into 27 CTA ranges of 8, so tiles are split into 2-3 k segments and CTAs
-    cross tile boundaries; partial sums are added in k order by the tile's
-    last segment.  A second call on the same inputs writes the same bytes."""
-    w = WL.Workload("pf-streamk", B=3, H=8, Hd=64, r=32, bits=8, L_cap=128, lens=0, E=1152)
+def test_odd_k_tile_count_repeats_bit_for_bit():
+    """E 1152 (18 k-tiles of 64, not a power of two) over 300 token rows (a
+    ragged third row tile) and 8 heads; a second call on the same inputs
+    writes the same bytes."""
+    w = WL.Workload("pf-oddk", B=3, H=8, Hd=64, r=32, bits=8, L_cap=128, lens=0, E=1152)
     ties, err, g, _ = _run(w, 100, [0, 5, 28], seed=31)
     assert err == 0 and list(g["lens"]) == [100, 105, 128]
     ties2, err2, g2, _ = _run(w, 100, [0, 5, 28], seed=31)
