@@ -42,9 +42,9 @@ namespace wsvd {
 namespace {
 
 constexpr int kGTok = 128;                    // tokens per tile (M of the score product)
-constexpr int kGConsumers = 128;              // four consumer warps
+constexpr int kGConsumers = 256;              // two consumer warpgroups (each half of the queries)
 constexpr int kGThreads = kGConsumers + 64;   // + producer warp + MMA warp
-constexpr int kGProducerWarp = 4, kGMmaWarp = 5;
+constexpr int kGProducerWarp = 8, kGMmaWarp = 9;
 constexpr int kMaxGroupedSplits = 64;
 constexpr int kQMax = 8355711;                // 127 (2^16 + 2^8 + 1): largest 3-digit signed value
 
@@ -183,6 +183,21 @@ __device__ __forceinline__ uint4 i4x8_to_h(uint32_t w) {
     o[k] = *reinterpret_cast<uint32_t*>(&h);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Stores N fp16 values (N / 2 packed pairs) at columns c0 .. c0 + N - 1 of a
+// row whose 8-column core-matrix chunks lie 128 bytes apart (c0 a multiple of N).
+template <int N>
+__device__ __forceinline__ void store_cols(uint32_t row, int c0, const uint32_t (&w)[N / 2]) {
+  const uint32_t a = row + (uint32_t)((c0 >> 3) * 128 + (c0 & 7) * 2);
+  if constexpr (N == 8) {
+    sts128(a, make_uint4(w[0], w[1], w[2], w[3]));
+  } else if constexpr (N == 4) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(w[0]), "r"(w[1]) : "memory");
+  } else {
+    static_assert(N == 2, "query counts per group: 2, 4 or 8");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(w[0]) : "memory");
+  }
 }
 
 // An integer below 2^22 in magnitude to fp32, exactly, on the FMA pipe:
@@ -434,43 +449,61 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     __syncwarp();
   } else {
     // ------------------------------------------------------------ consumers
-    const int t = tid;  // token slot of the tile, tensor-memory lane
+    // Two warpgroups: thread ct of 256 is token slot t = ct % 128 of the tile
+    // (tensor-memory lane t, warp quarter wq = warp % 4) for the queries of its
+    // group, q0 .. q0 + NQH - 1.  Group 0 widens the K codes of a staged tile,
+    // group 1 the V codes.
+    constexpr int NQH = NQ / 2;
+    const int ct = tid, grp = tid >> 7, t = tid & 127, wq = warp & 3, q0 = grp * NQH;
     wait(pready, 0);  // the group's steps (and planes) are staged
-    float step[NQ];
-    int nvis[NQ];  // rows visible to each query
+    float step[NQH];
+    int nvis[NQH];  // rows visible to each of this thread's queries
     const int vis_min = len - a.Tq + 1 + (qc * NQ) / a.G;  // the chunk's first query sees the fewest
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-      step[q] = stepv[q];
-      const int tq = (qc * NQ + q) / a.G;
-      nvis[q] = q < nq ? len - a.Tq + 1 + tq : 0;
+    for (int q = 0; q < NQH; ++q) {
+      const int qg = q0 + q;
+      step[q] = stepv[qg];
+      const int tq = (qc * NQ + qg) / a.G;
+      nvis[q] = qg < nq ? len - a.Tq + 1 + tq : 0;
     }
 
-    // Widen tile j of the ring into the operand buffers (slot j & 1).
+    // Widen tile j of the ring into the operand buffers (K codes: slot j & 1,
+    // group 0; V codes: slot j % NV, group 1).
     auto convert = [&](int j, float& sk, float& sv, int& pos) {
       const int s = j % S;
       wait(&full[s], (uint32_t)((j / S) & 1));
       const uint8_t* st = ring + (size_t)s * C::STAGE;
-      const uint32_t ak = s_ak + (uint32_t)((j & 1) * C::AK) + (uint32_t)((t >> 3) * 128 + (t & 7) * 16);
-      const uint32_t vc = s_vc + (uint32_t)((j % NV) * C::VC) + (uint32_t)((t >> 3) * C::LBO_V + (t & 7) * 16);
-      const uint32_t kr = smem_u32(st + t * RB), vr = smem_u32(st + kGTok * RB + t * RB);
+      if (grp == 0) {
+        const uint32_t ak = s_ak + (uint32_t)((j & 1) * C::AK) + (uint32_t)((t >> 3) * 128 + (t & 7) * 16);
+        const uint32_t kr = smem_u32(st + t * RB);
 #pragma unroll
-      for (int c = 0; c < RB / 16; ++c) {
-        const uint4 kv = lds128(kr + 16 * c), vv = lds128(vr + 16 * c);
-        if constexpr (CODEC == kCodecI8) {
-          sts128(ak + c * C::LBO_A, kv);
-          uint4 h0, h1;
-          i8x16_to_h(vv, h0, h1);
-          sts128(vc + (2 * c) * 128, h0);
-          sts128(vc + (2 * c + 1) * 128, h1);
-        } else {
-          const uint2 k0 = i4x8_to_i8(kv.x), k1 = i4x8_to_i8(kv.y), k2 = i4x8_to_i8(kv.z), k3 = i4x8_to_i8(kv.w);
-          sts128(ak + (2 * c) * C::LBO_A, make_uint4(k0.x, k0.y, k1.x, k1.y));
-          sts128(ak + (2 * c + 1) * C::LBO_A, make_uint4(k2.x, k2.y, k3.x, k3.y));
-          sts128(vc + (4 * c) * 128, i4x8_to_h(vv.x));
-          sts128(vc + (4 * c + 1) * 128, i4x8_to_h(vv.y));
-          sts128(vc + (4 * c + 2) * 128, i4x8_to_h(vv.z));
-          sts128(vc + (4 * c + 3) * 128, i4x8_to_h(vv.w));
+        for (int c = 0; c < RB / 16; ++c) {
+          const uint4 kv = lds128(kr + 16 * c);
+          if constexpr (CODEC == kCodecI8) {
+            sts128(ak + c * C::LBO_A, kv);
+          } else {
+            const uint2 k0 = i4x8_to_i8(kv.x), k1 = i4x8_to_i8(kv.y), k2 = i4x8_to_i8(kv.z), k3 = i4x8_to_i8(kv.w);
+            sts128(ak + (2 * c) * C::LBO_A, make_uint4(k0.x, k0.y, k1.x, k1.y));
+            sts128(ak + (2 * c + 1) * C::LBO_A, make_uint4(k2.x, k2.y, k3.x, k3.y));
+          }
+        }
+      } else {
+        const uint32_t vc = s_vc + (uint32_t)((j % NV) * C::VC) + (uint32_t)((t >> 3) * C::LBO_V + (t & 7) * 16);
+        const uint32_t vr = smem_u32(st + kGTok * RB + t * RB);
+#pragma unroll
+        for (int c = 0; c < RB / 16; ++c) {
+          const uint4 vv = lds128(vr + 16 * c);
+          if constexpr (CODEC == kCodecI8) {
+            uint4 h0, h1;
+            i8x16_to_h(vv, h0, h1);
+            sts128(vc + (2 * c) * 128, h0);
+            sts128(vc + (2 * c + 1) * 128, h1);
+          } else {
+            sts128(vc + (4 * c) * 128, i4x8_to_h(vv.x));
+            sts128(vc + (4 * c + 1) * 128, i4x8_to_h(vv.y));
+            sts128(vc + (4 * c + 2) * 128, i4x8_to_h(vv.z));
+            sts128(vc + (4 * c + 3) * 128, i4x8_to_h(vv.w));
+          }
         }
       }
       sk = lds_half_as_float(smem_u32(st + 2 * kGTok * RB + 2 * t));
@@ -484,16 +517,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 
     // Rows of the value accumulator this thread holds: M = 64 puts row j in
     // lane (j % 16) + 32 (j / 16), M = 128 row j in lane j.
-    const int orow = MO == 64 ? (lane < 16 ? warp * 16 + lane : -1) : t;
+    const int orow = MO == 64 ? (lane < 16 ? wq * 16 + lane : -1) : t;
     const bool holder = orow >= 0 && orow < R;
-    const bool warp_holds = MO == 64 ? warp * 16 < R : warp * 32 < R;
-    float l[NQ], acc[NQ];
+    const bool warp_holds = MO == 64 ? wq * 16 < R : wq * 32 < R;
+    const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+    float l[NQH], acc[NQH];
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
+    for (int q = 0; q < NQH; ++q) {
       l[q] = 0.f;
       acc[q] = 0.f;
     }
-    if (t < NQ) mrun[t] = kNegInf;  // ordered before its first use by the tile barriers
+    if (ct < NQ) mrun[ct] = kNegInf;  // ordered before its first use by the tile barriers
     // Fold tile j's value accumulator (scaled by 2^-e_j) into acc, rescaled
     // from the maxima before tile j to the maxima after it (the factor tile
     // j's softmax step broadcast: 0 while nothing was seen, 1 while a query
@@ -504,21 +538,25 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       tc05::fence_after_sync();
       if (warp_holds) {
         const int e = be[vb];
-        uint32_t v[(2 * NQ + 7) / 8 * 8];
-        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(2 * NS + vb * NO);
+        constexpr int NL = (NQH + 7) / 8 * 8;
+        uint32_t vh[NL], vl[NL];
+        const uint32_t ta = lane_base + (uint32_t)(2 * NS + vb * NO + q0);
 #pragma unroll
-        for (int c = 0; c < (2 * NQ + 7) / 8; ++c) {
+        for (int c = 0; c < NL / 8; ++c) {
           uint32_t w8[8];
           tc05::ld8(ta + 8 * c, w8);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[8 * c + k] = w8[k];
+          for (int k = 0; k < 8; ++k) vh[8 * c + k] = w8[k];
+          tc05::ld8(ta + NQ + 8 * c, w8);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) vl[8 * c + k] = w8[k];
         }
         tc05::wait_ld();
         const float unscale = __int_as_float((127 - e) << 23);
-        const float2* bj = bc + vb * NQ;
+        const float2* bj = bc + vb * NQ + q0;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const float d = (__uint_as_float(v[q]) + __uint_as_float(v[NQ + q])) * unscale;
+        for (int q = 0; q < NQH; ++q) {
+          const float d = (__uint_as_float(vh[q]) + __uint_as_float(vl[q])) * unscale;
           acc[q] = fmaf(acc[q], bj[q].y, d);
         }
       }
@@ -535,14 +573,15 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       float sk_n = 0.f, sv_n = 0.f;
       int pos_n = 0;
       if (i + 1 < ntiles) convert(i + 1, sk_n, sv_n, pos_n);
-      // scores of tile i
+      // scores of tile i: this thread's queries' three plane sums
       wait(&sready[i & 1], (uint32_t)((i >> 1) & 1));
       tc05::fence_after_sync();
-      uint32_t sv32[(3 * NQ + 7) / 8 * 8];
+      constexpr int NSV = (3 * NQH + 7) / 8 * 8;
+      uint32_t sv32[NSV];
       {
-        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((i & 1) * NS);
+        const uint32_t ta = lane_base + (uint32_t)((i & 1) * NS + 3 * q0);
 #pragma unroll
-        for (int c = 0; c < (3 * NQ + 7) / 8; ++c) {
+        for (int c = 0; c < NSV / 8; ++c) {
           uint32_t w8[8];
           tc05::ld8(ta + 8 * c, w8);
 #pragma unroll
@@ -550,41 +589,43 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         }
         tc05::wait_ld();
       }
-      float s[NQ];
+      float s[NQH];
       float* wm = wmax + (i & 1) * 4 * NQ;
       // Every row of a tile below the first query's horizon is visible to all
       // real queries: no per-query test there.
       if (nq == NQ && t_begin + (i + 1) * kGTok <= vis_min) {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) s[q] = plane_sum(sv32, q) * step[q] * sk_cur;
+        for (int q = 0; q < NQH; ++q) s[q] = plane_sum(sv32, q) * step[q] * sk_cur;
       } else {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) s[q] = pos_cur < nvis[q] ? plane_sum(sv32, q) * step[q] * sk_cur : kNegInf;
+        for (int q = 0; q < NQH; ++q) s[q] = pos_cur < nvis[q] ? plane_sum(sv32, q) * step[q] * sk_cur : kNegInf;
       }
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
+      for (int q = 0; q < NQH; ++q) {
         const float mx = warp_max_f32(s[q]);
-        if (lane == 0) wm[warp * NQ + q] = mx;
+        if (lane == 0) wm[wq * NQ + q0 + q] = mx;
       }
-      const uint32_t svb = pos_cur < len ? (uint32_t)__half_as_ushort(__float2half_rn(sv_cur)) : 0u;
-      const uint32_t svm = warp_max_u32(svb);
-      if (lane == 0) wsv[(i & 1) * 4 + warp] = svm;
+      if (grp == 0) {
+        const uint32_t svb = pos_cur < len ? (uint32_t)__half_as_ushort(__float2half_rn(sv_cur)) : 0u;
+        const uint32_t svm = warp_max_u32(svb);
+        if (lane == 0) wsv[(i & 1) * 4 + wq] = svm;
+      }
       tc05::fence_before_sync();
       named_barrier_sync(1, kGConsumers);
-      // One thread per query: the tile maximum over the four warps, the new
-      // running maximum and the rescale of the old one; one thread: the P~
+      // One thread per query: the tile maximum over the four warp quarters, the
+      // new running maximum and the rescale of the old one; one thread: the P~
       // scale 2^e that puts the largest s_V of the tile in [2^14, 2^15).
       float2* bi = bc + (i % NV) * NQ;
-      if (t < NQ) {
-        float tmax = wm[t];
+      if (ct < NQ) {
+        float tmax = wm[ct];
 #pragma unroll
-        for (int w = 1; w < 4; ++w) tmax = fmaxf(tmax, wm[w * NQ + t]);
-        const float mold = mrun[t], mnew = fmaxf(mold, tmax);
+        for (int w = 1; w < 4; ++w) tmax = fmaxf(tmax, wm[w * NQ + ct]);
+        const float mold = mrun[ct], mnew = fmaxf(mold, tmax);
         // .x: the maximum the tile's exponentials are taken against (0 while
         // the query sees nothing, so that -inf - .x stays -inf); .y: rescale
-        bi[t] = make_float2(mnew == kNegInf ? 0.f : mnew, mnew == kNegInf ? 1.f : ex2(mold - mnew));
-        mrun[t] = mnew;
-      } else if (t == kGConsumers - 1) {
+        bi[ct] = make_float2(mnew == kNegInf ? 0.f : mnew, mnew == kNegInf ? 1.f : ex2(mold - mnew));
+        mrun[ct] = mnew;
+      } else if (ct == kGConsumers - 1) {
         uint32_t svmax = 0;
 #pragma unroll
         for (int w = 0; w < 4; ++w) svmax = max(svmax, wsv[(i & 1) * 4 + w]);
@@ -594,12 +635,10 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
       named_barrier_sync(1, kGConsumers);
       const int e = be[i % NV];
       const float svs = (pos_cur < len) ? sv_cur * __int_as_float((127 + e) << 23) : 0.f;
-      uint32_t pw[NO / 2];  // fp16 pairs of the P~ row: hi[0..NQ), lo[0..NQ), zero padding
+      uint32_t ph[NQH / 2], pl[NQH / 2];  // fp16 pairs of this group's hi and lo P~ columns
 #pragma unroll
-      for (int k = NQ; k < NO / 2; ++k) pw[k] = 0u;
-#pragma unroll
-      for (int q = 0; q < NQ; q += 2) {
-        const float2 m0 = bi[q], m1 = bi[q + 1];
+      for (int q = 0; q < NQH; q += 2) {
+        const float2 m0 = bi[q0 + q], m1 = bi[q0 + q + 1];
         const float p0 = ex2(s[q] - m0.x), p1 = ex2(s[q + 1] - m1.x);  // 0 for a row the query does not see
         l[q] = fmaf(l[q], m0.y, p0);
         l[q + 1] = fmaf(l[q + 1], m1.y, p1);
@@ -607,13 +646,17 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
         const __half2 hi = __floats2half2_rn(t0, t1);
         const float2 hf = __half22float2(hi);
         const __half2 lo = __floats2half2_rn(t0 - hf.x, t1 - hf.y);
-        pw[q >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
-        pw[(NQ + q) >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+        ph[q >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+        pl[q >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
       }
+      // P~ row of token t: column c at byte (c / 8) * 128 + (c % 8) * 2 of the row's core-matrix run
       const uint32_t pa = s_p + (uint32_t)((i % NV) * C::PB) + (uint32_t)((t >> 3) * C::LBO_P + (t & 7) * 16);
+      store_cols<NQH>(pa, q0, ph);
+      store_cols<NQH>(pa, NQ + q0, pl);
+      if (grp == 1) {
 #pragma unroll
-      for (int c = 0; c < NO / 8; ++c)
-        sts128(pa + c * 128, make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
+        for (int c = 2 * NQ / 8; c < NO / 8; ++c) sts128(pa + c * 128, make_uint4(0u, 0u, 0u, 0u));
+      }
       tc05::fence_proxy_async_smem();
       mbar_arrive(&pfull[i % NV]);
       sk_cur = sk_n;
@@ -624,19 +667,19 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
 
     // CTA partial per query: (m, l, O[R])
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
+    for (int q = 0; q < NQH; ++q) {
       float v = l[q];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) lsum[warp * NQ + q] = v;
+      if (lane == 0) lsum[wq * NQ + q0 + q] = v;
     }
     if (holder)
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) res[q * (R + 2) + 2 + orow] = acc[q];
+      for (int q = 0; q < NQH; ++q) res[(q0 + q) * (R + 2) + 2 + orow] = acc[q];
     named_barrier_sync(1, kGConsumers);
-    if (t < NQ) {
-      res[t * (R + 2)] = mrun[t];
-      res[t * (R + 2) + 1] = ((lsum[t] + lsum[NQ + t]) + lsum[2 * NQ + t]) + lsum[3 * NQ + t];
+    if (ct < NQ) {
+      res[ct * (R + 2)] = mrun[ct];
+      res[ct * (R + 2) + 1] = ((lsum[ct] + lsum[NQ + ct]) + lsum[2 * NQ + ct]) + lsum[3 * NQ + ct];
     }
     named_barrier_sync(1, kGConsumers);
 
@@ -645,16 +688,16 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     bool finish = true;
     if (ncontrib > 1) {
       float* dst = a.partials + ((size_t)gidx * a.slot_stride + split) * NQ * (R + 2);
-      for (int e2 = t; e2 < nq * (R + 2); e2 += kGConsumers) dst[e2] = res[e2];
+      for (int e2 = ct; e2 < nq * (R + 2); e2 += kGConsumers) dst[e2] = res[e2];
       __threadfence();
       named_barrier_sync(1, kGConsumers);
-      if (t == 0) flag[0] = atomicAdd(&a.counters[gidx], 1) == ncontrib - 1;
+      if (ct == 0) flag[0] = atomicAdd(&a.counters[gidx], 1) == ncontrib - 1;
       named_barrier_sync(1, kGConsumers);
       finish = flag[0] != 0;
       if (finish) {  // last arriver: merge the splits in order
         __threadfence();
         const float* part = a.partials + (size_t)gidx * a.slot_stride * NQ * (R + 2);
-        for (int e2 = t; e2 < nq * (R + 1); e2 += kGConsumers) {
+        for (int e2 = ct; e2 < nq * (R + 1); e2 += kGConsumers) {
           const int ql = e2 / (R + 1), col = 1 + e2 % (R + 1);
           float M = kNegInf;
           for (int sp = 0; sp < ncontrib; ++sp) M = fmaxf(M, __ldcg(part + ((size_t)sp * NQ + ql) * (R + 2)));
@@ -666,11 +709,11 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
           res[ql * (R + 2) + col] = acc2;
         }
         named_barrier_sync(1, kGConsumers);
-        if (t == 0) atomicExch(&a.counters[gidx], 0);
+        if (ct == 0) atomicExch(&a.counters[gidx], 0);
       }
     }
     if (finish) {  // out_q = (O_q / l_q) . B_Vh
-      for (int idx = t; idx < nq * a.Hd; idx += kGConsumers) {
+      for (int idx = ct; idx < nq * a.Hd; idx += kGConsumers) {
         const int ql = idx / a.Hd, d = idx % a.Hd;
         const float* rq = fin + ql * (R + 2);
         const float inv = rq[1] > 0.f ? 1.f / rq[1] : 0.f;
