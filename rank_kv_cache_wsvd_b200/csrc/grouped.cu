@@ -22,13 +22,16 @@
 // both halves as separate columns of the accumulator.
 //
 // Per CTA (one (b, latent head, query chunk) and one run of 128-token tiles):
-//   warps 0-3  consumers; thread t <-> token t of a tile <-> tensor-memory lane t:
-//              widen the staged tile into the MMA operand layouts, read the
-//              scores, online softmax (exact per-tile maximum per query), write
-//              P~, and fold each tile's O into registers;
-//   warp 4     producer: 1-D bulk copies (TMA, no multicast) of codes + scales
+//   warps 0-7  consumers, two warpgroups each holding half of the queries;
+//              thread t of a group <-> token t of a tile <-> tensor-memory
+//              lane t: widen the staged tile into the MMA operand layouts
+//              (group 0 the K codes, group 1 the V codes), read the scores,
+//              online softmax (exact per-tile maximum per query), write P~,
+//              and fold each tile's O into registers;
+//   warp 8     producer: 1-D bulk copies (TMA, no multicast) of codes + scales
 //              into an mbarrier ring;
-//   warp 5     allocates tensor memory; one lane issues the MMAs.
+//   warp 9     allocates tensor memory and issues the MMAs (converged warp,
+//              one elected lane).
 // Split partials (m, l, O) merge last-arriver in split order (deterministic).
 #include <algorithm>
 #include <map>

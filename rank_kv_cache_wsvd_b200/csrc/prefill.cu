@@ -470,17 +470,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) prefill_gemm_kernel(const Pre
 
 // ------------------------------------------------------------------ 2'. GEMM + quantise on tcgen05
 // The same product and epilogue on the fifth-generation tensor cores, for
-// shapes whose 64- (r <= 64) or 128-column (r = 128) output tiles hold whole
-// heads of one side (K or V): 128 x BN output tiles, one CTA each.
+// shapes whose 64- or 128-column output tiles hold whole heads of one side
+// (K or V): 128 x BN output tiles, one CTA each (BN = 128 when H * r allows
+// and the tiles fill the device, else 64).
 //   warp 4   TMA producer: per 64-wide k-tile, the hi and lo activation tiles
 //            [128 x 64] (2-D tensor maps, 128-byte swizzle, K-major) and the
 //            weight tile [64 x BN] as BN / NG boxes of one head's NG columns
 //            (3-D tensor map over A [H][E][r], swizzle of NG * 2 bytes; the
 //            operand is N-major) into a four-stage mbarrier ring;
-//   warp 5   allocates tensor memory; one lane issues per k-tile four MMAs of
-//            the hi half into a fresh accumulator (one of NH, so that it runs
-//            up to NH k-tiles ahead of the epilogue) and four of the lo half
-//            into one accumulator kept over all of E;
+//   warp 5   allocates tensor memory and issues (converged, one elected
+//            lane) per k-tile four MMAs of the hi half into a fresh
+//            accumulator (one of NH, so that it runs up to NH k-tiles ahead
+//            of the epilogue) and four of the lo half into one accumulator
+//            kept over all of E;
 //   warps 0-3  thread t <-> output row t <-> tensor-memory lane t: add each
 //            k-tile's hi sum to an fp32 register total with a round-to-nearest
 //            add, then add the lo sum, undo p_m and quantise every head of the
@@ -520,14 +522,7 @@ struct TcArgs {
   int32_t* err;
 };
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-// Warp-level forms: a converged warp calls them, one elected lane issues.
+// TMA tile loads, warp-level: a converged warp calls them, one elected lane issues.
 __device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -547,15 +542,6 @@ __device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-
 template <int R, int BN_>
 __global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_xhi, const __grid_constant__ CUtensorMap tm_xlo,
@@ -575,7 +561,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* done = hfree + NH;   // every MMA of the tile has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.y * BN;
   const int HR = a.H * R;
   const int kv = n0 >= HR ? 1 : 0, nl = n0 - kv * HR;  // tile columns within the K or the V side

@@ -62,23 +62,7 @@ __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------- MMA
-// D[tmem] (+)= A[smem] . B[smem]^T, issued by one thread.
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accum)
-      : "memory");
-}
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accum)
-      : "memory");
-}
+// D[tmem] (+)= A[smem] . B[smem]^T.
 // Warp-level issue: every lane of a converged warp executes the call with the
 // same operands and one elected lane (the lowest) issues the instruction.
 // Issued this way an MMA costs what the tensor core needs for it; issued from
@@ -104,8 +88,9 @@ __device__ __forceinline__ void mma_i8_warp(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accum)
       : "memory");
 }
-// The commit of the MMAs the elected lane issued (the same lane: the lowest
-// of a converged warp).
+// Arrives once on `bar` when every MMA the elected lane issued before has
+// completed, their shared-memory reads included (the same lane: the lowest of
+// a converged warp).
 __device__ __forceinline__ void commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -113,14 +98,6 @@ __device__ __forceinline__ void commit_warp(uint64_t* bar) {
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
           static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
       : "memory");
-}
-
-// Arrives once on `bar` when every MMA this thread issued before has completed
-// (their shared-memory reads included).
-__device__ __forceinline__ void commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
-               : "memory");
 }
 
 // ---------------------------------------------------------------- loads
