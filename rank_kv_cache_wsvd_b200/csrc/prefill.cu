@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
                                                                      float* inv_p) {
   extern __shared__ __align__(16) float xs[];
   __shared__ float wmax[kRotThreads / 32];
+  griddep_launch_dependents();  // the GEMM behind may set up (it waits for this grid before reading)
   const int m = blockIdx.x, tid = threadIdx.x;
   const int E4 = E / 4;  // E is a multiple of 64: rows are whole 8-byte groups of four values
   const uint2* xr = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(x) + (size_t)m * E);
@@ -147,18 +148,21 @@ __global__ void __launch_bounds__(kRotThreads) prefill_rotate_kernel(const void*
   if (tid == 0) inv_p[m] = __uint_as_float((uint32_t)(127 - k) << 23);
 }
 
-// Register / shuffle version of the same rotation for rows of E = 128 * EPT
-// values (EPT a power of two <= 64) and blocks of at most 32 * EPT: 128
+// Register / shuffle version of the same rotation for rows of E = NT * EPT
+// values (EPT a power of two in [4, 64]) and blocks of at most 32 * EPT: NT
 // threads, thread i holds the EPT consecutive values i*EPT ..; butterfly
 // distances below EPT stay in registers, distances EPT .. 16*EPT are lane
 // exchanges inside the warp, so the only block-wide step is the maximum.
 // The arithmetic per value is the shared-memory kernel's (the same adds and
-// subtracts in the same stage order, the same normalisation, p_m and split).
-template <int EPT>
-__global__ void __launch_bounds__(128) prefill_rotate_reg_kernel(const void* x, int x_dtype, int E, int blk,
-                                                                 float hnorm, __half* xhi, __half* xlo,
-                                                                 float* inv_p) {
-  __shared__ float wmax[4];
+// subtracts in the same stage order, the same normalisation, p_m and split),
+// whatever NT.  More threads per row (fewer values each) keep more loads in
+// flight per SM: the kernel is bound by the latency of its row loads.
+template <int EPT, int NT>
+__global__ void __launch_bounds__(NT) prefill_rotate_reg_kernel(const void* x, int x_dtype, int E, int blk,
+                                                                float hnorm, __half* xhi, __half* xlo,
+                                                                float* inv_p) {
+  __shared__ float wmax[NT / 32];
+  griddep_launch_dependents();  // the GEMM behind may set up (it waits for this grid before reading)
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const uint16_t* xr = static_cast<const uint16_t*>(x) + (size_t)m * E + (size_t)tid * EPT;
   float v[EPT];
@@ -203,7 +207,9 @@ __global__ void __launch_bounds__(128) prefill_rotate_reg_kernel(const void* x, 
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (lane == 0) wmax[tid >> 5] = amax;
   __syncthreads();
-  amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  amax = wmax[0];
+#pragma unroll
+  for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, wmax[w]);
   int k = 0;
   if (amax > 0.f) {
     const int e = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 127;
@@ -561,6 +567,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* done = hfree + NH;   // every MMA of the tile has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
+  griddep_launch_dependents();  // the length advance behind may launch (it waits for this grid)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int m0 = blockIdx.x * kTcBM, n0 = blockIdx.y * BN;
   const int HR = a.H * R;
@@ -596,6 +603,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // one elected lane issues), so that the copies and MMAs issue at full rate.
   if (warp == 4) {  // ------------------------------------------------------ TMA producer
     const CUtensorMap* wmap = kv ? &tm_wv : &tm_wk;
+    griddep_wait();  // the split activations come from the rotation grid launched before this one
     for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % S;
       if (kt >= S) wait(&empty[s], (uint32_t)(((kt / S) - 1) & 1));
@@ -637,6 +645,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     wait(done, 0);  // every MMA has completed before the allocation is released
     __syncwarp();
   } else {  // -------------------------------------------------------- epilogue, thread = output row
+    griddep_wait();  // 1 / p_m comes from the rotation grid
     const int row = tid;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     float tot[BN];
@@ -792,8 +801,17 @@ cudaError_t launch_tc(const PrefillArgs& pa, const void* A_k, const void* A_v, i
   ta.lat_k = pa.lat_k; ta.lat_v = pa.lat_v; ta.scale_k = pa.scale_k; ta.scale_v = pa.scale_v; ta.err = err;
   const dim3 grid((unsigned)((pa.M + kTcBM - 1) / kTcBM), (unsigned)(pa.N / C::BN));
   (void)cudaGetLastError();
-  prefill_tc_kernel<R, BN><<<grid, kTcThreads, C::SMEM, s>>>(mh, ml, mk, mv, ta);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_tc_kernel<R, BN>, mh, ml, mk, mv, ta);
 }
 
 // Output tile width of the tcgen05 path: 128 columns when the tiles hold whole
@@ -811,6 +829,7 @@ int tc_tile_width(long long M, int H, int r) {
 
 // ------------------------------------------------------------------ 3. lengths
 __global__ void prefill_advance_kernel(int32_t* seq_lens, int B, int T, int L_cap, int32_t* err) {
+  griddep_wait();  // launched as a programmatic dependent of the GEMM, which reads the lengths
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int pos = seq_lens[b];
     if (pos >= 0 && (long long)pos + T <= L_cap) seq_lens[b] = pos + T;
@@ -878,17 +897,25 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
   __half* whi = reinterpret_cast<__half*>(w);
   __half* wlo = reinterpret_cast<__half*>(w + xbytes);
   float* winv = reinterpret_cast<float*>(w + 2 * xbytes);
-  const int ept = E / 128;
-  const bool reg_path = E % 128 == 0 && (ept & (ept - 1)) == 0 && ept >= 4 && ept <= 64 &&
-                        hadamard_block <= 32 * ept;
-  if (reg_path) {
-    switch (ept) {
-      case 4: prefill_rotate_reg_kernel<4><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
-      case 8: prefill_rotate_reg_kernel<8><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
-      case 16: prefill_rotate_reg_kernel<16><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
-      case 32: prefill_rotate_reg_kernel<32><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
-      default: prefill_rotate_reg_kernel<64><<<(unsigned)M, 128, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo, winv); break;
+  // Register path: the most threads per row (512, 256 or 128) that leave each
+  // a power-of-two run of 4 .. 64 values and a block within a warp's reach.
+  int nt = 0, ept = 0;
+  for (int cand = 512; cand >= 128 && !nt; cand >>= 1) {
+    const int e = E / cand;
+    if (E % cand == 0 && e >= 4 && e <= 64 && (e & (e - 1)) == 0 && hadamard_block <= 32 * e) {
+      nt = cand;
+      ept = e;
     }
+  }
+  if (nt) {
+#define WSVD_ROT(EPT_, NT_)                                                                                   \
+  if (ept == EPT_ && nt == NT_)                                                                               \
+    prefill_rotate_reg_kernel<EPT_, NT_><<<(unsigned)M, NT_, 0, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, \
+                                                                    wlo, winv);
+    WSVD_ROT(4, 128) WSVD_ROT(8, 128) WSVD_ROT(16, 128) WSVD_ROT(32, 128) WSVD_ROT(64, 128)
+    WSVD_ROT(4, 256) WSVD_ROT(8, 256) WSVD_ROT(16, 256) WSVD_ROT(32, 256) WSVD_ROT(64, 256)
+    WSVD_ROT(4, 512) WSVD_ROT(8, 512) WSVD_ROT(16, 512) WSVD_ROT(32, 512) WSVD_ROT(64, 512)
+#undef WSVD_ROT
   } else {
     prefill_rotate_kernel<<<(unsigned)M, kRotThreads, rot_smem, s>>>(x, x_dtype, E, hadamard_block, hnorm, whi, wlo,
                                                                      winv);
@@ -915,6 +942,18 @@ extern "C" int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, 
     const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)((N + kBN - 1) / kBN));
     prefill_gemm_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(a);
   }
-  prefill_advance_kernel<<<1, 128, 0, s>>>(seq_lens, B, T, L_cap, err);
+  {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, prefill_advance_kernel, seq_lens, B, T, L_cap, err) != cudaSuccess)
+      return WSVD_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? WSVD_OK : WSVD_ERR_CUDA;
 }
