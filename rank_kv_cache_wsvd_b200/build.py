@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libwsvd_b200.so")
 SOURCES = ["api.cu", "decode.cu", "shared.cu", "append.cu", "noalloc.cu", "fold.cu", "prefill.cu", "grouped.cu"]
-HEADERS = ["common.cuh", "wsvd_internal.h", "tc05.cuh"]
+HEADERS = ["common.cuh", "wsvd_internal.h", "tc05.cuh", "append_core.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
