@@ -61,7 +61,8 @@ def source_digest(files):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"append": ["append.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
+KERNEL_SOURCES = {"append": ["append.cu", "append_core.cuh", "common.cuh", "wsvd_internal.h", "api.cu"],
+                  "step": ["decode.cu", "append_core.cuh", "common.cuh", "wsvd_internal.h", "api.cu"],
                   "decode": ["decode.cu", "shared.cu", "common.cuh", "wsvd_internal.h", "api.cu"],
                   "prefill_gemm": ["prefill.cu", "common.cuh", "wsvd_internal.h", "tc05.cuh"],
                   "grouped": ["grouped.cu", "common.cuh", "wsvd_internal.h", "tc05.cuh"]}
@@ -199,9 +200,14 @@ class WsvdStep:
         else:
             self.q_host = torch.from_numpy(d.q_bits.view(np.int16).copy()).view(qdt).pin_memory()
         self.out_host = torch.empty((w.B, w.H, w.Hd), dtype=torch.float32).pin_memory()
-        # kernels per step: the append, and the decode's one or two (cluster kernel, or q' + split-L grid)
-        self.launches_per_step = (1 if self.has_append else 0) + W.wsvd_decode_launch_count(
-            w.B, w.H, w.Hd, w.r, w.bits, w.L_cap)
+        # kernels per step: one when the append and the decode run as one kernel, else the append and
+        # the decode's one or two (cluster kernel, or q' + split-L grid)
+        if self.has_append:
+            self.launches_per_step = W.wsvd_step_launch_count(w.B, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap,
+                                                              w.hadamard_block, w8)
+        else:
+            self.launches_per_step = W.wsvd_decode_launch_count(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap)
+        self.one_kernel = self.has_append and self.launches_per_step == 1
 
     def reset(self):
         self.lens.copy_(self.lens0)
@@ -852,7 +858,10 @@ def main():
     app_bytes = alg_bytes_append(w, w8) if st.has_append else 0
     per_app = t_app / args.steps
     per_dec = t_dec / args.steps
-    if st.has_append and per_app >= per_dec:
+    if st.one_kernel:
+        dom, nbytes, dur, launches = "step", app_bytes + dec_bytes, t_step / args.steps, \
+            "wsvd one-kernel step (append + decode, 1 launch)"
+    elif st.has_append and per_app >= per_dec:
         dom, nbytes, dur, launches = "append", app_bytes, per_app, "wsvd latent append (1 launch)"
     else:
         dom, nbytes, dur, launches = "decode", dec_bytes, per_dec, \
@@ -926,7 +935,9 @@ def main():
                        "attended_tokens_per_seq": [int(x) for x in st.lens_after],
                        "step": ("append + decode" if st.has_append else "decode"),
                        "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
-                       "launch": ("one wsvd_append_and_decode call per step (decode launched behind the "
+                       "launch": ("one wsvd_append_and_decode call per step (one kernel: append and decode); "
+                                  "events around the call" if st.one_kernel else
+                                  "one wsvd_append_and_decode call per step (decode launched behind the "
                                   "append as a programmatic dependent); events around the call"
                                   if st.has_append else "one wsvd_decode_attention call per step; events around it")},
             "step_us": ms_per_step * 1e3,

@@ -220,7 +220,7 @@ int wsvd_decode_attention_noalloc(int B, int H, int Hd, int r, int bits, int L_c
  *                           WSVD_ERR_UNSUPPORTED when the rotated slice,
  *                           B * E/c fp32 values, and the 32 KB row ring do
  *                           not fit in 200 KB of shared memory.
- *   r                       multiple of 8, at most 128, r * bits/8 % 4 == 0.
+ *   r                       8, 16, 32, 64 or 128.
  *   B                       1..16.
  *   seq_lens   [B]          int32, read and advanced in place.
  *   workspace               at least wsvd_append_workspace_size() bytes of
@@ -273,17 +273,25 @@ int wsvd_latent_prefill(int B, int T, int H, int E, int r, int bits, int L_cap, 
  * the cache including it; WSVD summaries, German §2.A and §2.C).  The pages
  * define no separate interface for it; the results are those of the two calls
  * made back to back, bit for bit.
- * The decode is launched as a programmatic dependent of the append: its launch
- * and its query projection q' = B_Kh . q overlap the append, and it reads
- * seq_lens and the cache only after the append grid has completed.  So q, B_k
- * and B_v must already be final when this call is made (they are read while
- * the append runs; the append itself never writes them).
+ * For one sequence (B = 1) whose decode takes the one-cluster-per-head path
+ * with the append's cluster size (short caches: each of the cluster's ranks
+ * holds at most one tile of rows), one kernel does both: cluster h projects
+ * head h's new K and V rows, the rank whose rows hold the new token quantises
+ * them, writes them to the cache and attends over them, and the other ranks
+ * attend over their rows meanwhile.  Otherwise the decode is launched as a
+ * programmatic dependent of the append: its launch and its query projection
+ * q' = B_Kh . q overlap the append, and it reads seq_lens and the cache only
+ * after the append grid has completed.  Either way q, B_k and B_v must
+ * already be final when this call is made (they are read while the append
+ * runs; the append itself never writes them).  wsvd_step_launch_count tells
+ * how many kernels a step takes for the given sizes on the current device.
  *   append_workspace   wsvd_append_workspace_size() bytes, contract as for
  *                      wsvd_latent_append;
  *   decode_workspace   wsvd_decode_workspace_size(B, H, r) bytes, contract as
  *                      for wsvd_decode_attention.
  * Every argument of both operations is validated before anything is launched;
  * the status codes are those of the two calls.                              */
+int wsvd_step_launch_count(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block, int w8);
 int wsvd_append_and_decode(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block,
                            const void* x, int x_dtype, const void* A_k, const void* A_v, int32_t* seq_lens,
                            uint8_t* lat_k, uint8_t* lat_v, void* scale_k, void* scale_v, const void* q,

@@ -35,6 +35,7 @@ SIGNATURES = {
     "shared_decode_workspace_size": (_c_size, [_c_int] * 3),
     "wsvd_append_workspace_size": (_c_size, []),
     "wsvd_decode_launch_count": (_c_int, [_c_int] * 6),
+    "wsvd_step_launch_count": (_c_int, [_c_int] * 9),
     "wsvd_decode_attention": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _c_size,
                                                                                         _p, _p]),
     "wsvd_decode_attention_noalloc": (_c_int, [_c_int] * 6 + [_p, _p, _c_int] + [_p] * 6 + [_c_float, _p, _p, _p]),
@@ -142,6 +143,12 @@ def wsvd_decode_workspace_size(B, H, r) -> int:
 def wsvd_decode_launch_count(B, H, Hd, r, bits, L_cap) -> int:
     """Kernels one wsvd_decode_attention call with these sizes launches on the current device."""
     return load().wsvd_decode_launch_count(B, H, Hd, r, bits, L_cap)
+
+
+def wsvd_step_launch_count(B, H, Hd, E, r, bits, L_cap, hadamard_block=128, w8=False) -> int:
+    """Kernels one wsvd_append_and_decode(_w8) call with these sizes launches on
+    the current device: 1 when the append and the decode run as one kernel."""
+    return load().wsvd_step_launch_count(B, H, Hd, E, r, bits, L_cap, hadamard_block, int(bool(w8)))
 
 
 def dense_decode_workspace_size(B, H, Hd) -> int:

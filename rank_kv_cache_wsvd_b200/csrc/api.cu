@@ -133,7 +133,9 @@ int prepare_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard
   if (hadamard_block < 1 || hadamard_block > 1024 || (hadamard_block & (hadamard_block - 1)))
     return WSVD_ERR_INVALID_ARG;
   if (E % hadamard_block) return WSVD_ERR_INVALID_ARG;
-  if (B > 16 || r % 8 || r > 128 || (r * bits / 8) % 4 || E > 65536) return WSVD_ERR_UNSUPPORTED;
+  // r / 8 column groups of 8 must divide a warp (the row walk and the lane reduction)
+  if (B > 16 || (r != 8 && r != 16 && r != 32 && r != 64 && r != 128) || (r * bits / 8) % 4 || E > 65536)
+    return WSVD_ERR_UNSUPPORTED;
   if (!x || !A_k || !A_v || !seq_lens || !lat_k || !lat_v || !scale_k || !scale_v || !workspace)
     return WSVD_ERR_INVALID_ARG;
   if (w8 && (!sA_k || !sA_v)) return WSVD_ERR_INVALID_ARG;
@@ -171,8 +173,11 @@ int run_step(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadama
   st = prepare_wsvd_decode(B, H, Hd, r, bits, L_cap, seq_lens, q, q_dtype, lat_k, lat_v, scale_k, scale_v, B_k, B_v,
                            sB_k, sB_v, w8, softmax_scale, out, decode_workspace, decode_workspace_bytes, err, &dp);
   if (st != WSVD_OK || B == 0) return st;
-  if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
   bind_workspace(&dp, decode_workspace);
+  bool fused = false;
+  if (launch_step_fused(ap, dp, as_stream(stream), &fused) != cudaSuccess) return WSVD_ERR_CUDA;
+  if (fused) return WSVD_OK;
+  if (launch_append(ap, as_stream(stream)) != cudaSuccess) return WSVD_ERR_CUDA;
   if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, as_stream(stream), true) !=
       cudaSuccess)
     return WSVD_ERR_CUDA;
@@ -318,6 +323,21 @@ int wsvd_decode_launch_count(int B, int H, int Hd, int r, int bits, int L_cap) {
   return decode_launch_count(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a);
 }
 
+int wsvd_step_launch_count(int B, int H, int Hd, int E, int r, int bits, int L_cap, int hadamard_block, int w8) {
+  if (B < 1 || H < 1 || E < 1 || L_cap < 0 || (bits != 8 && bits != 4) || r < 1 || (r * bits) % 8) return 0;
+  if (hadamard_block < 1 || (hadamard_block & (hadamard_block - 1)) || E % hadamard_block) return 0;
+  const int cl = append_cluster_size(E, hadamard_block);
+  if (cl < 1) return 0;
+  DecodeArgs a{};
+  a.B = B; a.H = H; a.Hd = Hd; a.W = r; a.L_cap = L_cap; a.w8 = w8 ? 1 : 0;
+  AppendArgs ap{};
+  ap.B = B; ap.H = H; ap.E = E; ap.r = r; ap.bits = bits; ap.L_cap = L_cap; ap.blk = hadamard_block;
+  ap.cluster = cl; ap.w8 = a.w8;
+  if (step_fused_applies(ap, a)) return 1;
+  const int n = decode_launch_count(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, a);
+  return n > 0 ? 1 + n : 0;
+}
+
 size_t wsvd_append_workspace_size(void) { return kAppendWorkspaceBytes; }
 
 int wsvd_latent_append(int B, int H, int E, int r, int bits, int L_cap, int hadamard_block, const void* x,
@@ -421,9 +441,11 @@ int wsvd_append_and_decode_host(int B, int H, int Hd, int E, int r, int bits, in
              cudaMemcpyAsync(q_dev, q_host, qbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
     return WSVD_ERR_CUDA;
   }
-  if (launch_append(ap, s) != cudaSuccess) return WSVD_ERR_CUDA;
   bind_workspace(&dp, w + l.dec);
-  if (launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, s, true) != cudaSuccess)
+  bool fused = false;
+  if (launch_step_fused(ap, dp, s, &fused) != cudaSuccess) return WSVD_ERR_CUDA;
+  if (!fused && (launch_append(ap, s) != cudaSuccess ||
+                 launch_decode(bits == 8 ? kCodecI8 : kCodecI4, r * bits / 8, kQProj, dp, s, true) != cudaSuccess))
     return WSVD_ERR_CUDA;
   if (!in_place && cudaMemcpyAsync(out_host, out_dev, obytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return WSVD_ERR_CUDA;

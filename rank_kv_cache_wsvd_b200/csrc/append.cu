@@ -123,7 +123,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
 #pragma unroll 1
       for (int k = 0; k < kRing; ++k) w.issue(ring, k, tid);  // re-stream (L2) for the next batch rows
     }
-    float acc[BB][8];
+    float2 acc[BB][4];
     stream_rows<BB, W8>(w, ring, xs, B, bb0, acc, tid);
     reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, slots + (size_t)bb0 * r, remote_slot + 4u * bb0 * r,
                    remote_bar, tid, block_sync);
@@ -164,7 +164,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     const size_t row = ((size_t)b * a.H + h) * a.L_cap + (ok ? pos : 0);
     const __half sh = quantise_append_row<W8>(slots + (size_t)b * r, (size_t)B * r, a.cluster, r, a.bits, a.hnorm,
                                               W8 ? (kv ? a.sAv : a.sAk) + (size_t)h * r : nullptr, ok,
-                                              (kv ? a.lat_v : a.lat_k) + row * RB, lane);
+                                              (kv ? a.lat_v : a.lat_k) + row * RB, nullptr, lane);
     if (lane == 0) {
       if (ok) (kv ? a.scale_v : a.scale_k)[row] = sh;
       else if (unit == 0) set_err(a.err, WSVD_DEVERR_CACHE_FULL);

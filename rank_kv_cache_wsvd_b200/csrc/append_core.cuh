@@ -46,61 +46,98 @@ struct RowWalk {
   }
 };
 
+// c[bb0 + bi][8 * cgi .. + 8] += xs[bb0 + bi][e] * A[e][8 * cgi .. + 8] for one
+// A row piece av (8 fp16 values, or 8 int8 codes in av.x, av.y); acc[bi][k]
+// holds columns 2k, 2k + 1 (packed fp32 FMAs, each lane rounded as fmaf).
+template <int BB, bool W8>
+__device__ __forceinline__ void accumulate_row(const uint4& av, const float* xs, int B, int bb0, int Ec, int e,
+                                               float2 (&acc)[BB][4]) {
+  float2 a[4];
+  if (W8) {  // int8 codes -> fp32, exact
+    a[0] = i8_pair(av.x ^ 0x80808080u, 0);
+    a[1] = i8_pair(av.x ^ 0x80808080u, 2);
+    a[2] = i8_pair(av.y ^ 0x80808080u, 0);
+    a[3] = i8_pair(av.y ^ 0x80808080u, 2);
+  } else {
+    a[0] = h2_pair(av.x);
+    a[1] = h2_pair(av.y);
+    a[2] = h2_pair(av.z);
+    a[3] = h2_pair(av.w);
+  }
+#pragma unroll
+  for (int bi = 0; bi < BB; ++bi) {
+    const float xv = (bb0 + bi < B) ? xs[(size_t)(bb0 + bi) * Ec + e] : 0.f;
+    const float2 x2 = make_float2(xv, xv);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[bi][k] = __ffma2_rn(x2, a[k], acc[bi][k]);
+  }
+}
+
 // Accumulate c[bb0 + bi][8 * cgi .. + 8] over this thread's rows, streaming
 // them through the ring (rows 0 .. kRing-1 already issued by the caller).
 template <int BB, bool W8>
 __device__ __forceinline__ void stream_rows(const RowWalk<W8>& w, uint4* ring, const float* xs, int B, int bb0,
-                                            float (&acc)[BB][8], int tid) {
+                                            float2 (&acc)[BB][4], int tid) {
 #pragma unroll
   for (int bi = 0; bi < BB; ++bi)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[bi][k] = 0.f;
+    for (int k = 0; k < 4; ++k) acc[bi][k] = make_float2(0.f, 0.f);
   for (int k = 0; k < w.nrows; ++k) {
     cp_async_wait_ring();  // this thread's group k is complete
     const uint4 av = ring[(size_t)(k % kRing) * kAppendThreads + tid];
-    float2 a01, a23, a45, a67;
-    if (W8) {  // int8 codes -> fp32, exact
-      a01 = i8_pair(av.x ^ 0x80808080u, 0);
-      a23 = i8_pair(av.x ^ 0x80808080u, 2);
-      a45 = i8_pair(av.y ^ 0x80808080u, 0);
-      a67 = i8_pair(av.y ^ 0x80808080u, 2);
-    } else {
-      a01 = h2_pair(av.x);
-      a23 = h2_pair(av.y);
-      a45 = h2_pair(av.z);
-      a67 = h2_pair(av.w);
-    }
-    const float af[8] = {a01.x, a01.y, a23.x, a23.y, a45.x, a45.y, a67.x, a67.y};
     // The slot is consumed (values in registers) before it is refilled.
     w.issue(ring, k + kRing, tid);
-    const int e = w.row(k);
-#pragma unroll
-    for (int bi = 0; bi < BB; ++bi) {
-      const float xv = (bb0 + bi < B) ? xs[(size_t)(bb0 + bi) * w.Ec + e] : 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[bi][j] = fmaf(xv, af[j], acc[bi][j]);
-    }
+    accumulate_row<BB, W8>(av, xs, B, bb0, w.Ec, w.row(k), acc);
   }
 }
 
-// Reduce acc over the CTA (threads sharing a column group, then warps) into
-// the slot rows bi < nb: a local store on the leader (remote_bar == 0), else an
-// st.async into the leader's slot at cluster address remote_dst that completes
-// 4 bytes per value on the leader's barrier.  Fixed summation order.
-template <int BB, typename Sync>
-__device__ __forceinline__ void reduce_cta(float (&acc)[BB][8], int ncg, int r, int nb, float* red, float* dst,
-                                           uint32_t remote_dst, uint32_t remote_bar, int tid, Sync sync) {
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int o = ncg; o < 32; o <<= 1)
+// Pairwise sums over the lanes that share a column group (lane % NCG), in
+// the order of a butterfly with partner lane ^ O for O = NCG, 2 NCG, ..., 16,
+// halving the values every round while more than one is left: each sum is
+// the one the full butterfly gives, bit for bit, with far fewer shuffles.
+// Returns the index of this lane's first value; it keeps NV >> rounds values
+// (at least one; lanes that differ only in the later rounds' bits then hold
+// the same sum).
+template <int NV, int O>
+__device__ __forceinline__ int reduce_scatter_lanes(float* v, int lane) {
+  if constexpr (O >= 32) {
+    return 0;
+  } else if constexpr (NV >= 2) {
+    constexpr int HALF = NV / 2;
+    const bool up = (lane & O) != 0;
 #pragma unroll
-    for (int bi = 0; bi < BB; ++bi)
+    for (int j = 0; j < HALF; ++j) {
+      const float send = up ? v[j] : v[j + HALF];
+      const float keep = up ? v[j + HALF] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+    }
+    return (up ? HALF : 0) + reduce_scatter_lanes<HALF, O * 2>(v, lane);
+  } else {
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+    return reduce_scatter_lanes<1, O * 2>(v, lane);
+  }
+}
+
+template <int BB, int NCG, typename Sync>
+__device__ __forceinline__ void reduce_cta_n(float2 (&acc)[BB][4], int r, int nb, float* red, float* dst,
+                                             uint32_t remote_dst, uint32_t remote_bar, int tid, Sync sync) {
+  constexpr int NV = BB * 8;
+  constexpr int ROUNDS = NCG == 1 ? 5 : NCG == 2 ? 4 : NCG == 4 ? 3 : NCG == 8 ? 2 : 1;
+  constexpr int KEPT = (NV >> ROUNDS) > 0 ? (NV >> ROUNDS) : 1;
+  const int warp = tid >> 5, lane = tid & 31, cgi = lane % NCG;
+  float v[NV];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[bi][k] += __shfl_xor_sync(0xffffffffu, acc[bi][k], o);
-  if (lane < ncg) {
+  for (int bi = 0; bi < BB; ++bi)
 #pragma unroll
-    for (int bi = 0; bi < BB; ++bi)
+    for (int k = 0; k < 4; ++k) {
+      v[bi * 8 + 2 * k] = acc[bi][k].x;
+      v[bi * 8 + 2 * k + 1] = acc[bi][k].y;
+    }
+  const int base = reduce_scatter_lanes<NV, NCG>(v, lane);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) red[(warp * BB + bi) * r + lane * 8 + k] = acc[bi][k];
+  for (int i = 0; i < KEPT; ++i) {
+    const int idx = base + i, bi = idx >> 3, k = idx & 7;
+    red[(warp * BB + bi) * r + cgi * 8 + k] = v[i];
   }
   sync();
   for (int idx = tid; idx < nb * r; idx += kAppendThreads) {
@@ -112,6 +149,24 @@ __device__ __forceinline__ void reduce_cta(float (&acc)[BB][8], int ncg, int r, 
     else dst[(size_t)bi * r + j] = s;
   }
   sync();
+}
+
+// Reduce acc over the CTA (threads sharing a column group, then warps) into
+// the slot rows bi < nb: a local store on the leader (remote_bar == 0), else an
+// st.async into the leader's slot at cluster address remote_dst that completes
+// 4 bytes per value on the leader's barrier.  Fixed summation order: within a
+// warp the butterfly over the lanes of a column group (partners at offsets
+// ncg, 2 ncg, ..., 16), then the warps in order.  ncg = r / 8 divides 32.
+template <int BB, typename Sync>
+__device__ __forceinline__ void reduce_cta(float2 (&acc)[BB][4], int ncg, int r, int nb, float* red, float* dst,
+                                           uint32_t remote_dst, uint32_t remote_bar, int tid, Sync sync) {
+  switch (ncg) {
+    case 1: reduce_cta_n<BB, 1>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
+    case 2: reduce_cta_n<BB, 2>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
+    case 4: reduce_cta_n<BB, 4>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
+    case 8: reduce_cta_n<BB, 8>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
+    default: reduce_cta_n<BB, 16>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
+  }
 }
 
 __device__ __forceinline__ float x_elem(uint32_t bits16, int dtype) {
@@ -204,12 +259,12 @@ __device__ __forceinline__ void rotate_x_slice(bool fast, const uint2 (&xraw)[kX
 // Quantise one finished row of one (b, h, K|V) unit, one warp: the cluster
 // ranks' partial sums (slots[q * stride + j], q = 0 .. nranks - 1) added in
 // rank order, times 1/sqrt(blk) (and the int8 weights' column scale), then the
-// append's fp32 decisions; codes and scale written at cache row `row` when
-// `ok`.  Returns the fp16 scale.
+// append's fp32 decisions; the codes are written to dst when `ok` (and to
+// dst2 too, when given).  Returns the fp16 scale.
 template <bool W8>
 __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t stride, int nranks, int r, int bits,
                                                       float hnorm, const float* colscale, bool ok, uint8_t* dst,
-                                                      int lane) {
+                                                      uint8_t* dst2, int lane) {
   const int Q = (bits == 8) ? 127 : 7;
   float cv[4];
   float amax = 0.f;
@@ -231,13 +286,21 @@ __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t
   const float sc = __half2float(sh);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
+    if (32 * k >= r) break;  // no column of this group (uniform across the warp)
     const int j = lane + 32 * k;
     const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(cv[k], sc)))) : 0;
     if (bits == 8) {
-      if (ok && j < r) dst[j] = (uint8_t)code;
+      if (ok && j < r) {
+        dst[j] = (uint8_t)code;
+        if (dst2) dst2[j] = (uint8_t)code;
+      }
     } else {
       const int hi = __shfl_down_sync(0xffffffffu, code, 1);  // column j + 1 (r is a multiple of 8)
-      if (ok && j < r && (lane & 1) == 0) dst[j / 2] = (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+      if (ok && j < r && (lane & 1) == 0) {
+        const uint8_t v = (uint8_t)((code & 0xF) | ((hi & 0xF) << 4));
+        dst[j / 2] = v;
+        if (dst2) dst2[j / 2] = v;
+      }
     }
   }
   return sh;

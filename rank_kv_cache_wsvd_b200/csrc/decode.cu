@@ -45,6 +45,7 @@
 
 #include <cooperative_groups.h>
 
+#include "append_core.cuh"
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -93,7 +94,8 @@ struct HelperArea {
   uint64_t bars[2 * NQ + 4];  // qready[NQ], qfree[NQ], resfull[2], resfree[2]
 };
 
-template <int CODEC, int VPT, int TPT, int NTOK>
+// SOVR: stage count override (0: as many stages as the ring budget holds).
+template <int CODEC, int VPT, int TPT, int NTOK, int SOVR = 0>
 struct Cfg {
   using CT = CodecT<CODEC>;
   static constexpr int kCB = VPT * CT::kBits / 8;  // bytes per lane per token
@@ -107,7 +109,8 @@ struct Cfg {
   static constexpr int kStageBytes = 2 * kCodeBytes + 2 * kScaleBytes;
   static constexpr int kStageBudget = kW <= 32 ? 73728 : 57344;  // ring bytes per CTA (two CTAs per SM)
   static constexpr int kStagesRaw = kStageBudget / kStageBytes;
-  static constexpr int kStages = kStagesRaw < 2 ? 2 : (kStagesRaw > 8 ? 8 : kStagesRaw);
+  static constexpr int kStages =
+      SOVR > 0 ? SOVR : (kStagesRaw < 2 ? 2 : (kStagesRaw > 8 ? 8 : kStagesRaw));
   static constexpr int kRedRaw = kConsumerWarps * TPT * (VPT + 2);
   static constexpr int kRedFloats = kRedRaw < kConsumerThreads ? kConsumerThreads : kRedRaw;
   static constexpr int kQW = VPT / 4;  // byte-plane words of q' per lane
@@ -137,7 +140,7 @@ struct Cfg {
   }
   // cluster kernel: operands, the leader's partial slots, then B_Vh
   __host__ __device__ static size_t cluster_seg_off() { return (kOffPre + 127) / 128 * 128; }
-  static size_t cluster_smem_bytes(int qmode, int Hd) {
+  __host__ __device__ static size_t cluster_smem_bytes(int qmode, int Hd) {
     return cluster_seg_off() + seg_bytes(qmode, kW, Hd) + (size_t)kMaxClusterSize * (kW + 2) * 4 +
            (qmode == kQDirect ? 0 : (size_t)kW * Hd * 2);
   }
@@ -346,7 +349,8 @@ __device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, con
                                             int j0, int jstep, int part) {
   const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * (a.w8 ? 1 : 2));
   const float* colscale = a.w8 ? a.sBk + (size_t)h * a.Hd : nullptr;  // int8 B_K: folded into q
-  const int cols = a.Hd >> 3;
+  const int cols = a.Hd >> 3;  // 4, 8, 16 or 32: a power of two, a multiple of 4
+  const int cmask = cols - 1;
   float amax = 0.f;
   auto qval = [&](int col) {
     const uint16_t qu = qsrc[col];
@@ -354,17 +358,32 @@ __device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, con
   };
   for (int j = j0; j < W; j += jstep) {
     float d = 0.f;
+    // columns ((k + j) mod cols) * 8 + part for k = 0, 1, ...: four loads ahead of four fmas
     if (colscale) {  // int8 B_K
       const int8_t* row = reinterpret_cast<const int8_t*>(sbuf) + (size_t)j * a.Hd;
-      for (int k = 0; k < cols; ++k) {
-        const int col = ((k + j) % cols) * 8 + part;
-        d = fmaf((float)row[col], qval(col) * colscale[col], d);
+      for (int k = 0; k < cols; k += 4) {
+        float bv[4], qv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = ((k + i + j) & cmask) * 8 + part;
+          bv[i] = (float)row[col];
+          qv[i] = qval(col) * colscale[col];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d = fmaf(bv[i], qv[i], d);
       }
     } else {
       const __half* row = reinterpret_cast<const __half*>(sbuf) + (size_t)j * a.Hd;
-      for (int k = 0; k < cols; ++k) {
-        const int col = ((k + j) % cols) * 8 + part;
-        d = fmaf(__half2float(row[col]), qval(col), d);
+      for (int k = 0; k < cols; k += 4) {
+        float bv[4], qv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = ((k + i + j) & cmask) * 8 + part;
+          bv[i] = __half2float(row[col]);
+          qv[i] = qval(col);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d = fmaf(bv[i], qv[i], d);
       }
     }
     d += __shfl_xor_sync(0xffffffffu, d, 1);
@@ -462,11 +481,12 @@ __device__ __forceinline__ void build_query(QState<CODEC, VPT>& qst, const uint8
   if constexpr (Cfg<CODEC, VPT, W / VPT, 1>::kNSeg == 2) qst.swap_halves(swapped_lane(tid & 31));
 }
 
-// One staged tile with n valid tokens: scores, lazy-rescaled online softmax and
-// the latent P.V accumulation of this lane's NTOK tokens.
+// One staged tile: scores, lazy-rescaled online softmax and the latent P.V
+// accumulation of this lane's NTOK tokens.  Tokens n0 <= tok < n are valid
+// (n0 > 0: the rest of a tile whose first rows were processed before).
 template <int CODEC, int VPT, int TPT, int NTOK>
 __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QState<CODEC, VPT>& qst, float& m,
-                                             float& l, float2* acc, int tid) {
+                                             float& l, float2* acc, int tid, int n0 = 0) {
   using C = Cfg<CODEC, VPT, TPT, NTOK>;
   using CT = typename C::CT;
   constexpr int T = C::kT, RB = C::kRB, CB = C::kCB, NSEG = C::kNSeg, TPP = C::kTPP, NP = VPT / 2;
@@ -482,7 +502,7 @@ __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QSt
     float d = qst.dot(seg);
 #pragma unroll
     for (int o = 1; o < TPT; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-    const bool valid = tok < n;
+    const bool valid = tok >= n0 && tok < n;
     const float skk = (CT::kScaled && valid) ? lds_half_as_float(smem_u32(sck + tok)) * qst.step : qst.step;
     sc[k] = valid ? d * skk : kNegInf;
     tmax = fmaxf(tmax, sc[k]);
@@ -497,7 +517,7 @@ __device__ __forceinline__ void process_tile(const uint8_t* st, int n, const QSt
 #pragma unroll
   for (int k = 0; k < NTOK; ++k) {
     const int tok = k * TPP + g_tok;
-    if (tok < n) {
+    if (tok >= n0 && tok < n) {
       const float p = ex2(sc[k] - m);
       l += p;
       const float wv = CT::kScaled ? p * lds_half_as_float(smem_u32(sck + T + tok)) : p;
@@ -1433,6 +1453,310 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
   finalize_out<W>(res, Bvh, a.out + ((size_t)b * a.H + h) * a.Hd, a.Hd, red, tid);
 }
 
+// ------------------------------------------------------------------ one-kernel step (one sequence)
+// The latent append and the decode of one step in one grid, for a single
+// sequence (B = 1) whose decode takes the cluster path with the append's
+// cluster size and at most one tile per rank.  Cluster h does head h's append
+// for K and V (rank q projects its E slice [q Ec, (q + 1) Ec), as the append
+// kernel's rank q) and head h's decode (rank q its token chunk, as the
+// cluster decode's rank q).  The append's partial rows go to the rank whose
+// chunk holds the new row (the owner) rather than to rank 0: the owner sums
+// them in rank order, quantises, writes the row to the cache and into its
+// staged tile, and adds that token to its softmax state after the tile's
+// other rows.  With one token per lane and tile, a lane's state after the two
+// passes is the one a single pass gives.  The owner also merges the ranks'
+// decode partials (in rank order, as rank 0 of the cluster decode does) and
+// writes out[h].  So every output equals that of the append kernel followed
+// by the cluster decode, bit for bit.
+//
+// Order of work.  Producer lane: barriers, then bulk copies of B_Kh and the
+// query and of this rank's A_Kh and A_Vh slices (contiguous blocks, four
+// chunks each with a barrier apiece; behind a grid that writes the query,
+// the query comes after the dependency wait).  Then the length (its load
+// overlaps the issue), which reaches the consumers through an mbarrier; B_Vh
+// (the merging rank); and, once the slices have landed, the cached rows of
+// the chunk below the new row.  Consumers: q' and the x slice rotation while
+// the copies land; the K and V projections of the slice chunk by chunk,
+// reduced across the CTA in one pass and stored into the owner's slots; the
+// old rows; the owner quantises and processes the new row; every rank but the
+// merging one sends its decode partial there, which merges and writes out[h].
+//
+// The length advance: each CTA's producer lane, after its read of seq_lens,
+// counts the CTA in the append's completion counter (acq_rel); the last of
+// the grid's CTAs stores the advanced length and resets the counter.
+constexpr int kStepChunks = 4;  // A slice chunks per unit, each with its own barrier
+struct StepLayout {
+  size_t slice_k, slice_v, xs, slots, red, bar, pos, total;
+};
+__host__ __device__ inline StepLayout step_layout(size_t base, int Ec, int r, int w8, int csize) {
+  auto up = [](size_t v, size_t a) { return (v + a - 1) / a * a; };
+  StepLayout L;
+  const size_t sb = (size_t)Ec * r * (w8 ? 1 : 2);
+  size_t o = up(base, 128);
+  L.slice_k = o;
+  o = up(o + sb, 128);
+  L.slice_v = o;
+  o = up(o + sb, 128);
+  L.xs = o;
+  o = up(o + (size_t)Ec * 4, 16);
+  L.slots = o;  // [csize][K, V][r]
+  o = up(o + (size_t)csize * 2 * r * 4, 16);
+  L.red = o;
+  o = up(o + (size_t)kAppendWarps * 2 * r * 4, 16);
+  L.bar = o;
+  o += (2 * kStepChunks + 2) * 8;
+  L.pos = o;
+  o += 16;
+  L.total = up(o, 128);
+  return L;
+}
+
+template <int CODEC, int VPT, int TPT, bool W8>
+__global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const DecodeArgs a, const AppendArgs ap) {
+  using C = Cfg<CODEC, VPT, TPT, 1, 1>;
+  constexpr int W = C::kW, NP = VPT / 2;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank(), csize = (int)cluster.num_blocks();
+  const int h = blockIdx.y;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stage = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* segfull = full + 2;  // (full[1], empty[1], segfull, aux[4]) as in the cluster decode
+  uint64_t* aux = segfull + 1;   // [0]: B_Vh staged, [1]: decode partials landed (merging rank)
+  float* qs = reinterpret_cast<float*>(smem + C::kOffQ);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* res = reinterpret_cast<float*>(smem + C::kOffRes);
+  float* misc = reinterpret_cast<float*>(smem + C::kOffMisc);
+  uint32_t* planes = reinterpret_cast<uint32_t*>(smem + C::kOffParts);
+  uint8_t* segbuf = smem + C::cluster_seg_off();
+  float* slots = reinterpret_cast<float*>(segbuf + seg_bytes(kQProj, W, a.Hd));  // [csize][W + 2]
+  __half* bvs = reinterpret_cast<__half*>(slots + (size_t)kMaxClusterSize * (W + 2));
+
+  const int r = ap.r, E = ap.E, Ec = E / csize, e0 = rank * Ec;
+  const StepLayout L = step_layout(C::cluster_smem_bytes(kQProj, a.Hd), Ec, r, W8, csize);
+  uint8_t* slice_k = smem + L.slice_k;
+  uint8_t* slice_v = smem + L.slice_v;
+  float* xs = reinterpret_cast<float*>(smem + L.xs);
+  float* aslots = reinterpret_cast<float*>(smem + L.slots);
+  float* ared = reinterpret_cast<float*>(smem + L.red);
+  // [u * kStepChunks + c]: chunk c of slice u landed; then the ranks' partial
+  // rows landed (owner), and the length known
+  uint64_t* abar = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* bar_part = abar + 2 * kStepChunks;
+  uint64_t* bar_pos = bar_part + 1;
+  int* pos_sm = reinterpret_cast<int*>(smem + L.pos);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = ((a.L_cap + csize - 1) / csize + 7) & ~7;
+  const int lo = min(a.L_cap, rank * chunk), hi = min(a.L_cap, lo + chunk);
+  const uint32_t piece = (uint32_t)Ec * r * (W8 ? 1 : 2) / kStepChunks;  // bytes per slice chunk
+  const int piece_rows = Ec / kStepChunks;
+
+  if (tid == kConsumerThreads) {
+    mbar_init(&full[0], 1);
+    mbar_init(segfull, 1);
+    mbar_init(&aux[0], 1);
+    mbar_init(&aux[1], 1);
+    for (int i = 0; i < 2 * kStepChunks + 2; ++i) mbar_init(&abar[i], 1);
+    fence_mbar_init();
+  }
+  cluster_arrive_relaxed();  // barriers initialised; waited on before any remote access
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      const int pos = ld_relaxed_gpu(ap.seq_lens);  // consumed below: the copies are issued meanwhile
+      const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
+      const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), qb = (uint32_t)a.Hd * 2;
+      const uint16_t* qh = static_cast<const uint16_t*>(a.q) + (size_t)h * a.Hd;
+      mbar_arrive_expect_tx(segfull, bb + qb);
+      bulk_g2s(segbuf, static_cast<const uint8_t*>(a.Bk) + (size_t)h * bb, bb, segfull, keep);
+      if (!ap.dep) bulk_g2s(segbuf + bb, qh, qb, segfull, keep);
+      for (int u = 0; u < 2; ++u) {
+        const uint8_t* src = static_cast<const uint8_t*>(u ? ap.Av : ap.Ak) + ((size_t)h * E + e0) * r * (W8 ? 1 : 2);
+        uint8_t* dst = u ? slice_v : slice_k;
+        for (int c = 0; c < kStepChunks; ++c) {
+          mbar_arrive_expect_tx(&abar[u * kStepChunks + c], piece);
+          bulk_g2s(dst + (size_t)c * piece, src + (size_t)c * piece, piece, &abar[u * kStepChunks + c], once);
+        }
+      }
+      if (ap.dep) {
+        griddep_wait();  // the query is written by the preceding grid
+        bulk_g2s(segbuf + bb, qh, qb, segfull, keep);
+      }
+      const bool ok = pos >= 0 && pos < a.L_cap;
+      const int lead = ok ? pos / chunk : 0;                   // the owner, which also merges
+      const int len_old = ok ? pos : clamp_len(pos, a.L_cap);  // rows final before the step
+      const int n_old = max(0, min(hi, len_old) - lo);          // of them in this rank's chunk
+      if (rank == lead && csize > 1) {
+        // the other ranks' partial rows (some may have landed already)
+        if (ok) mbar_arrive_expect_tx(bar_part, (uint32_t)((csize - 1) * 2 * r * 4));
+        mbar_arrive_expect_tx(&aux[1], (uint32_t)((csize - 1) * (W + 2) * 4));
+      }
+      *pos_sm = pos;
+      mbar_arrive(bar_pos);
+      if (rank == lead) {
+        mbar_arrive_expect_tx(&aux[0], bb);
+        for (uint32_t off = 0; off < bb; off += 32768)
+          bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, static_cast<const uint8_t*>(a.Bv) + (size_t)h * bb + off,
+                   min(32768u, bb - off), &aux[0], keep);
+      }
+      // The cached rows are read after this CTA's A slices have landed: they
+      // are needed only after the projection, and would compete with it for
+      // HBM bandwidth.
+      bool done = true;
+      for (int i = 0; i < 2 * kStepChunks; ++i) done = mbar_wait_bounded(&abar[i], 0) && done;
+      if (n_old > 0) {
+        const size_t row0 = (size_t)h * a.L_cap + lo;
+        const uint32_t cbytes = (uint32_t)n_old * C::kRB, sbytes = (uint32_t)((n_old + 7) & ~7) * 2u;
+        mbar_arrive_expect_tx(&full[0], 2 * cbytes + 2 * sbytes);
+        bulk_g2s(stage, a.lat_k + row0 * C::kRB, cbytes, &full[0], once);
+        bulk_g2s(stage + C::kCodeBytes, a.lat_v + row0 * C::kRB, cbytes, &full[0], once);
+        bulk_g2s(stage + 2 * C::kCodeBytes, a.scale_k + row0, sbytes, &full[0], once);
+        bulk_g2s(stage + 2 * C::kCodeBytes + C::kScaleBytes, a.scale_v + row0, sbytes, &full[0], once);
+      } else {
+        mbar_arrive(&full[0]);
+      }
+      if (ok) {
+        // This CTA's read of the length is complete (its value was used above).
+        const int prev = atom_add_acq_rel_gpu(ap.counter, 1);
+        if (prev == (int)(gridDim.x * gridDim.y) - 1) {
+          st_relaxed_gpu(ap.seq_lens, pos + 1);
+          st_relaxed_gpu(ap.counter, 0);
+        }
+      }
+      // No copy may still be landing when the CTA exits (the consumers may have
+      // given up on a barrier).
+      done = mbar_wait_bounded(&full[0], 0) && mbar_wait_bounded(segfull, 0) && done;
+      if (rank == lead) done = mbar_wait_bounded(&aux[0], 0) && done;
+      if (!done) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+    }
+    cluster_wait();
+    return;
+  }
+
+  // ---- consumers
+  bool timed_out = false;
+  auto cwait = [&](uint64_t* bar, uint32_t parity, bool cluster_scope) {
+    const uint64_t lim = timed_out ? 0ull : kWaitLimitNs;
+    const bool got = cluster_scope ? mbar_wait_cluster_bounded(bar, parity, lim) : mbar_wait_bounded(bar, parity, lim);
+    if (!got) {
+      if (!timed_out && lane == 0) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+      timed_out = true;
+    }
+  };
+  auto consumer_sync = []() { csync(); };
+  // x slice of the append (registers on the fast path)
+  const bool fast = x_fast_path(1, Ec, ap.blk);
+  uint2 xraw[kXChunks];
+  if (ap.dep) griddep_wait();  // x is written by the preceding grid
+  if (fast) load_x_slice(xraw, ap.x, 1, E, e0, Ec, warp, lane);
+
+  // q' and its byte planes, the rotated x slice
+  const int sub = tid % TPT;
+  QState<CODEC, VPT> qst;
+  cwait(segfull, 0, false);
+  build_query<CODEC, VPT, W, kQProj>(qst, segbuf, qs, misc, planes, a, tid, sub);
+  rotate_x_slice(fast, xraw, xs, ap.x, ap.x_dtype, 1, E, e0, Ec, ap.blk, tid, consumer_sync);
+
+  cwait(bar_pos, 0, false);
+  const int pos = timed_out ? -1 : *pos_sm;
+  const bool ok = pos >= 0 && pos < a.L_cap;
+  const int lead = ok ? pos / chunk : 0;
+  const bool own = ok && rank == lead;
+  const int len_old = ok ? pos : clamp_len(pos, a.L_cap);
+  const int n_old = max(0, min(hi, len_old) - lo);
+  if (!ok && rank == 0 && h == 0 && tid == 0) {
+    set_err(a.err, WSVD_DEVERR_CACHE_FULL);
+    if (pos < 0 || pos > a.L_cap) set_err(a.err, WSVD_DEVERR_LEN_RANGE);
+  }
+  cluster_wait();  // every CTA of the cluster has initialised its barriers
+
+  // the append: K and V projections of this rank's E slice, chunk by chunk,
+  // reduced in one pass into the owner's slots [rank][K, V]
+  if (ok) {
+    const int ncg = r / 8, nrg = kAppendThreads / ncg, rg = tid / ncg, cgi = tid % ncg;
+    const int nrows = rg < Ec ? (Ec - 1 - rg) / nrg + 1 : 0;
+    float2 cacc[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cacc[u][k] = make_float2(0.f, 0.f);
+      const uint8_t* sl = u ? slice_v : slice_k;
+      float2 (&cu)[1][4] = *reinterpret_cast<float2 (*)[1][4]>(&cacc[u][0]);
+      int landed = 0, bound = 0;  // chunks of this slice known to have landed; rows below bound are in
+      for (int k = 0, e = rg; k < nrows; ++k, e += nrg) {
+        while (e >= bound) {
+          cwait(&abar[u * kStepChunks + landed++], 0, false);
+          bound += piece_rows;
+        }
+        uint4 av;
+        if (W8) {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(sl + (size_t)e * r + cgi * 8);
+          av = make_uint4(v2.x, v2.y, 0u, 0u);
+        } else {
+          av = *reinterpret_cast<const uint4*>(sl + ((size_t)e * r + cgi * 8) * 2);
+        }
+        accumulate_row<1, W8>(av, xs, 1, 0, Ec, e, cu);
+      }
+    }
+    const bool remote = rank != lead;
+    float* dst = aslots + (size_t)rank * 2 * r;
+    reduce_cta<2>(cacc, ncg, r, 2, ared, dst, remote ? mapa_shared(dst, lead) : 0u,
+                  remote ? mapa_shared(bar_part, lead) : 0u, tid, consumer_sync);
+  }
+
+  // the rows of the chunk that precede the new one
+  float2 acc[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) acc[p] = make_float2(0.f, 0.f);
+  float m = kNegInf, l = 0.f;
+  cwait(&full[0], 0, false);
+  if (n_old > 0 && !timed_out) process_tile<CODEC, VPT, TPT, 1>(stage, n_old, qst, m, l, acc, tid);
+
+  if (own) {
+    // quantise the new row (warp 0: K, warp 1: V) into the cache and the staged tile
+    const int t = pos - lo;
+    if (warp < 2) {
+      const int u = warp;
+      if (csize > 1) cwait(bar_part, 0, true);
+      const size_t row = (size_t)h * a.L_cap + pos;
+      const int RB = r * ap.bits / 8;
+      uint8_t* tile_codes = stage + (size_t)u * C::kCodeBytes + (size_t)t * C::kRB;
+      const __half sh = quantise_append_row<W8>(aslots + (size_t)u * r, (size_t)2 * r, csize, r, ap.bits, ap.hnorm,
+                                                W8 ? (u ? ap.sAv : ap.sAk) + (size_t)h * r : nullptr, true,
+                                                (u ? ap.lat_v : ap.lat_k) + row * RB, tile_codes, lane);
+      if (lane == 0) {
+        (u ? ap.scale_v : ap.scale_k)[row] = sh;
+        reinterpret_cast<__half*>(stage + 2 * C::kCodeBytes + (size_t)u * C::kScaleBytes)[t] = sh;
+      }
+    }
+    csync();  // the new row is in the tile
+    if (!timed_out) process_tile<CODEC, VPT, TPT, 1>(stage, t + 1, qst, m, l, acc, tid, t);
+  }
+  reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
+  if (rank != lead) {
+    // Partial row straight into the merging rank's slot; each store completes
+    // its bytes on that rank's barrier.
+    const uint32_t rslot = mapa_shared(slots + (size_t)rank * (W + 2), lead), rbar = mapa_shared(&aux[1], lead);
+    for (int e = tid; e < W + 2; e += kConsumerThreads) st_async_f32(rslot + 4u * e, res[e], rbar);
+    return;
+  }
+
+  // the merging rank: the ranks' partials in rank order, up-projected through B_Vh
+  if (csize > 1) {
+    for (int e = tid; e < W + 2; e += kConsumerThreads) slots[(size_t)rank * (W + 2) + e] = res[e];
+    if (tid == 0 && !mbar_wait_cluster_bounded(&aux[1], 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+    csync();
+    merge_rows<W, false>(slots, csize, res, tid);
+  }
+  if (!mbar_wait_bounded(&aux[0], 0, timed_out ? 0ull : kWaitLimitNs) && lane == 0)
+    set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
+  const BvRef Bvh{bvs, a.w8, a.w8 ? a.sBv + (size_t)h * a.Hd : nullptr};
+  finalize_out<W>(res, Bvh, a.out + (size_t)h * a.Hd, a.Hd, red, tid);
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
@@ -1598,6 +1922,52 @@ bool plan_decode(int codec, int rowbytes, int qmode, const DecodeArgs& a, Plan* 
   return true;
 }
 
+
+// ---- one-kernel step: instantiated shapes (one token per lane and tile, r = 32)
+using StepFn = void (*)(const DecodeArgs, const AppendArgs);
+struct StepInfo {
+  StepFn fn;
+  int tile, rb;
+  size_t (*base)(int qmode, int Hd);  // the cluster decode's part of the shared memory
+};
+template <int CODEC, int VPT, int TPT, bool W8>
+StepInfo step_info() {
+  using C = Cfg<CODEC, VPT, TPT, 1, 1>;
+  return StepInfo{&step_cluster_kernel<CODEC, VPT, TPT, W8>, C::kT, C::kRB, &C::cluster_smem_bytes};
+}
+bool pick_step(int codec, int rowbytes, bool w8, StepInfo* si) {
+  if (codec == kCodecI8 && rowbytes == 32) {
+    *si = w8 ? step_info<kCodecI8, 32, 1, true>() : step_info<kCodecI8, 32, 1, false>();
+    return true;
+  }
+  if (codec == kCodecI4 && rowbytes == 16) {
+    *si = w8 ? step_info<kCodecI4, 32, 1, true>() : step_info<kCodecI4, 32, 1, false>();
+    return true;
+  }
+  return false;
+}
+struct StepPlan {
+  StepInfo si;
+  int csize;
+  size_t smem;
+};
+// The one-kernel step applies to one sequence whose decode takes the cluster
+// path with the append's cluster size, each rank's chunk within one tile, and
+// a shared-memory footprint that leaves two CTAs per SM.
+bool plan_step(const AppendArgs& ap, const DecodeArgs& a, StepPlan* sp) {
+  if (ap.B != 1 || a.B != 1 || a.H != ap.H || a.W != ap.r || a.L_cap != ap.L_cap || a.L_cap < 8 || a.H > 65535)
+    return false;
+  const int codec = ap.bits == 8 ? kCodecI8 : kCodecI4, rowbytes = ap.r * ap.bits / 8;
+  if (!pick_step(codec, rowbytes, ap.w8 != 0, &sp->si) || sp->si.rb != rowbytes || a.w8 != ap.w8) return false;
+  Plan pl;
+  if (!plan_decode(codec, rowbytes, kQProj, a, &pl) || !pl.cluster || pl.csize != ap.cluster) return false;
+  const int cs = ap.cluster;
+  const int chunk = ((a.L_cap + cs - 1) / cs + 7) & ~7;
+  if (chunk > sp->si.tile) return false;
+  sp->csize = cs;
+  sp->smem = step_layout(sp->si.base(kQProj, a.Hd), ap.E / cs, ap.r, ap.w8, cs).total;
+  return sp->smem <= 113 * 1024;
+}
 }  // namespace
 
 bool decode_supported(int codec, int rowbytes, int qmode) {
@@ -1660,6 +2030,36 @@ cudaError_t launch_decode(int codec, int rowbytes, int qmode, DecodeArgs a, cuda
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelExC(&cfg, pl.ki.fn, args);
+}
+
+bool step_fused_applies(const AppendArgs& ap, const DecodeArgs& a) {
+  StepPlan sp;
+  return plan_step(ap, a, &sp);
+}
+
+cudaError_t launch_step_fused(const AppendArgs& ap, const DecodeArgs& a, cudaStream_t stream, bool* launched) {
+  *launched = false;
+  StepPlan sp;
+  if (!plan_step(ap, a, &sp)) return cudaSuccess;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(sp.si.fn), sp.smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sp.csize, a.H, 1);
+  cfg.blockDim = dim3(kDecodeThreads, 1, 1);
+  cfg.dynamicSmemBytes = sp.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = sp.csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ap.dep ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, sp.si.fn, a, ap);
+  if (e == cudaSuccess) *launched = true;
+  return e;
 }
 
 }  // namespace wsvd

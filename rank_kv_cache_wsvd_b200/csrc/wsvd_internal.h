@@ -98,5 +98,11 @@ int decode_with_scratch(int B, int H, int Hd, int r, int bits, int L_cap, const 
                         void* scratch, size_t scratch_bytes, int32_t* err, cudaStream_t stream);
 size_t append_smem_bytes(int B, int E, int r, int cluster);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+// The append and the decode of one step as one cluster grid (decode.cu), for
+// one sequence on the cluster decode path; same results as launch_append then
+// launch_decode(after_append).  When the shapes do not allow it nothing is
+// queued and *launched is false.
+bool step_fused_applies(const AppendArgs& ap, const DecodeArgs& a);
+cudaError_t launch_step_fused(const AppendArgs& ap, const DecodeArgs& a, cudaStream_t stream, bool* launched);
 
 }  // namespace wsvd

@@ -96,6 +96,9 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.wsvd_latent_append(1, 4, 256, 16, 8, 8, 96, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 1
     assert lib.wsvd_latent_append(1, 4, 200, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 1
     assert lib.wsvd_latent_append(17, 4, 256, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 2
+    # r / 8 column groups must divide a warp: r = 24 or 40 is rejected
+    for r in (24, 40):
+        assert lib.wsvd_latent_append(1, 4, 256, r, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 256, None, None) == 2
     assert lib.wsvd_latent_append(1, 4, 256, 16, 8, 8, 128, p, 1, p, p, p, p, p, p, p, p, 8, None, None) == 4
     # dense / shared: unsupported widths
     assert lib.dense_decode_attention(1, 4, 48, 256, p, p, 0, p, p, 0.0, p, p, 1 << 22, None, None) == 2
@@ -109,6 +112,15 @@ def test_decode_launch_count_rejects_bad_sizes(lib):
     assert W.wsvd_decode_launch_count(1, 32, 128, 32, 5, 1600) == 0
     assert W.wsvd_decode_launch_count(1, 32, 128, 3, 4, 1600) == 0  # r * bits not a whole byte
     assert W.wsvd_decode_launch_count(1, 32, 128, 24, 8, 1600) == 0  # 24-byte rows are not instantiated
+
+
+def test_step_launch_count_rejects_bad_sizes(lib):
+    """wsvd_step_launch_count answers 0 for sizes the step would reject."""
+    assert W.wsvd_step_launch_count(0, 32, 128, 4096, 32, 8, 1600) == 0
+    assert W.wsvd_step_launch_count(1, 32, 128, 4096, 32, 5, 1600) == 0
+    assert W.wsvd_step_launch_count(1, 32, 128, 4096, 32, 8, 1600, hadamard_block=96) == 0  # not a power of two
+    assert W.wsvd_step_launch_count(1, 32, 128, 4000, 32, 8, 1600) == 0  # E not a multiple of the block
+    assert W.wsvd_step_launch_count(1, 32, 128, 4096, 24, 8, 1600) == 0  # 24-byte rows are not instantiated
 
 
 def test_prefill_workspace_and_host_validation(lib):

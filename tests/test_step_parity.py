@@ -1,8 +1,9 @@
-"""The one-call decode step, wsvd_append_and_decode: the latent append, then the
-decode launched behind it as a programmatic dependent (its launch and query
-projection overlap the append).  Its results must be those of the two calls
-made one after the other, bit for bit (cache rows, scales, lengths, output),
-and the oracle's two steps within the attention tolerance."""
+"""The one-call decode step, wsvd_append_and_decode: one kernel that appends
+and attends (one sequence on the cluster decode path), or the latent append
+followed by the decode launched behind it as a programmatic dependent.  Its
+results must be those of the two calls made one after the other, bit for bit
+(cache rows, scales, lengths, output), and the oracle's two steps within the
+attention tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -15,8 +16,20 @@ from oracle import wsvd_oracle as O
 pytestmark = pytest.mark.gpu
 
 CASES = {
-    # cluster decode path (few tiles), B = 1
+    # one kernel (cluster decode path, B = 1): the new row in the last rank's chunk
     "llava7b": (WL.LLAVA7B.with_(L_cap=1608), [1599]),
+    # one kernel: the new row is the first of rank 7's chunk (no cached rows before it there)
+    "llava7b-chunk-start": (WL.LLAVA7B, [1400]),
+    # one kernel: rank 4 owns the new row, ranks 5-7 hold no rows
+    "llava7b-middle": (WL.LLAVA7B, [803]),
+    # one kernel: empty cache, rank 0 (which also merges) owns the only row
+    "llava7b-first-row": (WL.LLAVA7B, [0]),
+    # one kernel, int4 cache, fp16 query
+    "int4-one-kernel": (WL.RAGGED.with_(B=1, H=8, E=2048, L_cap=1024), [700]),
+    # one kernel, two-CTA clusters (E 512 with 256-wide Hadamard blocks), x rotated in shared memory
+    "two-rank": (WL.PR1.with_(r=32, E=512, hadamard_block=256, L_cap=256), [77]),
+    # one kernel, one CTA per head
+    "one-rank": (WL.PR1.with_(r=32, E=256, hadamard_block=256, L_cap=128), [100]),
     # persistent decode path, a length at the last free row and a short one
     "long-r32": (WL.LONG[32].with_(L_cap=8192), [8000, 8191, 100, 4095]),
     # int4 cache, fp16 query, ragged lengths
@@ -71,6 +84,51 @@ def test_step_equals_append_then_decode(name):
     ref = O.wsvd_decode(d.q, lk, sk, lv, sv, d.Bk, d.Bv, nl, w.r, w.bits)
     assert np.array_equal(one["lens"].cpu().numpy(), np.asarray(lens0) + 1)
     assert_attention_close(out1.cpu().numpy(), ref, f"step {name}")
+
+
+ONE_KERNEL = ("llava7b", "llava7b-chunk-start", "llava7b-middle", "llava7b-first-row", "int4-one-kernel", "two-rank",
+              "one-rank")
+
+
+def test_step_launch_count_matches_the_path():
+    """One kernel for the single-sequence cluster-path cases, the append plus
+    the decode's launches otherwise."""
+    lc = W.wsvd_step_launch_count
+    for name, (w, _) in CASES.items():
+        n = lc(w.B, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block)
+        dn = W.wsvd_decode_launch_count(w.B, w.H, w.Hd, w.r, w.bits, w.L_cap)
+        assert n == (1 if name in ONE_KERNEL else 1 + dn), name
+    w = WL.LLAVA7B
+    assert lc(w.B, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block, w8=True) == 1
+    assert lc(2, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block) == 2  # two sequences: append + decode
+    assert lc(1, w.H, w.Hd, w.E, 16, w.bits, w.L_cap, w.hadamard_block) == 2  # two tokens per lane and tile
+    assert lc(0, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block) == 0
+
+
+@pytest.mark.parametrize("start", ["full", "negative"])
+def test_step_with_no_free_row_equals_the_two_calls(start):
+    """A full cache (length L_cap) or an invalid length: nothing is appended,
+    the error bits and the output are those of the two calls."""
+    w = WL.LLAVA7B
+    d, ai = _inputs(w, [w.L_cap - 1], seed=5)
+    d.seq_lens[:] = w.L_cap if start == "full" else -3
+    x = q_tensor(ai.x_bits[0], "bf16")
+    A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
+    q = q_tensor(d.q_bits, w.q_dtype)
+    two, one = _device_state(d), _device_state(d)
+    err2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    err1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    W.wsvd_latent_append(x, A_k, A_v, two["lens"], two["lat_k"], two["lat_v"], two["sk"], two["sv"], bits=w.bits,
+                         err=err2)
+    out2 = W.wsvd_decode_attention(q, two["lat_k"], two["lat_v"], two["sk"], two["sv"], B_k, B_v, two["lens"],
+                                   bits=w.bits, err=err2)
+    out1 = W.wsvd_append_and_decode(x, A_k, A_v, one["lens"], one["lat_k"], one["lat_v"], one["sk"], one["sv"], q,
+                                    B_k, B_v, bits=w.bits, err=err1)
+    torch.cuda.synchronize()
+    assert int(err1.item()) == int(err2.item()) != 0
+    for k in ("lat_k", "lat_v", "sk", "sv", "lens"):
+        assert torch.equal(one[k], two[k]), k
+    assert torch.equal(out1, out2)
 
 
 def test_step_validates_before_launching():

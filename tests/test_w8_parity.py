@@ -74,7 +74,9 @@ def test_w8_append_matches_oracle(name, w, lens0):
 
 
 def test_w8_step_equals_the_two_w8_calls_and_the_oracle():
-    for w, lens0 in ((WL.LLAVA7B.with_(L_cap=1608), [1599]),                    # cluster decode
+    w = WL.LLAVA7B
+    assert W.wsvd_step_launch_count(w.B, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block, w8=True) == 1
+    for w, lens0 in ((WL.LLAVA7B.with_(L_cap=1608), [1599]),                    # one kernel (cluster decode)
                      (WL.LONG[32].with_(L_cap=8192), [8000, 8191, 100, 4095])):  # split-L grid
         d = WL.decode_inputs(w, seed=21, lens=np.asarray(lens0) + 1)
         for b, n in enumerate(lens0):
