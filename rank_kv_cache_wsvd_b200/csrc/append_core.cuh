@@ -274,7 +274,9 @@ __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t
     cv[k] = 0.f;
     if (j < r) {
       float sum = 0.f;
-      for (int q = 0; q < nranks; ++q) sum += slots[(size_t)q * stride + j];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)  // clusters hold at most 8 ranks
+        if (q < nranks) sum += slots[(size_t)q * stride + j];
       cv[k] = sum * hnorm;
       if (W8) cv[k] *= colscale[j];  // column scale of int8 A
       amax = fmaxf(amax, fabsf(cv[k]));

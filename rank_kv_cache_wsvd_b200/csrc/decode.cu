@@ -1533,7 +1533,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
   float* slots = reinterpret_cast<float*>(segbuf + seg_bytes(kQProj, W, a.Hd));  // [csize][W + 2]
   __half* bvs = reinterpret_cast<__half*>(slots + (size_t)kMaxClusterSize * (W + 2));
 
-  const int r = ap.r, E = ap.E, Ec = E / csize, e0 = rank * Ec;
+  constexpr int r = W;  // the latent width (the host launches this kernel only when r == W)
+  const int E = ap.E, Ec = E / csize, e0 = rank * Ec;
   const StepLayout L = step_layout(C::cluster_smem_bytes(kQProj, a.Hd), Ec, r, W8, csize);
   uint8_t* slice_k = smem + L.slice_k;
   uint8_t* slice_v = smem + L.slice_v;
@@ -1703,8 +1704,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
     }
     const bool remote = rank != lead;
     float* dst = aslots + (size_t)rank * 2 * r;
-    reduce_cta<2>(cacc, ncg, r, 2, ared, dst, remote ? mapa_shared(dst, lead) : 0u,
-                  remote ? mapa_shared(bar_part, lead) : 0u, tid, consumer_sync);
+    reduce_cta_n<2, W / 8>(cacc, W, 2, ared, dst, remote ? mapa_shared(dst, lead) : 0u,
+                           remote ? mapa_shared(bar_part, lead) : 0u, tid, consumer_sync);
   }
 
   // the rows of the chunk that precede the new one
