@@ -260,16 +260,18 @@ __device__ __forceinline__ void rotate_x_slice(bool fast, const uint2 (&xraw)[kX
 // ranks' partial sums (slots[q * stride + j], q = 0 .. nranks - 1) added in
 // rank order, times 1/sqrt(blk) (and the int8 weights' column scale), then the
 // append's fp32 decisions; the codes are written to dst when `ok` (and to
-// dst2 too, when given).  Returns the fp16 scale.
-template <bool W8>
+// dst2 too, when given).  Returns the fp16 scale.  RMAX: a bound on r known
+// at compile time (128 covers every r; a caller with a fixed r passes it).
+template <bool W8, int RMAX = 128>
 __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t stride, int nranks, int r, int bits,
                                                       float hnorm, const float* colscale, bool ok, uint8_t* dst,
                                                       uint8_t* dst2, int lane) {
+  constexpr int KMAX = (RMAX + 31) / 32;  // column groups of 32 a lane may hold
   const int Q = (bits == 8) ? 127 : 7;
-  float cv[4];
+  float cv[KMAX];
   float amax = 0.f;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < KMAX; ++k) {
     const int j = lane + 32 * k;
     cv[k] = 0.f;
     if (j < r) {
@@ -287,7 +289,7 @@ __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t
   const __half sh = __float2half_rn(__fdiv_rn(amax, (float)Q));
   const float sc = __half2float(sh);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < KMAX; ++k) {
     if (32 * k >= r) break;  // no column of this group (uniform across the warp)
     const int j = lane + 32 * k;
     const int code = sc > 0.f ? max(-Q, min(Q, __float2int_rn(__fdiv_rn(cv[k], sc)))) : 0;

@@ -626,19 +626,32 @@ __device__ __forceinline__ void reduce_to_res(float m, float l, float2* acc, flo
 template <int W, bool GLOBAL>
 __device__ __forceinline__ float merge_elem(const float* part, int np, float M, int e) {
   float s2 = 0.f;
-  for (int p = 0; p < np; ++p) {
+  auto term = [&](int p) {
     const float mp = GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)];
     if (mp != kNegInf) {
       const float v = GLOBAL ? __ldcg(part + (size_t)p * (W + 2) + 1 + e) : part[(size_t)p * (W + 2) + 1 + e];
       s2 = fmaf(ex2(mp - M), v, s2);
     }
+  };
+  if constexpr (GLOBAL) {
+    for (int p = 0; p < np; ++p) term(p);
+  } else {  // a cluster's ranks: at most kMaxClusterSize rows, unrolled (same order)
+#pragma unroll
+    for (int p = 0; p < kMaxClusterSize; ++p)
+      if (p < np) term(p);
   }
   return s2;
 }
 template <int W, bool GLOBAL>
 __device__ __forceinline__ float merge_max(const float* part, int np) {
   float M = kNegInf;
-  for (int p = 0; p < np; ++p) M = fmaxf(M, GLOBAL ? __ldcg(part + (size_t)p * (W + 2)) : part[(size_t)p * (W + 2)]);
+  if constexpr (GLOBAL) {
+    for (int p = 0; p < np; ++p) M = fmaxf(M, __ldcg(part + (size_t)p * (W + 2)));
+  } else {
+#pragma unroll
+    for (int p = 0; p < kMaxClusterSize; ++p)
+      if (p < np) M = fmaxf(M, part[(size_t)p * (W + 2)]);
+  }
   return M;
 }
 // Thread-block version (consumer threads).
@@ -1725,7 +1738,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
       const size_t row = (size_t)h * a.L_cap + pos;
       const int RB = r * ap.bits / 8;
       uint8_t* tile_codes = stage + (size_t)u * C::kCodeBytes + (size_t)t * C::kRB;
-      const __half sh = quantise_append_row<W8>(aslots + (size_t)u * r, (size_t)2 * r, csize, r, ap.bits, ap.hnorm,
+      const __half sh = quantise_append_row<W8, W>(aslots + (size_t)u * r, (size_t)2 * r, csize, r, ap.bits, ap.hnorm,
                                                 W8 ? (u ? ap.sAv : ap.sAk) + (size_t)h * r : nullptr, true,
                                                 (u ? ap.lat_v : ap.lat_k) + row * RB, tile_codes, lane);
       if (lane == 0) {
@@ -1734,7 +1747,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
       }
     }
     csync();  // the new row is in the tile
-    if (!timed_out) process_tile<CODEC, VPT, TPT, 1>(stage, t + 1, qst, m, l, acc, tid, t);
+    // Only the warp holding the new token's lanes has a valid token in this
+    // pass; the other lanes' states would not change.
+    if (!timed_out && warp == (t * TPT) / 32) process_tile<CODEC, VPT, TPT, 1>(stage, t + 1, qst, m, l, acc, tid, t);
   }
   reduce_to_res<VPT, TPT, W, C::kNSeg>(m, l, acc, red, res, tid);
   if (rank != lead) {
