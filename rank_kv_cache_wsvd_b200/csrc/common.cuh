@@ -191,11 +191,6 @@ __device__ __forceinline__ float lds_half_as_float(uint32_t addr) {
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-// Release form: this thread's earlier memory accesses happen before whatever
-// the other CTAs do after their cluster_wait.
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
