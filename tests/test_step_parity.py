@@ -131,6 +131,38 @@ def test_step_with_no_free_row_equals_the_two_calls(start):
     assert torch.equal(out1, out2)
 
 
+@pytest.mark.parametrize("name", ["llava7b", "llava7b-chunk-start", "int4-one-kernel"])
+def test_step_ignores_rows_at_and_past_the_new_one(name):
+    """Rows from the new token's position on (the row the append writes, and
+    the cache's unused tail) hold random bytes: the step's output and the
+    rows it writes are those of a clean cache, bit for bit, and every byte
+    past the new row is left as it was."""
+    w, lens0 = CASES[name]
+    d, ai = _inputs(w, lens0, seed=41)
+    x = q_tensor(ai.x_bits[0], "bf16")
+    A_k, A_v, B_k, B_v = dev(ai.A_k), dev(ai.A_v), dev(d.Bk), dev(d.Bv)
+    q = q_tensor(d.q_bits, w.q_dtype)
+    clean = _device_state(d)
+    g = np.random.default_rng(7)
+    for b, n in enumerate(lens0):
+        for a in (d.lat_k, d.lat_v):
+            a[b, :, n:] = g.integers(0, 256, size=a[b, :, n:].shape, dtype=np.uint8)
+        for a in (d.scale_k, d.scale_v):
+            a[b, :, n:] = g.standard_normal(a[b, :, n:].shape).astype(np.float16) * 1e4
+    dirty = _device_state(d)
+    outs = [W.wsvd_append_and_decode(x, A_k, A_v, st["lens"], st["lat_k"], st["lat_v"], st["sk"], st["sv"], q, B_k,
+                                     B_v, bits=w.bits, hadamard_block=w.hadamard_block) for st in (clean, dirty)]
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]), name
+    for k in ("lat_k", "lat_v", "sk", "sv"):
+        for b, n in enumerate(lens0):
+            assert torch.equal(clean[k][b, :, :n + 1], dirty[k][b, :, :n + 1]), (name, k)
+    after = _device_state(d)  # the poisoned inputs, untouched
+    for k in ("lat_k", "lat_v", "sk", "sv"):
+        for b, n in enumerate(lens0):
+            assert torch.equal(dirty[k][b, :, n + 1:], after[k][b, :, n + 1:]), (name, k)
+
+
 def test_step_validates_before_launching():
     w, lens0 = CASES["llava7b"]
     d, ai = _inputs(w, lens0, seed=3)
