@@ -22,6 +22,8 @@ CASES = {
     "llava7b-chunk-start": (WL.LLAVA7B, [1400]),
     # one kernel: rank 4 owns the new row, ranks 5-7 hold no rows
     "llava7b-middle": (WL.LLAVA7B, [803]),
+    # one kernel: the new row is the last of rank 6's chunk (the last lane of the tile)
+    "llava7b-chunk-end": (WL.LLAVA7B, [1399]),
     # one kernel: empty cache, rank 0 (which also merges) owns the only row
     "llava7b-first-row": (WL.LLAVA7B, [0]),
     # one kernel, int4 cache, fp16 query
@@ -86,8 +88,8 @@ def test_step_equals_append_then_decode(name):
     assert_attention_close(out1.cpu().numpy(), ref, f"step {name}")
 
 
-ONE_KERNEL = ("llava7b", "llava7b-chunk-start", "llava7b-middle", "llava7b-first-row", "int4-one-kernel", "two-rank",
-              "one-rank")
+ONE_KERNEL = ("llava7b", "llava7b-chunk-start", "llava7b-middle", "llava7b-chunk-end", "llava7b-first-row",
+              "int4-one-kernel", "two-rank", "one-rank")
 
 
 def test_step_launch_count_matches_the_path():
@@ -195,7 +197,8 @@ def test_decode_launch_count_matches_the_path():
 
 @pytest.mark.parametrize("name,memory", [("llava7b", "pinned"), ("llava7b", "pinned-one-buffer"),
                                          ("llava7b", "pinned-direct"), ("llava7b", "pageable"), ("long-r32", "pinned"),
-                                         ("ragged-int4", "pinned"), ("ragged-int4", "pinned-direct")])
+                                         ("ragged-int4", "pinned"), ("ragged-int4", "pinned-direct"),
+                                         ("int4-one-kernel", "pinned"), ("int4-one-kernel", "pinned-direct")])
 def test_step_from_host_buffers_equals_device_step(name, memory):
     """wsvd_append_and_decode_host gives bit for bit what wsvd_append_and_decode
     gives on the same values already on the device, on two steps in a row

@@ -76,7 +76,10 @@ def test_w8_append_matches_oracle(name, w, lens0):
 def test_w8_step_equals_the_two_w8_calls_and_the_oracle():
     w = WL.LLAVA7B
     assert W.wsvd_step_launch_count(w.B, w.H, w.Hd, w.E, w.r, w.bits, w.L_cap, w.hadamard_block, w8=True) == 1
+    w4 = WL.RAGGED.with_(B=1, H=8, E=2048, L_cap=1024)
+    assert W.wsvd_step_launch_count(w4.B, w4.H, w4.Hd, w4.E, w4.r, w4.bits, w4.L_cap, w4.hadamard_block, w8=True) == 1
     for w, lens0 in ((WL.LLAVA7B.with_(L_cap=1608), [1599]),                    # one kernel (cluster decode)
+                     (WL.RAGGED.with_(B=1, H=8, E=2048, L_cap=1024), [700]),     # one kernel, int4 cache
                      (WL.LONG[32].with_(L_cap=8192), [8000, 8191, 100, 4095])):  # split-L grid
         d = WL.decode_inputs(w, seed=21, lens=np.asarray(lens0) + 1)
         for b, n in enumerate(lens0):
