@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include <map>
+#include <type_traits>
 #include <mutex>
 
 #include "append_core.cuh"
@@ -64,12 +65,14 @@ static __host__ __device__ inline AppendSmem append_layout(int B, int Ec, int r,
   return s;
 }
 
-template <int BB, bool W8>
+// R: the latent width, a compile-time constant of each instantiation.
+template <int BB, bool W8, int R>
 __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_group& cluster, uint8_t* smem,
                                             const AppendSmem& L) {
   const int rank = (int)cluster.block_rank();
   const int unit = blockIdx.y, h = unit >> 1, kv = unit & 1;
-  const int B = a.B, r = a.r, E = a.E;
+  constexpr int r = R;
+  const int B = a.B, E = a.E;
   const int Ec = E / a.cluster, e0 = rank * Ec;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint4* ring = reinterpret_cast<uint4*>(smem + L.ring_off);
@@ -125,8 +128,8 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     }
     float2 acc[BB][4];
     stream_rows<BB, W8>(w, ring, xs, B, bb0, acc, tid);
-    reduce_cta<BB>(acc, ncg, r, min(BB, B - bb0), red, slots + (size_t)bb0 * r, remote_slot + 4u * bb0 * r,
-                   remote_bar, tid, block_sync);
+    reduce_cta<BB, R / 8>(acc, r, min(BB, B - bb0), red, slots + (size_t)bb0 * r, remote_slot + 4u * bb0 * r,
+                          remote_bar, tid, block_sync);
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   // The A stream is done: a decode launched behind this kernel may now be
@@ -162,7 +165,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     const int pos = pos_sm[b];
     const bool ok = pos >= 0 && pos < a.L_cap;
     const size_t row = ((size_t)b * a.H + h) * a.L_cap + (ok ? pos : 0);
-    const __half sh = quantise_append_row<W8>(slots + (size_t)b * r, (size_t)B * r, a.cluster, r, a.bits, a.hnorm,
+    const __half sh = quantise_append_row<W8, R>(slots + (size_t)b * r, (size_t)B * r, a.cluster, r, a.bits, a.hnorm,
                                               W8 ? (kv ? a.sAv : a.sAk) + (size_t)h * r : nullptr, ok,
                                               (kv ? a.lat_v : a.lat_k) + row * RB, nullptr, lane);
     if (lane == 0) {
@@ -178,9 +181,21 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_kernel(const AppendA
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const AppendSmem L = append_layout(a.B, a.E / a.cluster, a.r, a.cluster);
-  if (a.B == 1) append_body<1, W8>(a, cluster, smem, L);
-  else if (a.B == 2) append_body<2, W8>(a, cluster, smem, L);
-  else append_body<4, W8>(a, cluster, smem, L);
+  // One body per latent width (r is 8, 16, 32, 64 or 128): the row walk, the
+  // reduction and the quantiser are then fixed at compile time.
+  auto run = [&](auto rtag) {
+    constexpr int R = decltype(rtag)::value;
+    if (a.B == 1) append_body<1, W8, R>(a, cluster, smem, L);
+    else if (a.B == 2) append_body<2, W8, R>(a, cluster, smem, L);
+    else append_body<4, W8, R>(a, cluster, smem, L);
+  };
+  switch (a.r) {
+    case 8: run(std::integral_constant<int, 8>{}); break;
+    case 16: run(std::integral_constant<int, 16>{}); break;
+    case 32: run(std::integral_constant<int, 32>{}); break;
+    case 64: run(std::integral_constant<int, 64>{}); break;
+    default: run(std::integral_constant<int, 128>{}); break;
+  }
 }
 
 int append_cluster_size(int E, int blk) {

@@ -118,8 +118,14 @@ __device__ __forceinline__ int reduce_scatter_lanes(float* v, int lane) {
   }
 }
 
+// Reduce acc over the CTA (threads sharing a column group, then warps) into
+// the slot rows bi < nb: a local store on the leader (remote_bar == 0), else an
+// st.async into the leader's slot at cluster address remote_dst that completes
+// 4 bytes per value on the leader's barrier.  Fixed summation order: within a
+// warp the butterfly over the lanes of a column group (partners at offsets
+// NCG, 2 NCG, ..., 16), then the warps in order.  NCG = r / 8 divides 32.
 template <int BB, int NCG, typename Sync>
-__device__ __forceinline__ void reduce_cta_n(float2 (&acc)[BB][4], int r, int nb, float* red, float* dst,
+__device__ __forceinline__ void reduce_cta(float2 (&acc)[BB][4], int r, int nb, float* red, float* dst,
                                              uint32_t remote_dst, uint32_t remote_bar, int tid, Sync sync) {
   constexpr int NV = BB * 8;
   constexpr int ROUNDS = NCG == 1 ? 5 : NCG == 2 ? 4 : NCG == 4 ? 3 : NCG == 8 ? 2 : 1;
@@ -151,23 +157,6 @@ __device__ __forceinline__ void reduce_cta_n(float2 (&acc)[BB][4], int r, int nb
   sync();
 }
 
-// Reduce acc over the CTA (threads sharing a column group, then warps) into
-// the slot rows bi < nb: a local store on the leader (remote_bar == 0), else an
-// st.async into the leader's slot at cluster address remote_dst that completes
-// 4 bytes per value on the leader's barrier.  Fixed summation order: within a
-// warp the butterfly over the lanes of a column group (partners at offsets
-// ncg, 2 ncg, ..., 16), then the warps in order.  ncg = r / 8 divides 32.
-template <int BB, typename Sync>
-__device__ __forceinline__ void reduce_cta(float2 (&acc)[BB][4], int ncg, int r, int nb, float* red, float* dst,
-                                           uint32_t remote_dst, uint32_t remote_bar, int tid, Sync sync) {
-  switch (ncg) {
-    case 1: reduce_cta_n<BB, 1>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
-    case 2: reduce_cta_n<BB, 2>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
-    case 4: reduce_cta_n<BB, 4>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
-    case 8: reduce_cta_n<BB, 8>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
-    default: reduce_cta_n<BB, 16>(acc, r, nb, red, dst, remote_dst, remote_bar, tid, sync); break;
-  }
-}
 
 __device__ __forceinline__ float x_elem(uint32_t bits16, int dtype) {
   return dtype == WSVD_DTYPE_BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((uint16_t)bits16));

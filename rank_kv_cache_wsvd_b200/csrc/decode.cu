@@ -1717,8 +1717,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
     }
     const bool remote = rank != lead;
     float* dst = aslots + (size_t)rank * 2 * r;
-    reduce_cta_n<2, W / 8>(cacc, W, 2, ared, dst, remote ? mapa_shared(dst, lead) : 0u,
-                           remote ? mapa_shared(bar_part, lead) : 0u, tid, consumer_sync);
+    reduce_cta<2, W / 8>(cacc, W, 2, ared, dst, remote ? mapa_shared(dst, lead) : 0u,
+                         remote ? mapa_shared(bar_part, lead) : 0u, tid, consumer_sync);
   }
 
   // the rows of the chunk that precede the new one

@@ -99,7 +99,7 @@ def test_long_context_64_steps(r):
     assert list(g["lens"].cpu().numpy()) == [74, 164, 214, 256]
 
 
-@pytest.mark.parametrize("bits,r", [(4, 32), (4, 64), (8, 128)])
+@pytest.mark.parametrize("bits,r", [(8, 8), (4, 16), (8, 16), (4, 32), (4, 64), (8, 128)])
 def test_formats(bits, r):
     w = WL.Workload("fmt", B=3, H=4, Hd=128, r=r, bits=bits, L_cap=16, lens=0, E=1024)
     ties, err, *_ = _run_steps(w, 4, [0, 5, 11], bits=bits)
