@@ -28,7 +28,6 @@
 #include <cooperative_groups.h>
 
 #include <map>
-#include <type_traits>
 #include <mutex>
 
 #include "append_core.cuh"
@@ -175,27 +174,19 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   }
 }
 
-// One kernel per weight format, so that each gets its own register allocation.
-template <bool W8>
+// One kernel per weight format and latent width (r is 8, 16, 32, 64 or 128):
+// each gets its own register allocation, the row walk, the reduction and the
+// quantiser are fixed at compile time, and each kernel holds only its own
+// bodies (a kernel with every width's bodies measured instruction-fetch
+// stalls at thirteen cycles per issued instruction).
+template <bool W8, int R>
 __global__ void __launch_bounds__(kAppendThreads, 4) append_kernel(const AppendArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
-  const AppendSmem L = append_layout(a.B, a.E / a.cluster, a.r, a.cluster);
-  // One body per latent width (r is 8, 16, 32, 64 or 128): the row walk, the
-  // reduction and the quantiser are then fixed at compile time.
-  auto run = [&](auto rtag) {
-    constexpr int R = decltype(rtag)::value;
-    if (a.B == 1) append_body<1, W8, R>(a, cluster, smem, L);
-    else if (a.B == 2) append_body<2, W8, R>(a, cluster, smem, L);
-    else append_body<4, W8, R>(a, cluster, smem, L);
-  };
-  switch (a.r) {
-    case 8: run(std::integral_constant<int, 8>{}); break;
-    case 16: run(std::integral_constant<int, 16>{}); break;
-    case 32: run(std::integral_constant<int, 32>{}); break;
-    case 64: run(std::integral_constant<int, 64>{}); break;
-    default: run(std::integral_constant<int, 128>{}); break;
-  }
+  const AppendSmem L = append_layout(a.B, a.E / a.cluster, R, a.cluster);
+  if (a.B == 1) append_body<1, W8, R>(a, cluster, smem, L);
+  else if (a.B == 2) append_body<2, W8, R>(a, cluster, smem, L);
+  else append_body<4, W8, R>(a, cluster, smem, L);
 }
 
 int append_cluster_size(int E, int blk) {
@@ -210,16 +201,24 @@ size_t append_smem_bytes(int B, int E, int r, int cluster) {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   const size_t smem = append_smem_bytes(a.B, a.E, a.r, a.cluster);
-  void (*kern)(const AppendArgs) = a.w8 ? append_kernel<true> : append_kernel<false>;
+  void (*kern)(const AppendArgs) = nullptr;
+  switch (a.r) {
+    case 8: kern = a.w8 ? append_kernel<true, 8> : append_kernel<false, 8>; break;
+    case 16: kern = a.w8 ? append_kernel<true, 16> : append_kernel<false, 16>; break;
+    case 32: kern = a.w8 ? append_kernel<true, 32> : append_kernel<false, 32>; break;
+    case 64: kern = a.w8 ? append_kernel<true, 64> : append_kernel<false, 64>; break;
+    case 128: kern = a.w8 ? append_kernel<true, 128> : append_kernel<false, 128>; break;
+    default: return cudaErrorInvalidValue;  // rejected by the argument checks before this
+  }
   {
     // Opt in to the dynamic shared memory once per device, kernel and size.
     static std::mutex mu;
-    static std::map<std::pair<int, int>, size_t> done;
+    static std::map<std::pair<int, const void*>, size_t> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_pair(dev, a.w8);
+    const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
     auto it = done.find(key);
     if (it == done.end() || it->second < smem) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
