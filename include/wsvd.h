@@ -377,10 +377,11 @@ void wsvd_step_host_graph_destroy(wsvd_step_graph* graph);
  * and the results are those of the fp16 entry points given those dequantised
  * weights (the kernels fold each scale in once: into q for B_k, after the
  * column sums for A and B_v).  The pages fix no granularity for the weight
- * scales; per output column is this library's reading.  Int8 matrices must be
- * 16-byte aligned; scales are read with plain loads.  Every other argument,
- * the workspace contracts and the status codes are those of the fp16 entry
- * points. */
+ * scales; per output column is this library's reading.  Int8 matrices and
+ * the B scales sB_k, sB_v must be 16-byte aligned (the decode stages a head's
+ * rows of them with bulk copies; else WSVD_ERR_INVALID_ARG); the A scales are
+ * read with plain loads.  Every other argument, the workspace contracts and
+ * the status codes are those of the fp16 entry points. */
 int wsvd_decode_attention_w8(int B, int H, int Hd, int r, int bits, int L_cap, const int32_t* seq_lens,
                              const void* q, int q_dtype, const uint8_t* lat_k, const uint8_t* lat_v,
                              const void* scale_k, const void* scale_v, const int8_t* B_k, const int8_t* B_v,

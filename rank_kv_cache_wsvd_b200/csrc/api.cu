@@ -110,6 +110,7 @@ int prepare_wsvd_decode(int B, int H, int Hd, int r, int bits, int L_cap, const 
   if (!aligned16(lat_k) || !aligned16(lat_v) || !aligned16(scale_k) || !aligned16(scale_v) ||
       !aligned16(B_k) || !aligned16(B_v))
     return WSVD_ERR_INVALID_ARG;
+  if (w8 && (!aligned16(sB_k) || !aligned16(sB_v))) return WSVD_ERR_INVALID_ARG;  // staged by bulk copies
   if (workspace_bytes < decode_ws_bytes(B, H, r)) return WSVD_ERR_WORKSPACE_TOO_SMALL;
   a->B = B; a->H = H; a->Hd = Hd; a->W = r; a->L_cap = L_cap; a->heads_share = 0;
   a->seq_lens = seq_lens; a->q = q; a->q_dtype = q_dtype;

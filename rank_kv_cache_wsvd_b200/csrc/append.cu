@@ -83,6 +83,9 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
   uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   int* pos_sm = reinterpret_cast<int*>(smem + L.pos_off);  // leader: seq_lens[b] as read at launch
 
+  // int8 weights: the leader's quantising lanes load their column scales now.
+  ColScales<R> cs;
+  if (W8 && rank == 0) cs.load((kv ? a.sAv : a.sAk) + (size_t)h * r, r, lane);
   // The leader reads the row positions first so that their latency is hidden.
   // No CTA writes seq_lens before every leader has counted itself done (below).
   if (rank == 0 && tid < B) pos_sm[tid] = ld_relaxed_gpu(a.seq_lens + tid);
@@ -165,8 +168,7 @@ __device__ __forceinline__ void append_body(const AppendArgs& a, cg::cluster_gro
     const bool ok = pos >= 0 && pos < a.L_cap;
     const size_t row = ((size_t)b * a.H + h) * a.L_cap + (ok ? pos : 0);
     const __half sh = quantise_append_row<W8, R>(slots + (size_t)b * r, (size_t)B * r, a.cluster, r, a.bits, a.hnorm,
-                                              W8 ? (kv ? a.sAv : a.sAk) + (size_t)h * r : nullptr, ok,
-                                              (kv ? a.lat_v : a.lat_k) + row * RB, nullptr, lane);
+                                                 cs, ok, (kv ? a.lat_v : a.lat_k) + row * RB, nullptr, lane);
     if (lane == 0) {
       if (ok) (kv ? a.scale_v : a.scale_k)[row] = sh;
       else if (unit == 0) set_err(a.err, WSVD_DEVERR_CACHE_FULL);

@@ -245,15 +245,27 @@ __device__ __forceinline__ void rotate_x_slice(bool fast, const uint2 (&xraw)[kX
   sync();
 }
 
+// The int8 weights' column scales of the columns a lane quantises (j = lane +
+// 32 k), loaded ahead of the quantiser so that their latency is hidden.
+template <int RMAX>
+struct ColScales {
+  static constexpr int K = (RMAX + 31) / 32;
+  float v[K];
+  __device__ __forceinline__ void load(const float* colscale, int r, int lane) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) v[k] = (lane + 32 * k < r) ? __ldg(colscale + lane + 32 * k) : 1.f;
+  }
+};
+
 // Quantise one finished row of one (b, h, K|V) unit, one warp: the cluster
 // ranks' partial sums (slots[q * stride + j], q = 0 .. nranks - 1) added in
-// rank order, times 1/sqrt(blk) (and the int8 weights' column scale), then the
-// append's fp32 decisions; the codes are written to dst when `ok` (and to
-// dst2 too, when given).  Returns the fp16 scale.  RMAX: a bound on r known
-// at compile time (128 covers every r; a caller with a fixed r passes it).
+// rank order, times 1/sqrt(blk) (and the int8 weights' column scale, from cs),
+// then the append's fp32 decisions; the codes are written to dst when `ok`
+// (and to dst2 too, when given).  Returns the fp16 scale.  RMAX: a bound on r
+// known at compile time (128 covers every r; a caller with a fixed r passes it).
 template <bool W8, int RMAX = 128>
 __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t stride, int nranks, int r, int bits,
-                                                      float hnorm, const float* colscale, bool ok, uint8_t* dst,
+                                                      float hnorm, const ColScales<RMAX>& cs, bool ok, uint8_t* dst,
                                                       uint8_t* dst2, int lane) {
   constexpr int KMAX = (RMAX + 31) / 32;  // column groups of 32 a lane may hold
   const int Q = (bits == 8) ? 127 : 7;
@@ -269,7 +281,7 @@ __device__ __forceinline__ __half quantise_append_row(const float* slots, size_t
       for (int q = 0; q < 8; ++q)  // clusters hold at most 8 ranks
         if (q < nranks) sum += slots[(size_t)q * stride + j];
       cv[k] = sum * hnorm;
-      if (W8) cv[k] *= colscale[j];  // column scale of int8 A
+      if (W8) cv[k] *= cs.v[k];  // column scale of int8 A
       amax = fmaxf(amax, fabsf(cv[k]));
     }
   }

@@ -348,7 +348,8 @@ __device__ __forceinline__ void csync() { named_barrier_sync(1, kConsumerThreads
 __device__ __forceinline__ float qprime_rows(const uint8_t* sbuf, float* qs, const DecodeArgs& a, int h, int W,
                                             int j0, int jstep, int part) {
   const uint16_t* qsrc = reinterpret_cast<const uint16_t*>(sbuf + (size_t)W * a.Hd * (a.w8 ? 1 : 2));
-  const float* colscale = a.w8 ? a.sBk + (size_t)h * a.Hd : nullptr;  // int8 B_K: folded into q
+  // int8 B_K: its column scales (staged after q) are folded into q
+  const float* colscale = a.w8 ? reinterpret_cast<const float*>(qsrc + a.Hd) : nullptr;
   const int cols = a.Hd >> 3;  // 4, 8, 16 or 32: a power of two, a multiple of 4
   const int cmask = cols - 1;
   float amax = 0.f;
@@ -702,10 +703,13 @@ __device__ __forceinline__ void issue_operands(uint8_t* dst, uint64_t* bar, cons
                                                uint64_t keep) {
   const size_t bh = (size_t)b * a.H + h;
   if (QMODE == kQProj) {
-    const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), qb = (uint32_t)a.Hd * 2;
-    mbar_arrive_expect_tx(bar, bb + qb);
+    // B_Kh, q and (int8 B_K) its column scales; the segment buffer holds
+    // W * Hd * 2 + Hd * 2 bytes, enough for the scales when B_K is int8.
+    const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), qb = (uint32_t)a.Hd * 2, sb = a.w8 ? (uint32_t)a.Hd * 4 : 0u;
+    mbar_arrive_expect_tx(bar, bb + qb + sb);
     bulk_g2s(dst, static_cast<const uint8_t*>(a.Bk) + (size_t)h * bb, bb, bar, keep);
     bulk_g2s(dst + bb, static_cast<const uint16_t*>(a.q) + bh * a.Hd, qb, bar, keep);
+    if (a.w8) bulk_g2s(dst + bb + qb, a.sBk + (size_t)h * a.Hd, sb, bar, keep);
   } else if (QMODE == kQDirect) {
     mbar_arrive_expect_tx(bar, (uint32_t)a.Hd * 2);
     bulk_g2s(dst, static_cast<const uint16_t*>(a.q) + bh * a.Hd, (uint32_t)a.Hd * 2, bar, keep);
@@ -1268,11 +1272,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     const uint64_t keep = l2_evict_last_policy();
     issue_operands<W, QMODE>(segbuf, segfull, a, b, h, keep);
     if (rank == 0 && a.Bv != nullptr) {
-      const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2);
-      mbar_arrive_expect_tx(&aux[0], bb);
+      // B_Vh, and (int8 B_V) its column scales after it
+      const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), sb = a.w8 ? (uint32_t)a.Hd * 4 : 0u;
+      mbar_arrive_expect_tx(&aux[0], bb + sb);
       for (uint32_t off = 0; off < bb; off += 32768)
         bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, static_cast<const uint8_t*>(a.Bv) + (size_t)h * bb + off,
                  min(32768u, bb - off), &aux[0], keep);
+      if (a.w8) bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + bb, a.sBv + (size_t)h * a.Hd, sb, &aux[0], keep);
     }
   }
   cluster_arrive_relaxed();  // barriers initialised; waited on before any remote access
@@ -1457,11 +1463,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
     csync();
     merge_rows<W, false>(slots, csize, res, tid);
   }
-  BvRef Bvh{nullptr, a.w8, a.w8 ? a.sBv + (size_t)h * a.Hd : nullptr};
+  BvRef Bvh{nullptr, a.w8, nullptr};
   if (a.Bv != nullptr) {
     if (!mbar_wait_bounded(&aux[0], 0, timed_out ? 0ull : kWaitLimitNs) && lane == 0)
       set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
     Bvh.p = bvs;
+    if (a.w8) Bvh.sv = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(bvs) + (size_t)W * a.Hd);
   }
   finalize_out<W>(res, Bvh, a.out + ((size_t)b * a.H + h) * a.Hd, a.Hd, red, tid);
 }
@@ -1584,8 +1591,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
       const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
       const uint32_t bb = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), qb = (uint32_t)a.Hd * 2;
       const uint16_t* qh = static_cast<const uint16_t*>(a.q) + (size_t)h * a.Hd;
-      mbar_arrive_expect_tx(segfull, bb + qb);
+      const uint32_t sb = a.w8 ? (uint32_t)a.Hd * 4 : 0u;  // int8 B_K / B_V: their column scales
+      mbar_arrive_expect_tx(segfull, bb + qb + sb);
       bulk_g2s(segbuf, static_cast<const uint8_t*>(a.Bk) + (size_t)h * bb, bb, segfull, keep);
+      if (a.w8) bulk_g2s(segbuf + bb + qb, a.sBk + (size_t)h * a.Hd, sb, segfull, keep);
       if (!ap.dep) bulk_g2s(segbuf + bb, qh, qb, segfull, keep);
       for (int u = 0; u < 2; ++u) {
         const uint8_t* src = static_cast<const uint8_t*>(u ? ap.Av : ap.Ak) + ((size_t)h * E + e0) * r * (W8 ? 1 : 2);
@@ -1611,10 +1620,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
       *pos_sm = pos;
       mbar_arrive(bar_pos);
       if (rank == lead) {
-        mbar_arrive_expect_tx(&aux[0], bb);
+        mbar_arrive_expect_tx(&aux[0], bb + sb);
         for (uint32_t off = 0; off < bb; off += 32768)
           bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + off, static_cast<const uint8_t*>(a.Bv) + (size_t)h * bb + off,
                    min(32768u, bb - off), &aux[0], keep);
+        if (a.w8) bulk_g2s(reinterpret_cast<uint8_t*>(bvs) + bb, a.sBv + (size_t)h * a.Hd, sb, &aux[0], keep);
       }
       // The cached rows are read after this CTA's A slices have landed: they
       // are needed only after the projection, and would compete with it for
@@ -1661,6 +1671,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
     }
   };
   auto consumer_sync = []() { csync(); };
+  // int8 weights: warps 0 and 1 (the quantisers of K and V, should this rank
+  // own the new row) load their column scales now.
+  ColScales<W> cs;
+  if (W8 && warp < 2) cs.load((warp ? ap.sAv : ap.sAk) + (size_t)h * r, r, lane);
   // x slice of the append (registers on the fast path)
   const bool fast = x_fast_path(1, Ec, ap.blk);
   uint2 xraw[kXChunks];
@@ -1739,8 +1753,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
       const int RB = r * ap.bits / 8;
       uint8_t* tile_codes = stage + (size_t)u * C::kCodeBytes + (size_t)t * C::kRB;
       const __half sh = quantise_append_row<W8, W>(aslots + (size_t)u * r, (size_t)2 * r, csize, r, ap.bits, ap.hnorm,
-                                                W8 ? (u ? ap.sAv : ap.sAk) + (size_t)h * r : nullptr, true,
-                                                (u ? ap.lat_v : ap.lat_k) + row * RB, tile_codes, lane);
+                                                   cs, true, (u ? ap.lat_v : ap.lat_k) + row * RB, tile_codes, lane);
       if (lane == 0) {
         (u ? ap.scale_v : ap.scale_k)[row] = sh;
         reinterpret_cast<__half*>(stage + 2 * C::kCodeBytes + (size_t)u * C::kScaleBytes)[t] = sh;
@@ -1769,7 +1782,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) step_cluster_kernel(const D
   }
   if (!mbar_wait_bounded(&aux[0], 0, timed_out ? 0ull : kWaitLimitNs) && lane == 0)
     set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
-  const BvRef Bvh{bvs, a.w8, a.w8 ? a.sBv + (size_t)h * a.Hd : nullptr};
+  const BvRef Bvh{bvs, a.w8,
+                  a.w8 ? reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(bvs) + (size_t)W * a.Hd)
+                       : nullptr};
   finalize_out<W>(res, Bvh, a.out + (size_t)h * a.Hd, a.Hd, red, tid);
 }
 

@@ -89,6 +89,11 @@ def test_host_validation_rejects_before_launch(lib):
     # workspace too small
     assert lib.wsvd_decode_attention(1, 4, 64, 16, 8, 256, p, p, 0, p, p, p, p, p, p, 0.0, p, p, 64,
                                      None, None) == 4
+    # int8 weights: the B scales are staged by bulk copies and must be 16-byte aligned
+    assert lib.wsvd_decode_attention_w8(1, 4, 64, 16, 8, 256, p, p, 0, p, p, p, p, p, p, bad, p, 0.0, p, p, 1 << 20,
+                                        None, None) == 1
+    assert lib.wsvd_decode_attention_w8(1, 4, 64, 16, 8, 256, p, p, 0, p, p, p, p, p, p, p, bad, 0.0, p, p, 1 << 20,
+                                        None, None) == 1
     # empty batch is a no-op
     assert lib.wsvd_decode_attention(0, 4, 64, 16, 8, 256, None, None, 0, None, None, None, None, None, None,
                                      0.0, None, None, 0, None, None) == 0
