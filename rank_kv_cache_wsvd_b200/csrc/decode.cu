@@ -968,12 +968,15 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
       if (stage_bv) {
         int lb, lh, lt;
         walk.locate(g_end - 1, lb, lh, lt);
-        const uint32_t bytes = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2);
-        mbar_arrive_expect_tx(bvbar, bytes);
+        // B_Vh, and (int8 B_V, half the bytes) its column scales after it
+        const uint32_t bytes = (uint32_t)W * a.Hd * (a.w8 ? 1 : 2), sbytes = a.w8 ? (uint32_t)a.Hd * 4 : 0u;
+        mbar_arrive_expect_tx(bvbar, bytes + sbytes);
         for (uint32_t off = 0; off < bytes; off += 32768)
           bulk_g2s(reinterpret_cast<uint8_t*>(bv_last) + off,
                    static_cast<const uint8_t*>(a.Bv) + (size_t)lh * bytes + off, min(32768u, bytes - off), bvbar,
                    keep);
+        if (a.w8)
+          bulk_g2s(reinterpret_cast<uint8_t*>(bv_last) + bytes, a.sBv + (size_t)lh * a.Hd, sbytes, bvbar, keep);
       }
       // Leave no copy in flight behind: wait (bounded) for the last uses of each buffer.
       if (stage_bv && !mbar_wait_bounded(bvbar, 0)) set_err(a.err, WSVD_DEVERR_PIPE_TIMEOUT);
@@ -1129,9 +1132,10 @@ __global__ void __launch_bounds__(kPersistThreads, 2) decode_kernel(const Decode
     float* outp = a.out + ((size_t)b_ * a.H + h_) * a.Hd;
     BvRef Bvh{nullptr, a.w8, a.w8 ? a.sBv + (size_t)h_ * a.Hd : nullptr};
     if (a.Bv != nullptr) {
-      if (C::bv_stage_bytes(a.Hd) > 0) {  // staged by the producer
+      if (C::bv_stage_bytes(a.Hd) > 0) {  // staged by the producer (with the int8 scales after it)
         wait(bvbar, 0);
         Bvh.p = bv_last;
+        if (a.w8) Bvh.sv = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(bv_last) + (size_t)W * a.Hd);
       } else {
         Bvh.p = static_cast<const uint8_t*>(a.Bv) + (size_t)h_ * W * a.Hd * (a.w8 ? 1 : 2);
       }
