@@ -388,6 +388,11 @@ __global__ void __launch_bounds__(kGThreads, 2) grouped_decode_kernel(const Grou
     // ------------------------------------------------------------ producer
     const uint64_t pol = l2_evict_first_policy();
     const int gidx = (b * a.Hkv + hkv) * a.nqc + qc;
+    {  // warm B_Vh in L2 for whichever split finishes the group (read at the very end)
+      const char* bv = reinterpret_cast<const char*>(a.Bv + (size_t)hkv * R * a.Hd);
+      const int bytes = R * a.Hd * 2;
+      for (int o = lane * 128; o < bytes; o += 32 * 128) prefetch_l2(bv + o);
+    }
     auto stage_planes = [&]() {  // the q' planes and steps (written by the preceding grid)
       griddep_wait();
       mbar_arrive_expect_tx_warp(pready, (uint32_t)C::QBLOCK);
