@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -54,10 +55,16 @@ def peaks():
 
 
 def source_digest(files):
+    """Digest of the kernel sources with comments and blank space removed, so
+    that an edit of comments alone does not retire a capture (the sources
+    hold no string literal with a comment marker)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "rank_kv_cache_wsvd_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "rank_kv_cache_wsvd_b200", "csrc", f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1493,17 +1493,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_cluster_kernel(const
 // writes out[h].  So every output equals that of the append kernel followed
 // by the cluster decode, bit for bit.
 //
-// Order of work.  Producer lane: barriers, then bulk copies of B_Kh and the
-// query and of this rank's A_Kh and A_Vh slices (contiguous blocks, four
-// chunks each with a barrier apiece; behind a grid that writes the query,
-// the query comes after the dependency wait).  Then the length (its load
-// overlaps the issue), which reaches the consumers through an mbarrier; B_Vh
-// (the merging rank); and, once the slices have landed, the cached rows of
-// the chunk below the new row.  Consumers: q' and the x slice rotation while
-// the copies land; the K and V projections of the slice chunk by chunk,
+// Order of work.  Producer lane: barriers, then bulk copies of B_Kh, the
+// query (and, for int8 B, B_K's column scales) and of this rank's A_Kh and
+// A_Vh slices (contiguous blocks, four chunks each with a barrier apiece;
+// behind a grid that writes the query, the query comes after the dependency
+// wait).  Then the length (its load overlaps the issue), which reaches the
+// consumers through an mbarrier; B_Vh (and its int8 column scales) into the
+// merging rank; and, once the slices have landed, the cached rows of the
+// chunk below the new row.  Consumers: q' and the x slice rotation while the
+// copies land (warps 0 and 1 load the int8 A column scales they would need
+// as quantisers); the K and V projections of the slice chunk by chunk,
 // reduced across the CTA in one pass and stored into the owner's slots; the
 // old rows; the owner quantises and processes the new row; every rank but the
 // merging one sends its decode partial there, which merges and writes out[h].
+// The latent width is a compile-time constant (r == W; the host checks it).
 //
 // The length advance: each CTA's producer lane, after its read of seq_lens,
 // counts the CTA in the append's completion counter (acq_rel); the last of
